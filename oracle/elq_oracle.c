@@ -1,0 +1,523 @@
+/*
+ * elq_oracle.c -- scalar CPU oracle of the quantized latent-MoE expert layer.
+ *
+ * TEST INFRASTRUCTURE ONLY (tests, the package smoke check and the benchmark's
+ * CPU-baseline leg).  Plain loops, one element at a time, in the order the
+ * definitions state.  Build flags: -O2 -ffp-contract=off -fno-fast-math, so
+ * that every fp32 operation below is one IEEE round-to-nearest operation and
+ * fmaf is the only fused one.  Readings R1-R14 are listed in elq_oracle.h.
+ */
+#include "elq_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* formats                                                                  */
+
+int orc_block_bytes(int fmt)
+{
+    switch (fmt) {
+    case ORC_Q4_0: return 18;
+    case ORC_Q8_0: return 34;
+    case ORC_Q8_1: return 36;
+    default: return 0;
+    }
+}
+
+int64_t orc_matrix_bytes(int fmt, int64_t rows, int64_t k)
+{
+    return rows * (k / 32) * (int64_t)orc_block_bytes(fmt);
+}
+
+/* fp32 -> fp16, round to nearest, ties to even (the loader's narrowing rule in
+ * "Q8 0 support", CONV1D).  Written from the IEEE 754 binary16 definition:
+ * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits, subnormals below
+ * 2^-14 with quantum 2^-24. */
+uint16_t orc_f32_to_f16(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, 4);
+    uint16_t sign = (uint16_t)((x >> 16) & 0x8000u);
+    uint32_t bexp = (x >> 23) & 0xFFu;
+    uint32_t frac = x & 0x7FFFFFu;
+    if (bexp == 0xFFu)                       /* inf or nan */
+        return (uint16_t)(sign | 0x7C00u | (frac ? 0x200u : 0u));
+    if (bexp == 0u)                          /* fp32 zero/subnormal < 2^-126 */
+        return sign;
+    int e = (int)bexp - 127;                 /* value = m * 2^(e-23) */
+    uint32_t m = frac | 0x800000u;           /* 24-bit significand */
+    if (e < -25)
+        return sign;                         /* below half the smallest subnormal */
+    int shift = (e >= -14) ? 13 : (-1 - e);  /* bits dropped from m */
+    uint32_t q = m >> shift;
+    uint32_t rem = m & ((1u << shift) - 1u);
+    uint32_t half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (q & 1u)))
+        q += 1u;
+    if (e >= -14) {                          /* normal result */
+        if (q == 0x800u) { q >>= 1; e += 1; }
+        int he = e + 15;
+        if (he >= 31)
+            return (uint16_t)(sign | 0x7C00u);
+        return (uint16_t)(sign | ((uint32_t)he << 10) | (q & 0x3FFu));
+    }
+    /* subnormal result; q == 0x400 is the smallest normal, encoded the same */
+    return (uint16_t)(sign | q);
+}
+
+float orc_f16_to_f32(uint16_t h)
+{
+    uint32_t sign = (uint32_t)(h & 0x8000u) << 16;
+    uint32_t he = (h >> 10) & 0x1Fu;
+    uint32_t hf = h & 0x3FFu;
+    float v;
+    if (he == 0u) {
+        v = (float)hf * 5.9604644775390625e-08f;   /* hf * 2^-24, exact */
+    } else if (he == 31u) {
+        uint32_t bits = 0x7F800000u | (hf << 13);
+        memcpy(&v, &bits, 4);
+    } else {
+        uint32_t bits = ((he - 15u + 127u) << 23) | (hf << 13);
+        memcpy(&v, &bits, 4);
+    }
+    uint32_t out;
+    memcpy(&out, &v, 4);
+    out |= sign;
+    memcpy(&v, &out, 4);
+    return v;
+}
+
+float orc_bf16_to_f32(uint16_t b)
+{
+    uint32_t bits = (uint32_t)b << 16;
+    float v;
+    memcpy(&v, &bits, 4);
+    return v;
+}
+
+/* R12: exp(x) by Cody and Waite's argument reduction (x = n ln2 + r with
+ * |r| <= ln2/2, ln2 carried as a high and a low fp32 part), the Taylor series
+ * of e^r to degree 7 evaluated by Horner's rule with fmaf, and an exact scaling
+ * by 2^n (two steps where the result is subnormal). */
+float orc_expf(float x)
+{
+    if (x != x) return x;
+    if (x > 88.72283935546875f) return INFINITY;          /* > ln(FLT_MAX) */
+    if (x < -103.972076416015625f) return 0.0f;           /* < ln(2^-150) */
+    const float log2e = 1.44269502162933349609375f;       /* fp32(1/ln 2) */
+    const float ln2_hi = 0.693145751953125f;              /* ln2, 16 significant bits */
+    const float ln2_lo = 1.428606765330187045037746429443359375e-06f; /* fp32(ln2 - ln2_hi) */
+    float n = rintf(x * log2e);
+    float r = fmaf(-n, ln2_hi, x);
+    r = fmaf(-n, ln2_lo, r);
+    /* 1/k! for k = 7 .. 2, each rounded to fp32 */
+    float p = 1.98412701138295233249664306640625e-04f;     /* 1/5040 */
+    p = fmaf(p, r, 1.388888922519981861114501953125e-03f); /* 1/720 */
+    p = fmaf(p, r, 8.333333767950534820556640625e-03f);    /* 1/120 */
+    p = fmaf(p, r, 4.16666679084300994873046875e-02f);     /* 1/24 */
+    p = fmaf(p, r, 1.6666667163372039794921875e-01f);      /* 1/6 */
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ni = (int)n;
+    if (ni > 127) {                                        /* p * 2^127 * 2^(n-127) */
+        uint32_t b1 = 254u << 23, b2 = (uint32_t)(ni - 127 + 127) << 23;
+        float s1, s2;
+        memcpy(&s1, &b1, 4);
+        memcpy(&s2, &b2, 4);
+        return (p * s1) * s2;
+    }
+    if (ni < -125) {                                       /* p * 2^(n+100) * 2^-100 */
+        uint32_t b1 = (uint32_t)(ni + 100 + 127) << 23, b2 = (uint32_t)(-100 + 127) << 23;
+        float s1, s2;
+        memcpy(&s1, &b1, 4);
+        memcpy(&s2, &b2, 4);
+        return (p * s1) * s2;
+    }
+    uint32_t b = (uint32_t)(ni + 127) << 23;
+    float s;
+    memcpy(&s, &b, 4);
+    return p * s;
+}
+
+/* R13: silu(g) = g / (1 + exp(-g)) */
+float orc_silu(float g)
+{
+    float e = orc_expf(-g);
+    float den = 1.0f + e;
+    return g / den;
+}
+
+/* ------------------------------------------------------------------------ */
+/* quantisers                                                               */
+
+static void put16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] = (uint8_t)(v >> 8); }
+static uint16_t get16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+
+/* R1-R3: q = clamp(round(x / d), -127, 127) with d = amax / 127 (fp32) */
+static void quant_sym8(const float* xb, float* d_out, int8_t* q, int* sumq)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        float a = fabsf(xb[i]);
+        if (a > amax) amax = a;
+    }
+    float d = amax / 127.0f;
+    int s = 0;
+    for (int i = 0; i < 32; ++i) {
+        int v = 0;
+        if (d != 0.0f) {
+            float r = roundf(xb[i] / d);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            v = (int)r;
+        }
+        q[i] = (int8_t)v;
+        s += v;
+    }
+    *d_out = d;
+    *sumq = s;
+}
+
+/* Q8_1 activation block: fp16 d, fp16 s = d * sum(q) (R4), int8 q[32] */
+void orc_quantize_q8_1(const float* x, int64_t n, uint8_t* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        float d;
+        int8_t q[32];
+        int sumq;
+        quant_sym8(x + 32 * b, &d, q, &sumq);
+        uint8_t* o = out + 36 * b;
+        put16(o, orc_f32_to_f16(d));
+        put16(o + 2, orc_f32_to_f16(d * (float)sumq));
+        memcpy(o + 4, q, 32);
+    }
+}
+
+/* Q8_0 weight block: fp16 d, int8 q[32] */
+void orc_quantize_q8_0(const float* x, int64_t n, uint8_t* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        float d;
+        int8_t q[32];
+        int sumq;
+        quant_sym8(x + 32 * b, &d, q, &sumq);
+        uint8_t* o = out + 34 * b;
+        put16(o, orc_f32_to_f16(d));
+        memcpy(o + 2, q, 32);
+    }
+}
+
+/* Q4_0 weight block (R5, R6): fp16 d = m / -8, nibbles q in [0, 15] */
+void orc_quantize_q4_0(const float* x, int64_t n, uint8_t* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const float* xb = x + 32 * b;
+        float amax = 0.0f, m = 0.0f;
+        for (int i = 0; i < 32; ++i) {
+            float a = fabsf(xb[i]);
+            if (a > amax) { amax = a; m = xb[i]; }
+        }
+        float d = m / -8.0f;
+        uint8_t q[32];
+        for (int i = 0; i < 32; ++i) {
+            int v = 8;
+            if (d != 0.0f) {
+                float r = roundf(xb[i] / d) + 8.0f;
+                if (r < 0.0f) r = 0.0f;
+                if (r > 15.0f) r = 15.0f;
+                v = (int)r;
+            }
+            q[i] = (uint8_t)v;
+        }
+        uint8_t* o = out + 18 * b;
+        put16(o, orc_f32_to_f16(d));
+        for (int j = 0; j < 16; ++j)
+            o[2 + j] = (uint8_t)(q[j] | (q[j + 16] << 4));
+    }
+}
+
+void orc_dequantize(int fmt, const uint8_t* blocks, int64_t n, double* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        double* ob = out + 32 * b;
+        if (fmt == ORC_Q8_0 || fmt == ORC_Q8_1) {
+            const uint8_t* p = blocks + (int64_t)orc_block_bytes(fmt) * b;
+            double d = (double)orc_f16_to_f32(get16(p));
+            const int8_t* q = (const int8_t*)(p + (fmt == ORC_Q8_0 ? 2 : 4));
+            for (int i = 0; i < 32; ++i) ob[i] = d * (double)q[i];
+        } else if (fmt == ORC_Q4_0) {
+            const uint8_t* p = blocks + 18 * b;
+            double d = (double)orc_f16_to_f32(get16(p));
+            for (int j = 0; j < 16; ++j) {
+                ob[j] = d * (double)((p[2 + j] & 0x0F) - 8);
+                ob[j + 16] = d * (double)((p[2 + j] >> 4) - 8);
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* block dots ("Q8 0 support", GPU EXPERT KERNELS; R7 for Q4_0)              */
+
+int32_t orc_block_isum(int wfmt, const uint8_t* w, const uint8_t* a)
+{
+    const int8_t* qa = (const int8_t*)(a + 4);
+    int32_t s = 0;
+    if (wfmt == ORC_Q8_0) {
+        const int8_t* qw = (const int8_t*)(w + 2);
+        for (int i = 0; i < 32; ++i) s += (int32_t)qw[i] * (int32_t)qa[i];
+    } else if (wfmt == ORC_Q4_0) {
+        for (int j = 0; j < 16; ++j) {
+            int lo = (w[2 + j] & 0x0F) - 8;
+            int hi = (w[2 + j] >> 4) - 8;
+            s += lo * (int32_t)qa[j] + hi * (int32_t)qa[j + 16];
+        }
+    }
+    return s;
+}
+
+float orc_block_term(int wfmt, const uint8_t* w, const uint8_t* a)
+{
+    float sc = orc_f16_to_f32(get16(w)) * orc_f16_to_f32(get16(a));
+    return (float)orc_block_isum(wfmt, w, a) * sc;
+}
+
+/* R8 */
+void orc_qmatmul(int wfmt, const uint8_t* W, int N, int K,
+                 const uint8_t* Xq, int T, float* Y)
+{
+    int nb = K / 32;
+    int wb = orc_block_bytes(wfmt);
+    for (int t = 0; t < T; ++t) {
+        const uint8_t* xr = Xq + (int64_t)t * nb * 36;
+        for (int n = 0; n < N; ++n) {
+            const uint8_t* wr = W + (int64_t)n * nb * wb;
+            float acc = 0.0f;
+            for (int c = 0; c < nb; c += 8) {
+                float part = 0.0f;
+                for (int kb = c; kb < c + 8 && kb < nb; ++kb) {
+                    const uint8_t* wk = wr + (int64_t)kb * wb;
+                    const uint8_t* ak = xr + (int64_t)kb * 36;
+                    int32_t isum = orc_block_isum(wfmt, wk, ak);
+                    float sc = orc_f16_to_f32(get16(wk)) * orc_f16_to_f32(get16(ak));
+                    part = fmaf((float)isum, sc, part);
+                }
+                acc = acc + part;
+            }
+            Y[(int64_t)t * N + n] = acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* router (R9-R11)                                                          */
+
+void orc_router_topk(const float* z, const float* Wr, const float* bias,
+                     int T, int L, int E, int k,
+                     int32_t* idx, float* w, float* logits)
+{
+    float* lg = (float*)malloc(sizeof(float) * (size_t)E);
+    char* taken = (char*)malloc((size_t)E);
+    for (int t = 0; t < T; ++t) {
+        const float* zt = z + (int64_t)t * L;
+        for (int e = 0; e < E; ++e) {
+            const float* we = Wr + (int64_t)e * L;
+            float part[32];
+            for (int j = 0; j < 32; ++j) {
+                float p = 0.0f;
+                for (int l = j; l < L; l += 32) p = fmaf(zt[l], we[l], p);
+                part[j] = p;
+            }
+            for (int off = 16; off >= 1; off /= 2) {
+                float nxt[32];
+                for (int j = 0; j < 32; ++j) nxt[j] = part[j] + part[j ^ off];
+                memcpy(part, nxt, sizeof(part));
+            }
+            float v = part[0];
+            if (bias) v = v + bias[e];
+            lg[e] = v;
+            if (logits) logits[(int64_t)t * E + e] = v;
+        }
+        memset(taken, 0, (size_t)E);
+        for (int j = 0; j < k; ++j) {          /* k largest, lower id on ties */
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || lg[e] > lg[best]) best = e;
+            }
+            taken[best] = 1;
+            idx[(int64_t)t * k + j] = best;
+        }
+        float l0 = lg[idx[(int64_t)t * k]];
+        float ex[64];
+        float sum = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            ex[j] = orc_expf(lg[idx[(int64_t)t * k + j]] - l0);
+            sum = sum + ex[j];
+        }
+        for (int j = 0; j < k; ++j) w[(int64_t)t * k + j] = ex[j] / sum;
+    }
+    free(lg);
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------ */
+/* bucketing                                                                */
+
+void orc_bucket(const int32_t* idx, int T, int k, int E,
+                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos)
+{
+    int P = T * k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int p = 0; p < P; ++p) counts[idx[p]] += 1;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int n = 0;
+    for (int e = 0; e < E; ++e)
+        for (int p = 0; p < P; ++p)
+            if (idx[p] == e) { perm[n] = p; pos[p] = n; ++n; }
+}
+
+/* ------------------------------------------------------------------------ */
+/* the layer                                                                */
+
+static int check_layer(const orc_layer* ly)
+{
+    if (ly->H % 32 || ly->L % 32 || ly->I % 32 || ly->E < 1 || ly->k < 1 ||
+        ly->k > ly->E || ly->k > 64)
+        return -2;
+    if (!orc_block_bytes(ly->du_fmt) || !orc_block_bytes(ly->ex_fmt) ||
+        ly->du_fmt == ORC_Q8_1 || ly->ex_fmt == ORC_Q8_1)
+        return -2;
+    return 0;
+}
+
+int orc_route(const orc_layer* ly, const float* x, int T, int32_t* idx, float* w)
+{
+    if (check_layer(ly)) return -2;
+    int H = ly->H, L = ly->L;
+    uint8_t* xq = (uint8_t*)malloc((size_t)T * (H / 32) * 36 + 1);
+    float* z = (float*)malloc(sizeof(float) * (size_t)T * L + 1);
+    orc_quantize_q8_1(x, (int64_t)T * H, xq);
+    orc_qmatmul(ly->du_fmt, ly->D, L, H, xq, T, z);
+    orc_router_topk(z, ly->router_w, ly->router_bias, T, L, ly->E, ly->k, idx, w, NULL);
+    free(xq);
+    free(z);
+    return 0;
+}
+
+int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trace* tr)
+{
+    if (check_layer(ly)) return -2;
+    int H = ly->H, L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    int P = T * k;
+    size_t xqb = (size_t)T * (H / 32) * 36, zqb = (size_t)T * (L / 32) * 36;
+    uint8_t* xq = (uint8_t*)malloc(xqb + 1);
+    float* z = (float*)malloc(sizeof(float) * (size_t)T * L + 1);
+    float* lg = (float*)malloc(sizeof(float) * (size_t)T * E + 1);
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)P + 1);
+    float* w = (float*)malloc(sizeof(float) * (size_t)P + 1);
+    uint8_t* zq = (uint8_t*)malloc(zqb + 1);
+    int32_t* counts = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    int32_t* offsets = (int32_t*)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (size_t)P + 1);
+    int32_t* pos = (int32_t*)malloc(sizeof(int32_t) * (size_t)P + 1);
+    float* g = (float*)malloc(sizeof(float) * (size_t)I);
+    float* u = (float*)malloc(sizeof(float) * (size_t)I);
+    float* h = (float*)malloc(sizeof(float) * (size_t)I);
+    uint8_t* hq = (uint8_t*)malloc((size_t)(I / 32) * 36);
+    float* o = (float*)malloc(sizeof(float) * (size_t)P * L + 1);
+    float* ylat = (float*)malloc(sizeof(float) * (size_t)T * L + 1);
+    uint8_t* ylq = (uint8_t*)malloc(zqb + 1);
+    int rc = 0;
+
+    /* a1, a2: x -> xq -> z */
+    orc_quantize_q8_1(x, (int64_t)T * H, xq);
+    orc_qmatmul(ly->du_fmt, ly->D, L, H, xq, T, z);
+    /* a3: router on the fp32 latent */
+    orc_router_topk(z, ly->router_w, ly->router_bias, T, L, E, k, idx, w, lg);
+    /* a4: latent activations for the experts */
+    orc_quantize_q8_1(z, (int64_t)T * L, zq);
+    /* a5 */
+    orc_bucket(idx, T, k, E, counts, offsets, perm, pos);
+    /* a6-a8, one (token, slot) pair at a time, in pair order */
+    for (int p = 0; p < P && rc == 0; ++p) {
+        int t = p / k, e = idx[p];
+        if (!ly->gate[e] || !ly->up[e] || !ly->down[e]) { rc = -1; break; }
+        const uint8_t* zt = zq + (size_t)t * (L / 32) * 36;
+        orc_qmatmul(ly->ex_fmt, ly->gate[e], I, L, zt, 1, g);
+        orc_qmatmul(ly->ex_fmt, ly->up[e], I, L, zt, 1, u);
+        for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
+        orc_quantize_q8_1(h, I, hq);
+        orc_qmatmul(ly->ex_fmt, ly->down[e], L, I, hq, 1, o + (size_t)p * L);
+        if (tr && tr->g) memcpy(tr->g + (size_t)p * I, g, sizeof(float) * (size_t)I);
+        if (tr && tr->u) memcpy(tr->u + (size_t)p * I, u, sizeof(float) * (size_t)I);
+        if (tr && tr->hq) memcpy(tr->hq + (size_t)p * (I / 32) * 36, hq, (size_t)(I / 32) * 36);
+    }
+    if (rc == 0) {
+        /* a9: weighted combine in rank order, then Q8_1 */
+        for (int t = 0; t < T; ++t)
+            for (int n = 0; n < L; ++n) {
+                float acc = 0.0f;
+                for (int j = 0; j < k; ++j)
+                    acc = fmaf(w[t * k + j], o[(size_t)(t * k + j) * L + n], acc);
+                ylat[(size_t)t * L + n] = acc;
+            }
+        orc_quantize_q8_1(ylat, (int64_t)T * L, ylq);
+        /* a10 */
+        orc_qmatmul(ly->du_fmt, ly->U, H, L, ylq, T, y);
+    }
+    if (tr) {
+        if (tr->xq) memcpy(tr->xq, xq, xqb);
+        if (tr->z) memcpy(tr->z, z, sizeof(float) * (size_t)T * L);
+        if (tr->logits) memcpy(tr->logits, lg, sizeof(float) * (size_t)T * E);
+        if (tr->idx) memcpy(tr->idx, idx, sizeof(int32_t) * (size_t)P);
+        if (tr->w) memcpy(tr->w, w, sizeof(float) * (size_t)P);
+        if (tr->zq) memcpy(tr->zq, zq, zqb);
+        if (tr->counts) memcpy(tr->counts, counts, sizeof(int32_t) * (size_t)E);
+        if (tr->offsets) memcpy(tr->offsets, offsets, sizeof(int32_t) * (size_t)(E + 1));
+        if (tr->perm) memcpy(tr->perm, perm, sizeof(int32_t) * (size_t)P);
+        if (tr->pos) memcpy(tr->pos, pos, sizeof(int32_t) * (size_t)P);
+        if (rc == 0) {
+            if (tr->o) memcpy(tr->o, o, sizeof(float) * (size_t)P * L);
+            if (tr->y_lat) memcpy(tr->y_lat, ylat, sizeof(float) * (size_t)T * L);
+            if (tr->ylq) memcpy(tr->ylq, ylq, zqb);
+        }
+    }
+    free(xq); free(z); free(lg); free(idx); free(w); free(zq); free(counts);
+    free(offsets); free(perm); free(pos); free(g); free(u); free(h); free(hq);
+    free(o); free(ylat); free(ylq);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* device arena layout, written out element by element                       */
+
+void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
+                    uint8_t* q_out, uint8_t* d_out)
+{
+    int nb = k / 32;
+    int wb = orc_block_bytes(fmt);
+    for (int row = 0; row < n_rows; ++row) {
+        int tile = row / 128, r = row % 128;
+        for (int kb = 0; kb < nb; ++kb) {
+            const uint8_t* blk = aos + ((int64_t)row * nb + kb) * wb;
+            int64_t slab = (int64_t)tile * nb + kb;
+            /* scale: fp16 at index slab*128 + r */
+            d_out[(slab * 128 + r) * 2] = blk[0];
+            d_out[(slab * 128 + r) * 2 + 1] = blk[1];
+            if (fmt == ORC_Q8_0) {
+                for (int i = 0; i < 32; ++i) {
+                    int64_t off = slab * 4096 + (r / 8) * 256 + (i / 16) * 128 + (r % 8) * 16 + (i % 16);
+                    q_out[off] = blk[2 + i];
+                }
+            } else {
+                for (int j = 0; j < 16; ++j)
+                    q_out[slab * 2048 + r * 16 + j] = blk[2 + j];
+            }
+        }
+    }
+}

@@ -1,0 +1,160 @@
+/*
+ * elq_oracle.h -- scalar CPU oracle of the quantized latent-MoE expert layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the slow, plain statement of what the
+ * layer computes, used by the test-suite, by the package's smoke check and by
+ * the benchmark's CPU-baseline leg.  It shares no code, header, table or
+ * constant with the CUDA library (quantized_latent_moe_b200/csrc); the two are
+ * written independently from the same definitions and compared element by
+ * element.
+ *
+ * Sources (page title, section):
+ *  - "edge0-strata/EDGE0.md", section "Changes from upstream Strata": latent-MoE
+ *    layers with dense D (hidden->latent) and U (latent->hidden) projections in
+ *    Q8 or Q4, latent sizes 1792 / 1280.
+ *  - "Q8 0 support - Pull Request #255 - Niko1221/Strata", section "GPU EXPERT
+ *    KERNELS": the Q8_0 block (qk 32) and the Q8_0 x Q8_1 block dot; section
+ *    "VERIFIED AGAINST AN ORACLE": GPU experts quantize activations to Q8_1.
+ *    Follow-up commit "per-role format lists": a min/offset term multiplies the
+ *    sum of the QUANTIZED activations, not the stored s.
+ *  - "Sync upstream Strata v0.1.39 into Lanes" (Strata-Lanes PR #24), SYCL-port
+ *    commit: the activation quantiser is byte-exact only with a correctly
+ *    rounded fp32 divide.  Q8_0 PR #255, "CONV1D": fp32 -> fp16 narrowing is
+ *    round-to-nearest-even.
+ *
+ * Block byte layouts (little endian):
+ *   Q8_0 : fp16 d, int8 q[32]                       34 B
+ *   Q4_0 : fp16 d, uint8 nib[16] (q[j] | q[j+16]<<4) 18 B
+ *   Q8_1 : fp16 d, fp16 s, int8 q[32]               36 B
+ *
+ * Readings where the pages are silent (each is the plainest one the rest
+ * supports):
+ *   R1 round(.) is round-half-away-from-zero (C roundf).
+ *   R2 d = amax / 127 and q = round(x / d) use an IEEE round-to-nearest fp32
+ *      divide; d == 0 gives q = 0; q is clamped to [-127, 127] (only reachable
+ *      when d is a tiny subnormal).
+ *   R3 q is computed with the fp32 d; the stored d is fp16(d) (RNE).
+ *   R4 Q8_1 s = fp16(d * (float)sum(q)).
+ *   R5 Q4_0: m = the element of largest |x| (lowest index on ties),
+ *      d = m / -8, q = clamp(round(x / d) + 8, 0, 15); d == 0 gives q = 8.
+ *   R6 Q4_0 nibble order: byte j = q[j] | q[j+16] << 4.
+ *   R7 Q4_0 x Q8_1: isum = sum (q4 - 8) * q8 (exact integer); s is unused.
+ *   R8 a row dot product accumulates in fp32 over chunks of 8 blocks:
+ *      sc = f32(d_w) * f32(d_a); part = fmaf((float)isum, sc, part) over the
+ *      blocks of a chunk in order from 0; acc = acc + part over the chunks in
+ *      order from 0.
+ *   R9 router logit = 32 strided fp32 partials (partial j takes l = j, j+32,
+ *      ... with fmaf), then an xor butterfly (16, 8, 4, 2, 1) of fp32 adds,
+ *      then + bias.  The router reads the unquantised fp32 latent z.
+ *   R10 bias takes part in selection and weights; top-k by logit descending,
+ *      lower expert id first on equal logits.
+ *   R11 weights = softmax over the k selected logits, in rank order.
+ *   R12 exp is this file's own orc_expf (Cody-Waite reduction, degree-7 Taylor
+ *      polynomial by fmaf, scaling by 2^n).
+ *   R13 SwiGLU: h = (g / (1 + exp(-g))) * u.
+ *   R14 combine: y_lat = sum_j fmaf(w_j, o_j, acc) over the k slots in rank
+ *      order from 0.
+ */
+#ifndef ELQ_ORACLE_H
+#define ELQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { ORC_Q4_0 = 2, ORC_Q8_0 = 8, ORC_Q8_1 = 9 };
+
+int      orc_block_bytes(int fmt);                /* 18, 34, 36; 0 if unknown */
+int64_t  orc_matrix_bytes(int fmt, int64_t rows, int64_t k);
+
+/* number formats */
+uint16_t orc_f32_to_f16(float x);                 /* round to nearest even */
+float    orc_f16_to_f32(uint16_t h);
+float    orc_bf16_to_f32(uint16_t b);
+float    orc_expf(float x);                       /* R12 */
+float    orc_silu(float g);                       /* R13 first factor */
+
+/* quantisers: n % 32 == 0, out holds n/32 blocks */
+void orc_quantize_q8_1(const float* x, int64_t n, uint8_t* out);
+void orc_quantize_q8_0(const float* x, int64_t n, uint8_t* out);
+void orc_quantize_q4_0(const float* x, int64_t n, uint8_t* out);
+/* fp64 dequantisers (self-checks) */
+void orc_dequantize(int fmt, const uint8_t* blocks, int64_t n, double* out);
+
+/* one weight block (Q8_0 or Q4_0) against one Q8_1 block */
+int32_t orc_block_isum(int wfmt, const uint8_t* wblk, const uint8_t* ablk);
+float   orc_block_term(int wfmt, const uint8_t* wblk, const uint8_t* ablk);
+
+/* Y[t][n] = row n of W (row-major AoS blocks, N rows x K) . Xq[t] (Q8_1, K)
+ * under R8; chunk = blocks per ordered chunk (8 in the layer). */
+void orc_qmatmul(int wfmt, const uint8_t* W, int N, int K,
+                 const uint8_t* Xq, int T, float* Y);
+
+/* router, R9-R11: idx [T][k], w [T][k], logits [T][E] (may be NULL) */
+void orc_router_topk(const float* z, const float* Wr, const float* bias,
+                     int T, int L, int E, int k,
+                     int32_t* idx, float* w, float* logits);
+
+/* token -> expert bucketing: counts [E], offsets [E+1] (exclusive scan),
+ * perm [T*k] pair ids sorted by (expert, pair id), pos [T*k] inverse. */
+void orc_bucket(const int32_t* idx, int T, int k, int E,
+                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos);
+
+/* One latent-MoE layer.  Weight matrices are row-major AoS blocks.
+ * gate/up/down are arrays of E pointers; an expert no token selects may be
+ * NULL. */
+typedef struct {
+    int H, L, E, k, I;
+    int du_fmt;                 /* format of D and U */
+    int ex_fmt;                 /* format of gate, up, down */
+    const uint8_t* D;           /* [L rows][H] */
+    const uint8_t* U;           /* [H rows][L] */
+    const float* router_w;      /* [E][L] fp32 */
+    const float* router_bias;   /* [E] or NULL */
+    const uint8_t* const* gate; /* E x [I rows][L] */
+    const uint8_t* const* up;   /* E x [I rows][L] */
+    const uint8_t* const* down; /* E x [L rows][I] */
+} orc_layer;
+
+/* Optional intermediates; any pointer may be NULL. */
+typedef struct {
+    uint8_t* xq;        /* [T][H/32] Q8_1 */
+    float*   z;         /* [T][L] */
+    float*   logits;    /* [T][E] */
+    int32_t* idx;       /* [T][k] */
+    float*   w;         /* [T][k] */
+    uint8_t* zq;        /* [T][L/32] Q8_1 */
+    int32_t* counts;    /* [E] */
+    int32_t* offsets;   /* [E+1] */
+    int32_t* perm;      /* [T*k] */
+    int32_t* pos;       /* [T*k] */
+    float*   g;         /* [T*k][I], pair order p = t*k + j */
+    float*   u;         /* [T*k][I] */
+    uint8_t* hq;        /* [T*k][I/32] Q8_1 */
+    float*   o;         /* [T*k][L] */
+    float*   y_lat;     /* [T][L] */
+    uint8_t* ylq;       /* [T][L/32] Q8_1 */
+} orc_trace;
+
+/* Returns 0, or -1 if a selected expert's weights are NULL, -2 on bad sizes. */
+int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y,
+                  orc_trace* tr);
+
+/* Only the routing half of the layer (x -> xq -> z -> idx, w), so that a caller
+ * can learn which experts a token set needs before supplying them. */
+int orc_route(const orc_layer* ly, const float* x, int T, int32_t* idx, float* w);
+
+/* The device arena layout, stated plainly (see elq.h of the library for the
+ * definition): rows in tiles of 128, per (tile, block) a 4096-byte Q8_0 slab
+ * in 8x16-byte core-matrix order, or a 2048-byte Q4_0 slab of 16-byte rows,
+ * and a 256-byte slab of fp16 scales.  aos is row-major AoS blocks.
+ * n_rows % 128 == 0. */
+void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
+                    uint8_t* q_out, uint8_t* d_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
