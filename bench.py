@@ -1,0 +1,465 @@
+#!/usr/bin/env python3
+"""Throughput of the quantized latent-MoE layer on B200.
+
+One step = one call of the whole layer (activation quantiser, D projection,
+router + top-k + bucketing, grouped gate/up + SwiGLU + requant, grouped down,
+weighted combine + requant, U projection) on one batch of synthetic input.
+The default workload is single-token decode: T=1, H=4096, latent L=1792, 128
+experts top-8, expert FFN I=1024, Q8_0 weights, bf16 input, router bias
+N(0, 1) per expert.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl elq|reference]
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+synchronize on both sides, timed with CUDA events on the launching stream; the
+max over ranks is taken.  Each rank runs its own replica on its own inputs
+(no data-path collective).  The working set per step is ~63 MB, below the
+126 MB L2, so the steps rotate over 8 distinct layer copies and 64 inputs:
+between two uses of the same weights 7 other layers' weights (~440 MB) pass
+through L2.
+
+--impl reference times the CPU oracle (the test-suite's scalar C statement of
+the layer) on the host cores on the same workload, one token per step.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent-MoE layer tokens/s; expert-weight HBM GB/s and % of B200 peak"
+KERNELS = ["quant_x", "proj_D", "router", "gate_up", "down", "combine", "proj_U"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4096)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="elq", choices=["elq", "reference"])
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--copies", type=int, default=8, help="distinct layer copies rotated over")
+    ap.add_argument("--inputs", type=int, default=64, help="distinct inputs rotated over")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded CPU-baseline sample")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_desc(wl):
+    return ("T=%d, H=%d, L=%d, E=%d, top-%d, I=%d, %s weights, %s input, router bias %s"
+            % (wl.T, wl.H, wl.L, wl.E, wl.k, wl.I, wl.fmt.upper(), wl.x_dtype, wl.bias))
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for (t, r) in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for (_, r) in self.rows[-3:]]
+        sm = [float(r[1]) for r in rows if len(r) > 2 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) > 2 and r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline and the reference arm)
+
+def oracle_setup(wl, n_tokens, gen_device):
+    import numpy as np
+    import oracle
+    from quantized_latent_moe_b200 import synth
+    fmt = {"q8_0": oracle.Q8_0, "q4_0": oracle.Q4_0}[wl.fmt]
+
+    def g(t):
+        return t.to("cpu").numpy()
+
+    dw = synth.dense_weights(wl, 0, device=gen_device)
+    w = {k: (None if v is None else g(v)) for k, v in dw.items()}
+    w["gate"] = None
+    ly = oracle.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, w)
+    xs = [g(synth.make_x(wl, step=s, device=gen_device).float()) for s in range(n_tokens)]
+    need = set()
+    for x in xs:
+        idx, _ = ly.route(x)
+        need |= set(idx.reshape(-1).tolist())
+    gate, up, down = [None] * wl.E, [None] * wl.E, [None] * wl.E
+    for e in sorted(need):
+        a, b, c = synth.expert_weights(wl, e, 0, device=gen_device)
+        gate[e], up[e], down[e] = g(a), g(b), g(c)
+    ly.set_experts({"gate": gate, "up": up, "down": down}, sorted(need))
+    return ly, xs
+
+
+def oracle_run(ly, xs, steps, threads):
+    """Run `steps` oracle layer calls (token s % len(xs) each) over `threads`
+    host threads (the C calls release the GIL); returns wall seconds."""
+    n = max(1, threads)
+    share = [steps // n + (1 if i < steps % n else 0) for i in range(n)]
+    start = [sum(share[:i]) for i in range(n)]
+
+    def work(i):
+        for s in range(start[i], start[i] + share[i]):
+            ly.forward(xs[s % len(xs)])
+
+    ths = [threading.Thread(target=work, args=(i,)) for i in range(n)]
+    t0 = time.perf_counter()
+    for t in ths:
+        t.start()
+    for t in ths:
+        t.join()
+    return time.perf_counter() - t0
+
+
+def host_threads():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(n, 32))
+
+
+def cpu_baseline(wl, seconds, gen_device):
+    ly, xs = oracle_setup(wl, 2, gen_device)
+    threads = host_threads()
+    t1 = oracle_run(ly, xs, threads, threads)          # calibration: one token per thread
+    steps = max(threads, int(seconds / max(t1, 1e-6) * threads))
+    dt = oracle_run(ly, xs, steps, threads)
+    return {"value": steps * wl.T / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d single-token %s layer calls (2 distinct tokens, their %d experts "
+                      "pre-quantised by the oracle), %.1f s wall on %d host threads"
+                      % (steps, wl.name, sum(g is not None for g in ly.gate), dt, threads)}
+
+
+def run_reference(args):
+    from quantized_latent_moe_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    gen = "cpu"
+    try:
+        import torch
+        if torch.cuda.is_available():
+            gen = "cuda"
+    except Exception:
+        pass
+    ly, xs = oracle_setup(wl, 2, gen)
+    threads = host_threads()
+    oracle_run(ly, xs, args.warmup, threads)
+    dt = oracle_run(ly, xs, args.steps, threads)
+    value = args.steps * wl.T / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic", "config": {"workload": "%s: %s" % (wl.name, workload_desc(wl)),
+                                        "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "each step: one single-token layer call of the scalar C oracle "
+                                   "(2 distinct tokens alternating), steps spread over %d host threads"
+                                   % threads},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_latent_moe_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """dram bytes per launch of `kernel` from the committed ncu summary, only if
+    it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_elq(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_latent_moe_b200 import build, elq, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    elq.lib()
+    wl = synth.WORKLOADS[args.workload]
+    fmt = elq.FMT[wl.fmt]
+    stream = torch.cuda.current_stream()
+
+    # distinct layer copies (layer index = copy + 8 * rank) and inputs
+    layers = []
+    for c in range(args.copies):
+        li = c + args.copies * rank
+        dw = synth.dense_weights(wl, li, device=dev)
+        rb = dw["router_bias"]
+        ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, dw["router_w"],
+                                None if rb is None else rb.to(dev), device=dev)
+        ly.set_dense(dw["D"], dw["U"])
+        for e0 in range(0, wl.E, 32):
+            n = min(32, wl.E - e0)
+            ws_ = [synth.expert_weights(wl, e, li, device=dev) for e in range(e0, e0 + n)]
+            ly.set_experts(e0, torch.stack([w[0] for w in ws_]), torch.stack([w[1] for w in ws_]),
+                           torch.stack([w[2] for w in ws_]))
+            del ws_
+        layers.append(ly)
+        del dw
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    S = args.inputs
+    xs = [synth.make_x(wl, step=s + 1000 * rank, device=dev) for s in range(S)]
+    ys = [torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev) for _ in range(2)]
+    ws = layers[0].workspace(wl.T)
+    for ly in layers[1:]:
+        ly._ws[wl.T] = ws          # steps are serial on the stream: one workspace serves all
+
+    def step(i, y=None):
+        elq.moe_layer(layers[i % args.copies], xs[i % S], ys[i % 2] if y is None else y, ws)
+
+    # eager warm-up of every (layer, input) pairing used, then a graph of G steps
+    for i in range(max(args.copies, 2)):
+        step(i)
+    torch.cuda.synchronize()
+    assert elq.workspace_status(ws) == 0
+    G = math.lcm(args.copies, S, 2)
+    graphs = {}
+
+    def graph_for(n, start):
+        key = (n, start % G)
+        if key not in graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(start, start + n):
+                    step(i)
+            graphs[key] = g
+        return graphs[key]
+
+    def run_steps(k, start=0):
+        done = 0
+        while done < k:
+            n = min(G, k - done)
+            graph_for(n, start + done).replay()
+            done += n
+        return start + k
+
+    launches_per_step = elq.lib().elq_layer_kernel_count()
+    pos = run_steps(args.warmup)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = Clocks(local)
+    time.sleep(0.3)
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    pos = run_steps(args.steps, pos)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    dev_ms = e0.elapsed_time(e1)
+
+    # end to end through the C ABI with host buffers: pinned x in, y out, every step
+    x_host = [x.cpu().pin_memory() for x in xs[:8]]
+    y_host = torch.empty(wl.T, wl.H, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    y_dev = torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev)
+    for i in range(8):
+        x_dev.copy_(x_host[i % 8], non_blocking=True)
+        elq.moe_layer(layers[i % args.copies], x_dev, y_dev, ws)
+        y_host.copy_(y_dev, non_blocking=True)
+        stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        x_dev.copy_(x_host[i % 8], non_blocking=True)
+        elq.moe_layer(layers[i % args.copies], x_dev, y_dev, ws)
+        y_host.copy_(y_dev, non_blocking=True)
+        stream.synchronize()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+
+    # per-kernel device time: the same steps with an event after every kernel
+    nk = launches_per_step
+    prof_steps = min(args.steps, 1024)
+    per = [[] for _ in range(nk)]
+    GP = min(G, 64)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(GP)]
+    gp = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gp):
+        for i in range(GP):
+            elq.moe_layer_profiled(layers[i % args.copies], xs[i % S], ys[i % 2], evs[i], ws)
+    gp.replay()
+    torch.cuda.synchronize()
+    for _ in range(max(1, prof_steps // GP)):
+        gp.replay()
+        torch.cuda.synchronize()
+        for i in range(GP):
+            for j in range(nk):
+                per[j].append(evs[i][j].elapsed_time(evs[i][j + 1]))
+    t_wall1 = time.time()
+    clocks = clk.stop(t_wall0, t_wall1)
+    kern_ms = [statistics.mean(v) for v in per]
+
+    # routed experts per step (for the algorithmic bytes of the expert kernels)
+    n_act = []
+    for i in range(min(S, 64)):
+        elq.moe_layer(layers[0], xs[i], ys[0], ws)
+        torch.cuda.synchronize()
+        n_act.append(int(elq.workspace_view(layers[0], wl.T, "n_act", ws).item()))
+    act = statistics.mean(n_act)
+
+    # max over ranks
+    t = torch.tensor([dev_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev_ms, e2e_ms = t.tolist()
+
+    if rank == 0:
+        blk = 34 if wl.fmt == "q8_0" else 18
+        nb_L, nb_H, nb_I = wl.L // 32, wl.H // 32, wl.I // 32
+        gu_w = act * 2 * wl.I * nb_L * blk
+        dn_w = act * wl.L * nb_I * blk
+        du_w = (wl.L * nb_H + wl.H * nb_L) * blk
+        rt_w = wl.E * wl.L * 4
+        P = wl.T * wl.k
+        gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
+        tokens = args.steps * wl.T * world
+        value = tokens / (dev_ms / 1e3)
+        peak, peak_kind = peaks()
+        gu_ms = kern_ms[KERNELS.index("gate_up")]
+        dn_ms = kern_ms[KERNELS.index("down")]
+        achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+        step_s = dev_ms / 1e3 / args.steps
+        layer_bytes = gu_w + dn_w + du_w + rt_w
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic (seeded counter-hash normals; random-init weights of the layer's shape)",
+            "config": {"workload": "%s: %s" % (wl.name, workload_desc(wl)),
+                       "global_batch": wl.T * world, "parallelism": "replicas" if world > 1 else "1 GPU",
+                       "layer_copies": args.copies, "inputs": S,
+                       "l2": "inputs larger than L2: %d layer copies x ~%.0f MB touched per step rotate, "
+                             "%.0f MB between reuses of a layer (L2 126 MB)"
+                             % (args.copies, layer_bytes / 1e6, (args.copies - 1) * layer_bytes / 1e6),
+                       "cuda_graph": "%d steps per graph, programmatic dependent launch" % G},
+            "expert_weight_gbs": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9,
+            "expert_weight_frac": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / peak,
+            "layer_weight_gbs": layer_bytes / step_s / 1e9,
+            "layer_weight_frac": layer_bytes / step_s / 1e9 / peak,
+            "kernel_ms": dict(zip(KERNELS, kern_ms)),
+            "distinct_experts_per_step": act,
+            "roofline": {"bound": "hbm", "kernel": "k_qgemv<Q8_0> gate/up (+SwiGLU, Q8_1)",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic_for("gate_up"),
+                         "algorithmic_bytes_per_launch": gu_bytes},
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": xs[0].numel() * xs[0].element_size(),
+                    "d2h_bytes_per_step": wl.T * wl.H * 4},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, "cuda")
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        del g
+    del gp
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args)
+        return
+    run_elq(args)
+
+
+if __name__ == "__main__":
+    main()

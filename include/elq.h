@@ -1,0 +1,250 @@
+/*
+ * elq.h -- C ABI of the quantized latent-MoE expert layer for B200 (sm_100a).
+ *
+ * The layer (page "edge0-strata/EDGE0.md", section "Changes from upstream
+ * Strata"): a dense D projection (hidden H -> latent L, L = 1792 or 1280), a
+ * router with top-k over E experts, per-expert gate/up -> SwiGLU -> down in the
+ * latent space, and a dense U projection (latent -> hidden).  Weights are
+ * Q8_0 or Q4_0 blocks of 32 values; activations are quantised to Q8_1 ("Q8 0
+ * support - Pull Request #255 - Niko1221/Strata", section "VERIFIED AGAINST AN
+ * ORACLE": the GPU experts quantise activations to Q8_1; section "GPU EXPERT
+ * KERNELS": the Q8_0 x Q8_1 block dot).
+ *
+ * Conventions shared by every call
+ *  - Pointers named as device pointers are CUDA device memory owned by the
+ *    caller.  The library allocates nothing, keeps no state between calls and
+ *    never synchronises the stream.  `stream` is a cudaStream_t (NULL = legacy
+ *    default stream).
+ *  - Device pointers must be 16-byte aligned unless stated otherwise.
+ *  - Every call validates its arguments on the host before it enqueues any
+ *    work, and returns ELQ_OK or a negative elq_status.  On an error nothing is
+ *    enqueued and no output is written.  Launch failures return ELQ_ERR_CUDA.
+ *    Faults inside kernels surface at the caller's next synchronisation.
+ *  - Calls that take a workspace `ws` use it for intermediates.  It must be at
+ *    least the size the matching *_workspace_bytes call returns, 256-byte
+ *    aligned, and ZERO-FILLED before its first use; every call leaves its
+ *    counters at zero again, so a workspace can be reused without clearing.
+ *    Two calls that share a workspace must not overlap on the GPU.
+ *  - Floating-point results follow a fixed accumulation order (below), so the
+ *    same inputs always give the same bits, whatever the launch shape.
+ *
+ * Block formats (little endian)
+ *   Q8_0 : fp16 d, int8 q[32]                    x = d * q            34 B
+ *   Q4_0 : fp16 d, uint8 nib[16]                 x = d * (q - 8)      18 B
+ *          byte j holds q[j] (low nibble) and q[j+16] (high nibble)
+ *   Q8_1 : fp16 d, fp16 s, int8 q[32]            s = d * sum(q)       36 B
+ *   Quantisation of a block: amax = max |x|; Q8: d = amax / 127 (fp32,
+ *   correctly rounded), q = round-half-away(x / d) (correctly rounded divide),
+ *   d stored as fp16 (round to nearest even); Q4_0: m = the element of largest
+ *   |x| (lowest index on ties), d = m / -8, q = clamp(round(x / d) + 8, 0, 15).
+ *   A zero scale gives all-zero codes (Q4_0: 8).
+ *
+ * Arithmetic
+ *   Block dot of a weight block with a Q8_1 block: isum = sum q_w * q_a (Q4_0:
+ *   sum (q_w - 8) * q_a, with the quantised activations' own sum, not s), an
+ *   exact int32.  A row dot over K = 32 * nb accumulates, for each run of 8
+ *   blocks in order, part = fmaf((float)isum, f32(d_w) * f32(d_a), part) from
+ *   0, and adds the runs' parts in order into an fp32 sum from 0.
+ *   Router logit: 32 lane-strided fp32 fmaf partials, an xor butterfly of adds
+ *   (16, 8, 4, 2, 1), plus the bias.  Top-k by logit, lower expert id first on
+ *   ties; weights are the softmax over the k selected logits.  exp() is the
+ *   library's own (Cody-Waite reduction, degree-7 Taylor polynomial).
+ *   SwiGLU h = (g / (1 + exp(-g))) * u; the weighted combine sums
+ *   fmaf(w_j, o_j, acc) over the k slots in rank order.
+ *
+ * Device weight arena ("tile-slab" layout)
+ *   A matrix of n_rows x k (n_rows % 128 == 0, k % 32 == 0, nb = k / 32) is
+ *   stored as tiles of 128 rows.  For tile t and block column kb, slab
+ *   s = t * nb + kb holds:
+ *     q : Q8_0 -- 4096 bytes at q + 4096 s: the 128 x 32 int8 codes as 8-row x
+ *         16-byte core matrices; code i of local row r sits at byte
+ *         (r/8)*256 + (i/16)*128 + (r%8)*16 + (i%16).  This is the K-major,
+ *         no-swizzle operand layout of the tcgen05 tensor cores (leading byte
+ *         offset 128, stride byte offset 256), so a slab is one bulk copy.
+ *         Q4_0 -- 2048 bytes at q + 2048 s: local row r's 16 nibble bytes at
+ *         byte 16 r, in the block's own order.
+ *     d : 128 fp16 scales at d + 256 s (local row r at element r).
+ *   q and d must be 256-byte aligned.
+ *
+ * Layer weights
+ *   D      : L rows x H;   U : H rows x L  (any weight format each)
+ *   router : fp32 [E][L], optional fp32 bias [E]
+ *   gate_up: E * 2I rows x L; expert e owns rows [2I e, 2I (e+1)); its tile j
+ *            holds gate rows 64j .. 64j+63 then up rows 64j .. 64j+63.
+ *            I % 64 == 0.
+ *   down   : E * L rows x I; expert e owns rows [L e, L (e+1)).
+ */
+#ifndef ELQ_H
+#define ELQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ELQ_OK = 0,
+    ELQ_ERR_INVALID_ARG = -1,   /* null pointer, bad size, k > E, ... */
+    ELQ_ERR_UNSUPPORTED = -2,   /* format or shape the kernels do not take */
+    ELQ_ERR_ALIGNMENT = -3,     /* a pointer is not aligned as required */
+    ELQ_ERR_WORKSPACE = -4,     /* workspace missing or too small */
+    ELQ_ERR_CUDA = -5,          /* a CUDA runtime call failed */
+    ELQ_ERR_TIMEOUT = -6        /* a bounded device wait ran out */
+} elq_status;
+
+typedef enum {                  /* GGUF type ids */
+    ELQ_F32 = 0,
+    ELQ_Q4_0 = 2,
+    ELQ_Q8_0 = 8,
+    ELQ_Q8_1 = 9,
+    ELQ_BF16 = 30
+} elq_type;
+
+/* One quantised matrix in the tile-slab arena (device pointers q, d). */
+typedef struct {
+    int32_t fmt;                /* ELQ_Q8_0 or ELQ_Q4_0 */
+    int32_t n_rows;             /* multiple of 128 */
+    int32_t k;                  /* multiple of 32 */
+    int32_t reserved;
+    const void* q;
+    const void* d;
+} elq_qmat;
+
+/* One latent-MoE layer.  The struct lives in host memory; every pointer in it
+ * is device memory. */
+typedef struct {
+    int32_t H, L, E, k, I;
+    int32_t reserved;
+    elq_qmat D;                 /* L x H  */
+    elq_qmat U;                 /* H x L  */
+    const float* router_w;      /* [E][L] */
+    const float* router_bias;   /* [E] or NULL */
+    elq_qmat gate_up;           /* E*2I x L, interleaved by 64-row halves */
+    elq_qmat down;              /* E*L x I */
+} elq_layer;
+
+/* ---- status ------------------------------------------------------------ */
+
+/* Static English text of a status code. */
+const char* elq_status_string(int32_t status);
+
+/* ABI version (increments on any change of this header). */
+int32_t elq_version(void);
+
+/* ---- arena preparation (not part of a layer call) ------------------------ */
+
+/* Bytes of the arena arrays of an n_rows x k matrix in format fmt.  Returns
+ * q_bytes + d_bytes, or 0 for an unsupported format/shape.  Either out
+ * pointer may be NULL. */
+size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k,
+                       size_t* q_bytes, size_t* d_bytes);
+
+/* Repack row-major GGUF-style AoS blocks (device, n_rows x k/32 blocks of
+ * 34 B (Q8_0) or 18 B (Q4_0), no alignment requirement) into the arena. */
+elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t k,
+                          void* q_out, void* d_out, void* stream);
+
+/* Quantise fp32 weights (device, row-major n_rows x k) into the arena with the
+ * format's own quantiser (block rules above). */
+elq_status elq_quantize_weights(int32_t fmt, const float* w, int32_t n_rows, int32_t k,
+                                void* q_out, void* d_out, void* stream);
+
+/* Quantise E experts' fp32 gate and up matrices (device, [E][I][L] each) into
+ * one gate_up arena (E*2I rows x L, interleaved as described above). */
+elq_status elq_quantize_gate_up(int32_t fmt, const float* gate, const float* up,
+                                int32_t E, int32_t I, int32_t L,
+                                void* q_out, void* d_out, void* stream);
+
+/* ---- the hot path --------------------------------------------------------- */
+
+/* Q8_1 activation quantiser (a1, a4).  x: device [rows][cols] fp32 (x_type
+ * ELQ_F32) or bf16 (ELQ_BF16), cols % 32 == 0, 4-byte aligned.  out: device
+ * rows*cols/32 Q8_1 blocks (36 B each, row-major, 4-byte aligned). */
+elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_t cols,
+                             void* out_q8_1, void* stream);
+
+/* Router (a3): logits = W_r z + bias, top-k, softmax over the k.  z: device fp32
+ * [T][L] (unquantised latent), w_router [E][L], bias [E] or NULL.  idx: device
+ * int32 [T][k] in rank order; weights fp32 [T][k]; logits fp32 [T][E] or NULL.
+ * 1 <= k <= min(E, 32), E <= 1024, L % 32 == 0. */
+elq_status elq_router_topk(const float* z, const float* w_router, const float* bias,
+                           int32_t T, int32_t L, int32_t E, int32_t k,
+                           int32_t* idx, float* weights, float* logits, void* stream);
+
+/* Token -> expert bucketing (a5): counts [E], offsets [E+1] (exclusive scan),
+ * perm [T*k] = pair ids p = t*k + j sorted by (expert, p), pos [T*k] its
+ * inverse.  All device int32. */
+elq_status elq_route_bucket(const int32_t* idx, int32_t T, int32_t k, int32_t E,
+                            int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* pos, void* stream);
+
+/* Latent projection (a2 with D, a10 with U): y[t][n] = row n of w . x[t].
+ * x_q8_1: device T rows of w->k/32 Q8_1 blocks; y: device fp32 [T][w->n_rows]. */
+size_t elq_latent_proj_workspace_bytes(const elq_qmat* w, int32_t T);
+elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped experts (a5-a9): bucketing, gate/up with SwiGLU and Q8_1 requant,
+ * down, and the weighted combine.  z_q8_1: device T rows of L/32 Q8_1 blocks;
+ * idx, weights: device [T][k] as elq_router_topk writes them; y_lat: device
+ * fp32 [T][L].  Uses layer->L, E, k, I, gate_up and down. */
+elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1,
+                                   const int32_t* idx, const float* weights, int32_t T,
+                                   float* y_lat, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer (a1-a10): x device [T][H] fp32 or bf16 -> y device fp32
+ * [T][H]. */
+size_t elq_workspace_bytes(const elq_layer* layer, int32_t T);
+elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T,
+                         float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernels one elq_moe_layer call launches, in order: activation
+ * quantiser, D projection (+ latent Q8_1), router (+ top-k, bucketing),
+ * gate/up (+ SwiGLU, Q8_1), down, combine (+ Q8_1), U projection. */
+int32_t elq_layer_kernel_count(void);
+
+/* elq_moe_layer that also records CUDA events on the stream: events[0] before
+ * the first kernel and events[i] after kernel i (i = 1 .. kernel count), so
+ * that elapsed times between consecutive events give each kernel's device
+ * time.  events: host array of n_events >= kernel count + 1 cudaEvent_t.
+ * Kernels launched this way do not overlap their prologues with the previous
+ * kernel (no programmatic dependent launch). */
+elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t x_type, int32_t T,
+                                  float* y, void* ws, size_t ws_bytes, void* const* events,
+                                  int32_t n_events, void* stream);
+
+/* Intermediates of an elq_moe_layer call inside its workspace, for tests and
+ * measurement.  `which`: 0 xq (Q8_1 of x), 1 z (fp32 [T][L]), 2 zq, 3 logits
+ * (fp32 [T][E]), 4 idx (int32 [T][k]), 5 weights (fp32 [T][k]), 6 counts
+ * (int32 [E]), 7 offsets (int32 [E+1]), 8 perm (int32 [T*k]), 9 pos, 10 hq
+ * (Q8_1 [T*k][I/32], by pair position), 11 o (fp32 [T*k][L], by position),
+ * 12 y_lat (fp32 [T][L]), 13 ylq (Q8_1), 14 number of routed experts (int32).
+ * Sets *offset (bytes from the workspace start) and *bytes; returns ELQ_OK or
+ * ELQ_ERR_INVALID_ARG.  The values are those of the last call on that
+ * workspace once the stream has reached its end. */
+elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which,
+                              size_t* offset, size_t* bytes);
+
+/* Reads the workspace's device error word after the stream has been
+ * synchronised by the caller (blocking copy of 4 bytes); returns ELQ_OK or
+ * ELQ_ERR_TIMEOUT, and clears the word. */
+elq_status elq_workspace_status(void* ws, void* stream);
+
+/* ---- test entry points ----------------------------------------------------- */
+
+/* Single-block dots ("Q8 0 support", GPU EXPERT KERNELS: block-dot parity to
+ * 1e-7): for i < nblocks, isum[i] and term[i] = (float)isum * (f32(d_w) *
+ * f32(d_a)) of AoS weight block i (wfmt Q8_0 or Q4_0) against Q8_1 block i.
+ * All device pointers, no alignment requirement. */
+elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q8_1,
+                                int64_t nblocks, int32_t* isum, float* term, void* stream);
+
+/* Runs the library's own exp on n fp32 values (device in -> out). */
+elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ELQ_H */

@@ -1,0 +1,168 @@
+// elq_device.cuh -- device helpers of the sm_100a kernels: number formats,
+// the library's own exp, block quantisation of one warp's 32 values, and the
+// bulk-copy / mbarrier primitives (inline PTX) with bounded waits.
+//
+// Every fp32 operation whose rounding is part of the layer's definition is
+// written with an explicit round-to-nearest intrinsic (__fmul_rn, __fadd_rn,
+// __fdiv_rn, __fmaf_rn); the library is also compiled with -fmad=false so no
+// other multiply-add is contracted.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace elq {
+
+constexpr int kTileRows = 128;     // rows per arena tile
+constexpr int kChunk = 8;          // blocks per ordered accumulation chunk
+constexpr int kQ80Slab = 4096;     // bytes of one Q8_0 (tile, block) slab
+constexpr int kQ40Slab = 2048;     // bytes of one Q4_0 (tile, block) slab
+constexpr int kScaleSlab = 256;    // bytes of one slab's 128 fp16 scales
+
+// Device error word codes (first int32 of a workspace).
+constexpr int kErrTimeout = 1;
+
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+// exp(x): Cody-Waite reduction x = n ln2 + r (ln2 as a 16-bit high part and
+// an fp32 low part), e^r by its Taylor series to degree 7 in Horner form with
+// fused multiply-adds, then an exact scaling by 2^n, split in two where the
+// result is subnormal or near overflow.
+__device__ __forceinline__ float exp_f32(float x) {
+    if (x != x) return x;
+    if (x > 88.72283935546875f) return __int_as_float(0x7f800000);
+    if (x < -103.972076416015625f) return 0.0f;
+    const float n = rintf(__fmul_rn(x, 1.44269502162933349609375f));
+    float r = __fmaf_rn(-n, 0.693145751953125f, x);
+    r = __fmaf_rn(-n, 1.428606765330187045037746429443359375e-06f, r);
+    float p = 1.98412701138295233249664306640625e-04f;
+    p = __fmaf_rn(p, r, 1.388888922519981861114501953125e-03f);
+    p = __fmaf_rn(p, r, 8.333333767950534820556640625e-03f);
+    p = __fmaf_rn(p, r, 4.16666679084300994873046875e-02f);
+    p = __fmaf_rn(p, r, 1.6666667163372039794921875e-01f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ni = (int)n;
+    if (ni > 127)
+        return __fmul_rn(__fmul_rn(p, __int_as_float(254 << 23)), __int_as_float((ni - 127 + 127) << 23));
+    if (ni < -125)
+        return __fmul_rn(__fmul_rn(p, __int_as_float((ni + 100 + 127) << 23)), __int_as_float(27 << 23));
+    return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+}
+
+__device__ __forceinline__ float silu_f32(float g) {
+    const float e = exp_f32(-g);
+    return __fdiv_rn(g, __fadd_rn(1.0f, e));
+}
+
+// Quantise one 32-value block held one value per lane (lane i = element i)
+// into a Q8_1 block at dst (4-byte aligned): fp16 d, fp16 s, int8 q[32].
+__device__ __forceinline__ void warp_quant_q8_1(float v, uint8_t* dst) {
+    const int lane = threadIdx.x & 31;
+    float amax = fabsf(v);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float d = __fdiv_rn(amax, 127.0f);
+    int q = 0;
+    if (d != 0.0f) {
+        float r = roundf(__fdiv_rn(v, d));
+        r = fminf(fmaxf(r, -127.0f), 127.0f);
+        q = (int)r;
+    }
+    int s = q;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    // gather 4 codes per lane into one word: lane j (< 8) writes codes 4j..4j+3
+    const uint32_t b = (uint32_t)(q & 0xff);
+    const uint32_t b0 = __shfl_sync(0xffffffffu, b, (lane * 4 + 0) & 31);
+    const uint32_t b1 = __shfl_sync(0xffffffffu, b, (lane * 4 + 1) & 31);
+    const uint32_t b2 = __shfl_sync(0xffffffffu, b, (lane * 4 + 2) & 31);
+    const uint32_t b3 = __shfl_sync(0xffffffffu, b, (lane * 4 + 3) & 31);
+    if (lane < 8)
+        reinterpret_cast<uint32_t*>(dst + 4)[lane] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    if (lane == 0) {
+        const uint32_t dh = f2h(d);
+        const uint32_t sh = f2h(__fmul_rn(d, (float)s));
+        reinterpret_cast<uint32_t*>(dst)[0] = dh | (sh << 16);
+    }
+}
+
+// ---- bulk copies and mbarriers (sm_90+ PTX, used on sm_100a) ------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Global -> shared bulk copy completing on an mbarrier's transaction count.
+// dst, src 16-byte aligned, bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for an mbarrier phase: gives up after budget_ns of wall time
+// (and a hard cap on polls), records kErrTimeout in *err and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
+                                                  uint64_t budget_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 0; i < (1u << 26); ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 255 && global_timer_ns() - t0 > budget_ns) break;
+    }
+    if (err) atomicExch(err, kErrTimeout);
+    return false;
+}
+
+// Programmatic dependent launch: wait for the upstream grid's memory, and let
+// the downstream grid start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    return *reinterpret_cast<const uint4*>(p);
+}
+
+}  // namespace elq

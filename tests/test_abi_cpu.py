@@ -1,0 +1,116 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol include/elq.h declares, reports its sizes, and refuses bad arguments on
+the host before any launch (every case here fails validation, so nothing is
+ever enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_latent_moe_b200 import build, elq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return elq.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "elq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(elq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(elq.SIGNATURES)
+
+
+def test_status_strings_and_version(L):
+    assert L.elq_version() == 1
+    assert L.elq_status_string(0) == b"ok"
+    assert L.elq_status_string(-4).startswith(b"workspace")
+    assert L.elq_status_string(123) == b"unknown status"
+
+
+def test_arena_bytes(L):
+    q, d = elq.SZ(), elq.SZ()
+    # an expert of the pages' synthetic 2560/640 shape: gate+up as 1280 rows? use the D of the decode shape
+    assert L.elq_arena_bytes(8, 1792, 4096, ctypes.byref(q), ctypes.byref(d)) == 1792 * 128 * 34
+    assert q.value == 1792 * 128 * 32 and d.value == 1792 * 128 * 2
+    assert L.elq_arena_bytes(2, 1280, 3072, None, None) == 1280 * 96 * 18
+    assert L.elq_arena_bytes(8, 100, 64, None, None) == 0          # rows not a multiple of 128
+    assert L.elq_arena_bytes(8, 128, 48, None, None) == 0          # k not a multiple of 32
+    assert L.elq_arena_bytes(3, 128, 64, None, None) == 0          # unknown format
+
+
+def _qm(fmt, rows, k, q=1 << 20, d=2 << 20):
+    return elq.QMat(fmt, rows, k, 0, q, d)
+
+
+def _layer(H=512, L_=256, E=8, k=2, I=256, fmt=8, **over):
+    base = 1 << 24
+    ly = elq.LayerC(H, L_, E, k, I, 0, _qm(fmt, L_, H, base, base + 4096), _qm(fmt, H, L_, base + 8192, base + 12288),
+                    base + 16384, None, _qm(fmt, E * 2 * I, L_, base + 20480, base + 24576),
+                    _qm(fmt, E * L_, I, base + 28672, base + 32768))
+    for k_, v in over.items():
+        setattr(ly, k_, v)
+    return ly
+
+
+def test_layer_validation(L):
+    ws_small = ctypes.c_void_p(1 << 26)
+    x = ctypes.c_void_p(1 << 27)
+    y = ctypes.c_void_p(1 << 28)
+    good = _layer()
+    assert L.elq_workspace_bytes(ctypes.byref(good), 4) > 0
+    # workspace too small -> refused before any launch
+    assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, ws_small, 16, None) == -4
+    assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, None, 1 << 30, None) == -4
+    assert L.elq_moe_layer(ctypes.byref(good), None, 0, 4, y, ws_small, 1 << 30, None) == -1
+    assert L.elq_moe_layer(ctypes.byref(good), x, 5, 4, y, ws_small, 1 << 30, None) == -2
+    assert L.elq_moe_layer(ctypes.byref(good), ctypes.c_void_p((1 << 27) + 2), 0, 4, y, ws_small, 1 << 30, None) == -3
+    assert L.elq_moe_layer(ctypes.byref(_layer(k=9)), x, 0, 4, y, ws_small, 1 << 30, None) == -1
+    assert L.elq_moe_layer(ctypes.byref(_layer(fmt=9)), x, 0, 4, y, ws_small, 1 << 30, None) == -2
+    assert L.elq_moe_layer(ctypes.byref(_layer(I=96)), x, 0, 4, y, ws_small, 1 << 30, None) == -2
+    bad = _layer()
+    bad.D = _qm(8, 256, 512, (1 << 20) + 16)
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws_small, 1 << 30, None) == -3
+    bad = _layer()
+    bad.U = _qm(8, 512, 128)
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws_small, 1 << 30, None) == -1
+    bad = _layer()
+    bad.router_w = None
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws_small, 1 << 30, None) == -1
+    assert L.elq_moe_layer(None, x, 0, 4, y, ws_small, 1 << 30, None) == -1
+    assert L.elq_moe_layer(ctypes.byref(good), x, 0, -1, y, ws_small, 1 << 30, None) == -1
+
+
+def test_other_entry_validation(L):
+    p = ctypes.c_void_p(1 << 24)
+    assert L.elq_quantize_q8_1(p, 0, 4, 48, p, None) == -2          # cols % 32
+    assert L.elq_quantize_q8_1(p, 7, 4, 64, p, None) == -2          # x type
+    assert L.elq_quantize_q8_1(None, 0, 4, 64, p, None) == -1
+    assert L.elq_quantize_q8_1(ctypes.c_void_p((1 << 24) + 1), 0, 4, 64, p, None) == -3
+    assert L.elq_router_topk(p, p, None, 1, 64, 8, 9, p, p, p, None) == -1     # k > E
+    assert L.elq_router_topk(p, p, None, 1, 64, 64, 33, p, p, p, None) == -2   # k > 32
+    assert L.elq_router_topk(p, p, None, 1, 64, 8, 2, p, p, None, None) == -1  # logits required
+    assert L.elq_route_bucket(p, 4, 2, 8, None, p, p, p, None) == -1
+    assert L.elq_route_bucket(p, 4, 9, 8, p, p, p, p, None) == -1
+    qm = _qm(8, 256, 512)
+    assert L.elq_latent_proj(ctypes.byref(qm), p, 2, p, None, 0, None) == -4
+    assert L.elq_latent_proj(ctypes.byref(_qm(4, 256, 512)), p, 2, p, p, 1 << 30, None) == -2
+    assert L.elq_latent_proj(ctypes.byref(_qm(8, 200, 512)), p, 2, p, p, 1 << 30, None) == -2
+    assert L.elq_arena_pack(8, p, 100, 64, p, p, None) == -2
+    assert L.elq_arena_pack(8, p, 128, 64, ctypes.c_void_p((1 << 24) + 16), p, None) == -3
+    assert L.elq_quantize_weights(2, p, 128, 40, p, p, None) == -2
+    assert L.elq_quantize_gate_up(8, p, p, 2, 96, 64, p, p, None) == -2
+    assert L.elq_test_block_isums(9, p, p, 4, p, p, None) == -2
+    assert L.elq_workspace_status(None, None) == -1
