@@ -39,7 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "latent-MoE layer tokens/s; expert-weight HBM GB/s and % of B200 peak"
-KERNELS = ["quant_x", "proj_D", "router", "gate_up", "down", "combine", "proj_U"]
+KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
+KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 
 
 def parse():
@@ -316,7 +317,8 @@ def run_elq(args):
             done += n
         return start + k
 
-    launches_per_step = elq.lib().elq_layer_kernel_count()
+    launches_per_step = layers[0].kernel_count(wl.T)
+    KERNELS = KERNELS_SMALL_T if launches_per_step == 5 else KERNELS_LARGE_T
     pos = run_steps(args.warmup)
     torch.cuda.synchronize()
     if world > 1:
@@ -359,24 +361,30 @@ def run_elq(args):
     torch.cuda.synchronize()
     e2e_ms = f0.elapsed_time(f1)
 
-    # per-kernel device time: the same steps with an event after every kernel
+    # per-kernel device time: the same steps with an event after every kernel.
+    # Eager launches behind a queued GPU sleep, so the host runs ahead and the
+    # kernels execute back to back (events cannot be timed inside a graph).
     nk = launches_per_step
     prof_steps = min(args.steps, 1024)
     per = [[] for _ in range(nk)]
-    GP = min(G, 64)
+    GP = 32
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(GP)]
-    gp = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gp):
-        for i in range(GP):
-            elq.moe_layer_profiled(layers[i % args.copies], xs[i % S], ys[i % 2], evs[i], ws)
-    gp.replay()
+    for row in evs:             # torch creates the CUDA event at its first record
+        for ev in row:
+            ev.record(stream)
     torch.cuda.synchronize()
-    for _ in range(max(1, prof_steps // GP)):
-        gp.replay()
+    done = 0
+    while done < prof_steps:
+        n = min(GP, prof_steps - done)
+        torch.cuda._sleep(20_000_000)
+        for i in range(n):
+            j = done + i
+            elq.moe_layer_profiled(layers[j % args.copies], xs[j % S], ys[j % 2], evs[i], ws)
         torch.cuda.synchronize()
-        for i in range(GP):
+        for i in range(n):
             for j in range(nk):
                 per[j].append(evs[i][j].elapsed_time(evs[i][j + 1]))
+        done += n
     t_wall1 = time.time()
     clocks = clk.stop(t_wall0, t_wall1)
     kern_ms = [statistics.mean(v) for v in per]
@@ -443,9 +451,7 @@ def run_elq(args):
         if world == 1 and not args.no_cpu:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, "cuda")
         print(json.dumps(line), flush=True)
-    for g in graphs.values():
-        del g
-    del gp
+    graphs.clear()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

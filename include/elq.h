@@ -54,17 +54,19 @@
  *
  * Device weight arena ("tile-slab" layout)
  *   A matrix of n_rows x k (n_rows % 128 == 0, k % 32 == 0, nb = k / 32) is
- *   stored as tiles of 128 rows.  For tile t and block column kb, slab
- *   s = t * nb + kb holds:
- *     q : Q8_0 -- 4096 bytes at q + 4096 s: the 128 x 32 int8 codes as 8-row x
- *         16-byte core matrices; code i of local row r sits at byte
- *         (r/8)*256 + (i/16)*128 + (r%8)*16 + (i%16).  This is the K-major,
- *         no-swizzle operand layout of the tcgen05 tensor cores (leading byte
- *         offset 128, stride byte offset 256), so a slab is one bulk copy.
- *         Q4_0 -- 2048 bytes at q + 2048 s: local row r's 16 nibble bytes at
- *         byte 16 r, in the block's own order.
- *     d : 128 fp16 scales at d + 256 s (local row r at element r).
- *   q and d must be 256-byte aligned.
+ *   stored as tiles of 128 rows, each tile as four slices of 32 rows, and each
+ *   slice as its nb blocks one after another.  For tile t, slice s (rows
+ *   128 t + 32 s .. +31), block kb and local row r (0..31):
+ *     q : Q8_0 -- a 1024-byte piece at q + t*nb*4096 + s*nb*1024 + kb*1024;
+ *         code i of row r sits at byte (r/8)*256 + (i/16)*128 + (r%8)*16 +
+ *         (i%16) of the piece: 8-row x 16-byte core matrices, the K-major
+ *         no-swizzle operand layout of the tcgen05 tensor cores.
+ *         Q4_0 -- a 512-byte piece at q + t*nb*2048 + s*nb*512 + kb*512; row
+ *         r's 16 nibble bytes at byte 16 r of the piece, in the block's order.
+ *     d : fp16 scale at element t*nb*128 + s*nb*32 + kb*32 + r.
+ *   So the 8 blocks of a 32-row slice that one warp of the decode kernels
+ *   reads are one contiguous bulk copy.  q and d must be 256-byte aligned.
+ *   The layer's matrices (and elq_latent_proj's) need k % 128 == 0.
  *
  * Layer weights
  *   D      : L rows x H;   U : H rows x L  (any weight format each)
@@ -200,10 +202,12 @@ size_t elq_workspace_bytes(const elq_layer* layer, int32_t T);
 elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T,
                          float* y, void* ws, size_t ws_bytes, void* stream);
 
-/* Number of kernels one elq_moe_layer call launches, in order: activation
- * quantiser, D projection (+ latent Q8_1), router (+ top-k, bucketing),
- * gate/up (+ SwiGLU, Q8_1), down, combine (+ Q8_1), U projection. */
-int32_t elq_layer_kernel_count(void);
+/* Number of kernels one elq_moe_layer call launches at this T (0 if the
+ * layer is invalid), in order: [activation quantiser, for T > 8], D projection
+ * (quantising x itself for T <= 8; + latent Q8_1), router (+ top-k,
+ * bucketing), gate/up (+ SwiGLU, Q8_1), down (+ weighted combine, Q8_1), U
+ * projection. */
+int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T);
 
 /* elq_moe_layer that also records CUDA events on the stream: events[0] before
  * the first kernel and events[i] after kernel i (i = 1 .. kernel count), so

@@ -494,7 +494,15 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trac
 }
 
 /* ------------------------------------------------------------------------ */
-/* device arena layout, written out element by element                       */
+/* device arena layout, written out element by element.
+ * Rows in tiles of 128, each tile in four slices of 32 rows; per (tile,
+ * slice) the blocks kb = 0 .. nb-1 follow one another:
+ *   Q8_0 codes: 1024 bytes per (tile, slice, kb) at
+ *       tile*nb*4096 + slice*nb*1024 + kb*1024 + (r/8)*256 + (i/16)*128 + (r%8)*16 + (i%16)
+ *       for local row r (0..31) of the slice and code i (0..31) of the block;
+ *   Q4_0 codes: 512 bytes per (tile, slice, kb) at
+ *       tile*nb*2048 + slice*nb*512 + kb*512 + r*16 + j (the block's 16 nibble bytes);
+ *   scales: fp16 element tile*nb*128 + slice*nb*32 + kb*32 + r. */
 
 void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
                     uint8_t* q_out, uint8_t* d_out)
@@ -502,21 +510,20 @@ void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
     int nb = k / 32;
     int wb = orc_block_bytes(fmt);
     for (int row = 0; row < n_rows; ++row) {
-        int tile = row / 128, r = row % 128;
+        int tile = row / 128, slice = (row % 128) / 32, r = row % 32;
         for (int kb = 0; kb < nb; ++kb) {
             const uint8_t* blk = aos + ((int64_t)row * nb + kb) * wb;
-            int64_t slab = (int64_t)tile * nb + kb;
-            /* scale: fp16 at index slab*128 + r */
-            d_out[(slab * 128 + r) * 2] = blk[0];
-            d_out[(slab * 128 + r) * 2 + 1] = blk[1];
+            int64_t sel = (int64_t)tile * nb * 128 + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r;
+            d_out[sel * 2] = blk[0];
+            d_out[sel * 2 + 1] = blk[1];
             if (fmt == ORC_Q8_0) {
-                for (int i = 0; i < 32; ++i) {
-                    int64_t off = slab * 4096 + (r / 8) * 256 + (i / 16) * 128 + (r % 8) * 16 + (i % 16);
-                    q_out[off] = blk[2 + i];
-                }
+                int64_t base = (int64_t)tile * nb * 4096 + (int64_t)slice * nb * 1024 + (int64_t)kb * 1024;
+                for (int i = 0; i < 32; ++i)
+                    q_out[base + (r / 8) * 256 + (i / 16) * 128 + (r % 8) * 16 + (i % 16)] = blk[2 + i];
             } else {
+                int64_t base = (int64_t)tile * nb * 2048 + (int64_t)slice * nb * 512 + (int64_t)kb * 512;
                 for (int j = 0; j < 16; ++j)
-                    q_out[slab * 2048 + r * 16 + j] = blk[2 + j];
+                    q_out[base + r * 16 + j] = blk[2 + j];
             }
         }
     }

@@ -146,11 +146,11 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y,
  * can learn which experts a token set needs before supplying them. */
 int orc_route(const orc_layer* ly, const float* x, int T, int32_t* idx, float* w);
 
-/* The device arena layout, stated plainly (see elq.h of the library for the
- * definition): rows in tiles of 128, per (tile, block) a 4096-byte Q8_0 slab
- * in 8x16-byte core-matrix order, or a 2048-byte Q4_0 slab of 16-byte rows,
- * and a 256-byte slab of fp16 scales.  aos is row-major AoS blocks.
- * n_rows % 128 == 0. */
+/* The device arena layout, stated plainly (the definition is written out in
+ * elq_oracle.c): tiles of 128 rows, four 32-row slices per tile, per slice
+ * its blocks one after another (1024-byte Q8_0 or 512-byte Q4_0 pieces) and a
+ * parallel array of fp16 scales.  aos is row-major AoS blocks; n_rows % 128
+ * == 0. */
 void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
                     uint8_t* q_out, uint8_t* d_out);
 

@@ -17,7 +17,9 @@ namespace {
 
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per bounded device wait
 constexpr int kMaxDevices = 64;
-constexpr int kLayerKernels = 7;   // quant, D, router, gate/up, down, combine, U
+constexpr int kRouterSmemMax = 200 * 1024;           // dynamic shared memory cap of router/bucket
+constexpr int kGemvSmemMax = 225 * 1024;             // dynamic shared memory cap of the GEMV
+constexpr int kRawMaxT = 8;                          // D quantises x itself up to this many tokens
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -37,15 +39,18 @@ int sm_count() {
 
 // Opt a kernel in to large dynamic shared memory once per device.
 template <typename K>
-cudaError_t smem_optin(K kern, int bytes, uint64_t* done_mask_per_dev) {
+cudaError_t smem_optin(K kern, int bytes, bool* done_per_dev) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && (done_mask_per_dev[dev] >> 0 & 1ull)) return cudaSuccess;
+    if (dev >= 0 && dev < kMaxDevices && done_per_dev[dev]) return cudaSuccess;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done_mask_per_dev[dev] |= 1ull;
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done_per_dev[dev] = true;
     return e;
 }
+
+bool g_optin_w8[kMaxDevices], g_optin_w2[kMaxDevices], g_optin_router[kMaxDevices], g_optin_bucket[kMaxDevices],
+    g_optin_topk[kMaxDevices];
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
@@ -73,7 +78,7 @@ elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k) {
     if (!w) return ELQ_ERR_INVALID_ARG;
     if (!fmt_ok(w->fmt)) return ELQ_ERR_UNSUPPORTED;
     if (w->n_rows != rows || w->k != k || rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
-    if (rows % kTileRows || k % 32) return ELQ_ERR_UNSUPPORTED;
+    if (rows % kTileRows || k % 128) return ELQ_ERR_UNSUPPORTED;
     if (!w->q || !w->d) return ELQ_ERR_INVALID_ARG;
     if (!aligned(w->q, 256) || !aligned(w->d, 256)) return ELQ_ERR_ALIGNMENT;
     return ELQ_OK;
@@ -82,56 +87,75 @@ elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k) {
 // ---------------------------------------------------------------------------
 // GEMV planning
 
-struct GemvPlan {
-    int split;      // 1: per-chunk units with ordered partial completion
-    int grid;
-    size_t partial_bytes;
-    size_t counter_ints;
+struct WPlan {
+    int warps, stages, tokcap, stage_bytes, act_off, act_bytes, scratch_bytes, smem, grid;
+    int nchunks, tiles;
+    size_t partial_bytes, counter_ints;
 };
 
-// groups_max: upper bound on active groups (1 for dense); tok_rows: rows of
-// the partial buffer's token dimension (T or P).
-GemvPlan plan_gemv(int n_rows_per_group, int k, int groups_max, int64_t tok_rows) {
-    GemvPlan p;
-    const int sms = sm_count();
-    const int tiles = n_rows_per_group / kTileRows;
-    const int nchunks = (k / 32 + kChunk - 1) / kChunk;
-    const int64_t units_whole = (int64_t)groups_max * tiles;
-    p.split = (units_whole < 2 * sms && nchunks > 1) ? 1 : 0;
-    p.grid = sms;
-    p.partial_bytes = p.split ? (size_t)nchunks * tok_rows * tiles * kTileRows * sizeof(float) : 0;
-    p.counter_ints = p.split ? (size_t)groups_max * tiles : 0;
+// rows_per_group: matrix rows of one group; k: reduction length; groups_max:
+// bound on active groups; tok_rows: rows of the partial buffer's token
+// dimension (T or T*k); tokmax: most tokens one group can hold.
+WPlan plan_w(int fmt, int x_mode, int rows_per_group, int k, int groups_max, int64_t tok_rows, int tokmax) {
+    WPlan p;
+    p.tiles = rows_per_group / kTileRows;
+    p.nchunks = (k / 32 + kChunk - 1) / kChunk;
+    p.tokcap = std::max(1, std::min(tokmax, kTokMax));
+    p.act_bytes = (x_mode == X_RAW_F32) ? 1024 : (x_mode == X_RAW_BF16) ? 512 : kChunk * 36;
+    const int codes = kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
+    p.act_off = codes + kChunk * 64;
+    p.stage_bytes = (int)round_up((size_t)p.act_off + (size_t)p.tokcap * p.act_bytes, 128);
+    p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)p.tokcap * 288, 128) : 0;
+    static const int cand[][2] = {{8, 3}, {8, 2}, {4, 2}, {2, 2}, {1, 2}};
+    p.warps = 0;
+    for (const auto& c : cand) {
+        const long need = 512 + (long)c[0] * (c[1] * p.stage_bytes + p.scratch_bytes);
+        if (need <= kGemvSmemMax) {
+            p.warps = c[0];
+            p.stages = c[1];
+            p.smem = (int)need;
+            break;
+        }
+    }
+    p.grid = sm_count();
+    p.partial_bytes = (size_t)p.nchunks * tok_rows * p.tiles * kTileRows * sizeof(float);
+    p.counter_ints = (size_t)groups_max * p.tiles;
     return p;
 }
 
-uint64_t g_smem_done_q80[kMaxDevices], g_smem_done_q40[kMaxDevices], g_smem_done_router[kMaxDevices],
-    g_smem_done_bucket[kMaxDevices];
-
-cudaError_t launch_gemv(const GemvArgs& g, int fmt, int grid, cudaStream_t s, bool pdl) {
+cudaError_t launch_w(WArgs g, int fmt, const WPlan& p, cudaStream_t s, bool pdl) {
+    g.stages = p.stages;
+    g.tokcap = p.tokcap;
+    g.stage_bytes = p.stage_bytes;
+    g.act_off = p.act_off;
+    g.act_bytes = p.act_bytes;
+    g.scratch_bytes = p.scratch_bytes;
+    g.nchunks = p.nchunks;
+    g.tiles = p.tiles;
+    g.budget_ns = kWaitBudgetNs;
+    if (p.warps == 0) return cudaErrorInvalidConfiguration;
     if (fmt == ELQ_Q8_0) {
-        cudaError_t e = smem_optin(k_qgemv<8>, GemvSmem<8>::kTotal, g_smem_done_q80);
+        cudaError_t e = smem_optin(k_wgemv<8>, kGemvSmemMax, g_optin_w8);
         if (e != cudaSuccess) return e;
-        return launch(k_qgemv<8>, dim3(grid), dim3(kGemvThreads), GemvSmem<8>::kTotal, s, pdl, g);
+        return launch(k_wgemv<8>, dim3(p.grid), dim3(32 * p.warps), p.smem, s, pdl, g);
     }
-    cudaError_t e = smem_optin(k_qgemv<2>, GemvSmem<2>::kTotal, g_smem_done_q40);
+    cudaError_t e = smem_optin(k_wgemv<2>, kGemvSmemMax, g_optin_w2);
     if (e != cudaSuccess) return e;
-    return launch(k_qgemv<2>, dim3(grid), dim3(kGemvThreads), GemvSmem<2>::kTotal, s, pdl, g);
+    return launch(k_wgemv<2>, dim3(p.grid), dim3(32 * p.warps), p.smem, s, pdl, g);
 }
 
-GemvArgs dense_args(const elq_qmat* w, int T, const void* x, int out_mode, float* y, uint8_t* yq,
-                    const GemvPlan& pl, float* partial, int* counters, int* err) {
-    GemvArgs g;
+WArgs dense_w(const elq_qmat* w, int T, const void* x, int x_mode, int64_t x_row, int out_mode, float* y,
+              uint8_t* yq, float* partial, int* counters, int* err) {
+    WArgs g;
     std::memset(&g, 0, sizeof(g));
     g.q = static_cast<const uint8_t*>(w->q);
     g.d = static_cast<const uint16_t*>(w->d);
     g.nb = w->k / 32;
-    g.tiles = w->n_rows / kTileRows;
-    g.nchunks = (g.nb + kChunk - 1) / kChunk;
-    g.split = pl.split;
-    g.T = T;
     g.kslots = 1;
-    g.x = static_cast<const uint8_t*>(x);
-    g.x_mode = X_DENSE;
+    g.T = T;
+    g.x = x;
+    g.x_mode = x_mode;
+    g.x_row = x_row;
     g.out_mode = out_mode;
     g.y = y;
     g.y_ld = w->n_rows;
@@ -141,7 +165,6 @@ GemvArgs dense_args(const elq_qmat* w, int T, const void* x, int out_mode, float
     g.part_tok = T;
     g.counters = counters;
     g.err = err;
-    g.budget_ns = kWaitBudgetNs;
     return g;
 }
 
@@ -162,29 +185,30 @@ struct ProjWs {
     int* err;
     int* counters;
     float* partial;
+    WPlan plan;
     size_t total;
 };
 
-ProjWs proj_layout(const elq_qmat* w, int T, void* base, GemvPlan* plan_out) {
-    GemvPlan pl = plan_gemv(w->n_rows, w->k, 1, T);
-    Carve c;
+ProjWs proj_layout(const elq_qmat* w, int T, void* base) {
     ProjWs ws;
-    ws.err = c.take<int>(base, 256 + pl.counter_ints * sizeof(int));
+    ws.plan = plan_w(w->fmt, X_Q81_TOKEN, w->n_rows, w->k, 1, T, T);
+    Carve c;
+    ws.err = c.take<int>(base, (64 + ws.plan.counter_ints) * sizeof(int));
     ws.counters = ws.err ? ws.err + 64 : nullptr;
-    ws.partial = c.take<float>(base, pl.partial_bytes);
+    ws.partial = c.take<float>(base, ws.plan.partial_bytes);
     ws.total = c.off;
-    if (plan_out) *plan_out = pl;
     return ws;
 }
 
 struct LayerWs {
     int* err;               // error word, then counters
     int* cnt_router;        // ceil(T/8) + 1
-    int* cnt_d;             // D projection tiles
-    int* cnt_gu;            // gate/up (group, tile)
-    int* cnt_dn;            // down
-    int* cnt_u;             // U projection
-    uint8_t* xq;
+    int* cnt_d;
+    int* cnt_gu;
+    int* cnt_dn;
+    int* cnt_u;
+    int* cnt_comb;          // [T][L/128]
+    uint8_t* xq;            // only when T > kRawMaxT
     float* z;
     uint8_t* zq;
     float* logits;
@@ -196,22 +220,25 @@ struct LayerWs {
     float* ylat;
     uint8_t* ylq;
     float* partial;
-    GemvPlan pd, pgu, pdn, pu;
+    WPlan pd, pgu, pdn, pu;
+    bool raw;
     size_t total;
 };
 
-LayerWs layer_layout(const elq_layer* ly, int T, void* base) {
+LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     LayerWs w;
     const int H = ly->H, L = ly->L, E = ly->E, k = ly->k, I = ly->I;
     const int64_t P = (int64_t)T * k;
     const int gmax = (int)std::min<int64_t>(E, P);
-    w.pd = plan_gemv(L, H, 1, T);
-    w.pgu = plan_gemv(2 * I, L, gmax, P);
-    w.pdn = plan_gemv(L, I, gmax, P);
-    w.pu = plan_gemv(H, L, 1, T);
+    w.raw = T <= kRawMaxT;
+    const int dmode = w.raw ? (x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32) : X_Q81_TOKEN;
+    w.pd = plan_w(ly->D.fmt, dmode, L, H, 1, T, T);
+    w.pgu = plan_w(ly->gate_up.fmt, X_Q81_PAIR_TOKEN, 2 * I, L, gmax, P, T);
+    w.pdn = plan_w(ly->down.fmt, X_Q81_POSITION, L, I, gmax, P, T);
+    w.pu = plan_w(ly->U.fmt, X_Q81_TOKEN, H, L, 1, T, T);
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     const size_t n_cnt = 64 + (rblocks + 1) + w.pd.counter_ints + w.pgu.counter_ints + w.pdn.counter_ints +
-                         w.pu.counter_ints;
+                         w.pu.counter_ints + (size_t)T * (L / kTileRows);
     Carve c;
     w.err = c.take<int>(base, n_cnt * sizeof(int));
     int* cur = w.err ? w.err + 64 : nullptr;
@@ -221,7 +248,8 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base) {
     w.cnt_gu = adv(w.pgu.counter_ints);
     w.cnt_dn = adv(w.pdn.counter_ints);
     w.cnt_u = adv(w.pu.counter_ints);
-    w.xq = c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
+    w.cnt_comb = adv((size_t)T * (L / kTileRows));
+    w.xq = w.raw ? nullptr : c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
     w.z = c.take<float>(base, (size_t)T * L * 4);
     w.zq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
     w.logits = c.take<float>(base, (size_t)T * E * 4);
@@ -251,7 +279,7 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     if (H <= 0 || L <= 0 || E <= 0 || k <= 0 || I <= 0) return ELQ_ERR_INVALID_ARG;
     if (k > E) return ELQ_ERR_INVALID_ARG;
     if (k > 32 || E > 1024) return ELQ_ERR_UNSUPPORTED;
-    if (H % kTileRows || L % kTileRows || I % 64) return ELQ_ERR_UNSUPPORTED;
+    if (H % kTileRows || L % kTileRows || I % kTileRows) return ELQ_ERR_UNSUPPORTED;
     if ((int64_t)T * k > (int64_t)1 << 30) return ELQ_ERR_UNSUPPORTED;
     elq_status s;
     if ((s = check_qmat(&ly->D, L, H)) != ELQ_OK) return s;
@@ -266,31 +294,75 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
 
 size_t router_smem(int T, int L, int E) {
     const int nt = std::min(T, kRouterTok);
-    size_t a = (size_t)nt * L * 4;
-    size_t b = (size_t)kRouterWarps * E * 4;
+    const size_t a = (size_t)(nt + kRouterWarps) * L * 4;
+    const size_t b = (size_t)kRouterWarps * E * 4;
     return std::max(a, b);
 }
+
+bool router_shape_ok(int T, int L, int E) { return router_smem(T, L, E) <= (size_t)kRouterSmemMax; }
 
 cudaError_t launch_router(const float* z, const float* w, const float* bias, int T, int L, int E, int k,
                           int32_t* idx, float* wts, float* logits, int* cnt, bool do_bucket, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* pos, int32_t* act, int32_t* n_act,
-                          cudaStream_t s, bool pdl) {
+                          cudaStream_t s, bool pdl, int* err = nullptr) {
     RouterArgs a;
-    a.z = z; a.w = w; a.bias = bias; a.T = T; a.L = L; a.E = E; a.k = k;
-    a.idx = idx; a.wts = wts; a.logits = logits;
+    std::memset(&a, 0, sizeof(a));
+    a.err = err;
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     a.cnt_tok = cnt;
     a.cnt_all = cnt ? cnt + rblocks : nullptr;
     a.do_bucket = do_bucket ? 1 : 0;
     a.counts = counts; a.offsets = offsets; a.perm = perm; a.pos = pos; a.act = act; a.n_act = n_act;
-    const size_t sm = router_smem(T, L, E);
-    cudaError_t e = smem_optin(k_router, 227 * 1024, g_smem_done_router);
+    cudaError_t e = smem_optin(k_router, kRouterSmemMax, g_optin_router);
     if (e != cudaSuccess) return e;
     dim3 grid((E + kRouterWarps - 1) / kRouterWarps, rblocks);
-    return launch(k_router, grid, dim3(kRouterWarps * 32), sm, s, pdl, a);
+    return launch(k_router, grid, dim3(kRouterWarps * 32), router_smem(T, L, E), s, pdl, a);
 }
 
-bool router_shape_ok(int T, int L, int E) { return router_smem(T, L, E) <= 227 * 1024; }
+// Kernel sequence of the grouped experts (gate/up, then down with the combine)
+// routing_early_down: the routing was produced two kernels before the down
+// projection (by the router, not by a bucketing kernel right before gate/up
+// whose completion the down kernel could not otherwise rely on).
+elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, const float* wts,
+                       float* y_lat, cudaStream_t s, bool pdl, const std::function<bool()>& mark,
+                       bool routing_early_down) {
+    const int L = ly->L, k = ly->k, I = ly->I;
+    const int64_t P = (int64_t)T * k;
+    WArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.q = static_cast<const uint8_t*>(ly->gate_up.q);
+    g.d = static_cast<const uint16_t*>(ly->gate_up.d);
+    g.nb = L / 32;
+    g.q_gstride = (int64_t)(2 * I / kTileRows) * g.nb * slab_bytes(ly->gate_up.fmt);
+    g.d_gstride = (int64_t)(2 * I / kTileRows) * g.nb * kTileRows;
+    g.act = w.act; g.n_act = w.n_act; g.offsets = w.offsets; g.perm = w.perm; g.kslots = k; g.T = T;
+    g.x = zq; g.x_mode = X_Q81_PAIR_TOKEN;
+    g.out_mode = OUT_SWIGLU;
+    g.yq = w.hq; g.yq_ld = I / 32;
+    g.partial = w.partial; g.part_tok = P; g.counters = w.cnt_gu; g.err = w.err;
+    if (launch_w(g, ly->gate_up.fmt, w.pgu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    WArgs h;
+    std::memset(&h, 0, sizeof(h));
+    h.q = static_cast<const uint8_t*>(ly->down.q);
+    h.d = static_cast<const uint16_t*>(ly->down.d);
+    h.nb = I / 32;
+    h.q_gstride = (int64_t)(L / kTileRows) * h.nb * slab_bytes(ly->down.fmt);
+    h.d_gstride = (int64_t)(L / kTileRows) * h.nb * kTileRows;
+    h.act = w.act; h.n_act = w.n_act; h.offsets = w.offsets; h.perm = w.perm; h.kslots = k; h.T = T;
+    h.x = w.hq; h.x_mode = X_Q81_POSITION;
+    h.out_mode = OUT_F32_COMBINE;
+    h.y = w.o; h.y_ld = L;
+    h.wts = wts; h.pos = w.pos; h.cnt_comb = w.cnt_comb; h.ylat = y_lat; h.ylq = w.ylq;
+    h.partial = w.partial; h.part_tok = P; h.counters = w.cnt_dn; h.err = w.err;
+    h.routing_early = routing_early_down ? 1 : 0;
+    if (launch_w(h, ly->down.fmt, w.pdn, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    return ELQ_OK;
+}
+
+elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
+                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events);
+
+int layer_kernels(int T) { return T <= kRawMaxT ? 5 : 6; }
 
 }  // namespace
 
@@ -402,13 +474,15 @@ elq_status elq_router_topk(const float* z, const float* w_router, const float* b
     if (k > 32 || E > 1024 || L % 32) return ELQ_ERR_UNSUPPORTED;
     if (T == 0) return ELQ_OK;
     if (!z || !w_router || !idx || !weights || !logits) return ELQ_ERR_INVALID_ARG;
-    if (!aligned(z, 4) || !aligned(w_router, 4) || (bias && !aligned(bias, 4)) || !aligned(idx, 4) ||
+    if (!aligned(z, 16) || !aligned(w_router, 16) || (bias && !aligned(bias, 4)) || !aligned(idx, 4) ||
         !aligned(weights, 4) || !aligned(logits, 4))
         return ELQ_ERR_ALIGNMENT;
     if (!router_shape_ok(T, L, E)) return ELQ_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_router(z, w_router, bias, T, L, E, k, idx, weights, logits, nullptr, false, nullptr,
                                   nullptr, nullptr, nullptr, nullptr, nullptr, s, false);
+    if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    e = smem_optin(k_topk, kRouterSmemMax, g_optin_topk);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
     e = launch(k_topk, dim3((T + 3) / 4), dim3(128), (size_t)4 * E * 4, s, true, (const float*)logits, (int)T,
                (int)E, (int)k, idx, weights);
@@ -425,7 +499,7 @@ elq_status elq_route_bucket(const int32_t* idx, int32_t T, int32_t k, int32_t E,
         (pos && !aligned(pos, 4)))
         return ELQ_ERR_ALIGNMENT;
     const int nw = 32;
-    cudaError_t e = smem_optin(k_bucket, 227 * 1024, g_smem_done_bucket);
+    cudaError_t e = smem_optin(k_bucket, kRouterSmemMax, g_optin_bucket);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
     e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, static_cast<cudaStream_t>(stream), false, idx,
                (int)(T * k), (int)E, counts, offsets, perm, pos, (int32_t*)nullptr, (int32_t*)nullptr);
@@ -433,9 +507,9 @@ elq_status elq_route_bucket(const int32_t* idx, int32_t T, int32_t k, int32_t E,
 }
 
 size_t elq_latent_proj_workspace_bytes(const elq_qmat* w, int32_t T) {
-    if (!w || T <= 0 || check_qmat(w, w->n_rows, w->k) == ELQ_ERR_UNSUPPORTED) return 0;
-    if (!fmt_ok(w->fmt) || w->n_rows <= 0 || w->k <= 0 || w->n_rows % kTileRows || w->k % 32) return 0;
-    return proj_layout(w, T, nullptr, nullptr).total;
+    if (!w || T <= 0) return 0;
+    if (!fmt_ok(w->fmt) || w->n_rows <= 0 || w->k <= 0 || w->n_rows % kTileRows || w->k % 128) return 0;
+    return proj_layout(w, T, nullptr).total;
 }
 
 elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y, void* ws, size_t ws_bytes,
@@ -446,66 +520,18 @@ elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, flo
     if (T < 0) return ELQ_ERR_INVALID_ARG;
     if (T == 0) return ELQ_OK;
     if (!x_q8_1 || !y) return ELQ_ERR_INVALID_ARG;
-    if (!aligned(x_q8_1, 4) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
-    GemvPlan pl;
-    ProjWs lay = proj_layout(w, T, ws, &pl);
+    if (!aligned(x_q8_1, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
+    ProjWs lay = proj_layout(w, T, ws);
     if (!ws || ws_bytes < lay.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
-    GemvArgs g = dense_args(w, T, x_q8_1, OUT_F32, y, nullptr, pl, lay.partial, lay.counters, lay.err);
-    return cuda_status(launch_gemv(g, w->fmt, pl.grid, static_cast<cudaStream_t>(stream), false));
+    WArgs g = dense_w(w, T, x_q8_1, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, lay.partial, lay.counters, lay.err);
+    return cuda_status(launch_w(g, w->fmt, lay.plan, static_cast<cudaStream_t>(stream), false));
 }
 
 size_t elq_workspace_bytes(const elq_layer* layer, int32_t T) {
     if (check_layer(layer, T) != ELQ_OK || T <= 0) return 0;
-    return layer_layout(layer, T, nullptr).total;
-}
-
-static elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, float* y_lat,
-                              cudaStream_t s, bool pdl, std::function<bool()> mark = std::function<bool()>()) {
-    auto marked = [&]() { return !mark || mark(); };
-    const int L = ly->L, k = ly->k, I = ly->I;
-    const int64_t P = (int64_t)T * k;
-    // a6 + a7: gate/up with SwiGLU and Q8_1 requant -> hq by pair position
-    GemvArgs g;
-    std::memset(&g, 0, sizeof(g));
-    g.q = static_cast<const uint8_t*>(ly->gate_up.q);
-    g.d = static_cast<const uint16_t*>(ly->gate_up.d);
-    g.nb = L / 32;
-    g.tiles = 2 * I / kTileRows;
-    g.nchunks = (g.nb + kChunk - 1) / kChunk;
-    g.q_gstride = (int64_t)g.tiles * g.nb * slab_bytes(ly->gate_up.fmt);
-    g.d_gstride = (int64_t)g.tiles * g.nb * kTileRows;
-    g.split = w.pgu.split;
-    g.act = w.act; g.n_act = w.n_act; g.offsets = w.offsets; g.perm = w.perm; g.kslots = k; g.T = T;
-    g.x = zq; g.x_mode = X_PAIR_TOKEN;
-    g.out_mode = OUT_SWIGLU;
-    g.yq = w.hq; g.yq_ld = I / 32;
-    g.partial = w.partial; g.part_tok = P; g.counters = w.cnt_gu; g.err = w.err; g.budget_ns = kWaitBudgetNs;
-    cudaError_t e = launch_gemv(g, ly->gate_up.fmt, w.pgu.grid, s, pdl);
-    if (e != cudaSuccess || !marked()) return ELQ_ERR_CUDA;
-    // a8: down -> o by pair position
-    GemvArgs h;
-    std::memset(&h, 0, sizeof(h));
-    h.q = static_cast<const uint8_t*>(ly->down.q);
-    h.d = static_cast<const uint16_t*>(ly->down.d);
-    h.nb = I / 32;
-    h.tiles = L / kTileRows;
-    h.nchunks = (h.nb + kChunk - 1) / kChunk;
-    h.q_gstride = (int64_t)h.tiles * h.nb * slab_bytes(ly->down.fmt);
-    h.d_gstride = (int64_t)h.tiles * h.nb * kTileRows;
-    h.split = w.pdn.split;
-    h.act = w.act; h.n_act = w.n_act; h.offsets = w.offsets; h.perm = w.perm; h.kslots = k; h.T = T;
-    h.x = w.hq; h.x_mode = X_POSITION;
-    h.out_mode = OUT_F32;
-    h.y = w.o; h.y_ld = L;
-    h.partial = w.partial; h.part_tok = P; h.counters = w.cnt_dn; h.err = w.err; h.budget_ns = kWaitBudgetNs;
-    e = launch_gemv(h, ly->down.fmt, w.pdn.grid, s, pdl);
-    if (e != cudaSuccess || !marked()) return ELQ_ERR_CUDA;
-    // a9: combine + Q8_1
-    e = launch(k_combine, dim3(T, (L + 255) / 256), dim3(256), 0, s, pdl, (const float*)w.o,
-               (const int32_t*)w.pos, (const float*)w.wts, k, L, y_lat, w.ylq);
-    if (e != cudaSuccess || !marked()) return ELQ_ERR_CUDA;
-    return ELQ_OK;
+    // the larger of the two input types' layouts
+    return std::max(layer_layout(layer, T, nullptr, ELQ_F32).total, layer_layout(layer, T, nullptr, ELQ_BF16).total);
 }
 
 elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, const int32_t* idx,
@@ -515,72 +541,22 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     if (st != ELQ_OK) return st;
     if (T == 0) return ELQ_OK;
     if (!z_q8_1 || !idx || !weights || !y_lat) return ELQ_ERR_INVALID_ARG;
-    if (!aligned(z_q8_1, 4) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y_lat, 16))
+    if (!aligned(z_q8_1, 16) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y_lat, 16))
         return ELQ_ERR_ALIGNMENT;
-    LayerWs w = layer_layout(layer, T, ws);
+    LayerWs w = layer_layout(layer, T, ws, ELQ_F32);
     if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int E = layer->E, k = layer->k;
     const int64_t P = (int64_t)T * k;
-    // bucketing on one CTA; the combine reads the caller's weights
     const int nw = 32;
-    cudaError_t e = smem_optin(k_bucket, 227 * 1024, g_smem_done_bucket);
+    cudaError_t e = smem_optin(k_bucket, kRouterSmemMax, g_optin_bucket);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
-    e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, s, false, idx, (int)P, E, w.counts,
-               w.offsets, w.perm, w.pos, w.act, w.n_act);
+    e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, s, false, idx, (int)P, E, w.counts, w.offsets,
+               w.perm, w.pos, w.act, w.n_act);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
-    LayerWs w2 = w;
-    w2.wts = const_cast<float*>(weights);
-    return run_experts(layer, w2, T, static_cast<const uint8_t*>(z_q8_1), y_lat, s, true);
-}
-
-static elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
-                            size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
-    elq_status st = check_layer(layer, T);
-    if (st != ELQ_OK) return st;
-    if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
-    if (T == 0) return ELQ_OK;
-    if (!x || !y) return ELQ_ERR_INVALID_ARG;
-    if (!aligned(x, 4) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
-    if (events && n_events < kLayerKernels + 1) return ELQ_ERR_INVALID_ARG;
-    if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
-    LayerWs w = layer_layout(layer, T, ws);
-    if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
-    if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int H = layer->H, L = layer->L, E = layer->E, k = layer->k;
-    int ev = 0;
-    auto mark = [&]() -> bool {
-        if (!events) return true;
-        return cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s) == cudaSuccess;
-    };
-    const bool pdl = (events == nullptr);
-    cudaError_t e;
-    if (!mark()) return ELQ_ERR_CUDA;
-    // a1
-    const int64_t nblk = (int64_t)T * (H / 32);
-    if (x_type == ELQ_BF16)
-        e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x, nblk,
-                   w.xq);
-    else
-        e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
-                   nblk, w.xq);
-    if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
-    // a2 + a4: z and zq
-    GemvArgs gd = dense_args(&layer->D, T, w.xq, OUT_F32_Q81, w.z, w.zq, w.pd, w.partial, w.cnt_d, w.err);
-    if (launch_gemv(gd, layer->D.fmt, w.pd.grid, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
-    // a3 + a5
-    e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits, w.cnt_router,
-                      true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl);
-    if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
-    // a6 - a9
-    st = run_experts(layer, w, T, w.zq, w.ylat, s, pdl, events ? [&]() { return mark(); } : std::function<bool()>());
-    if (st != ELQ_OK) return st;
-    // a10
-    GemvArgs gu = dense_args(&layer->U, T, w.ylq, OUT_F32, y, nullptr, w.pu, w.partial, w.cnt_u, w.err);
-    if (launch_gemv(gu, layer->U.fmt, w.pu.grid, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
-    return ELQ_OK;
+    return run_experts(layer, w, T, static_cast<const uint8_t*>(z_q8_1), weights, y_lat, s, true,
+                       []() { return true; }, true);
 }
 
 elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
@@ -588,12 +564,16 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
     return run_layer(layer, x, x_type, T, y, ws, ws_bytes, stream, nullptr, 0);
 }
 
-int32_t elq_layer_kernel_count(void) { return kLayerKernels; }
+int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T) {
+    if (check_layer(layer, T) != ELQ_OK || T <= 0) return 0;
+    return layer_kernels(T);
+}
 
 elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y,
                                   void* ws, size_t ws_bytes, void* const* events, int32_t n_events, void* stream) {
-    if (!events) return ELQ_ERR_INVALID_ARG;
-    for (int i = 0; i < n_events && i < kLayerKernels + 1; ++i)
+    if (!events || T <= 0) return ELQ_ERR_INVALID_ARG;
+    if (n_events < layer_kernels(T) + 1) return ELQ_ERR_INVALID_ARG;
+    for (int i = 0; i < layer_kernels(T) + 1; ++i)
         if (!events[i]) return ELQ_ERR_INVALID_ARG;
     return run_layer(layer, x, x_type, T, y, ws, ws_bytes, stream, events, n_events);
 }
@@ -601,7 +581,7 @@ elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t
 elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, size_t* offset, size_t* bytes) {
     if (check_layer(layer, T) != ELQ_OK || T <= 0 || !offset || !bytes) return ELQ_ERR_INVALID_ARG;
     char* const base = reinterpret_cast<char*>((uintptr_t)1 << 40);   // only offsets are taken
-    LayerWs w = layer_layout(layer, T, base);
+    LayerWs w = layer_layout(layer, T, base, ELQ_F32);
     const size_t Tz = (size_t)T, P = (size_t)T * layer->k, L = layer->L, H = layer->H, E = layer->E,
                  I = layer->I;
     const void* p = nullptr;
@@ -624,6 +604,7 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, 
     case 14: p = w.n_act; n = 4; break;
     default: return ELQ_ERR_INVALID_ARG;
     }
+    if (!p) return ELQ_ERR_INVALID_ARG;   // not materialised at this T
     *offset = (size_t)(static_cast<const char*>(p) - base);
     *bytes = n;
     return ELQ_OK;
@@ -661,3 +642,60 @@ elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream) {
 }
 
 }  // extern "C"
+
+namespace {
+
+elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
+                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
+    elq_status st = check_layer(layer, T);
+    if (st != ELQ_OK) return st;
+    if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
+    if (T == 0) return ELQ_OK;
+    if (!x || !y) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
+    if (events && n_events < layer_kernels(T) + 1) return ELQ_ERR_INVALID_ARG;
+    if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
+    LayerWs w = layer_layout(layer, T, ws, x_type);
+    if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int H = layer->H, L = layer->L, E = layer->E, k = layer->k;
+    int ev = 0;
+    std::function<bool()> mark = [&]() -> bool {
+        if (!events) return true;
+        return cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s) == cudaSuccess;
+    };
+    const bool pdl = (events == nullptr);
+    cudaError_t e;
+    if (!mark()) return ELQ_ERR_CUDA;
+    // a1 + a2 + a4: D projection of x (quantised by the GEMV itself at small T)
+    WArgs gd;
+    if (w.raw) {
+        gd = dense_w(&layer->D, T, x, x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32, H, OUT_F32_Q81, w.z, w.zq,
+                     w.partial, w.cnt_d, w.err);
+    } else {
+        const int64_t nblk = (int64_t)T * (H / 32);
+        if (x_type == ELQ_BF16)
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        else
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        gd = dense_w(&layer->D, T, w.xq, X_Q81_TOKEN, 0, OUT_F32_Q81, w.z, w.zq, w.partial, w.cnt_d, w.err);
+    }
+    if (launch_w(gd, layer->D.fmt, w.pd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    // a3 + a5
+    e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits, w.cnt_router,
+                      true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl, w.err);
+    if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    // a6 - a9
+    st = run_experts(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark, pdl);
+    if (st != ELQ_OK) return st;
+    // a10
+    WArgs gu = dense_w(&layer->U, T, w.ylq, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, w.partial, w.cnt_u, w.err);
+    if (launch_w(gu, layer->U.fmt, w.pu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    return ELQ_OK;
+}
+
+}  // namespace

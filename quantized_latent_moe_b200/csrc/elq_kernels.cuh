@@ -3,9 +3,9 @@
 //   k_quant_weights   arena preparation from fp32 weights
 //   k_arena_pack      arena preparation from GGUF-style AoS blocks
 //   k_router          a3 (+a5)  logits, top-k, softmax, bucketing
-//   k_bucket          a5 standalone
-//   k_qgemv           a2/a6/a7/a8/a10  grouped quantised GEMV over the arena
-//   k_combine         a9  weighted combine + Q8_1
+//   k_topk, k_bucket  a3 / a5 standalone
+//   k_wgemv           a2 (+a1, a4) / a6 + a7 / a8 + a9 / a10: grouped quantised
+//                     GEMV over the arena, one warp per 32-row unit
 #pragma once
 
 #include "elq_device.cuh"
@@ -66,8 +66,8 @@ __global__ void __launch_bounds__(256) k_quant_weights(const float* __restrict__
         x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
     }
     const int64_t tile = row / kTileRows;
-    const int r = (int)(row % kTileRows);
-    const int64_t slab = tile * nb + kb;
+    const int slice = (int)(row % kTileRows) / 32, r = (int)(row % 32);
+    const int64_t sel = tile * nb * kTileRows + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r;
     if (FMT == 8) {
         float amax = 0.0f;
 #pragma unroll
@@ -82,10 +82,11 @@ __global__ void __launch_bounds__(256) k_quant_weights(const float* __restrict__
             if (dd != 0.0f) v = (int)fminf(fmaxf(roundf(__fdiv_rn(x[i], dd)), -127.0f), 127.0f);
             words[i >> 2] |= (uint32_t)(v & 0xff) << (8 * (i & 3));
         }
-        uint8_t* dst = q + slab * kQ80Slab + (r >> 3) * 256 + (r & 7) * 16;
+        uint8_t* dst = q + tile * nb * kQ80Slab + (int64_t)slice * nb * 1024 + (int64_t)kb * 1024 + (r >> 3) * 256 +
+                       (r & 7) * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
         *reinterpret_cast<uint4*>(dst + 128) = make_uint4(words[4], words[5], words[6], words[7]);
-        d[slab * kTileRows + r] = f2h(dd);
+        d[sel] = f2h(dd);
     } else {
         float amax = 0.0f, m = 0.0f;
 #pragma unroll
@@ -105,9 +106,9 @@ __global__ void __launch_bounds__(256) k_quant_weights(const float* __restrict__
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             words[j >> 2] |= (uint32_t)(qv[j] | (qv[j + 16] << 4)) << (8 * (j & 3));
-        uint8_t* dst = q + slab * kQ40Slab + r * 16;
+        uint8_t* dst = q + tile * nb * kQ40Slab + (int64_t)slice * nb * 512 + (int64_t)kb * 512 + r * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
-        d[slab * kTileRows + r] = f2h(dd);
+        d[sel] = f2h(dd);
     }
 }
 
@@ -122,18 +123,19 @@ __global__ void __launch_bounds__(256) k_arena_pack(const uint8_t* __restrict__ 
     const int kb = (int)(id % nb);
     const uint8_t* src = aos + id * bb;
     const int64_t tile = row / kTileRows;
-    const int r = (int)(row % kTileRows);
-    const int64_t slab = tile * nb + kb;
-    d[slab * kTileRows + r] = (uint16_t)(src[0] | (src[1] << 8));
+    const int slice = (int)(row % kTileRows) / 32, r = (int)(row % 32);
+    d[tile * nb * kTileRows + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r] = (uint16_t)(src[0] | (src[1] << 8));
     uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const int nq = (FMT == 8) ? 32 : 16;
     for (int i = 0; i < nq; ++i) words[i >> 2] |= (uint32_t)src[2 + i] << (8 * (i & 3));
     if (FMT == 8) {
-        uint8_t* dst = q + slab * kQ80Slab + (r >> 3) * 256 + (r & 7) * 16;
+        uint8_t* dst = q + tile * nb * kQ80Slab + (int64_t)slice * nb * 1024 + (int64_t)kb * 1024 + (r >> 3) * 256 +
+                       (r & 7) * 16;
         *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
         *reinterpret_cast<uint4*>(dst + 128) = make_uint4(words[4], words[5], words[6], words[7]);
     } else {
-        *reinterpret_cast<uint4*>(q + slab * kQ40Slab + r * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+        *reinterpret_cast<uint4*>(q + tile * nb * kQ40Slab + (int64_t)slice * nb * 512 + (int64_t)kb * 512 + r * 16) =
+            make_uint4(words[0], words[1], words[2], words[3]);
     }
 }
 
@@ -240,12 +242,15 @@ struct RouterArgs {
     int* cnt_all;     // [1]
     int do_bucket;
     int32_t *counts, *offsets, *perm, *pos, *act, *n_act;
+    int* err;         // device error word or NULL
 };
+
+constexpr uint64_t kRouterBudgetNs = 2000000000ull;
 
 // Top-k of one token's logits (in shared memory, lg[0..E)) by one warp, then
 // the softmax over the k selected in rank order.  Lane j ends with rank j.
 __device__ __forceinline__ void warp_topk_softmax(const float* lg, int E, int k, int32_t* idx_out,
-                                                  float* w_out) {
+                                                  float* w_out, int32_t* idx_sm = nullptr) {
     const int lane = threadIdx.x & 31;
     uint32_t taken = 0;
     float sel_v = 0.0f;
@@ -274,37 +279,99 @@ __device__ __forceinline__ void warp_topk_softmax(const float* lg, int E, int k,
     if (lane < k) {
         idx_out[lane] = sel_e;
         w_out[lane] = __fdiv_rn(ex, sum);
+        if (idx_sm) idx_sm[lane] = sel_e;
+    }
+}
+
+// a5 for at most 64 pairs by one warp: the rank of pair p is the number of
+// pairs (e', p') before (e, p) in (expert, pair id) order; counts and offsets
+// are direct counts.  idx_sm: the pairs' experts in shared memory.
+__device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* counts, int32_t* offsets,
+                                  int32_t* perm, int32_t* pos, int32_t* act, int32_t* n_act) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int p = lane + 32 * h;
+        if (p < P) {
+            const int e = idx_sm[p];
+            int r = 0;
+            for (int q = 0; q < P; ++q) {
+                const int eq = idx_sm[q];
+                r += (eq < e) || (eq == e && q < p);
+            }
+            perm[r] = p;
+            pos[p] = r;
+        }
+    }
+    int n = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        int c = 0, lt = 0;
+        for (int q = 0; q < P; ++q) {
+            const int eq = idx_sm[q];
+            c += (eq == e);
+            lt += (eq < e);
+        }
+        if (e < E) {
+            counts[e] = c;
+            offsets[e] = lt;
+        }
+        const bool on = (e < E) && c > 0;
+        const unsigned b = __ballot_sync(kFull, on);
+        if (on && act) act[n + __popc(b & ((1u << lane) - 1u))] = e;
+        n += __popc(b);
+    }
+    if (lane == 0) {
+        offsets[E] = P;
+        if (n_act) *n_act = n;
     }
 }
 
 __global__ void __launch_bounds__(128) k_router(RouterArgs a) {
-    extern __shared__ float rsm[];
+    extern __shared__ __align__(128) float rsm[];   // [4][L] router rows, then [<=8][L] latent rows
+    __shared__ __align__(8) uint64_t rbar;
     __shared__ int s_last;
-    pdl_wait();
+    __shared__ int32_t s_idx[64];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.y * kRouterTok;
     const int nt = min(kRouterTok, a.T - t0);
-    for (int i = threadIdx.x; i < nt * a.L; i += blockDim.x) rsm[i] = a.z[(int64_t)t0 * a.L + i];
+    const int e0 = blockIdx.x * kRouterWarps;
+    const int ne = min(kRouterWarps, a.E - e0);
+    float* wsm = rsm;
+    float* zsm = rsm + kRouterWarps * a.L;
+    if (threadIdx.x == 0) {
+        mbar_init(&rbar, 1);
+        fence_barrier_init();
+    }
     __syncthreads();
-    const int e = blockIdx.x * kRouterWarps + warp;
-    if (e < a.E) {
-        const float* wr = a.w + (int64_t)e * a.L;
-        const float b = a.bias ? a.bias[e] : 0.0f;
+    // router rows do not depend on the upstream kernel: start them first
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&rbar, (uint32_t)(ne + nt) * a.L * 4u);
+        bulk_g2s(wsm, a.w + (int64_t)e0 * a.L, (uint32_t)ne * a.L * 4u, &rbar);
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) bulk_g2s(zsm, a.z + (int64_t)t0 * a.L, (uint32_t)nt * a.L * 4u, &rbar);
+    if (!mbar_wait_bounded(&rbar, 0, a.err, kRouterBudgetNs)) {
+        mbar_wait_bounded(&rbar, 0, nullptr, kRouterBudgetNs);
+        return;
+    }
+    const int e = e0 + warp;
+    if (warp < ne) {
+        const float* wr = wsm + warp * a.L;
+        const float b = a.bias ? __ldg(a.bias + e) : 0.0f;
         for (int tt = 0; tt < nt; ++tt) {
-            const float* zt = rsm + tt * a.L;
+            const float* zt = zsm + tt * a.L;
             float p = 0.0f;
-            for (int l = lane; l < a.L; l += 32) p = __fmaf_rn(zt[l], __ldg(wr + l), p);
+            for (int l = lane; l < a.L; l += 32) p = __fmaf_rn(zt[l], wr[l], p);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(kFull, p, o));
             if (a.bias) p = __fadd_rn(p, b);
             if (lane == 0) a.logits[(int64_t)(t0 + tt) * a.E + e] = p;
         }
     }
-    if (!a.cnt_tok) {       // logits only; k_topk follows
-        pdl_trigger();
-        return;
-    }
     __syncthreads();
+    if (!a.cnt_tok) return;     // logits only; k_topk follows
     if (threadIdx.x == 0) {
         __threadfence();
         s_last = (atomicAdd(&a.cnt_tok[blockIdx.y], 1) == (int)gridDim.x - 1);
@@ -312,18 +379,22 @@ __global__ void __launch_bounds__(128) k_router(RouterArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    const bool small = a.do_bucket && gridDim.y == 1 && a.T * a.k <= 64;
     float* lg = rsm + warp * a.E;
     for (int tt = warp; tt < nt; tt += kRouterWarps) {
         const int t = t0 + tt;
         for (int x = lane; x < a.E; x += 32) lg[x] = __ldcg(a.logits + (int64_t)t * a.E + x);
         __syncwarp();
-        warp_topk_softmax(lg, a.E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k);
+        warp_topk_softmax(lg, a.E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k,
+                          small ? s_idx + t * a.k : nullptr);
         __syncwarp();
     }
     __syncthreads();
     if (threadIdx.x == 0) a.cnt_tok[blockIdx.y] = 0;
-    if (!a.do_bucket) {
-        pdl_trigger();
+    if (!a.do_bucket) return;
+    if (small) {
+        if (warp == 0)
+            bucket_warp_small(s_idx, a.T * a.k, a.E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act);
         return;
     }
     if (threadIdx.x == 0) {
@@ -336,7 +407,6 @@ __global__ void __launch_bounds__(128) k_router(RouterArgs a) {
     bucket_cta(a.idx, a.T * a.k, a.E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act,
                reinterpret_cast<int*>(rsm));
     if (threadIdx.x == 0) *a.cnt_all = 0;
-    pdl_trigger();
 }
 
 // Standalone top-k + softmax: one warp per token over logits [T][E].
@@ -355,385 +425,467 @@ __global__ void __launch_bounds__(128) k_topk(const float* __restrict__ logits, 
 }
 
 // ============================================================================
-// Grouped quantised GEMV (dp4a) over the tile-slab arena.
+// Grouped quantised GEMV (dp4a) over the slice-major arena -- one warp per
+// work unit.
 //
-// Work unit: (group a, tile, chunk range).  A group is one expert with its
-// pairs (from the bucketing) or the whole dense matrix with all T tokens.
-// split == 1: a unit is one chunk of 8 blocks; its per-chunk partial sums go
-//   to a partial buffer and the last unit of a tile to arrive (atomic counter)
-//   adds the chunks' partials in order and runs the epilogue.
-// split == 0: a unit is a whole tile; chunk partials are added in order in
-//   shared memory and the same CTA runs the epilogue.
-// Units are dealt to the persistent CTAs in contiguous ranges.  Each step
-// (unit, 32-token block, chunk) streams its weight slabs (<= 32 KB of codes +
-// 2 KB of scales) into a ring of shared-memory stages with two bulk copies
-// completing on an mbarrier; the activations of the step's tokens are staged
-// next to them.  Warp w owns rows 16w .. 16w+15 of the tile.
+// A unit is (group a, 128-row tile, chunk c of 8 blocks, 32-row slice s).  A
+// group is one expert with the pairs the bucketing gave it, or the whole dense
+// matrix with all T tokens.  Lane l owns row 32 s + l of the tile.
+//
+// Each warp runs its own ring of shared-memory stages: for a unit it issues
+// bulk copies (completing on the stage's mbarrier) of the slice's codes for the
+// chunk (8 KB Q8_0 / 4 KB Q4_0, contiguous), its fp16 scales (512 B) and, per
+// token, the chunk's activation slice (8 Q8_1 blocks, or 256 raw values that
+// it quantises itself).  The unit's weights are loaded into registers once and
+// reused for every token.  The per-chunk partial sums go to a partial buffer;
+// the warp completing the last of a tile's units (an atomic counter per tile)
+// adds the chunks in order and runs the epilogue.  No block-wide barrier is
+// taken after the start.  Work is dealt to the persistent CTAs in contiguous
+// unit ranges; inside a CTA the warps take units from a shared counter.
 // ============================================================================
-constexpr int kGemvThreads = 256;
-constexpr int kGemvStages = 4;
-constexpr int kTokBlock = 32;      // tokens per token block
-constexpr int kTokPass = 4;        // tokens per register pass
+constexpr int kTokMax = 32;        // tokens a unit stages at once
 
-enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2 };
-enum { X_DENSE = 0, X_PAIR_TOKEN = 1, X_POSITION = 2 };
+enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2, OUT_F32_COMBINE = 3 };
+enum { X_Q81_TOKEN = 0, X_Q81_PAIR_TOKEN = 1, X_Q81_POSITION = 2, X_RAW_F32 = 3, X_RAW_BF16 = 4 };
 
-struct GemvArgs {
+struct WArgs {
     const uint8_t* q;           // arena codes of group 0
     const uint16_t* d;          // arena scales of group 0
-    int64_t q_gstride;          // bytes between groups
+    int64_t q_gstride;          // bytes between groups (experts)
     int64_t d_gstride;          // fp16 elements between groups
-    int nb, tiles, nchunks, split;
-    const int32_t* act;         // active experts (NULL: one dense group)
+    int nb, tiles, nchunks;
+    const int32_t* act;         // active experts, NULL for one dense group
     const int32_t* n_act;
-    const int32_t* offsets;     // [E+1] pair offsets (NULL: dense)
+    const int32_t* offsets;     // [E+1] pair offsets, NULL for dense
     const int32_t* perm;
-    int kslots;                 // k: token of pair p is p / k
+    int kslots;                 // top-k: token of pair p is p / k
     int T;
-    const uint8_t* x;           // Q8_1 rows, nb blocks each
+    const void* x;
     int x_mode;
+    int64_t x_row;              // elements per raw input row (X_RAW_*)
     int out_mode;
-    float* y;                   // fp32 out rows (token or position), ld y_ld
+    float* y;                   // fp32 rows (token or pair position)
     int64_t y_ld;
-    uint8_t* yq;                // Q8_1 out rows, yq_ld blocks each
-    int64_t yq_ld;
-    float* partial;             // split: [nchunks][part_tok][tiles*128]
+    uint8_t* yq;                // Q8_1 rows
+    int64_t yq_ld;              // blocks per Q8_1 row
+    // OUT_F32_COMBINE: weighted combine of each token's k rows of y
+    const float* wts;
+    const int32_t* pos;
+    int* cnt_comb;              // [T][tiles], zero on entry/exit
+    float* ylat;
+    uint8_t* ylq;
+    float* partial;             // [nchunks][part_tok][tiles*128]
     int64_t part_tok;
-    int* counters;              // split: per (group slot, tile), zero on entry/exit
+    int* counters;              // [groups][tiles], zero on entry/exit
     int* err;
     uint64_t budget_ns;
+    int stages, tokcap;
+    int stage_bytes, act_off, act_bytes, scratch_bytes;
+    // routing (act/offsets/perm) was complete before this grid was launched:
+    // the prologue may read it before the grid dependency is resolved
+    int routing_early;
 };
 
 template <int FMT>
-struct GemvSmem {
-    static constexpr int kSlab = (FMT == 8) ? kQ80Slab : kQ40Slab;
-    static constexpr int kStageQ = kSlab * kChunk;
-    static constexpr int kStage = kStageQ + kScaleSlab * kChunk;
-    static constexpr int kStagesBytes = kStage * kGemvStages;
-    static constexpr int kAq = kStagesBytes;                           // int8 [32 tok][8 kb][32]
-    static constexpr int kAd = kAq + kTokBlock * kChunk * 32;          // float [32][8]
-    static constexpr int kAs = kAd + kTokBlock * kChunk * 4;           // int [32][8]
-    static constexpr int kAcc = kAs + kTokBlock * kChunk * 4;          // float [32][128]
-    static constexpr int kBar = kAcc + kTokBlock * kTileRows * 4;      // uint64 [stages]
-    static constexpr int kTotal = kBar + 8 * kGemvStages + 16;
+struct WSlice {
+    static constexpr int kCodes = (FMT == 8) ? 1024 : 512;   // bytes per (slice, block)
 };
 
-struct GemvUnit {
-    int a, tile, c0, c1;
-    int e, tok0, ntok;          // tok0: first pair position (experts) or 0
-    bool valid;
+struct WUnit {
+    int a, tile, c, s, e, tok0, ntok, kbn;
 };
 
-__device__ __forceinline__ GemvUnit gemv_unit(const GemvArgs& g, int64_t u, int64_t u_end) {
-    GemvUnit r;
-    r.valid = u < u_end;
-    if (!r.valid) return r;
-    const int per_group = g.tiles * (g.split ? g.nchunks : 1);
-    r.a = (int)(u / per_group);
-    const int rem = (int)(u % per_group);
-    r.tile = g.split ? rem / g.nchunks : rem;
-    r.c0 = g.split ? rem % g.nchunks : 0;
-    r.c1 = g.split ? r.c0 + 1 : g.nchunks;
-    r.e = g.act ? __ldg(g.act + r.a) : 0;
+__device__ __forceinline__ WUnit wunit(const WArgs& g, int u) {
+    WUnit r;
+    const int per_tile = g.nchunks * 4;
+    const int per_group = g.tiles * per_tile;
+    r.a = u / per_group;
+    int rem = u - r.a * per_group;
+    r.tile = rem / per_tile;
+    rem -= r.tile * per_tile;
+    r.c = rem >> 2;
+    r.s = rem & 3;
+    r.e = g.act ? __ldcg(g.act + r.a) : 0;
     if (g.offsets) {
-        r.tok0 = __ldg(g.offsets + r.e);
-        r.ntok = __ldg(g.offsets + r.e + 1) - r.tok0;
+        r.tok0 = __ldcg(g.offsets + r.e);
+        r.ntok = __ldcg(g.offsets + r.e + 1) - r.tok0;
     } else {
         r.tok0 = 0;
         r.ntok = g.T;
     }
+    r.kbn = min(kChunk, g.nb - r.c * kChunk);
     return r;
 }
 
-// Step cursor over (unit, token block, chunk) in order.
-struct GemvCursor {
-    GemvUnit un;
-    int64_t u, u_end;
-    int tb, c;
-    __device__ __forceinline__ void start(const GemvArgs& g, int64_t u0, int64_t u1) {
-        u = u0;
-        u_end = u1;
-        un = gemv_unit(g, u, u_end);
-        tb = 0;
-        c = un.valid ? un.c0 : 0;
-    }
-    __device__ __forceinline__ bool valid() const { return un.valid; }
-    __device__ __forceinline__ void advance(const GemvArgs& g) {
-        if (++c < un.c1) return;
-        c = un.c0;
-        if (++tb * kTokBlock < un.ntok) return;
-        tb = 0;
-        ++u;
-        un = gemv_unit(g, u, u_end);
-        c = un.valid ? un.c0 : 0;
-    }
-};
-
-template <int FMT>
-__device__ __forceinline__ void gemv_issue(const GemvArgs& g, const GemvCursor& cu, uint8_t* stage,
-                                           uint64_t* bar) {
-    using S = GemvSmem<FMT>;
-    const int kbn = min(kChunk, g.nb - cu.c * kChunk);
-    const int64_t slab0 = (int64_t)cu.un.tile * g.nb + (int64_t)cu.c * kChunk;
-    const uint8_t* qs = g.q + cu.un.e * g.q_gstride + slab0 * S::kSlab;
-    const uint16_t* ds = g.d + cu.un.e * g.d_gstride + slab0 * kTileRows;
-    const uint32_t qb = (uint32_t)(kbn * S::kSlab), db = (uint32_t)(kbn * kScaleSlab);
-    mbar_arrive_expect_tx(bar, qb + db);
-    bulk_g2s(stage, qs, qb, bar);
-    bulk_g2s(stage + S::kStageQ, ds, db, bar);
+__device__ __forceinline__ int64_t wunit_xrow(const WArgs& g, const WUnit& un, int i) {
+    const int tp = un.tok0 + i;
+    if (g.x_mode == X_Q81_PAIR_TOKEN) return __ldcg(g.perm + tp) / g.kslots;
+    return tp;   // token (dense) or pair position
 }
 
-// Epilogue of one token block of a tile from acc[tok][row] in shared memory.
-__device__ __forceinline__ void gemv_epilogue(const GemvArgs& g, const GemvUnit& un, int tb, int ntb,
-                                              const float* acc) {
+// Bytes of one token's activation slice for a chunk of kbn blocks.
+__device__ __forceinline__ uint32_t wact_bytes(const WArgs& g, int kbn) {
+    if (g.x_mode == X_RAW_F32) return (uint32_t)kbn * 128u;
+    if (g.x_mode == X_RAW_BF16) return (uint32_t)kbn * 64u;
+    return (uint32_t)kbn * 36u;
+}
+
+template <int FMT>
+__device__ __forceinline__ void wissue_weights(const WArgs& g, const WUnit& un, uint8_t* stage, uint64_t* bar,
+                                               int ntok_pass) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t cb = (uint32_t)(un.kbn * SL::kCodes), sb = (uint32_t)(un.kbn * 64);
+    if (lane == 0) mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)ntok_pass * wact_bytes(g, un.kbn));
+    __syncwarp();
+    if (lane == 0) {
+        const uint8_t* src = g.q + un.e * g.q_gstride +
+                             ((int64_t)un.tile * g.nb * 4 + (int64_t)un.s * g.nb + (int64_t)un.c * kChunk) * SL::kCodes;
+        bulk_g2s(stage, src, cb, bar);
+    } else if (lane == 1) {
+        const uint16_t* src = g.d + un.e * g.d_gstride + (int64_t)un.tile * g.nb * kTileRows +
+                              (int64_t)un.s * g.nb * 32 + (int64_t)un.c * kChunk * 32;
+        bulk_g2s(stage + kChunk * SL::kCodes, src, sb, bar);
+    }
+}
+
+__device__ __forceinline__ void wissue_acts(const WArgs& g, const WUnit& un, uint8_t* act_area, uint64_t* bar,
+                                            int first, int ntok_pass) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t ab = wact_bytes(g, un.kbn);
+    for (int i = lane; i < ntok_pass; i += 32) {
+        const int64_t row = wunit_xrow(g, un, first + i);
+        const uint8_t* src;
+        if (g.x_mode == X_RAW_F32)
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)un.c * 256) * 4;
+        else if (g.x_mode == X_RAW_BF16)
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)un.c * 256) * 2;
+        else
+            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + (int64_t)un.c * kChunk) * 36;
+        bulk_g2s(act_area + i * g.act_bytes, src, ab, bar);
+    }
+}
+
+// Epilogue of a finished tile (all chunk partials present) by one warp.  The
+// chunk partials of up to 16 chunks are loaded before any is added, so the
+// L2 round trips overlap; the adds then run in chunk order.
+__device__ void wepilogue(const WArgs& g, const WUnit& un) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows_total = (int64_t)g.tiles * kTileRows;
+    for (int i = 0; i < un.ntok; ++i) {
+        const int64_t tokidx = (int64_t)un.tok0 + i;
+        float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const float* pb = g.partial + tokidx * rows_total + (int64_t)un.tile * kTileRows + lane;
+        const int64_t cstride = g.part_tok * rows_total;
+        for (int c0 = 0; c0 < g.nchunks; c0 += 16) {
+            float t[16][4];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                if (c0 + c < g.nchunks) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) t[c][q] = __ldcg(pb + (int64_t)(c0 + c) * cstride + 32 * q);
+                }
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                if (c0 + c < g.nchunks) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) v[q] = __fadd_rn(v[q], t[c][q]);
+                }
+        }
+        if (g.out_mode == OUT_SWIGLU) {
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const float h = __fmul_rn(silu_f32(v[hb]), v[2 + hb]);
+                warp_quant_q8_1(h, g.yq + (tokidx * g.yq_ld + un.tile * 2 + hb) * 36);
+            }
+            continue;
+        }
+        float* yr = g.y + tokidx * g.y_ld + (int64_t)un.tile * kTileRows + lane;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) yr[32 * q] = v[q];
+        if (g.out_mode == OUT_F32_Q81) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                warp_quant_q8_1(v[q], g.yq + (tokidx * g.yq_ld + un.tile * 4 + q) * 36);
+        } else if (g.out_mode == OUT_F32_COMBINE) {
+            // the pair's rows of this tile are out: count them for the token
+            __threadfence();
+            __syncwarp();
+            const int p = __ldcg(g.perm + tokidx);
+            const int t = p / g.kslots;
+            int last = 0;
+            if (lane == 0) {
+                int* cnt = g.cnt_comb + (int64_t)t * g.tiles + un.tile;
+                last = (atomicAdd(cnt, 1) == g.kslots - 1);
+                if (last) *cnt = 0;
+            }
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {
+                __threadfence();
+                const int L = g.tiles * kTileRows;
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int j0 = 0; j0 < g.kslots; j0 += 8) {
+                    float ov[8][4], wv[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < g.kslots) {
+                            const int pj = t * g.kslots + j0 + j;
+                            wv[j] = __ldcg(g.wts + pj);
+                            const float* orow =
+                                g.y + (int64_t)__ldcg(g.pos + pj) * g.y_ld + (int64_t)un.tile * kTileRows + lane;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) ov[j][q] = __ldcg(orow + 32 * q);
+                        }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < g.kslots) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) acc[q] = __fmaf_rn(wv[j], ov[j][q], acc[q]);
+                        }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    g.ylat[(int64_t)t * L + un.tile * kTileRows + 32 * q + lane] = acc[q];
+                    warp_quant_q8_1(acc[q], g.ylq + ((int64_t)t * (L / 32) + un.tile * 4 + q) * 36);
+                }
+            }
+        }
+    }
+}
+
+// Completion of a batch of this warp's finished units (held one per lane in
+// `pending`): one fence for all their partial stores, one atomic per unit;
+// the warp then runs the epilogue of every tile it completed.
+__device__ __forceinline__ void wcomplete(const WArgs& g, int pending, int npend) {
+    const int lane = threadIdx.x & 31;
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane < npend) {
+        const WUnit un = wunit(g, pending);
+        int* cnt = g.counters + (int64_t)un.a * g.tiles + un.tile;
+        last = (atomicAdd(cnt, 1) == g.nchunks * 4 - 1);
+        if (last) *cnt = 0;
+    }
+    unsigned m = __ballot_sync(kFull, last);
+    if (m) __threadfence();
+    while (m) {
+        const int j = __ffs(m) - 1;
+        m &= m - 1;
+        const int u = __shfl_sync(kFull, pending, j);
+        wepilogue(g, wunit(g, u));
+    }
+    __syncwarp();
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
+    using SL = WSlice<FMT>;
+    extern __shared__ __align__(128) uint8_t wsm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t orow0 = (int64_t)un.tok0 + tb * kTokBlock;   // token (dense) or position (experts)
-    if (g.out_mode == OUT_SWIGLU) {
-        for (int i = warp; i < ntb * 2; i += kGemvThreads / 32) {
-            const int tok = i >> 1, hb = i & 1;
-            const float gv = acc[tok * kTileRows + hb * 32 + lane];
-            const float uv = acc[tok * kTileRows + 64 + hb * 32 + lane];
-            const float h = __fmul_rn(silu_f32(gv), uv);
-            warp_quant_q8_1(h, g.yq + ((orow0 + tok) * g.yq_ld + un.tile * 2 + hb) * 36);
-        }
-        return;
-    }
-    for (int i = threadIdx.x; i < ntb * kTileRows; i += kGemvThreads) {
-        const int tok = i / kTileRows, r = i % kTileRows;
-        g.y[(orow0 + tok) * g.y_ld + (int64_t)un.tile * kTileRows + r] = acc[i];
-    }
-    if (g.out_mode == OUT_F32_Q81) {
-        for (int i = warp; i < ntb * 4; i += kGemvThreads / 32) {
-            const int tok = i >> 2, b = i & 3;
-            warp_quant_q8_1(acc[tok * kTileRows + b * 32 + lane],
-                            g.yq + ((orow0 + tok) * g.yq_ld + un.tile * 4 + b) * 36);
-        }
-    }
-}
+    const int S = g.stages;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wsm);                 // [nwarps][S]
+    int* unit_of = reinterpret_cast<int*>(wsm + 8 * 8 * 4);             // [nwarps][S], S <= 4
+    int* s_next = reinterpret_cast<int*>(wsm + 8 * 8 * 4 + 8 * 4 * 4);
+    uint8_t* stages = wsm + 512 + (size_t)warp * (S * g.stage_bytes + g.scratch_bytes);
+    uint8_t* scratch = stages + S * g.stage_bytes;
+    uint64_t* mybar = bars + warp * 4;
+    int* myunit = unit_of + warp * 4;
 
-template <int FMT>
-__global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(GemvArgs g) {
-    using S = GemvSmem<FMT>;
-    extern __shared__ __align__(128) uint8_t gsm[];
-    uint8_t* stages = gsm;
-    int8_t* aq = reinterpret_cast<int8_t*>(gsm + S::kAq);
-    float* ad = reinterpret_cast<float*>(gsm + S::kAd);
-    int* as = reinterpret_cast<int*>(gsm + S::kAs);
-    float* acc = reinterpret_cast<float*>(gsm + S::kAcc);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(gsm + S::kBar);
-    __shared__ int s_flag;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        for (int s = 0; s < kGemvStages; ++s) mbar_init(&bars[s], 1);
-        fence_barrier_init();
-    }
+    if (threadIdx.x == 0) *s_next = 0;
+    if (lane <= S) mbar_init(&mybar[lane], 1);     // S ring stages + one for extra token passes
+    if (lane == 0) fence_barrier_init();
     __syncthreads();
-    pdl_wait();
 
-    // this CTA's unit range
-    const int64_t n_groups = g.act ? (int64_t)__ldg(g.n_act) : 1;
-    const int64_t n_units = n_groups * g.tiles * (g.split ? g.nchunks : 1);
-    const int64_t u0 = n_units * blockIdx.x / gridDim.x;
-    const int64_t u1 = n_units * (blockIdx.x + 1) / gridDim.x;
-    if (u0 >= u1) return;
+    const bool dense = (g.act == nullptr);
+    const bool early = dense || g.routing_early;
+    int64_t n_units = 0, u0 = 0, u1 = 0;
+    auto range = [&]() {
+        const int64_t groups = dense ? 1 : (int64_t)__ldcg(g.n_act);
+        n_units = groups * g.tiles * g.nchunks * 4;
+        u0 = n_units * blockIdx.x / gridDim.x;
+        u1 = n_units * (blockIdx.x + 1) / gridDim.x;
+    };
+    auto grab = [&]() -> int {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(s_next, 1);
+        u = __shfl_sync(kFull, u, 0) + (int)u0;
+        return (u < u1) ? u : -1;
+    };
+    const int tokcap = g.tokcap;
 
-    GemvCursor prod, cons;
-    int issued = 0;
-    if (tid == 0) {
-        prod.start(g, u0, u1);
-        for (int s = 0; s < kGemvStages && prod.valid(); ++s) {
-            gemv_issue<FMT>(g, prod, stages + s * S::kStage, &bars[s]);
-            prod.advance(g);
-            ++issued;
+    // prologue: fill the ring.  Weights do not depend on the upstream kernel
+    // (and the routing, when it was complete before this grid started), so
+    // their copies start before the grid dependency is resolved.
+    if (early) {
+        range();
+        for (int st = 0; st < S; ++st) {
+            const int u = grab();
+            if (lane == 0) myunit[st] = u;
+            if (u >= 0) {
+                const WUnit un = wunit(g, u);
+                wissue_weights<FMT>(g, un, stages + st * g.stage_bytes, &mybar[st], min(un.ntok, tokcap));
+            }
         }
-    }
-    cons.start(g, u0, u1);
-
-    // lane -> (row, byte offset within a slab)
-    int row, woff;
-    if (FMT == 8) {
-        const int r16 = lane & 15, kg = lane >> 4;
-        row = warp * 16 + r16;
-        woff = (row >> 3) * 256 + kg * 128 + (row & 7) * 16;
+        pdl_wait();
+        pdl_trigger();
+        __syncwarp();
+        for (int st = 0; st < S; ++st) {
+            const int u = myunit[st];
+            if (u >= 0) {
+                const WUnit un = wunit(g, u);
+                wissue_acts(g, un, stages + st * g.stage_bytes + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+            }
+        }
     } else {
-        const int half = lane & 1;
-        row = warp * 16 + (lane >> 1);
-        woff = row * 16 + half * 8;
+        pdl_wait();
+        pdl_trigger();
+        range();
+        for (int st = 0; st < S; ++st) {
+            const int u = grab();
+            if (lane == 0) myunit[st] = u;
+            if (u >= 0) {
+                const WUnit un = wunit(g, u);
+                uint8_t* stg = stages + st * g.stage_bytes;
+                wissue_weights<FMT>(g, un, stg, &mybar[st], min(un.ntok, tokcap));
+                wissue_acts(g, un, stg + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+            }
+        }
     }
-    const bool owner = (FMT == 8) ? (lane < 16) : ((lane & 1) == 0);
-    const int aoff = (FMT == 8) ? (lane >> 4) * 16 : (lane & 1) * 8;
+    __syncwarp();
 
+    const int64_t rows_total = (int64_t)g.tiles * kTileRows;
+    uint32_t xuse = 0;          // uses of the extra barrier (its phase parity)
     bool ok = true;
-    for (int step = 0; cons.valid(); ++step) {
-        const GemvUnit un = cons.un;
-        const int tb = cons.tb, c = cons.c;
-        const int ntb = min(kTokBlock, un.ntok - tb * kTokBlock);
-        const int kbn = min(kChunk, g.nb - c * kChunk);
-        const int stg = step % kGemvStages;
-
-        // stage this step's activations: (token, block) -> codes, scale, code sum
-        for (int i = tid; i < ntb * kbn; i += kGemvThreads) {
-            const int tok = i / kbn, kb = i % kbn;
-            const int tokpos = un.tok0 + tb * kTokBlock + tok;
-            int64_t xrow;
-            if (g.x_mode == X_DENSE) xrow = tokpos;
-            else if (g.x_mode == X_PAIR_TOKEN) xrow = __ldg(g.perm + tokpos) / g.kslots;
-            else xrow = tokpos;
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(
-                g.x + (xrow * g.nb + (int64_t)c * kChunk + kb) * 36);
-            const uint32_t dsw = __ldg(src);
-            uint32_t* dst = reinterpret_cast<uint32_t*>(aq + (tok * kChunk + kb) * 32);
-            int sum = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t v = __ldg(src + 1 + j);
-                dst[j] = v;
-                sum = __dp4a((int)v, 0x01010101, sum);
-            }
-            ad[tok * kChunk + kb] = h2f((uint16_t)(dsw & 0xffff));
-            as[tok * kChunk + kb] = sum;
+    int it = 0;
+    int pending = -1, npend = 0; // finished units awaiting their completion count (one per lane)
+    for (;; ++it) {
+        const int st = it % S;
+        const int u = myunit[st];
+        if (u < 0) break;
+        if (!mbar_wait_bounded(&mybar[st], (uint32_t)((it / S) & 1), g.err, g.budget_ns)) {
+            ok = false;
+            break;
         }
-        if (tid == 0) s_flag = mbar_wait_bounded(&bars[stg], (step / kGemvStages) & 1, g.err, g.budget_ns);
-        __syncthreads();
-        if (!s_flag) { ok = false; break; }
+        const WUnit un = wunit(g, u);
+        uint8_t* stg = stages + st * g.stage_bytes;
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(stg + kChunk * SL::kCodes);
 
-        const uint8_t* sq = stages + stg * S::kStage;
-        const uint16_t* sd = reinterpret_cast<const uint16_t*>(sq + S::kStageQ);
-        for (int tp = 0; tp < ntb; tp += kTokPass) {
-            float part[kTokPass];
+        // the slice's weights for this chunk, in registers (signed 8-bit codes)
+        int w[kChunk][8];
+        float dw[kChunk];
 #pragma unroll
-            for (int t = 0; t < kTokPass; ++t) part[t] = 0.0f;
-            for (int kb = 0; kb < kbn; ++kb) {
-                const float dw = h2f(sd[kb * kTileRows + row]);
+        for (int kb = 0; kb < kChunk; ++kb) {
+            if (kb < un.kbn) {
+                dw[kb] = h2f(sc[kb * 32 + lane]);
                 if (FMT == 8) {
-                    const uint4 w = lds128(sq + kb * kQ80Slab + woff);
-#pragma unroll
-                    for (int t = 0; t < kTokPass; ++t) {
-                        if (tp + t < ntb) {
-                            const int ai = (tp + t) * kChunk + kb;
-                            const uint4 av = lds128(aq + ai * 32 + aoff);
-                            int s = __dp4a((int)w.x, (int)av.x, 0);
-                            s = __dp4a((int)w.y, (int)av.y, s);
-                            s = __dp4a((int)w.z, (int)av.z, s);
-                            s = __dp4a((int)w.w, (int)av.w, s);
-                            s += __shfl_xor_sync(kFull, s, 16);
-                            part[t] = __fmaf_rn(__int2float_rn(s), __fmul_rn(dw, ad[ai]), part[t]);
-                        }
-                    }
+                    const uint8_t* cp = stg + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
+                    const uint4 a = lds128(cp), b = lds128(cp + 128);
+                    w[kb][0] = (int)a.x; w[kb][1] = (int)a.y; w[kb][2] = (int)a.z; w[kb][3] = (int)a.w;
+                    w[kb][4] = (int)b.x; w[kb][5] = (int)b.y; w[kb][6] = (int)b.z; w[kb][7] = (int)b.w;
                 } else {
-                    const uint2 w = *reinterpret_cast<const uint2*>(sq + kb * kQ40Slab + woff);
-                    const int lo0 = (int)(w.x & 0x0F0F0F0Fu), lo1 = (int)(w.y & 0x0F0F0F0Fu);
-                    const int hi0 = (int)((w.x >> 4) & 0x0F0F0F0Fu), hi1 = (int)((w.y >> 4) & 0x0F0F0F0Fu);
+                    const uint4 a = lds128(stg + kb * 512 + lane * 16);
+                    const uint32_t v[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                    for (int t = 0; t < kTokPass; ++t) {
-                        if (tp + t < ntb) {
-                            const int ai = (tp + t) * kChunk + kb;
-                            const uint2 al = *reinterpret_cast<const uint2*>(aq + ai * 32 + aoff);
-                            const uint2 ah = *reinterpret_cast<const uint2*>(aq + ai * 32 + 16 + aoff);
-                            int s = __dp4a(lo0, (int)al.x, 0);
-                            s = __dp4a(lo1, (int)al.y, s);
-                            s = __dp4a(hi0, (int)ah.x, s);
-                            s = __dp4a(hi1, (int)ah.y, s);
-                            s += __shfl_xor_sync(kFull, s, 1);
-                            s -= 8 * as[ai];
-                            part[t] = __fmaf_rn(__int2float_rn(s), __fmul_rn(dw, ad[ai]), part[t]);
-                        }
+                    for (int j = 0; j < 4; ++j) {
+                        // nibbles q (0..15) -> signed bytes q - 8, without borrows between bytes
+                        const uint32_t lo = v[j] & 0x0F0F0F0Fu, hi = (v[j] >> 4) & 0x0F0F0F0Fu;
+                        w[kb][j] = (int)(((lo | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
+                        w[kb][4 + j] = (int)(((hi | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
                     }
                 }
-            }
-            if (owner) {
+            } else {
+                dw[kb] = 0.0f;
 #pragma unroll
-                for (int t = 0; t < kTokPass; ++t) {
-                    if (tp + t < ntb) {
-                        const int tok = tp + t;
-                        if (g.split) {
-                            const int64_t tokidx = (int64_t)un.tok0 + tb * kTokBlock + tok;
-                            __stcg(g.partial + ((int64_t)c * g.part_tok + tokidx) * ((int64_t)g.tiles * kTileRows) +
-                                       (int64_t)un.tile * kTileRows + row,
-                                   part[t]);
-                        } else {
-                            float* ap = acc + tok * kTileRows + row;
-                            *ap = (c == un.c0) ? __fadd_rn(0.0f, part[t]) : __fadd_rn(*ap, part[t]);
-                        }
-                    }
+                for (int j = 0; j < 8; ++j) w[kb][j] = 0;
+            }
+        }
+        __syncwarp();
+
+        for (int first = 0; first < un.ntok; first += tokcap) {
+            const int np = min(tokcap, un.ntok - first);
+            if (first > 0) {
+                // more tokens than one staging holds: reload the activation area
+                __syncwarp();
+                fence_proxy_async();
+                uint64_t* xb = &mybar[S];
+                if (lane == 0) mbar_arrive_expect_tx(xb, (uint32_t)np * wact_bytes(g, un.kbn));
+                __syncwarp();
+                wissue_acts(g, un, stg + g.act_off, xb, first, np);
+                const bool got = mbar_wait_bounded(xb, xuse & 1u, g.err, g.budget_ns);
+                ++xuse;
+                if (!got) {
+                    ok = false;
+                    break;
                 }
             }
-        }
-        __syncthreads();   // stage and activations consumed
-        if (tid == 0 && prod.valid()) {
-            fence_proxy_async();
-            gemv_issue<FMT>(g, prod, stages + stg * S::kStage, &bars[stg]);
-            prod.advance(g);
-            ++issued;
-        }
-
-        const bool last_chunk = (c + 1 == un.c1);
-        const bool last_tb = ((tb + 1) * kTokBlock >= un.ntok);
-        if (!g.split && last_chunk) {
-            gemv_epilogue(g, un, tb, ntb, acc);
-            __syncthreads();
-        }
-        if (g.split && last_chunk && last_tb) {
-            // ordered completion of the tile: the last unit to arrive finishes it
-            if (tid == 0) {
-                __threadfence();
-                int* cnt = g.counters + (int64_t)un.a * g.tiles + un.tile;
-                const int old = atomicAdd(cnt, 1);
-                s_flag = (old == g.nchunks - 1);
-                if (s_flag) *cnt = 0;
-            }
-            __syncthreads();
-            if (s_flag) {
-                __threadfence();
-                for (int tb2 = 0; tb2 * kTokBlock < un.ntok; ++tb2) {
-                    const int n2 = min(kTokBlock, un.ntok - tb2 * kTokBlock);
-                    for (int i = tid; i < n2 * kTileRows; i += kGemvThreads) {
-                        const int tok = i / kTileRows, r = i % kTileRows;
-                        const int64_t tokidx = (int64_t)un.tok0 + tb2 * kTokBlock + tok;
-                        float s = 0.0f;
-                        for (int cc = 0; cc < g.nchunks; ++cc)
-                            s = __fadd_rn(s, __ldcg(g.partial + ((int64_t)cc * g.part_tok + tokidx) *
-                                                                   ((int64_t)g.tiles * kTileRows) +
-                                                    (int64_t)un.tile * kTileRows + r));
-                        acc[i] = s;
+            const uint8_t* abase = stg + g.act_off;
+            if (g.x_mode == X_RAW_F32 || g.x_mode == X_RAW_BF16) {
+                // quantise the raw slices to Q8_1 in this warp's scratch
+                for (int t = 0; t < np; ++t)
+                    for (int kb = 0; kb < un.kbn; ++kb) {
+                        float v;
+                        if (g.x_mode == X_RAW_F32)
+                            v = reinterpret_cast<const float*>(abase + t * g.act_bytes)[kb * 32 + lane];
+                        else
+                            v = __bfloat162float(
+                                reinterpret_cast<const __nv_bfloat16*>(abase + t * g.act_bytes)[kb * 32 + lane]);
+                        warp_quant_q8_1(v, scratch + (t * kChunk + kb) * 36);
                     }
-                    __syncthreads();
-                    gemv_epilogue(g, un, tb2, n2, acc);
-                    __syncthreads();
+                __syncwarp();
+                abase = scratch;
+            }
+            const int astride = (g.x_mode == X_RAW_F32 || g.x_mode == X_RAW_BF16) ? kChunk * 36 : g.act_bytes;
+            for (int t = 0; t < np; ++t) {
+                const uint8_t* ab = abase + t * astride;
+                float part = 0.0f;
+#pragma unroll
+                for (int kb = 0; kb < kChunk; ++kb) {
+                    if (kb < un.kbn) {
+                        const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36 + 4);
+                        int isum = 0;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) isum = __dp4a(w[kb][j], (int)aw[j], isum);
+                        const float da = h2f(*reinterpret_cast<const uint16_t*>(ab + kb * 36));
+                        part = __fmaf_rn(__int2float_rn(isum), __fmul_rn(dw[kb], da), part);
+                    }
                 }
+                const int64_t tokidx = (int64_t)un.tok0 + first + t;
+                __stcg(g.partial + ((int64_t)un.c * g.part_tok + tokidx) * rows_total + (int64_t)un.tile * kTileRows +
+                           un.s * 32 + lane,
+                       part);
             }
         }
-        cons.advance(g);
-    }
-    if (!ok && tid == 0) {
-        // drain: wait (bounded) for every copy still in flight before exiting
-        for (int s = 0; s < issued && s < kGemvStages; ++s) {
-            const int st = issued - 1 - s;
-            mbar_wait_bounded(&bars[st % kGemvStages], (st / kGemvStages) & 1, nullptr, g.budget_ns);
+        if (!ok) break;
+        // stage consumed: refill it with this warp's next unit
+        __syncwarp();
+        fence_proxy_async();
+        {
+            const int nu = grab();
+            if (lane == 0) myunit[st] = nu;
+            if (nu >= 0) {
+                const WUnit nn = wunit(g, nu);
+                wissue_weights<FMT>(g, nn, stg, &mybar[st], min(nn.ntok, tokcap));
+                wissue_acts(g, nn, stg + g.act_off, &mybar[st], 0, min(nn.ntok, tokcap));
+            }
+        }
+        // completion of the tile (the last of its 4 * nchunks units runs the
+        // epilogue), batched per warp so that one fence covers many units
+        if (lane == npend) pending = u;
+        if (++npend == 32) {
+            wcomplete(g, pending, npend);
+            npend = 0;
         }
     }
-    pdl_trigger();
-}
-
-// ============================================================================
-// a9 -- weighted combine in rank order, then Q8_1.  Grid (T, ceil(L/256)).
-// ============================================================================
-__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ o, const int32_t* __restrict__ pos,
-                                                 const float* __restrict__ w, int k, int L,
-                                                 float* __restrict__ ylat, uint8_t* __restrict__ ylq) {
-    pdl_wait();
-    const int t = blockIdx.x;
-    const int n = blockIdx.y * 256 + threadIdx.x;
-    if (n >= L) return;   // L % 32 == 0: whole warps leave together
-    float acc = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        const int p = __ldg(pos + t * k + j);
-        acc = __fmaf_rn(__ldg(w + t * k + j), __ldcg(o + (int64_t)p * L + n), acc);
+    if (ok && npend) wcomplete(g, pending, npend);
+    if (!ok) {
+        // drain: wait (bounded) for this warp's copies still in flight
+        for (int k = 0; k < S; ++k) {
+            const int j = it + k;
+            if (myunit[j % S] >= 0) mbar_wait_bounded(&mybar[j % S], (uint32_t)((j / S) & 1), nullptr, g.budget_ns);
+        }
+        if (xuse) mbar_wait_bounded(&mybar[S], (xuse - 1) & 1u, nullptr, g.budget_ns);
     }
-    ylat[(int64_t)t * L + n] = acc;
-    warp_quant_q8_1(acc, ylq + ((int64_t)t * (L / 32) + n / 32) * 36);
-    pdl_trigger();
 }
 
 // ============================================================================

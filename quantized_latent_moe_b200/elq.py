@@ -57,7 +57,7 @@ SIGNATURES = {
     "elq_workspace_bytes": (SZ, [ctypes.POINTER(LayerC), I32]),
     "elq_moe_layer": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V]),
     "elq_workspace_status": (I32, [V, V]),
-    "elq_layer_kernel_count": (I32, []),
+    "elq_layer_kernel_count": (I32, [ctypes.POINTER(LayerC), I32]),
     "elq_workspace_view": (I32, [ctypes.POINTER(LayerC), I32, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "elq_moe_layer_profiled": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V, I32, V]),
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
@@ -183,6 +183,10 @@ class Layer:
                       self.router_w.data_ptr(),
                       None if self.router_bias is None else self.router_bias.data_ptr(),
                       self.gate_up.struct(), self.down.struct())
+
+    def kernel_count(self, T: int) -> int:
+        s = self.struct()
+        return int(_lib().elq_layer_kernel_count(ctypes.byref(s), T))
 
     def workspace_bytes(self, T: int) -> int:
         s = self.struct()

@@ -71,6 +71,9 @@ def test_layer_validation(L):
     y = ctypes.c_void_p(1 << 28)
     good = _layer()
     assert L.elq_workspace_bytes(ctypes.byref(good), 4) > 0
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 4) == 5
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 9) == 6
+    assert L.elq_layer_kernel_count(None, 4) == 0
     # workspace too small -> refused before any launch
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, ws_small, 16, None) == -4
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, None, 1 << 30, None) == -4
@@ -108,6 +111,7 @@ def test_other_entry_validation(L):
     assert L.elq_latent_proj(ctypes.byref(qm), p, 2, p, None, 0, None) == -4
     assert L.elq_latent_proj(ctypes.byref(_qm(4, 256, 512)), p, 2, p, p, 1 << 30, None) == -2
     assert L.elq_latent_proj(ctypes.byref(_qm(8, 200, 512)), p, 2, p, p, 1 << 30, None) == -2
+    assert L.elq_latent_proj(ctypes.byref(_qm(8, 256, 96)), p, 2, p, p, 1 << 30, None) == -2   # k % 128
     assert L.elq_arena_pack(8, p, 100, 64, p, p, None) == -2
     assert L.elq_arena_pack(8, p, 128, 64, ctypes.c_void_p((1 << 24) + 16), p, None) == -3
     assert L.elq_quantize_weights(2, p, 128, 40, p, p, None) == -2

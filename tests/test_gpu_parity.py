@@ -111,8 +111,8 @@ def test_gate_up_interleave(E, orc):
 
 
 @pytest.mark.parametrize("fmt", [8, 2])
-@pytest.mark.parametrize("N,K,T", [(128, 32, 1), (256, 288, 3), (1792, 4096, 1), (384, 1280, 6),
-                                   (512, 512, 33), (128, 2048, 32), (4096, 1792, 2)])
+@pytest.mark.parametrize("N,K,T", [(128, 128, 1), (256, 384, 3), (1792, 4096, 1), (384, 1280, 6),
+                                   (512, 512, 33), (128, 2048, 32), (4096, 1792, 2), (256, 640, 70)])
 def test_latent_proj_exact(E, orc, fmt, N, K, T):
     W = _gen(5, N + K, (N, K), 0.02)
     X = _gen(6, T, (T, K))
@@ -162,6 +162,26 @@ def test_bucket_exact(E, orc, T, k, E_):
         assert np.array_equal(a.cpu().numpy(), b)
 
 
+def _check_intermediates(E, ly, T, tr):
+    """Every intermediate of the last layer call against the oracle's trace."""
+    v = lambda n: E.workspace_view(ly, T, n).cpu().numpy()
+    assert np.array_equal(v("z").reshape(T, -1), tr["z"])
+    assert np.array_equal(v("zq").reshape(T, -1), tr["zq"])
+    assert np.array_equal(v("logits").reshape(T, -1), tr["logits"])
+    assert np.array_equal(v("idx").reshape(T, -1), tr["idx"])
+    assert np.array_equal(v("weights").reshape(T, -1), tr["w"])
+    assert np.array_equal(v("counts"), tr["counts"])
+    assert np.array_equal(v("offsets"), tr["offsets"])
+    assert np.array_equal(v("perm"), tr["perm"])
+    assert np.array_equal(v("pos"), tr["pos"])
+    # hq and o are stored by pair position on the GPU, by pair id in the trace
+    pos = tr["pos"]
+    assert np.array_equal(v("hq").reshape(T * ly.k, -1)[pos], tr["hq"])
+    assert np.array_equal(v("o").reshape(T * ly.k, -1)[pos], tr["o"])
+    assert np.array_equal(v("y_lat").reshape(T, -1), tr["y_lat"])
+    assert np.array_equal(v("ylq").reshape(T, -1), tr["ylq"])
+
+
 @pytest.mark.parametrize("name", ["tiny", "decode", "verify"])
 def test_layer_exact(E, orc, name):
     wl = synth.WORKLOADS[name]
@@ -170,9 +190,26 @@ def test_layer_exact(E, orc, name):
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
     assert E.workspace_status(ly.workspace(wl.T)) == 0
     ol = oracle_layer(orc, wl, experts=[])
-    ref = oracle_forward(orc, ol, wl, x.float().numpy())
+    tr = oracle_forward(orc, ol, wl, x.float().numpy(), trace=True)
+    ref = tr["y"]
     assert max_abs_rel(y, ref) <= TOL
+    _check_intermediates(E, ly, wl.T, tr)
     assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 9), ("tiny", 33), ("verify", 12)])
+def test_layer_exact_larger_T(E, orc, name, T):
+    """Above 8 tokens the activation quantiser runs as its own kernel."""
+    wl = synth.WORKLOADS[name]
+    ly = gpu_layer(wl)
+    x = synth.make_x(wl, T=T)
+    y = E.moe_layer(ly, x.cuda()).cpu().numpy()
+    ol = oracle_layer(orc, wl, experts=[])
+    tr = oracle_forward(orc, ol, wl, x.float().numpy(), trace=True)
+    _check_intermediates(E, ly, T, tr)
+    xq = E.workspace_view(ly, T, "xq").cpu().numpy().reshape(T, -1)
+    assert np.array_equal(xq, tr["xq"])
+    assert np.array_equal(y, tr["y"])
 
 
 def test_layer_repeat_and_ragged_T(E, orc):
@@ -180,7 +217,7 @@ def test_layer_repeat_and_ragged_T(E, orc):
     wl = synth.WORKLOADS["tiny"]
     ly = gpu_layer(wl)
     ol = oracle_layer(orc, wl)
-    for T in (1, 3, 9, 33, 4, 4):
+    for T in (1, 3, 8, 9, 33, 4, 4, 40):
         x = synth.normal(wl.seed, 77 + T, (T, wl.H))
         y = E.moe_layer(ly, x.cuda()).cpu().numpy()
         ref = ol.forward(x.numpy())

@@ -324,17 +324,25 @@ def test_byte_sizes_from_pages(orc):
 def test_arena_pack_spot_positions(orc):
     r = _rng(10)
     n, K = 256, 96
-    aos = r.integers(0, 256, n * (K // 32) * 34).astype(np.uint8)
-    q, d = orc.arena_pack(8, aos, n, K)
-    blk = aos.reshape(n, K // 32, 34)
     nb = K // 32
-    # row 9, block 2, byte 17: tile 0, slab 2, (9//8)*256 + (17//16)*128 + (9%8)*16 + 1
-    assert q[2 * 4096 + 256 + 128 + 16 + 1] == blk[9, 2, 2 + 17]
-    # row 130 (tile 1, r = 2), block 0, byte 0
-    assert q[(1 * nb + 0) * 4096 + 0 + 0 + 2 * 16] == blk[130, 0, 2]
-    assert bytes(d[((1 * nb + 1) * 128 + 2) * 2:][:2]) == bytes(blk[130, 1, 0:2])
+    aos = r.integers(0, 256, n * nb * 34).astype(np.uint8)
+    q, d = orc.arena_pack(8, aos, n, K)
+    blk = aos.reshape(n, nb, 34)
+    # row 9 (tile 0, slice 0, r 9), block 2, code 17:
+    #   0 + 0 + 2*1024 + (9//8)*256 + (17//16)*128 + (9%8)*16 + 1
+    assert q[2 * 1024 + 256 + 128 + 16 + 1] == blk[9, 2, 2 + 17]
+    # row 130 (tile 1, slice 0, r 2), block 0, code 0
+    assert q[1 * nb * 4096 + 0 + 0 + 2 * 16] == blk[130, 0, 2]
+    # row 200 (tile 1, slice 2, r 8), block 1, code 31
+    assert q[1 * nb * 4096 + 2 * nb * 1024 + 1 * 1024 + 1 * 256 + 128 + 0 + 15] == blk[200, 1, 2 + 31]
+    # scale of row 130, block 1
+    sel = 1 * nb * 128 + 0 + 1 * 32 + 2
+    assert bytes(d[2 * sel:2 * sel + 2]) == bytes(blk[130, 1, 0:2])
     assert np.array_equal(np.sort(q), np.sort(blk[:, :, 2:].reshape(-1)))
     aos4 = r.integers(0, 256, n * nb * 18).astype(np.uint8)
-    q4, _ = orc.arena_pack(2, aos4, n, K)
+    q4, d4 = orc.arena_pack(2, aos4, n, K)
     b4 = aos4.reshape(n, nb, 18)
-    assert q4[(1 * nb + 2) * 2048 + 5 * 16 + 7] == b4[133, 2, 2 + 7]
+    # row 133 (tile 1, slice 0, r 5), block 2, nibble byte 7
+    assert q4[1 * nb * 2048 + 0 + 2 * 512 + 5 * 16 + 7] == b4[133, 2, 2 + 7]
+    # row 255 (tile 1, slice 3, r 31), block 0, byte 0
+    assert q4[1 * nb * 2048 + 3 * nb * 512 + 0 + 31 * 16] == b4[255, 0, 2]
