@@ -308,6 +308,8 @@ cudaError_t launch_router(const float* z, const float* w, const float* bias, int
     RouterArgs a;
     std::memset(&a, 0, sizeof(a));
     a.err = err;
+    a.z = z; a.w = w; a.bias = bias; a.T = T; a.L = L; a.E = E; a.k = k;
+    a.idx = idx; a.wts = wts; a.logits = logits;
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     a.cnt_tok = cnt;
     a.cnt_all = cnt ? cnt + rblocks : nullptr;
