@@ -188,6 +188,29 @@ size_t elq_latent_proj_workspace_bytes(const elq_qmat* w, int32_t T);
 elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* elq_latent_proj without a workspace, for callers that cannot allocate
+ * device memory: code embedded in a host engine whose plugin interface hands
+ * over only input and output pointers, engines that reserve all of HBM up
+ * front for the resident expert arena and forbid allocation afterwards, and
+ * callers that may not call cudaMalloc between setting up and running their
+ * decode loop.  The paper has no counterpart; this is a calling convention of
+ * this library.
+ *  - The scratch (error word, tile counters, chunk partial sums) is one
+ *    file-scope device array of 4 MiB (4,194,304 bytes) that every GPU which
+ *    loads the library holds until the process exits.  A shape whose scratch
+ *    (elq_latent_proj_workspace_bytes) exceeds it returns ELQ_ERR_WORKSPACE;
+ *    e.g. a 1792 x 4096 Q8_0 matrix fits up to 36 tokens.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call clears the error word and the counters on its stream (a
+ *    cudaMemsetAsync) before its kernel; nothing is allocated or freed.
+ *  - All calls share the one array: calls that overlap on the GPU (different
+ *    streams, or several host threads) race and give wrong results.  Order
+ *    them on one stream. */
+elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y,
+                                   void* stream);
+
 /* Grouped experts (a5-a9): bucketing, gate/up with SwiGLU and Q8_1 requant,
  * down, and the weighted combine.  z_q8_1: device T rows of L/32 Q8_1 blocks;
  * idx, weights: device [T][k] as elq_router_topk writes them; y_lat: device

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <functional>
+#include <mutex>
 
 #include "../../include/elq.h"
 #include "elq_kernels.cuh"
@@ -644,6 +645,60 @@ elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free latent projection.  Its scratch (error word, tile counters,
+// chunk partial sums) lives in one file-scope device array instead of a
+// caller-provided workspace.  In host code the array's name only stands for
+// the symbol: its device address is looked up with cudaGetSymbolAddress, once
+// per device, with that device current.
+
+namespace {
+constexpr size_t kStaticScratchBytes = (size_t)4 << 20;   // 4 MiB, held by every GPU that loads the library
+}
+
+static __device__ __align__(256) unsigned char g_elq_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices];
+
+elq_status static_scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ELQ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return ELQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_elq_static_scratch) != cudaSuccess || !p) return ELQ_ERR_CUDA;
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return ELQ_OK;
+}
+}  // namespace
+
+extern "C" elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y,
+                                              void* stream) {
+    if (!w) return ELQ_ERR_INVALID_ARG;
+    elq_status st = check_qmat(w, w->n_rows, w->k);
+    if (st != ELQ_OK) return st;
+    if (T < 0) return ELQ_ERR_INVALID_ARG;
+    if (T == 0) return ELQ_OK;
+    if (!x_q8_1 || !y) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(x_q8_1, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
+    if (proj_layout(w, T, nullptr).total > kStaticScratchBytes) return ELQ_ERR_WORKSPACE;
+    void* base = nullptr;
+    if ((st = static_scratch_address(&base)) != ELQ_OK) return st;
+    ProjWs lay = proj_layout(w, T, base);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: the error word and the
+    // tile counters must start at zero
+    if (cudaMemsetAsync(lay.err, 0, (64 + lay.plan.counter_ints) * sizeof(int), s) != cudaSuccess)
+        return ELQ_ERR_CUDA;
+    WArgs g = dense_w(w, T, x_q8_1, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, lay.partial, lay.counters, lay.err);
+    return cuda_status(launch_w(g, w->fmt, lay.plan, s, false));
+}
 
 namespace {
 

@@ -53,6 +53,7 @@ SIGNATURES = {
     "elq_route_bucket": (I32, [V, I32, I32, I32, V, V, V, V, V]),
     "elq_latent_proj_workspace_bytes": (SZ, [ctypes.POINTER(QMat), I32]),
     "elq_latent_proj": (I32, [ctypes.POINTER(QMat), V, I32, V, V, SZ, V]),
+    "elq_latent_proj_noalloc": (I32, [ctypes.POINTER(QMat), V, I32, V, V]),
     "elq_moe_experts_grouped": (I32, [ctypes.POINTER(LayerC), V, V, V, I32, V, V, SZ, V]),
     "elq_workspace_bytes": (SZ, [ctypes.POINTER(LayerC), I32]),
     "elq_moe_layer": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V]),
@@ -251,6 +252,19 @@ def latent_proj(m: QMatrix, xq: torch.Tensor, T: int, ws=None, stream=None) -> t
         ws = ws[off:off + n]
     _ck(_lib().elq_latent_proj(ctypes.byref(s), _ptr(xq), T, _ptr(y), _ptr(ws), ws.numel(),
                                _stream(stream)), "elq_latent_proj")
+    return y
+
+
+def latent_proj_noalloc(m: QMatrix, xq: torch.Tensor, T: int, y: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """elq_latent_proj_noalloc: the projection with the library's own static
+    scratch instead of a workspace (for callers that cannot allocate).  Calls
+    share that scratch, so they must not overlap on the GPU."""
+    s = m.struct()
+    if y is None:
+        y = torch.empty(T, m.n_rows, dtype=torch.float32, device=m.q.device)
+    _ck(_lib().elq_latent_proj_noalloc(ctypes.byref(s), _ptr(xq), T, _ptr(y), _stream(stream)),
+        "elq_latent_proj_noalloc")
     return y
 
 

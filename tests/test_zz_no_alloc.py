@@ -1,0 +1,46 @@
+"""The allocation-free projection entry point, elq_latent_proj_noalloc.
+
+It serves callers that cannot allocate device memory (an engine plugin given
+only input and output pointers, an engine that reserves all of HBM for its
+resident weights up front): its scratch is a static device array of the
+library.  This file runs last so that a failure here leaves every other test
+already run; it also passes on its own in a fresh process.
+"""
+import pytest
+import torch
+
+from quantized_latent_moe_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def E():
+    from quantized_latent_moe_b200 import build, elq
+    build.build()
+    elq.lib()
+    assert torch.cuda.is_available()
+    return elq
+
+
+@pytest.mark.parametrize("fmt,N,K,T", [(8, 1792, 4096, 1), (8, 4096, 1792, 3), (2, 1280, 3072, 6)])
+def test_noalloc_matches_workspace_entry(E, fmt, N, K, T):
+    W = synth.normal(11, N + K, (N, K), 0.02).cuda()
+    X = synth.normal(12, T, (T, K)).cuda()
+    m = E.QMatrix.from_f32(W, fmt)
+    xq = E.quantize_q8_1(X)
+    ref = E.latent_proj(m, xq, T)
+    # two calls in a row share (and leave behind) the same static scratch
+    for _ in range(2):
+        y = E.latent_proj_noalloc(m, xq, T)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref)      # the projection tests' tolerance: bit-identical
+
+
+def test_noalloc_rejects_oversize(E):
+    N, K, T = 4096, 1792, 64             # 7 chunks x 64 tokens x 4096 rows x 4 B > 4 MiB
+    m = E.QMatrix(8, N, K)
+    xq = torch.zeros(T, K // 32 * 36, dtype=torch.uint8, device="cuda")
+    with pytest.raises(E.ElqError) as ex:
+        E.latent_proj_noalloc(m, xq, T)
+    assert ex.value.status == -4
