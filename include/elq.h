@@ -226,10 +226,12 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
                          float* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels one elq_moe_layer call launches at this T (0 if the
- * layer is invalid), in order: [activation quantiser, for T > 8], D projection
- * (quantising x itself for T <= 8; + latent Q8_1), router (+ top-k,
- * bucketing), gate/up (+ SwiGLU, Q8_1), down (+ weighted combine, Q8_1), U
- * projection. */
+ * layer is invalid).  Decode/verify path, in order: [activation quantiser,
+ * for T > 8], D projection (quantising x itself for T <= 8; + latent Q8_1),
+ * router (+ top-k, bucketing), gate/up (+ SwiGLU, Q8_1), down (+ weighted
+ * combine, Q8_1), U projection.  Tensor-core path (T >= 64 and every matrix
+ * Q8_0): activation quantiser, x packing, D, router, slot map, z packing,
+ * gate/up, down (+ combine), U. */
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T);
 
 /* elq_moe_layer that also records CUDA events on the stream: events[0] before
@@ -248,6 +250,8 @@ elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t
  * (int32 [E]), 7 offsets (int32 [E+1]), 8 perm (int32 [T*k]), 9 pos, 10 hq
  * (Q8_1 [T*k][I/32], by pair position), 11 o (fp32 [T*k][L], by position),
  * 12 y_lat (fp32 [T][L]), 13 ylq (Q8_1), 14 number of routed experts (int32).
+ * On the tensor-core path (T >= 64, all matrices Q8_0) hq and o are kept in
+ * padded per-expert slots instead, and their views return ELQ_ERR_INVALID_ARG.
  * Sets *offset (bytes from the workspace start) and *bytes; returns ELQ_OK or
  * ELQ_ERR_INVALID_ARG.  The values are those of the last call on that
  * workspace once the stream has reached its end. */

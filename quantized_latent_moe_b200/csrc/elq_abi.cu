@@ -10,7 +10,7 @@
 #include <mutex>
 
 #include "../../include/elq.h"
-#include "elq_kernels.cuh"
+#include "elq_tc.cuh"
 
 using namespace elq;
 
@@ -21,6 +21,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kRouterSmemMax = 200 * 1024;           // dynamic shared memory cap of router/bucket
 constexpr int kGemvSmemMax = 225 * 1024;             // dynamic shared memory cap of the GEMV
 constexpr int kRawMaxT = 8;                          // D quantises x itself up to this many tokens
+constexpr int kTcMinT = 64;                          // tensor-core path from this many tokens (Q8_0 weights)
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -182,23 +183,75 @@ struct Carve {
     }
 };
 
+int64_t round16(int64_t x) { return (x + 15) / 16 * 16; }
+
+bool tc_path(int fmt, int T) { return fmt == ELQ_Q8_0 && T >= kTcMinT; }
+
 struct ProjWs {
     int* err;
     int* counters;
     float* partial;
+    uint8_t* bq;            // tensor-core path: packed activations
+    float* bd;
+    int64_t bstride;
+    bool tc;
     WPlan plan;
     size_t total;
 };
 
 ProjWs proj_layout(const elq_qmat* w, int T, void* base) {
     ProjWs ws;
+    ws.tc = tc_path(w->fmt, T);
     ws.plan = plan_w(w->fmt, X_Q81_TOKEN, w->n_rows, w->k, 1, T, T);
+    if (ws.tc) {
+        ws.plan.partial_bytes = 0;
+        ws.plan.counter_ints = 0;
+    }
     Carve c;
     ws.err = c.take<int>(base, (64 + ws.plan.counter_ints) * sizeof(int));
     ws.counters = ws.err ? ws.err + 64 : nullptr;
     ws.partial = c.take<float>(base, ws.plan.partial_bytes);
+    ws.bstride = round16(T);
+    const int nb = w->k / 32;
+    ws.bq = ws.tc ? c.take<uint8_t>(base, (size_t)nb * ws.bstride * 32) : nullptr;
+    ws.bd = ws.tc ? c.take<float>(base, (size_t)nb * ws.bstride * 4) : nullptr;
     ws.total = c.off;
     return ws;
+}
+
+bool g_optin_tc[kMaxDevices];
+
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s, bool pdl) {
+    const int64_t n = a.bstride * a.nb;
+    return launch(k_pack_b, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, a);
+}
+
+cudaError_t launch_tc(TcArgs g, cudaStream_t s, bool pdl) {
+    g.budget_ns = kWaitBudgetNs;
+    cudaError_t e = smem_optin(k_tcgemm, kTcSmem, g_optin_tc);
+    if (e != cudaSuccess) return e;
+    return launch(k_tcgemm, dim3(sm_count()), dim3(kTcThreads), (size_t)kTcSmem, s, pdl, g);
+}
+
+TcArgs dense_tc(const elq_qmat* w, int T, const uint8_t* bq, const float* bd, int64_t bstride, int out_mode,
+                float* y, uint8_t* yq, int* err) {
+    TcArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.q = static_cast<const uint8_t*>(w->q);
+    g.d = static_cast<const uint16_t*>(w->d);
+    g.nb = w->k / 32;
+    g.rtiles = w->n_rows / kTileRows;
+    g.T = T;
+    g.bq = bq;
+    g.bd = bd;
+    g.bstride = bstride;
+    g.out_mode = out_mode;
+    g.y = y;
+    g.y_ld = w->n_rows;
+    g.yq = yq;
+    g.yq_ld = w->n_rows / 32;
+    g.err = err;
+    return g;
 }
 
 struct LayerWs {
@@ -221,6 +274,13 @@ struct LayerWs {
     float* ylat;
     uint8_t* ylq;
     float* partial;
+    // tensor-core path
+    bool tc;
+    int64_t tstride, sstride;   // slots of the dense (tokens) and the expert (pairs, padded) B buffers
+    uint8_t *bxq, *bzq, *bhq, *byq;
+    float *bxd, *bzd, *bhd, *byd;
+    int32_t *slot_off, *tt_off, *pair_slot;
+    int* cnt_comb_tc;
     WPlan pd, pgu, pdn, pu;
     bool raw;
     size_t total;
@@ -231,6 +291,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     const int H = ly->H, L = ly->L, E = ly->E, k = ly->k, I = ly->I;
     const int64_t P = (int64_t)T * k;
     const int gmax = (int)std::min<int64_t>(E, P);
+    w.tc = tc_path(ly->D.fmt, T) && tc_path(ly->U.fmt, T) && tc_path(ly->gate_up.fmt, T) && tc_path(ly->down.fmt, T);
     w.raw = T <= kRawMaxT;
     const int dmode = w.raw ? (x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32) : X_Q81_TOKEN;
     w.pd = plan_w(ly->D.fmt, dmode, L, H, 1, T, T);
@@ -266,9 +327,34 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.o = c.take<float>(base, (size_t)P * L * 4);
     w.ylat = c.take<float>(base, (size_t)T * L * 4);
     w.ylq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
-    const size_t part = std::max(std::max(w.pd.partial_bytes, w.pgu.partial_bytes),
-                                 std::max(w.pdn.partial_bytes, w.pu.partial_bytes));
-    w.partial = c.take<float>(base, part);
+    w.tstride = round16(T);
+    w.sstride = round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
+    if (!w.tc) {
+        const size_t part = std::max(std::max(w.pd.partial_bytes, w.pgu.partial_bytes),
+                                     std::max(w.pdn.partial_bytes, w.pu.partial_bytes));
+        w.partial = c.take<float>(base, part);
+        w.bxq = w.bzq = w.bhq = w.byq = nullptr;
+        w.bxd = w.bzd = w.bhd = w.byd = nullptr;
+        w.slot_off = w.tt_off = w.pair_slot = nullptr;
+        w.cnt_comb_tc = nullptr;
+    } else {
+        w.partial = nullptr;
+        const int nbH = H / 32, nbL = L / 32, nbI = I / 32;
+        w.bxq = c.take<uint8_t>(base, (size_t)nbH * w.tstride * 32);
+        w.bxd = c.take<float>(base, (size_t)nbH * w.tstride * 4);
+        w.bzq = c.take<uint8_t>(base, (size_t)nbL * w.sstride * 32);
+        w.bzd = c.take<float>(base, (size_t)nbL * w.sstride * 4);
+        w.bhq = c.take<uint8_t>(base, (size_t)nbI * w.sstride * 32);
+        w.bhd = c.take<float>(base, (size_t)nbI * w.sstride * 4);
+        w.byq = c.take<uint8_t>(base, (size_t)nbL * w.tstride * 32);
+        w.byd = c.take<float>(base, (size_t)nbL * w.tstride * 4);
+        w.slot_off = c.take<int32_t>(base, (size_t)(E + 1) * 4);
+        w.tt_off = c.take<int32_t>(base, (size_t)(E + 1) * 4);
+        w.pair_slot = c.take<int32_t>(base, (size_t)P * 4);
+        w.cnt_comb_tc = c.take<int>(base, (size_t)T * (L / 32) * 4);
+        // o is stored by slot on this path
+        w.o = c.take<float>(base, (size_t)w.sstride * L * 4);
+    }
     w.total = c.off;
     return w;
 }
@@ -365,7 +451,76 @@ elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8
 elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
                      size_t ws_bytes, void* stream, void* const* events, int32_t n_events);
 
-int layer_kernels(int T) { return T <= kRawMaxT ? 5 : 6; }
+// Tensor-core experts: slots from the routing, gathered z codes, gate/up (+SwiGLU
+// into the packed hq buffer), down (+combine into y_lat, Q8_1 rows and the
+// packed buffer the U projection reads).
+elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, const float* wts,
+                          float* y_lat, cudaStream_t s, bool pdl, const std::function<bool()>& mark) {
+    const int L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    const int P = T * k;
+    if (launch(k_tc_route, dim3(1), dim3(1024), 0, s, pdl, (const int32_t*)w.offsets, (const int32_t*)w.act,
+               (const int32_t*)w.n_act, (const int32_t*)w.idx, (const int32_t*)w.pos, P, E, w.slot_off, w.tt_off,
+               w.pair_slot) != cudaSuccess ||
+        !mark())
+        return ELQ_ERR_CUDA;
+    PackArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    pa.x = zq;
+    pa.nb = L / 32;
+    pa.mode = PACK_PAIRS;
+    pa.offsets = w.offsets;
+    pa.slot_off = w.slot_off;
+    pa.perm = w.perm;
+    pa.kslots = k;
+    pa.E = E;
+    pa.bq = w.bzq;
+    pa.bd = w.bzd;
+    pa.bstride = w.sstride;
+    if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    TcArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.q = static_cast<const uint8_t*>(ly->gate_up.q);
+    g.d = static_cast<const uint16_t*>(ly->gate_up.d);
+    g.nb = L / 32;
+    g.rtiles = 2 * I / kTileRows;
+    g.q_gstride = (int64_t)g.rtiles * g.nb * kQ80Slab;
+    g.d_gstride = (int64_t)g.rtiles * g.nb * kTileRows;
+    g.act = w.act; g.n_act = w.n_act; g.slot_off = w.slot_off; g.offsets = w.offsets; g.tt_off = w.tt_off;
+    g.T = T;
+    g.bq = w.bzq; g.bd = w.bzd; g.bstride = w.sstride;
+    g.out_mode = TC_OUT_SWIGLU;
+    g.cq = w.bhq; g.cd = w.bhd; g.cstride = w.sstride;
+    g.err = w.err;
+    if (launch_tc(g, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    TcArgs h;
+    std::memset(&h, 0, sizeof(h));
+    h.q = static_cast<const uint8_t*>(ly->down.q);
+    h.d = static_cast<const uint16_t*>(ly->down.d);
+    h.nb = I / 32;
+    h.rtiles = L / kTileRows;
+    h.q_gstride = (int64_t)h.rtiles * h.nb * kQ80Slab;
+    h.d_gstride = (int64_t)h.rtiles * h.nb * kTileRows;
+    h.act = w.act; h.n_act = w.n_act; h.slot_off = w.slot_off; h.offsets = w.offsets; h.tt_off = w.tt_off;
+    h.T = T;
+    h.bq = w.bhq; h.bd = w.bhd; h.bstride = w.sstride;
+    h.out_mode = TC_OUT_F32_COMBINE;
+    h.y = w.o; h.y_ld = L;
+    h.cq = w.byq; h.cd = w.byd; h.cstride = w.tstride;
+    h.wts = wts; h.perm = w.perm; h.pair_slot = w.pair_slot; h.kslots = k; h.cnt_comb = w.cnt_comb_tc;
+    h.ylat = y_lat; h.ylq = w.ylq;
+    h.err = w.err;
+    if (launch_tc(h, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    return ELQ_OK;
+}
+
+bool layer_tc(const elq_layer* ly, int T) {
+    return tc_path(ly->D.fmt, T) && tc_path(ly->U.fmt, T) && tc_path(ly->gate_up.fmt, T) && tc_path(ly->down.fmt, T);
+}
+
+int layer_kernels(const elq_layer* ly, int T) {
+    if (layer_tc(ly, T)) return 9;
+    return T <= kRawMaxT ? 5 : 6;
+}
 
 }  // namespace
 
@@ -527,8 +682,23 @@ elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, flo
     ProjWs lay = proj_layout(w, T, ws);
     if (!ws || ws_bytes < lay.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (lay.tc) {
+        PackArgs pa;
+        std::memset(&pa, 0, sizeof(pa));
+        pa.x = static_cast<const uint8_t*>(x_q8_1);
+        pa.nb = w->k / 32;
+        pa.mode = PACK_DENSE;
+        pa.T = T;
+        pa.bq = lay.bq;
+        pa.bd = lay.bd;
+        pa.bstride = lay.bstride;
+        if (launch_pack(pa, s, false) != cudaSuccess) return ELQ_ERR_CUDA;
+        TcArgs g = dense_tc(w, T, lay.bq, lay.bd, lay.bstride, TC_OUT_F32, y, nullptr, lay.err);
+        return cuda_status(launch_tc(g, s, true));
+    }
     WArgs g = dense_w(w, T, x_q8_1, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, lay.partial, lay.counters, lay.err);
-    return cuda_status(launch_w(g, w->fmt, lay.plan, static_cast<cudaStream_t>(stream), false));
+    return cuda_status(launch_w(g, w->fmt, lay.plan, s, false));
 }
 
 size_t elq_workspace_bytes(const elq_layer* layer, int32_t T) {
@@ -558,6 +728,12 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, s, false, idx, (int)P, E, w.counts, w.offsets,
                w.perm, w.pos, w.act, w.n_act);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    if (w.tc) {
+        // the slot map reads idx from the workspace copy the layer call would have
+        if (cudaMemcpyAsync(w.idx, idx, (size_t)P * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return ELQ_ERR_CUDA;
+        return run_experts_tc(layer, w, T, static_cast<const uint8_t*>(z_q8_1), weights, y_lat, s, true,
+                              []() { return true; });
+    }
     return run_experts(layer, w, T, static_cast<const uint8_t*>(z_q8_1), weights, y_lat, s, true,
                        []() { return true; }, true);
 }
@@ -569,14 +745,15 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
 
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T) {
     if (check_layer(layer, T) != ELQ_OK || T <= 0) return 0;
-    return layer_kernels(T);
+    return layer_kernels(layer, T);
 }
 
 elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y,
                                   void* ws, size_t ws_bytes, void* const* events, int32_t n_events, void* stream) {
-    if (!events || T <= 0) return ELQ_ERR_INVALID_ARG;
-    if (n_events < layer_kernels(T) + 1) return ELQ_ERR_INVALID_ARG;
-    for (int i = 0; i < layer_kernels(T) + 1; ++i)
+    if (!events || T <= 0 || check_layer(layer, T) != ELQ_OK) return ELQ_ERR_INVALID_ARG;
+    const int nk = layer_kernels(layer, T);
+    if (n_events < nk + 1) return ELQ_ERR_INVALID_ARG;
+    for (int i = 0; i < nk + 1; ++i)
         if (!events[i]) return ELQ_ERR_INVALID_ARG;
     return run_layer(layer, x, x_type, T, y, ws, ws_bytes, stream, events, n_events);
 }
@@ -600,8 +777,8 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, 
     case 7: p = w.offsets; n = (E + 1) * 4; break;
     case 8: p = w.perm; n = P * 4; break;
     case 9: p = w.pos; n = P * 4; break;
-    case 10: p = w.hq; n = P * (I / 32) * 36; break;
-    case 11: p = w.o; n = P * L * 4; break;
+    case 10: p = w.tc ? nullptr : w.hq; n = P * (I / 32) * 36; break;
+    case 11: p = w.tc ? nullptr : w.o; n = P * L * 4; break;
     case 12: p = w.ylat; n = Tz * L * 4; break;
     case 13: p = w.ylq; n = Tz * (L / 32) * 36; break;
     case 14: p = w.n_act; n = 4; break;
@@ -710,7 +887,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     if (T == 0) return ELQ_OK;
     if (!x || !y) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
-    if (events && n_events < layer_kernels(T) + 1) return ELQ_ERR_INVALID_ARG;
+    if (events && n_events < layer_kernels(layer, T) + 1) return ELQ_ERR_INVALID_ARG;
     if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
     LayerWs w = layer_layout(layer, T, ws, x_type);
     if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
@@ -725,6 +902,38 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     const bool pdl = (events == nullptr);
     cudaError_t e;
     if (!mark()) return ELQ_ERR_CUDA;
+    if (w.tc) {
+        // prefill: a1 quantiser, packed x, D on the tensor cores (z, zq), router,
+        // then the tensor-core experts and U
+        const int64_t nblk = (int64_t)T * (H / 32);
+        if (x_type == ELQ_BF16)
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        else
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        PackArgs pa;
+        std::memset(&pa, 0, sizeof(pa));
+        pa.x = w.xq;
+        pa.nb = H / 32;
+        pa.mode = PACK_DENSE;
+        pa.T = T;
+        pa.bq = w.bxq;
+        pa.bd = w.bxd;
+        pa.bstride = w.tstride;
+        if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32_Q81, w.z, w.zq, w.err);
+        if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits,
+                          w.cnt_router, true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl, w.err);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        st = run_experts_tc(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark);
+        if (st != ELQ_OK) return st;
+        TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, TC_OUT_F32, y, nullptr, w.err);
+        if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        return ELQ_OK;
+    }
     // a1 + a2 + a4: D projection of x (quantised by the GEMV itself at small T)
     WArgs gd;
     if (w.raw) {

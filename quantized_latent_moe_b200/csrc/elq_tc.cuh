@@ -1,0 +1,599 @@
+// elq_tc.cuh -- the prefill path: grouped int8 GEMM on the 5th-generation
+// tensor cores (tcgen05.mma kind::i8, accumulators in TMEM).
+//
+// A Q8_0 x Q8_1 row dot needs, for every 32-wide block, its exact int32 sum
+// rescaled by f32(d_w) * f32(d_a) and added in a fixed order (8-block chunks,
+// see elq.h).  One MMA with K = 32 is exactly one block, so each block's MMA
+// writes a fresh TMEM accumulator (no accumulation inside the tensor core) and
+// the epilogue warps drain it and apply the ordered fp32 rescale.
+//
+// CTA: warp 0 issues the bulk copies, warp 1 issues the MMAs (one elected
+// thread each), warps 2..9 drain TMEM (warp w reads TMEM lanes 32*(w%4) ..
+// +31, i.e. weight rows; warps 2..5 take tokens 0..31 of the tile, warps 6..9
+// tokens 32..63).  Tile = 128 weight rows x up to 64 tokens x all K.
+//
+// Operands in shared memory use the K-major, no-swizzle canonical layout:
+// 8-row x 16-byte core matrices, LBO = 128 B (next core matrix along K), SBO =
+// 256 B (next 8 rows).  A weight tile's block kb is assembled from the four
+// 1 KB slice pieces of the arena; the activations come pre-packed in the same
+// layout ("B buffers": [kb][slot/8][2][8][16] codes and [kb][slot] fp32 scales).
+#pragma once
+
+#include "elq_kernels.cuh"
+
+namespace elq {
+
+// ---- tcgen05 primitives ----------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] = A[smem] x B[smem]^T (int8 x int8 -> int32), accumulate if acc != 0.
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+// Arrive (once) on an mbarrier when all MMAs this thread issued so far are done.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Bounded mbarrier wait taken by lane 0 for the whole warp (the result is the
+// same in every lane, so warp-collective instructions after it stay converged).
+__device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity, int* err, uint64_t budget_ns) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, err, budget_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Shared-memory matrix descriptor: K-major, no swizzle, version 1.
+__device__ __forceinline__ uint64_t umma_desc(const void* p, uint32_t lbo, uint32_t sbo) {
+    const uint64_t a = smem_addr(p);
+    return ((a >> 4) & 0x3FFFull) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor: s8 x s8 -> s32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_i8(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- B buffers: Q8_1 rows -> canonical slots ---------------------------------
+//
+// Slot s of a B buffer holds one activation row: for block kb its 32 codes at
+// bq + kb*bstride*32 + (s/8)*256 + (c/16)*128 + (s%8)*16 + c%16, its scale at
+// bd[kb*bstride + s].  Slots without a row hold zeros.
+
+enum { PACK_DENSE = 0, PACK_PAIRS = 1 };
+
+struct PackArgs {
+    const uint8_t* x;           // Q8_1 AoS rows, nb blocks each
+    int nb;
+    int mode;
+    int T;                      // PACK_DENSE: rows 0 .. T-1 -> slots 0 .. T-1
+    // PACK_PAIRS: expert e's pairs perm[off[e] + i] go to slot slot_off[e] + i; row = pair / k
+    const int32_t* offsets;
+    const int32_t* slot_off;
+    const int32_t* perm;
+    int kslots, E;
+    uint8_t* bq;
+    float* bd;
+    int64_t bstride;            // slots in the buffer (multiple of 16)
+};
+
+// One thread per (slot, block).
+__global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
+    pdl_wait();
+    const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= a.bstride * a.nb) return;
+    const int64_t slot = id / a.nb;
+    const int kb = (int)(id % a.nb);
+    int64_t row = -1;
+    if (a.mode == PACK_DENSE) {
+        if (slot < a.T) row = slot;
+    } else {
+        // the expert whose padded slot range holds this slot
+        int lo = 0, hi = a.E;   // slot_off[lo] <= slot < slot_off[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldcg(a.slot_off + mid) <= slot) lo = mid; else hi = mid;
+        }
+        const int i = (int)(slot - __ldcg(a.slot_off + lo));
+        const int n = __ldcg(a.offsets + lo + 1) - __ldcg(a.offsets + lo);
+        if (i < n) row = __ldcg(a.perm + __ldcg(a.offsets + lo) + i) / a.kslots;
+    }
+    uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
+    float dd = 0.0f;
+    if (row >= 0) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(a.x + (row * a.nb + kb) * 36);
+        const uint32_t w0 = __ldcg(src);
+        lo4 = make_uint4(__ldcg(src + 1), __ldcg(src + 2), __ldcg(src + 3), __ldcg(src + 4));
+        hi4 = make_uint4(__ldcg(src + 5), __ldcg(src + 6), __ldcg(src + 7), __ldcg(src + 8));
+        dd = h2f((uint16_t)(w0 & 0xffff));
+    }
+    uint8_t* dst = a.bq + (int64_t)kb * a.bstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
+    *reinterpret_cast<uint4*>(dst) = lo4;
+    *reinterpret_cast<uint4*>(dst + 128) = hi4;
+    a.bd[(int64_t)kb * a.bstride + slot] = dd;
+    pdl_trigger();
+}
+
+constexpr int kTcN = 64;            // tokens per tile
+
+// ---- routing -> padded slots -------------------------------------------------
+// slot_off[e] = sum over e' < e of roundup(count(e'), 16); tt_off[a] = sum over
+// active experts a' < a of ceil(count / 64); pair_slot[p] = the slot of pair p.
+// One CTA.
+__global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const int32_t* act, const int32_t* n_act,
+                                                   const int32_t* idx, const int32_t* pos, int P, int E,
+                                                   int32_t* slot_off, int32_t* tt_off, int32_t* pair_slot) {
+    pdl_wait();
+    __shared__ int s_slot[1025];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+        int local = 0;
+        for (int e = e0; e < e1; ++e) local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + 15) & ~15;
+        int incl = local;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int e = e0; e < e1; ++e) {
+            s_slot[e] = run;
+            slot_off[e] = run;
+            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + 15) & ~15;
+        }
+        if (lane == 31) {
+            s_slot[E] = incl;
+            slot_off[E] = incl;
+        }
+    } else if (warp == 1) {
+        const int na = __ldcg(n_act);
+        const int per = (na + 31) / 32;
+        const int a0 = min(na, lane * per), a1 = min(na, a0 + per);
+        int local = 0;
+        for (int a = a0; a < a1; ++a) {
+            const int e = __ldcg(act + a);
+            local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + kTcN - 1) / kTcN;
+        }
+        int incl = local;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int a = a0; a < a1; ++a) {
+            tt_off[a] = run;
+            const int e = __ldcg(act + a);
+            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + kTcN - 1) / kTcN;
+        }
+        if (lane == 31) tt_off[na] = incl;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        const int e = __ldcg(idx + p);
+        pair_slot[p] = s_slot[e] + __ldcg(pos + p) - __ldcg(offsets + e);
+    }
+    pdl_trigger();
+}
+
+// ---- the GEMM ------------------------------------------------------------------
+
+constexpr int kTcKS = 4;            // blocks per pipeline stage
+constexpr int kTcStages = 4;
+constexpr int kTcBufs = 4;          // TMEM accumulators of kTcN columns
+constexpr int kTcThreads = 320;
+constexpr int kTcStageA = kTcKS * 4096;
+constexpr int kTcStageB = kTcKS * kTcN * 32;
+constexpr int kTcStageDw = kTcKS * kTileRows * 2;
+constexpr int kTcStageDa = kTcKS * kTcN * 4;
+constexpr int kTcStage = kTcStageA + kTcStageB + kTcStageDw + kTcStageDa;
+constexpr int kTcXchg = kTcN * 64 * 4;                     // SwiGLU exchange of the up rows
+constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg;
+
+enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3 };
+
+struct TcArgs {
+    const uint8_t* q;           // weight arena of group 0
+    const uint16_t* d;
+    int64_t q_gstride, d_gstride;
+    int nb, rtiles;
+    // groups: dense (act == NULL: one group of T tokens in slots 0 .. T-1) or
+    // the routed experts (slot_off/counts per expert, tt_off per active expert)
+    const int32_t* act;
+    const int32_t* n_act;
+    const int32_t* slot_off;    // [E+1]
+    const int32_t* offsets;     // [E+1] pair offsets (tokens per expert = difference)
+    const int32_t* tt_off;      // [E+1] token tiles before active expert a
+    int T;
+    // B operand
+    const uint8_t* bq;
+    const float* bd;
+    int64_t bstride;
+    // outputs
+    int out_mode;
+    float* y;                   // fp32 rows, by token (dense) or slot (experts)
+    int64_t y_ld;
+    uint8_t* yq;                // Q8_1 AoS rows (TC_OUT_F32_Q81)
+    int64_t yq_ld;
+    uint8_t* cq;                // canonical B buffer written by the epilogue (SWIGLU: hq; COMBINE: ylq)
+    float* cd;
+    int64_t cstride;
+    // combine (down): weights, the slot of each pair, per (token, 32-row block) counters
+    const float* wts;
+    const int32_t* perm;        // pair of each position (experts)
+    const int32_t* pair_slot;   // [T*k] slot of each pair
+    int kslots;
+    int* cnt_comb;              // [T][L/32]
+    float* ylat;
+    uint8_t* ylq;               // Q8_1 AoS of y_lat
+    int* err;
+    uint64_t budget_ns;
+};
+
+struct TcUnit {
+    int rt, e, slot0, nvalid, ncols;
+    bool valid;
+};
+
+__device__ __forceinline__ TcUnit tc_unit(const TcArgs& g, int u) {
+    TcUnit r;
+    r.rt = u % g.rtiles;
+    const int q = u / g.rtiles;
+    if (!g.act) {
+        r.e = 0;
+        r.slot0 = q * kTcN;
+        r.nvalid = min(kTcN, g.T - r.slot0);
+    } else {
+        const int na = __ldcg(g.n_act);
+        int lo = 0, hi = na;    // tt_off[lo] <= q < tt_off[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldcg(g.tt_off + mid) <= q) lo = mid; else hi = mid;
+        }
+        r.e = __ldcg(g.act + lo);
+        const int tt = q - __ldcg(g.tt_off + lo);
+        r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
+        const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
+        r.nvalid = min(kTcN, cnt - tt * kTcN);
+    }
+    r.ncols = (r.nvalid + 15) & ~15;
+    r.valid = r.nvalid > 0;
+    return r;
+}
+
+__device__ __forceinline__ int tc_units(const TcArgs& g) {
+    if (!g.act) return ((g.T + kTcN - 1) / kTcN) * g.rtiles;
+    return __ldcg(g.tt_off + __ldcg(g.n_act)) * g.rtiles;
+}
+
+// Write one 32-value Q8_1 block (held one value per lane) into a canonical B
+// buffer at (slot, kb): the warp-level quantiser, then the canonical scatter.
+__device__ __forceinline__ void warp_quant_canonical(float v, uint8_t* cq, float* cd, int64_t cstride,
+                                                     int64_t slot, int kb, uint8_t* scratch36) {
+    const int lane = threadIdx.x & 31;
+    warp_quant_q8_1(v, scratch36);
+    __syncwarp();
+    uint8_t* dst = cq + (int64_t)kb * cstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
+    if (lane < 8) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(scratch36 + 4)[lane];
+        reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] = w;
+    }
+    if (lane == 0) cd[(int64_t)kb * cstride + slot] = h2f(*reinterpret_cast<const uint16_t*>(scratch36));
+    __syncwarp();
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
+    extern __shared__ __align__(1024) uint8_t tcsm[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(tcsm);            // [stages]
+    uint64_t* empty = full + kTcStages;                             // [stages]
+    uint64_t* tfull = empty + kTcStages;                            // [bufs]
+    uint64_t* tempty = tfull + kTcBufs;                             // [bufs]
+    uint64_t* xfull = tempty + kTcBufs;                             // up rows handed over (4 warps)
+    uint64_t* xempty = xfull + 1;                                   // ... and taken (4 warps)
+    uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(xempty + 1);
+    int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
+    uint8_t* scratch = tcsm + 512;                                  // 8 warps x 36 B quantiser scratch
+    uint8_t* stages = tcsm + 1024;
+    float* xchg = reinterpret_cast<float*>(tcsm + 1024 + kTcStages * kTcStage);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + 8);      // the MMA commit + 8 epilogue warps
+        }
+        for (int b = 0; b < kTcBufs; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        mbar_init(xfull, 4);
+        mbar_init(xempty, 4);
+        *abort_sm = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_sm, kTcBufs * kTcN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_sm;
+    pdl_wait();
+
+    const int n_units = tc_units(g);
+    const int u0 = (int)((int64_t)n_units * blockIdx.x / gridDim.x);
+    const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
+    const int kstages = g.nb / kTcKS;
+    volatile int* abort_v = abort_sm;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int it = 0;
+            for (int u = u0; u < u1 && !*abort_v; ++u) {
+                const TcUnit un = tc_unit(g, u);
+                if (!un.valid) continue;
+                const uint8_t* qa = g.q + un.e * g.q_gstride + (int64_t)un.rt * g.nb * 4096;
+                const uint16_t* da = g.d + un.e * g.d_gstride + (int64_t)un.rt * g.nb * kTileRows;
+                for (int ks = 0; ks < kstages; ++ks, ++it) {
+                    const int s = it % kTcStages;
+                    if (it >= kTcStages &&
+                        !mbar_wait_bounded(&empty[s], (uint32_t)((it / kTcStages - 1) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    uint8_t* st = stages + s * kTcStage;
+                    const uint32_t bbytes = (uint32_t)un.ncols * 32u, dabytes = (uint32_t)un.ncols * 4u;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)kTcStageA + kTcStageDw + kTcKS * (bbytes + dabytes));
+                    const int kb0 = ks * kTcKS;
+                    for (int kl = 0; kl < kTcKS; ++kl)
+                        for (int sl = 0; sl < 4; ++sl)
+                            bulk_g2s(st + kl * 4096 + sl * 1024, qa + ((int64_t)sl * g.nb + kb0 + kl) * 1024, 1024,
+                                     &full[s]);
+                    for (int sl = 0; sl < 4; ++sl)
+                        bulk_g2s(st + kTcStageA + sl * kTcKS * 64, da + (int64_t)sl * g.nb * 32 + kb0 * 32,
+                                 kTcKS * 64, &full[s]);
+                    for (int kl = 0; kl < kTcKS; ++kl) {
+                        const int kb = kb0 + kl;
+                        bulk_g2s(st + kTcStageA + kTcStageDw + kl * kTcN * 32,
+                                 g.bq + (int64_t)kb * g.bstride * 32 + (int64_t)un.slot0 * 32, bbytes, &full[s]);
+                        bulk_g2s(st + kTcStageA + kTcStageDw + kTcStageB + kl * kTcN * 4,
+                                 g.bd + (int64_t)kb * g.bstride + un.slot0, dabytes, &full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int it = 0, mc = 0;
+            for (int u = u0; u < u1 && !*abort_v; ++u) {
+                const TcUnit un = tc_unit(g, u);
+                if (!un.valid) continue;
+                const uint32_t idesc = umma_idesc_i8(128, un.ncols);
+                for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
+                    const int s = it % kTcStages;
+                    if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t* st = stages + s * kTcStage;
+                    for (int kl = 0; kl < kTcKS; ++kl, ++mc) {
+                        const int b = mc % kTcBufs;
+                        if (mc >= kTcBufs &&
+                            !mbar_wait_bounded(&tempty[b], (uint32_t)((mc / kTcBufs - 1) & 1), g.err, g.budget_ns)) {
+                            *abort_v = 1;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
+                        const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
+                        umma_i8(tmem + (uint32_t)(b * kTcN), adesc, bdesc, idesc, 0u);
+                        umma_commit(&tfull[b]);
+                    }
+                    umma_commit(&empty[s]);
+                }
+            }
+            // let the last MMAs finish before the accumulators are freed
+            if (mc > 0) {
+                const int last = mc - 1;
+                mbar_wait_bounded(&tfull[last % kTcBufs], (uint32_t)((last / kTcBufs) & 1), nullptr, g.budget_ns);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int ew = warp - 2;              // 0..7
+        const int sp = warp & 3;              // TMEM lane quarter this warp may read
+        const int half = ew >> 2;             // tokens 32*half .. +31
+        const int row = sp * 32 + lane;       // weight row within the tile
+        uint8_t* qs = scratch + ew * 64;
+        int it = 0, ec = 0, xc = 0;
+        for (int u = u0; u < u1 && !*abort_v; ++u) {
+            const TcUnit un = tc_unit(g, u);
+            if (!un.valid) continue;
+            float acc[32], part[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) { acc[j] = 0.0f; part[j] = 0.0f; }
+            const bool active = half * 32 < un.ncols;
+            bool ok = true;
+            for (int ks = 0; ks < kstages; ++ks, ++it) {
+                const int s = it % kTcStages;
+                const uint8_t* st = stages + s * kTcStage;
+                // the scales of this stage were written by the bulk copies
+                if (!warp_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
+                const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
+                for (int kl = 0; kl < kTcKS; ++kl, ++ec) {
+                    const int b = ec % kTcBufs;
+                    if (!warp_wait_bounded(&tfull[b], (uint32_t)((ec / kTcBufs) & 1), g.err, g.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(b * kTcN + half * 32), r);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[b]);
+                    const int kb = ks * kTcKS + kl;
+                    if (active) {
+                        const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
+                        const float* dak = das + kl * kTcN + half * 32;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            part[j] = __fmaf_rn(__int2float_rn((int)r[j]), __fmul_rn(dw, dak[j]), part[j]);
+                    }
+                    if ((kb & (kChunk - 1)) == kChunk - 1 || kb == g.nb - 1) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            acc[j] = __fadd_rn(acc[j], part[j]);
+                            part[j] = 0.0f;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (!ok) break;
+            }
+            if (!ok) {
+                *abort_v = 1;
+                break;
+            }
+            // ---- outputs of the tile ----
+            const int nv = un.nvalid;
+            const int64_t slot0 = un.slot0;
+            if (g.out_mode == TC_OUT_SWIGLU) {
+                // rows 0..63 gate, 64..127 up (interleaved arena): the up warps hand their values over
+                if (sp >= 2) {
+                    if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) xchg[(half * 32 + j) * 64 + (sp - 2) * 32 + lane] = acc[j];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xfull);
+                } else {
+                    if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = half * 32 + j;
+                        if (t >= nv) break;
+                        const float uv = xchg[t * 64 + sp * 32 + lane];
+                        const float h = __fmul_rn(silu_f32(acc[j]), uv);
+                        warp_quant_canonical(h, g.cq, g.cd, g.cstride, slot0 + t, un.rt * 2 + sp, qs);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(xempty);
+                }
+                ++xc;
+                continue;
+            }
+            for (int j = 0; j < 32; ++j) {
+                const int t = half * 32 + j;
+                if (t >= nv) break;
+                const int64_t orow = slot0 + t;
+                g.y[orow * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
+                if (g.out_mode == TC_OUT_F32_Q81)
+                    warp_quant_q8_1(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
+            }
+            if (g.out_mode == TC_OUT_F32_COMBINE) {
+                // each (token, 32-row block) is combined by the warp that writes its last expert row block
+                __threadfence();
+                __syncwarp();
+                const int L = g.rtiles * kTileRows;
+                for (int j = 0; j < 32; ++j) {
+                    const int t = half * 32 + j;
+                    if (t >= nv) break;
+                    // the pair in this slot: slot = slot_off[e] + i, pair = perm[offsets[e] + i]
+                    const int i = (int)(slot0 + t - __ldcg(g.slot_off + un.e));
+                    const int p = __ldcg(g.perm + __ldcg(g.offsets + un.e) + i);
+                    const int tok = p / g.kslots;
+                    const int blk = un.rt * 4 + sp;
+                    int last = 0;
+                    if (lane == 0) {
+                        int* cnt = g.cnt_comb + (int64_t)tok * (L / 32) + blk;
+                        last = (atomicAdd(cnt, 1) == g.kslots - 1);
+                        if (last) *cnt = 0;
+                    }
+                    last = __shfl_sync(kFull, last, 0);
+                    if (!last) continue;
+                    __threadfence();
+                    float a2 = 0.0f;
+                    for (int jj = 0; jj < g.kslots; ++jj) {
+                        const int pj = tok * g.kslots + jj;
+                        const float o = __ldcg(g.y + (int64_t)__ldcg(g.pair_slot + pj) * g.y_ld + blk * 32 + lane);
+                        a2 = __fmaf_rn(__ldcg(g.wts + pj), o, a2);
+                    }
+                    g.ylat[(int64_t)tok * L + blk * 32 + lane] = a2;
+                    warp_quant_q8_1(a2, g.ylq + ((int64_t)tok * (L / 32) + blk) * 36);
+                    __syncwarp();
+                    if (g.cq) {
+                        // the same block, packed for the U projection (slot = token)
+                        uint8_t* dst = g.cq + (int64_t)blk * g.cstride * 32 + ((int64_t)tok >> 3) * 256 + (tok & 7) * 16;
+                        const uint8_t* srcb = g.ylq + ((int64_t)tok * (L / 32) + blk) * 36;
+                        if (lane < 8)
+                            reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] =
+                                reinterpret_cast<const uint32_t*>(srcb + 4)[lane];
+                        if (lane == 0)
+                            g.cd[(int64_t)blk * g.cstride + tok] = h2f(*reinterpret_cast<const uint16_t*>(srcb));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTcBufs * kTcN);
+    pdl_trigger();
+}
+
+}  // namespace elq
