@@ -41,6 +41,9 @@ sys.path.insert(0, ROOT)
 METRIC = "latent-MoE layer tokens/s; expert-weight HBM GB/s and % of B200 peak"
 KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
+KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "proj_U"]
+KERNEL_NAMES = {"gate_up": {5: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)",
+                            9: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"}}
 
 
 def parse():
@@ -218,6 +221,15 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # the CUDA path
 
+def tensor_peak_int8():
+    """Dense int8 tensor peak: the measured bf16 GEMM rate (burst) x 2, the
+    nominal int8 : bf16 ratio of B200 (4.5 vs 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return 2.0 * float(json.load(open(p))["bf16_tflops"]), "measured bf16 x 2"
+    return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
 def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_latent_moe_b200", "csrc")
@@ -297,6 +309,8 @@ def run_elq(args):
     torch.cuda.synchronize()
     assert elq.workspace_status(ws) == 0
     G = math.lcm(args.copies, S, 2)
+    if wl.T > 64:
+        G = min(G, 16)
     graphs = {}
 
     def graph_for(n, start):
@@ -318,7 +332,7 @@ def run_elq(args):
         return start + k
 
     launches_per_step = layers[0].kernel_count(wl.T)
-    KERNELS = KERNELS_SMALL_T if launches_per_step == 5 else KERNELS_LARGE_T
+    KERNELS = {5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[launches_per_step]
     pos = run_steps(args.warmup)
     torch.cuda.synchronize()
     if world > 1:
@@ -340,11 +354,12 @@ def run_elq(args):
 
     # end to end through the C ABI with host buffers: pinned x in, y out, every step
     x_host = [x.cpu().pin_memory() for x in xs[:8]]
+    nh = len(x_host)
     y_host = torch.empty(wl.T, wl.H, dtype=torch.float32).pin_memory()
     x_dev = torch.empty_like(xs[0])
     y_dev = torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev)
     for i in range(8):
-        x_dev.copy_(x_host[i % 8], non_blocking=True)
+        x_dev.copy_(x_host[i % nh], non_blocking=True)
         elq.moe_layer(layers[i % args.copies], x_dev, y_dev, ws)
         y_host.copy_(y_dev, non_blocking=True)
         stream.synchronize()
@@ -353,7 +368,7 @@ def run_elq(args):
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for i in range(args.steps):
-        x_dev.copy_(x_host[i % 8], non_blocking=True)
+        x_dev.copy_(x_host[i % nh], non_blocking=True)
         elq.moe_layer(layers[i % args.copies], x_dev, y_dev, ws)
         y_host.copy_(y_dev, non_blocking=True)
         stream.synchronize()
@@ -411,15 +426,28 @@ def run_elq(args):
         du_w = (wl.L * nb_H + wl.H * nb_L) * blk
         rt_w = wl.E * wl.L * 4
         P = wl.T * wl.k
-        gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
         tokens = args.steps * wl.T * world
         value = tokens / (dev_ms / 1e3)
-        peak, peak_kind = peaks()
+        hbm_peak, peak_kind = peaks()
         gu_ms = kern_ms[KERNELS.index("gate_up")]
         dn_ms = kern_ms[KERNELS.index("down")]
-        achieved = gu_bytes / (gu_ms / 1e3) / 1e9
         step_s = dev_ms / 1e3 / args.steps
         layer_bytes = gu_w + dn_w + du_w + rt_w
+        if launches_per_step == 9:
+            # tensor-core path: gate/up is a contraction; int8 peak = measured bf16 x the nominal 2x ratio
+            gu_ops = 2.0 * (2 * wl.I) * P * wl.L
+            tpk, tkind = tensor_peak_int8()
+            achieved = gu_ops / (gu_ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][9], "achieved": achieved, "peak": tpk,
+                    "peak_kind": tkind, "unit": "TOPS (int8)", "frac": achieved / tpk,
+                    "traffic": traffic_for("gate_up_tc"), "algorithmic_ops_per_launch": gu_ops,
+                    "algorithmic_bytes_per_launch": gu_w}
+        else:
+            gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
+            achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": KERNEL_NAMES["gate_up"][launches_per_step], "achieved": achieved,
+                    "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "traffic": traffic_for("gate_up"), "algorithmic_bytes_per_launch": gu_bytes}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
@@ -433,15 +461,12 @@ def run_elq(args):
                              % (args.copies, layer_bytes / 1e6, (args.copies - 1) * layer_bytes / 1e6),
                        "cuda_graph": "%d steps per graph, programmatic dependent launch" % G},
             "expert_weight_gbs": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9,
-            "expert_weight_frac": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / peak,
+            "expert_weight_frac": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / hbm_peak,
             "layer_weight_gbs": layer_bytes / step_s / 1e9,
-            "layer_weight_frac": layer_bytes / step_s / 1e9 / peak,
+            "layer_weight_frac": layer_bytes / step_s / 1e9 / hbm_peak,
             "kernel_ms": dict(zip(KERNELS, kern_ms)),
             "distinct_experts_per_step": act,
-            "roofline": {"bound": "hbm", "kernel": "k_qgemv<Q8_0> gate/up (+SwiGLU, Q8_1)",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic_for("gate_up"),
-                         "algorithmic_bytes_per_launch": gu_bytes},
+            "roofline": roof,
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": xs[0].numel() * xs[0].element_size(),
                     "d2h_bytes_per_step": wl.T * wl.H * 4},

@@ -195,11 +195,12 @@ elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, flo
  * callers that may not call cudaMalloc between setting up and running their
  * decode loop.  The paper has no counterpart; this is a calling convention of
  * this library.
- *  - The scratch (error word, tile counters, chunk partial sums) is one
- *    file-scope device array of 4 MiB (4,194,304 bytes) that every GPU which
- *    loads the library holds until the process exits.  A shape whose scratch
- *    (elq_latent_proj_workspace_bytes) exceeds it returns ELQ_ERR_WORKSPACE;
- *    e.g. a 1792 x 4096 Q8_0 matrix fits up to 36 tokens.
+ *  - It always runs the GEMV kernel, whatever T.  Its scratch (error word,
+ *    tile counters, and the chunk partial sums: k/256 chunks x T x n_rows x 4
+ *    bytes) is one file-scope device array of 4 MiB (4,194,304 bytes) that
+ *    every GPU which loads the library holds until the process exits.  A
+ *    shape whose scratch exceeds it returns ELQ_ERR_WORKSPACE; e.g. a
+ *    1792 x 4096 Q8_0 matrix fits up to 36 tokens.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make
  *    that first call before any stream capture.

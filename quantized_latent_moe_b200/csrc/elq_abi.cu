@@ -199,9 +199,11 @@ struct ProjWs {
     size_t total;
 };
 
-ProjWs proj_layout(const elq_qmat* w, int T, void* base) {
+// allow_tc: whether the tensor-core path may be chosen (the allocation-free
+// entry point always runs the GEMV its scratch bound is stated for).
+ProjWs proj_layout(const elq_qmat* w, int T, void* base, bool allow_tc = true) {
     ProjWs ws;
-    ws.tc = tc_path(w->fmt, T);
+    ws.tc = allow_tc && tc_path(w->fmt, T);
     ws.plan = plan_w(w->fmt, X_Q81_TOKEN, w->n_rows, w->k, 1, T, T);
     if (ws.tc) {
         ws.plan.partial_bytes = 0;
@@ -864,10 +866,10 @@ extern "C" elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q
     if (T == 0) return ELQ_OK;
     if (!x_q8_1 || !y) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x_q8_1, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
-    if (proj_layout(w, T, nullptr).total > kStaticScratchBytes) return ELQ_ERR_WORKSPACE;
+    if (proj_layout(w, T, nullptr, false).total > kStaticScratchBytes) return ELQ_ERR_WORKSPACE;
     void* base = nullptr;
     if ((st = static_scratch_address(&base)) != ELQ_OK) return st;
-    ProjWs lay = proj_layout(w, T, base);
+    ProjWs lay = proj_layout(w, T, base, false);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the array keeps the previous call's contents: the error word and the
     // tile counters must start at zero

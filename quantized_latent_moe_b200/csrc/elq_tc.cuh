@@ -73,6 +73,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 consecutive TMEM columns of this thread's lane := v.
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Exact int32 -> fp32 for |s| < 2^22 without the (slow) conversion unit: the
+// integer s + 0x4B400000 is the bit pattern of the float 1.5 * 2^23 + s, so
+// one fp32 subtraction of 1.5 * 2^23 recovers s exactly.
+constexpr uint32_t kAccSeed = 0x4B400000u;
+constexpr float kAccSeedF = 12582912.0f;
+
 // Bounded mbarrier wait taken by lane 0 for the whole warp (the result is the
 // same in every lane, so warp-collective instructions after it stay converged).
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity, int* err, uint64_t budget_ns) {
@@ -218,15 +234,18 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
 // ---- the GEMM ------------------------------------------------------------------
 
 constexpr int kTcKS = 4;            // blocks per pipeline stage
-constexpr int kTcStages = 4;
-constexpr int kTcBufs = 4;          // TMEM accumulators of kTcN columns
+constexpr int kTcTileRowsPad = 129; // padded row count of the SwiGLU transpose (no bank conflicts)
+constexpr int kTcStages = 6;
+constexpr int kTcBufs = 8;          // TMEM accumulators of kTcN columns (all 512 columns), two groups of kTcKS
+constexpr int kTcGroups = kTcBufs / kTcKS;
 constexpr int kTcThreads = 320;
 constexpr int kTcStageA = kTcKS * 4096;
 constexpr int kTcStageB = kTcKS * kTcN * 32;
 constexpr int kTcStageDw = kTcKS * kTileRows * 2;
 constexpr int kTcStageDa = kTcKS * kTcN * 4;
 constexpr int kTcStage = kTcStageA + kTcStageB + kTcStageDw + kTcStageDa;
-constexpr int kTcXchg = kTcN * 64 * 4;                     // SwiGLU exchange of the up rows
+constexpr int kTcXld = kTcTileRowsPad;
+constexpr int kTcXchg = kTcN * kTcXld * 4;                  // SwiGLU transpose: [token][row], padded rows
 constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg;
 
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3 };
@@ -325,9 +344,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     extern __shared__ __align__(1024) uint8_t tcsm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(tcsm);            // [stages]
     uint64_t* empty = full + kTcStages;                             // [stages]
-    uint64_t* tfull = empty + kTcStages;                            // [bufs]
-    uint64_t* tempty = tfull + kTcBufs;                             // [bufs]
-    uint64_t* xfull = tempty + kTcBufs;                             // up rows handed over (4 warps)
+    uint64_t* tfull = empty + kTcStages;                            // [groups]: a stage's MMAs are done
+    uint64_t* tempty = tfull + kTcGroups;                           // [groups]: its accumulators drained
+    uint64_t* xfull = tempty + kTcGroups;                           // up rows handed over (4 warps)
     uint64_t* xempty = xfull + 1;                                   // ... and taken (4 warps)
     uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(xempty + 1);
     int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
@@ -341,12 +360,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + 8);      // the MMA commit + 8 epilogue warps
         }
-        for (int b = 0; b < kTcBufs; ++b) {
+        for (int b = 0; b < kTcGroups; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
         }
-        mbar_init(xfull, 4);
-        mbar_init(xempty, 4);
+        mbar_init(xfull, 8);
+        mbar_init(xempty, 8);
         *abort_sm = 0;
         fence_barrier_init();
     }
@@ -405,40 +424,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        // stage `it` goes to accumulator group it % 2 (kTcKS buffers, one per block)
         if (lane == 0) {
-            int it = 0, mc = 0;
+            int it = 0;
             for (int u = u0; u < u1 && !*abort_v; ++u) {
                 const TcUnit un = tc_unit(g, u);
                 if (!un.valid) continue;
                 const uint32_t idesc = umma_idesc_i8(128, un.ncols);
                 for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
-                    const int s = it % kTcStages;
+                    const int s = it % kTcStages, gr = it % kTcGroups;
+                    if (it >= kTcGroups &&
+                        !mbar_wait_bounded(&tempty[gr], (uint32_t)((it / kTcGroups - 1) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
                     if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns)) {
                         *abort_v = 1;
                         break;
                     }
                     tc_fence_after();
                     const uint8_t* st = stages + s * kTcStage;
-                    for (int kl = 0; kl < kTcKS; ++kl, ++mc) {
-                        const int b = mc % kTcBufs;
-                        if (mc >= kTcBufs &&
-                            !mbar_wait_bounded(&tempty[b], (uint32_t)((mc / kTcBufs - 1) & 1), g.err, g.budget_ns)) {
-                            *abort_v = 1;
-                            break;
-                        }
-                        tc_fence_after();
+                    for (int kl = 0; kl < kTcKS; ++kl) {
                         const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
                         const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
-                        umma_i8(tmem + (uint32_t)(b * kTcN), adesc, bdesc, idesc, 0u);
-                        umma_commit(&tfull[b]);
+                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 0u);
                     }
+                    umma_commit(&tfull[gr]);
                     umma_commit(&empty[s]);
                 }
             }
             // let the last MMAs finish before the accumulators are freed
-            if (mc > 0) {
-                const int last = mc - 1;
-                mbar_wait_bounded(&tfull[last % kTcBufs], (uint32_t)((last / kTcBufs) & 1), nullptr, g.budget_ns);
+            if (it > 0) {
+                const int last = it - 1;
+                mbar_wait_bounded(&tfull[last % kTcGroups], (uint32_t)((last / kTcGroups) & 1), nullptr, g.budget_ns);
             }
         }
     } else {
@@ -448,7 +466,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
         const int half = ew >> 2;             // tokens 32*half .. +31
         const int row = sp * 32 + lane;       // weight row within the tile
         uint8_t* qs = scratch + ew * 64;
-        int it = 0, ec = 0, xc = 0;
+        int it = 0, xc = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
             const TcUnit un = tc_unit(g, u);
             if (!un.valid) continue;
@@ -457,36 +475,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
             for (int j = 0; j < 32; ++j) { acc[j] = 0.0f; part[j] = 0.0f; }
             const bool active = half * 32 < un.ncols;
             bool ok = true;
+            const uint32_t tlane = (uint32_t)(sp * 32) << 16;
             for (int ks = 0; ks < kstages; ++ks, ++it) {
-                const int s = it % kTcStages;
+                const int s = it % kTcStages, gr = it % kTcGroups;
                 const uint8_t* st = stages + s * kTcStage;
-                // the scales of this stage were written by the bulk copies
-                if (!warp_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns)) {
+                // the stage's scales (bulk copies) and its accumulators (MMAs)
+                if (!warp_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns) ||
+                    !warp_wait_bounded(&tfull[gr], (uint32_t)((it / kTcGroups) & 1), g.err, g.budget_ns)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
                 const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
                 const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
-                for (int kl = 0; kl < kTcKS; ++kl, ++ec) {
-                    const int b = ec % kTcBufs;
-                    if (!warp_wait_bounded(&tfull[b], (uint32_t)((ec / kTcBufs) & 1), g.err, g.budget_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint32_t r[32];
-                    tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(b * kTcN + half * 32), r);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[b]);
+                uint32_t rc[32], rn[32];
+                const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + half * 32);
+                tmem_ld32(tb, rc);
+                tmem_ld_wait();
+#pragma unroll
+                for (int kl = 0; kl < kTcKS; ++kl) {
+                    if (kl + 1 < kTcKS) tmem_ld32(tb + (uint32_t)((kl + 1) * kTcN), rn);   // overlaps the rescale
                     const int kb = ks * kTcKS + kl;
                     if (active) {
                         const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
-                        const float* dak = das + kl * kTcN + half * 32;
+                        const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + half * 32);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            part[j] = __fmaf_rn(__int2float_rn((int)r[j]), __fmul_rn(dw, dak[j]), part[j]);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 dv = dak[j4];
+                            const float da4[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int j = 4 * j4 + q;
+                                const float isum = __fsub_rn(__uint_as_float(rc[j] + kAccSeed), kAccSeedF);
+                                part[j] = __fmaf_rn(isum, __fmul_rn(dw, da4[q]), part[j]);
+                            }
+                        }
                     }
                     if ((kb & (kChunk - 1)) == kChunk - 1 || kb == g.nb - 1) {
 #pragma unroll
@@ -495,10 +518,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                             part[j] = 0.0f;
                         }
                     }
+                    if (kl + 1 < kTcKS) {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) rc[j] = rn[j];
+                    }
                 }
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive(&tempty[gr]);
+                    mbar_arrive(&empty[s]);
+                }
             }
             if (!ok) {
                 *abort_v = 1;
@@ -508,82 +539,118 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
             const int nv = un.nvalid;
             const int64_t slot0 = un.slot0;
             if (g.out_mode == TC_OUT_SWIGLU) {
-                // rows 0..63 gate, 64..127 up (interleaved arena): the up warps hand their values over
-                if (sp >= 2) {
-                    if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
-                        *abort_v = 1;
-                        break;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) xchg[(half * 32 + j) * 64 + (sp - 2) * 32 + lane] = acc[j];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(xfull);
-                } else {
-                    if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
-                        *abort_v = 1;
-                        break;
-                    }
-                    for (int j = 0; j < 32; ++j) {
-                        const int t = half * 32 + j;
-                        if (t >= nv) break;
-                        const float uv = xchg[t * 64 + sp * 32 + lane];
-                        const float h = __fmul_rn(silu_f32(acc[j]), uv);
-                        warp_quant_canonical(h, g.cq, g.cd, g.cstride, slot0 + t, un.rt * 2 + sp, qs);
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(xempty);
+                // transpose the tile's accumulators through shared memory ([token][row], padded), then
+                // each of the first 128 epilogue threads builds one Q8_1 block of h = silu(gate) * up:
+                // h row 32*hb + i of token t takes gate row 32*hb + i and up row 64 + 32*hb + i
+                if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
+                    *abort_v = 1;
+                    break;
                 }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) xchg[(half * 32 + j) * kTcXld + row] = acc[j];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xfull);
+                if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
+                    *abort_v = 1;
+                    break;
+                }
+                const int task = ew * 32 + lane;            // 0 .. 255: (token, h block)
+                const int t = task >> 1, hb = task & 1;
+                if (task < 2 * kTcN && t < nv) {
+                    const float* gr = xchg + t * kTcXld + hb * 32;
+                    const float* ur = gr + 64;
+                    float h[32];
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
+                        amax = fmaxf(amax, fabsf(h[i]));
+                    }
+                    const float d = __fdiv_rn(amax, 127.0f);
+                    uint32_t wq[8];
+                    int sum = 0;
+#pragma unroll
+                    for (int w4 = 0; w4 < 8; ++w4) wq[w4] = 0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        int q = 0;
+                        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(h[i], d)), -127.0f), 127.0f);
+                        sum += q;
+                        wq[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+                    }
+                    (void)sum;
+                    const int64_t slot = slot0 + t;
+                    const int kbh = un.rt * 2 + hb;
+                    uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                    *reinterpret_cast<uint4*>(dst + 128) = make_uint4(wq[4], wq[5], wq[6], wq[7]);
+                    // the activation scale as the down projection reads it: fp32 of the stored fp16
+                    g.cd[(int64_t)kbh * g.cstride + slot] = __half2float(__float2half_rn(d));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xempty);
                 ++xc;
                 continue;
             }
+#pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int t = half * 32 + j;
-                if (t >= nv) break;
-                const int64_t orow = slot0 + t;
-                g.y[orow * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
-                if (g.out_mode == TC_OUT_F32_Q81)
-                    warp_quant_q8_1(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
+                if (t < nv) {
+                    const int64_t orow = slot0 + t;
+                    g.y[orow * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
+                    if (g.out_mode == TC_OUT_F32_Q81)
+                        warp_quant_q8_1(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
+                }
             }
             if (g.out_mode == TC_OUT_F32_COMBINE) {
-                // each (token, 32-row block) is combined by the warp that writes its last expert row block
+                // each (token, 32-row block) is combined by the warp that writes its last expert row
+                // block: lane j counts token 32*half + j, all counters of the warp at once
                 __threadfence();
                 __syncwarp();
                 const int L = g.rtiles * kTileRows;
-                for (int j = 0; j < 32; ++j) {
-                    const int t = half * 32 + j;
-                    if (t >= nv) break;
-                    // the pair in this slot: slot = slot_off[e] + i, pair = perm[offsets[e] + i]
-                    const int i = (int)(slot0 + t - __ldcg(g.slot_off + un.e));
+                const int blk = un.rt * 4 + sp;
+                const int tj = half * 32 + lane;
+                int tok = 0, last = 0;
+                if (tj < nv) {
+                    const int i = (int)(slot0 + tj - __ldcg(g.slot_off + un.e));
                     const int p = __ldcg(g.perm + __ldcg(g.offsets + un.e) + i);
-                    const int tok = p / g.kslots;
-                    const int blk = un.rt * 4 + sp;
-                    int last = 0;
-                    if (lane == 0) {
-                        int* cnt = g.cnt_comb + (int64_t)tok * (L / 32) + blk;
-                        last = (atomicAdd(cnt, 1) == g.kslots - 1);
-                        if (last) *cnt = 0;
-                    }
-                    last = __shfl_sync(kFull, last, 0);
-                    if (!last) continue;
-                    __threadfence();
+                    tok = p / g.kslots;
+                    int* cnt = g.cnt_comb + (int64_t)tok * (L / 32) + blk;
+                    last = (atomicAdd(cnt, 1) == g.kslots - 1);
+                    if (last) *cnt = 0;
+                }
+                unsigned m = __ballot_sync(kFull, last);
+                if (m) __threadfence();
+                while (m) {
+                    const int j = __ffs(m) - 1;
+                    m &= m - 1;
+                    const int tk = __shfl_sync(kFull, tok, j);
                     float a2 = 0.0f;
-                    for (int jj = 0; jj < g.kslots; ++jj) {
-                        const int pj = tok * g.kslots + jj;
-                        const float o = __ldcg(g.y + (int64_t)__ldcg(g.pair_slot + pj) * g.y_ld + blk * 32 + lane);
-                        a2 = __fmaf_rn(__ldcg(g.wts + pj), o, a2);
+                    for (int j0 = 0; j0 < g.kslots; j0 += 8) {
+                        float ov[8], wv[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (j0 + q < g.kslots) {
+                                const int pj = tk * g.kslots + j0 + q;
+                                wv[q] = __ldcg(g.wts + pj);
+                                ov[q] = __ldcg(g.y + (int64_t)__ldcg(g.pair_slot + pj) * g.y_ld + blk * 32 + lane);
+                            }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (j0 + q < g.kslots) a2 = __fmaf_rn(wv[q], ov[q], a2);
                     }
-                    g.ylat[(int64_t)tok * L + blk * 32 + lane] = a2;
-                    warp_quant_q8_1(a2, g.ylq + ((int64_t)tok * (L / 32) + blk) * 36);
+                    g.ylat[(int64_t)tk * L + blk * 32 + lane] = a2;
+                    warp_quant_q8_1(a2, g.ylq + ((int64_t)tk * (L / 32) + blk) * 36);
                     __syncwarp();
                     if (g.cq) {
                         // the same block, packed for the U projection (slot = token)
-                        uint8_t* dst = g.cq + (int64_t)blk * g.cstride * 32 + ((int64_t)tok >> 3) * 256 + (tok & 7) * 16;
-                        const uint8_t* srcb = g.ylq + ((int64_t)tok * (L / 32) + blk) * 36;
+                        uint8_t* dst = g.cq + (int64_t)blk * g.cstride * 32 + ((int64_t)tk >> 3) * 256 + (tk & 7) * 16;
+                        const uint8_t* srcb = g.ylq + ((int64_t)tk * (L / 32) + blk) * 36;
                         if (lane < 8)
                             reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] =
                                 reinterpret_cast<const uint32_t*>(srcb + 4)[lane];
                         if (lane == 0)
-                            g.cd[(int64_t)blk * g.cstride + tok] = h2f(*reinterpret_cast<const uint16_t*>(srcb));
+                            g.cd[(int64_t)blk * g.cstride + tk] = h2f(*reinterpret_cast<const uint16_t*>(srcb));
                     }
                 }
             }

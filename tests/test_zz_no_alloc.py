@@ -23,7 +23,8 @@ def E():
     return elq
 
 
-@pytest.mark.parametrize("fmt,N,K,T", [(8, 1792, 4096, 1), (8, 4096, 1792, 3), (2, 1280, 3072, 6)])
+@pytest.mark.parametrize("fmt,N,K,T", [(8, 1792, 4096, 1), (8, 4096, 1792, 3), (2, 1280, 3072, 6),
+                                       (8, 256, 512, 64)])
 def test_noalloc_matches_workspace_entry(E, fmt, N, K, T):
     W = synth.normal(11, N + K, (N, K), 0.02).cuda()
     X = synth.normal(12, T, (T, K)).cuda()
