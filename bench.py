@@ -42,8 +42,10 @@ METRIC = "latent-MoE layer tokens/s; expert-weight HBM GB/s and % of B200 peak"
 KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "proj_U"]
+KERNELS_FUSED = ["layer"]
 KERNEL_NAMES = {"gate_up": {5: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)",
-                            9: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"}}
+                            9: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
+                "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 
 
 def parse():
@@ -57,6 +59,10 @@ def parse():
     ap.add_argument("--inputs", type=int, default=64, help="distinct inputs rotated over")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded CPU-baseline sample")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="small T as the single persistent kernel instead of the separate-kernel sequence")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="no nvidia-smi sampling (for runs under a profiler; the line is then not a bench value)")
     return ap.parse_args()
 
 
@@ -283,6 +289,8 @@ def run_elq(args):
         ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, dw["router_w"],
                                 None if rb is None else rb.to(dev), device=dev)
         ly.set_dense(dw["D"], dw["U"])
+        if args.fused:
+            ly.flags = elq.LAYER_FUSED
         for e0 in range(0, wl.E, 32):
             n = min(32, wl.E - e0)
             ws_ = [synth.expert_weights(wl, e, li, device=dev) for e in range(e0, e0 + n)]
@@ -298,7 +306,7 @@ def run_elq(args):
     ys = [torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev) for _ in range(2)]
     ws = layers[0].workspace(wl.T)
     for ly in layers[1:]:
-        ly._ws[wl.T] = ws          # steps are serial on the stream: one workspace serves all
+        ly.share_workspace(wl.T, ws)   # steps are serial on the stream: one workspace serves all
 
     def step(i, y=None):
         elq.moe_layer(layers[i % args.copies], xs[i % S], ys[i % 2] if y is None else y, ws)
@@ -332,12 +340,12 @@ def run_elq(args):
         return start + k
 
     launches_per_step = layers[0].kernel_count(wl.T)
-    KERNELS = {5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[launches_per_step]
+    KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[launches_per_step]
     pos = run_steps(args.warmup)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = Clocks(local)
+    clk = None if args.no_clocks else Clocks(local)
     time.sleep(0.3)
     t_wall0 = time.time()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -401,7 +409,7 @@ def run_elq(args):
                 per[j].append(evs[i][j].elapsed_time(evs[i][j + 1]))
         done += n
     t_wall1 = time.time()
-    clocks = clk.stop(t_wall0, t_wall1)
+    clocks = {"sampled": False} if clk is None else clk.stop(t_wall0, t_wall1)
     kern_ms = [statistics.mean(v) for v in per]
 
     # routed experts per step (for the algorithmic bytes of the expert kernels)
@@ -429,11 +437,25 @@ def run_elq(args):
         tokens = args.steps * wl.T * world
         value = tokens / (dev_ms / 1e3)
         hbm_peak, peak_kind = peaks()
-        gu_ms = kern_ms[KERNELS.index("gate_up")]
-        dn_ms = kern_ms[KERNELS.index("down")]
         step_s = dev_ms / 1e3 / args.steps
         layer_bytes = gu_w + dn_w + du_w + rt_w
-        if launches_per_step == 9:
+        # activations the layer must read or write once: x, y, and the Q8_1 rows between the steps
+        x_bytes = wl.T * wl.H * (2 if wl.x_dtype == "bf16" else 4)
+        act_bytes = x_bytes + wl.T * wl.H * 4 + wl.T * nb_L * 36 * 2 + P * nb_I * 36
+        if launches_per_step == 1:
+            lay_ms = kern_ms[0]
+            gu_ms = dn_ms = None
+            lb = layer_bytes + act_bytes
+            achieved = lb / (lay_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": KERNEL_NAMES["layer"][1], "achieved": achieved, "peak": hbm_peak,
+                    "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "traffic": traffic_for("layer"), "algorithmic_bytes_per_launch": lb}
+        else:
+            gu_ms = kern_ms[KERNELS.index("gate_up")]
+            dn_ms = kern_ms[KERNELS.index("down")]
+        if launches_per_step == 1:
+            pass
+        elif launches_per_step == 9:
             # tensor-core path: gate/up is a contraction; int8 peak = measured bf16 x the nominal 2x ratio
             gu_ops = 2.0 * (2 * wl.I) * P * wl.L
             tpk, tkind = tensor_peak_int8()
@@ -459,9 +481,11 @@ def run_elq(args):
                        "l2": "inputs larger than L2: %d layer copies x ~%.0f MB touched per step rotate, "
                              "%.0f MB between reuses of a layer (L2 126 MB)"
                              % (args.copies, layer_bytes / 1e6, (args.copies - 1) * layer_bytes / 1e6),
-                       "cuda_graph": "%d steps per graph, programmatic dependent launch" % G},
-            "expert_weight_gbs": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9,
-            "expert_weight_frac": (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / hbm_peak,
+                       "cuda_graph": "%d steps per graph%s" % (
+                           G, ", one cooperative launch per step" if launches_per_step == 1
+                           else ", programmatic dependent launch")},
+            "expert_weight_gbs": None if gu_ms is None else (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9,
+            "expert_weight_frac": None if gu_ms is None else (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / hbm_peak,
             "layer_weight_gbs": layer_bytes / step_s / 1e9,
             "layer_weight_frac": layer_bytes / step_s / 1e9 / hbm_peak,
             "kernel_ms": dict(zip(KERNELS, kern_ms)),

@@ -114,11 +114,21 @@ typedef struct {
     const void* d;
 } elq_qmat;
 
+/* elq_layer.flags bits. */
+enum {
+    /* Run small token counts (T <= 8, T * k <= 64) as one cooperative
+     * persistent kernel instead of the separate-kernel sequence (same
+     * results, bit for bit).  Off by default: on B200 it measures slower
+     * than the sequence (its phase-to-phase handoffs through global memory
+     * cost more than the launches they replace). */
+    ELQ_LAYER_FUSED = 1
+};
+
 /* One latent-MoE layer.  The struct lives in host memory; every pointer in it
  * is device memory. */
 typedef struct {
     int32_t H, L, E, k, I;
-    int32_t reserved;
+    int32_t flags;              /* ELQ_LAYER_* bits, 0 by default */
     elq_qmat D;                 /* L x H  */
     elq_qmat U;                 /* H x L  */
     const float* router_w;      /* [E][L] */
@@ -227,12 +237,15 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
                          float* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels one elq_moe_layer call launches at this T (0 if the
- * layer is invalid).  Decode/verify path, in order: [activation quantiser,
- * for T > 8], D projection (quantising x itself for T <= 8; + latent Q8_1),
- * router (+ top-k, bucketing), gate/up (+ SwiGLU, Q8_1), down (+ weighted
- * combine, Q8_1), U projection.  Tensor-core path (T >= 64 and every matrix
- * Q8_0): activation quantiser, x packing, D, router, slot map, z packing,
- * gate/up, down (+ combine), U. */
+ * layer is invalid).  Fused small-T path (ELQ_LAYER_FUSED set, T <= 8,
+ * T * k <= 64, D and U in one format, gate/up and down in one format, the
+ * shared-memory plan fits): 1, a cooperative persistent kernel running the
+ * whole layer.  Decode/verify path otherwise, in order: [activation
+ * quantiser, for T > 8], D projection (quantising x itself for T <= 8; +
+ * latent Q8_1), router (+ top-k, bucketing), gate/up (+ SwiGLU, Q8_1), down
+ * (+ weighted combine, Q8_1), U projection.  Tensor-core path (T >= 64 and
+ * every matrix Q8_0): activation quantiser, x packing, D, router, slot map, z
+ * packing, gate/up, down (+ combine), U. */
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T);
 
 /* elq_moe_layer that also records CUDA events on the stream: events[0] before
@@ -265,6 +278,18 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which,
 elq_status elq_workspace_status(void* ws, void* stream);
 
 /* ---- test entry points ----------------------------------------------------- */
+
+/* Failure detection of the fused small-T kernel: runs the layer exactly as
+ * elq_moe_layer's fused path would, except that the routing is never
+ * published, so every wait for it runs out after budget_ns (1 ms .. 2 s) of
+ * device time.  The kernel then lets its own copies in flight land and
+ * returns; the workspace error word reads ELQ_ERR_TIMEOUT afterwards (see
+ * elq_workspace_status) and the workspace must be zero-filled again before
+ * its next use.  y is left undefined.  ELQ_ERR_UNSUPPORTED when the layer at
+ * this T does not take the fused path. */
+elq_status elq_test_fused_timeout(const elq_layer* layer, const void* x, int32_t x_type, int32_t T,
+                                  float* y, void* ws, size_t ws_bytes, uint64_t budget_ns,
+                                  void* stream);
 
 /* Single-block dots ("Q8 0 support", GPU EXPERT KERNELS: block-dot parity to
  * 1e-7): for i < nblocks, isum[i] and term[i] = (float)isum * (f32(d_w) *

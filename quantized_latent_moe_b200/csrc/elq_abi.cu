@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "../../include/elq.h"
+#include "elq_decode.cuh"
 #include "elq_tc.cuh"
 
 using namespace elq;
@@ -51,8 +52,26 @@ cudaError_t smem_optin(K kern, int bytes, bool* done_per_dev) {
     return e;
 }
 
-bool g_optin_w8[kMaxDevices], g_optin_w2[kMaxDevices], g_optin_router[kMaxDevices], g_optin_bucket[kMaxDevices],
-    g_optin_topk[kMaxDevices];
+bool g_optin_router[kMaxDevices], g_optin_bucket[kMaxDevices],
+    g_optin_topk[kMaxDevices], g_optin_dec[4][kMaxDevices];
+
+// Cooperative launch: every CTA of the grid is resident at once.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                        Args... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
@@ -125,6 +144,29 @@ WPlan plan_w(int fmt, int x_mode, int rows_per_group, int k, int groups_max, int
     return p;
 }
 
+// One kernel per (format, activation mode, output mode): each launch runs
+// only its own code paths, which keeps its instruction footprint small.
+template <int FMT, int XM, int OM>
+cudaError_t launch_w_t(const WArgs& g, const WPlan& p, cudaStream_t s, bool pdl) {
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_wgemv<FMT, XM, OM>, kGemvSmemMax, optin);
+    if (e != cudaSuccess) return e;
+    return launch(k_wgemv<FMT, XM, OM>, dim3(p.grid), dim3(32 * p.warps), p.smem, s, pdl, g);
+}
+
+template <int FMT>
+cudaError_t launch_w_f(const WArgs& g, const WPlan& p, cudaStream_t s, bool pdl) {
+    switch (g.x_mode * 16 + g.out_mode) {
+    case X_RAW_BF16 * 16 + OUT_F32_Q81: return launch_w_t<FMT, X_RAW_BF16, OUT_F32_Q81>(g, p, s, pdl);
+    case X_RAW_F32 * 16 + OUT_F32_Q81: return launch_w_t<FMT, X_RAW_F32, OUT_F32_Q81>(g, p, s, pdl);
+    case X_Q81_TOKEN * 16 + OUT_F32_Q81: return launch_w_t<FMT, X_Q81_TOKEN, OUT_F32_Q81>(g, p, s, pdl);
+    case X_Q81_TOKEN * 16 + OUT_F32: return launch_w_t<FMT, X_Q81_TOKEN, OUT_F32>(g, p, s, pdl);
+    case X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU: return launch_w_t<FMT, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl);
+    case X_Q81_POSITION * 16 + OUT_F32_COMBINE: return launch_w_t<FMT, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_w(WArgs g, int fmt, const WPlan& p, cudaStream_t s, bool pdl) {
     g.stages = p.stages;
     g.tokcap = p.tokcap;
@@ -136,14 +178,7 @@ cudaError_t launch_w(WArgs g, int fmt, const WPlan& p, cudaStream_t s, bool pdl)
     g.tiles = p.tiles;
     g.budget_ns = kWaitBudgetNs;
     if (p.warps == 0) return cudaErrorInvalidConfiguration;
-    if (fmt == ELQ_Q8_0) {
-        cudaError_t e = smem_optin(k_wgemv<8>, kGemvSmemMax, g_optin_w8);
-        if (e != cudaSuccess) return e;
-        return launch(k_wgemv<8>, dim3(p.grid), dim3(32 * p.warps), p.smem, s, pdl, g);
-    }
-    cudaError_t e = smem_optin(k_wgemv<2>, kGemvSmemMax, g_optin_w2);
-    if (e != cudaSuccess) return e;
-    return launch(k_wgemv<2>, dim3(p.grid), dim3(32 * p.warps), p.smem, s, pdl, g);
+    return fmt == ELQ_Q8_0 ? launch_w_f<8>(g, p, s, pdl) : launch_w_f<2>(g, p, s, pdl);
 }
 
 WArgs dense_w(const elq_qmat* w, int T, const void* x, int x_mode, int64_t x_row, int out_mode, float* y,
@@ -256,6 +291,55 @@ TcArgs dense_tc(const elq_qmat* w, int T, const uint8_t* bq, const float* bd, in
     return g;
 }
 
+// The fused small-T kernel's shared-memory plan.
+constexpr int kDecSmemMax = 227 * 1024;
+
+struct DecPlanH {
+    bool ok;
+    int stages, stage_bytes, xq_chunks, header, smem;
+};
+
+// Chunks of x the largest CTA share of the D units (numbered chunk-major)
+// spans, on a grid of `grid` CTAs.
+int dec_xq_chunks(int tiles, int nchunks, int grid) {
+    const int per_chunk = tiles * 4;
+    const int n = per_chunk * nchunks;
+    int most = 0;
+    for (int b = 0; b < grid; ++b) {
+        const int u0 = (int)((int64_t)n * b / grid), u1 = (int)((int64_t)n * (b + 1) / grid);
+        if (u1 > u0) most = std::max(most, (u1 - 1) / per_chunk - u0 / per_chunk + 1);
+    }
+    return most;
+}
+
+DecPlanH plan_dec(const elq_layer* ly, int T) {
+    DecPlanH d;
+    std::memset(&d, 0, sizeof(d));
+    if (!(ly->flags & ELQ_LAYER_FUSED)) return d;
+    if (T < 1 || T > kDecMaxT || (int64_t)T * ly->k > kDecMaxPairs) return d;
+    if (ly->D.fmt != ly->U.fmt || ly->gate_up.fmt != ly->down.fmt) return d;
+    if (ly->L / kTileRows > 64) return d;            // latent tiles the shared-memory mirror follows
+    auto codes = [](int fmt) { return kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512); };
+    const size_t acts = (size_t)T * kChunk * 36;
+    size_t need = std::max((size_t)codes(ly->D.fmt), (size_t)codes(ly->gate_up.fmt)) + kChunk * 64 + acts;
+    need = std::max(need, (size_t)ly->L * 4);       // a router row
+    need = std::max(need, (size_t)4096 + 256);      // the top-k and bucketing scratch
+    d.stage_bytes = (int)round_up(need, 128);
+    d.xq_chunks = dec_xq_chunks(ly->L / kTileRows, (ly->H / 32 + kChunk - 1) / kChunk, sm_count());
+    const size_t xq = round_up((size_t)d.xq_chunks * acts, 128);
+    d.header = dec_header_bytes(ly->L, ly->I);
+    for (int st = kDecMaxStages; st >= 2; --st) {
+        const size_t sm = (size_t)d.header + xq + (size_t)kDecWarps * st * d.stage_bytes;
+        if (sm <= (size_t)kDecSmemMax) {
+            d.stages = st;
+            d.smem = (int)sm;
+            d.ok = true;
+            break;
+        }
+    }
+    return d;
+}
+
 struct LayerWs {
     int* err;               // error word, then counters
     int* cnt_router;        // ceil(T/8) + 1
@@ -276,6 +360,12 @@ struct LayerWs {
     float* ylat;
     uint8_t* ylq;
     float* partial;
+    // fused small-T path (one persistent kernel)
+    bool fused;
+    DecPlanH dec;
+    int* sync;
+    int4* grp;
+    float* part_d;          // D chunk partials (fused path)
     // tensor-core path
     bool tc;
     int64_t tstride, sstride;   // slots of the dense (tokens) and the expert (pairs, padded) B buffers
@@ -301,8 +391,11 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.pdn = plan_w(ly->down.fmt, X_Q81_POSITION, L, I, gmax, P, T);
     w.pu = plan_w(ly->U.fmt, X_Q81_TOKEN, H, L, 1, T, T);
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
+    w.dec = plan_dec(ly, T);
+    w.fused = !w.tc && w.dec.ok;
+    const size_t n_sync = w.fused ? (size_t)dec_sync_ints(T, L, I) : 0;
     const size_t n_cnt = 64 + (rblocks + 1) + w.pd.counter_ints + w.pgu.counter_ints + w.pdn.counter_ints +
-                         w.pu.counter_ints + (size_t)T * (L / kTileRows);
+                         w.pu.counter_ints + (size_t)T * (L / kTileRows) + n_sync;
     Carve c;
     w.err = c.take<int>(base, n_cnt * sizeof(int));
     int* cur = w.err ? w.err + 64 : nullptr;
@@ -313,6 +406,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.cnt_dn = adv(w.pdn.counter_ints);
     w.cnt_u = adv(w.pu.counter_ints);
     w.cnt_comb = adv((size_t)T * (L / kTileRows));
+    w.sync = w.fused ? adv(n_sync) : nullptr;
     w.xq = w.raw ? nullptr : c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
     w.z = c.take<float>(base, (size_t)T * L * 4);
     w.zq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
@@ -331,7 +425,21 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.ylq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
     w.tstride = round16(T);
     w.sstride = round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
-    if (!w.tc) {
+    w.grp = nullptr;
+    w.part_d = nullptr;
+    if (w.fused) {
+        w.grp = c.take<int4>(base, (size_t)E * sizeof(int4));
+        // D's chunk partials; the region also serves the separate-kernel
+        // entry points that share this layout
+        const size_t part = std::max(std::max(w.pd.partial_bytes, w.pgu.partial_bytes),
+                                     std::max(w.pdn.partial_bytes, w.pu.partial_bytes));
+        w.partial = c.take<float>(base, part);
+        w.part_d = w.partial;
+        w.bxq = w.bzq = w.bhq = w.byq = nullptr;
+        w.bxd = w.bzd = w.bhd = w.byd = nullptr;
+        w.slot_off = w.tt_off = w.pair_slot = nullptr;
+        w.cnt_comb_tc = nullptr;
+    } else if (!w.tc) {
         const size_t part = std::max(std::max(w.pd.partial_bytes, w.pgu.partial_bytes),
                                      std::max(w.pdn.partial_bytes, w.pu.partial_bytes));
         w.partial = c.take<float>(base, part);
@@ -368,6 +476,7 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     if (H <= 0 || L <= 0 || E <= 0 || k <= 0 || I <= 0) return ELQ_ERR_INVALID_ARG;
     if (k > E) return ELQ_ERR_INVALID_ARG;
     if (k > 32 || E > 1024) return ELQ_ERR_UNSUPPORTED;
+    if (ly->flags & ~ELQ_LAYER_FUSED) return ELQ_ERR_INVALID_ARG;
     if (H % kTileRows || L % kTileRows || I % kTileRows) return ELQ_ERR_UNSUPPORTED;
     if ((int64_t)T * k > (int64_t)1 << 30) return ELQ_ERR_UNSUPPORTED;
     elq_status s;
@@ -410,15 +519,9 @@ cudaError_t launch_router(const float* z, const float* w, const float* bias, int
     return launch(k_router, grid, dim3(kRouterWarps * 32), router_smem(T, L, E), s, pdl, a);
 }
 
-// Kernel sequence of the grouped experts (gate/up, then down with the combine)
-// routing_early_down: the routing was produced two kernels before the down
-// projection (by the router, not by a bucketing kernel right before gate/up
-// whose completion the down kernel could not otherwise rely on).
-elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, const float* wts,
-                       float* y_lat, cudaStream_t s, bool pdl, const std::function<bool()>& mark,
-                       bool routing_early_down) {
+// Grouped gate/up over the routed pairs: SwiGLU epilogue into hq.
+WArgs gate_up_args(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, float* partial) {
     const int L = ly->L, k = ly->k, I = ly->I;
-    const int64_t P = (int64_t)T * k;
     WArgs g;
     std::memset(&g, 0, sizeof(g));
     g.q = static_cast<const uint8_t*>(ly->gate_up.q);
@@ -430,8 +533,14 @@ elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8
     g.x = zq; g.x_mode = X_Q81_PAIR_TOKEN;
     g.out_mode = OUT_SWIGLU;
     g.yq = w.hq; g.yq_ld = I / 32;
-    g.partial = w.partial; g.part_tok = P; g.counters = w.cnt_gu; g.err = w.err;
-    if (launch_w(g, ly->gate_up.fmt, w.pgu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    g.partial = partial; g.part_tok = (int64_t)T * k; g.counters = w.cnt_gu; g.err = w.err;
+    return g;
+}
+
+// Grouped down over the routed pairs: o by pair position, weighted combine
+// into y_lat and its Q8_1 rows.
+WArgs down_args(const elq_layer* ly, const LayerWs& w, int T, const float* wts, float* y_lat, float* partial) {
+    const int L = ly->L, k = ly->k, I = ly->I;
     WArgs h;
     std::memset(&h, 0, sizeof(h));
     h.q = static_cast<const uint8_t*>(ly->down.q);
@@ -444,10 +553,81 @@ elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8
     h.out_mode = OUT_F32_COMBINE;
     h.y = w.o; h.y_ld = L;
     h.wts = wts; h.pos = w.pos; h.cnt_comb = w.cnt_comb; h.ylat = y_lat; h.ylq = w.ylq;
-    h.partial = w.partial; h.part_tok = P; h.counters = w.cnt_dn; h.err = w.err;
+    h.partial = partial; h.part_tok = (int64_t)T * k; h.counters = w.cnt_dn; h.err = w.err;
+    return h;
+}
+
+// Kernel sequence of the grouped experts (gate/up, then down with the combine)
+// routing_early_down: the routing was produced two kernels before the down
+// projection (by the router, not by a bucketing kernel right before gate/up
+// whose completion the down kernel could not otherwise rely on).
+elq_status run_experts(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, const float* wts,
+                       float* y_lat, cudaStream_t s, bool pdl, const std::function<bool()>& mark,
+                       bool routing_early_down) {
+    WArgs g = gate_up_args(ly, w, T, zq, w.partial);
+    if (launch_w(g, ly->gate_up.fmt, w.pgu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    WArgs h = down_args(ly, w, T, wts, y_lat, w.partial);
     h.routing_early = routing_early_down ? 1 : 0;
     if (launch_w(h, ly->down.fmt, w.pdn, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
     return ELQ_OK;
+}
+
+// The fused small-T layer: one cooperative launch of k_decode_layer.
+template <int FDU, int FEX>
+cudaError_t launch_fused_t(const DecArgs& a, const DecPlanH& p, cudaStream_t s) {
+    const int slot = (FDU == 8 ? 2 : 0) + (FEX == 8 ? 1 : 0);
+    cudaError_t e = smem_optin(k_decode_layer<FDU, FEX>, kDecSmemMax, g_optin_dec[slot]);
+    if (e != cudaSuccess) return e;
+    return launch_coop(k_decode_layer<FDU, FEX>, dim3(sm_count()), dim3(kDecWarps * 32), (size_t)p.smem, s, a);
+}
+
+elq_status run_fused(const elq_layer* ly, const LayerWs& w, const void* x, int32_t x_type, int T, float* y,
+                     cudaStream_t s, uint64_t budget_ns = kWaitBudgetNs, bool withhold_routing = false) {
+    const int H = ly->H, L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    const DecPlanH& p = w.dec;
+    if (!p.ok) return ELQ_ERR_UNSUPPORTED;
+    DecArgs a;
+    std::memset(&a, 0, sizeof(a));
+    // D reads the Q8_1 of x each CTA makes in shared memory
+    a.dproj = dense_w(&ly->D, T, nullptr, X_Q81_TOKEN, 0, OUT_F32_Q81, w.z, w.zq, w.part_d, w.cnt_d, w.err);
+    a.dproj.tiles = w.pd.tiles;
+    a.dproj.nchunks = w.pd.nchunks;
+    a.dproj.act_off = kChunk * (ly->D.fmt == ELQ_Q8_0 ? 1024 : 512) + kChunk * 64;
+    a.dproj.act_bytes = kChunk * 36;
+    a.dproj.stage_bytes = p.stage_bytes;
+    a.dproj.stages = p.stages;
+    a.dproj.tokcap = T;
+    a.dproj.budget_ns = budget_ns;
+    a.gu_q = static_cast<const uint8_t*>(ly->gate_up.q);
+    a.gu_d = static_cast<const uint16_t*>(ly->gate_up.d);
+    a.gu_qs = (int64_t)(2 * I / kTileRows) * (L / 32) * slab_bytes(ly->gate_up.fmt);
+    a.gu_ds = (int64_t)(2 * I / kTileRows) * (L / 32) * kTileRows;
+    a.dn_q = static_cast<const uint8_t*>(ly->down.q);
+    a.dn_d = static_cast<const uint16_t*>(ly->down.d);
+    a.dn_qs = (int64_t)(L / kTileRows) * (I / 32) * slab_bytes(ly->down.fmt);
+    a.dn_ds = (int64_t)(L / kTileRows) * (I / 32) * kTileRows;
+    a.u_q = static_cast<const uint8_t*>(ly->U.q);
+    a.u_d = static_cast<const uint16_t*>(ly->U.d);
+    a.T = T; a.H = H; a.L = L; a.E = E; a.k = k; a.I = I;
+    a.rw = ly->router_w; a.rb = ly->router_bias;
+    a.z = w.z; a.logits = w.logits; a.idx = w.idx; a.wts = w.wts;
+    a.counts = w.counts; a.offsets = w.offsets; a.perm = w.perm; a.pos = w.pos; a.act = w.act; a.n_act = w.n_act;
+    a.grp = w.grp;
+    a.zq = w.zq; a.hq = w.hq; a.o = w.o; a.ylat = w.ylat; a.ylq = w.ylq; a.y = y;
+    a.sync = w.sync;
+    a.err = w.err;
+    a.budget_ns = budget_ns;
+    a.withhold_routing = withhold_routing ? 1 : 0;
+    a.x = x;
+    a.x_bf16 = (x_type == ELQ_BF16) ? 1 : 0;
+    a.stages = p.stages; a.stage_bytes = p.stage_bytes; a.xq_chunks = p.xq_chunks; a.header = p.header;
+    cudaError_t e;
+    const bool du8 = ly->D.fmt == ELQ_Q8_0, ex8 = ly->gate_up.fmt == ELQ_Q8_0;
+    if (du8 && ex8) e = launch_fused_t<8, 8>(a, p, s);
+    else if (du8) e = launch_fused_t<8, 2>(a, p, s);
+    else if (ex8) e = launch_fused_t<2, 8>(a, p, s);
+    else e = launch_fused_t<2, 2>(a, p, s);
+    return cuda_status(e);
 }
 
 elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
@@ -519,8 +699,11 @@ bool layer_tc(const elq_layer* ly, int T) {
     return tc_path(ly->D.fmt, T) && tc_path(ly->U.fmt, T) && tc_path(ly->gate_up.fmt, T) && tc_path(ly->down.fmt, T);
 }
 
+bool layer_fused(const elq_layer* ly, int T) { return !layer_tc(ly, T) && plan_dec(ly, T).ok; }
+
 int layer_kernels(const elq_layer* ly, int T) {
     if (layer_tc(ly, T)) return 9;
+    if (layer_fused(ly, T)) return 1;
     return T <= kRawMaxT ? 5 : 6;
 }
 
@@ -804,6 +987,21 @@ elq_status elq_workspace_status(void* ws, void* stream) {
     return ELQ_ERR_TIMEOUT;
 }
 
+elq_status elq_test_fused_timeout(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y,
+                                  void* ws, size_t ws_bytes, uint64_t budget_ns, void* stream) {
+    elq_status st = check_layer(layer, T);
+    if (st != ELQ_OK) return st;
+    if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
+    if (T <= 0 || !x || !y) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return ELQ_ERR_ALIGNMENT;
+    if (budget_ns < 1000000ull || budget_ns > kWaitBudgetNs) return ELQ_ERR_INVALID_ARG;
+    LayerWs w = layer_layout(layer, T, ws, x_type);
+    if (!w.fused) return ELQ_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
+    return run_fused(layer, w, x, x_type, T, y, static_cast<cudaStream_t>(stream), budget_ns, true);
+}
+
 elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q8_1, int64_t nblocks,
                                 int32_t* isum, float* term, void* stream) {
     if (!fmt_ok(wfmt)) return ELQ_ERR_UNSUPPORTED;
@@ -904,6 +1102,11 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     const bool pdl = (events == nullptr);
     cudaError_t e;
     if (!mark()) return ELQ_ERR_CUDA;
+    if (w.fused) {
+        st = run_fused(layer, w, x, x_type, T, y, s);
+        if (st != ELQ_OK) return st;
+        return mark() ? ELQ_OK : ELQ_ERR_CUDA;
+    }
     if (w.tc) {
         // prefill: a1 quantiser, packed x, D on the tensor cores (z, zq), router,
         // then the tensor-core experts and U

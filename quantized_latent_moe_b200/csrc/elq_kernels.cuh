@@ -286,8 +286,10 @@ __device__ __forceinline__ void warp_topk_softmax(const float* lg, int E, int k,
 // a5 for at most 64 pairs by one warp: the rank of pair p is the number of
 // pairs (e', p') before (e, p) in (expert, pair id) order; counts and offsets
 // are direct counts.  idx_sm: the pairs' experts in shared memory.
+// grp (optional): per active group a, (expert, first position, pairs).
 __device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* counts, int32_t* offsets,
-                                  int32_t* perm, int32_t* pos, int32_t* act, int32_t* n_act) {
+                                  int32_t* perm, int32_t* pos, int32_t* act, int32_t* n_act,
+                                  int4* grp = nullptr) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -319,6 +321,7 @@ __device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* 
         const bool on = (e < E) && c > 0;
         const unsigned b = __ballot_sync(kFull, on);
         if (on && act) act[n + __popc(b & ((1u << lane) - 1u))] = e;
+        if (on && grp) grp[n + __popc(b & ((1u << lane) - 1u))] = make_int4(e, lt, c, 0);
         n += __popc(b);
     }
     if (lane == 0) {
@@ -474,6 +477,7 @@ struct WArgs {
     int* cnt_comb;              // [T][tiles], zero on entry/exit
     float* ylat;
     uint8_t* ylq;
+    int* comb_done;             // [tiles] tokens combined per latent tile, or NULL
     float* partial;             // [nchunks][part_tok][tiles*128]
     int64_t part_tok;
     int* counters;              // [groups][tiles], zero on entry/exit
@@ -517,26 +521,28 @@ __device__ __forceinline__ WUnit wunit(const WArgs& g, int u) {
     return r;
 }
 
+template <int XM>
 __device__ __forceinline__ int64_t wunit_xrow(const WArgs& g, const WUnit& un, int i) {
     const int tp = un.tok0 + i;
-    if (g.x_mode == X_Q81_PAIR_TOKEN) return __ldcg(g.perm + tp) / g.kslots;
+    if (XM == X_Q81_PAIR_TOKEN) return __ldcg(g.perm + tp) / g.kslots;
     return tp;   // token (dense) or pair position
 }
 
 // Bytes of one token's activation slice for a chunk of kbn blocks.
-__device__ __forceinline__ uint32_t wact_bytes(const WArgs& g, int kbn) {
-    if (g.x_mode == X_RAW_F32) return (uint32_t)kbn * 128u;
-    if (g.x_mode == X_RAW_BF16) return (uint32_t)kbn * 64u;
+template <int XM>
+__device__ __forceinline__ uint32_t wact_bytes(int kbn) {
+    if (XM == X_RAW_F32) return (uint32_t)kbn * 128u;
+    if (XM == X_RAW_BF16) return (uint32_t)kbn * 64u;
     return (uint32_t)kbn * 36u;
 }
 
-template <int FMT>
+template <int FMT, int XM>
 __device__ __forceinline__ void wissue_weights(const WArgs& g, const WUnit& un, uint8_t* stage, uint64_t* bar,
                                                int ntok_pass) {
     using SL = WSlice<FMT>;
     const int lane = threadIdx.x & 31;
     const uint32_t cb = (uint32_t)(un.kbn * SL::kCodes), sb = (uint32_t)(un.kbn * 64);
-    if (lane == 0) mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)ntok_pass * wact_bytes(g, un.kbn));
+    if (lane == 0) mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)ntok_pass * wact_bytes<XM>(un.kbn));
     __syncwarp();
     if (lane == 0) {
         const uint8_t* src = g.q + un.e * g.q_gstride +
@@ -549,16 +555,17 @@ __device__ __forceinline__ void wissue_weights(const WArgs& g, const WUnit& un, 
     }
 }
 
+template <int XM>
 __device__ __forceinline__ void wissue_acts(const WArgs& g, const WUnit& un, uint8_t* act_area, uint64_t* bar,
                                             int first, int ntok_pass) {
     const int lane = threadIdx.x & 31;
-    const uint32_t ab = wact_bytes(g, un.kbn);
+    const uint32_t ab = wact_bytes<XM>(un.kbn);
     for (int i = lane; i < ntok_pass; i += 32) {
-        const int64_t row = wunit_xrow(g, un, first + i);
+        const int64_t row = wunit_xrow<XM>(g, un, first + i);
         const uint8_t* src;
-        if (g.x_mode == X_RAW_F32)
+        if (XM == X_RAW_F32)
             src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)un.c * 256) * 4;
-        else if (g.x_mode == X_RAW_BF16)
+        else if (XM == X_RAW_BF16)
             src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)un.c * 256) * 2;
         else
             src = static_cast<const uint8_t*>(g.x) + (row * g.nb + (int64_t)un.c * kChunk) * 36;
@@ -566,9 +573,91 @@ __device__ __forceinline__ void wissue_acts(const WArgs& g, const WUnit& un, uin
     }
 }
 
+// The unit's slice of weights (in its stage) into registers: w[kb][j] holds
+// the signed 8-bit codes 4j..4j+3 of block kb of this lane's row, dw[kb] its
+// scale; blocks past kbn are zero.
+template <int FMT>
+__device__ __forceinline__ void wload_regs(const uint8_t* stg, int kbn, int (&w)[kChunk][8], float (&dw)[kChunk]) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(stg + kChunk * SL::kCodes);
+#pragma unroll
+    for (int kb = 0; kb < kChunk; ++kb) {
+        if (kb < kbn) {
+            dw[kb] = h2f(sc[kb * 32 + lane]);
+            if (FMT == 8) {
+                const uint8_t* cp = stg + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
+                const uint4 a = lds128(cp), b = lds128(cp + 128);
+                w[kb][0] = (int)a.x; w[kb][1] = (int)a.y; w[kb][2] = (int)a.z; w[kb][3] = (int)a.w;
+                w[kb][4] = (int)b.x; w[kb][5] = (int)b.y; w[kb][6] = (int)b.z; w[kb][7] = (int)b.w;
+            } else {
+                const uint4 a = lds128(stg + kb * 512 + lane * 16);
+                const uint32_t v[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    // nibbles q (0..15) -> signed bytes q - 8, without borrows between bytes
+                    const uint32_t lo = v[j] & 0x0F0F0F0Fu, hi = (v[j] >> 4) & 0x0F0F0F0Fu;
+                    w[kb][j] = (int)(((lo | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
+                    w[kb][4 + j] = (int)(((hi | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
+                }
+            }
+        } else {
+            dw[kb] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[kb][j] = 0;
+        }
+    }
+}
+
+// The row dot products of one unit with np staged tokens (the unit's tokens
+// first .. first + np - 1), each chunk partial stored to the partial buffer.
+// Raw activations are first quantised to Q8_1 in the warp's scratch.
+template <int XM>
+__device__ __forceinline__ void wdots(const WArgs& g, const WUnit& un, const int (&w)[kChunk][8],
+                                      const float (&dw)[kChunk], const uint8_t* abase, int np, int first,
+                                      uint8_t* scratch) {
+    const int lane = threadIdx.x & 31;
+    int astride = g.act_bytes;
+    if (XM == X_RAW_F32 || XM == X_RAW_BF16) {
+        for (int t = 0; t < np; ++t)
+            for (int kb = 0; kb < un.kbn; ++kb) {
+                float v;
+                if (XM == X_RAW_F32)
+                    v = reinterpret_cast<const float*>(abase + t * g.act_bytes)[kb * 32 + lane];
+                else
+                    v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(abase + t * g.act_bytes)[kb * 32 + lane]);
+                warp_quant_q8_1(v, scratch + (t * kChunk + kb) * 36);
+            }
+        __syncwarp();
+        abase = scratch;
+        astride = kChunk * 36;
+    }
+    const int64_t rows_total = (int64_t)g.tiles * kTileRows;
+    for (int t = 0; t < np; ++t) {
+        const uint8_t* ab = abase + t * astride;
+        float part = 0.0f;
+#pragma unroll
+        for (int kb = 0; kb < kChunk; ++kb) {
+            if (kb < un.kbn) {
+                const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36 + 4);
+                int isum = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) isum = __dp4a(w[kb][j], (int)aw[j], isum);
+                const float da = h2f(*reinterpret_cast<const uint16_t*>(ab + kb * 36));
+                part = __fmaf_rn(__int2float_rn(isum), __fmul_rn(dw[kb], da), part);
+            }
+        }
+        const int64_t tokidx = (int64_t)un.tok0 + first + t;
+        __stcg(g.partial + ((int64_t)un.c * g.part_tok + tokidx) * rows_total + (int64_t)un.tile * kTileRows +
+                   un.s * 32 + lane,
+               part);
+    }
+}
+
 // Epilogue of a finished tile (all chunk partials present) by one warp.  The
 // chunk partials of up to 16 chunks are loaded before any is added, so the
 // L2 round trips overlap; the adds then run in chunk order.
+template <int OM>
 __device__ void wepilogue(const WArgs& g, const WUnit& un) {
     const int lane = threadIdx.x & 31;
     const int64_t rows_total = (int64_t)g.tiles * kTileRows;
@@ -592,7 +681,7 @@ __device__ void wepilogue(const WArgs& g, const WUnit& un) {
                     for (int q = 0; q < 4; ++q) v[q] = __fadd_rn(v[q], t[c][q]);
                 }
         }
-        if (g.out_mode == OUT_SWIGLU) {
+        if (OM == OUT_SWIGLU) {
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
                 const float h = __fmul_rn(silu_f32(v[hb]), v[2 + hb]);
@@ -603,11 +692,11 @@ __device__ void wepilogue(const WArgs& g, const WUnit& un) {
         float* yr = g.y + tokidx * g.y_ld + (int64_t)un.tile * kTileRows + lane;
 #pragma unroll
         for (int q = 0; q < 4; ++q) yr[32 * q] = v[q];
-        if (g.out_mode == OUT_F32_Q81) {
+        if (OM == OUT_F32_Q81) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 warp_quant_q8_1(v[q], g.yq + (tokidx * g.yq_ld + un.tile * 4 + q) * 36);
-        } else if (g.out_mode == OUT_F32_COMBINE) {
+        } else if (OM == OUT_F32_COMBINE) {
             // the pair's rows of this tile are out: count them for the token
             __threadfence();
             __syncwarp();
@@ -648,6 +737,13 @@ __device__ void wepilogue(const WArgs& g, const WUnit& un) {
                     g.ylat[(int64_t)t * L + un.tile * kTileRows + 32 * q + lane] = acc[q];
                     warp_quant_q8_1(acc[q], g.ylq + ((int64_t)t * (L / 32) + un.tile * 4 + q) * 36);
                 }
+                if (g.comb_done) {
+                    // consumers in this grid read ylq with bulk copies
+                    fence_proxy_async_global();
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicAdd(g.comb_done + un.tile, 1);
+                }
             }
         }
     }
@@ -656,6 +752,7 @@ __device__ void wepilogue(const WArgs& g, const WUnit& un) {
 // Completion of a batch of this warp's finished units (held one per lane in
 // `pending`): one fence for all their partial stores, one atomic per unit;
 // the warp then runs the epilogue of every tile it completed.
+template <int OM>
 __device__ __forceinline__ void wcomplete(const WArgs& g, int pending, int npend) {
     const int lane = threadIdx.x & 31;
     __threadfence();
@@ -673,14 +770,13 @@ __device__ __forceinline__ void wcomplete(const WArgs& g, int pending, int npend
         const int j = __ffs(m) - 1;
         m &= m - 1;
         const int u = __shfl_sync(kFull, pending, j);
-        wepilogue(g, wunit(g, u));
+        wepilogue<OM>(g, wunit(g, u));
     }
     __syncwarp();
 }
 
-template <int FMT>
+template <int FMT, int XM, int OM>
 __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
-    using SL = WSlice<FMT>;
     extern __shared__ __align__(128) uint8_t wsm[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = g.stages;
@@ -724,7 +820,7 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             if (lane == 0) myunit[st] = u;
             if (u >= 0) {
                 const WUnit un = wunit(g, u);
-                wissue_weights<FMT>(g, un, stages + st * g.stage_bytes, &mybar[st], min(un.ntok, tokcap));
+                wissue_weights<FMT, XM>(g, un, stages + st * g.stage_bytes, &mybar[st], min(un.ntok, tokcap));
             }
         }
         pdl_wait();
@@ -734,7 +830,7 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             const int u = myunit[st];
             if (u >= 0) {
                 const WUnit un = wunit(g, u);
-                wissue_acts(g, un, stages + st * g.stage_bytes + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+                wissue_acts<XM>(g, un, stages + st * g.stage_bytes + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
             }
         }
     } else {
@@ -747,14 +843,13 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             if (u >= 0) {
                 const WUnit un = wunit(g, u);
                 uint8_t* stg = stages + st * g.stage_bytes;
-                wissue_weights<FMT>(g, un, stg, &mybar[st], min(un.ntok, tokcap));
-                wissue_acts(g, un, stg + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+                wissue_weights<FMT, XM>(g, un, stg, &mybar[st], min(un.ntok, tokcap));
+                wissue_acts<XM>(g, un, stg + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
             }
         }
     }
     __syncwarp();
 
-    const int64_t rows_total = (int64_t)g.tiles * kTileRows;
     uint32_t xuse = 0;          // uses of the extra barrier (its phase parity)
     bool ok = true;
     int it = 0;
@@ -769,37 +864,10 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
         }
         const WUnit un = wunit(g, u);
         uint8_t* stg = stages + st * g.stage_bytes;
-        const uint16_t* sc = reinterpret_cast<const uint16_t*>(stg + kChunk * SL::kCodes);
 
-        // the slice's weights for this chunk, in registers (signed 8-bit codes)
         int w[kChunk][8];
         float dw[kChunk];
-#pragma unroll
-        for (int kb = 0; kb < kChunk; ++kb) {
-            if (kb < un.kbn) {
-                dw[kb] = h2f(sc[kb * 32 + lane]);
-                if (FMT == 8) {
-                    const uint8_t* cp = stg + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
-                    const uint4 a = lds128(cp), b = lds128(cp + 128);
-                    w[kb][0] = (int)a.x; w[kb][1] = (int)a.y; w[kb][2] = (int)a.z; w[kb][3] = (int)a.w;
-                    w[kb][4] = (int)b.x; w[kb][5] = (int)b.y; w[kb][6] = (int)b.z; w[kb][7] = (int)b.w;
-                } else {
-                    const uint4 a = lds128(stg + kb * 512 + lane * 16);
-                    const uint32_t v[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // nibbles q (0..15) -> signed bytes q - 8, without borrows between bytes
-                        const uint32_t lo = v[j] & 0x0F0F0F0Fu, hi = (v[j] >> 4) & 0x0F0F0F0Fu;
-                        w[kb][j] = (int)(((lo | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
-                        w[kb][4 + j] = (int)(((hi | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
-                    }
-                }
-            } else {
-                dw[kb] = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) w[kb][j] = 0;
-            }
-        }
+        wload_regs<FMT>(stg, un.kbn, w, dw);
         __syncwarp();
 
         for (int first = 0; first < un.ntok; first += tokcap) {
@@ -809,9 +877,9 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
                 __syncwarp();
                 fence_proxy_async();
                 uint64_t* xb = &mybar[S];
-                if (lane == 0) mbar_arrive_expect_tx(xb, (uint32_t)np * wact_bytes(g, un.kbn));
+                if (lane == 0) mbar_arrive_expect_tx(xb, (uint32_t)np * wact_bytes<XM>(un.kbn));
                 __syncwarp();
-                wissue_acts(g, un, stg + g.act_off, xb, first, np);
+                wissue_acts<XM>(g, un, stg + g.act_off, xb, first, np);
                 const bool got = mbar_wait_bounded(xb, xuse & 1u, g.err, g.budget_ns);
                 ++xuse;
                 if (!got) {
@@ -819,42 +887,7 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
                     break;
                 }
             }
-            const uint8_t* abase = stg + g.act_off;
-            if (g.x_mode == X_RAW_F32 || g.x_mode == X_RAW_BF16) {
-                // quantise the raw slices to Q8_1 in this warp's scratch
-                for (int t = 0; t < np; ++t)
-                    for (int kb = 0; kb < un.kbn; ++kb) {
-                        float v;
-                        if (g.x_mode == X_RAW_F32)
-                            v = reinterpret_cast<const float*>(abase + t * g.act_bytes)[kb * 32 + lane];
-                        else
-                            v = __bfloat162float(
-                                reinterpret_cast<const __nv_bfloat16*>(abase + t * g.act_bytes)[kb * 32 + lane]);
-                        warp_quant_q8_1(v, scratch + (t * kChunk + kb) * 36);
-                    }
-                __syncwarp();
-                abase = scratch;
-            }
-            const int astride = (g.x_mode == X_RAW_F32 || g.x_mode == X_RAW_BF16) ? kChunk * 36 : g.act_bytes;
-            for (int t = 0; t < np; ++t) {
-                const uint8_t* ab = abase + t * astride;
-                float part = 0.0f;
-#pragma unroll
-                for (int kb = 0; kb < kChunk; ++kb) {
-                    if (kb < un.kbn) {
-                        const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36 + 4);
-                        int isum = 0;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) isum = __dp4a(w[kb][j], (int)aw[j], isum);
-                        const float da = h2f(*reinterpret_cast<const uint16_t*>(ab + kb * 36));
-                        part = __fmaf_rn(__int2float_rn(isum), __fmul_rn(dw[kb], da), part);
-                    }
-                }
-                const int64_t tokidx = (int64_t)un.tok0 + first + t;
-                __stcg(g.partial + ((int64_t)un.c * g.part_tok + tokidx) * rows_total + (int64_t)un.tile * kTileRows +
-                           un.s * 32 + lane,
-                       part);
-            }
+            wdots<XM>(g, un, w, dw, stg + g.act_off, np, first, scratch);
         }
         if (!ok) break;
         // stage consumed: refill it with this warp's next unit
@@ -865,19 +898,19 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             if (lane == 0) myunit[st] = nu;
             if (nu >= 0) {
                 const WUnit nn = wunit(g, nu);
-                wissue_weights<FMT>(g, nn, stg, &mybar[st], min(nn.ntok, tokcap));
-                wissue_acts(g, nn, stg + g.act_off, &mybar[st], 0, min(nn.ntok, tokcap));
+                wissue_weights<FMT, XM>(g, nn, stg, &mybar[st], min(nn.ntok, tokcap));
+                wissue_acts<XM>(g, nn, stg + g.act_off, &mybar[st], 0, min(nn.ntok, tokcap));
             }
         }
         // completion of the tile (the last of its 4 * nchunks units runs the
         // epilogue), batched per warp so that one fence covers many units
         if (lane == npend) pending = u;
         if (++npend == 32) {
-            wcomplete(g, pending, npend);
+            wcomplete<OM>(g, pending, npend);
             npend = 0;
         }
     }
-    if (ok && npend) wcomplete(g, pending, npend);
+    if (ok && npend) wcomplete<OM>(g, pending, npend);
     if (!ok) {
         // drain: wait (bounded) for this warp's copies still in flight
         for (int k = 0; k < S; ++k) {

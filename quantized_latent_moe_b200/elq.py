@@ -16,6 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libelq.so")
 
 F32, Q4_0, Q8_0, Q8_1, BF16 = 0, 2, 8, 9, 30
+LAYER_FUSED = 1            # elq_layer.flags: small T as one persistent kernel
 FMT = {"q8_0": Q8_0, "q4_0": Q4_0}
 SLAB = {Q8_0: 4096, Q4_0: 2048}
 
@@ -33,7 +34,7 @@ class QMat(ctypes.Structure):
 
 class LayerC(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("L", ctypes.c_int32), ("E", ctypes.c_int32),
-                ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("D", QMat), ("U", QMat), ("router_w", ctypes.c_void_p),
                 ("router_bias", ctypes.c_void_p), ("gate_up", QMat), ("down", QMat)]
 
@@ -63,6 +64,7 @@ SIGNATURES = {
     "elq_moe_layer_profiled": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V, I32, V]),
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
     "elq_test_expf": (I32, [V, V, I64, V]),
+    "elq_test_fused_timeout": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, ctypes.c_uint64, V]),
 }
 
 
@@ -146,6 +148,7 @@ class Layer:
         self.D, self.U, self.gate_up, self.down = D, U, gate_up, down
         self.router_w = router_w.contiguous()
         self.router_bias = None if router_bias is None else router_bias.contiguous()
+        self.flags = 0          # LAYER_FUSED: small T as one persistent kernel
         self._ws = {}
 
     @classmethod
@@ -180,7 +183,7 @@ class Layer:
                                         _stream(stream)), "elq_quantize_weights")
 
     def struct(self) -> LayerC:
-        return LayerC(self.H, self.L, self.E, self.k, self.I, 0, self.D.struct(), self.U.struct(),
+        return LayerC(self.H, self.L, self.E, self.k, self.I, self.flags, self.D.struct(), self.U.struct(),
                       self.router_w.data_ptr(),
                       None if self.router_bias is None else self.router_bias.data_ptr(),
                       self.gate_up.struct(), self.down.struct())
@@ -194,7 +197,9 @@ class Layer:
         return int(_lib().elq_workspace_bytes(ctypes.byref(s), T))
 
     def workspace(self, T: int) -> torch.Tensor:
-        ws = self._ws.get(T)
+        """A zero-filled device workspace for T tokens (cached per T and flags)."""
+        key = (T, self.flags)
+        ws = self._ws.get(key)
         if ws is None:
             n = self.workspace_bytes(T)
             if n == 0:
@@ -202,8 +207,13 @@ class Layer:
             ws = torch.zeros(n + 256, dtype=torch.uint8, device=self.router_w.device)
             off = (-ws.data_ptr()) % 256
             ws = ws[off:off + n]
-            self._ws[T] = ws
+            self._ws[key] = ws
         return ws
+
+    def share_workspace(self, T: int, ws: torch.Tensor):
+        """Use `ws` (another layer's workspace of the same shape) for T tokens:
+        calls that run one after another on one stream may share it."""
+        self._ws[(T, self.flags)] = ws
 
 
 # --------------------------------------------------------------------------
@@ -340,6 +350,19 @@ def test_block_isums(wfmt: int, w_aos: torch.Tensor, xq: torch.Tensor, n: int, s
     _ck(_lib().elq_test_block_isums(wfmt, _ptr(w_aos), _ptr(xq), n, _ptr(isum), _ptr(term),
                                     _stream(stream)), "elq_test_block_isums")
     return isum, term
+
+
+def test_fused_timeout(layer: Layer, x: torch.Tensor, ws: torch.Tensor, budget_ns: int,
+                       stream=None) -> int:
+    """The fused layer kernel with its routing withheld: returns the call's
+    status (the kernel's own outcome is in the workspace error word)."""
+    x = x.contiguous()
+    T = x.shape[0]
+    xt = {torch.float32: F32, torch.bfloat16: BF16}[x.dtype]
+    y = torch.empty(T, layer.H, dtype=torch.float32, device=x.device)
+    s = layer.struct()
+    return int(_lib().elq_test_fused_timeout(ctypes.byref(s), _ptr(x), xt, T, _ptr(y), _ptr(ws), ws.numel(),
+                                             budget_ns, _stream(stream)))
 
 
 def test_expf(x: torch.Tensor, stream=None) -> torch.Tensor:

@@ -71,9 +71,20 @@ def test_layer_validation(L):
     y = ctypes.c_void_p(1 << 28)
     good = _layer()
     assert L.elq_workspace_bytes(ctypes.byref(good), 4) > 0
+    # the separate-kernel sequence by default; one fused kernel on request for
+    # T <= 8 and T*k <= 64
     assert L.elq_layer_kernel_count(ctypes.byref(good), 4) == 5
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(flags=1)), 4) == 1
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(k=8, flags=1)), 8) == 1  # 64 pairs
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(k=8, flags=1)), 9) == 6  # T > 8
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(E=128, k=16, flags=1)), 8) == 5  # 128 pairs
     assert L.elq_layer_kernel_count(ctypes.byref(good), 9) == 6
     assert L.elq_layer_kernel_count(None, 4) == 0
+    # the fused path keeps its phase flags and counters in the workspace
+    assert L.elq_workspace_bytes(ctypes.byref(_layer(flags=1)), 4) > L.elq_workspace_bytes(ctypes.byref(good), 4)
+    # unknown flag bits are refused
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(flags=2)), 4) == 0
+    assert L.elq_moe_layer(ctypes.byref(_layer(flags=6)), x, 0, 4, y, ws_small, 1 << 30, None) == -1
     # workspace too small -> refused before any launch
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, ws_small, 16, None) == -4
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, 4, y, None, 1 << 30, None) == -4

@@ -182,10 +182,16 @@ def _check_intermediates(E, ly, T, tr):
     assert np.array_equal(v("ylq").reshape(T, -1), tr["ylq"])
 
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("name", ["tiny", "decode", "verify"])
-def test_layer_exact(E, orc, name):
+def test_layer_exact(E, orc, name, fused):
+    """Every intermediate and the output, on the fused single-kernel path and
+    on the separate-kernel sequence."""
     wl = synth.WORKLOADS[name]
     ly = gpu_layer(wl)
+    if fused:
+        ly.flags = E.LAYER_FUSED
+    assert ly.kernel_count(wl.T) == (1 if fused else 5)
     x = synth.make_x(wl)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
     assert E.workspace_status(ly.workspace(wl.T)) == 0
