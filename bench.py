@@ -51,8 +51,8 @@ KERNEL_NAMES = {"gate_up": {5: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)", 6: "k_wg
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4096)
-    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 4096; the stack: 64)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default 64; the stack: 4)")
     ap.add_argument("--impl", default="elq", choices=["elq", "reference"])
     ap.add_argument("--workload", default="decode")
     ap.add_argument("--copies", type=int, default=8, help="distinct layer copies rotated over")
@@ -215,7 +215,7 @@ def run_reference(args):
     threads = host_threads()
     oracle_run(ly, xs, args.warmup, threads)
     dt = oracle_run(ly, xs, args.steps, threads)
-    value = args.steps * tok / dt
+    value = args.steps * tok / dt / wl.layers      # a stack step runs every layer
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
@@ -224,8 +224,10 @@ def run_reference(args):
                                         "parallelism": "host threads"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": "each step: one layer call of %d token(s) on the scalar C oracle "
-                                   "(2 distinct inputs alternating), steps spread over %d host threads"
-                                   % (tok, threads)},
+                                   "(2 distinct inputs alternating), steps spread over %d host threads%s"
+                                   % (tok, threads, "" if wl.layers == 1 else
+                                      "; tokens/s of the %d-layer stack = one layer's rate / %d"
+                                      % (wl.layers, wl.layers))},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -513,14 +515,208 @@ def run_elq(args):
         dist.destroy_process_group()
 
 
+def run_stack(args):
+    """The resident stack: each step runs one batch of T new tokens through all
+    of the workload's layers on one fp32 residual stream (elq_moe_stack)."""
+    import torch
+    import torch.distributed as dist
+
+    from quantized_latent_moe_b200 import build, elq, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    elq.lib()
+    wl = synth.WORKLOADS[args.workload]
+    fmt = elq.FMT[wl.fmt]
+    stream = torch.cuda.current_stream()
+    layers = []
+    for l in range(wl.layers):
+        li = l + 1000 * rank
+        dw = synth.dense_weights(wl, li, device=dev)
+        rb = dw["router_bias"]
+        ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, dw["router_w"],
+                                None if rb is None else rb.to(dev), device=dev)
+        ly.set_dense(dw["D"], dw["U"])
+        for e0 in range(0, wl.E, 32):
+            ws_ = [synth.expert_weights(wl, e, li, device=dev) for e in range(e0, min(wl.E, e0 + 32))]
+            ly.set_experts(e0, torch.stack([w[0] for w in ws_]), torch.stack([w[1] for w in ws_]),
+                           torch.stack([w[2] for w in ws_]))
+            del ws_
+        layers.append(ly)
+        del dw
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    S = min(args.inputs, 16)
+    xs = [synth.make_x(wl, step=s + 1000 * rank, device=dev) for s in range(S)]
+    h = torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev)
+    ws = layers[0].stack_workspace(wl.T)
+    lws = ws[:layers[0].workspace_bytes(wl.T)]        # its first part is the layer workspace
+    for ly in layers:
+        ly.share_workspace(wl.T, lws)
+
+    def step(i):
+        elq.moe_stack(layers, xs[i % S], h, ws)
+
+    for i in range(2):
+        step(i)
+    torch.cuda.synchronize()
+    assert elq.workspace_status(ws) == 0
+    G = 4
+    graphs = {}
+
+    def run_steps(k, start=0):
+        done = 0
+        while done < k:
+            n = min(G, k - done)
+            key = (n, (start + done) % S)
+            if key not in graphs:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for i in range(start + done, start + done + n):
+                        step(i)
+                graphs[key] = g
+            graphs[key].replay()
+            done += n
+        return start + k
+
+    pos = run_steps(args.warmup)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = None if args.no_clocks else Clocks(local)
+    time.sleep(0.3)
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    pos = run_steps(args.steps, pos)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    dev_ms = e0.elapsed_time(e1)
+    # end to end: pinned tokens in, the residual stream out, every step
+    x_host = [x.cpu().pin_memory() for x in xs[:4]]
+    h_host = torch.empty(wl.T, wl.H, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        x_dev.copy_(x_host[i % len(x_host)], non_blocking=True)
+        elq.moe_stack(layers, x_dev, h, ws)
+        h_host.copy_(h, non_blocking=True)
+        stream.synchronize()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    # per-kernel times of one layer at this T (first layer, eager, behind a GPU sleep)
+    nk = layers[0].kernel_count(wl.T)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
+    for ev in evs:
+        ev.record(stream)
+    torch.cuda.synchronize()
+    per = [[] for _ in range(nk)]
+    for r in range(16):
+        torch.cuda._sleep(2_000_000)
+        elq.moe_layer_profiled(layers[r % len(layers)], xs[r % S], h, evs, lws)
+        torch.cuda.synchronize()
+        for j in range(nk):
+            per[j].append(evs[j].elapsed_time(evs[j + 1]))
+    t_wall1 = time.time()
+    clocks = {"sampled": False} if clk is None else clk.stop(t_wall0, t_wall1)
+    kern_ms = [statistics.mean(v) for v in per]
+    # routed experts of every layer on one step (layer by layer on the same residual stream)
+    n_act = []
+    h.copy_(xs[0].float())
+    for ly in layers:
+        hl = h.clone()
+        elq.moe_stack([ly], hl, h, ws)
+        torch.cuda.synchronize()
+        n_act.append(int(elq.workspace_view(ly, wl.T, "n_act", lws).item()))
+    t = torch.tensor([dev_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev_ms, e2e_ms = t.tolist()
+    if rank == 0:
+        blk = 34 if wl.fmt == "q8_0" else 18
+        nb_L, nb_H, nb_I = wl.L // 32, wl.H // 32, wl.I // 32
+        per_layer_dense = (wl.L * nb_H + wl.H * nb_L) * blk + wl.E * wl.L * 4
+        expert_bytes = [a * (2 * wl.I * nb_L + wl.L * nb_I) * blk for a in n_act]
+        step_bytes = sum(expert_bytes) + wl.layers * per_layer_dense
+        tokens = args.steps * wl.T * world
+        value = tokens / (dev_ms / 1e3)
+        hbm_peak, peak_kind = peaks()
+        step_s = dev_ms / 1e3 / args.steps
+        names = KERNELS_LARGE_T if nk == 6 else KERNELS_SMALL_T
+        gu_ms = kern_ms[names.index("gate_up")]
+        P = wl.T * wl.k
+        gu_bytes = n_act[0] * 2 * wl.I * nb_L * blk + wl.T * nb_L * 36 + P * nb_I * 36
+        achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic (seeded counter-hash normals; random-init weights of the layer's shape)",
+            "config": {"workload": "%s: %d layers on one fp32 residual stream, %s"
+                                   % (wl.name, wl.layers, workload_desc(wl)),
+                       "global_batch": wl.T * world, "parallelism": "replicas" if world > 1 else "1 GPU",
+                       "inputs": S, "l2": "inputs larger than L2: %.1f GB of weights touched per step"
+                                         % (step_bytes / 1e9),
+                       "cuda_graph": "%d steps per graph" % G},
+            "layer_weight_gbs": step_bytes / step_s / 1e9,
+            "layer_weight_frac": step_bytes / step_s / 1e9 / hbm_peak,
+            "kernel_ms": dict(zip(names, kern_ms)),
+            "distinct_experts_per_layer": statistics.mean(n_act),
+            "roofline": {"bound": "hbm", "kernel": "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1), T=%d" % wl.T,
+                         "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None, "algorithmic_bytes_per_launch": gu_bytes},
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": xs[0].numel() * xs[0].element_size(),
+                    "d2h_bytes_per_step": wl.T * wl.H * 4},
+            "gpu_launches": (1 + wl.layers * (1 + nk)) * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu:
+            cb = cpu_baseline(wl, args.cpu_seconds, "cuda")
+            cb["value"] /= wl.layers
+            cb["sample"] += "; tokens/s of the whole stack = one layer's rate / %d layers" % wl.layers
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
+    from quantized_latent_moe_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = wl.steps if wl.layers > 1 else 4096
+    if args.warmup is None:
+        args.warmup = 4 if wl.layers > 1 else 64
     if args.impl == "reference":
         if int(os.environ.get("WORLD_SIZE", "1")) > 1 and int(os.environ.get("RANK", "0")) != 0:
             return
         run_reference(args)
         return
-    run_elq(args)
+    if wl.layers > 1:
+        run_stack(args)
+    else:
+        run_elq(args)
 
 
 if __name__ == "__main__":

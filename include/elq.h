@@ -236,6 +236,26 @@ size_t elq_workspace_bytes(const elq_layer* layer, int32_t T);
 elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T,
                          float* y, void* ws, size_t ws_bytes, void* stream);
 
+/* A stack of layers on one residual stream.  The pages give no rule for it;
+ * the reading taken: h = fp32(x), then for l = 0 .. n_layers-1,
+ * h = h + layer_l(rms(h)), where rms(h) is each row divided by
+ * sqrt(mean(h^2) + 1e-6) (no learned scale; the sum of squares by 32
+ * lane-strided fused multiply-adds and an xor butterfly of adds, every step
+ * IEEE round-to-nearest fp32).  Without the normalisation the stack diverges:
+ * a layer's output grows with the square of its input.
+ * layers: host array of n_layers layers of identical shapes and formats (their
+ * pointers device memory); x: device [T][H] fp32 or bf16 (the new tokens);
+ * h: device [T][H] fp32 output.  ws: one workspace of
+ * elq_stack_workspace_bytes(&layers[0], T) bytes, shared by the layers in
+ * turn (the layer workspace, then the normalised input).  The separate-kernel
+ * path at every T below the tensor-core threshold (T < 64; larger T returns
+ * ELQ_ERR_UNSUPPORTED; ELQ_LAYER_FUSED is ignored here).  Launches
+ * 1 + n_layers * (1 + the layer's separate-kernel count) kernels.
+ * Validation as elq_moe_layer, before anything is enqueued. */
+elq_status elq_moe_stack(const elq_layer* layers, int32_t n_layers, const void* x, int32_t x_type,
+                         int32_t T, float* h, void* ws, size_t ws_bytes, void* stream);
+size_t elq_stack_workspace_bytes(const elq_layer* layer, int32_t T);
+
 /* Number of kernels one elq_moe_layer call launches at this T (0 if the
  * layer is invalid).  Fused small-T path (ELQ_LAYER_FUSED set, T <= 8,
  * T * k <= 64, D and U in one format, gate/up and down in one format, the

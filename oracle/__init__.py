@@ -84,6 +84,7 @@ def _declare(L):
                                ctypes.c_int, P]),
         "orc_router_topk": (None, [P, P, P] + [ctypes.c_int] * 4 + [P, P, P]),
         "orc_bucket": (None, [P] + [ctypes.c_int] * 3 + [P, P, P, P]),
+        "orc_rmsnorm": (None, [P, ctypes.c_int, ctypes.c_int, P]),
         "orc_moe_layer": (ctypes.c_int, [ctypes.POINTER(OrcLayer), P, ctypes.c_int,
                                          P, ctypes.POINTER(OrcTrace)]),
         "orc_route": (ctypes.c_int, [ctypes.POINTER(OrcLayer), P, ctypes.c_int, P, P]),
@@ -173,6 +174,15 @@ def router_topk(z, Wr, bias, k: int):
     logits = np.empty((T, E), np.float32)
     lib().orc_router_topk(_p(z), _p(Wr), _p(b), T, L, E, k, _p(idx), _p(w), _p(logits))
     return idx, w, logits
+
+
+def rmsnorm(h):
+    """Rows of h divided by sqrt(mean(h^2) + 1e-6) (the stack's layer input)."""
+    h = _f32(h)
+    T, H = h.shape
+    out = np.empty((T, H), np.float32)
+    lib().orc_rmsnorm(_p(h), T, H, _p(out))
+    return out
 
 
 def bucket(idx: np.ndarray, E: int):

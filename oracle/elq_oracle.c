@@ -341,6 +341,10 @@ void orc_router_topk(const float* z, const float* Wr, const float* bias,
             lg[e] = v;
             if (logits) logits[(int64_t)t * E + e] = v;
         }
+        /* R18: a NaN logit ranks as -infinity (in the selection and in the
+         * softmax), so the k chosen ids are always valid and distinct */
+        for (int e = 0; e < E; ++e)
+            if (isnan(lg[e])) lg[e] = -INFINITY;
         memset(taken, 0, (size_t)E);
         for (int j = 0; j < k; ++j) {          /* k largest, lower id on ties */
             int best = -1;
@@ -526,5 +530,30 @@ void orc_arena_pack(int fmt, const uint8_t* aos, int n_rows, int k,
                     q_out[base + r * 16 + j] = blk[2 + j];
             }
         }
+    }
+}
+
+/* RMS normalisation of the rows of h [T][H] (the stack's reading): the sum of
+ * squares as 32 partials (partial j takes i = j, j+32, ... with fmaf), an xor
+ * butterfly (16, 8, 4, 2, 1) of adds, ms = sum / H, r = sqrtf(ms + 1e-6f),
+ * out_i = h_i / r. */
+void orc_rmsnorm(const float* h, int T, int H, float* out)
+{
+    for (int t = 0; t < T; ++t) {
+        const float* hr = h + (int64_t)t * H;
+        float part[32];
+        for (int j = 0; j < 32; ++j) {
+            float p = 0.0f;
+            for (int i = j; i < H; i += 32) p = fmaf(hr[i], hr[i], p);
+            part[j] = p;
+        }
+        for (int off = 16; off >= 1; off /= 2) {
+            float nxt[32];
+            for (int j = 0; j < 32; ++j) nxt[j] = part[j] + part[j ^ off];
+            memcpy(part, nxt, sizeof(part));
+        }
+        const float ms = part[0] / (float)H;
+        const float r = sqrtf(ms + 1e-6f);
+        for (int i = 0; i < H; ++i) out[(int64_t)t * H + i] = hr[i] / r;
     }
 }

@@ -54,6 +54,8 @@
  *   R13 SwiGLU: h = (g / (1 + exp(-g))) * u.
  *   R14 combine: y_lat = sum_j fmaf(w_j, o_j, acc) over the k slots in rank
  *      order from 0.
+ *   R18 a NaN router logit ranks as -infinity, in the selection and in the
+ *       softmax (ties still by lower id), so the chosen ids are always valid.
  */
 #ifndef ELQ_ORACLE_H
 #define ELQ_ORACLE_H
@@ -92,7 +94,8 @@ float   orc_block_term(int wfmt, const uint8_t* wblk, const uint8_t* ablk);
 void orc_qmatmul(int wfmt, const uint8_t* W, int N, int K,
                  const uint8_t* Xq, int T, float* Y);
 
-/* router, R9-R11: idx [T][k], w [T][k], logits [T][E] (may be NULL) */
+/* router, R9-R11 and R18 (a NaN logit ranks as -infinity): idx [T][k],
+ * w [T][k], logits [T][E] (may be NULL; raw values) */
 void orc_router_topk(const float* z, const float* Wr, const float* bias,
                      int T, int L, int E, int k,
                      int32_t* idx, float* w, float* logits);
@@ -145,6 +148,11 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y,
 /* Only the routing half of the layer (x -> xq -> z -> idx, w), so that a caller
  * can learn which experts a token set needs before supplying them. */
 int orc_route(const orc_layer* ly, const float* x, int T, int32_t* idx, float* w);
+
+/* The stack's layer input: each row of h divided by sqrt(mean(h^2) + 1e-6),
+ * the sum of squares in the R9 order (32 strided fmaf partials, xor
+ * butterfly of adds). */
+void orc_rmsnorm(const float* h, int T, int H, float* out);
 
 /* The device arena layout, stated plainly (the definition is written out in
  * elq_oracle.c): tiles of 128 rows, four 32-row slices per tile, per slice

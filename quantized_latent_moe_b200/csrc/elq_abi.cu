@@ -161,6 +161,7 @@ cudaError_t launch_w_f(const WArgs& g, const WPlan& p, cudaStream_t s, bool pdl)
     case X_RAW_F32 * 16 + OUT_F32_Q81: return launch_w_t<FMT, X_RAW_F32, OUT_F32_Q81>(g, p, s, pdl);
     case X_Q81_TOKEN * 16 + OUT_F32_Q81: return launch_w_t<FMT, X_Q81_TOKEN, OUT_F32_Q81>(g, p, s, pdl);
     case X_Q81_TOKEN * 16 + OUT_F32: return launch_w_t<FMT, X_Q81_TOKEN, OUT_F32>(g, p, s, pdl);
+    case X_Q81_TOKEN * 16 + OUT_F32_ADD: return launch_w_t<FMT, X_Q81_TOKEN, OUT_F32_ADD>(g, p, s, pdl);
     case X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU: return launch_w_t<FMT, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl);
     case X_Q81_POSITION * 16 + OUT_F32_COMBINE: return launch_w_t<FMT, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
     default: return cudaErrorInvalidValue;
@@ -631,7 +632,7 @@ elq_status run_fused(const elq_layer* ly, const LayerWs& w, const void* x, int32
 }
 
 elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
-                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events);
+                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events, bool residual = false);
 
 // Tensor-core experts: slots from the routing, gathered z codes, gate/up (+SwiGLU
 // into the packed hq buffer), down (+combine into y_lat, Q8_1 rows and the
@@ -928,6 +929,51 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
     return run_layer(layer, x, x_type, T, y, ws, ws_bytes, stream, nullptr, 0);
 }
 
+elq_status elq_moe_stack(const elq_layer* layers, int32_t n_layers, const void* x, int32_t x_type, int32_t T,
+                         float* h, void* ws, size_t ws_bytes, void* stream) {
+    if (!layers || n_layers <= 0) return ELQ_ERR_INVALID_ARG;
+    if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
+    for (int l = 0; l < n_layers; ++l) {
+        const elq_status st = check_layer(&layers[l], T);
+        if (st != ELQ_OK) return st;
+        const elq_layer& a = layers[l];
+        const elq_layer& b = layers[0];
+        if (a.H != b.H || a.L != b.L || a.E != b.E || a.k != b.k || a.I != b.I || a.D.fmt != b.D.fmt ||
+            a.U.fmt != b.U.fmt || a.gate_up.fmt != b.gate_up.fmt || a.down.fmt != b.down.fmt ||
+            (a.router_bias == nullptr) != (b.router_bias == nullptr))
+            return ELQ_ERR_INVALID_ARG;
+    }
+    if (T == 0) return ELQ_OK;
+    if (layer_tc(&layers[0], T)) return ELQ_ERR_UNSUPPORTED;
+    if (!x || !h) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(h, 16)) return ELQ_ERR_ALIGNMENT;
+    if (!router_shape_ok(T, layers[0].L, layers[0].E)) return ELQ_ERR_UNSUPPORTED;
+    const size_t lay = layer_layout(&layers[0], T, nullptr, ELQ_F32).total;
+    const size_t need = lay + round_up((size_t)T * layers[0].H * 4, 256);
+    if (!ws || ws_bytes < need) return ELQ_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
+    float* xn = reinterpret_cast<float*>(static_cast<char*>(ws) + lay);   // the normalised layer input
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int H = layers[0].H;
+    const int64_t n = (int64_t)T * H;
+    const dim3 grid((unsigned)((n + 255) / 256));
+    cudaError_t e = (x_type == ELQ_BF16) ? launch(k_to_f32<true>, grid, dim3(256), 0, s, false, x, n, h)
+                                         : launch(k_to_f32<false>, grid, dim3(256), 0, s, false, x, n, h);
+    if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    for (int l = 0; l < n_layers; ++l) {
+        e = launch(k_rmsnorm, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, s, false, (const float*)h, T, H, xn);
+        if (e != cudaSuccess) return ELQ_ERR_CUDA;
+        const elq_status st = run_layer(&layers[l], xn, ELQ_F32, T, h, ws, lay, stream, nullptr, 0, true);
+        if (st != ELQ_OK) return st;
+    }
+    return ELQ_OK;
+}
+
+size_t elq_stack_workspace_bytes(const elq_layer* layer, int32_t T) {
+    if (check_layer(layer, T) != ELQ_OK || T <= 0) return 0;
+    return layer_layout(layer, T, nullptr, ELQ_F32).total + round_up((size_t)T * layer->H * 4, 256);
+}
+
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T) {
     if (check_layer(layer, T) != ELQ_OK || T <= 0) return 0;
     return layer_kernels(layer, T);
@@ -1079,8 +1125,9 @@ extern "C" elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q
 
 namespace {
 
+// residual: y = y + layer(x) (the stack; the separate-kernel GEMV path only)
 elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int32_t T, float* y, void* ws,
-                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events) {
+                     size_t ws_bytes, void* stream, void* const* events, int32_t n_events, bool residual) {
     elq_status st = check_layer(layer, T);
     if (st != ELQ_OK) return st;
     if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
@@ -1102,7 +1149,8 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     const bool pdl = (events == nullptr);
     cudaError_t e;
     if (!mark()) return ELQ_ERR_CUDA;
-    if (w.fused) {
+    if (residual && w.tc) return ELQ_ERR_UNSUPPORTED;
+    if (w.fused && !residual) {
         st = run_fused(layer, w, x, x_type, T, y, s);
         if (st != ELQ_OK) return st;
         return mark() ? ELQ_OK : ELQ_ERR_CUDA;
@@ -1164,7 +1212,8 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     st = run_experts(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark, pdl);
     if (st != ELQ_OK) return st;
     // a10
-    WArgs gu = dense_w(&layer->U, T, w.ylq, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, w.partial, w.cnt_u, w.err);
+    WArgs gu = dense_w(&layer->U, T, w.ylq, X_Q81_TOKEN, 0, residual ? OUT_F32_ADD : OUT_F32, y, nullptr, w.partial,
+                       w.cnt_u, w.err);
     if (launch_w(gu, layer->U.fmt, w.pu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
     return ELQ_OK;
 }

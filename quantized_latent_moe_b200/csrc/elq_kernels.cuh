@@ -260,7 +260,8 @@ __device__ __forceinline__ void warp_topk_softmax(const float* lg, int E, int k,
         int be = 0x7fffffff;
         for (int i = 0, x = lane; x < E; ++i, x += 32) {
             if (taken & (1u << i)) continue;
-            const float v = lg[x];
+            const float v0 = lg[x];
+            const float v = (v0 != v0) ? -INFINITY : v0;   // R18: a NaN logit ranks as -inf
             if (v > bv || (v == bv && x < be)) { bv = v; be = x; }
         }
 #pragma unroll
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(128) k_topk(const float* __restrict__ logits, 
 // ============================================================================
 constexpr int kTokMax = 32;        // tokens a unit stages at once
 
-enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2, OUT_F32_COMBINE = 3 };
+enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2, OUT_F32_COMBINE = 3, OUT_F32_ADD = 4 };
 enum { X_Q81_TOKEN = 0, X_Q81_PAIR_TOKEN = 1, X_Q81_POSITION = 2, X_RAW_F32 = 3, X_RAW_BF16 = 4 };
 
 struct WArgs {
@@ -690,6 +691,12 @@ __device__ void wepilogue(const WArgs& g, const WUnit& un) {
             continue;
         }
         float* yr = g.y + tokidx * g.y_ld + (int64_t)un.tile * kTileRows + lane;
+        if (OM == OUT_F32_ADD) {
+            // residual stream: y = y + the rows (fp32)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) yr[32 * q] = __fadd_rn(yr[32 * q], v[q]);
+            continue;
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) yr[32 * q] = v[q];
         if (OM == OUT_F32_Q81) {
@@ -919,6 +926,33 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
         }
         if (xuse) mbar_wait_bounded(&mybar[S], (xuse - 1) & 1u, nullptr, g.budget_ns);
     }
+}
+
+// RMS normalisation of each row of h (one warp per row): lane j sums h_i^2
+// for i = j, j + 32, ... with fused multiply-adds, an xor butterfly (16 .. 1)
+// of adds gives the total, ms = total / H, r = sqrt(ms + 1e-6), out_i =
+// h_i / r (every operation IEEE round-to-nearest).
+__global__ void __launch_bounds__(256) k_rmsnorm(const float* __restrict__ h, int T, int H, float* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* hr = h + (int64_t)t * H;
+    float p = 0.0f;
+    for (int i = lane; i < H; i += 32) p = __fmaf_rn(hr[i], hr[i], p);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+    const float ms = __fdiv_rn(p, (float)H);
+    const float r = __fsqrt_rn(__fadd_rn(ms, 1e-6f));
+    float* orow = out + (int64_t)t * H;
+    for (int i = lane; i < H; i += 32) orow[i] = __fdiv_rn(hr[i], r);
+}
+
+// The residual stream's first value: fp32 copy of x (bf16 or fp32).
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_to_f32(const void* __restrict__ x, int64_t n, float* __restrict__ h) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    h[i] = BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[i]) : static_cast<const float*>(x)[i];
 }
 
 // ============================================================================

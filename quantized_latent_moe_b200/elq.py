@@ -58,6 +58,8 @@ SIGNATURES = {
     "elq_moe_experts_grouped": (I32, [ctypes.POINTER(LayerC), V, V, V, I32, V, V, SZ, V]),
     "elq_workspace_bytes": (SZ, [ctypes.POINTER(LayerC), I32]),
     "elq_moe_layer": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V]),
+    "elq_moe_stack": (I32, [ctypes.POINTER(LayerC), I32, V, I32, I32, V, V, SZ, V]),
+    "elq_stack_workspace_bytes": (SZ, [ctypes.POINTER(LayerC), I32]),
     "elq_workspace_status": (I32, [V, V]),
     "elq_layer_kernel_count": (I32, [ctypes.POINTER(LayerC), I32]),
     "elq_workspace_view": (I32, [ctypes.POINTER(LayerC), I32, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
@@ -210,6 +212,21 @@ class Layer:
             self._ws[key] = ws
         return ws
 
+    def stack_workspace(self, T: int) -> torch.Tensor:
+        """A zero-filled workspace for elq_moe_stack over layers of this shape."""
+        key = ("stack", T)
+        ws = self._ws.get(key)
+        if ws is None:
+            s = self.struct()
+            n = int(_lib().elq_stack_workspace_bytes(ctypes.byref(s), T))
+            if n == 0:
+                raise ElqError(-1, "elq_stack_workspace_bytes")
+            ws = torch.zeros(n + 256, dtype=torch.uint8, device=self.router_w.device)
+            off = (-ws.data_ptr()) % 256
+            ws = ws[off:off + n]
+            self._ws[key] = ws
+        return ws
+
     def share_workspace(self, T: int, ws: torch.Tensor):
         """Use `ws` (another layer's workspace of the same shape) for T tokens:
         calls that run one after another on one stream may share it."""
@@ -303,6 +320,22 @@ def moe_layer(layer: Layer, x: torch.Tensor, y: torch.Tensor | None = None, ws=N
     _ck(_lib().elq_moe_layer(ctypes.byref(s), _ptr(x), xt, T, _ptr(y), _ptr(ws), ws.numel(),
                              _stream(stream)), "elq_moe_layer")
     return y
+
+
+def moe_stack(layers, x: torch.Tensor, h: torch.Tensor | None = None, ws=None, stream=None) -> torch.Tensor:
+    """h = fp32(x), then h = h + layer(rms(h)) for each layer in turn (one
+    residual stream, fp32).  All layers of one shape; one workspace serves them."""
+    x = x.contiguous()
+    T = x.shape[0]
+    xt = {torch.float32: F32, torch.bfloat16: BF16}[x.dtype]
+    if h is None:
+        h = torch.empty(T, layers[0].H, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = layers[0].stack_workspace(T)
+    arr = (LayerC * len(layers))(*[ly.struct() for ly in layers])
+    _ck(_lib().elq_moe_stack(arr, len(layers), _ptr(x), xt, T, _ptr(h), _ptr(ws), ws.numel(), _stream(stream)),
+        "elq_moe_stack")
+    return h
 
 
 def moe_layer_profiled(layer: Layer, x: torch.Tensor, y: torch.Tensor, events, ws=None,

@@ -107,6 +107,23 @@ def test_layer_validation(L):
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, -1, y, ws_small, 1 << 30, None) == -1
 
 
+def test_stack_validation(L):
+    ws = ctypes.c_void_p(1 << 26)
+    x = ctypes.c_void_p(1 << 27)
+    h = ctypes.c_void_p(1 << 28)
+    arr = (elq.LayerC * 2)(_layer(), _layer())
+    # refused before any launch: bad counts, mixed shapes, unsupported T, input type, workspace
+    assert L.elq_moe_stack(arr, 0, x, 0, 4, h, ws, 1 << 30, None) == -1
+    assert L.elq_moe_stack(None, 2, x, 0, 4, h, ws, 1 << 30, None) == -1
+    mixed = (elq.LayerC * 2)(_layer(), _layer(I=512))
+    assert L.elq_moe_stack(mixed, 2, x, 0, 4, h, ws, 1 << 30, None) == -1
+    assert L.elq_moe_stack(arr, 2, x, 0, 64, h, ws, 1 << 30, None) == -2       # tensor-core sizes
+    assert L.elq_moe_stack(arr, 2, x, 5, 4, h, ws, 1 << 30, None) == -2
+    assert L.elq_moe_stack(arr, 2, x, 0, 4, h, ws, 16, None) == -4
+    assert L.elq_moe_stack(arr, 2, ctypes.c_void_p((1 << 27) + 4), 0, 4, h, ws, 1 << 30, None) == -3
+    assert L.elq_moe_stack(arr, 2, x, 0, 0, h, ws, 1 << 30, None) == 0         # nothing to do
+
+
 def test_other_entry_validation(L):
     p = ctypes.c_void_p(1 << 24)
     assert L.elq_quantize_q8_1(p, 0, 4, 48, p, None) == -2          # cols % 32

@@ -241,3 +241,38 @@ def test_experts_grouped_exact(E, orc):
     w = torch.from_numpy(tr["w"]).cuda()
     y_lat = E.moe_experts_grouped(ly, zq, idx, w).cpu().numpy()
     assert np.array_equal(y_lat, tr["y_lat"])
+
+
+def test_router_nan_inputs_give_valid_ids(E, orc):
+    """R18 on the GPU: NaN latent rows and a NaN bias route exactly as the
+    oracle's (NaN ranks as -inf), so no invalid expert id reaches the
+    bucketing or the expert kernels."""
+    T, L, E_, k = 5, 1792, 128, 8
+    z = _gen(9, 600, (T, L))
+    z[1, 100] = float("nan")
+    w = _gen(9, 601, (E_, L), 0.02)
+    b = _gen(9, 602, E_)
+    ref_idx0, _, _ = orc.router_topk(z[:1].numpy(), w.numpy(), b.numpy(), k)
+    b[int(ref_idx0[0, 0])] = float("nan")
+    idx, wts, lg = E.router_topk(z.cuda(), w.cuda(), b.cuda(), k)
+    ridx, rw, rlg = orc.router_topk(z.numpy(), w.numpy(), b.numpy(), k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.array_equal(wts.cpu().numpy(), rw, equal_nan=True)
+    assert np.array_equal(lg.cpu().numpy(), rlg, equal_nan=True)
+    assert ridx[1].tolist() == list(range(k)) and int(ref_idx0[0, 0]) not in ridx[0].tolist()
+
+
+def test_layer_with_a_nan_token(E, orc):
+    """A NaN token does not fault the layer; the other tokens' outputs are
+    exactly the oracle's."""
+    wl = synth.WORKLOADS["tiny"]
+    ly = gpu_layer(wl)
+    ol = oracle_layer(orc, wl)
+    for T in (3, 12):
+        x = synth.normal(wl.seed, 610 + T, (T, wl.H))
+        x[1, 3] = float("nan")
+        y = E.moe_layer(ly, x.cuda()).cpu().numpy()
+        assert E.workspace_status(ly.workspace(T)) == 0
+        ref = ol.forward(x.numpy())
+        keep = [t for t in range(T) if t != 1]
+        assert np.array_equal(y[keep], ref[keep])

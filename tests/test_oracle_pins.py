@@ -346,3 +346,57 @@ def test_arena_pack_spot_positions(orc):
     assert q4[1 * nb * 2048 + 0 + 2 * 512 + 5 * 16 + 7] == b4[133, 2, 2 + 7]
     # row 255 (tile 1, slice 3, r 31), block 0, byte 0
     assert q4[1 * nb * 2048 + 3 * nb * 512 + 0 + 31 * 16] == b4[255, 0, 2]
+
+
+# ---- R18: NaN router logits rank as -infinity --------------------------------
+
+def test_router_nan_logits_rank_last(orc):
+    rng = np.random.default_rng(11)
+    L, E, k = 64, 8, 3
+    Wr = rng.normal(size=(E, L)).astype(np.float32)
+    z = rng.normal(size=(2, L)).astype(np.float32)
+    z[1, 7] = np.nan                                   # token 1: every logit NaN
+    idx, w, logits = orc.router_topk(z, Wr, None, k)
+    assert np.isnan(logits[1]).all()
+    assert idx[1].tolist() == [0, 1, 2]                # all tie at -inf: lower ids first
+    # a NaN bias removes that expert from the choice of a finite token
+    ref_idx, _, _ = orc.router_topk(z[:1], Wr, None, k)
+    bias = np.zeros(E, np.float32)
+    bias[ref_idx[0, 0]] = np.nan
+    idx2, w2, _ = orc.router_topk(z[:1], Wr, bias, k)
+    assert ref_idx[0, 0] not in idx2[0].tolist()
+    assert np.isfinite(w2).all() and abs(float(w2.sum()) - 1.0) < 1e-6
+    assert idx2[0, :k - 1].tolist() == ref_idx[0, 1:].tolist()
+
+
+# ---- the stack's RMS normalisation -------------------------------------------
+
+def test_rmsnorm_constant_row_closed_form(orc):
+    for c, H in ((3.0, 64), (0.5, 4096), (-2.0, 1792)):
+        h = np.full((1, H), c, np.float32)
+        ms = np.float32(c * c)                         # the sum of H equal squares is exact here
+        r = np.sqrt(ms + np.float32(1e-6), dtype=np.float32)
+        assert np.array_equal(orc.rmsnorm(h), np.full((1, H), np.float32(c) / r, np.float32))
+
+
+def test_rmsnorm_single_spike(orc):
+    H = 256
+    h = np.zeros((1, H), np.float32)
+    h[0, 77] = 16.0
+    out = orc.rmsnorm(h)
+    r = np.sqrt(np.float32(256.0 / H) + np.float32(1e-6), dtype=np.float32)
+    assert out[0, 77] == np.float32(16.0) / r and np.count_nonzero(out) == 1
+
+
+def test_rmsnorm_against_fp64(orc):
+    rng = np.random.default_rng(5)
+    h = (rng.normal(size=(6, 4096)) * np.array([[1e-3], [1.0], [7.0], [100.0], [0.3], [42.0]])).astype(np.float32)
+    out = orc.rmsnorm(h).astype(np.float64)
+    hd = h.astype(np.float64)
+    ref = hd / np.sqrt((hd * hd).mean(axis=1, keepdims=True) + 1e-6)
+    assert np.abs(out - ref).max() <= 4e-6 * np.abs(ref).max()
+    # unit RMS afterwards where eps is negligible; 1/sqrt(2) where mean(h^2) == eps
+    rms = np.sqrt((out * out).mean(axis=1))
+    assert np.allclose(rms[1:], 1.0, rtol=1e-5)
+    ms0 = (hd[0] * hd[0]).mean()
+    assert abs(rms[0] - np.sqrt(ms0 / (ms0 + 1e-6))) < 1e-6
