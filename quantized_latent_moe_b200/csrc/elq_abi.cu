@@ -117,6 +117,11 @@ struct WPlan {
 // rows_per_group: matrix rows of one group; k: reduction length; groups_max:
 // bound on active groups; tok_rows: rows of the partial buffer's token
 // dimension (T or T*k); tokmax: most tokens one group can hold.
+constexpr int kDenseTg = 8;   // tokens per group of a dense projection (the groups share the weights)
+constexpr int kGroupTok = 8;  // tokens staged per unit for an expert group (more take extra passes)
+
+int dense_groups(int T) { return (T + kDenseTg - 1) / kDenseTg; }
+
 WPlan plan_w(int fmt, int x_mode, int rows_per_group, int k, int groups_max, int64_t tok_rows, int tokmax) {
     WPlan p;
     p.tiles = rows_per_group / kTileRows;
@@ -203,6 +208,7 @@ WArgs dense_w(const elq_qmat* w, int T, const void* x, int x_mode, int64_t x_row
     g.part_tok = T;
     g.counters = counters;
     g.err = err;
+    g.dense_tg = kDenseTg;
     return g;
 }
 
@@ -240,7 +246,7 @@ struct ProjWs {
 ProjWs proj_layout(const elq_qmat* w, int T, void* base, bool allow_tc = true) {
     ProjWs ws;
     ws.tc = allow_tc && tc_path(w->fmt, T);
-    ws.plan = plan_w(w->fmt, X_Q81_TOKEN, w->n_rows, w->k, 1, T, T);
+    ws.plan = plan_w(w->fmt, X_Q81_TOKEN, w->n_rows, w->k, dense_groups(T), T, std::min(T, kDenseTg));
     if (ws.tc) {
         ws.plan.partial_bytes = 0;
         ws.plan.counter_ints = 0;
@@ -387,10 +393,10 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.tc = tc_path(ly->D.fmt, T) && tc_path(ly->U.fmt, T) && tc_path(ly->gate_up.fmt, T) && tc_path(ly->down.fmt, T);
     w.raw = T <= kRawMaxT;
     const int dmode = w.raw ? (x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32) : X_Q81_TOKEN;
-    w.pd = plan_w(ly->D.fmt, dmode, L, H, 1, T, T);
-    w.pgu = plan_w(ly->gate_up.fmt, X_Q81_PAIR_TOKEN, 2 * I, L, gmax, P, T);
-    w.pdn = plan_w(ly->down.fmt, X_Q81_POSITION, L, I, gmax, P, T);
-    w.pu = plan_w(ly->U.fmt, X_Q81_TOKEN, H, L, 1, T, T);
+    w.pd = plan_w(ly->D.fmt, dmode, L, H, dense_groups(T), T, std::min(T, kDenseTg));
+    w.pgu = plan_w(ly->gate_up.fmt, X_Q81_PAIR_TOKEN, 2 * I, L, gmax, P, std::min(T, kGroupTok));
+    w.pdn = plan_w(ly->down.fmt, X_Q81_POSITION, L, I, gmax, P, std::min(T, kGroupTok));
+    w.pu = plan_w(ly->U.fmt, X_Q81_TOKEN, H, L, dense_groups(T), T, std::min(T, kDenseTg));
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     w.dec = plan_dec(ly, T);
     w.fused = !w.tc && w.dec.ok;

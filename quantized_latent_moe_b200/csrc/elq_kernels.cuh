@@ -482,6 +482,7 @@ struct WArgs {
     float* partial;             // [nchunks][part_tok][tiles*128]
     int64_t part_tok;
     int* counters;              // [groups][tiles], zero on entry/exit
+    int dense_tg;               // dense: tokens per group (the token groups share the weights); 0 = all T
     int* err;
     uint64_t budget_ns;
     int stages, tokcap;
@@ -500,6 +501,14 @@ struct WUnit {
     int a, tile, c, s, e, tok0, ntok, kbn;
 };
 
+// A warp's cache of the last group it decoded: its expert, first pair
+// position and pair count, and (lane i < ntok) the token of its pair i.  The
+// units a warp takes run in group order, so one L2 round trip per group
+// replaces one per unit.
+struct WGroupCache {
+    int a, e, tok0, ntok, tok;
+};
+
 __device__ __forceinline__ WUnit wunit(const WArgs& g, int u) {
     WUnit r;
     const int per_tile = g.nchunks * 4;
@@ -515,8 +524,46 @@ __device__ __forceinline__ WUnit wunit(const WArgs& g, int u) {
         r.tok0 = __ldcg(g.offsets + r.e);
         r.ntok = __ldcg(g.offsets + r.e + 1) - r.tok0;
     } else {
-        r.tok0 = 0;
-        r.ntok = g.T;
+        const int tg = g.dense_tg > 0 ? g.dense_tg : g.T;
+        r.tok0 = r.a * tg;
+        r.ntok = min(tg, g.T - r.tok0);
+    }
+    r.kbn = min(kChunk, g.nb - r.c * kChunk);
+    return r;
+}
+
+// wunit through the warp's group cache (all lanes call it with the same u).
+template <int XM>
+__device__ __forceinline__ WUnit wunit_c(const WArgs& g, int u, WGroupCache& c) {
+    WUnit r;
+    const int per_tile = g.nchunks * 4;
+    const int per_group = g.tiles * per_tile;
+    r.a = u / per_group;
+    int rem = u - r.a * per_group;
+    r.tile = rem / per_tile;
+    rem -= r.tile * per_tile;
+    r.c = rem >> 2;
+    r.s = rem & 3;
+    if (g.act) {
+        if (c.a != r.a) {
+            c.a = r.a;
+            c.e = __ldcg(g.act + r.a);
+            c.tok0 = __ldcg(g.offsets + c.e);
+            c.ntok = __ldcg(g.offsets + c.e + 1) - c.tok0;
+            c.tok = 0;
+            if (XM == X_Q81_PAIR_TOKEN) {
+                const int lane = threadIdx.x & 31;
+                if (lane < c.ntok) c.tok = __ldcg(g.perm + c.tok0 + lane) / g.kslots;
+            }
+        }
+        r.e = c.e;
+        r.tok0 = c.tok0;
+        r.ntok = c.ntok;
+    } else {
+        const int tg = g.dense_tg > 0 ? g.dense_tg : g.T;
+        r.e = 0;
+        r.tok0 = r.a * tg;
+        r.ntok = min(tg, g.T - r.tok0);
     }
     r.kbn = min(kChunk, g.nb - r.c * kChunk);
     return r;
@@ -558,11 +605,13 @@ __device__ __forceinline__ void wissue_weights(const WArgs& g, const WUnit& un, 
 
 template <int XM>
 __device__ __forceinline__ void wissue_acts(const WArgs& g, const WUnit& un, uint8_t* act_area, uint64_t* bar,
-                                            int first, int ntok_pass) {
+                                            int first, int ntok_pass, const WGroupCache* c = nullptr) {
     const int lane = threadIdx.x & 31;
     const uint32_t ab = wact_bytes<XM>(un.kbn);
     for (int i = lane; i < ntok_pass; i += 32) {
-        const int64_t row = wunit_xrow<XM>(g, un, first + i);
+        const int64_t row = (XM == X_Q81_PAIR_TOKEN && c && first == 0 && i < 32 && c->a == un.a)
+                                ? (int64_t)c->tok
+                                : wunit_xrow<XM>(g, un, first + i);
         const uint8_t* src;
         if (XM == X_RAW_F32)
             src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)un.c * 256) * 4;
@@ -804,7 +853,8 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
     const bool early = dense || g.routing_early;
     int64_t n_units = 0, u0 = 0, u1 = 0;
     auto range = [&]() {
-        const int64_t groups = dense ? 1 : (int64_t)__ldcg(g.n_act);
+        const int64_t groups = dense ? (g.dense_tg > 0 ? (g.T + g.dense_tg - 1) / g.dense_tg : 1)
+                                     : (int64_t)__ldcg(g.n_act);
         n_units = groups * g.tiles * g.nchunks * 4;
         u0 = n_units * blockIdx.x / gridDim.x;
         u1 = n_units * (blockIdx.x + 1) / gridDim.x;
@@ -816,6 +866,10 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
         return (u < u1) ? u : -1;
     };
     const int tokcap = g.tokcap;
+    WGroupCache gcache{-1, 0, 0, 0, 0};
+    // completions are counted in batches; heavier units (more tokens each)
+    // count sooner, so that tile epilogues spread over the warps
+    const int cbatch = max(1, 32 / max(1, tokcap));
 
     // prologue: fill the ring.  Weights do not depend on the upstream kernel
     // (and the routing, when it was complete before this grid started), so
@@ -826,7 +880,7 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             const int u = grab();
             if (lane == 0) myunit[st] = u;
             if (u >= 0) {
-                const WUnit un = wunit(g, u);
+                const WUnit un = wunit_c<XM>(g, u, gcache);
                 wissue_weights<FMT, XM>(g, un, stages + st * g.stage_bytes, &mybar[st], min(un.ntok, tokcap));
             }
         }
@@ -836,8 +890,8 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
         for (int st = 0; st < S; ++st) {
             const int u = myunit[st];
             if (u >= 0) {
-                const WUnit un = wunit(g, u);
-                wissue_acts<XM>(g, un, stages + st * g.stage_bytes + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+                const WUnit un = wunit_c<XM>(g, u, gcache);
+                wissue_acts<XM>(g, un, stages + st * g.stage_bytes + g.act_off, &mybar[st], 0, min(un.ntok, tokcap), &gcache);
             }
         }
     } else {
@@ -848,10 +902,10 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             const int u = grab();
             if (lane == 0) myunit[st] = u;
             if (u >= 0) {
-                const WUnit un = wunit(g, u);
+                const WUnit un = wunit_c<XM>(g, u, gcache);
                 uint8_t* stg = stages + st * g.stage_bytes;
                 wissue_weights<FMT, XM>(g, un, stg, &mybar[st], min(un.ntok, tokcap));
-                wissue_acts<XM>(g, un, stg + g.act_off, &mybar[st], 0, min(un.ntok, tokcap));
+                wissue_acts<XM>(g, un, stg + g.act_off, &mybar[st], 0, min(un.ntok, tokcap), &gcache);
             }
         }
     }
@@ -869,7 +923,7 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             ok = false;
             break;
         }
-        const WUnit un = wunit(g, u);
+        const WUnit un = wunit_c<XM>(g, u, gcache);
         uint8_t* stg = stages + st * g.stage_bytes;
 
         int w[kChunk][8];
@@ -904,15 +958,15 @@ __global__ void __launch_bounds__(256, 1) k_wgemv(WArgs g) {
             const int nu = grab();
             if (lane == 0) myunit[st] = nu;
             if (nu >= 0) {
-                const WUnit nn = wunit(g, nu);
+                const WUnit nn = wunit_c<XM>(g, nu, gcache);
                 wissue_weights<FMT, XM>(g, nn, stg, &mybar[st], min(nn.ntok, tokcap));
-                wissue_acts<XM>(g, nn, stg + g.act_off, &mybar[st], 0, min(nn.ntok, tokcap));
+                wissue_acts<XM>(g, nn, stg + g.act_off, &mybar[st], 0, min(nn.ntok, tokcap), &gcache);
             }
         }
         // completion of the tile (the last of its 4 * nchunks units runs the
         // epilogue), batched per warp so that one fence covers many units
         if (lane == npend) pending = u;
-        if (++npend == 32) {
+        if (++npend == cbatch) {
             wcomplete<OM>(g, pending, npend);
             npend = 0;
         }
