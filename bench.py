@@ -266,6 +266,17 @@ def traffic_for(kernel):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(values, world, device):
+    """Each rank's device times -> the max over ranks (every rank gets it);
+    the job is as slow as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_elq(args):
     import torch
     import torch.distributed as dist
@@ -430,10 +441,7 @@ def run_elq(args):
     act = statistics.mean(n_act)
 
     # max over ranks
-    t = torch.tensor([dev_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    dev_ms, e2e_ms = t.tolist()
+    dev_ms, e2e_ms = max_over_ranks([dev_ms, e2e_ms], world, dev)
 
     if rank == 0:
         blk = 34 if wl.fmt == "q8_0" else 18
@@ -645,10 +653,7 @@ def run_stack(args):
         elq.moe_stack([ly], hl, h, ws)
         torch.cuda.synchronize()
         n_act.append(int(elq.workspace_view(ly, wl.T, "n_act", lws).item()))
-    t = torch.tensor([dev_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    dev_ms, e2e_ms = t.tolist()
+    dev_ms, e2e_ms = max_over_ranks([dev_ms, e2e_ms], world, dev)
     if rank == 0:
         blk = 34 if wl.fmt == "q8_0" else 18
         nb_L, nb_H, nb_I = wl.L // 32, wl.H // 32, wl.I // 32
