@@ -664,7 +664,7 @@ def run_stack(args):
         value = tokens / (dev_ms / 1e3)
         hbm_peak, peak_kind = peaks()
         step_s = dev_ms / 1e3 / args.steps
-        names = KERNELS_LARGE_T if nk == 6 else KERNELS_SMALL_T
+        names = {5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[nk]
         gu_ms = kern_ms[names.index("gate_up")]
         P = wl.T * wl.k
         gu_bytes = n_act[0] * 2 * wl.I * nb_L * blk + wl.T * nb_L * 36 + P * nb_I * 36

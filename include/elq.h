@@ -247,10 +247,10 @@ elq_status elq_moe_layer(const elq_layer* layer, const void* x, int32_t x_type, 
  * pointers device memory); x: device [T][H] fp32 or bf16 (the new tokens);
  * h: device [T][H] fp32 output.  ws: one workspace of
  * elq_stack_workspace_bytes(&layers[0], T) bytes, shared by the layers in
- * turn (the layer workspace, then the normalised input).  The separate-kernel
- * path at every T below the tensor-core threshold (T < 64; larger T returns
- * ELQ_ERR_UNSUPPORTED; ELQ_LAYER_FUSED is ignored here).  Launches
- * 1 + n_layers * (1 + the layer's separate-kernel count) kernels.
+ * turn (the layer workspace, then the normalised input).  Each layer takes
+ * the path elq_moe_layer would (ELQ_LAYER_FUSED is ignored here); the last
+ * projection adds into h.  Launches 1 + n_layers * (1 + the layer's kernel
+ * count without ELQ_LAYER_FUSED) kernels.
  * Validation as elq_moe_layer, before anything is enqueued. */
 elq_status elq_moe_stack(const elq_layer* layers, int32_t n_layers, const void* x, int32_t x_type,
                          int32_t T, float* h, void* ws, size_t ws_bytes, void* stream);
@@ -263,7 +263,7 @@ size_t elq_stack_workspace_bytes(const elq_layer* layer, int32_t T);
  * whole layer.  Decode/verify path otherwise, in order: [activation
  * quantiser, for T > 8], D projection (quantising x itself for T <= 8; +
  * latent Q8_1), router (+ top-k, bucketing), gate/up (+ SwiGLU, Q8_1), down
- * (+ weighted combine, Q8_1), U projection.  Tensor-core path (T >= 64 and
+ * (+ weighted combine, Q8_1), U projection.  Tensor-core path (T >= 16 and
  * every matrix Q8_0): activation quantiser, x packing, D, router, slot map, z
  * packing, gate/up, down (+ combine), U. */
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T);
@@ -284,7 +284,7 @@ elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t
  * (int32 [E]), 7 offsets (int32 [E+1]), 8 perm (int32 [T*k]), 9 pos, 10 hq
  * (Q8_1 [T*k][I/32], by pair position), 11 o (fp32 [T*k][L], by position),
  * 12 y_lat (fp32 [T][L]), 13 ylq (Q8_1), 14 number of routed experts (int32).
- * On the tensor-core path (T >= 64, all matrices Q8_0) hq and o are kept in
+ * On the tensor-core path (T >= 16, all matrices Q8_0) hq and o are kept in
  * padded per-expert slots instead, and their views return ELQ_ERR_INVALID_ARG.
  * Sets *offset (bytes from the workspace start) and *bytes; returns ELQ_OK or
  * ELQ_ERR_INVALID_ARG.  The values are those of the last call on that

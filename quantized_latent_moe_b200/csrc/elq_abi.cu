@@ -22,7 +22,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kRouterSmemMax = 200 * 1024;           // dynamic shared memory cap of router/bucket
 constexpr int kGemvSmemMax = 225 * 1024;             // dynamic shared memory cap of the GEMV
 constexpr int kRawMaxT = 8;                          // D quantises x itself up to this many tokens
-constexpr int kTcMinT = 64;                          // tensor-core path from this many tokens (Q8_0 weights)
+constexpr int kTcMinT = 16;                          // tensor-core path from this many tokens (Q8_0 weights)
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -950,7 +950,6 @@ elq_status elq_moe_stack(const elq_layer* layers, int32_t n_layers, const void* 
             return ELQ_ERR_INVALID_ARG;
     }
     if (T == 0) return ELQ_OK;
-    if (layer_tc(&layers[0], T)) return ELQ_ERR_UNSUPPORTED;
     if (!x || !h) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(h, 16)) return ELQ_ERR_ALIGNMENT;
     if (!router_shape_ok(T, layers[0].L, layers[0].E)) return ELQ_ERR_UNSUPPORTED;
@@ -1155,7 +1154,6 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     const bool pdl = (events == nullptr);
     cudaError_t e;
     if (!mark()) return ELQ_ERR_CUDA;
-    if (residual && w.tc) return ELQ_ERR_UNSUPPORTED;
     if (w.fused && !residual) {
         st = run_fused(layer, w, x, x_type, T, y, s);
         if (st != ELQ_OK) return st;
@@ -1189,7 +1187,8 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         st = run_experts_tc(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark);
         if (st != ELQ_OK) return st;
-        TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, TC_OUT_F32, y, nullptr, w.err);
+        TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, residual ? TC_OUT_F32_ADD : TC_OUT_F32, y,
+                             nullptr, w.err);
         if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         return ELQ_OK;
     }

@@ -248,7 +248,7 @@ constexpr int kTcXld = kTcTileRowsPad;
 constexpr int kTcXchg = kTcN * kTcXld * 4;                  // SwiGLU transpose: [token][row], padded rows
 constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg;
 
-enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3 };
+enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
 
 struct TcArgs {
     const uint8_t* q;           // weight arena of group 0
@@ -597,7 +597,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                 const int t = half * 32 + j;
                 if (t < nv) {
                     const int64_t orow = slot0 + t;
-                    g.y[orow * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
+                    float* yp = g.y + orow * g.y_ld + (int64_t)un.rt * kTileRows + row;
+                    // TC_OUT_F32_ADD: the residual stream, y = y + the rows (fp32)
+                    *yp = (g.out_mode == TC_OUT_F32_ADD) ? __fadd_rn(*yp, acc[j]) : acc[j];
                     if (g.out_mode == TC_OUT_F32_Q81)
                         warp_quant_q8_1(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
                 }

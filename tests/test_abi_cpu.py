@@ -79,6 +79,9 @@ def test_layer_validation(L):
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(k=8, flags=1)), 9) == 6  # T > 8
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(E=128, k=16, flags=1)), 8) == 5  # 128 pairs
     assert L.elq_layer_kernel_count(ctypes.byref(good), 9) == 6
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 15) == 6
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 16) == 9                 # tensor cores from 16 tokens
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(fmt=2)), 32) == 6         # Q4_0 stays on the GEMV path
     assert L.elq_layer_kernel_count(None, 4) == 0
     # the fused path keeps its phase flags and counters in the workspace
     assert L.elq_workspace_bytes(ctypes.byref(_layer(flags=1)), 4) > L.elq_workspace_bytes(ctypes.byref(good), 4)
@@ -117,7 +120,7 @@ def test_stack_validation(L):
     assert L.elq_moe_stack(None, 2, x, 0, 4, h, ws, 1 << 30, None) == -1
     mixed = (elq.LayerC * 2)(_layer(), _layer(I=512))
     assert L.elq_moe_stack(mixed, 2, x, 0, 4, h, ws, 1 << 30, None) == -1
-    assert L.elq_moe_stack(arr, 2, x, 0, 64, h, ws, 1 << 30, None) == -2       # tensor-core sizes
+    assert L.elq_moe_stack(arr, 2, x, 0, 64, h, ws, 16, None) == -4           # tensor-core sizes too
     assert L.elq_moe_stack(arr, 2, x, 5, 4, h, ws, 1 << 30, None) == -2
     assert L.elq_moe_stack(arr, 2, x, 0, 4, h, ws, 16, None) == -4
     assert L.elq_moe_stack(arr, 2, ctypes.c_void_p((1 << 27) + 4), 0, 4, h, ws, 1 << 30, None) == -3

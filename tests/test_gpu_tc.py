@@ -1,4 +1,4 @@
-"""Parity of the tensor-core path (tcgen05 kind::i8, T >= 64, Q8_0 weights)
+"""Parity of the tensor-core path (tcgen05 kind::i8, T >= 16, Q8_0 weights)
 with the CPU oracle, through the C ABI."""
 import numpy as np
 import pytest
