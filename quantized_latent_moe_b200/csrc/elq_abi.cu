@@ -270,11 +270,25 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s, bool pdl) {
     return launch(k_pack_b, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, a);
 }
 
+// One kernel per output mode: each launch carries only its own epilogue.
+template <int OM>
+cudaError_t launch_tc_t(const TcArgs& g, cudaStream_t s, bool pdl) {
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_tcgemm<OM>, kTcSmem, optin);
+    if (e != cudaSuccess) return e;
+    return launch(k_tcgemm<OM>, dim3(sm_count()), dim3(kTcThreads), (size_t)kTcSmem, s, pdl, g);
+}
+
 cudaError_t launch_tc(TcArgs g, cudaStream_t s, bool pdl) {
     g.budget_ns = kWaitBudgetNs;
-    cudaError_t e = smem_optin(k_tcgemm, kTcSmem, g_optin_tc);
-    if (e != cudaSuccess) return e;
-    return launch(k_tcgemm, dim3(sm_count()), dim3(kTcThreads), (size_t)kTcSmem, s, pdl, g);
+    switch (g.out_mode) {
+    case TC_OUT_F32: return launch_tc_t<TC_OUT_F32>(g, s, pdl);
+    case TC_OUT_F32_Q81: return launch_tc_t<TC_OUT_F32_Q81>(g, s, pdl);
+    case TC_OUT_SWIGLU: return launch_tc_t<TC_OUT_SWIGLU>(g, s, pdl);
+    case TC_OUT_F32_COMBINE: return launch_tc_t<TC_OUT_F32_COMBINE>(g, s, pdl);
+    case TC_OUT_F32_ADD: return launch_tc_t<TC_OUT_F32_ADD>(g, s, pdl);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 TcArgs dense_tc(const elq_qmat* w, int T, const uint8_t* bq, const float* bd, int64_t bstride, int out_mode,

@@ -326,6 +326,14 @@ __device__ __forceinline__ int tc_units(const TcArgs& g) {
 
 // Write one 32-value Q8_1 block (held one value per lane) into a canonical B
 // buffer at (slot, kb): the warp-level quantiser, then the canonical scatter.
+// Out-of-line pieces of the epilogues, called from 32-way unrolled loops:
+// one copy of their code instead of 32 (the kernels' instruction footprint).
+__device__ __noinline__ void tc_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
+__device__ __noinline__ float tc_swiglu(float g, float u) { return __fmul_rn(silu_f32(g), u); }
+__device__ __noinline__ int tc_qcode(float h, float d) {
+    return (int)fminf(fmaxf(roundf(__fdiv_rn(h, d)), -127.0f), 127.0f);
+}
+
 __device__ __forceinline__ void warp_quant_canonical(float v, uint8_t* cq, float* cd, int64_t cstride,
                                                      int64_t slot, int kb, uint8_t* scratch36) {
     const int lane = threadIdx.x & 31;
@@ -340,6 +348,7 @@ __device__ __forceinline__ void warp_quant_canonical(float v, uint8_t* cq, float
     __syncwarp();
 }
 
+template <int OM>
 __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     extern __shared__ __align__(1024) uint8_t tcsm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(tcsm);            // [stages]
@@ -538,7 +547,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
             // ---- outputs of the tile ----
             const int nv = un.nvalid;
             const int64_t slot0 = un.slot0;
-            if (g.out_mode == TC_OUT_SWIGLU) {
+            if (OM == TC_OUT_SWIGLU) {
                 // transpose the tile's accumulators through shared memory ([token][row], padded), then
                 // each of the first 128 epilogue threads builds one Q8_1 block of h = silu(gate) * up:
                 // h row 32*hb + i of token t takes gate row 32*hb + i and up row 64 + 32*hb + i
@@ -563,7 +572,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     float amax = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
+                        h[i] = tc_swiglu(gr[i], ur[i]);
                         amax = fmaxf(amax, fabsf(h[i]));
                     }
                     const float d = __fdiv_rn(amax, 127.0f);
@@ -574,7 +583,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         int q = 0;
-                        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(h[i], d)), -127.0f), 127.0f);
+                        if (d != 0.0f) q = tc_qcode(h[i], d);
                         sum += q;
                         wq[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
                     }
@@ -599,12 +608,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     const int64_t orow = slot0 + t;
                     float* yp = g.y + orow * g.y_ld + (int64_t)un.rt * kTileRows + row;
                     // TC_OUT_F32_ADD: the residual stream, y = y + the rows (fp32)
-                    *yp = (g.out_mode == TC_OUT_F32_ADD) ? __fadd_rn(*yp, acc[j]) : acc[j];
-                    if (g.out_mode == TC_OUT_F32_Q81)
-                        warp_quant_q8_1(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
+                    *yp = (OM == TC_OUT_F32_ADD) ? __fadd_rn(*yp, acc[j]) : acc[j];
+                    if (OM == TC_OUT_F32_Q81)
+                        tc_quant(acc[j], g.yq + (orow * g.yq_ld + un.rt * 4 + sp) * 36);
                 }
             }
-            if (g.out_mode == TC_OUT_F32_COMBINE) {
+            if (OM == TC_OUT_F32_COMBINE) {
                 // each (token, 32-row block) is combined by the warp that writes its last expert row
                 // block: lane j counts token 32*half + j, all counters of the warp at once
                 __threadfence();
