@@ -71,6 +71,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// 16 consecutive TMEM columns of this thread's lane (32x32b shape).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive TMEM columns of this thread's lane := v.
@@ -238,7 +249,9 @@ constexpr int kTcTileRowsPad = 129; // padded row count of the SwiGLU transpose 
 constexpr int kTcStages = 6;
 constexpr int kTcBufs = 8;          // TMEM accumulators of kTcN columns (all 512 columns), two groups of kTcKS
 constexpr int kTcGroups = kTcBufs / kTcKS;
-constexpr int kTcThreads = 320;
+constexpr int kTcEpiWarps = 16;     // epilogue warps: 4 TMEM lane quarters x 4 column quarters
+constexpr int kTcEpiCols = 16;      // accumulator columns (tokens) per epilogue warp
+constexpr int kTcThreads = 32 * (2 + kTcEpiWarps);
 constexpr int kTcStageA = kTcKS * 4096;
 constexpr int kTcStageB = kTcKS * kTcN * 32;
 constexpr int kTcStageDw = kTcKS * kTileRows * 2;
@@ -247,6 +260,7 @@ constexpr int kTcStage = kTcStageA + kTcStageB + kTcStageDw + kTcStageDa;
 constexpr int kTcXld = kTcTileRowsPad;
 constexpr int kTcXchg = kTcN * kTcXld * 4;                  // SwiGLU transpose: [token][row], padded rows
 constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg;
+static_assert(kTcEpiWarps * kTcEpiCols == 4 * kTcN, "the epilogue warps cover the 128 x 64 tile");
 
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
 
@@ -324,28 +338,14 @@ __device__ __forceinline__ int tc_units(const TcArgs& g) {
     return __ldcg(g.tt_off + __ldcg(g.n_act)) * g.rtiles;
 }
 
-// Write one 32-value Q8_1 block (held one value per lane) into a canonical B
-// buffer at (slot, kb): the warp-level quantiser, then the canonical scatter.
-// Out-of-line pieces of the epilogues, called from 32-way unrolled loops:
-// one copy of their code instead of 32 (the kernels' instruction footprint).
+
+// Out-of-line pieces of the epilogues, called from unrolled loops: one copy
+// of their code instead of one per column (the kernels' instruction
+// footprint).
 __device__ __noinline__ void tc_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
 __device__ __noinline__ float tc_swiglu(float g, float u) { return __fmul_rn(silu_f32(g), u); }
 __device__ __noinline__ int tc_qcode(float h, float d) {
     return (int)fminf(fmaxf(roundf(__fdiv_rn(h, d)), -127.0f), 127.0f);
-}
-
-__device__ __forceinline__ void warp_quant_canonical(float v, uint8_t* cq, float* cd, int64_t cstride,
-                                                     int64_t slot, int kb, uint8_t* scratch36) {
-    const int lane = threadIdx.x & 31;
-    warp_quant_q8_1(v, scratch36);
-    __syncwarp();
-    uint8_t* dst = cq + (int64_t)kb * cstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
-    if (lane < 8) {
-        const uint32_t w = reinterpret_cast<const uint32_t*>(scratch36 + 4)[lane];
-        reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] = w;
-    }
-    if (lane == 0) cd[(int64_t)kb * cstride + slot] = h2f(*reinterpret_cast<const uint16_t*>(scratch36));
-    __syncwarp();
 }
 
 template <int OM>
@@ -355,11 +355,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     uint64_t* empty = full + kTcStages;                             // [stages]
     uint64_t* tfull = empty + kTcStages;                            // [groups]: a stage's MMAs are done
     uint64_t* tempty = tfull + kTcGroups;                           // [groups]: its accumulators drained
-    uint64_t* xfull = tempty + kTcGroups;                           // up rows handed over (4 warps)
-    uint64_t* xempty = xfull + 1;                                   // ... and taken (4 warps)
+    uint64_t* xfull = tempty + kTcGroups;                           // the tile handed over (epilogue warps)
+    uint64_t* xempty = xfull + 1;                                   // ... and taken
     uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(xempty + 1);
     int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
-    uint8_t* scratch = tcsm + 512;                                  // 8 warps x 36 B quantiser scratch
     uint8_t* stages = tcsm + 1024;
     float* xchg = reinterpret_cast<float*>(tcsm + 1024 + kTcStages * kTcStage);
 
@@ -367,14 +366,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     if (threadIdx.x == 0) {
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + 8);      // the MMA commit + 8 epilogue warps
+            mbar_init(&empty[s], 1 + kTcEpiWarps);   // the MMA commit + the epilogue warps
         }
         for (int b = 0; b < kTcGroups; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);
+            mbar_init(&tempty[b], kTcEpiWarps);
         }
-        mbar_init(xfull, 8);
-        mbar_init(xempty, 8);
+        mbar_init(xfull, kTcEpiWarps);
+        mbar_init(xempty, kTcEpiWarps);
         *abort_sm = 0;
         fence_barrier_init();
     }
@@ -470,19 +469,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
         }
     } else {
         // ---------------- epilogue ----------------
-        const int ew = warp - 2;              // 0..7
+        const int ew = warp - 2;              // 0 .. kTcEpiWarps-1
         const int sp = warp & 3;              // TMEM lane quarter this warp may read
-        const int half = ew >> 2;             // tokens 32*half .. +31
+        const int c0 = (ew >> 2) * kTcEpiCols;   // its accumulator columns (tokens) c0 .. c0+15
         const int row = sp * 32 + lane;       // weight row within the tile
-        uint8_t* qs = scratch + ew * 64;
         int it = 0, xc = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
             const TcUnit un = tc_unit(g, u);
             if (!un.valid) continue;
-            float acc[32], part[32];
+            float acc[kTcEpiCols], part[kTcEpiCols];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) { acc[j] = 0.0f; part[j] = 0.0f; }
-            const bool active = half * 32 < un.ncols;
+            for (int j = 0; j < kTcEpiCols; ++j) { acc[j] = 0.0f; part[j] = 0.0f; }
+            const bool active = c0 < un.ncols;
             bool ok = true;
             const uint32_t tlane = (uint32_t)(sp * 32) << 16;
             for (int ks = 0; ks < kstages; ++ks, ++it) {
@@ -497,19 +495,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                 tc_fence_after();
                 const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
                 const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
-                uint32_t rc[32], rn[32];
-                const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + half * 32);
-                tmem_ld32(tb, rc);
+                uint32_t rc[kTcEpiCols], rn[kTcEpiCols];
+                const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + c0);
+                tmem_ld16(tb, rc);
                 tmem_ld_wait();
 #pragma unroll
                 for (int kl = 0; kl < kTcKS; ++kl) {
-                    if (kl + 1 < kTcKS) tmem_ld32(tb + (uint32_t)((kl + 1) * kTcN), rn);   // overlaps the rescale
+                    if (kl + 1 < kTcKS) tmem_ld16(tb + (uint32_t)((kl + 1) * kTcN), rn);   // overlaps the rescale
                     const int kb = ks * kTcKS + kl;
                     if (active) {
                         const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
-                        const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + half * 32);
+                        const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
 #pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
+                        for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
                             const float4 dv = dak[j4];
                             const float da4[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
@@ -522,7 +520,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     }
                     if ((kb & (kChunk - 1)) == kChunk - 1 || kb == g.nb - 1) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
+                        for (int j = 0; j < kTcEpiCols; ++j) {
                             acc[j] = __fadd_rn(acc[j], part[j]);
                             part[j] = 0.0f;
                         }
@@ -530,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     if (kl + 1 < kTcKS) {
                         tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) rc[j] = rn[j];
+                        for (int j = 0; j < kTcEpiCols; ++j) rc[j] = rn[j];
                     }
                 }
                 tc_fence_before();
@@ -556,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     break;
                 }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) xchg[(half * 32 + j) * kTcXld + row] = acc[j];
+                for (int j = 0; j < kTcEpiCols; ++j) xchg[(c0 + j) * kTcXld + row] = acc[j];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(xfull);
                 if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
@@ -602,8 +600,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                 continue;
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int t = half * 32 + j;
+            for (int j = 0; j < kTcEpiCols; ++j) {
+                const int t = c0 + j;
                 if (t < nv) {
                     const int64_t orow = slot0 + t;
                     float* yp = g.y + orow * g.y_ld + (int64_t)un.rt * kTileRows + row;
@@ -615,14 +613,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
             }
             if (OM == TC_OUT_F32_COMBINE) {
                 // each (token, 32-row block) is combined by the warp that writes its last expert row
-                // block: lane j counts token 32*half + j, all counters of the warp at once
+                // block: lane j < 16 counts token c0 + j, all counters of the warp at once
                 __threadfence();
                 __syncwarp();
                 const int L = g.rtiles * kTileRows;
                 const int blk = un.rt * 4 + sp;
-                const int tj = half * 32 + lane;
+                const int tj = c0 + lane;
                 int tok = 0, last = 0;
-                if (tj < nv) {
+                if (lane < kTcEpiCols && tj < nv) {
                     const int i = (int)(slot0 + tj - __ldcg(g.slot_off + un.e));
                     const int p = __ldcg(g.perm + __ldcg(g.offsets + un.e) + i);
                     tok = p / g.kslots;
