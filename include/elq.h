@@ -70,7 +70,7 @@
  *
  * Layer weights
  *   D      : L rows x H;   U : H rows x L  (any weight format each)
- *   router : fp32 [E][L], optional fp32 bias [E]
+ *   router : fp32 [E][L], optional fp32 bias [E]; L <= 2048
  *   gate_up: E * 2I rows x L; expert e owns rows [2I e, 2I (e+1)); its tile j
  *            holds gate rows 64j .. 64j+63 then up rows 64j .. 64j+63.
  *            I % 64 == 0.
@@ -180,7 +180,8 @@ elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_
 /* Router (a3): logits = W_r z + bias, top-k, softmax over the k.  z: device fp32
  * [T][L] (unquantised latent), w_router [E][L], bias [E] or NULL.  idx: device
  * int32 [T][k] in rank order; weights fp32 [T][k]; logits fp32 [T][E] or NULL.
- * 1 <= k <= min(E, 32), E <= 1024, L % 32 == 0. */
+ * 1 <= k <= min(E, 32), E <= 1024, L % 32 == 0, L <= 2048 (each lane of the
+ * router kernel holds its L/32 weights of a router row in registers). */
 elq_status elq_router_topk(const float* z, const float* w_router, const float* bias,
                            int32_t T, int32_t L, int32_t E, int32_t k,
                            int32_t* idx, float* weights, float* logits, void* stream);

@@ -496,7 +496,7 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     const int H = ly->H, L = ly->L, E = ly->E, k = ly->k, I = ly->I;
     if (H <= 0 || L <= 0 || E <= 0 || k <= 0 || I <= 0) return ELQ_ERR_INVALID_ARG;
     if (k > E) return ELQ_ERR_INVALID_ARG;
-    if (k > 32 || E > 1024) return ELQ_ERR_UNSUPPORTED;
+    if (k > 32 || E > 1024 || L > kRouterMaxL) return ELQ_ERR_UNSUPPORTED;
     if (ly->flags & ~ELQ_LAYER_FUSED) return ELQ_ERR_INVALID_ARG;
     if (H % kTileRows || L % kTileRows || I % kTileRows) return ELQ_ERR_UNSUPPORTED;
     if ((int64_t)T * k > (int64_t)1 << 30) return ELQ_ERR_UNSUPPORTED;
@@ -511,14 +511,32 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     return ELQ_OK;
 }
 
-size_t router_smem(int T, int L, int E) {
-    const int nt = std::min(T, kRouterTok);
-    const size_t a = (size_t)(nt + kRouterWarps) * L * 4;
-    const size_t b = (size_t)kRouterWarps * E * 4;
-    return std::max(a, b);
+// Router launch shape: 4 experts per CTA and one token block each while that
+// grid stays within two CTAs per SM; beyond, 16 experts per CTA and about one
+// CTA per SM, each streaming several token blocks.
+struct RouterShape {
+    int nw, gx, gy, stages;
+};
+
+RouterShape router_shape(int T, int E) {
+    RouterShape r;
+    const int rblocks = (T + kRouterTok - 1) / kRouterTok;
+    const int sms = sm_count();
+    r.nw = ((int64_t)rblocks * ((E + 3) / 4) <= 2 * (int64_t)sms) ? 4 : kRouterMaxWarps;
+    r.gx = (E + r.nw - 1) / r.nw;
+    r.gy = r.nw == 4 ? rblocks : std::min(rblocks, std::max(1, sms / r.gx));
+    r.stages = r.gy < rblocks ? 2 : 1;
+    return r;
 }
 
-bool router_shape_ok(int T, int L, int E) { return router_smem(T, L, E) <= (size_t)kRouterSmemMax; }
+size_t router_smem(int T, int L, int E) {
+    const RouterShape r = router_shape(T, E);
+    return (size_t)r.stages * std::min(T, kRouterTok) * L * 4 + (size_t)r.nw * E * 4;
+}
+
+bool router_shape_ok(int T, int L, int E) {
+    return L <= kRouterMaxL && router_smem(T, L, E) <= (size_t)kRouterSmemMax;
+}
 
 cudaError_t launch_router(const float* z, const float* w, const float* bias, int T, int L, int E, int k,
                           int32_t* idx, float* wts, float* logits, int* cnt, bool do_bucket, int32_t* counts,
@@ -536,8 +554,8 @@ cudaError_t launch_router(const float* z, const float* w, const float* bias, int
     a.counts = counts; a.offsets = offsets; a.perm = perm; a.pos = pos; a.act = act; a.n_act = n_act;
     cudaError_t e = smem_optin(k_router, kRouterSmemMax, g_optin_router);
     if (e != cudaSuccess) return e;
-    dim3 grid((E + kRouterWarps - 1) / kRouterWarps, rblocks);
-    return launch(k_router, grid, dim3(kRouterWarps * 32), router_smem(T, L, E), s, pdl, a);
+    const RouterShape r = router_shape(T, E);
+    return launch(k_router, dim3(r.gx, r.gy), dim3(r.nw * 32), router_smem(T, L, E), s, pdl, a);
 }
 
 // Grouped gate/up over the routed pairs: SwiGLU epilogue into hq.
@@ -835,7 +853,7 @@ elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_
 elq_status elq_router_topk(const float* z, const float* w_router, const float* bias, int32_t T, int32_t L,
                            int32_t E, int32_t k, int32_t* idx, float* weights, float* logits, void* stream) {
     if (T < 0 || L <= 0 || E <= 0 || k <= 0 || k > E) return ELQ_ERR_INVALID_ARG;
-    if (k > 32 || E > 1024 || L % 32) return ELQ_ERR_UNSUPPORTED;
+    if (k > 32 || E > 1024 || L % 32 || L > kRouterMaxL) return ELQ_ERR_UNSUPPORTED;
     if (T == 0) return ELQ_OK;
     if (!z || !w_router || !idx || !weights || !logits) return ELQ_ERR_INVALID_ARG;
     if (!aligned(z, 16) || !aligned(w_router, 16) || (bias && !aligned(bias, 4)) || !aligned(idx, 4) ||

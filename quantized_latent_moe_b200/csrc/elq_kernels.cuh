@@ -223,12 +223,18 @@ __global__ void k_bucket(const int32_t* idx, int P, int E, int32_t* counts, int3
 
 // ============================================================================
 // a3 -- router: logits (R9 order), top-k (lower id on ties), softmax over the
-// k selected; optionally a5 by the last CTA.  Grid (ceil(E/4), ceil(T/8)),
-// 128 threads: one warp per expert, 8 tokens per CTA.  The last CTA of a
-// token block does that block's top-k; the last token block buckets.
+// k selected; optionally a5 by the last CTA.  A block of nw warps (4 or 16)
+// holds nw experts, one per warp, each lane keeping its L/32 lane-strided
+// router weights in registers (L <= 2048).  Grid (ceil(E/nw), gy): CTA (x, y)
+// streams the token blocks y, y + gy, ... (8 tokens each) through a bulk-copy
+// ring of one or two stages, so that a latent row is read once per CTA and
+// reused by all its experts.  The last CTA to finish a token block does its
+// top-k; the last token block buckets.
 // ============================================================================
-constexpr int kRouterWarps = 4;
 constexpr int kRouterTok = 8;
+constexpr int kRouterJ = 64;          // register-held router weights per lane
+constexpr int kRouterMaxL = 32 * kRouterJ;
+constexpr int kRouterMaxWarps = 16;
 
 struct RouterArgs {
     const float* z;
@@ -331,86 +337,129 @@ __device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* 
     }
 }
 
-__global__ void __launch_bounds__(128) k_router(RouterArgs a) {
-    extern __shared__ __align__(128) float rsm[];   // [4][L] router rows, then [<=8][L] latent rows
-    __shared__ __align__(8) uint64_t rbar;
-    __shared__ int s_last;
+__global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
+    extern __shared__ __align__(128) float rsm[];   // [stages][<=8][L] latent rows, then [nw][E] scratch
+    __shared__ __align__(8) uint64_t rbar[2];
+    __shared__ int s_last, s_all;
     __shared__ int32_t s_idx[64];
+    const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.y * kRouterTok;
-    const int nt = min(kRouterTok, a.T - t0);
-    const int e0 = blockIdx.x * kRouterWarps;
-    const int ne = min(kRouterWarps, a.E - e0);
-    float* wsm = rsm;
-    float* zsm = rsm + kRouterWarps * a.L;
+    const int L = a.L, E = a.E;
+    const int nj = L >> 5;
+    const int rblocks = (a.T + kRouterTok - 1) / kRouterTok;
+    const int gy = (int)gridDim.y;
+    const int nmine = (rblocks - (int)blockIdx.y + gy - 1) / gy;   // >= 1: gridDim.y <= rblocks
+    const int stages = (gy < rblocks) ? 2 : 1;
+    const int rows = min(a.T, kRouterTok);
+    float* scr = rsm + (size_t)stages * rows * L;
+    const int e = (int)blockIdx.x * nw + warp;
+    const bool has_e = e < E;
+    // the router rows do not depend on the upstream kernel: load them first
+    float wr[kRouterJ];
+    {
+        const float* wrow = a.w + (int64_t)(has_e ? e : 0) * L + lane;
+#pragma unroll
+        for (int j = 0; j < kRouterJ; ++j) wr[j] = (has_e && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
+    }
+    const float bias = (has_e && a.bias) ? __ldg(a.bias + e) : 0.0f;
     if (threadIdx.x == 0) {
-        mbar_init(&rbar, 1);
+        for (int st = 0; st < stages; ++st) mbar_init(&rbar[st], 1);
         fence_barrier_init();
     }
     __syncthreads();
-    // router rows do not depend on the upstream kernel: start them first
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&rbar, (uint32_t)(ne + nt) * a.L * 4u);
-        bulk_g2s(wsm, a.w + (int64_t)e0 * a.L, (uint32_t)ne * a.L * 4u, &rbar);
-    }
     pdl_wait();
     pdl_trigger();
-    if (threadIdx.x == 0) bulk_g2s(zsm, a.z + (int64_t)t0 * a.L, (uint32_t)nt * a.L * 4u, &rbar);
-    if (!mbar_wait_bounded(&rbar, 0, a.err, kRouterBudgetNs)) {
-        mbar_wait_bounded(&rbar, 0, nullptr, kRouterBudgetNs);
-        return;
-    }
-    const int e = e0 + warp;
-    if (warp < ne) {
-        const float* wr = wsm + warp * a.L;
-        const float b = a.bias ? __ldg(a.bias + e) : 0.0f;
-        for (int tt = 0; tt < nt; ++tt) {
-            const float* zt = zsm + tt * a.L;
-            float p = 0.0f;
-            for (int l = lane; l < a.L; l += 32) p = __fmaf_rn(zt[l], wr[l], p);
+    // thread 0: token block number i of this CTA into stage i % stages
+    auto issue = [&](int i) {
+        const int t0 = ((int)blockIdx.y + i * gy) * kRouterTok;
+        const uint32_t bytes = (uint32_t)min(kRouterTok, a.T - t0) * (uint32_t)L * 4u;
+        uint64_t* bar = &rbar[i & (stages - 1)];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(rsm + (size_t)(i & (stages - 1)) * rows * L, a.z + (int64_t)t0 * L, bytes, bar);
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < min(stages, nmine); ++i) issue(i);
+    const bool small = a.do_bucket && rblocks == 1 && a.T * a.k <= 64;
+    for (int i = 0; i < nmine; ++i) {
+        const int b = (int)blockIdx.y + i * gy;
+        const int t0 = b * kRouterTok;
+        const int nt = min(kRouterTok, a.T - t0);
+        const bool ok = mbar_wait_bounded(&rbar[i & (stages - 1)], (uint32_t)(i / stages) & 1u, a.err,
+                                          kRouterBudgetNs);
+        if (!__syncthreads_and(ok)) {
+            // drain this CTA's copies still in flight, then give up
+            for (int q = i; q < min(i + stages, nmine); ++q)
+                mbar_wait_bounded(&rbar[q & (stages - 1)], (uint32_t)(q / stages) & 1u, nullptr, kRouterBudgetNs);
+            return;
+        }
+        if (has_e) {
+            const float* zs = rsm + (size_t)(i & (stages - 1)) * rows * L + lane;
+            for (int tt = 0; tt < nt; tt += 2) {
+                const float* z0 = zs + tt * L;
+                const float* z1 = zs + min(tt + 1, nt - 1) * L;
+                float p0 = 0.0f, p1 = 0.0f;
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(kFull, p, o));
-            if (a.bias) p = __fadd_rn(p, b);
-            if (lane == 0) a.logits[(int64_t)(t0 + tt) * a.E + e] = p;
+                for (int j = 0; j < kRouterJ; ++j) {
+                    if (j < nj) {
+                        p0 = __fmaf_rn(z0[32 * j], wr[j], p0);
+                        p1 = __fmaf_rn(z1[32 * j], wr[j], p1);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    p0 = __fadd_rn(p0, __shfl_xor_sync(kFull, p0, o));
+                    p1 = __fadd_rn(p1, __shfl_xor_sync(kFull, p1, o));
+                }
+                if (a.bias) {
+                    p0 = __fadd_rn(p0, bias);
+                    p1 = __fadd_rn(p1, bias);
+                }
+                if (lane == 0) {
+                    a.logits[(int64_t)(t0 + tt) * E + e] = p0;
+                    if (tt + 1 < nt) a.logits[(int64_t)(t0 + tt + 1) * E + e] = p1;
+                }
+            }
+        }
+        __syncthreads();                       // the stage is consumed: refill it
+        if (threadIdx.x == 0 && i + stages < nmine) issue(i + stages);
+        if (!a.cnt_tok) continue;              // logits only; k_topk follows
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last = (atomicAdd(&a.cnt_tok[b], 1) == (int)gridDim.x - 1);
+        }
+        __syncthreads();
+        if (!s_last) continue;
+        __threadfence();
+        float* lg = scr + (size_t)warp * E;
+        for (int tt = warp; tt < nt; tt += nw) {
+            const int t = t0 + tt;
+            for (int x = lane; x < E; x += 32) lg[x] = __ldcg(a.logits + (int64_t)t * E + x);
+            __syncwarp();
+            warp_topk_softmax(lg, E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k,
+                              small ? s_idx + t * a.k : nullptr);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            a.cnt_tok[b] = 0;
+            s_all = 0;
+            if (a.do_bucket && !small) {
+                __threadfence();
+                s_all = (atomicAdd(a.cnt_all, 1) == rblocks - 1);
+            }
+        }
+        __syncthreads();
+        if (!a.do_bucket) continue;
+        if (small) {
+            if (warp == 0)
+                bucket_warp_small(s_idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act);
+        } else if (s_all) {
+            __threadfence();
+            bucket_cta(a.idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act,
+                       reinterpret_cast<int*>(scr));
+            if (threadIdx.x == 0) *a.cnt_all = 0;
         }
     }
-    __syncthreads();
-    if (!a.cnt_tok) return;     // logits only; k_topk follows
-    if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = (atomicAdd(&a.cnt_tok[blockIdx.y], 1) == (int)gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    const bool small = a.do_bucket && gridDim.y == 1 && a.T * a.k <= 64;
-    float* lg = rsm + warp * a.E;
-    for (int tt = warp; tt < nt; tt += kRouterWarps) {
-        const int t = t0 + tt;
-        for (int x = lane; x < a.E; x += 32) lg[x] = __ldcg(a.logits + (int64_t)t * a.E + x);
-        __syncwarp();
-        warp_topk_softmax(lg, a.E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k,
-                          small ? s_idx + t * a.k : nullptr);
-        __syncwarp();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) a.cnt_tok[blockIdx.y] = 0;
-    if (!a.do_bucket) return;
-    if (small) {
-        if (warp == 0)
-            bucket_warp_small(s_idx, a.T * a.k, a.E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act);
-        return;
-    }
-    if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = (atomicAdd(a.cnt_all, 1) == (int)gridDim.y - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    bucket_cta(a.idx, a.T * a.k, a.E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act,
-               reinterpret_cast<int*>(rsm));
-    if (threadIdx.x == 0) *a.cnt_all = 0;
 }
 
 // Standalone top-k + softmax: one warp per token over logits [T][E].

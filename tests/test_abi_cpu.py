@@ -83,6 +83,8 @@ def test_layer_validation(L):
     assert L.elq_layer_kernel_count(ctypes.byref(good), 16) == 9                 # tensor cores from 16 tokens
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(fmt=2)), 32) == 6         # Q4_0 stays on the GEMV path
     assert L.elq_layer_kernel_count(None, 4) == 0
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(L_=2176)), 4) == 0      # router rows: L <= 2048
+    assert L.elq_layer_kernel_count(ctypes.byref(_layer(L_=2048)), 4) == 5
     # the fused path keeps its phase flags and counters in the workspace
     assert L.elq_workspace_bytes(ctypes.byref(_layer(flags=1)), 4) > L.elq_workspace_bytes(ctypes.byref(good), 4)
     # unknown flag bits are refused
@@ -136,6 +138,7 @@ def test_other_entry_validation(L):
     assert L.elq_router_topk(p, p, None, 1, 64, 8, 9, p, p, p, None) == -1     # k > E
     assert L.elq_router_topk(p, p, None, 1, 64, 64, 33, p, p, p, None) == -2   # k > 32
     assert L.elq_router_topk(p, p, None, 1, 64, 8, 2, p, p, None, None) == -1  # logits required
+    assert L.elq_router_topk(p, p, None, 1, 2080, 8, 2, p, p, p, None) == -2  # L > 2048
     assert L.elq_route_bucket(p, 4, 2, 8, None, p, p, p, None) == -1
     assert L.elq_route_bucket(p, 4, 9, 8, p, p, p, p, None) == -1
     qm = _qm(8, 256, 512)

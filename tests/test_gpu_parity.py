@@ -124,7 +124,8 @@ def test_latent_proj_exact(E, orc, fmt, N, K, T):
 
 
 @pytest.mark.parametrize("T,L,E_,k,bias", [(1, 1792, 128, 8, True), (6, 1280, 128, 8, False),
-                                            (37, 256, 8, 2, False), (5, 64, 33, 32, True)])
+                                            (37, 256, 8, 2, False), (5, 64, 33, 32, True),
+                                            (300, 256, 128, 8, True), (2000, 64, 33, 32, True)])
 def test_router_exact(E, orc, T, L, E_, k, bias):
     z = _gen(7, T, (T, L), 1.3)
     W = _gen(7, 100 + L, (E_, L), 0.02)
@@ -222,6 +223,29 @@ def test_layer_exact_larger_T(E, orc, name, T):
     xq = E.workspace_view(ly, T, "xq").cpu().numpy().reshape(T, -1)
     assert np.array_equal(xq, tr["xq"])
     assert np.array_equal(y, tr["y"])
+
+
+STREAMED = [synth.Workload("wide", 11, 200, 512, 256, 128, 8, 128, synth.Q8_0, synth.F32, "zipf"),
+            synth.Workload("wide4", 12, 160, 512, 256, 128, 8, 128, synth.Q4_0, synth.F32, "normal"),
+            synth.Workload("tiny1500", 0, 1500, 512, 256, 8, 2, 256, synth.Q8_0, synth.F32, "none")]
+
+
+@pytest.mark.parametrize("wl", STREAMED, ids=[w.name for w in STREAMED])
+def test_layer_streamed_router(E, orc, wl):
+    """Token counts at which the router runs 16 experts per CTA and a CTA
+    streams several 8-token blocks through its two-stage ring (top-k by the
+    last CTA to finish each block, bucketing by the last block): every routing
+    output, every intermediate and y equal the oracle's."""
+    ly = gpu_layer(wl)
+    x = synth.make_x(wl)
+    y = E.moe_layer(ly, x.cuda()).cpu().numpy()
+    assert E.workspace_status(ly.workspace(wl.T)) == 0
+    ol = oracle_layer(orc, wl)
+    tr = ol.forward(x.float().numpy(), trace=True)
+    _check_intermediates(E, ly, wl.T, tr)
+    assert np.array_equal(y, tr["y"])
+    y2 = E.moe_layer(ly, x.cuda()).cpu().numpy()        # the counters reset themselves
+    assert np.array_equal(y2, y)
 
 
 def test_layer_repeat_and_ragged_T(E, orc):
