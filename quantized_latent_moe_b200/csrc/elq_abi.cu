@@ -541,10 +541,9 @@ bool router_shape_ok(int T, int L, int E) {
 cudaError_t launch_router(const float* z, const float* w, const float* bias, int T, int L, int E, int k,
                           int32_t* idx, float* wts, float* logits, int* cnt, bool do_bucket, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* pos, int32_t* act, int32_t* n_act,
-                          cudaStream_t s, bool pdl, int* err = nullptr) {
+                          cudaStream_t s, bool pdl) {
     RouterArgs a;
     std::memset(&a, 0, sizeof(a));
-    a.err = err;
     a.z = z; a.w = w; a.bias = bias; a.T = T; a.L = L; a.E = E; a.k = k;
     a.idx = idx; a.wts = wts; a.logits = logits;
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
@@ -1215,7 +1214,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32_Q81, w.z, w.zq, w.err);
         if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits,
-                          w.cnt_router, true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl, w.err);
+                          w.cnt_router, true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         st = run_experts_tc(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark);
         if (st != ELQ_OK) return st;
@@ -1243,7 +1242,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     if (launch_w(gd, layer->D.fmt, w.pd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
     // a3 + a5
     e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits, w.cnt_router,
-                      true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl, w.err);
+                      true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl);
     if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
     // a6 - a9
     st = run_experts(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark, pdl);

@@ -154,7 +154,18 @@ __device__ void bucket_cta(const int32_t* idx, int P, int E, int32_t* counts, in
     __syncthreads();
     const int seg = (P + nw - 1) / nw;
     const int s0 = min(P, warp * seg), s1 = min(P, s0 + seg);
-    for (int p = s0 + lane; p < s1; p += 32) atomicAdd(&hist[warp * E + __ldcg(idx + p)], 1);
+    // 8 chunks of 32 pairs loaded ahead of their updates
+    for (int c0 = s0; c0 < s1; c0 += 256) {
+        int ev[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = c0 + 32 * u + lane;
+            ev[u] = p < s1 ? __ldcg(idx + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (ev[u] >= 0) atomicAdd(&hist[warp * E + ev[u]], 1);
+    }
     __syncthreads();
     if (warp == 0) {
         const int per = (E + 31) / 32;
@@ -184,20 +195,29 @@ __device__ void bucket_cta(const int32_t* idx, int P, int E, int32_t* counts, in
         if (lane == 31) offsets[E] = incl;
     }
     __syncthreads();
-    for (int c0 = s0; c0 < s1; c0 += 32) {
-        const int p = c0 + lane;
-        const bool v = p < s1;
-        const int e = v ? __ldcg(idx + p) : -1 - lane;
-        const unsigned m = __match_any_sync(kFull, e);
-        if (v) {
-            const int r = __popc(m & ((1u << lane) - 1u));
-            const int posn = hist[warp * E + e] + r;
-            perm[posn] = p;
-            pos[p] = posn;
+    for (int c0 = s0; c0 < s1; c0 += 256) {
+        int ev[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = c0 + 32 * u + lane;
+            ev[u] = p < s1 ? __ldcg(idx + p) : -1 - lane;
         }
-        __syncwarp();
-        if (v && lane == __ffs(m) - 1) hist[warp * E + e] += __popc(m);
-        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = c0 + 32 * u + lane;
+            const bool v = p < s1;
+            const int e = ev[u];
+            const unsigned m = __match_any_sync(kFull, e);
+            if (v) {
+                const int r = __popc(m & ((1u << lane) - 1u));
+                const int posn = hist[warp * E + e] + r;
+                perm[posn] = p;
+                pos[p] = posn;
+            }
+            __syncwarp();
+            if (v && lane == __ffs(m) - 1) hist[warp * E + e] += __popc(m);
+            __syncwarp();
+        }
     }
     __syncthreads();
     if (act && warp == 0) {
@@ -226,7 +246,7 @@ __global__ void k_bucket(const int32_t* idx, int P, int E, int32_t* counts, int3
 // k selected; optionally a5 by the last CTA.  A block of nw warps (4 or 16)
 // holds nw experts, one per warp, each lane keeping its L/32 lane-strided
 // router weights in registers (L <= 2048).  Grid (ceil(E/nw), gy): CTA (x, y)
-// streams the token blocks y, y + gy, ... (8 tokens each) through a bulk-copy
+// streams the token blocks y, y + gy, ... (8 tokens each) through a cp.async
 // ring of one or two stages, so that a latent row is read once per CTA and
 // reused by all its experts.  The last CTA to finish a token block does its
 // top-k; the last token block buckets.
@@ -248,10 +268,7 @@ struct RouterArgs {
     int* cnt_all;     // [1]
     int do_bucket;
     int32_t *counts, *offsets, *perm, *pos, *act, *n_act;
-    int* err;         // device error word or NULL
 };
-
-constexpr uint64_t kRouterBudgetNs = 2000000000ull;
 
 // Top-k of one token's logits (in shared memory, lg[0..E)) by one warp, then
 // the softmax over the k selected in rank order.  Lane j ends with rank j.
@@ -339,7 +356,6 @@ __device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* 
 
 __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
     extern __shared__ __align__(128) float rsm[];   // [stages][<=8][L] latent rows, then [nw][E] scratch
-    __shared__ __align__(8) uint64_t rbar[2];
     __shared__ int s_last, s_all;
     __shared__ int32_t s_idx[64];
     const int nw = blockDim.x >> 5;
@@ -362,36 +378,32 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
         for (int j = 0; j < kRouterJ; ++j) wr[j] = (has_e && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
     }
     const float bias = (has_e && a.bias) ? __ldg(a.bias + e) : 0.0f;
-    if (threadIdx.x == 0) {
-        for (int st = 0; st < stages; ++st) mbar_init(&rbar[st], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
     pdl_wait();
     pdl_trigger();
-    // thread 0: token block number i of this CTA into stage i % stages
+    // token block number i of this CTA into stage i % stages: one cp.async
+    // group per block (an empty group past the last block keeps the count)
     auto issue = [&](int i) {
-        const int t0 = ((int)blockIdx.y + i * gy) * kRouterTok;
-        const uint32_t bytes = (uint32_t)min(kRouterTok, a.T - t0) * (uint32_t)L * 4u;
-        uint64_t* bar = &rbar[i & (stages - 1)];
-        mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(rsm + (size_t)(i & (stages - 1)) * rows * L, a.z + (int64_t)t0 * L, bytes, bar);
+        if (i < nmine) {
+            const int t0 = ((int)blockIdx.y + i * gy) * kRouterTok;
+            const int n16 = min(kRouterTok, a.T - t0) * (L >> 2);
+            const float* src = a.z + (int64_t)t0 * L;
+            float* dst = rsm + (size_t)(i & (stages - 1)) * rows * L;
+            for (int c = threadIdx.x; c < n16; c += blockDim.x) cp_async16(dst + 4 * c, src + 4 * c);
+        }
+        cp_async_commit();
     };
-    if (threadIdx.x == 0)
-        for (int i = 0; i < min(stages, nmine); ++i) issue(i);
+    issue(0);
+    if (stages == 2) issue(1);
     const bool small = a.do_bucket && rblocks == 1 && a.T * a.k <= 64;
     for (int i = 0; i < nmine; ++i) {
         const int b = (int)blockIdx.y + i * gy;
         const int t0 = b * kRouterTok;
         const int nt = min(kRouterTok, a.T - t0);
-        const bool ok = mbar_wait_bounded(&rbar[i & (stages - 1)], (uint32_t)(i / stages) & 1u, a.err,
-                                          kRouterBudgetNs);
-        if (!__syncthreads_and(ok)) {
-            // drain this CTA's copies still in flight, then give up
-            for (int q = i; q < min(i + stages, nmine); ++q)
-                mbar_wait_bounded(&rbar[q & (stages - 1)], (uint32_t)(q / stages) & 1u, nullptr, kRouterBudgetNs);
-            return;
-        }
+        if (stages == 2)
+            cp_async_wait<1>();
+        else
+            cp_async_wait<0>();
+        __syncthreads();
         if (has_e) {
             const float* zs = rsm + (size_t)(i & (stages - 1)) * rows * L + lane;
             for (int tt = 0; tt < nt; tt += 2) {
@@ -421,7 +433,7 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
             }
         }
         __syncthreads();                       // the stage is consumed: refill it
-        if (threadIdx.x == 0 && i + stages < nmine) issue(i + stages);
+        if (stages == 2) issue(i + 2);
         if (!a.cnt_tok) continue;              // logits only; k_topk follows
         if (threadIdx.x == 0) {
             __threadfence();
