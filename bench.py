@@ -684,7 +684,8 @@ def run_stack(args):
             "layer_weight_frac": step_bytes / step_s / 1e9 / hbm_peak,
             "kernel_ms": dict(zip(names, kern_ms)),
             "distinct_experts_per_layer": statistics.mean(n_act),
-            "roofline": {"bound": "hbm", "kernel": "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1), T=%d" % wl.T,
+            "roofline": {"bound": "hbm", "kernel": ("k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU), T=%d" if nk == 9
+                                                   else "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1), T=%d") % wl.T,
                          "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": None, "algorithmic_bytes_per_launch": gu_bytes},
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",

@@ -248,13 +248,15 @@ __global__ void k_bucket(const int32_t* idx, int P, int E, int32_t* counts, int3
 // router weights in registers (L <= 2048).  Grid (ceil(E/nw), gy): CTA (x, y)
 // streams the token blocks y, y + gy, ... (8 tokens each) through a cp.async
 // ring of one or two stages, so that a latent row is read once per CTA and
-// reused by all its experts.  The last CTA to finish a token block does its
-// top-k; the last token block buckets.
+// reused by all its experts.  Each token block's top-k is done once all gx
+// CTAs have finished it, normally by its owner CTA (rotating over x) after
+// that CTA's stream; the last top-k buckets.
 // ============================================================================
 constexpr int kRouterTok = 8;
 constexpr int kRouterJ = 64;          // register-held router weights per lane
 constexpr int kRouterMaxL = 32 * kRouterJ;
 constexpr int kRouterMaxWarps = 16;
+constexpr int kRouterOwnWords = 32;   // deferred top-k list: the first 1024 blocks of a CTA
 
 struct RouterArgs {
     const float* z;
@@ -358,6 +360,7 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
     extern __shared__ __align__(128) float rsm[];   // [stages][<=8][L] latent rows, then [nw][E] scratch
     __shared__ int s_last, s_all;
     __shared__ int32_t s_idx[64];
+    __shared__ uint32_t s_own[kRouterOwnWords];   // blocks of this CTA whose top-k it owns
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = a.L, E = a.E;
@@ -395,6 +398,46 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
     issue(0);
     if (stages == 2) issue(1);
     const bool small = a.do_bucket && rblocks == 1 && a.T * a.k <= 64;
+    const bool claims = stages == 2;                       // CTAs stream several blocks
+    const int target = claims ? (int)gridDim.x : (int)gridDim.x - 1;   // counter before the last increment
+    // top-k + softmax of token block b (all threads; its logits are complete),
+    // then the arrival that makes the last token block's owner bucket
+    auto topk_block = [&](int b) {
+        const int t0 = b * kRouterTok;
+        const int nt = min(kRouterTok, a.T - t0);
+        __threadfence();
+        float* lg = scr + (size_t)warp * E;
+        for (int tt = warp; tt < nt; tt += nw) {
+            const int t = t0 + tt;
+            for (int x = lane; x < E; x += 32) lg[x] = __ldcg(a.logits + (int64_t)t * E + x);
+            __syncwarp();
+            warp_topk_softmax(lg, E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k,
+                              small ? s_idx + t * a.k : nullptr);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            a.cnt_tok[b] = 0;
+            s_all = 0;
+            if (a.do_bucket && !small) {
+                __threadfence();
+                s_all = (atomicAdd(a.cnt_all, 1) == rblocks - 1);
+            }
+        }
+        __syncthreads();
+        if (!a.do_bucket) return;
+        if (small) {
+            if (warp == 0)
+                bucket_warp_small(s_idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act);
+        } else if (s_all) {
+            __threadfence();
+            bucket_cta(a.idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act,
+                       reinterpret_cast<int*>(scr));
+            if (threadIdx.x == 0) *a.cnt_all = 0;
+        }
+        __syncthreads();
+    };
+    for (int i = threadIdx.x; i < kRouterOwnWords; i += blockDim.x) s_own[i] = 0u;
     for (int i = 0; i < nmine; ++i) {
         const int b = (int)blockIdx.y + i * gy;
         const int t0 = b * kRouterTok;
@@ -435,43 +478,45 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
         __syncthreads();                       // the stage is consumed: refill it
         if (stages == 2) issue(i + 2);
         if (!a.cnt_tok) continue;              // logits only; k_topk follows
+        // arrival.  When CTAs stream several blocks, block b's counter takes
+        // gx + 1 increments: one arrival per CTA of its token blocks, plus a
+        // claim by its owner CTA (x = i % gx) after that CTA's stream, and
+        // whoever makes the last increment does the top-k -- in practice the
+        // owner, so that the top-k work is spread over the CTAs whatever order
+        // they arrive in.  With one block per CTA the last arrival does it.
+        // An arrival that completes the count defers its top-k to the end of
+        // its own stream.
         if (threadIdx.x == 0) {
             __threadfence();
-            s_last = (atomicAdd(&a.cnt_tok[b], 1) == (int)gridDim.x - 1);
-        }
-        __syncthreads();
-        if (!s_last) continue;
-        __threadfence();
-        float* lg = scr + (size_t)warp * E;
-        for (int tt = warp; tt < nt; tt += nw) {
-            const int t = t0 + tt;
-            for (int x = lane; x < E; x += 32) lg[x] = __ldcg(a.logits + (int64_t)t * E + x);
-            __syncwarp();
-            warp_topk_softmax(lg, E, a.k, a.idx + (int64_t)t * a.k, a.wts + (int64_t)t * a.k,
-                              small ? s_idx + t * a.k : nullptr);
-            __syncwarp();
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            a.cnt_tok[b] = 0;
-            s_all = 0;
-            if (a.do_bucket && !small) {
-                __threadfence();
-                s_all = (atomicAdd(a.cnt_all, 1) == rblocks - 1);
+            const bool last = atomicAdd(&a.cnt_tok[b], 1) == target;
+            if (i < 32 * kRouterOwnWords) {
+                if (last) s_own[i >> 5] |= 1u << (i & 31);
+            } else {
+                s_last = last;
             }
         }
-        __syncthreads();
-        if (!a.do_bucket) continue;
-        if (small) {
-            if (warp == 0)
-                bucket_warp_small(s_idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act);
-        } else if (s_all) {
-            __threadfence();
-            bucket_cta(a.idx, a.T * a.k, E, a.counts, a.offsets, a.perm, a.pos, a.act, a.n_act,
-                       reinterpret_cast<int*>(scr));
-            if (threadIdx.x == 0) *a.cnt_all = 0;
+        if (i >= 32 * kRouterOwnWords) {       // past the deferred list: inline
+            __syncthreads();
+            if (s_last) topk_block(b);
+            __syncthreads();
         }
     }
+    if (!a.cnt_tok) return;
+    if (claims) {
+        for (int i = (int)blockIdx.x; i < nmine; i += (int)gridDim.x) {
+            const int b = (int)blockIdx.y + i * gy;
+            if (threadIdx.x == 0) {
+                __threadfence();
+                s_last = atomicAdd(&a.cnt_tok[b], 1) == target;
+            }
+            __syncthreads();
+            if (s_last) topk_block(b);
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    for (int i = 0; i < min(nmine, 32 * kRouterOwnWords); ++i)
+        if ((s_own[i >> 5] >> (i & 31)) & 1u) topk_block((int)blockIdx.y + i * gy);
 }
 
 // Standalone top-k + softmax: one warp per token over logits [T][E].
