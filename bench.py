@@ -43,7 +43,7 @@ KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "proj_U"]
 KERNELS_FUSED = ["layer"]
-KERNEL_NAMES = {"gate_up": {5: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1)",
+KERNEL_NAMES = {"gate_up": {5: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
                             9: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 
@@ -253,15 +253,15 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel):
+def traffic_for(kernel, workload):
     """dram bytes per launch of `kernel` from the committed ncu summary, only if
-    it was taken on the current kernel sources."""
+    it was taken on the current kernel sources and on this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash() or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -466,7 +466,7 @@ def run_elq(args):
             achieved = lb / (lay_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": KERNEL_NAMES["layer"][1], "achieved": achieved, "peak": hbm_peak,
                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "traffic": traffic_for("layer"), "algorithmic_bytes_per_launch": lb}
+                    "traffic": traffic_for("layer", wl.name), "algorithmic_bytes_per_launch": lb}
         else:
             gu_ms = kern_ms[KERNELS.index("gate_up")]
             dn_ms = kern_ms[KERNELS.index("down")]
@@ -479,14 +479,15 @@ def run_elq(args):
             achieved = gu_ops / (gu_ms / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][9], "achieved": achieved, "peak": tpk,
                     "peak_kind": tkind, "unit": "TOPS (int8)", "frac": achieved / tpk,
-                    "traffic": traffic_for("gate_up_tc"), "algorithmic_ops_per_launch": gu_ops,
+                    "traffic": traffic_for("gate_up_tc", wl.name), "algorithmic_ops_per_launch": gu_ops,
                     "algorithmic_bytes_per_launch": gu_w}
         else:
             gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
             achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-            roof = {"bound": "hbm", "kernel": KERNEL_NAMES["gate_up"][launches_per_step], "achieved": achieved,
+            roof = {"bound": "hbm", "kernel": KERNEL_NAMES["gate_up"][launches_per_step].format(fmt=wl.fmt.upper()),
+                    "achieved": achieved,
                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "traffic": traffic_for("gate_up"), "algorithmic_bytes_per_launch": gu_bytes}
+                    "traffic": traffic_for("gate_up", wl.name), "algorithmic_bytes_per_launch": gu_bytes}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
@@ -685,7 +686,8 @@ def run_stack(args):
             "kernel_ms": dict(zip(names, kern_ms)),
             "distinct_experts_per_layer": statistics.mean(n_act),
             "roofline": {"bound": "hbm", "kernel": ("k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU), T=%d" if nk == 9
-                                                   else "k_wgemv<Q8_0> gate/up (+SwiGLU, Q8_1), T=%d") % wl.T,
+                                                   else "k_wgemv<" + wl.fmt.upper() + "> gate/up (+SwiGLU, Q8_1), T=%d")
+                                                  % wl.T,
                          "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": None, "algorithmic_bytes_per_launch": gu_bytes},
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
