@@ -20,6 +20,11 @@
  *    work, and returns ELQ_OK or a negative elq_status.  On an error nothing is
  *    enqueued and no output is written.  Launch failures return ELQ_ERR_CUDA.
  *    Faults inside kernels surface at the caller's next synchronisation.
+ *  - No tokens (T = 0, or rows = 0) is a valid call: it checks its other
+ *    arguments, then returns ELQ_OK without enqueuing anything or reading its
+ *    data pointers, which may then be NULL; the *_workspace_bytes calls return
+ *    0.  elq_route_bucket is the exception: it still writes zero counts and
+ *    offsets.
  *  - Calls that take a workspace `ws` use it for intermediates.  It must be at
  *    least the size the matching *_workspace_bytes call returns, 256-byte
  *    aligned, and ZERO-FILLED before its first use; every call leaves its

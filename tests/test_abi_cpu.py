@@ -129,6 +129,30 @@ def test_stack_validation(L):
     assert L.elq_moe_stack(arr, 2, x, 0, 0, h, ws, 1 << 30, None) == 0         # nothing to do
 
 
+def test_empty_inputs_return_ok_without_work(L):
+    """T = 0 (no tokens): each entry point still validates its other arguments,
+    then returns ELQ_OK without a launch (no GPU is touched here) and without
+    reading its data pointers."""
+    p = ctypes.c_void_p(1 << 24)
+    good = _layer()
+    assert L.elq_moe_layer(ctypes.byref(good), None, 0, 0, None, None, 0, None) == 0
+    assert L.elq_moe_layer(ctypes.byref(good), None, 30, 0, None, None, 0, None) == 0     # bf16 input
+    assert L.elq_moe_layer(ctypes.byref(good), None, 5, 0, None, None, 0, None) == -2     # input type still checked
+    assert L.elq_moe_layer(ctypes.byref(_layer(k=9)), None, 0, 0, None, None, 0, None) == -1   # layer still checked
+    assert L.elq_moe_experts_grouped(ctypes.byref(good), None, None, None, 0, None, None, 0, None) == 0
+    assert L.elq_router_topk(None, None, None, 0, 64, 8, 2, None, None, None, None) == 0
+    assert L.elq_router_topk(None, None, None, 0, 64, 8, 9, None, None, None, None) == -1  # k > E still checked
+    assert L.elq_quantize_q8_1(None, 0, 0, 64, None, None) == 0
+    qm = _qm(8, 256, 512)
+    assert L.elq_latent_proj(ctypes.byref(qm), None, 0, None, None, 0, None) == 0
+    assert L.elq_latent_proj_noalloc(ctypes.byref(qm), None, 0, None, None) == 0
+    assert L.elq_latent_proj(ctypes.byref(qm), p, -1, p, p, 1 << 30, None) == -1
+    # no tokens need no workspace
+    assert L.elq_workspace_bytes(ctypes.byref(good), 0) == 0
+    assert L.elq_latent_proj_workspace_bytes(ctypes.byref(qm), 0) == 0
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 0) == 0
+
+
 def test_other_entry_validation(L):
     p = ctypes.c_void_p(1 << 24)
     assert L.elq_quantize_q8_1(p, 0, 4, 48, p, None) == -2          # cols % 32
