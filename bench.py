@@ -236,13 +236,37 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # the CUDA path
 
+_INT8_PEAK = None
+
+
 def tensor_peak_int8():
-    """Dense int8 tensor peak: the measured bf16 GEMM rate (burst) x 2, the
-    nominal int8 : bf16 ratio of B200 (4.5 vs 2.25 PFLOP/s)."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        return 2.0 * float(json.load(open(p))["bf16_tflops"]), "measured bf16 x 2"
-    return 2.0 * 1590.0, "fallback bf16 x 2"
+    """Dense int8 tensor-core peak (TOPS), measured on this GPU: one CTA per
+    SM issuing back-to-back tcgen05.mma kind::i8 (M=128, N=256, K=32) from
+    shared memory into TMEM (elq_test_mma_i8_rate), timed with CUDA events
+    on the launching stream after a warm-up launch; the best of five launches
+    (a burst figure, like the measured bf16 peak)."""
+    global _INT8_PEAK
+    if _INT8_PEAK is not None:
+        return _INT8_PEAK
+    import torch
+    from quantized_latent_moe_b200 import elq
+    stream = torch.cuda.current_stream()
+    n_mma = 32768
+    ops = 2.0 * 128 * 256 * 32 * n_mma * elq.sm_count()
+    elq.test_mma_i8_rate(256)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _, err = elq.test_mma_i8_rate(n_mma)
+        e1.record(stream)
+        e1.synchronize()
+        if int(err.item()) != 0:
+            raise RuntimeError("int8 rate kernel: a bounded wait ran out")
+        best = max(best, ops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    _INT8_PEAK = (best, "measured int8 (tcgen05.mma kind::i8 M128 N256 K32 loop, one CTA per SM, best of 5)")
+    return _INT8_PEAK
 
 
 def source_hash():
@@ -275,6 +299,80 @@ def max_over_ranks(values, world, device):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.tolist()
+
+
+class GraphSet:
+    """CUDA graphs of n consecutive steps, keyed by (n, first step mod period):
+    step(i) depends on i only through i mod period, so one graph serves every
+    run of n steps starting at the same phase.  prepare() captures (and
+    replays once) every graph a later run() will use, so that a timed run()
+    replays graphs and never captures one."""
+
+    def __init__(self, G, step, period=None):
+        self.G, self.step = G, step
+        self.period = G if period is None else period
+        self.graphs = {}
+
+    def keys(self, k, start):
+        out, done = [], 0
+        while done < k:
+            n = min(self.G, k - done)
+            out.append((n, (start + done) % self.period))
+            done += n
+        return out
+
+    def _get(self, key):
+        import torch
+        g = self.graphs.get(key)
+        if g is None:
+            n, ph = key
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(ph, ph + n):
+                    self.step(i)
+            self.graphs[key] = g
+        return g
+
+    def prepare(self, k, start):
+        for key in dict.fromkeys(self.keys(k, start)):
+            if key not in self.graphs:
+                self._get(key).replay()
+
+    def run(self, k, start=0):
+        for key in self.keys(k, start):
+            self._get(key).replay()
+        return start + k
+
+    def long_run(self, stream, start, min_ms=300.0, min_steps=400):
+        """Device time per step over a long run of full graphs: replays for at
+        least min_ms of warm-up, then at least min_steps steps and min_ms,
+        each replay timed with CUDA events on the launching stream; the
+        median over replays (ms per step)."""
+        import torch
+        key = (self.G, start % self.period)
+        g = self._get(key)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        t0 = time.perf_counter()
+        while (time.perf_counter() - t0) * 1e3 < min_ms:
+            g.replay()
+            torch.cuda.synchronize()
+        per, steps, total = [], 0, 0.0
+        while steps < min_steps or total < min_ms:
+            ev[0].record(stream)
+            g.replay()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            ms = ev[0].elapsed_time(ev[1])
+            per.append(ms / self.G)
+            steps += self.G
+            total += ms
+        return {"ms_per_step_median": statistics.median(per), "ms_per_step_mean": total / steps,
+                "steps": steps, "replays": len(per), "warmup_ms": min_ms,
+                "note": "median over replays of %d-step graphs after at least %.0f ms of warm-up"
+                        % (self.G, min_ms)}
+
+    def clear(self):
+        self.graphs.clear()
 
 
 def run_elq(args):
@@ -339,29 +437,14 @@ def run_elq(args):
     G = math.lcm(args.copies, S, 2)
     if wl.T > 64:
         G = min(G, 16)
-    graphs = {}
-
-    def graph_for(n, start):
-        key = (n, start % G)
-        if key not in graphs:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for i in range(start, start + n):
-                    step(i)
-            graphs[key] = g
-        return graphs[key]
-
-    def run_steps(k, start=0):
-        done = 0
-        while done < k:
-            n = min(G, k - done)
-            graph_for(n, start + done).replay()
-            done += n
-        return start + k
+    graphs = GraphSet(G, step)
 
     launches_per_step = layers[0].kernel_count(wl.T)
     KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[launches_per_step]
-    pos = run_steps(args.warmup)
+    pos = graphs.run(args.warmup)
+    # every graph the timed steps replay is captured, instantiated and
+    # replayed once here: the timed region holds replays only
+    graphs.prepare(args.steps, pos)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -373,12 +456,13 @@ def run_elq(args):
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    pos = run_steps(args.steps, pos)
+    pos = graphs.run(args.steps, pos)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     dev_ms = e0.elapsed_time(e1)
+    long_run = graphs.long_run(stream, pos)
 
     # end to end through the C ABI with host buffers: pinned x in, y out, every step
     x_host = [x.cpu().pin_memory() for x in xs[:8]]
@@ -499,9 +583,11 @@ def run_elq(args):
                        "l2": "inputs larger than L2: %d layer copies x ~%.0f MB touched per step rotate, "
                              "%.0f MB between reuses of a layer (L2 126 MB)"
                              % (args.copies, layer_bytes / 1e6, (args.copies - 1) * layer_bytes / 1e6),
-                       "cuda_graph": "%d steps per graph%s" % (
+                       "cuda_graph": "%d steps per graph%s; every graph captured and replayed once before "
+                                     "the timed region" % (
                            G, ", one cooperative launch per step" if launches_per_step == 1
                            else ", programmatic dependent launch")},
+            "long_run": long_run,
             "expert_weight_gbs": None if gu_ms is None else (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9,
             "expert_weight_frac": None if gu_ms is None else (gu_w + dn_w) / ((gu_ms + dn_ms) / 1e3) / 1e9 / hbm_peak,
             "layer_weight_gbs": layer_bytes / step_s / 1e9,
@@ -581,24 +667,9 @@ def run_stack(args):
     torch.cuda.synchronize()
     assert elq.workspace_status(ws) == 0
     G = 4
-    graphs = {}
-
-    def run_steps(k, start=0):
-        done = 0
-        while done < k:
-            n = min(G, k - done)
-            key = (n, (start + done) % S)
-            if key not in graphs:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for i in range(start + done, start + done + n):
-                        step(i)
-                graphs[key] = g
-            graphs[key].replay()
-            done += n
-        return start + k
-
-    pos = run_steps(args.warmup)
+    graphs = GraphSet(G, step, period=S)
+    pos = graphs.run(args.warmup)
+    graphs.prepare(args.steps, pos)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -610,7 +681,7 @@ def run_stack(args):
     if world > 1:
         dist.barrier()
     e0.record(stream)
-    pos = run_steps(args.steps, pos)
+    pos = graphs.run(args.steps, pos)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -680,7 +751,8 @@ def run_stack(args):
                        "global_batch": wl.T * world, "parallelism": "replicas" if world > 1 else "1 GPU",
                        "inputs": S, "l2": "inputs larger than L2: %.1f GB of weights touched per step"
                                          % (step_bytes / 1e9),
-                       "cuda_graph": "%d steps per graph" % G},
+                       "cuda_graph": "%d steps per graph; every graph captured and replayed once before "
+                                     "the timed region" % G},
             "layer_weight_gbs": step_bytes / step_s / 1e9,
             "layer_weight_frac": step_bytes / step_s / 1e9 / hbm_peak,
             "kernel_ms": dict(zip(names, kern_ms)),
@@ -708,8 +780,26 @@ def run_stack(args):
         dist.destroy_process_group()
 
 
+def spawn_ranks(n):
+    """`bench.py --gpus N` run directly (no torchrun around it): relaunch this
+    command as N ranks, one per GPU, under torch.distributed.run on this node;
+    rank 0 prints the line.  Returns the launcher's exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
     from quantized_latent_moe_b200 import synth
     wl = synth.WORKLOADS[args.workload]
     if args.steps is None:

@@ -12,9 +12,13 @@
  *
  * Conventions shared by every call
  *  - Pointers named as device pointers are CUDA device memory owned by the
- *    caller.  The library allocates nothing, keeps no state between calls and
- *    never synchronises the stream.  `stream` is a cudaStream_t (NULL = legacy
- *    default stream).
+ *    caller.  The library allocates no memory and never synchronises the
+ *    stream (elq_workspace_status and elq_latent_proj_noalloc_status are the
+ *    documented blocking exceptions).  The state it keeps between calls is
+ *    per device and read-only after the first call there: the SM count, the
+ *    kernels' shared-memory opt-ins, and, for elq_latent_proj_noalloc only,
+ *    the address of its file-scope 4 MiB scratch array (below).  `stream` is
+ *    a cudaStream_t (NULL = legacy default stream).
  *  - Device pointers must be 16-byte aligned unless stated otherwise.
  *  - Every call validates its arguments on the host before it enqueues any
  *    work, and returns ELQ_OK or a negative elq_status.  On an error nothing is
@@ -224,9 +228,19 @@ elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, flo
  *    cudaMemsetAsync) before its kernel; nothing is allocated or freed.
  *  - All calls share the one array: calls that overlap on the GPU (different
  *    streams, or several host threads) race and give wrong results.  Order
- *    them on one stream. */
+ *    them on one stream.
+ *  - A bounded device wait that runs out (2 s) leaves y undefined and sets the
+ *    array's error word, which elq_latent_proj_noalloc_status reads; the next
+ *    call clears it. */
 elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q8_1, int32_t T, float* y,
                                    void* stream);
+
+/* Outcome of the last elq_latent_proj_noalloc call on the current device:
+ * copies the static array's error word to the host (blocking: it
+ * synchronises `stream`, which must be the stream of that call) and returns
+ * ELQ_OK, or ELQ_ERR_TIMEOUT if one of that call's bounded waits ran out.
+ * Allocates nothing; the word is cleared by the next noalloc call. */
+elq_status elq_latent_proj_noalloc_status(void* stream);
 
 /* Grouped experts (a5-a9): bucketing, gate/up with SwiGLU and Q8_1 requant,
  * down, and the weighted combine.  z_q8_1: device T rows of L/32 Q8_1 blocks;
@@ -323,6 +337,20 @@ elq_status elq_test_fused_timeout(const elq_layer* layer, const void* x, int32_t
  * All device pointers, no alignment requirement. */
 elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q8_1,
                                 int64_t nblocks, int32_t* isum, float* term, void* stream);
+
+/* The int8 tensor-core rate, for the roofline's peak: one CTA per SM, each
+ * issuing n_mma (>= 2) tcgen05.mma kind::i8 instructions of M = 128, N = 256,
+ * K = 32 back to back (2 * 128 * 256 * 32 integer operations each) from fixed
+ * shared-memory operands into TMEM, then waiting (bounded, 2 s) for them.
+ * The caller times the launch on `stream` (CUDA events) and divides the
+ * operations, n_mma * elq_sm_count() * 2097152, by the time.  sink: device
+ * int32 [elq_sm_count()], one accumulator word per CTA; err: device int32,
+ * zero before the call, ELQ_ERR_TIMEOUT's code 1 if a wait ran out. */
+elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
+
+/* Streaming multiprocessors of the current device (the grid the persistent
+ * kernels use). */
+int32_t elq_sm_count(void);
 
 /* Runs the library's own exp on n fp32 values (device in -> out). */
 elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream);

@@ -1095,6 +1095,18 @@ elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q
     return cuda_status(cudaGetLastError());
 }
 
+elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream) {
+    if (n_mma < 2 || !sink || !err) return ELQ_ERR_INVALID_ARG;
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_test_mma_i8_rate, kRateSmem, optin);
+    if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    return cuda_status(launch(k_test_mma_i8_rate, dim3(sm_count()), dim3(128), (size_t)kRateSmem,
+                              static_cast<cudaStream_t>(stream), false, (int)n_mma, (int*)sink, (int*)err,
+                              kWaitBudgetNs));
+}
+
+int32_t elq_sm_count(void) { return sm_count(); }
+
 elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream) {
     if (n < 0) return ELQ_ERR_INVALID_ARG;
     if (n == 0) return ELQ_OK;
@@ -1157,6 +1169,18 @@ extern "C" elq_status elq_latent_proj_noalloc(const elq_qmat* w, const void* x_q
         return ELQ_ERR_CUDA;
     WArgs g = dense_w(w, T, x_q8_1, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, lay.partial, lay.counters, lay.err);
     return cuda_status(launch_w(g, w->fmt, lay.plan, s, false));
+}
+
+extern "C" elq_status elq_latent_proj_noalloc_status(void* stream) {
+    void* base = nullptr;
+    elq_status st = static_scratch_address(&base);
+    if (st != ELQ_OK) return st;
+    // the error word is the first int of the array (proj_layout's first carve)
+    int v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, base, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ELQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ELQ_ERR_CUDA;
+    return v == 0 ? ELQ_OK : ELQ_ERR_TIMEOUT;
 }
 
 namespace {

@@ -266,8 +266,8 @@ struct RouterArgs {
     int32_t* idx;
     float* wts;
     float* logits;
-    int* cnt_tok;     // [gridDim.y], zero on entry, zero on exit
-    int* cnt_all;     // [1]
+    int* cnt_tok;     // [rblocks]: one per 8-token block; zero on entry and exit
+    int* cnt_all;     // [1], right after cnt_tok (cnt_tok + rblocks); zero on entry and exit
     int do_bucket;
     int32_t *counts, *offsets, *perm, *pos, *act, *n_act;
 };

@@ -672,4 +672,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     pdl_trigger();
 }
 
+// ---- measurement: the int8 tensor-core rate ------------------------------------
+//
+// One CTA per SM (the launch asks for enough shared memory to keep it alone),
+// one thread issuing n_mma back-to-back tcgen05.mma kind::i8 of M=128, N=256,
+// K=32 (one int8 block of 128 x 256 outputs, 2 * 128 * 256 * 32 operations)
+// from two fixed shared-memory operand tiles into two alternating TMEM
+// accumulators, then one commit.  The operands' values do not matter for the
+// rate; the sink receives one accumulator word per CTA so the work is
+// observable.  Every wait is bounded.
+constexpr int kRateN = 256;
+constexpr int kRateSmem = 150 * 1024;
+
+__global__ void __launch_bounds__(128, 1) k_test_mma_i8_rate(int n_mma, int* sink, int* err, uint64_t budget_ns) {
+    extern __shared__ __align__(1024) uint8_t rsm_[];
+    uint64_t* done = reinterpret_cast<uint64_t*>(rsm_);
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(rsm_ + 8);
+    uint8_t* a = rsm_ + 1024;                 // 128 x 32 codes
+    uint8_t* b = a + 128 * 32;                // 256 x 32 codes
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (128 + kRateN) * 32 / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(a)[i] = 0x01010101u * (uint32_t)((i & 7) + 1);
+    if (threadIdx.x == 0) {
+        mbar_init(done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase, 2 * kRateN);
+        tmem_relinquish();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tbase;
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = umma_idesc_i8(128, kRateN);
+        const uint64_t ad = umma_desc(a, 128, 256), bd = umma_desc(b, 128, 256);
+        for (int i = 0; i < n_mma; ++i)
+            umma_i8(tmem + (uint32_t)((i & 1) * kRateN), ad, bd, idesc, i >= 2 ? 1u : 0u);
+        umma_commit(done);
+    }
+    __syncwarp();
+    const bool ok = warp_wait_bounded(done, 0, err, budget_ns);
+    tc_fence_after();
+    if (warp == 0) {
+        uint32_t r[16];
+        tmem_ld16(tmem, r);
+        tmem_ld_wait();
+        if (ok && threadIdx.x == 0) sink[blockIdx.x] = (int)r[0];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 2 * kRateN);
+}
+
 }  // namespace elq

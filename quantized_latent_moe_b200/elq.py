@@ -55,6 +55,7 @@ SIGNATURES = {
     "elq_latent_proj_workspace_bytes": (SZ, [ctypes.POINTER(QMat), I32]),
     "elq_latent_proj": (I32, [ctypes.POINTER(QMat), V, I32, V, V, SZ, V]),
     "elq_latent_proj_noalloc": (I32, [ctypes.POINTER(QMat), V, I32, V, V]),
+    "elq_latent_proj_noalloc_status": (I32, [V]),
     "elq_moe_experts_grouped": (I32, [ctypes.POINTER(LayerC), V, V, V, I32, V, V, SZ, V]),
     "elq_workspace_bytes": (SZ, [ctypes.POINTER(LayerC), I32]),
     "elq_moe_layer": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V]),
@@ -66,6 +67,8 @@ SIGNATURES = {
     "elq_moe_layer_profiled": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, V, I32, V]),
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
     "elq_test_expf": (I32, [V, V, I64, V]),
+    "elq_test_mma_i8_rate": (I32, [I32, V, V, V]),
+    "elq_sm_count": (I32, []),
     "elq_test_fused_timeout": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, ctypes.c_uint64, V]),
 }
 
@@ -295,6 +298,12 @@ def latent_proj_noalloc(m: QMatrix, xq: torch.Tensor, T: int, y: torch.Tensor | 
     return y
 
 
+def latent_proj_noalloc_status(stream=None) -> int:
+    """Blocking: the outcome of the last elq_latent_proj_noalloc call on this
+    device (0, or the timeout status)."""
+    return int(_lib().elq_latent_proj_noalloc_status(_stream(stream)))
+
+
 def moe_experts_grouped(layer: Layer, zq: torch.Tensor, idx: torch.Tensor, w: torch.Tensor,
                         stream=None) -> torch.Tensor:
     T = idx.shape[0]
@@ -396,6 +405,20 @@ def test_fused_timeout(layer: Layer, x: torch.Tensor, ws: torch.Tensor, budget_n
     s = layer.struct()
     return int(_lib().elq_test_fused_timeout(ctypes.byref(s), _ptr(x), xt, T, _ptr(y), _ptr(ws), ws.numel(),
                                              budget_ns, _stream(stream)))
+
+
+def test_mma_i8_rate(n_mma: int, device="cuda", stream=None):
+    """Launches the int8 tensor-core rate kernel (elq_test_mma_i8_rate) on the
+    current stream; returns (sink, err) device tensors.  The caller times it."""
+    n = int(_lib().elq_sm_count())
+    sink = torch.zeros(n, dtype=torch.int32, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    _ck(_lib().elq_test_mma_i8_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_i8_rate")
+    return sink, err
+
+
+def sm_count() -> int:
+    return int(_lib().elq_sm_count())
 
 
 def test_expf(x: torch.Tensor, stream=None) -> torch.Tensor:

@@ -46,3 +46,41 @@ def test_gemv_label_names_the_format():
         label = bench.KERNEL_NAMES["gate_up"][5].format(fmt=wl.fmt.upper())
         assert ("Q4_0" in label) == (wl.fmt == "q4_0"), label
         assert ("Q8_0" in label) == (wl.fmt == "q8_0"), label
+
+
+class _FakeGraph:
+    def replay(self):
+        pass
+
+
+def test_timed_run_replays_only_prepared_graphs(monkeypatch):
+    """The driver's warm-up and step counts (5 and 20 with 64-step graphs):
+    prepare() captures every graph the timed run() replays, so the timed
+    region never captures one."""
+    captured = []
+
+    def fake_get(self, key):
+        if key not in self.graphs:
+            captured.append(key)
+            self.graphs[key] = _FakeGraph()
+        return self.graphs[key]
+
+    monkeypatch.setattr(bench.GraphSet, "_get", fake_get)
+    for G, period, warm, steps in ((64, 64, 5, 20), (64, 64, 64, 4096), (16, 16, 3, 37), (4, 16, 4, 64)):
+        gs = bench.GraphSet(G, lambda i: None, period=period)
+        pos = gs.run(warm)
+        gs.prepare(steps, pos)
+        before = list(captured)
+        end = gs.run(steps, pos)
+        assert captured == before, (G, warm, steps)
+        assert end == warm + steps
+        assert sum(n for n, _ in gs.keys(steps, pos)) == steps
+        captured.clear()
+
+
+def test_graph_keys_follow_the_step_phase():
+    gs = bench.GraphSet(64, lambda i: None)
+    assert gs.keys(20, 5) == [(20, 5)]
+    assert gs.keys(130, 5) == [(64, 5), (64, 5), (2, 5)]
+    gs = bench.GraphSet(4, lambda i: None, period=16)
+    assert gs.keys(10, 14) == [(4, 14), (4, 2), (2, 6)]

@@ -80,3 +80,13 @@ def test_tc_prefill_full_size_sampled(E, orc):
     idx = E.workspace_view(ly, wl.T, "idx").cpu().numpy().reshape(wl.T, -1)
     assert np.array_equal(idx[sample], ref["idx"])
     assert np.array_equal(y[sample], ref["y"])
+
+
+def test_int8_rate_kernel_runs(E):
+    """The measurement kernel behind the int8 peak: no wait runs out, and every
+    CTA's accumulator word is the same nonzero value (same operands)."""
+    sink, err = E.test_mma_i8_rate(64)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    s = sink.cpu()
+    assert (s == s[0]).all() and int(s[0]) != 0

@@ -78,6 +78,22 @@ def _ulp32(x):
     return 2.0 ** (math.floor(math.log2(x)) - 23)
 
 
+def test_bf16_to_f32_matches_torch(orc):
+    """Every bf16 bit pattern widens to the fp32 torch's bfloat16 conversion
+    gives (NaNs: a NaN), plus values fixed by the format: 0x3F80 = 1.0,
+    0xC000 = -2.0, 0x7F80 = +inf, 0x0001 = 2^-133 (the smallest subnormal)."""
+    import torch
+    bits = np.arange(65536, dtype=np.uint16)
+    ref = torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).float().numpy()
+    got = np.array([orc.lib().orc_bf16_to_f32(int(b)) for b in bits], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    f = orc.lib().orc_bf16_to_f32
+    assert f(0x3F80) == 1.0 and f(0xC000) == -2.0 and f(0x7F80) == math.inf
+    assert f(0x0001) == 2.0 ** -133
+
+
 def test_expf_within_two_ulp_of_fp64(orc):
     r = _rng(1)
     xs = np.concatenate([np.linspace(-20, 20, 4001), r.uniform(-87, 88, 3000),
