@@ -11,6 +11,7 @@
 
 #include "../../include/elq.h"
 #include "elq_decode.cuh"
+#include "elq_sgemv.cuh"
 #include "elq_tc.cuh"
 
 using namespace elq;
@@ -213,6 +214,163 @@ WArgs dense_w(const elq_qmat* w, int T, const void* x, int x_mode, int64_t x_row
 }
 
 // ---------------------------------------------------------------------------
+// Small-T cluster GEMV planning (k_sgemv)
+
+struct SPlan {
+    bool ok;
+    int C, Cg, cpc, stages, stage_bytes, act_off, act_bytes, scratch_bytes, pbuf_off, route_off, smem, clusters;
+    int nchunks, ipg;
+};
+
+constexpr int kSSmemMax = 227 * 1024;
+
+// rows_per_group: matrix rows of one group; K: reduction length; groups_max:
+// bound on the groups; routed: an expert projection (a group table in shared
+// memory).
+SPlan plan_s(int fmt, int x_mode, bool swiglu, int rows_per_group, int K, int groups_max, int T, bool routed) {
+    SPlan p;
+    std::memset(&p, 0, sizeof(p));
+    if (T < 1 || T > kSMaxT || groups_max < 1 || groups_max > kSMaxPairs) return p;
+    const int nb = K / 32;
+    p.nchunks = (nb + kChunk - 1) / kChunk;
+    p.ipg = swiglu ? rows_per_group / 64 : rows_per_group / 32;
+    const int64_t n_items = (int64_t)groups_max * p.ipg;
+    const int sms = sm_count();
+    const int halves = swiglu ? 2 : 1;
+    // split an item's chunks over Cg CTAs until there are CTAs for every SM
+    // (and at most 16 chunks, one per warp, per CTA)
+    int Cg = 1;
+    while (Cg < p.nchunks && halves * Cg * 2 <= kSMaxCluster &&
+           ((p.nchunks + Cg - 1) / Cg > kSMaxWarps || n_items * halves * Cg < sms))
+        Cg *= 2;
+    if ((p.nchunks + Cg - 1) / Cg > kSMaxWarps) return p;
+    p.Cg = Cg;
+    p.C = Cg * halves;
+    p.cpc = (p.nchunks + Cg - 1) / Cg;
+    const int codes = kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
+    p.act_off = codes + kChunk * 64;
+    p.act_bytes = x_mode == X_RAW_F32 ? 1024 : x_mode == X_RAW_BF16 ? 512 : kChunk * 36;
+    p.stage_bytes = (int)round_up((size_t)p.act_off + (size_t)T * p.act_bytes, 128);
+    p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)T * kChunk * 36, 128) : 0;
+    const int pbuf = 2 * halves * p.nchunks * T * 128;
+    const int route = routed ? (int)round_up((size_t)kSRouteBytes, 128) : 0;
+    auto smem_for = [&](int st) { return kSHeader + p.cpc * (st * p.stage_bytes + p.scratch_bytes) + pbuf + route; };
+    // resident CTAs per SM: shared memory (1 KB reserved per CTA), warps, and
+    // registers at the launch bound's 64 per thread
+    auto per_sm = [&](int smem) {
+        const int a = (228 * 1024) / (smem + 1024);
+        const int b = 32 / p.cpc, c = 64 / p.cpc;
+        return std::max(0, std::min(std::min(a, b), std::min(c, 32)));
+    };
+    auto clusters_for = [&](int st) {
+        const int64_t cap = std::max<int64_t>(1, (int64_t)per_sm(smem_for(st)) * sms / p.C);
+        return (int)std::min<int64_t>(n_items, cap);
+    };
+    if (smem_for(1) > kSSmemMax) return p;
+    // rounds of items per cluster: one stage exposes the latency of each
+    // round (later rounds' weights come from L2, prefetched at the start),
+    // two stages hide every other round but fit fewer CTAs
+    const int64_t r1 = (n_items + clusters_for(1) - 1) / clusters_for(1);
+    p.stages = 1;
+    if (smem_for(2) <= kSSmemMax) {
+        const int64_t r2 = (n_items + clusters_for(2) - 1) / clusters_for(2);
+        if (r2 + 1 < 2 * r1) p.stages = 2;
+    }
+    p.clusters = clusters_for(p.stages);
+    p.pbuf_off = kSHeader + p.cpc * (p.stages * p.stage_bytes + p.scratch_bytes);
+    p.route_off = p.pbuf_off + pbuf;
+    p.smem = smem_for(p.stages);
+    p.ok = true;
+    return p;
+}
+
+template <int FMT, int XM, int OM>
+cudaError_t launch_s_t(const SArgs& g, const SPlan& p, cudaStream_t s, bool pdl) {
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_sgemv<FMT, XM, OM>, kSSmemMax, optin);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(p.clusters * p.C));
+    cfg.blockDim = dim3((unsigned)(32 * p.cpc));
+    cfg.dynamicSmemBytes = (size_t)p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (p.C > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)p.C;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, k_sgemv<FMT, XM, OM>, g);
+}
+
+template <int FMT>
+cudaError_t launch_s_f(const SArgs& g, int x_mode, int out_mode, const SPlan& p, cudaStream_t s, bool pdl) {
+    switch (x_mode * 16 + out_mode) {
+    case X_RAW_BF16 * 16 + OUT_F32_Q81: return launch_s_t<FMT, X_RAW_BF16, OUT_F32_Q81>(g, p, s, pdl);
+    case X_RAW_F32 * 16 + OUT_F32_Q81: return launch_s_t<FMT, X_RAW_F32, OUT_F32_Q81>(g, p, s, pdl);
+    case X_Q81_TOKEN * 16 + OUT_F32: return launch_s_t<FMT, X_Q81_TOKEN, OUT_F32>(g, p, s, pdl);
+    case X_Q81_TOKEN * 16 + OUT_F32_ADD: return launch_s_t<FMT, X_Q81_TOKEN, OUT_F32_ADD>(g, p, s, pdl);
+    case X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU: return launch_s_t<FMT, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl);
+    case X_Q81_POSITION * 16 + OUT_F32_COMBINE: return launch_s_t<FMT, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_s(SArgs g, int fmt, int x_mode, int out_mode, const SPlan& p, cudaStream_t s, bool pdl) {
+    if (!p.ok) return cudaErrorInvalidConfiguration;
+    g.nchunks = p.nchunks;
+    g.items_per_group = p.ipg;
+    g.C = p.C;
+    g.Cg = p.Cg;
+    g.cpc = p.cpc;
+    g.stages = p.stages;
+    g.stage_bytes = p.stage_bytes;
+    g.act_off = p.act_off;
+    g.act_bytes = p.act_bytes;
+    g.scratch_bytes = p.scratch_bytes;
+    g.pbuf_off = p.pbuf_off;
+    g.route_off = p.route_off;
+    g.budget_ns = kWaitBudgetNs;
+    const int64_t ctas = (int64_t)p.clusters * p.C;
+    for (int r = 0; r < 3; ++r)
+        g.pf_share[r] = g.pf[r] ? (int64_t)round_up((size_t)((g.pf_bytes[r] + ctas - 1) / ctas), 256) : 0;
+    return fmt == ELQ_Q8_0 ? launch_s_f<8>(g, x_mode, out_mode, p, s, pdl) : launch_s_f<2>(g, x_mode, out_mode, p, s, pdl);
+}
+
+// A dense projection of T <= 8 tokens on k_sgemv.
+SArgs dense_s(const elq_qmat* w, int T, const void* x, int64_t x_row, float* y, uint8_t* yq, int* err) {
+    SArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.q = static_cast<const uint8_t*>(w->q);
+    g.d = static_cast<const uint16_t*>(w->d);
+    g.nb = w->k / 32;
+    g.groups_max = 1;
+    g.route = ROUTE_NONE;
+    g.T = T;
+    g.k = 1;
+    g.x = x;
+    g.x_row = x_row;
+    g.y = y;
+    g.y_ld = w->n_rows;
+    g.yq = yq;
+    g.yq_ld = w->n_rows / 32;
+    g.err = err;
+    g.early = 1;
+    return g;
+}
+
+// ---------------------------------------------------------------------------
 // Workspace layouts
 
 struct Carve {
@@ -396,6 +554,11 @@ struct LayerWs {
     int* cnt_comb_tc;
     WPlan pd, pgu, pdn, pu;
     bool raw;
+    // small-T path: cluster router (k_route_small) and cluster GEMV (k_sgemv)
+    bool small;
+    SPlan sd, sgu, sdn, su;
+    int rs_C, rs_epc;
+    int32_t* gtok;          // [groups][8] tokens of each routed group's pairs
     size_t total;
 };
 
@@ -414,9 +577,21 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     w.dec = plan_dec(ly, T);
     w.fused = !w.tc && w.dec.ok;
+    w.small = false;
+    w.rs_C = 1;
+    while ((E + w.rs_C - 1) / w.rs_C > 8 && w.rs_C < kSMaxCluster) w.rs_C *= 2;
+    w.rs_epc = (E + w.rs_C - 1) / w.rs_C;
+    if (!w.tc && !w.fused && w.raw && P <= kSMaxPairs && w.rs_epc <= kSMaxWarps &&
+        rs_smem_bytes(T, L, E) + 16 <= kSSmemMax) {
+        w.sd = plan_s(ly->D.fmt, dmode, false, L, H, 1, T, false);
+        w.sgu = plan_s(ly->gate_up.fmt, X_Q81_PAIR_TOKEN, true, 2 * I, L, gmax, T, true);
+        w.sdn = plan_s(ly->down.fmt, X_Q81_POSITION, false, L, I, gmax, T, true);
+        w.su = plan_s(ly->U.fmt, X_Q81_TOKEN, false, H, L, 1, T, false);
+        w.small = w.sd.ok && w.sgu.ok && w.sdn.ok && w.su.ok;
+    }
     const size_t n_sync = w.fused ? (size_t)dec_sync_ints(T, L, I) : 0;
     const size_t n_cnt = 64 + (rblocks + 1) + w.pd.counter_ints + w.pgu.counter_ints + w.pdn.counter_ints +
-                         w.pu.counter_ints + (size_t)T * (L / kTileRows) + n_sync;
+                         w.pu.counter_ints + (size_t)T * (L / 32) + n_sync;
     Carve c;
     w.err = c.take<int>(base, n_cnt * sizeof(int));
     int* cur = w.err ? w.err + 64 : nullptr;
@@ -426,7 +601,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.cnt_gu = adv(w.pgu.counter_ints);
     w.cnt_dn = adv(w.pdn.counter_ints);
     w.cnt_u = adv(w.pu.counter_ints);
-    w.cnt_comb = adv((size_t)T * (L / kTileRows));
+    w.cnt_comb = adv((size_t)T * (L / 32));     // per (token, 32-row block): covers the per-tile use too
     w.sync = w.fused ? adv(n_sync) : nullptr;
     w.xq = w.raw ? nullptr : c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
     w.z = c.take<float>(base, (size_t)T * L * 4);
@@ -447,7 +622,12 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.tstride = round16(T);
     w.sstride = round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
     w.grp = nullptr;
+    w.gtok = nullptr;
     w.part_d = nullptr;
+    if (w.small) {
+        w.grp = c.take<int4>(base, (size_t)gmax * sizeof(int4));
+        w.gtok = c.take<int32_t>(base, (size_t)gmax * kSMaxT * 4);
+    }
     if (w.fused) {
         w.grp = c.take<int4>(base, (size_t)E * sizeof(int4));
         // D's chunk partials; the region also serves the separate-kernel
@@ -593,6 +773,97 @@ WArgs down_args(const elq_layer* ly, const LayerWs& w, int T, const float* wts, 
     h.wts = wts; h.pos = w.pos; h.cnt_comb = w.cnt_comb; h.ylat = y_lat; h.ylq = w.ylq;
     h.partial = partial; h.part_tok = (int64_t)T * k; h.counters = w.cnt_dn; h.err = w.err;
     return h;
+}
+
+// The expert projections on k_sgemv.  route: ROUTE_GROUPS (the layer call:
+// the group table k_route_small wrote) or ROUTE_ARRAYS (the bucketed arrays
+// in the workspace; wts the caller's).
+SArgs gate_up_s(const elq_layer* ly, const LayerWs& w, int T, int route, const uint8_t* zq) {
+    const int L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    SArgs g;
+    std::memset(&g, 0, sizeof(g));
+    g.q = static_cast<const uint8_t*>(ly->gate_up.q);
+    g.d = static_cast<const uint16_t*>(ly->gate_up.d);
+    g.nb = L / 32;
+    g.q_gstride = (int64_t)(2 * I / kTileRows) * g.nb * slab_bytes(ly->gate_up.fmt);
+    g.d_gstride = (int64_t)(2 * I / kTileRows) * g.nb * kTileRows;
+    g.groups_max = (int)std::min<int64_t>(E, (int64_t)T * k);
+    g.route = route;
+    g.T = T; g.E = E; g.k = k;
+    g.act = w.act; g.n_act = w.n_act; g.offsets = w.offsets; g.perm = w.perm; g.pos = w.pos;
+    g.grp = w.grp; g.gtok = w.gtok;
+    g.x = zq;
+    g.yq = w.hq; g.yq_ld = I / 32;
+    // the routed experts' down matrices, for the next kernel
+    g.pfe_q = static_cast<const uint8_t*>(ly->down.q);
+    g.pfe_d = reinterpret_cast<const uint8_t*>(ly->down.d);
+    g.pfe_qs = (int64_t)(L / kTileRows) * (I / 32) * slab_bytes(ly->down.fmt);
+    g.pfe_ds = (int64_t)(L / kTileRows) * (I / 32) * kScaleSlab;
+    g.L = L;
+    g.err = w.err;
+    g.early = 0;
+    return g;
+}
+
+SArgs down_s(const elq_layer* ly, const LayerWs& w, int T, int route, const float* wts, float* y_lat) {
+    const int L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    SArgs h;
+    std::memset(&h, 0, sizeof(h));
+    h.q = static_cast<const uint8_t*>(ly->down.q);
+    h.d = static_cast<const uint16_t*>(ly->down.d);
+    h.nb = I / 32;
+    h.q_gstride = (int64_t)(L / kTileRows) * h.nb * slab_bytes(ly->down.fmt);
+    h.d_gstride = (int64_t)(L / kTileRows) * h.nb * kTileRows;
+    h.groups_max = (int)std::min<int64_t>(E, (int64_t)T * k);
+    h.route = route;
+    h.T = T; h.E = E; h.k = k;
+    h.act = w.act; h.n_act = w.n_act; h.offsets = w.offsets; h.perm = w.perm; h.pos = w.pos;
+    h.grp = w.grp; h.gtok = w.gtok;
+    h.wts = wts;
+    h.x = w.hq;
+    h.y = w.o; h.y_ld = L;
+    h.cnt_comb = w.cnt_comb; h.ylat = y_lat; h.ylq = w.ylq; h.L = L;
+    h.err = w.err;
+    // the routing is complete before this kernel's upstream (gate/up) starts
+    h.early = 1;
+    return h;
+}
+
+// The small-T cluster router: one cluster of rs_C CTAs of rs_epc warps.
+cudaError_t launch_route_small(const elq_layer* ly, const LayerWs& w, int T, cudaStream_t s, bool pdl) {
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_route_small, kSSmemMax, optin);
+    if (e != cudaSuccess) return e;
+    RSArgs r;
+    std::memset(&r, 0, sizeof(r));
+    r.z = w.z; r.w = ly->router_w; r.bias = ly->router_bias;
+    r.T = T; r.L = ly->L; r.E = ly->E; r.k = ly->k; r.C = w.rs_C; r.epc = w.rs_epc;
+    r.logits = w.logits; r.idx = w.idx; r.wts = w.wts;
+    r.counts = w.counts; r.offsets = w.offsets; r.perm = w.perm; r.pos = w.pos; r.act = w.act; r.n_act = w.n_act;
+    r.grp = w.grp; r.gtok = w.gtok;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)w.rs_C);
+    cfg.blockDim = dim3((unsigned)(32 * w.rs_epc));
+    cfg.dynamicSmemBytes = (size_t)rs_smem_bytes(T, ly->L, ly->E) + 16;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (w.rs_C > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)w.rs_C;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, k_route_small, r);
 }
 
 // Kernel sequence of the grouped experts (gate/up, then down with the combine)
@@ -920,6 +1191,12 @@ elq_status elq_latent_proj(const elq_qmat* w, const void* x_q8_1, int32_t T, flo
         TcArgs g = dense_tc(w, T, lay.bq, lay.bd, lay.bstride, TC_OUT_F32, y, nullptr, lay.err);
         return cuda_status(launch_tc(g, s, true));
     }
+    if (T <= kSMaxT) {
+        const SPlan sp = plan_s(w->fmt, X_Q81_TOKEN, false, w->n_rows, w->k, 1, T, false);
+        if (sp.ok)
+            return cuda_status(launch_s(dense_s(w, T, x_q8_1, 0, y, nullptr, lay.err), w->fmt, X_Q81_TOKEN, OUT_F32,
+                                        sp, s, false));
+    }
     WArgs g = dense_w(w, T, x_q8_1, X_Q81_TOKEN, 0, OUT_F32, y, nullptr, lay.partial, lay.counters, lay.err);
     return cuda_status(launch_w(g, w->fmt, lay.plan, s, false));
 }
@@ -951,6 +1228,18 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, s, false, idx, (int)P, E, w.counts, w.offsets,
                w.perm, w.pos, w.act, w.n_act);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    if (!w.tc && T <= kSMaxT && P <= kSMaxPairs) {
+        const int gmax = (int)std::min<int64_t>(E, P);
+        const SPlan pgu = plan_s(layer->gate_up.fmt, X_Q81_PAIR_TOKEN, true, 2 * layer->I, layer->L, gmax, T, true);
+        const SPlan pdn = plan_s(layer->down.fmt, X_Q81_POSITION, false, layer->L, layer->I, gmax, T, true);
+        if (pgu.ok && pdn.ok) {
+            if (launch_s(gate_up_s(layer, w, T, ROUTE_ARRAYS, static_cast<const uint8_t*>(z_q8_1)),
+                         layer->gate_up.fmt, X_Q81_PAIR_TOKEN, OUT_SWIGLU, pgu, s, true) != cudaSuccess)
+                return ELQ_ERR_CUDA;
+            return cuda_status(launch_s(down_s(layer, w, T, ROUTE_ARRAYS, weights, y_lat), layer->down.fmt,
+                                        X_Q81_POSITION, OUT_F32_COMBINE, pdn, s, true));
+        }
+    }
     if (w.tc) {
         // the slot map reads idx from the workspace copy the layer call would have
         if (cudaMemcpyAsync(w.idx, idx, (size_t)P * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return ELQ_ERR_CUDA;
@@ -1245,6 +1534,37 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, residual ? TC_OUT_F32_ADD : TC_OUT_F32, y,
                              nullptr, w.err);
         if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        return ELQ_OK;
+    }
+    if (w.small) {
+        // a1 + a2 + a4: D (x quantised in the kernel; z, zq), asking L2 for
+        // the router rows and U, which later kernels of the layer read
+        const int dmode = x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32;
+        SArgs gd = dense_s(&layer->D, T, x, H, w.z, w.zq, w.err);
+        gd.pf[0] = reinterpret_cast<const uint8_t*>(layer->router_w);
+        gd.pf_bytes[0] = (int64_t)E * L * 4;
+        gd.pf[1] = static_cast<const uint8_t*>(layer->U.q);
+        gd.pf_bytes[1] = (int64_t)(H / kTileRows) * (L / 32) * slab_bytes(layer->U.fmt);
+        gd.pf[2] = static_cast<const uint8_t*>(layer->U.d);
+        gd.pf_bytes[2] = (int64_t)(H / kTileRows) * (L / 32) * kScaleSlab;
+        if (launch_s(gd, layer->D.fmt, dmode, OUT_F32_Q81, w.sd, s, pdl) != cudaSuccess || !mark())
+            return ELQ_ERR_CUDA;
+        // a3 + a5: the cluster router (logits, top-k, softmax, bucketing, group table)
+        if (launch_route_small(layer, w, T, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        // a6 + a7, then a8 + a9
+        if (launch_s(gate_up_s(layer, w, T, ROUTE_GROUPS, w.zq), layer->gate_up.fmt, X_Q81_PAIR_TOKEN, OUT_SWIGLU,
+                     w.sgu, s, pdl) != cudaSuccess ||
+            !mark())
+            return ELQ_ERR_CUDA;
+        if (launch_s(down_s(layer, w, T, ROUTE_GROUPS, w.wts, w.ylat), layer->down.fmt, X_Q81_POSITION,
+                     OUT_F32_COMBINE, w.sdn, s, pdl) != cudaSuccess ||
+            !mark())
+            return ELQ_ERR_CUDA;
+        // a10
+        SArgs gu = dense_s(&layer->U, T, w.ylq, 0, y, nullptr, w.err);
+        if (launch_s(gu, layer->U.fmt, X_Q81_TOKEN, residual ? OUT_F32_ADD : OUT_F32, w.su, s, pdl) != cudaSuccess ||
+            !mark())
+            return ELQ_ERR_CUDA;
         return ELQ_OK;
     }
     // a1 + a2 + a4: D projection of x (quantised by the GEMV itself at small T)

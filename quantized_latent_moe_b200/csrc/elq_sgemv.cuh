@@ -1,0 +1,727 @@
+// elq_sgemv.cuh -- grouped quantised GEMV for small token counts (T <= 8,
+// T * k <= 64) with the split-K reduction inside a thread-block cluster.
+//
+// Work item: one 32-row slice of a group (the dense matrix, or one routed
+// expert) over all of K -- or, for the gate/up projection, the gate slice and
+// the up slice whose rows meet in one SwiGLU block.  A cluster of C CTAs
+// takes an item; each CTA takes a contiguous run of the item's 8-block chunks,
+// one chunk per warp.  A warp bulk-copies its chunk's codes and scales (one
+// 8 KB / 4 KB contiguous piece of the arena plus 512 B) and its tokens'
+// activation slices into its shared-memory stage, computes the chunk partial
+// of each token (dp4a, then the chunk's ordered fused multiply-adds), and
+// stores it into the partial buffer of the cluster's first CTA through
+// distributed shared memory.  One cluster barrier later that CTA adds the
+// chunk partials in chunk order and runs the epilogue.  No partial sum goes
+// through global memory and no global counter is taken, except by the down
+// projection's weighted combine, whose k pairs come from different items.
+//
+// Clusters are persistent: cluster i takes items i, i + n, i + 2n, ... and
+// each warp keeps up to two items' copies in flight.  Weights that do not
+// depend on the upstream kernel are requested before the grid dependency
+// wait.  Each CTA also asks L2 to prefetch its share of weights a later
+// kernel of the layer reads (the router rows and U during D; the routed
+// experts' down matrices during gate/up), so that those kernels find them in
+// L2.
+//
+// Routing.  k_route_small (one cluster) computes the router logits, gathers
+// them in its first CTA through distributed shared memory, and there takes
+// the top-k, the softmax and the bucketing of the T * k <= 64 pairs, writing
+// the routing arrays and a table of the routed groups (expert, first pair
+// position, pairs, and each pair's token).  The expert kernels read that
+// table (or build it from the bucketed arrays of the grouped-experts call)
+// into shared memory once per CTA.
+#pragma once
+
+#include "elq_kernels.cuh"
+
+namespace elq {
+
+constexpr int kSMaxT = 8;            // tokens of a dense group / pairs of an expert group
+constexpr int kSMaxPairs = 64;       // T * k
+constexpr int kSMaxWarps = 16;
+constexpr int kSMaxCluster = 8;
+constexpr int kSHeader = 512;        // mbarriers [warps][2] and the routing scalars
+
+enum { ROUTE_NONE = 0, ROUTE_ARRAYS = 1, ROUTE_GROUPS = 2 };
+
+// ---- cluster primitives --------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The shared-memory address in CTA `rank` of this cluster that corresponds to
+// the local shared-memory address `a`.
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void dsmem_st(uint32_t a, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+// Every thread of every CTA of the cluster: arrive (release), then wait (acquire).
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+struct SArgs {
+    // weights: codes of slice s of tile t, blocks 8c .. 8c+7, of group e at
+    // q + e*q_gstride + ((t*nb*4) + s*nb + 8c) * codes-per-block-slice
+    const uint8_t* q;
+    const uint16_t* d;
+    int64_t q_gstride, d_gstride;
+    int nb, nchunks;
+    int items_per_group;     // slices (or slice pairs, SwiGLU) per group
+    int groups_max;          // bound on the groups (dense: 1)
+    int C, Cg, cpc, stages;  // cluster size, CTAs per slice, chunks (= warps) per CTA, ring depth
+    int stage_bytes, act_off, act_bytes, scratch_bytes, pbuf_off, route_off;
+    // routing
+    int route;
+    int T, E, k;
+    const int32_t *act, *n_act, *offsets, *perm, *pos;   // ROUTE_ARRAYS
+    const int4* grp;                             // ROUTE_GROUPS: per group (expert, first position, pairs, 0)
+    const int32_t* gtok;                         // ROUTE_GROUPS: [group][8] token of each pair
+    const float* wts;                            // combine weights [T][k]
+    // activations
+    const void* x;
+    int64_t x_row;                               // raw inputs: elements per row
+    // outputs
+    float* y;
+    int64_t y_ld;
+    uint8_t* yq;
+    int64_t yq_ld;
+    int* cnt_comb;                               // [T][L/32], zero on entry and exit
+    float* ylat;
+    uint8_t* ylq;
+    int L;
+    // L2 prefetch: up to three fixed ranges, and one per-expert pair of ranges
+    const uint8_t* pf[3];
+    int64_t pf_bytes[3];
+    int64_t pf_share[3];                         // bytes per CTA (a multiple of 256)
+    const uint8_t* pfe_q;
+    const uint8_t* pfe_d;
+    int64_t pfe_qs, pfe_ds;                      // bytes per expert (multiples of 256)
+    int* err;
+    uint64_t budget_ns;
+    int early;               // weights and routing do not depend on the upstream grid
+};
+
+// Shared-memory table of the routed groups (expert modes): the count, then
+// per group (expert, first pair position, pairs, 0) and the token of each of
+// its pairs (a group holds at most one pair per token, so at most kSMaxT).
+constexpr int kSRouteBytes = 16 + kSMaxPairs * 16 + kSMaxPairs * kSMaxT * 4;
+
+__device__ __forceinline__ int* sr_nact(uint8_t* rs) { return reinterpret_cast<int*>(rs); }
+__device__ __forceinline__ int4* sr_grp(uint8_t* rs) { return reinterpret_cast<int4*>(rs + 16); }
+__device__ __forceinline__ int32_t* sr_tok(uint8_t* rs) { return reinterpret_cast<int32_t*>(rs + 16 + kSMaxPairs * 16); }
+
+// Prefetch into L2 the part [lo, hi) of a byte range (lo, hi multiples of 16).
+__device__ __forceinline__ void l2_prefetch_range(const uint8_t* base, int64_t lo, int64_t hi) {
+    for (int64_t p = lo; p < hi; p += 65536) {
+        const int64_t rem = hi - p;
+        const uint32_t n = (uint32_t)(rem < 65536 ? rem : 65536);
+        bulk_prefetch_l2(base + p, n);
+    }
+}
+
+// This CTA's share of n bytes when every CTA of the grid takes `share`
+// consecutive bytes (share: a multiple of 256, fixed by the host).
+__device__ __forceinline__ void share_of(int64_t n, int64_t share, int64_t& lo, int64_t& hi) {
+    lo = (int64_t)blockIdx.x * share;
+    hi = lo + share < n ? lo + share : n;
+}
+
+// Fills the group table from global memory (all threads; ends with a
+// CTA barrier).  ROUTE_GROUPS: the router's table; ROUTE_ARRAYS: built from
+// the bucketed arrays (act, offsets, perm).
+__device__ void s_load_groups(const SArgs& g, uint8_t* rs) {
+    if (g.route == ROUTE_GROUPS) {
+        const int na = __ldcg(g.n_act);
+        for (int i = threadIdx.x; i < na; i += blockDim.x) sr_grp(rs)[i] = __ldcg(g.grp + i);
+        for (int i = threadIdx.x; i < na * kSMaxT; i += blockDim.x) sr_tok(rs)[i] = __ldcg(g.gtok + i);
+        if (threadIdx.x == 0) *sr_nact(rs) = na;
+    } else {
+        const int na = __ldcg(g.n_act);
+        for (int a = threadIdx.x; a < na; a += blockDim.x) {
+            const int e = __ldcg(g.act + a);
+            const int o0 = __ldcg(g.offsets + e);
+            const int n = __ldcg(g.offsets + e + 1) - o0;
+            sr_grp(rs)[a] = make_int4(e, o0, n, 0);
+            for (int i = 0; i < n && i < kSMaxT; ++i) sr_tok(rs)[a * kSMaxT + i] = __ldcg(g.perm + o0 + i) / g.k;
+        }
+        if (threadIdx.x == 0) *sr_nact(rs) = na;
+    }
+    __syncthreads();
+}
+
+// Group a: (expert, first pair position, pairs); dense: (0, 0, T).
+__device__ __forceinline__ int4 sgroup(const SArgs& g, const uint8_t* rs, int a) {
+    if (g.route == ROUTE_NONE) return make_int4(0, 0, g.T, 0);
+    return reinterpret_cast<const int4*>(rs + 16)[a];
+}
+
+__device__ __forceinline__ int s_n_groups(const SArgs& g, const uint8_t* rs) {
+    return g.route == ROUTE_NONE ? 1 : *reinterpret_cast<const int*>(rs);
+}
+
+// Token of pair i of group a.
+__device__ __forceinline__ int s_tok(const uint8_t* rs, int a, int i) {
+    return reinterpret_cast<const int32_t*>(rs + 16 + kSMaxPairs * 16)[a * kSMaxT + i];
+}
+
+// The unit of this warp in item `item`: slice, chunk and group.
+struct SUnit {
+    int a, tile, s, hb, c, kbn;
+    int4 grp;                // expert, first position, pairs
+    bool has;                // this warp has a chunk of the item
+};
+
+template <int OM>
+__device__ __forceinline__ SUnit s_unit(const SArgs& g, const uint8_t* rs, int item, int rank, int warp) {
+    SUnit u;
+    u.a = item / g.items_per_group;
+    const int ip = item - u.a * g.items_per_group;
+    if (OM == OUT_SWIGLU) {
+        u.tile = ip >> 1;
+        u.hb = ip & 1;
+        u.s = (rank / g.Cg) * 2 + u.hb;
+    } else {
+        u.tile = ip >> 2;
+        u.s = ip & 3;
+        u.hb = 0;
+    }
+    u.c = (rank % g.Cg) * g.cpc + warp;
+    u.has = warp < g.cpc && u.c < g.nchunks;
+    u.kbn = u.has ? min(kChunk, g.nb - u.c * kChunk) : 0;
+    u.grp = sgroup(g, rs, u.a);
+    return u;
+}
+
+template <int XM>
+__device__ __forceinline__ uint32_t s_act_bytes(int kbn) {
+    if (XM == X_RAW_F32) return (uint32_t)kbn * 128u;
+    if (XM == X_RAW_BF16) return (uint32_t)kbn * 64u;
+    return (uint32_t)kbn * 36u;
+}
+
+template <int FMT, int XM>
+__device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, uint8_t* stg, uint64_t* bar) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    const uint32_t cb = (uint32_t)(u.kbn * SL::kCodes), sb = (uint32_t)(u.kbn * 64);
+    if (lane == 0) mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * s_act_bytes<XM>(u.kbn));
+    __syncwarp();
+    if (lane == 0) {
+        const uint8_t* src = g.q + u.grp.x * g.q_gstride +
+                             ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + (int64_t)u.c * kChunk) * SL::kCodes;
+        bulk_g2s(stg, src, cb, bar);
+    } else if (lane == 1) {
+        const uint16_t* src = g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows +
+                              (int64_t)u.s * g.nb * 32 + (int64_t)u.c * kChunk * 32;
+        bulk_g2s(stg + kChunk * SL::kCodes, src, sb, bar);
+    }
+}
+
+template <int XM>
+__device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, const SUnit& u, uint8_t* act,
+                                             uint64_t* bar) {
+    const int lane = threadIdx.x & 31;
+    if (lane < u.grp.z) {
+        int64_t row;
+        if (XM == X_Q81_PAIR_TOKEN) row = s_tok(rs, u.a, lane);
+        else if (XM == X_Q81_POSITION) row = u.grp.y + lane;
+        else row = lane;
+        const uint8_t* src;
+        if (XM == X_RAW_F32)
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)u.c * 256) * 4;
+        else if (XM == X_RAW_BF16)
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)u.c * 256) * 2;
+        else
+            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + (int64_t)u.c * kChunk) * 36;
+        bulk_g2s(act + lane * g.act_bytes, src, s_act_bytes<XM>(u.kbn), bar);
+    }
+}
+
+// Q8_1 of one token's chunk of raw activations (kbn blocks of 32 values at
+// src, fp32 or bf16) into kbn 36-byte blocks at dst, all blocks at once:
+// lane l takes values 8 (l % 4) .. +7 of block l / 4.  Same arithmetic as
+// the one-block warp quantiser: amax, d = amax / 127, q = clamp(round(x /
+// d)), s = fp16(d * sum q).  The loops stay rolled: a short body keeps the
+// code a warp runs once small (these kernels are bound by its fetch).
+template <bool BF16>
+__device__ __forceinline__ float raw_at(const uint8_t* src, int i) {
+    return BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(src)[i])
+                : reinterpret_cast<const float*>(src)[i];
+}
+
+template <bool BF16>
+__device__ __noinline__ void warp_quant_chunk(const uint8_t* src, int kbn, uint8_t* dst) {
+    const int lane = threadIdx.x & 31;
+    const int b = lane >> 2, qd = lane & 3;
+    const bool on = b < kbn;
+    const int i0 = b * 32 + qd * 8;
+    float amax = 0.0f;
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, on ? fabsf(raw_at<BF16>(src, i0 + i)) : 0.0f);
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const float d = __fdiv_rn(amax, 127.0f);
+    uint32_t w0 = 0, w1 = 0;
+    int sum = 0;
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        int q = 0;
+        if (on && d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(raw_at<BF16>(src, i0 + i), d)), -127.0f), 127.0f);
+        sum += q;
+        const uint32_t bq = (uint32_t)(q & 0xff) << (8 * (i & 3));
+        if (i < 4) w0 |= bq; else w1 |= bq;
+    }
+    sum += __shfl_xor_sync(kFull, sum, 1);
+    sum += __shfl_xor_sync(kFull, sum, 2);
+    if (on) {
+        uint32_t* o = reinterpret_cast<uint32_t*>(dst + b * 36 + 4 + qd * 8);
+        o[0] = w0;
+        o[1] = w1;
+        if (qd == 0) {
+            const uint32_t dh = f2h(d);
+            const uint32_t sh = f2h(__fmul_rn(d, (float)sum));
+            *reinterpret_cast<uint32_t*>(dst + b * 36) = dh | (sh << 16);
+        }
+    }
+}
+
+// Block kb of this lane's row from the stage: signed 8-bit codes in w[0..7]
+// (codes 4j .. 4j+3 in w[j]) and the scale.
+template <int FMT>
+__device__ __forceinline__ void s_block(const uint8_t* stg, int kb, int (&w)[8], float& dw) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    dw = h2f(reinterpret_cast<const uint16_t*>(stg + kChunk * SL::kCodes)[kb * 32 + lane]);
+    if (FMT == 8) {
+        const uint8_t* cp = stg + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
+        const uint4 a = lds128(cp), b = lds128(cp + 128);
+        w[0] = (int)a.x; w[1] = (int)a.y; w[2] = (int)a.z; w[3] = (int)a.w;
+        w[4] = (int)b.x; w[5] = (int)b.y; w[6] = (int)b.z; w[7] = (int)b.w;
+    } else {
+        const uint4 a = lds128(stg + kb * 512 + lane * 16);
+        const uint32_t v[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            // nibbles q (0..15) -> signed bytes q - 8, without borrows between bytes
+            const uint32_t lo = v[j] & 0x0F0F0F0Fu, hi = (v[j] >> 4) & 0x0F0F0F0Fu;
+            w[j] = (int)(((lo | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
+            w[4 + j] = (int)(((hi | 0x80808080u) - 0x08080808u) ^ 0x80808080u);
+        }
+    }
+}
+
+// Chunk partials of the unit's tokens into the first CTA's partial buffer:
+// token t's value of this lane's row goes to the shared-memory address
+// `dst + (t * 32 + lane) * 4` of that CTA.  For each token the blocks are
+// taken in order (part = fmaf(isum, d_w * d_a, part)), the block's codes read
+// again from the stage per token.  Raw activations are first quantised to
+// Q8_1 in the warp's scratch.
+template <int FMT, int XM>
+__device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uint8_t* stg, uint8_t* scratch,
+                                       uint32_t dst) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t* abase = stg + g.act_off;
+    int astride = g.act_bytes;
+    const int nt = u.grp.z;
+    if (XM == X_RAW_F32 || XM == X_RAW_BF16) {
+#pragma unroll 1
+        for (int t = 0; t < nt; ++t)
+            warp_quant_chunk<XM == X_RAW_BF16>(abase + t * g.act_bytes, u.kbn, scratch + t * kChunk * 36);
+        __syncwarp();
+        abase = scratch;
+        astride = kChunk * 36;
+    }
+#pragma unroll 1
+    for (int t = 0; t < nt; ++t) {
+        const uint8_t* ab = abase + t * astride;
+        int isum[kChunk];
+        float sc[kChunk];
+        // the blocks' integer sums and scale products are independent: all
+        // loads of the chunk are in flight together
+#pragma unroll
+        for (int kb = 0; kb < kChunk; ++kb) {
+            isum[kb] = 0;
+            sc[kb] = 0.0f;
+            if (kb < u.kbn) {
+                int w[8];
+                float dw;
+                s_block<FMT>(stg, kb, w, dw);
+                // a 36-byte Q8_1 block: 4-byte aligned only (d, s, then 8 words of codes)
+                const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) isum[kb] = __dp4a(w[j], (int)aw[1 + j], isum[kb]);
+                sc[kb] = __fmul_rn(dw, h2f((uint16_t)(aw[0] & 0xffff)));
+            }
+        }
+        // then the chunk's ordered chain of fused multiply-adds
+        float part = 0.0f;
+#pragma unroll
+        for (int kb = 0; kb < kChunk; ++kb)
+            if (kb < u.kbn) part = __fmaf_rn(__int2float_rn(isum[kb]), sc[kb], part);
+        dsmem_st(dst + (uint32_t)((t * 32 + lane) * 4), part);
+    }
+}
+
+// One out-of-line copy each of the epilogues' quantiser and SwiGLU.
+__device__ __noinline__ void s_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
+__device__ __noinline__ float s_swiglu(float g, float u) { return __fmul_rn(silu_f32(g), u); }
+
+// The item's epilogue in the cluster's first CTA: per token (warps take
+// tokens in turn) the chunk partials in chunk order, then the output mode.
+// pb: this item's partial buffer [units][T][32].
+template <int OM>
+__device__ void s_epilogue(const SArgs& g, const uint8_t* rs, const SUnit& u, const float* pb) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    const int T = g.T;
+    const int nt = u.grp.z;
+    const int row = u.tile * kTileRows + u.s * 32 + lane;      // row of the group's matrix
+    for (int t = warp; t < nt; t += nw) {
+        float acc = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < g.nchunks; ++c) acc = __fadd_rn(acc, pb[(c * T + t) * 32 + lane]);
+        const int64_t pp = (int64_t)u.grp.y + t;                // token (dense) or pair position
+        if (OM == OUT_SWIGLU) {
+            // the up slice's partials follow the gate slice's
+            float up = 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < g.nchunks; ++c) up = __fadd_rn(up, pb[((g.nchunks + c) * T + t) * 32 + lane]);
+            s_quant(s_swiglu(acc, up), g.yq + (pp * g.yq_ld + u.tile * 2 + u.hb) * 36);
+            continue;
+        }
+        float* yr = g.y + pp * g.y_ld + row;
+        if (OM == OUT_F32_ADD) {
+            *yr = __fadd_rn(*yr, acc);
+            continue;
+        }
+        *yr = acc;
+        if (OM == OUT_F32_Q81) {
+            s_quant(acc, g.yq + (pp * g.yq_ld + u.tile * 4 + u.s) * 36);
+        } else if (OM == OUT_F32_COMBINE) {
+            // this pair's 32 rows of o are out: count them for the token; the
+            // last of the token's k pairs combines this 32-row block
+            __threadfence();
+            __syncwarp();
+            const int tok = s_tok(rs, u.a, t);
+            const int blk = u.tile * 4 + u.s;
+            int last = 0;
+            if (lane == 0) {
+                int* cnt = g.cnt_comb + (int64_t)tok * (g.L / 32) + blk;
+                last = (atomicAdd(cnt, 1) == g.k - 1);
+                if (last) *cnt = 0;
+            }
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {
+                __threadfence();
+                float a2 = 0.0f;
+                for (int j0 = 0; j0 < g.k; j0 += 8) {
+                    float ov[8], wv[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < g.k) {
+                            const int pj = tok * g.k + j0 + j;
+                            wv[j] = __ldcg(g.wts + pj);
+                            const int pos = __ldcg(g.pos + pj);
+                            ov[j] = __ldcg(g.y + (int64_t)pos * g.y_ld + row);
+                        }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < g.k) a2 = __fmaf_rn(wv[j], ov[j], a2);
+                }
+                g.ylat[(int64_t)tok * g.L + row] = a2;
+                s_quant(a2, g.ylq + ((int64_t)tok * (g.L / 32) + blk) * 36);
+            }
+        }
+    }
+}
+
+// Prefetch into L2 this CTA's share of the routed experts' ranges (group a's
+// expert e: bytes [0, len) at base + e * len; len a multiple of 256; groups
+// taken in order, the total split evenly over the grid's CTAs).
+__device__ __forceinline__ void s_prefetch_experts(const SArgs& g, const uint8_t* rs, int na, const uint8_t* base,
+                                                   int64_t len) {
+    const uint32_t len_u = (uint32_t)(len >> 8);
+    const uint32_t total_u = (uint32_t)na * len_u;
+    const uint32_t share_u = (total_u + gridDim.x - 1) / gridDim.x;
+    uint32_t lo = blockIdx.x * share_u;
+    const uint32_t hi = min(total_u, lo + share_u);
+    while (lo < hi) {
+        const uint32_t a = lo / len_u;
+        const uint32_t end = min(hi, (a + 1) * len_u);
+        const int e = sgroup(g, rs, (int)a).x;
+        const int64_t off = (int64_t)(lo - a * len_u) << 8;
+        l2_prefetch_range(base + (int64_t)e * len, off, off + ((int64_t)(end - lo) << 8));
+        lo = end;
+    }
+}
+
+// Prefetch into L2 the weights of this warp's unit in every item of its
+// cluster from `m0` on (the items the ring has not requested yet), so that
+// HBM streams them while the ring works through the earlier ones.
+template <int FMT, int OM>
+__device__ __forceinline__ void s_prefetch_own(const SArgs& g, const uint8_t* rs, int n_items, int cid, int ncl,
+                                               int m0, int rank, int warp) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    if (lane > 1) return;
+    for (int item = cid + m0 * ncl; item < n_items; item += ncl) {
+        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
+        if (!u.has) return;
+        if (lane == 0)
+            bulk_prefetch_l2(g.q + u.grp.x * g.q_gstride +
+                                 ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + (int64_t)u.c * kChunk) * SL::kCodes,
+                             (uint32_t)(u.kbn * SL::kCodes));
+        else
+            bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows +
+                                 (int64_t)u.s * g.nb * 32 + (int64_t)u.c * kChunk * 32,
+                             (uint32_t)(u.kbn * 64));
+    }
+}
+
+// ============================================================================
+// a3 + a5 for T <= 8, T * k <= 64: the router as one cluster of C CTAs.
+// CTA r holds experts r * epc .. +epc-1, one per warp, each lane keeping its
+// L/32 lane-strided router weights in registers; a logit is that lane's fmaf
+// chain over z, the xor butterfly of adds, plus the bias (the router's
+// order).  The logits go to global memory and, through distributed shared
+// memory, to the first CTA, which then ranks them (top-k, lower id first on
+// ties, NaN as -inf), takes the softmax over the k in rank order, buckets the
+// pairs, and writes the routing arrays and the group table.
+// ============================================================================
+struct RSArgs {
+    const float* z;          // [T][L]
+    const float* w;          // [E][L]
+    const float* bias;       // [E] or NULL
+    int T, L, E, k, C, epc;
+    float* logits;           // [T][E]
+    int32_t* idx;            // [T][k]
+    float* wts;              // [T][k]
+    int32_t *counts, *offsets, *perm, *pos, *act, *n_act;
+    int4* grp;               // [groups]
+    int32_t* gtok;           // [groups][8]
+};
+
+__host__ __device__ constexpr int rs_smem_bytes(int T, int L, int E) {
+    // z rows, logits [T][E], top-k ids and values, bucket scratch
+    return T * L * 4 + T * E * 4 + 64 * 4 * 2 + (2 * E + 1) * 4 + 64 * 4 * 2 + 64 * 16 + 16;
+}
+
+__global__ void __launch_bounds__(kSMaxWarps * 32, 1) k_route_small(RSArgs a) {
+    extern __shared__ __align__(16) float rsm_small[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, L = a.L, E = a.E, k = a.k, P = T * k;
+    const int rank = a.C > 1 ? (int)cluster_rank() : 0;
+    float* zs = rsm_small;                          // [T][L]
+    float* lg = zs + T * L;                         // [T][E] (first CTA)
+    int32_t* sidx = reinterpret_cast<int32_t*>(lg + T * E);   // [64]
+    float* sval = reinterpret_cast<float*>(sidx + 64);        // [64]
+    int32_t* scount = reinterpret_cast<int32_t*>(sval + 64);  // [E], then offsets [E+1]
+    int32_t* soff = scount + E;
+    int32_t* sperm = soff + E + 1;                  // [64]
+    int32_t* spos = sperm + 64;                     // [64]
+    int4* sgrp = reinterpret_cast<int4*>(((uintptr_t)(spos + 64) + 15) & ~(uintptr_t)15);   // [64]
+    int* snact = reinterpret_cast<int*>(sgrp + 64);
+    const int e = rank * a.epc + warp;
+    const bool has_e = warp < a.epc && e < E;
+    const int nj = L >> 5;
+    // the router rows do not depend on the upstream kernel
+    float wr[kRouterJ];
+    {
+        const float* wrow = a.w + (int64_t)(has_e ? e : 0) * L + lane;
+#pragma unroll
+        for (int j = 0; j < kRouterJ; ++j) wr[j] = (has_e && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
+    }
+    const float bias = (has_e && a.bias) ? __ldg(a.bias + e) : 0.0f;
+    // every CTA of the cluster is running before any distributed store
+    if (a.C > 1) cluster_barrier();
+    pdl_wait();
+    pdl_trigger();
+    for (int i = threadIdx.x; i < T * L / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(zs)[i] = __ldcg(reinterpret_cast<const float4*>(a.z) + i);
+    __syncthreads();
+    if (has_e) {
+        const uint32_t lg_lead = a.C > 1 ? dsmem_map(smem_addr(lg), 0) : smem_addr(lg);
+        for (int t = 0; t < T; ++t) {
+            const float* zr = zs + t * L + lane;
+            float p = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kRouterJ; ++j)
+                if (j < nj) p = __fmaf_rn(zr[32 * j], wr[j], p);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(kFull, p, o));
+            if (a.bias) p = __fadd_rn(p, bias);
+            if (lane == 0) {
+                a.logits[(int64_t)t * E + e] = p;
+                dsmem_st(lg_lead + (uint32_t)((t * E + e) * 4), p);
+            }
+        }
+    }
+    if (a.C > 1) cluster_barrier(); else __syncthreads();
+    if (rank != 0) return;
+    // ---- the first CTA: top-k by rank, softmax, bucketing ----
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+        const float v0 = lg[i];
+        lg[i] = (v0 != v0) ? -INFINITY : v0;          // a NaN logit ranks as -inf
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+        const int t = i / E, ee = i - t * E;
+        const float* row = lg + t * E;
+        const float v = row[ee];
+        int r = 0;
+        for (int j = 0; j < E; ++j) r += (row[j] > v) | ((row[j] == v) & (j < ee));
+        if (r < k) {
+            sidx[t * k + r] = ee;
+            sval[t * k + r] = v;
+        }
+    }
+    __syncthreads();
+    for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) {
+        const float sel = lane < k ? sval[t * k + lane] : 0.0f;
+        const float l0 = __shfl_sync(kFull, sel, 0);
+        const float ex = lane < k ? exp_f32(__fsub_rn(sel, l0)) : 0.0f;
+        float sum = 0.0f;
+        for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, __shfl_sync(kFull, ex, j));
+        if (lane < k) {
+            a.idx[t * k + lane] = sidx[t * k + lane];
+            a.wts[t * k + lane] = __fdiv_rn(ex, sum);
+        }
+    }
+    if (warp == 0) bucket_warp_small(sidx, P, E, scount, soff, sperm, spos, nullptr, snact, sgrp);
+    __syncthreads();
+    const int na = *snact;
+    for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        a.perm[i] = sperm[i];
+        a.pos[i] = spos[i];
+    }
+    for (int i = threadIdx.x; i < E; i += blockDim.x) a.counts[i] = scount[i];
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) a.offsets[i] = soff[i];
+    for (int i = threadIdx.x; i < na; i += blockDim.x) {
+        const int4 gq = sgrp[i];
+        a.act[i] = gq.x;
+        a.grp[i] = gq;
+        for (int j = 0; j < gq.z && j < kSMaxT; ++j) a.gtok[i * kSMaxT + j] = sperm[gq.y + j] / k;
+    }
+    if (threadIdx.x == 0) *a.n_act = na;
+}
+
+template <int FMT, int XM, int OM>
+__global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
+    extern __shared__ __align__(128) uint8_t ssm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = g.stages;
+    const int rank = g.C > 1 ? (int)cluster_rank() : 0;
+    const int cid = (int)blockIdx.x / g.C;
+    const int ncl = (int)gridDim.x / g.C;
+    uint64_t* mybar = reinterpret_cast<uint64_t*>(ssm) + warp * 2;
+    uint8_t* rs = ssm + g.route_off;
+    uint8_t* stages = ssm + kSHeader + (size_t)warp * (S * g.stage_bytes + g.scratch_bytes);
+    uint8_t* scratch = stages + S * g.stage_bytes;
+    float* pbuf = reinterpret_cast<float*>(ssm + g.pbuf_off);
+    const int units = (OM == OUT_SWIGLU ? 2 : 1) * g.nchunks;
+    const uint32_t pb_local = smem_addr(pbuf);
+    const uint32_t pb_lead = g.C > 1 ? dsmem_map(pb_local, 0) : pb_local;
+    // this warp's unit index in the partial buffer
+    const int uidx = (OM == OUT_SWIGLU ? (rank / g.Cg) * g.nchunks : 0) + (rank % g.Cg) * g.cpc + warp;
+
+    if (lane < S) mbar_init(&mybar[lane], 1);
+    if (lane == 0) fence_barrier_init();
+    // every CTA of the cluster is running (its shared memory may be written
+    // by the others) before the first distributed shared-memory store
+    if (g.C > 1) cluster_barrier(); else __syncthreads();
+
+    int n_items = 0;
+    auto issue_w = [&](int m) {
+        const int item = cid + m * ncl;
+        if (item >= n_items) return;
+        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
+        if (u.has) s_issue_weights<FMT, XM>(g, u, stages + (m % S) * g.stage_bytes, &mybar[m % S]);
+    };
+    auto issue_a = [&](int m) {
+        const int item = cid + m * ncl;
+        if (item >= n_items) return;
+        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
+        if (u.has) s_issue_acts<XM>(g, rs, u, stages + (m % S) * g.stage_bytes + g.act_off, &mybar[m % S]);
+    };
+    // L2 prefetch of the fixed ranges a later kernel reads (by the last warp)
+    auto prefetch_fixed = [&]() {
+        if (warp == (int)(blockDim.x >> 5) - 1 && lane < 3 && g.pf[lane]) {
+            int64_t lo, hi;
+            share_of(g.pf_bytes[lane], g.pf_share[lane], lo, hi);
+            l2_prefetch_range(g.pf[lane], lo, hi);
+        }
+    };
+    if (g.early) {
+        // weights (and, for the down projection, the routing, complete
+        // before the upstream gate/up started) do not depend on the upstream grid
+        if (g.route != ROUTE_NONE) s_load_groups(g, rs);
+        n_items = s_n_groups(g, rs) * g.items_per_group;
+        for (int m = 0; m < S; ++m) issue_w(m);
+        pdl_wait();
+        pdl_trigger();
+        for (int m = 0; m < S; ++m) issue_a(m);
+        s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank, warp);
+        prefetch_fixed();
+    } else {
+        pdl_wait();
+        pdl_trigger();
+        if (g.route != ROUTE_NONE) s_load_groups(g, rs);
+        n_items = s_n_groups(g, rs) * g.items_per_group;
+        for (int m = 0; m < S; ++m) {
+            issue_w(m);
+            issue_a(m);
+        }
+        s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank, warp);
+        prefetch_fixed();
+        if (g.pfe_q && warp == (int)(blockDim.x >> 5) - 1 && lane < 2) {
+            const int na = s_n_groups(g, rs);
+            if (lane == 0) s_prefetch_experts(g, rs, na, g.pfe_q, g.pfe_qs);
+            else s_prefetch_experts(g, rs, na, g.pfe_d, g.pfe_ds);
+        }
+    }
+
+    bool ok = true;
+    int m_fail = -1;
+    for (int m = 0;; ++m) {
+        const int item = cid + m * ncl;
+        if (item >= n_items) break;
+        const int st = m % S;
+        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
+        uint8_t* stg = stages + st * g.stage_bytes;
+        if (u.has && ok) {
+            const bool got = mbar_wait_bounded(&mybar[st], (uint32_t)((m / S) & 1), g.err, g.budget_ns);
+            ok = __all_sync(kFull, got);
+            if (!ok) m_fail = m;
+            if (ok) s_dots<FMT, XM>(g, u, stg, scratch, pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128));
+            // the stage is consumed: refill it with this warp's item m + S
+            __syncwarp();
+            fence_proxy_async();
+            if (ok) {
+                issue_w(m + S);
+                issue_a(m + S);
+            }
+        }
+        // every chunk partial of the item is in the first CTA
+        if (g.C > 1) cluster_barrier(); else __syncthreads();
+        if (rank == 0) s_epilogue<OM>(g, rs, u, pbuf + (size_t)(m & 1) * units * g.T * 32);
+    }
+    if (!ok) {
+        // drain: wait (bounded) for this warp's copies still in flight (the
+        // one that ran out and the S - 1 issued after it)
+        for (int j = m_fail; j < m_fail + S; ++j) {
+            const int item = cid + j * ncl;
+            if (item >= n_items) continue;
+            const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
+            if (u.has) mbar_wait_bounded(&mybar[j % S], (uint32_t)((j / S) & 1), nullptr, g.budget_ns);
+        }
+    }
+}
+
+}  // namespace elq

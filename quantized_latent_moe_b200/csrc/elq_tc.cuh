@@ -94,6 +94,47 @@ __device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 16 consecutive TMEM columns of this thread's lane := v.
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+// Pairs of fp32 values in one 64-bit register and the packed two-wide fp32
+// operations on them: each half is one IEEE round-to-nearest operation, the
+// same result as the scalar instruction, at half the instruction count.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // Exact int32 -> fp32 for |s| < 2^22 without the (slow) conversion unit: the
 // integer s + 0x4B400000 is the bit pattern of the float 1.5 * 2^23 + s, so
 // one fp32 subtraction of 1.5 * 2^23 recovers s exactly.
@@ -307,23 +348,35 @@ struct TcUnit {
     bool valid;
 };
 
+// Units of a group (the dense matrix, or one routed expert with its n_q
+// token tiles) run row tile by row tile, each row tile against all n_q token
+// tiles in turn: a weight tile is read from HBM once and its next uses follow
+// at once (from L2), while a group's token tiles (at most a few hundred KB)
+// stay in L2 across its row tiles.
 __device__ __forceinline__ TcUnit tc_unit(const TcArgs& g, int u) {
     TcUnit r;
-    r.rt = u % g.rtiles;
-    const int q = u / g.rtiles;
+    int tt;
     if (!g.act) {
+        const int n_q = (g.T + kTcN - 1) / kTcN;
+        r.rt = u / n_q;
+        tt = u - r.rt * n_q;
         r.e = 0;
-        r.slot0 = q * kTcN;
+        r.slot0 = tt * kTcN;
         r.nvalid = min(kTcN, g.T - r.slot0);
     } else {
+        const int q = u / g.rtiles;
         const int na = __ldcg(g.n_act);
-        int lo = 0, hi = na;    // tt_off[lo] <= q < tt_off[hi]
+        int lo = 0, hi = na;    // tt_off[lo] <= q < tt_off[hi]: the group's units are [tt_off[lo], tt_off[lo+1]) * rtiles
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
             if (__ldcg(g.tt_off + mid) <= q) lo = mid; else hi = mid;
         }
         r.e = __ldcg(g.act + lo);
-        const int tt = q - __ldcg(g.tt_off + lo);
+        const int base = __ldcg(g.tt_off + lo);
+        const int n_q = __ldcg(g.tt_off + lo + 1) - base;
+        const int v = u - base * g.rtiles;
+        r.rt = v / n_q;
+        tt = v - r.rt * n_q;
         r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
         const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
         r.nvalid = min(kTcN, cnt - tt * kTcN);
@@ -385,6 +438,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_sm;
+    if (warp >= 2) {
+        // every accumulator starts at the seed: an MMA then leaves seed + isum,
+        // the bit pattern of the float 1.5 * 2^23 + isum (see kAccSeed)
+        const uint32_t tb = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(((warp - 2) >> 2) * kTcEpiCols);
+#pragma unroll
+        for (int b = 0; b < kTcBufs; ++b) tmem_st16_const(tb + (uint32_t)(b * kTcN), kAccSeed);
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
     pdl_wait();
 
     const int n_units = tc_units(g);
@@ -455,7 +519,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     for (int kl = 0; kl < kTcKS; ++kl) {
                         const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
                         const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
-                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 0u);
+                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 1u);
                     }
                     umma_commit(&tfull[gr]);
                     umma_commit(&empty[s]);
@@ -477,12 +541,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
         for (int u = u0; u < u1 && !*abort_v; ++u) {
             const TcUnit un = tc_unit(g, u);
             if (!un.valid) continue;
-            float acc[kTcEpiCols], part[kTcEpiCols];
+            // accumulator pairs (columns 2j, 2j+1)
+            uint64_t acc2[kTcEpiCols / 2], part2[kTcEpiCols / 2];
 #pragma unroll
-            for (int j = 0; j < kTcEpiCols; ++j) { acc[j] = 0.0f; part[j] = 0.0f; }
-            const bool active = c0 < un.ncols;
+            for (int j = 0; j < kTcEpiCols / 2; ++j) { acc2[j] = 0ull; part2[j] = 0ull; }
             bool ok = true;
             const uint32_t tlane = (uint32_t)(sp * 32) << 16;
+            const uint64_t seed2 = f2_pack(kAccSeedF, kAccSeedF);
             for (int ks = 0; ks < kstages; ++ks, ++it) {
                 const int s = it % kTcStages, gr = it % kTcGroups;
                 const uint8_t* st = stages + s * kTcStage;
@@ -495,40 +560,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                 tc_fence_after();
                 const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
                 const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
-                uint32_t rc[kTcEpiCols], rn[kTcEpiCols];
                 const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + c0);
-                tmem_ld16(tb, rc);
-                tmem_ld_wait();
 #pragma unroll
                 for (int kl = 0; kl < kTcKS; ++kl) {
-                    if (kl + 1 < kTcKS) tmem_ld16(tb + (uint32_t)((kl + 1) * kTcN), rn);   // overlaps the rescale
-                    const int kb = ks * kTcKS + kl;
-                    if (active) {
-                        const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
-                        const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
+                    uint32_t rc[kTcEpiCols];
+                    tmem_ld16(tb + (uint32_t)(kl * kTcN), rc);
+                    tmem_ld_wait();
+                    // block kl of the stage: part = fmaf(isum, d_w * d_a, part) per column, two at a time
+                    const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
+                    const uint64_t dw2 = f2_pack(dw, dw);
+                    const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
 #pragma unroll
-                        for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
-                            const float4 dv = dak[j4];
-                            const float da4[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int j = 4 * j4 + q;
-                                const float isum = __fsub_rn(__uint_as_float(rc[j] + kAccSeed), kAccSeedF);
-                                part[j] = __fmaf_rn(isum, __fmul_rn(dw, da4[q]), part[j]);
-                            }
-                        }
+                    for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
+                        const float4 dv = dak[j4];
+                        const uint64_t i0 = f2_sub(f2_pack(__uint_as_float(rc[4 * j4]), __uint_as_float(rc[4 * j4 + 1])), seed2);
+                        const uint64_t i1 =
+                            f2_sub(f2_pack(__uint_as_float(rc[4 * j4 + 2]), __uint_as_float(rc[4 * j4 + 3])), seed2);
+                        part2[2 * j4] = f2_fma(i0, f2_mul(dw2, f2_pack(dv.x, dv.y)), part2[2 * j4]);
+                        part2[2 * j4 + 1] = f2_fma(i1, f2_mul(dw2, f2_pack(dv.z, dv.w)), part2[2 * j4 + 1]);
                     }
-                    if ((kb & (kChunk - 1)) == kChunk - 1 || kb == g.nb - 1) {
+                }
+                // the group's accumulators back to the seed for its next MMAs
 #pragma unroll
-                        for (int j = 0; j < kTcEpiCols; ++j) {
-                            acc[j] = __fadd_rn(acc[j], part[j]);
-                            part[j] = 0.0f;
-                        }
-                    }
-                    if (kl + 1 < kTcKS) {
-                        tmem_ld_wait();
+                for (int kl = 0; kl < kTcKS; ++kl) tmem_st16_const(tb + (uint32_t)(kl * kTcN), kAccSeed);
+                tmem_st_wait();
+                // a run of 8 blocks ends with every second stage (and with the last)
+                if ((ks & 1) || ks == kstages - 1) {
 #pragma unroll
-                        for (int j = 0; j < kTcEpiCols; ++j) rc[j] = rn[j];
+                    for (int j = 0; j < kTcEpiCols / 2; ++j) {
+                        acc2[j] = f2_add(acc2[j], part2[j]);
+                        part2[j] = 0ull;
                     }
                 }
                 tc_fence_before();
@@ -538,6 +599,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     mbar_arrive(&empty[s]);
                 }
             }
+            float acc[kTcEpiCols];
+#pragma unroll
+            for (int j = 0; j < kTcEpiCols / 2; ++j) f2_unpack(acc2[j], acc[2 * j], acc[2 * j + 1]);
             if (!ok) {
                 *abort_v = 1;
                 break;

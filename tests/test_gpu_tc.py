@@ -62,24 +62,68 @@ def test_tc_experts_grouped_exact(E, orc):
     assert np.array_equal(y_lat, tr["y_lat"])
 
 
-def test_tc_prefill_full_size_sampled(E, orc):
+def _threads(fn, parts):
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        return list(ex.map(fn, parts))
+
+
+def test_tc_prefill_full_size(E, orc):
     """The prefill workload at full size (T=2048, 128 experts, Zipf-skewed
-    router): all routing decisions and sampled tokens' outputs against the
-    oracle computing those tokens alone (the layer is token-wise independent)."""
+    router), through the layer call:
+     - z and its Q8_1 rows for all 2048 tokens against the oracle's quantised
+       matmul (the oracle quantises x and D itself);
+     - the routing of all 2048 tokens (logits, idx, weights) against the
+       oracle's router on the oracle's z, and the bucket arrays against the
+       oracle's bucketing of those ids;
+     - y for sampled tokens, the oracle computing them alone (the layer is
+       token-wise independent): the last pair of every expert group (each lands
+       in that expert's last, usually partial, 64-token tile), every token of
+       the smallest group, the first and last tokens of the largest, tokens 0
+       and 2047."""
     wl = synth.WORKLOADS["prefill"]
     ly = gpu_layer(wl)
     x = synth.make_x(wl)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
     assert E.workspace_status(ly.workspace(wl.T)) == 0
-    counts = E.workspace_view(ly, wl.T, "counts").cpu().numpy()
-    assert counts.sum() == wl.T * wl.k and counts.max() <= wl.T
-    ol = oracle_layer(orc, wl, experts=[])
-    sample = [0, 1, 511, 1024, 2047]
-    xs = x.float().numpy()[sample]
-    ref = oracle_forward(orc, ol, wl, xs, trace=True)
-    idx = E.workspace_view(ly, wl.T, "idx").cpu().numpy().reshape(wl.T, -1)
-    assert np.array_equal(idx[sample], ref["idx"])
-    assert np.array_equal(y[sample], ref["y"])
+    v = lambda n: E.workspace_view(ly, wl.T, n).cpu().numpy()
+    T, L, H, k = wl.T, wl.L, wl.H, wl.k
+    # z for every token (rows of tokens split over host threads)
+    dw = synth.dense_weights(wl, 0)
+    Dq = orc.quantize(8, dw["D"].numpy())
+    xq = orc.quantize(orc.Q8_1, x.float().numpy())
+    assert np.array_equal(v("xq").reshape(T, -1), xq)
+    rows = [(t0, min(T, t0 + 128)) for t0 in range(0, T, 128)]
+    zs = _threads(lambda r: orc.qmatmul(8, Dq, L, H, xq[r[0]:r[1]], r[1] - r[0]), rows)
+    z_ref = np.concatenate(zs)
+    assert np.array_equal(v("z").reshape(T, L), z_ref)
+    assert np.array_equal(v("zq").reshape(T, -1), orc.quantize(orc.Q8_1, z_ref))
+    # routing of every token
+    ridx, rw, rlg = orc.router_topk(z_ref, dw["router_w"].numpy(), dw["router_bias"].numpy(), k)
+    assert np.array_equal(v("logits").reshape(T, -1), rlg)
+    idx = v("idx").reshape(T, k)
+    assert np.array_equal(idx, ridx)
+    assert np.array_equal(v("weights").reshape(T, k), rw)
+    counts, offsets, perm, pos = orc.bucket(ridx, wl.E)
+    assert np.array_equal(v("counts"), counts) and np.array_equal(v("offsets"), offsets)
+    assert np.array_equal(v("perm"), perm) and np.array_equal(v("pos"), pos)
+    # sampled outputs
+    sample = {0, T - 1}
+    for e in range(wl.E):
+        if counts[e]:
+            sample.add(int(perm[offsets[e + 1] - 1]) // k)
+    e_min = int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    e_max = int(np.argmax(counts))
+    sample |= {int(p) // k for p in perm[offsets[e_min]:offsets[e_min + 1]]}
+    sample |= {int(perm[offsets[e_max]]) // k, int(perm[offsets[e_max + 1] - 1]) // k}
+    sample = sorted(sample)
+    ol = oracle_layer(orc, wl, experts=sorted(set(ridx[sample].reshape(-1).tolist())))
+    xs = x.float().numpy()
+    parts = [sample[i:i + 8] for i in range(0, len(sample), 8)]
+    ref = np.concatenate(_threads(lambda ts: ol.forward(xs[ts]), parts))
+    assert max_abs_rel(y[sample], ref) <= 1e-3
+    assert np.array_equal(y[sample], ref)
 
 
 def test_int8_rate_kernel_runs(E):
