@@ -218,7 +218,8 @@ WArgs dense_w(const elq_qmat* w, int T, const void* x, int x_mode, int64_t x_row
 
 struct SPlan {
     bool ok;
-    int C, Cg, cpc, stages, stage_bytes, act_off, act_bytes, scratch_bytes, pbuf_off, route_off, smem, clusters;
+    int C, Cg, cpc, stages, stage_bytes, scales_off, acts_off, act_row, scratch_bytes, pbuf_off, route_off, smem,
+        clusters;
     int nchunks, ipg;
 };
 
@@ -247,14 +248,18 @@ SPlan plan_s(int fmt, int x_mode, bool swiglu, int rows_per_group, int K, int gr
     p.Cg = Cg;
     p.C = Cg * halves;
     p.cpc = (p.nchunks + Cg - 1) / Cg;
-    const int codes = kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
-    p.act_off = codes + kChunk * 64;
-    p.act_bytes = x_mode == X_RAW_F32 ? 1024 : x_mode == X_RAW_BF16 ? 512 : kChunk * 36;
-    p.stage_bytes = (int)round_up((size_t)p.act_off + (size_t)T * p.act_bytes, 128);
+    // one stage of a CTA: the codes and scales of its cpc chunks, then each
+    // token's activations over the same blocks
+    const int codes = p.cpc * kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
+    const int ablock = x_mode == X_RAW_F32 ? 128 : x_mode == X_RAW_BF16 ? 64 : 36;
+    p.scales_off = codes;
+    p.acts_off = (int)round_up((size_t)codes + (size_t)p.cpc * kChunk * 64, 128);
+    p.act_row = p.cpc * kChunk * ablock;
+    p.stage_bytes = (int)round_up((size_t)p.acts_off + (size_t)T * p.act_row, 128);
     p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)T * kChunk * 36, 128) : 0;
     const int pbuf = 2 * halves * p.nchunks * T * 128;
     const int route = routed ? (int)round_up((size_t)kSRouteBytes, 128) : 0;
-    auto smem_for = [&](int st) { return kSHeader + p.cpc * (st * p.stage_bytes + p.scratch_bytes) + pbuf + route; };
+    auto smem_for = [&](int st) { return kSHeader + st * p.stage_bytes + p.cpc * p.scratch_bytes + pbuf + route; };
     // resident CTAs per SM: shared memory (1 KB reserved per CTA), warps, and
     // registers at the launch bound's 64 per thread
     auto per_sm = [&](int smem) {
@@ -277,7 +282,7 @@ SPlan plan_s(int fmt, int x_mode, bool swiglu, int rows_per_group, int K, int gr
         if (r2 + 1 < 2 * r1) p.stages = 2;
     }
     p.clusters = clusters_for(p.stages);
-    p.pbuf_off = kSHeader + p.cpc * (p.stages * p.stage_bytes + p.scratch_bytes);
+    p.pbuf_off = kSHeader + p.stages * p.stage_bytes + p.cpc * p.scratch_bytes;
     p.route_off = p.pbuf_off + pbuf;
     p.smem = smem_for(p.stages);
     p.ok = true;
@@ -336,8 +341,9 @@ cudaError_t launch_s(SArgs g, int fmt, int x_mode, int out_mode, const SPlan& p,
     g.cpc = p.cpc;
     g.stages = p.stages;
     g.stage_bytes = p.stage_bytes;
-    g.act_off = p.act_off;
-    g.act_bytes = p.act_bytes;
+    g.scales_off = p.scales_off;
+    g.acts_off = p.acts_off;
+    g.act_row = p.act_row;
     g.scratch_bytes = p.scratch_bytes;
     g.pbuf_off = p.pbuf_off;
     g.route_off = p.route_off;

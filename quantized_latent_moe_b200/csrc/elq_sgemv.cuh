@@ -76,7 +76,9 @@ struct SArgs {
     int items_per_group;     // slices (or slice pairs, SwiGLU) per group
     int groups_max;          // bound on the groups (dense: 1)
     int C, Cg, cpc, stages;  // cluster size, CTAs per slice, chunks (= warps) per CTA, ring depth
-    int stage_bytes, act_off, act_bytes, scratch_bytes, pbuf_off, route_off;
+    // one stage of a CTA: codes [cpc][8 blocks], scales [cpc][8 blocks][32],
+    // then per token its activations over the CTA's blocks (act_row bytes each)
+    int stage_bytes, scales_off, acts_off, act_row, scratch_bytes, pbuf_off, route_off;
     // routing
     int route;
     int T, E, k;
@@ -199,34 +201,46 @@ __device__ __forceinline__ SUnit s_unit(const SArgs& g, const uint8_t* rs, int i
     return u;
 }
 
+// Bytes of one activation block (32 values) in the input's form.
 template <int XM>
-__device__ __forceinline__ uint32_t s_act_bytes(int kbn) {
-    if (XM == X_RAW_F32) return (uint32_t)kbn * 128u;
-    if (XM == X_RAW_BF16) return (uint32_t)kbn * 64u;
-    return (uint32_t)kbn * 36u;
+__device__ __forceinline__ uint32_t s_act_block() {
+    return XM == X_RAW_F32 ? 128u : XM == X_RAW_BF16 ? 64u : 36u;
 }
 
+// The CTA's blocks of an item: [kb0, kb0 + nblk) of slice (tile, s), the
+// chunks (rank % Cg) * cpc .. +cpc-1 (clipped to the matrix).
+struct SRange {
+    int kb0, nblk;
+};
+__device__ __forceinline__ SRange s_range(const SArgs& g, int rank) {
+    SRange r;
+    r.kb0 = (rank % g.Cg) * g.cpc * kChunk;
+    r.nblk = max(0, min(g.nb, r.kb0 + g.cpc * kChunk) - r.kb0);
+    return r;
+}
+
+// One stage of a CTA in three kinds of bulk copies: the codes of all its
+// chunks (contiguous in the arena), their scales, and per token its
+// activations over the same blocks.  Thread 0 arms the stage's barrier with
+// every byte and issues the weights; lanes 0 .. ntok-1 of warp 0 the
+// activations (s_issue_acts).
 template <int FMT, int XM>
-__device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, uint8_t* stg, uint64_t* bar) {
+__device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, const SRange& r, uint8_t* stg,
+                                                uint64_t* bar) {
     using SL = WSlice<FMT>;
-    const int lane = threadIdx.x & 31;
-    const uint32_t cb = (uint32_t)(u.kbn * SL::kCodes), sb = (uint32_t)(u.kbn * 64);
-    if (lane == 0) mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * s_act_bytes<XM>(u.kbn));
-    __syncwarp();
-    if (lane == 0) {
-        const uint8_t* src = g.q + u.grp.x * g.q_gstride +
-                             ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + (int64_t)u.c * kChunk) * SL::kCodes;
-        bulk_g2s(stg, src, cb, bar);
-    } else if (lane == 1) {
-        const uint16_t* src = g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows +
-                              (int64_t)u.s * g.nb * 32 + (int64_t)u.c * kChunk * 32;
-        bulk_g2s(stg + kChunk * SL::kCodes, src, sb, bar);
-    }
+    const uint32_t cb = (uint32_t)(r.nblk * SL::kCodes), sb = (uint32_t)(r.nblk * 64);
+    mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * (uint32_t)r.nblk * s_act_block<XM>());
+    bulk_g2s(stg, g.q + u.grp.x * g.q_gstride + ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
+             cb, bar);
+    bulk_g2s(stg + g.scales_off,
+             g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows + (int64_t)u.s * g.nb * 32 +
+                 (int64_t)r.kb0 * 32,
+             sb, bar);
 }
 
 template <int XM>
-__device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, const SUnit& u, uint8_t* act,
-                                             uint64_t* bar) {
+__device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, const SUnit& u, const SRange& r,
+                                             uint8_t* stg, uint64_t* bar) {
     const int lane = threadIdx.x & 31;
     if (lane < u.grp.z) {
         int64_t row;
@@ -235,12 +249,12 @@ __device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, 
         else row = lane;
         const uint8_t* src;
         if (XM == X_RAW_F32)
-            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)u.c * 256) * 4;
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)r.kb0 * 32) * 4;
         else if (XM == X_RAW_BF16)
-            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)u.c * 256) * 2;
+            src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)r.kb0 * 32) * 2;
         else
-            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + (int64_t)u.c * kChunk) * 36;
-        bulk_g2s(act + lane * g.act_bytes, src, s_act_bytes<XM>(u.kbn), bar);
+            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + r.kb0) * 36;
+        bulk_g2s(stg + g.acts_off + lane * g.act_row, src, (uint32_t)r.nblk * s_act_block<XM>(), bar);
     }
 }
 
@@ -292,20 +306,19 @@ __device__ __noinline__ void warp_quant_chunk(const uint8_t* src, int kbn, uint8
     }
 }
 
-// Block kb of this lane's row from the stage: signed 8-bit codes in w[0..7]
-// (codes 4j .. 4j+3 in w[j]) and the scale.
+// Block kb of this lane's row: signed 8-bit codes in w[0..7] (codes 4j ..
+// 4j+3 in w[j]) from the chunk's codes, and its scale.
 template <int FMT>
-__device__ __forceinline__ void s_block(const uint8_t* stg, int kb, int (&w)[8], float& dw) {
-    using SL = WSlice<FMT>;
+__device__ __forceinline__ void s_block(const uint8_t* codes, const uint16_t* scales, int kb, int (&w)[8], float& dw) {
     const int lane = threadIdx.x & 31;
-    dw = h2f(reinterpret_cast<const uint16_t*>(stg + kChunk * SL::kCodes)[kb * 32 + lane]);
+    dw = h2f(scales[kb * 32 + lane]);
     if (FMT == 8) {
-        const uint8_t* cp = stg + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
+        const uint8_t* cp = codes + kb * 1024 + (lane >> 3) * 256 + (lane & 7) * 16;
         const uint4 a = lds128(cp), b = lds128(cp + 128);
         w[0] = (int)a.x; w[1] = (int)a.y; w[2] = (int)a.z; w[3] = (int)a.w;
         w[4] = (int)b.x; w[5] = (int)b.y; w[6] = (int)b.z; w[7] = (int)b.w;
     } else {
-        const uint4 a = lds128(stg + kb * 512 + lane * 16);
+        const uint4 a = lds128(codes + kb * 512 + lane * 16);
         const uint32_t v[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -326,14 +339,19 @@ __device__ __forceinline__ void s_block(const uint8_t* stg, int kb, int (&w)[8],
 template <int FMT, int XM>
 __device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uint8_t* stg, uint8_t* scratch,
                                        uint32_t dst) {
+    using SL = WSlice<FMT>;
     const int lane = threadIdx.x & 31;
-    const uint8_t* abase = stg + g.act_off;
-    int astride = g.act_bytes;
+    const int warp = threadIdx.x >> 5;
+    // this warp's chunk inside the CTA's stage
+    const uint8_t* codes = stg + warp * kChunk * SL::kCodes;
+    const uint16_t* scales = reinterpret_cast<const uint16_t*>(stg + g.scales_off) + warp * kChunk * 32;
+    const uint8_t* abase = stg + g.acts_off + warp * kChunk * s_act_block<XM>();
+    int astride = g.act_row;
     const int nt = u.grp.z;
     if (XM == X_RAW_F32 || XM == X_RAW_BF16) {
 #pragma unroll 1
         for (int t = 0; t < nt; ++t)
-            warp_quant_chunk<XM == X_RAW_BF16>(abase + t * g.act_bytes, u.kbn, scratch + t * kChunk * 36);
+            warp_quant_chunk<XM == X_RAW_BF16>(abase + t * g.act_row, u.kbn, scratch + t * kChunk * 36);
         __syncwarp();
         abase = scratch;
         astride = kChunk * 36;
@@ -352,7 +370,7 @@ __device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uin
             if (kb < u.kbn) {
                 int w[8];
                 float dw;
-                s_block<FMT>(stg, kb, w, dw);
+                s_block<FMT>(codes, scales, kb, w, dw);
                 // a 36-byte Q8_1 block: 4-byte aligned only (d, s, then 8 words of codes)
                 const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36);
 #pragma unroll
@@ -462,26 +480,23 @@ __device__ __forceinline__ void s_prefetch_experts(const SArgs& g, const uint8_t
     }
 }
 
-// Prefetch into L2 the weights of this warp's unit in every item of its
-// cluster from `m0` on (the items the ring has not requested yet), so that
-// HBM streams them while the ring works through the earlier ones.
+// Prefetch into L2 this CTA's weights in every item of its cluster from `m0`
+// on (the items the ring has not requested yet), so that HBM streams them
+// while the ring works through the earlier ones.  Thread 0.
 template <int FMT, int OM>
 __device__ __forceinline__ void s_prefetch_own(const SArgs& g, const uint8_t* rs, int n_items, int cid, int ncl,
-                                               int m0, int rank, int warp) {
+                                               int m0, int rank) {
     using SL = WSlice<FMT>;
-    const int lane = threadIdx.x & 31;
-    if (lane > 1) return;
+    const SRange r = s_range(g, rank);
+    if (r.nblk <= 0) return;
     for (int item = cid + m0 * ncl; item < n_items; item += ncl) {
-        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
-        if (!u.has) return;
-        if (lane == 0)
-            bulk_prefetch_l2(g.q + u.grp.x * g.q_gstride +
-                                 ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + (int64_t)u.c * kChunk) * SL::kCodes,
-                             (uint32_t)(u.kbn * SL::kCodes));
-        else
-            bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows +
-                                 (int64_t)u.s * g.nb * 32 + (int64_t)u.c * kChunk * 32,
-                             (uint32_t)(u.kbn * 64));
+        const SUnit u = s_unit<OM>(g, rs, item, rank, 0);
+        bulk_prefetch_l2(g.q + u.grp.x * g.q_gstride +
+                             ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
+                         (uint32_t)(r.nblk * SL::kCodes));
+        bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows + (int64_t)u.s * g.nb * 32 +
+                             (int64_t)r.kb0 * 32,
+                         (uint32_t)(r.nblk * 64));
     }
 }
 
@@ -620,35 +635,43 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
     const int rank = g.C > 1 ? (int)cluster_rank() : 0;
     const int cid = (int)blockIdx.x / g.C;
     const int ncl = (int)gridDim.x / g.C;
-    uint64_t* mybar = reinterpret_cast<uint64_t*>(ssm) + warp * 2;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ssm);            // [S] stage barriers
+    volatile int* bad = reinterpret_cast<volatile int*>(ssm + 64);
     uint8_t* rs = ssm + g.route_off;
-    uint8_t* stages = ssm + kSHeader + (size_t)warp * (S * g.stage_bytes + g.scratch_bytes);
-    uint8_t* scratch = stages + S * g.stage_bytes;
+    uint8_t* stages = ssm + kSHeader;
+    uint8_t* scratch = ssm + kSHeader + (size_t)S * g.stage_bytes + (size_t)warp * g.scratch_bytes;
     float* pbuf = reinterpret_cast<float*>(ssm + g.pbuf_off);
     const int units = (OM == OUT_SWIGLU ? 2 : 1) * g.nchunks;
     const uint32_t pb_local = smem_addr(pbuf);
     const uint32_t pb_lead = g.C > 1 ? dsmem_map(pb_local, 0) : pb_local;
     // this warp's unit index in the partial buffer
     const int uidx = (OM == OUT_SWIGLU ? (rank / g.Cg) * g.nchunks : 0) + (rank % g.Cg) * g.cpc + warp;
+    const SRange rng = s_range(g, rank);
+    const bool cta_has = rng.nblk > 0;
 
-    if (lane < S) mbar_init(&mybar[lane], 1);
-    if (lane == 0) fence_barrier_init();
+    if (threadIdx.x < S) mbar_init(&bars[threadIdx.x], 1);
+    if (threadIdx.x == 0) {
+        *bad = 0;
+        fence_barrier_init();
+    }
     // every CTA of the cluster is running (its shared memory may be written
     // by the others) before the first distributed shared-memory store
     if (g.C > 1) cluster_barrier(); else __syncthreads();
 
     int n_items = 0;
-    auto issue_w = [&](int m) {
+    int issued = -1;                 // thread 0: the last item whose copies went out
+    auto issue_w = [&](int m) {      // thread 0
         const int item = cid + m * ncl;
-        if (item >= n_items) return;
-        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
-        if (u.has) s_issue_weights<FMT, XM>(g, u, stages + (m % S) * g.stage_bytes, &mybar[m % S]);
+        if (item >= n_items || !cta_has) return;
+        const SUnit u = s_unit<OM>(g, rs, item, rank, 0);
+        s_issue_weights<FMT, XM>(g, u, rng, stages + (m % S) * g.stage_bytes, &bars[m % S]);
+        issued = m;
     };
-    auto issue_a = [&](int m) {
+    auto issue_a = [&](int m) {      // warp 0
         const int item = cid + m * ncl;
-        if (item >= n_items) return;
-        const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
-        if (u.has) s_issue_acts<XM>(g, rs, u, stages + (m % S) * g.stage_bytes + g.act_off, &mybar[m % S]);
+        if (item >= n_items || !cta_has) return;
+        const SUnit u = s_unit<OM>(g, rs, item, rank, 0);
+        s_issue_acts<XM>(g, rs, u, rng, stages + (m % S) * g.stage_bytes, &bars[m % S]);
     };
     // L2 prefetch of the fixed ranges a later kernel reads (by the last warp)
     auto prefetch_fixed = [&]() {
@@ -663,22 +686,28 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         // before the upstream gate/up started) do not depend on the upstream grid
         if (g.route != ROUTE_NONE) s_load_groups(g, rs);
         n_items = s_n_groups(g, rs) * g.items_per_group;
-        for (int m = 0; m < S; ++m) issue_w(m);
+        if (threadIdx.x == 0)
+            for (int m = 0; m < S; ++m) issue_w(m);
         pdl_wait();
         pdl_trigger();
-        for (int m = 0; m < S; ++m) issue_a(m);
-        s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank, warp);
+        __syncwarp();
+        if (warp == 0)
+            for (int m = 0; m < S; ++m) issue_a(m);
+        if (threadIdx.x == 0) s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank);
         prefetch_fixed();
     } else {
         pdl_wait();
         pdl_trigger();
         if (g.route != ROUTE_NONE) s_load_groups(g, rs);
         n_items = s_n_groups(g, rs) * g.items_per_group;
-        for (int m = 0; m < S; ++m) {
-            issue_w(m);
-            issue_a(m);
+        if (warp == 0) {
+            for (int m = 0; m < S; ++m) {
+                if (lane == 0) issue_w(m);
+                __syncwarp();
+                issue_a(m);
+            }
+            if (lane == 0) s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank);
         }
-        s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank, warp);
         prefetch_fixed();
         if (g.pfe_q && warp == (int)(blockDim.x >> 5) - 1 && lane < 2) {
             const int na = s_n_groups(g, rs);
@@ -687,40 +716,38 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         }
     }
 
-    bool ok = true;
-    int m_fail = -1;
     for (int m = 0;; ++m) {
         const int item = cid + m * ncl;
         if (item >= n_items) break;
         const int st = m % S;
         const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
-        uint8_t* stg = stages + st * g.stage_bytes;
-        if (u.has && ok) {
-            const bool got = mbar_wait_bounded(&mybar[st], (uint32_t)((m / S) & 1), g.err, g.budget_ns);
-            ok = __all_sync(kFull, got);
-            if (!ok) m_fail = m;
-            if (ok) s_dots<FMT, XM>(g, u, stg, scratch, pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128));
-            // the stage is consumed: refill it with this warp's item m + S
-            __syncwarp();
-            fence_proxy_async();
-            if (ok) {
-                issue_w(m + S);
-                issue_a(m + S);
+        const uint8_t* stg = stages + st * g.stage_bytes;
+        if (u.has && !*bad) {
+            const bool got = mbar_wait_bounded(&bars[st], (uint32_t)((m / S) & 1), g.err, g.budget_ns);
+            if (!__all_sync(kFull, got)) {
+                if (lane == 0) *bad = 1;
+            } else {
+                s_dots<FMT, XM>(g, u, stg, scratch, pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128));
             }
         }
-        // every chunk partial of the item is in the first CTA
+        // every chunk partial of the item is in the first CTA, and every warp
+        // of this CTA is done with the stage
         if (g.C > 1) cluster_barrier(); else __syncthreads();
+        // refill the stage with this CTA's item m + S
+        if (warp == 0 && !*bad) {
+            if (lane == 0) {
+                fence_proxy_async();
+                issue_w(m + S);
+            }
+            __syncwarp();
+            issue_a(m + S);
+        }
         if (rank == 0) s_epilogue<OM>(g, rs, u, pbuf + (size_t)(m & 1) * units * g.T * 32);
     }
-    if (!ok) {
-        // drain: wait (bounded) for this warp's copies still in flight (the
-        // one that ran out and the S - 1 issued after it)
-        for (int j = m_fail; j < m_fail + S; ++j) {
-            const int item = cid + j * ncl;
-            if (item >= n_items) continue;
-            const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
-            if (u.has) mbar_wait_bounded(&mybar[j % S], (uint32_t)((j / S) & 1), nullptr, g.budget_ns);
-        }
+    if (*bad && threadIdx.x == 0) {
+        // drain: wait (bounded) for the last copies of every stage
+        for (int m = (issued - S + 1 > 0 ? issued - S + 1 : 0); m <= issued; ++m)
+            mbar_wait_bounded(&bars[m % S], (uint32_t)((m / S) & 1), nullptr, g.budget_ns);
     }
 }
 
