@@ -1,6 +1,8 @@
 // elq_abi.cu -- the C ABI declared in include/elq.h: host-side validation,
 // workspace layout and kernel launches.  No allocation, no synchronisation
 // (except elq_workspace_status, which is documented as blocking).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -443,8 +445,52 @@ cudaError_t launch_tc_t(const TcArgs& g, cudaStream_t s, bool pdl) {
     return launch(k_tcgemm<OM>, dim3(sm_count()), dim3(kTcThreads), (size_t)kTcSmem, s, pdl, g);
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, cuuint32_t rank, const void* base, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* box) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+    if (!fn) return false;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The four tensor maps of a k_tcgemm launch (layouts in TcArgs).  n_groups:
+// the matrices of the arena (the experts, or 1).
+bool tc_maps(TcArgs& g, int n_groups) {
+    const cuuint64_t nb = (cuuint64_t)g.nb, tiles = (cuuint64_t)n_groups * g.rtiles;
+    const cuuint64_t slots = (cuuint64_t)g.bstride;
+    const cuuint64_t da[4] = {256, 4, nb, tiles}, sa[3] = {nb * 1024, 1024, nb * 4096};
+    const cuuint32_t ba[4] = {256, 4, kTcKS, 1};
+    const cuuint64_t dd[4] = {32, 4, nb, tiles}, sd[3] = {nb * 64, 64, nb * 256};
+    const cuuint32_t bdd[4] = {32, 4, kTcKS, 1};
+    const cuuint64_t db[3] = {64, slots / 8, nb}, sb[2] = {256, slots * 32};
+    const cuuint32_t bb[3] = {64, kTcN / 8, kTcKS};
+    const cuuint64_t dbd[2] = {slots, nb}, sbd[1] = {slots * 4};
+    const cuuint32_t bbd[2] = {kTcN, kTcKS};
+    return encode_map(&g.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.q, da, sa, ba) &&
+           encode_map(&g.tm_d, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, g.d, dd, sd, bdd) &&
+           encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, g.bq, db, sb, bb) &&
+           encode_map(&g.tm_bd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, g.bd, dbd, sbd, bbd);
+}
+
 cudaError_t launch_tc(TcArgs g, cudaStream_t s, bool pdl) {
     g.budget_ns = kWaitBudgetNs;
+    if (!tc_maps(g, g.n_groups)) return cudaErrorInvalidValue;
     switch (g.out_mode) {
     case TC_OUT_F32: return launch_tc_t<TC_OUT_F32>(g, s, pdl);
     case TC_OUT_F32_Q81: return launch_tc_t<TC_OUT_F32_Q81>(g, s, pdl);
@@ -463,6 +509,7 @@ TcArgs dense_tc(const elq_qmat* w, int T, const uint8_t* bq, const float* bd, in
     g.d = static_cast<const uint16_t*>(w->d);
     g.nb = w->k / 32;
     g.rtiles = w->n_rows / kTileRows;
+    g.n_groups = 1;
     g.T = T;
     g.bq = bq;
     g.bd = bd;
@@ -584,8 +631,10 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.dec = plan_dec(ly, T);
     w.fused = !w.tc && w.dec.ok;
     w.small = false;
+    // the cluster router: up to 8 CTAs (the portable cluster size), as few
+    // experts per CTA as that allows (at most 16, one per warp)
     w.rs_C = 1;
-    while ((E + w.rs_C - 1) / w.rs_C > 8 && w.rs_C < kSMaxCluster) w.rs_C *= 2;
+    while ((E + w.rs_C - 1) / w.rs_C > 4 && w.rs_C < kSMaxCluster) w.rs_C *= 2;
     w.rs_epc = (E + w.rs_C - 1) / w.rs_C;
     if (!w.tc && !w.fused && w.raw && P <= kSMaxPairs && w.rs_epc <= kSMaxWarps &&
         rs_smem_bytes(T, L, E) + 16 <= kSSmemMax) {
@@ -980,6 +1029,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     g.d = static_cast<const uint16_t*>(ly->gate_up.d);
     g.nb = L / 32;
     g.rtiles = 2 * I / kTileRows;
+    g.n_groups = E;
     g.q_gstride = (int64_t)g.rtiles * g.nb * kQ80Slab;
     g.d_gstride = (int64_t)g.rtiles * g.nb * kTileRows;
     g.act = w.act; g.n_act = w.n_act; g.slot_off = w.slot_off; g.offsets = w.offsets; g.tt_off = w.tt_off;
@@ -995,6 +1045,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     h.d = static_cast<const uint16_t*>(ly->down.d);
     h.nb = I / 32;
     h.rtiles = L / kTileRows;
+    h.n_groups = E;
     h.q_gstride = (int64_t)h.rtiles * h.nb * kQ80Slab;
     h.d_gstride = (int64_t)h.rtiles * h.nb * kTileRows;
     h.act = w.act; h.n_act = w.n_act; h.slot_off = w.slot_off; h.offsets = w.offsets; h.tt_off = w.tt_off;

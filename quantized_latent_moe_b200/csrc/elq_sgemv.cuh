@@ -586,13 +586,27 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 1) k_route_small(RSArgs a) {
         lg[i] = (v0 != v0) ? -INFINITY : v0;          // a NaN logit ranks as -inf
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
-        const int t = i / E, ee = i - t * E;
-        const float* row = lg + t * E;
-        const float v = row[ee];
+    // rank of candidate (t, e): four lanes each count over a quarter of the
+    // row, two shuffles add the quarters
+    const int nq = (T * E + 7) / 8 * 8;             // candidates, padded so every lane quartet is whole
+    for (int base = 0; base < nq * 4; base += (int)blockDim.x) {
+        const int id = base + (int)threadIdx.x;
+        const int c = id >> 2, qd = id & 3;
         int r = 0;
-        for (int j = 0; j < E; ++j) r += (row[j] > v) | ((row[j] == v) & (j < ee));
-        if (r < k) {
+        float v = 0.0f;
+        int ee = 0, t = 0;
+        const bool live = c < T * E;
+        if (live) {
+            t = c / E;
+            ee = c - t * E;
+            const float* row = lg + t * E;
+            v = row[ee];
+            const int j0 = qd * ((E + 3) >> 2), j1 = min(E, j0 + ((E + 3) >> 2));
+            for (int j = j0; j < j1; ++j) r += (row[j] > v) | ((row[j] == v) & (j < ee));
+        }
+        r += __shfl_xor_sync(kFull, r, 1);
+        r += __shfl_xor_sync(kFull, r, 2);
+        if (live && qd == 0 && r < k) {
             sidx[t * k + r] = ee;
             sval[t * k + r] = v;
         }
@@ -611,20 +625,31 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 1) k_route_small(RSArgs a) {
     }
     if (warp == 0) bucket_warp_small(sidx, P, E, scount, soff, sperm, spos, nullptr, snact, sgrp);
     __syncthreads();
+    // the routing out to global memory: group table first (the expert
+    // kernels wait for it), then the arrays of the bucketing
     const int na = *snact;
-    for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    for (int i = threadIdx.x; i < na * kSMaxT; i += blockDim.x) {
+        const int ga = i / kSMaxT, j = i - ga * kSMaxT;
+        const int4 gq = sgrp[ga];
+        if (j == 0) {
+            a.grp[ga] = gq;
+            a.act[ga] = gq.x;
+        }
+        if (j < gq.z) a.gtok[i] = sperm[gq.y + j] / k;
+    }
+    if (threadIdx.x == 0) *a.n_act = na;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+        if (i < P) {
+            a.perm[i] = sperm[i];
+            a.pos[i] = spos[i];
+        }
+        if (i < E) a.counts[i] = scount[i];
+        a.offsets[i] = soff[i];
+    }
+    for (int i = threadIdx.x + E + 1; i < P; i += blockDim.x) {
         a.perm[i] = sperm[i];
         a.pos[i] = spos[i];
     }
-    for (int i = threadIdx.x; i < E; i += blockDim.x) a.counts[i] = scount[i];
-    for (int i = threadIdx.x; i <= E; i += blockDim.x) a.offsets[i] = soff[i];
-    for (int i = threadIdx.x; i < na; i += blockDim.x) {
-        const int4 gq = sgrp[i];
-        a.act[i] = gq.x;
-        a.grp[i] = gq;
-        for (int j = 0; j < gq.z && j < kSMaxT; ++j) a.gtok[i * kSMaxT + j] = sperm[gq.y + j] / k;
-    }
-    if (threadIdx.x == 0) *a.n_act = na;
 }
 
 template <int FMT, int XM, int OM>

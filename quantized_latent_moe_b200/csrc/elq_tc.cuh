@@ -19,6 +19,8 @@
 // layout ("B buffers": [kb][slot/8][2][8][16] codes and [kb][slot] fp32 scales).
 #pragma once
 
+#include <cuda.h>
+
 #include "elq_kernels.cuh"
 
 namespace elq {
@@ -57,6 +59,32 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Tiled tensor copies global -> shared through a tensor map (a kernel
+// parameter), completing on an mbarrier's transaction count.  No multicast.
+// The innermost coordinate is always 0 or 16-byte aligned here.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_addr(bar))
+        : "memory");
 }
 
 // 32 consecutive 32-bit TMEM columns of this thread's lane.
@@ -306,10 +334,19 @@ static_assert(kTcEpiWarps * kTcEpiCols == 4 * kTcN, "the epilogue warps cover th
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
 
 struct TcArgs {
+    // tensor maps of one stage's four copies (host-encoded):
+    //  tm_a : weight codes, uint32 [tiles][nb][4 slices][256] with strides
+    //         (nb*4096, 1024, nb*1024) bytes; box [1][4][4][256] lands as
+    //         [block][slice][1 KB], the MMA's A layout
+    //  tm_d : weight scales, uint16 [tiles][nb][4][32]; box -> [block][slice][32]
+    //  tm_b : packed activation codes, uint32 [nb][slots/8][64]; box [4][8][64]
+    //  tm_bd: activation scales, fp32 [nb][slots]; box [4][64]
+    CUtensorMap tm_a, tm_d, tm_b, tm_bd;
     const uint8_t* q;           // weight arena of group 0
     const uint16_t* d;
     int64_t q_gstride, d_gstride;
     int nb, rtiles;
+    int n_groups;               // matrices in the arena (the experts, or 1)
     // groups: dense (act == NULL: one group of T tokens in slots 0 .. T-1) or
     // the routed experts (slot_off/counts per expert, tt_off per active expert)
     const int32_t* act;
@@ -402,7 +439,7 @@ __device__ __noinline__ int tc_qcode(float h, float d) {
 }
 
 template <int OM>
-__global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
+__global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant__ TcArgs g) {
     extern __shared__ __align__(1024) uint8_t tcsm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(tcsm);            // [stages]
     uint64_t* empty = full + kTcStages;                             // [stages]
@@ -474,23 +511,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                         break;
                     }
                     uint8_t* st = stages + s * kTcStage;
-                    const uint32_t bbytes = (uint32_t)un.ncols * 32u, dabytes = (uint32_t)un.ncols * 4u;
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)kTcStageA + kTcStageDw + kTcKS * (bbytes + dabytes));
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)kTcStage);
                     const int kb0 = ks * kTcKS;
-                    for (int kl = 0; kl < kTcKS; ++kl)
-                        for (int sl = 0; sl < 4; ++sl)
-                            bulk_g2s(st + kl * 4096 + sl * 1024, qa + ((int64_t)sl * g.nb + kb0 + kl) * 1024, 1024,
-                                     &full[s]);
-                    for (int sl = 0; sl < 4; ++sl)
-                        bulk_g2s(st + kTcStageA + sl * kTcKS * 64, da + (int64_t)sl * g.nb * 32 + kb0 * 32,
-                                 kTcKS * 64, &full[s]);
-                    for (int kl = 0; kl < kTcKS; ++kl) {
-                        const int kb = kb0 + kl;
-                        bulk_g2s(st + kTcStageA + kTcStageDw + kl * kTcN * 32,
-                                 g.bq + (int64_t)kb * g.bstride * 32 + (int64_t)un.slot0 * 32, bbytes, &full[s]);
-                        bulk_g2s(st + kTcStageA + kTcStageDw + kTcStageB + kl * kTcN * 4,
-                                 g.bd + (int64_t)kb * g.bstride + un.slot0, dabytes, &full[s]);
-                    }
+                    const int tile = un.e * g.rtiles + un.rt;
+                    tma_load_4d(st, &g.tm_a, 0, 0, kb0, tile, &full[s]);
+                    tma_load_4d(st + kTcStageA, &g.tm_d, 0, 0, kb0, tile, &full[s]);
+                    tma_load_3d(st + kTcStageA + kTcStageDw, &g.tm_b, 0, un.slot0 >> 3, kb0, &full[s]);
+                    tma_load_2d(st + kTcStageA + kTcStageDw + kTcStageB, &g.tm_bd, un.slot0, kb0, &full[s]);
                 }
             }
         }
@@ -567,7 +594,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(TcArgs g) {
                     tmem_ld16(tb + (uint32_t)(kl * kTcN), rc);
                     tmem_ld_wait();
                     // block kl of the stage: part = fmaf(isum, d_w * d_a, part) per column, two at a time
-                    const float dw = h2f(dws[sp * kTcKS * 32 + kl * 32 + lane]);
+                    const float dw = h2f(dws[kl * kTileRows + sp * 32 + lane]);
                     const uint64_t dw2 = f2_pack(dw, dw);
                     const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
 #pragma unroll
