@@ -573,6 +573,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 #pragma unroll
             for (int j = 0; j < kTcEpiCols / 2; ++j) { acc2[j] = 0ull; part2[j] = 0ull; }
             bool ok = true;
+            const bool active = c0 < un.ncols;
             const uint32_t tlane = (uint32_t)(sp * 32) << 16;
             const uint64_t seed2 = f2_pack(kAccSeedF, kAccSeedF);
             for (int ks = 0; ks < kstages; ++ks, ++it) {
@@ -588,29 +589,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                 const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
                 const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
                 const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + c0);
+                // column groups past the tile's tokens hold no MMA result (and keep the seed)
+                if (active) {
 #pragma unroll
-                for (int kl = 0; kl < kTcKS; ++kl) {
-                    uint32_t rc[kTcEpiCols];
-                    tmem_ld16(tb + (uint32_t)(kl * kTcN), rc);
-                    tmem_ld_wait();
-                    // block kl of the stage: part = fmaf(isum, d_w * d_a, part) per column, two at a time
-                    const float dw = h2f(dws[kl * kTileRows + sp * 32 + lane]);
-                    const uint64_t dw2 = f2_pack(dw, dw);
-                    const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
+                    for (int kp = 0; kp < kTcKS; kp += 2) {
+                        // two blocks' accumulators per wait
+                        uint32_t rc[2][kTcEpiCols];
+                        tmem_ld16(tb + (uint32_t)(kp * kTcN), rc[0]);
+                        tmem_ld16(tb + (uint32_t)((kp + 1) * kTcN), rc[1]);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
-                        const float4 dv = dak[j4];
-                        const uint64_t i0 = f2_sub(f2_pack(__uint_as_float(rc[4 * j4]), __uint_as_float(rc[4 * j4 + 1])), seed2);
-                        const uint64_t i1 =
-                            f2_sub(f2_pack(__uint_as_float(rc[4 * j4 + 2]), __uint_as_float(rc[4 * j4 + 3])), seed2);
-                        part2[2 * j4] = f2_fma(i0, f2_mul(dw2, f2_pack(dv.x, dv.y)), part2[2 * j4]);
-                        part2[2 * j4 + 1] = f2_fma(i1, f2_mul(dw2, f2_pack(dv.z, dv.w)), part2[2 * j4 + 1]);
+                        for (int h = 0; h < 2; ++h) {
+                            const int kl = kp + h;
+                            // block kl of the stage: part = fmaf(isum, d_w * d_a, part) per column, two at a time
+                            const float dw = h2f(dws[kl * kTileRows + sp * 32 + lane]);
+                            const uint64_t dw2 = f2_pack(dw, dw);
+                            const float4* dak = reinterpret_cast<const float4*>(das + kl * kTcN + c0);
+#pragma unroll
+                            for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
+                                const float4 dv = dak[j4];
+                                const uint64_t i0 = f2_sub(
+                                    f2_pack(__uint_as_float(rc[h][4 * j4]), __uint_as_float(rc[h][4 * j4 + 1])), seed2);
+                                const uint64_t i1 = f2_sub(
+                                    f2_pack(__uint_as_float(rc[h][4 * j4 + 2]), __uint_as_float(rc[h][4 * j4 + 3])), seed2);
+                                part2[2 * j4] = f2_fma(i0, f2_mul(dw2, f2_pack(dv.x, dv.y)), part2[2 * j4]);
+                                part2[2 * j4 + 1] = f2_fma(i1, f2_mul(dw2, f2_pack(dv.z, dv.w)), part2[2 * j4 + 1]);
+                            }
+                        }
                     }
-                }
-                // the group's accumulators back to the seed for its next MMAs
+                    // the group's accumulators back to the seed for its next MMAs
 #pragma unroll
-                for (int kl = 0; kl < kTcKS; ++kl) tmem_st16_const(tb + (uint32_t)(kl * kTcN), kAccSeed);
-                tmem_st_wait();
+                    for (int kl = 0; kl < kTcKS; ++kl) tmem_st16_const(tb + (uint32_t)(kl * kTcN), kAccSeed);
+                    tmem_st_wait();
+                }
                 // a run of 8 blocks ends with every second stage (and with the last)
                 if ((ks & 1) || ks == kstages - 1) {
 #pragma unroll
@@ -638,7 +649,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
             const int64_t slot0 = un.slot0;
             if (OM == TC_OUT_SWIGLU) {
                 // transpose the tile's accumulators through shared memory ([token][row], padded), then
-                // each of the first 128 epilogue threads builds one Q8_1 block of h = silu(gate) * up:
+                // the epilogue threads build the Q8_1 blocks of h = silu(gate) * up, four per block:
                 // h row 32*hb + i of token t takes gate row 32*hb + i and up row 64 + 32*hb + i
                 if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
                     *abort_v = 1;
@@ -652,38 +663,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     *abort_v = 1;
                     break;
                 }
-                const int task = ew * 32 + lane;            // 0 .. 255: (token, h block)
-                const int t = task >> 1, hb = task & 1;
-                if (task < 2 * kTcN && t < nv) {
-                    const float* gr = xchg + t * kTcXld + hb * 32;
-                    const float* ur = gr + 64;
-                    float h[32];
+                // all 512 epilogue threads: four lanes per (token, h block),
+                // eight values each; amax and the code sum by two shuffles
+                {
+                    const int task = ew * 32 + lane;        // 0 .. 511
+                    const int b = task >> 2, qd = task & 3;  // block (token t, half hb), quarter
+                    const int t = b >> 1, hb = b & 1;
+                    const bool on = t < nv;
+                    float h[8];
                     float amax = 0.0f;
+                    if (on) {
+                        const float* gr = xchg + t * kTcXld + hb * 32 + qd * 8;
+                        const float* ur = gr + 64;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        h[i] = tc_swiglu(gr[i], ur[i]);
-                        amax = fmaxf(amax, fabsf(h[i]));
+                        for (int i = 0; i < 8; ++i) {
+                            h[i] = tc_swiglu(gr[i], ur[i]);
+                            amax = fmaxf(amax, fabsf(h[i]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) h[i] = 0.0f;
                     }
+                    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+                    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
                     const float d = __fdiv_rn(amax, 127.0f);
-                    uint32_t wq[8];
-                    int sum = 0;
+                    uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-                    for (int w4 = 0; w4 < 8; ++w4) wq[w4] = 0;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         int q = 0;
                         if (d != 0.0f) q = tc_qcode(h[i], d);
-                        sum += q;
-                        wq[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+                        if (i < 4) w0 |= (uint32_t)(q & 0xff) << (8 * i);
+                        else w1 |= (uint32_t)(q & 0xff) << (8 * (i - 4));
                     }
-                    (void)sum;
-                    const int64_t slot = slot0 + t;
-                    const int kbh = un.rt * 2 + hb;
-                    uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
-                    *reinterpret_cast<uint4*>(dst + 128) = make_uint4(wq[4], wq[5], wq[6], wq[7]);
-                    // the activation scale as the down projection reads it: fp32 of the stored fp16
-                    g.cd[(int64_t)kbh * g.cstride + slot] = __half2float(__float2half_rn(d));
+                    if (on) {
+                        const int64_t slot = slot0 + t;
+                        const int kbh = un.rt * 2 + hb;
+                        // codes 8 qd .. 8 qd + 7 of the slot's 32: first or second 16-byte half, low or high 8 bytes
+                        uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 32 + (slot >> 3) * 256 + (qd >> 1) * 128 +
+                                       (slot & 7) * 16 + (qd & 1) * 8;
+                        *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+                        // the activation scale as the down projection reads it: fp32 of the stored fp16
+                        if (qd == 0) g.cd[(int64_t)kbh * g.cstride + slot] = __half2float(__float2half_rn(d));
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(xempty);
