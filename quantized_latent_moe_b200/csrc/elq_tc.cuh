@@ -433,10 +433,7 @@ __device__ __forceinline__ int tc_units(const TcArgs& g) {
 // of their code instead of one per column (the kernels' instruction
 // footprint).
 __device__ __noinline__ void tc_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
-__device__ __noinline__ float tc_swiglu(float g, float u) { return __fmul_rn(silu_f32(g), u); }
-__device__ __noinline__ int tc_qcode(float h, float d) {
-    return (int)fminf(fmaxf(roundf(__fdiv_rn(h, d)), -127.0f), 127.0f);
-}
+
 
 template <int OM>
 __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant__ TcArgs g) {
@@ -677,7 +674,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                         const float* ur = gr + 64;
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            h[i] = tc_swiglu(gr[i], ur[i]);
+                            h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
                             amax = fmaxf(amax, fabsf(h[i]));
                         }
                     } else {
@@ -691,7 +688,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         int q = 0;
-                        if (d != 0.0f) q = tc_qcode(h[i], d);
+                        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(h[i], d)), -127.0f), 127.0f);
                         if (i < 4) w0 |= (uint32_t)(q & 0xff) << (8 * i);
                         else w1 |= (uint32_t)(q & 0xff) << (8 * (i - 4));
                     }
