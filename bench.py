@@ -41,10 +41,11 @@ sys.path.insert(0, ROOT)
 METRIC = "latent-MoE layer tokens/s; expert-weight HBM GB/s and % of B200 peak"
 KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
-KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "proj_U"]
+KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "combine",
+              "proj_U"]
 KERNELS_FUSED = ["layer"]
 KERNEL_NAMES = {"gate_up": {5: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
-                            9: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
+                            10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 
 
@@ -440,7 +441,7 @@ def run_elq(args):
     graphs = GraphSet(G, step)
 
     launches_per_step = layers[0].kernel_count(wl.T)
-    KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[launches_per_step]
+    KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 10: KERNELS_TC}[launches_per_step]
     pos = graphs.run(args.warmup)
     # every graph the timed steps replay is captured, instantiated and
     # replayed once here: the timed region holds replays only
@@ -556,12 +557,12 @@ def run_elq(args):
             dn_ms = kern_ms[KERNELS.index("down")]
         if launches_per_step == 1:
             pass
-        elif launches_per_step == 9:
+        elif launches_per_step == 10:
             # tensor-core path: gate/up is a contraction; int8 peak = measured bf16 x the nominal 2x ratio
             gu_ops = 2.0 * (2 * wl.I) * P * wl.L
             tpk, tkind = tensor_peak_int8()
             achieved = gu_ops / (gu_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][9], "achieved": achieved, "peak": tpk,
+            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][10], "achieved": achieved, "peak": tpk,
                     "peak_kind": tkind, "unit": "TOPS (int8)", "frac": achieved / tpk,
                     "traffic": traffic_for("gate_up_tc", wl.name), "algorithmic_ops_per_launch": gu_ops,
                     "algorithmic_bytes_per_launch": gu_w}
@@ -736,7 +737,7 @@ def run_stack(args):
         value = tokens / (dev_ms / 1e3)
         hbm_peak, peak_kind = peaks()
         step_s = dev_ms / 1e3 / args.steps
-        names = {5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 9: KERNELS_TC}[nk]
+        names = {5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 10: KERNELS_TC}[nk]
         gu_ms = kern_ms[names.index("gate_up")]
         P = wl.T * wl.k
         gu_bytes = n_act[0] * 2 * wl.I * nb_L * blk + wl.T * nb_L * 36 + P * nb_I * 36
@@ -757,7 +758,7 @@ def run_stack(args):
             "layer_weight_frac": step_bytes / step_s / 1e9 / hbm_peak,
             "kernel_ms": dict(zip(names, kern_ms)),
             "distinct_experts_per_layer": statistics.mean(n_act),
-            "roofline": {"bound": "hbm", "kernel": ("k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU), T=%d" if nk == 9
+            "roofline": {"bound": "hbm", "kernel": ("k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU), T=%d" if nk == 10
                                                    else "k_wgemv<" + wl.fmt.upper() + "> gate/up (+SwiGLU, Q8_1), T=%d")
                                                   % wl.T,
                          "achieved": achieved, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",

@@ -285,7 +285,7 @@ size_t elq_stack_workspace_bytes(const elq_layer* layer, int32_t T);
  * latent Q8_1), router (+ top-k, bucketing), gate/up (+ SwiGLU, Q8_1), down
  * (+ weighted combine, Q8_1), U projection.  Tensor-core path (T >= 16 and
  * every matrix Q8_0): activation quantiser, x packing, D, router, slot map, z
- * packing, gate/up, down (+ combine), U. */
+ * packing, gate/up, down, weighted combine, U. */
 int32_t elq_layer_kernel_count(const elq_layer* layer, int32_t T);
 
 /* elq_moe_layer that also records CUDA events on the stream: events[0] before

@@ -1051,13 +1051,17 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     h.act = w.act; h.n_act = w.n_act; h.slot_off = w.slot_off; h.offsets = w.offsets; h.tt_off = w.tt_off;
     h.T = T;
     h.bq = w.bhq; h.bd = w.bhd; h.bstride = w.sstride;
-    h.out_mode = TC_OUT_F32_COMBINE;
+    h.out_mode = TC_OUT_F32;           // o by slot; the combine follows
     h.y = w.o; h.y_ld = L;
-    h.cq = w.byq; h.cd = w.byd; h.cstride = w.tstride;
-    h.wts = wts; h.perm = w.perm; h.pair_slot = w.pair_slot; h.kslots = k; h.cnt_comb = w.cnt_comb_tc;
-    h.ylat = y_lat; h.ylq = w.ylq;
     h.err = w.err;
     if (launch_tc(h, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    CombArgs c;
+    std::memset(&c, 0, sizeof(c));
+    c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
+    c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
+    const int64_t warps = (int64_t)T * (L / 32);
+    if (launch(k_tc_combine, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+        return ELQ_ERR_CUDA;
     return ELQ_OK;
 }
 
@@ -1068,7 +1072,7 @@ bool layer_tc(const elq_layer* ly, int T) {
 bool layer_fused(const elq_layer* ly, int T) { return !layer_tc(ly, T) && plan_dec(ly, T).ok; }
 
 int layer_kernels(const elq_layer* ly, int T) {
-    if (layer_tc(ly, T)) return 9;
+    if (layer_tc(ly, T)) return 10;
     if (layer_fused(ly, T)) return 1;
     return T <= kRawMaxT ? 5 : 6;
 }

@@ -781,6 +781,57 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
     pdl_trigger();
 }
 
+// ---- a9 on the tensor-core path: the weighted combine --------------------------
+//
+// One warp per (token, 32-row latent block), lane = row: y_lat = fmaf(w_j,
+// o_j, y_lat) over the token's k pairs in rank order (o read by the pair's
+// slot), then its Q8_1 block, written both row-major (ylq) and into the
+// packed buffer the U projection reads (slot = token).
+struct CombArgs {
+    const float* o;             // [slots][L] by slot
+    const float* wts;           // [T][k]
+    const int32_t* pair_slot;   // [T*k]
+    int T, L, k;
+    float* ylat;                // [T][L]
+    uint8_t* ylq;               // [T][L/32] Q8_1
+    uint8_t* cq;                // packed codes [L/32][cstride]
+    float* cd;                  // packed scales [L/32][cstride]
+    int64_t cstride;
+};
+
+__global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nbl = a.L / 32;
+    if (wid >= (int64_t)a.T * nbl) return;
+    const int t = (int)(wid / nbl), blk = (int)(wid - (int64_t)t * nbl);
+    float acc = 0.0f;
+    for (int j0 = 0; j0 < a.k; j0 += 8) {
+        float ov[8], wv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (j0 + q < a.k) {
+                const int pj = t * a.k + j0 + q;
+                wv[q] = __ldg(a.wts + pj);
+                ov[q] = __ldcg(a.o + (int64_t)__ldg(a.pair_slot + pj) * a.L + blk * 32 + lane);
+            }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (j0 + q < a.k) acc = __fmaf_rn(wv[q], ov[q], acc);
+    }
+    a.ylat[(int64_t)t * a.L + blk * 32 + lane] = acc;
+    uint8_t* qb = a.ylq + ((int64_t)t * nbl + blk) * 36;
+    warp_quant_q8_1(acc, qb);
+    __syncwarp();
+    // the same block, packed for the U projection
+    uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 32 + ((int64_t)t >> 3) * 256 + (t & 7) * 16;
+    if (lane < 8)
+        reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] = reinterpret_cast<const uint32_t*>(qb + 4)[lane];
+    if (lane == 0) a.cd[(int64_t)blk * a.cstride + t] = h2f(*reinterpret_cast<const uint16_t*>(qb));
+}
+
 // ---- measurement: the int8 tensor-core rate ------------------------------------
 //
 // One CTA per SM (the launch asks for enough shared memory to keep it alone),

@@ -80,7 +80,7 @@ def test_layer_validation(L):
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(E=128, k=16, flags=1)), 8) == 5  # 128 pairs
     assert L.elq_layer_kernel_count(ctypes.byref(good), 9) == 6
     assert L.elq_layer_kernel_count(ctypes.byref(good), 15) == 6
-    assert L.elq_layer_kernel_count(ctypes.byref(good), 16) == 9                 # tensor cores from 16 tokens
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 16) == 10                # tensor cores from 16 tokens
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(fmt=2)), 32) == 6         # Q4_0 stays on the GEMV path
     assert L.elq_layer_kernel_count(None, 4) == 0
     assert L.elq_layer_kernel_count(ctypes.byref(_layer(L_=2176)), 4) == 0      # router rows: L <= 2048

@@ -177,7 +177,7 @@ def _check_intermediates(E, ly, T, tr):
     assert np.array_equal(v("pos"), tr["pos"])
     # hq and o are stored by pair position on the GPU, by pair id in the trace
     # (the tensor-core path keeps them in padded per-expert slots instead)
-    if ly.kernel_count(T) != 9:
+    if ly.kernel_count(T) != 10:
         pos = tr["pos"]
         assert np.array_equal(v("hq").reshape(T * ly.k, -1)[pos], tr["hq"])
         assert np.array_equal(v("o").reshape(T * ly.k, -1)[pos], tr["o"])
@@ -210,13 +210,13 @@ def test_layer_exact(E, orc, name, fused):
                                     ("verify", 24)])
 def test_layer_exact_larger_T(E, orc, name, T):
     """Above 8 tokens the activation quantiser runs as its own kernel; from 16
-    tokens Q8_0 layers take the tensor-core path (nine kernels), Q4_0 layers
+    tokens Q8_0 layers take the tensor-core path (ten kernels), Q4_0 layers
     stay on the GEMV path."""
     wl = synth.WORKLOADS[name]
     ly = gpu_layer(wl)
     x = synth.make_x(wl, T=T)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
-    assert ly.kernel_count(T) == (9 if (wl.fmt == "q8_0" and T >= 16) else 6)
+    assert ly.kernel_count(T) == (10 if (wl.fmt == "q8_0" and T >= 16) else 6)
     ol = oracle_layer(orc, wl, experts=[])
     tr = oracle_forward(orc, ol, wl, x.float().numpy(), trace=True)
     _check_intermediates(E, ly, T, tr)

@@ -34,7 +34,7 @@ def test_tc_latent_proj_exact(E, orc, N, K, T):
 def test_tc_layer_tiny_exact(E, orc, T):
     wl = synth.WORKLOADS["tiny"]
     ly = gpu_layer(wl)
-    assert ly.kernel_count(T) == 9
+    assert ly.kernel_count(T) == 10
     x = synth.make_x(wl, T=T)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
     assert E.workspace_status(ly.workspace(T)) == 0
