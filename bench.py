@@ -44,7 +44,8 @@ KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "combine",
               "proj_U"]
 KERNELS_FUSED = ["layer"]
-KERNEL_NAMES = {"gate_up": {5: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)", 6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
+KERNEL_NAMES = {"gate_up": {5: "k_sgemv<{fmt}> gate/up (cluster GEMV, +SwiGLU, Q8_1)",
+                            6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
                             10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 

@@ -82,14 +82,45 @@ def test_stack_matches_layer_calls(E, orc):
     assert torch.equal(h, r)
 
 
-def test_stack_stays_finite_over_48_layers(E):
-    """With the normalised layer input the residual stream of the stack
-    workload's shape stays finite over all 48 layers (unnormalised, a layer's
-    output grows with the square of its input and the stream diverges)."""
+def _oracle_layer_on_demand(orc, wl, layer):
+    """Oracle layer whose experts are drawn when a routing needs them (drawn
+    by the input recipe on the GPU and copied over: the same bits as on the
+    host; the oracle quantises them itself)."""
+    from helpers import ORC_FMT
+    dw = synth.dense_weights(wl, layer)
+    w = {kk: (None if v is None else v.numpy()) for kk, v in dw.items()}
+    w["gate"] = None
+    return orc.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, ORC_FMT[wl.fmt], ORC_FMT[wl.fmt], w)
+
+
+def _add_experts_drawn_on_gpu(ol, wl, experts, layer):
+    g, u, d = [None] * wl.E, [None] * wl.E, [None] * wl.E
+    for e in experts:
+        if ol.gate[e] is None:
+            a, b, c = synth.expert_weights(wl, int(e), layer, device="cuda")
+            g[e], u[e], d[e] = a.cpu().numpy(), b.cpu().numpy(), c.cpu().numpy()
+    ol.set_experts({"gate": g, "up": u, "down": d}, [e for e in experts if g[e] is not None])
+
+
+def test_stack_48_layers_steps_0_and_63(E, orc):
+    """The stack workload at full depth: 48 distinct layers (each with its own
+    128 experts, about 36 GB of arena), the step-0 and step-63 token batches
+    of 32 tokens each; the oracle follows two tokens of each step through all
+    48 layers (rms-normalised input, fp32 residual), drawing each layer's
+    experts as its routing needs them.  Exact, and finite everywhere."""
     wl = synth.WORKLOADS["stack"]
-    base = gpu_layer(wl, layer=0)
-    layers = [base] * wl.layers
-    x = synth.make_x(wl, step=3).cuda()
-    h = E.moe_stack(layers, x)
-    assert torch.isfinite(h).all()
-    assert E.workspace_status(base.stack_workspace(wl.T)) == 0
+    layers = [gpu_layer(wl, layer=l) for l in range(wl.layers)]
+    ols = [_oracle_layer_on_demand(orc, wl, l) for l in range(wl.layers)]
+    for step, rows in ((0, [0, 31]), (wl.steps - 1, [5, 17])):
+        x = synth.make_x(wl, step=step)
+        h = E.moe_stack(layers, x.cuda()).cpu().numpy()
+        assert E.workspace_status(layers[0].stack_workspace(wl.T)) == 0
+        assert np.isfinite(h).all()
+        r = x.float().numpy()[rows]
+        for l in range(wl.layers):
+            ol = ols[l]
+            xn = orc.rmsnorm(r)
+            idx, _ = ol.route(xn)
+            _add_experts_drawn_on_gpu(ol, wl, sorted(set(idx.reshape(-1).tolist())), l)
+            r = (r + ol.forward(xn)).astype(np.float32)
+        assert np.array_equal(h[rows], r), step
