@@ -65,6 +65,8 @@ def parse():
                     help="small T as the single persistent kernel instead of the separate-kernel sequence")
     ap.add_argument("--no-clocks", action="store_true",
                     help="no nvidia-smi sampling (for runs under a profiler; the line is then not a bench value)")
+    ap.add_argument("--no-long", action="store_true",
+                    help="skip the long-run median (for runs under a profiler)")
     return ap.parse_args()
 
 
@@ -464,7 +466,7 @@ def run_elq(args):
     if world > 1:
         dist.barrier()
     dev_ms = e0.elapsed_time(e1)
-    long_run = graphs.long_run(stream, pos)
+    long_run = None if args.no_long else graphs.long_run(stream, pos)
 
     # end to end through the C ABI with host buffers: pinned x in, y out, every step
     x_host = [x.cpu().pin_memory() for x in xs[:8]]
