@@ -273,6 +273,36 @@ def tensor_peak_int8():
     return _INT8_PEAK
 
 
+_F32X2_RATE = None
+
+
+def f32x2_rate():
+    """Packed fp32 instructions per second (fma.rn.f32x2, each two fused
+    multiply-adds), measured on this GPU: 2 CTAs of 1024 threads per SM, 8
+    independent chains per thread (elq_test_f32x2_rate), timed with CUDA
+    events on the launching stream; the best of five launches."""
+    global _F32X2_RATE
+    if _F32X2_RATE is not None:
+        return _F32X2_RATE
+    import torch
+    from quantized_latent_moe_b200 import elq
+    stream = torch.cuda.current_stream()
+    n = 4096
+    instr = 2.0 * elq.sm_count() * 1024 * n * 8
+    elq.test_f32x2_rate(64)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        elq.test_f32x2_rate(n)
+        e1.record(stream)
+        e1.synchronize()
+        best = max(best, instr / (e0.elapsed_time(e1) / 1e3))
+    _F32X2_RATE = best
+    return best
+
+
 def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_latent_moe_b200", "csrc")
@@ -569,6 +599,25 @@ def run_elq(args):
                     "peak_kind": tkind, "unit": "TOPS (int8)", "frac": achieved / tpk,
                     "traffic": traffic_for("gate_up_tc", wl.name), "algorithmic_ops_per_launch": gu_ops,
                     "algorithmic_bytes_per_launch": gu_w}
+            # the launch's three bounds: int8 tensor ops, HBM bytes, and the
+            # fp32 epilogue (per 32-value block of every output element one
+            # int-to-float subtract, one scale product and one fused
+            # multiply-add, as packed pairs: 1.5 fma.rn.f32x2-rate
+            # instructions per element-block)
+            gu_io = gu_w + wl.T * nb_L * 36 + P * nb_I * 36
+            elem_blocks = float(P) * (2 * wl.I) * nb_L
+            f2r = f32x2_rate()
+            t_tensor = gu_ops / (tpk * 1e12)
+            t_hbm = gu_io / (hbm_peak * 1e9)
+            t_epi = elem_blocks * 1.5 / f2r
+            t_meas = gu_ms / 1e3
+            roof["fractions"] = {
+                "tensor": t_tensor / t_meas, "hbm": t_hbm / t_meas, "epilogue": t_epi / t_meas,
+                "max_bound": max(t_tensor, t_hbm, t_epi) / t_meas,
+                "bound_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6, "epilogue": t_epi * 1e6},
+                "f32x2_instr_per_s": f2r, "hbm_bytes_per_launch": gu_io, "element_blocks_per_launch": elem_blocks,
+                "note": "each fraction = that bound's time / the launch's event-timed time; the epilogue bound "
+                        "uses the measured fma.rn.f32x2 instruction rate"}
         else:
             gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
             achieved = gu_bytes / (gu_ms / 1e3) / 1e9

@@ -348,6 +348,13 @@ elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q
  * zero before the call, ELQ_ERR_TIMEOUT's code 1 if a wait ran out. */
 elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
 
+/* The packed fp32 rate, for the tensor-core epilogue's bound: 2 * SM count
+ * CTAs of 1024 threads, each thread running n iterations of 8 independent
+ * fma.rn.f32x2 instructions.  The caller times the launch on `stream` and
+ * divides 2 * elq_sm_count() * 1024 * n * 8 instructions by the time.  sink:
+ * device fp32 [2 * elq_sm_count() * 1024]. */
+elq_status elq_test_f32x2_rate(int32_t n, float* sink, void* stream);
+
 /* Streaming multiprocessors of the current device (the grid the persistent
  * kernels use). */
 int32_t elq_sm_count(void);

@@ -1455,6 +1455,12 @@ elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void
                               kWaitBudgetNs));
 }
 
+elq_status elq_test_f32x2_rate(int32_t n, float* sink, void* stream) {
+    if (n < 1 || !sink) return ELQ_ERR_INVALID_ARG;
+    return cuda_status(launch(k_test_f32x2_rate, dim3(2 * sm_count()), dim3(1024), 0,
+                              static_cast<cudaStream_t>(stream), false, (int)n, sink));
+}
+
 int32_t elq_sm_count(void) { return sm_count(); }
 
 elq_status elq_test_expf(const float* in, float* out, int64_t n, void* stream) {

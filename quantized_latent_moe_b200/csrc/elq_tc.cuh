@@ -888,4 +888,28 @@ __global__ void __launch_bounds__(128, 1) k_test_mma_i8_rate(int n_mma, int* sin
     if (warp == 0) tmem_dealloc(tmem, 2 * kRateN);
 }
 
+// ---- measurement: the packed fp32 rate --------------------------------------
+//
+// Every thread runs n iterations of 8 independent chains of fma.rn.f32x2
+// (each instruction two fused multiply-adds); one word per thread lands in
+// sink so that the work is observable.  The caller times the launch and
+// divides threads * n * 8 instructions by the time: the epilogue bound of the
+// tensor-core GEMM is counted in these instructions.
+__global__ void __launch_bounds__(1024) k_test_f32x2_rate(int n, float* sink) {
+    uint64_t a[8], b = f2_pack(1.0000001f, 0.9999999f), c = f2_pack(1e-7f, -1e-7f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = f2_pack((float)threadIdx.x + j, (float)blockIdx.x - j);
+    for (int i = 0; i < n; ++i) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[j] = f2_fma(a[j], b, c);
+    }
+    float lo, hi, acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        f2_unpack(a[j], lo, hi);
+        acc = __fadd_rn(acc, __fadd_rn(lo, hi));
+    }
+    sink[(int64_t)blockIdx.x * blockDim.x + threadIdx.x] = acc;
+}
+
 }  // namespace elq

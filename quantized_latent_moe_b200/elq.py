@@ -69,6 +69,7 @@ SIGNATURES = {
     "elq_test_expf": (I32, [V, V, I64, V]),
     "elq_test_mma_i8_rate": (I32, [I32, V, V, V]),
     "elq_sm_count": (I32, []),
+    "elq_test_f32x2_rate": (I32, [I32, V, V]),
     "elq_test_fused_timeout": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, ctypes.c_uint64, V]),
 }
 
@@ -415,6 +416,14 @@ def test_mma_i8_rate(n_mma: int, device="cuda", stream=None):
     err = torch.zeros(1, dtype=torch.int32, device=device)
     _ck(_lib().elq_test_mma_i8_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_i8_rate")
     return sink, err
+
+
+def test_f32x2_rate(n: int, device="cuda", stream=None) -> torch.Tensor:
+    """Launches the packed-fp32 rate kernel (elq_test_f32x2_rate) on the
+    current stream; returns its sink.  The caller times it."""
+    sink = torch.empty(2 * sm_count() * 1024, dtype=torch.float32, device=device)
+    _ck(_lib().elq_test_f32x2_rate(n, _ptr(sink), _stream(stream)), "elq_test_f32x2_rate")
+    return sink
 
 
 def sm_count() -> int:

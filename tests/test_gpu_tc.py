@@ -134,3 +134,11 @@ def test_int8_rate_kernel_runs(E):
     assert int(err.item()) == 0
     s = sink.cpu()
     assert (s == s[0]).all() and int(s[0]) != 0
+
+
+def test_f32x2_rate_kernel_runs(E):
+    """The measurement kernel behind the epilogue bound runs and leaves
+    finite values."""
+    sink = E.test_f32x2_rate(16)
+    torch.cuda.synchronize()
+    assert torch.isfinite(sink).all()
