@@ -3,7 +3,7 @@
 Only the tests, the package's ``smoke()`` check and the benchmark's CPU
 baseline leg may use this package.  The CUDA library never imports, links or
 calls it, and it imports nothing from the CUDA library.  What it computes is
-stated in ``elq_oracle.h`` (readings R1-R14) and written out in
+stated in ``elq_oracle.h`` (readings R1-R21) and written out in
 ``elq_oracle.c`` as plain loops; this module only builds the C file with gcc
 and marshals numpy arrays into it.
 """
@@ -20,8 +20,8 @@ SRC = os.path.join(HERE, "elq_oracle.c")
 HDR = os.path.join(HERE, "elq_oracle.h")
 LIB = os.path.join(HERE, "libelq_oracle.so")
 
-Q4_0, Q8_0, Q8_1 = 2, 8, 9
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q8_1: 36}
+Q4_0, Q8_0, Q8_1, NVFP4 = 2, 8, 9, 100
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q8_1: 36, NVFP4: 18}
 
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC",
           "-shared", "-Wall", "-Wextra"]
@@ -57,7 +57,9 @@ class OrcLayer(ctypes.Structure):
                 ("k", ctypes.c_int), ("I", ctypes.c_int),
                 ("du_fmt", ctypes.c_int), ("ex_fmt", ctypes.c_int),
                 ("D", P), ("U", P), ("router_w", P), ("router_bias", P),
-                ("gate", P), ("up", P), ("down", P)]
+                ("gate", P), ("up", P), ("down", P),
+                ("gate_g", P), ("up_g", P), ("down_g", P),
+                ("act_gz", F32), ("act_gh", F32)]
 
 
 class OrcTrace(ctypes.Structure):
@@ -89,6 +91,14 @@ def _declare(L):
                                          P, ctypes.POINTER(OrcTrace)]),
         "orc_route": (ctypes.c_int, [ctypes.POINTER(OrcLayer), P, ctypes.c_int, P, P]),
         "orc_arena_pack": (None, [ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P]),
+        "orc_f32_to_e2m1": (ctypes.c_uint8, [F32]),
+        "orc_e2m1_to_f32": (F32, [ctypes.c_uint8]),
+        "orc_f32_to_e4m3": (ctypes.c_uint8, [F32]),
+        "orc_e4m3_to_f32": (F32, [ctypes.c_uint8]),
+        "orc_nvfp4_global": (F32, [P, I64]),
+        "orc_quantize_nvfp4": (None, [P, I64, F32, P]),
+        "orc_dequantize_nvfp4": (None, [P, I64, F32, P]),
+        "orc_qmatmul_nvfp4": (None, [P, F32, ctypes.c_int, ctypes.c_int, P, F32, ctypes.c_int, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -196,6 +206,53 @@ def bucket(idx: np.ndarray, E: int):
     return counts, offsets, perm, pos
 
 
+def f32_to_e2m1(x: float) -> int:
+    return int(lib().orc_f32_to_e2m1(float(x)))
+
+
+def e2m1_to_f32(c: int) -> float:
+    return float(lib().orc_e2m1_to_f32(int(c)))
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().orc_f32_to_e4m3(float(x)))
+
+
+def e4m3_to_f32(b: int) -> float:
+    return float(lib().orc_e4m3_to_f32(int(b)))
+
+
+def nvfp4_global(x) -> float:
+    """Global scale of a weight matrix: amax / (6 * 448), 1 when all zero (R20)."""
+    x = _f32(x)
+    return float(lib().orc_nvfp4_global(_p(x), x.size))
+
+
+def quantize_nvfp4(x, g: float = 1.0) -> np.ndarray:
+    """fp32 array (last dim % 32 == 0) -> 18-byte NVFP4 blocks under global scale g."""
+    x = _f32(x)
+    out = np.empty(x.shape[:-1] + (x.shape[-1] // 32 * 18,), np.uint8)
+    lib().orc_quantize_nvfp4(_p(x), x.size, float(g), _p(out))
+    return out
+
+
+def dequantize_nvfp4(blocks: np.ndarray, n: int, g: float) -> np.ndarray:
+    blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
+    out = np.empty(n, np.float64)
+    lib().orc_dequantize_nvfp4(_p(blocks), n, float(g), _p(out))
+    return out
+
+
+def qmatmul_nvfp4(W: np.ndarray, gw: float, N: int, K: int, Xq: np.ndarray, T: int,
+                  ga: float = 1.0) -> np.ndarray:
+    W = np.ascontiguousarray(W, np.uint8)
+    Xq = np.ascontiguousarray(Xq, np.uint8)
+    assert W.size == N * (K // 32) * 18 and Xq.size == T * (K // 32) * 18
+    Y = np.empty((T, N), np.float32)
+    lib().orc_qmatmul_nvfp4(_p(W), float(gw), N, K, _p(Xq), float(ga), T, _p(Y))
+    return Y
+
+
 def arena_pack(fmt: int, aos: np.ndarray, n_rows: int, k: int):
     aos = np.ascontiguousarray(aos, np.uint8)
     nb = k // 32
@@ -223,12 +280,26 @@ class Layer:
         self.gate = [None] * E
         self.up = [None] * E
         self.down = [None] * E
+        # NVFP4 experts: one global scale per expert gate/up pair and per down (R20)
+        self.gate_g = np.ones(E, np.float32)
+        self.down_g = np.ones(E, np.float32)
+        # and static global scales of the experts' NVFP4 inputs z and h
+        self.act_gz = float(w.get("act_gz", 1.0))
+        self.act_gh = float(w.get("act_gh", 1.0))
         self.set_experts(w, range(E))
 
     def set_experts(self, w, experts):
         for e in experts:
             g = w["gate"][e] if w.get("gate") is not None else None
             if g is None:
+                continue
+            if self.ex_fmt == NVFP4:
+                gu = np.concatenate([_f32(g).ravel(), _f32(w["up"][e]).ravel()])
+                self.gate_g[e] = nvfp4_global(gu)
+                self.down_g[e] = nvfp4_global(w["down"][e])
+                self.gate[e] = quantize_nvfp4(g, self.gate_g[e])
+                self.up[e] = quantize_nvfp4(w["up"][e], self.gate_g[e])
+                self.down[e] = quantize_nvfp4(w["down"][e], self.down_g[e])
                 continue
             self.gate[e] = quantize(self.ex_fmt, g)
             self.up[e] = quantize(self.ex_fmt, w["up"][e])
@@ -243,7 +314,8 @@ class Layer:
         return OrcLayer(self.H, self.L, self.E, self.k, self.I, self.du_fmt, self.ex_fmt,
                         _p(self.D), _p(self.U), _p(self.router_w), _p(self.router_bias),
                         ctypes.cast(self._g, P), ctypes.cast(self._u, P),
-                        ctypes.cast(self._d, P))
+                        ctypes.cast(self._d, P), _p(self.gate_g), _p(self.gate_g),
+                        _p(self.down_g), self.act_gz, self.act_gh)
 
     def route(self, x):
         x = _f32(x)
@@ -265,14 +337,15 @@ class Layer:
         tr = None
         bufs = {}
         if trace:
+            xb = 18 if self.ex_fmt == NVFP4 else 36
             bufs = dict(
                 xq=np.empty((T, H // 32 * 36), np.uint8), z=np.empty((T, L), np.float32),
                 logits=np.empty((T, E), np.float32), idx=np.empty((T, k), np.int32),
-                w=np.empty((T, k), np.float32), zq=np.empty((T, L // 32 * 36), np.uint8),
+                w=np.empty((T, k), np.float32), zq=np.empty((T, L // 32 * xb), np.uint8),
                 counts=np.empty(E, np.int32), offsets=np.empty(E + 1, np.int32),
                 perm=np.empty(P_, np.int32), pos=np.empty(P_, np.int32),
                 g=np.empty((P_, I), np.float32), u=np.empty((P_, I), np.float32),
-                hq=np.empty((P_, I // 32 * 36), np.uint8), o=np.empty((P_, L), np.float32),
+                hq=np.empty((P_, I // 32 * xb), np.uint8), o=np.empty((P_, L), np.float32),
                 y_lat=np.empty((T, L), np.float32), ylq=np.empty((T, L // 32 * 36), np.uint8))
             tr = OrcTrace(**{n: _p(a) for n, a in bufs.items()})
         s = self._struct()

@@ -22,6 +22,7 @@ int orc_block_bytes(int fmt)
     case ORC_Q4_0: return 18;
     case ORC_Q8_0: return 34;
     case ORC_Q8_1: return 36;
+    case ORC_NVFP4: return 18;
     default: return 0;
     }
 }
@@ -313,6 +314,175 @@ void orc_qmatmul(int wfmt, const uint8_t* W, int N, int K,
 }
 
 /* ------------------------------------------------------------------------ */
+/* NVFP4 (page "edge0-strata", section "Changes from upstream Strata": the  */
+/* Edge0 latent experts are NVFP4).  The pages name the format only; the    */
+/* readings R19-R21 in elq_oracle.h fix the rest.                           */
+
+/* E2M1 magnitudes by code 0..7 (sign in bit 3). */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+/* R19: fp32 -> E2M1, round to nearest with ties to the even code, finite
+ * values saturate at 6, the sign kept (a negative value rounding to 0 gives
+ * code 8, -0).  Written as the intervals of the grid's midpoints. */
+uint8_t orc_f32_to_e2m1(float v)
+{
+    uint8_t sign = (v < 0.0f) ? 8u : 0u;
+    float a = fabsf(v);
+    uint8_t c;
+    if (!(a > 0.25f)) c = 0;           /* also NaN */
+    else if (a < 0.75f) c = 1;
+    else if (a <= 1.25f) c = 2;
+    else if (a < 1.75f) c = 3;
+    else if (a <= 2.5f) c = 4;
+    else if (a < 3.5f) c = 5;
+    else if (a <= 5.0f) c = 6;
+    else c = 7;
+    return (uint8_t)(sign | c);
+}
+
+float orc_e2m1_to_f32(uint8_t c)
+{
+    float m = kE2M1[c & 7u];
+    return (c & 8u) ? -m : m;
+}
+
+/* R19: unsigned fp32 -> E4M3 (1 sign bit, 4 exponent bits with bias 7, 3
+ * fraction bits; no infinity, 0x7F is NaN), round to nearest even, finite
+ * values saturate at 448 (0x7E); NaN and non-positive values give 0.
+ * Written from the format's definition: normals 2^(e-7) * (1 + f/8) for
+ * e = 1..15, subnormals f * 2^-9. */
+uint8_t orc_f32_to_e4m3(float v)
+{
+    if (!(v > 0.0f)) return 0;
+    if (v >= 448.0f) return 0x7E;
+    uint32_t x;
+    memcpy(&x, &v, 4);
+    int e = (int)((x >> 23) & 0xFFu) - 127;       /* v = m * 2^(e-23), m 24 bits */
+    uint32_t m = (x & 0x7FFFFFu) | (((x >> 23) & 0xFFu) ? 0x800000u : 0u);
+    if (((x >> 23) & 0xFFu) == 0u) e = -126;       /* fp32 subnormal (underflows to 0 below) */
+    /* the quantum is 2^-9 below 2^-6 and 2^(e-3) above: drop bits of m */
+    int shift = (e >= -6) ? 20 : 20 + (-6 - e);    /* fraction bits kept: 3, fewer when subnormal */
+    if (shift > 24) return 0;                      /* below half the smallest subnormal */
+    uint32_t q = m >> shift;
+    uint32_t rem = m & ((1u << shift) - 1u);
+    uint32_t half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (q & 1u))) q += 1u;
+    /* q is the significand on the grid: 8..16 for normals (16 = next exponent),
+     * 0..8 for subnormals (8 = the smallest normal) */
+    int ee;
+    uint32_t f;
+    if (e >= -6) {
+        ee = e + 7;
+        if (q == 16u) { ee += 1; q = 8u; }
+        f = q - 8u;
+    } else {
+        if (q == 8u) { ee = 1; f = 0u; }
+        else { ee = 0; f = q; }
+    }
+    if (ee > 15 || (ee == 15 && f == 7u)) return 0x7E;   /* saturate */
+    return (uint8_t)((ee << 3) | f);
+}
+
+float orc_e4m3_to_f32(uint8_t b)
+{
+    int e = (b >> 3) & 15, f = b & 7;
+    if (e == 15 && f == 7) return NAN;
+    if (e == 0) return ldexpf((float)f, -9);
+    return ldexpf(1.0f + (float)f / 8.0f, e - 7);
+}
+
+/* R20: global scale of a weight matrix: amax / (6 * 448) (fp32 divide), 1 for
+ * an all-zero matrix.  Activations take 1. */
+float orc_nvfp4_global(const float* x, int64_t n)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    return amax > 0.0f ? amax / 2688.0f : 1.0f;
+}
+
+/* R20: blocks of 32 values (two 16-value micro-blocks), 18 bytes each: the
+ * two E4M3 scales, then 16 bytes of codes, value 2j in the low nibble of
+ * byte j and value 2j+1 in its high nibble.  Micro-block scale s =
+ * e4m3(amax / 6 / g) (fp32 divides), code = e2m1(x / (dec(s) * g)) (fp32
+ * product and divide); a zero scale gives zero codes. */
+void orc_quantize_nvfp4(const float* x, int64_t n, float g, uint8_t* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const float* xb = x + 32 * b;
+        uint8_t* o = out + 18 * b;
+        uint8_t codes[32];
+        for (int mb = 0; mb < 2; ++mb) {
+            float amax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(xb[16 * mb + i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t sb = orc_f32_to_e4m3((amax / 6.0f) / g);
+            o[mb] = sb;
+            float ds = orc_e4m3_to_f32(sb);
+            float den = ds * g;
+            for (int i = 0; i < 16; ++i)
+                codes[16 * mb + i] = (den != 0.0f) ? orc_f32_to_e2m1(xb[16 * mb + i] / den) : 0u;
+        }
+        for (int j = 0; j < 16; ++j)
+            o[2 + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+    }
+}
+
+/* value i of an NVFP4 block, as the doubled integer 2 * e2m1 (exact) */
+static int nv_code2(const uint8_t* blk, int i)
+{
+    uint8_t c = (uint8_t)((blk[2 + i / 2] >> ((i & 1) * 4)) & 0x0Fu);
+    static const int mag2[8] = {0, 1, 2, 3, 4, 6, 8, 12};
+    return (c & 8u) ? -mag2[c & 7u] : mag2[c & 7u];
+}
+
+void orc_dequantize_nvfp4(const uint8_t* blocks, int64_t n, float g, double* out)
+{
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const uint8_t* p = blocks + 18 * b;
+        for (int i = 0; i < 32; ++i)
+            out[32 * b + i] = (double)nv_code2(p, i) * 0.5 * (double)orc_e4m3_to_f32(p[i / 16]) * (double)g;
+    }
+}
+
+/* R21: Y[t][n] = row n of W (NVFP4, global gw) . X[t] (NVFP4, global ga).
+ * Per 16-value micro-block m: isum = sum (2 w)(2 a) exact, sc = dec(sw) *
+ * dec(sa); part = fmaf((float)isum, sc, part) over the micro-blocks of a
+ * chunk of 8 blocks (16 micro-blocks) in order from 0; acc = acc + part over
+ * the chunks in order from 0; y = acc * ((gw * ga) * 0.25). */
+void orc_qmatmul_nvfp4(const uint8_t* W, float gw, int N, int K, const uint8_t* X, float ga,
+                       int T, float* Y)
+{
+    int nb = K / 32;
+    float gq = (gw * ga) * 0.25f;
+    for (int t = 0; t < T; ++t) {
+        const uint8_t* xr = X + (int64_t)t * nb * 18;
+        for (int n = 0; n < N; ++n) {
+            const uint8_t* wr = W + (int64_t)n * nb * 18;
+            float acc = 0.0f;
+            for (int c = 0; c < nb; c += 8) {
+                float part = 0.0f;
+                for (int kb = c; kb < c + 8 && kb < nb; ++kb)
+                    for (int mb = 0; mb < 2; ++mb) {
+                        const uint8_t* wk = wr + (int64_t)kb * 18;
+                        const uint8_t* ak = xr + (int64_t)kb * 18;
+                        int32_t isum = 0;
+                        for (int i = 16 * mb; i < 16 * mb + 16; ++i) isum += nv_code2(wk, i) * nv_code2(ak, i);
+                        float sc = orc_e4m3_to_f32(wk[mb]) * orc_e4m3_to_f32(ak[mb]);
+                        part = fmaf((float)isum, sc, part);
+                    }
+                acc = acc + part;
+            }
+            Y[(int64_t)t * N + n] = acc * gq;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* router (R9-R11)                                                          */
 
 void orc_router_topk(const float* z, const float* Wr, const float* bias,
@@ -394,7 +564,10 @@ static int check_layer(const orc_layer* ly)
         ly->k > ly->E || ly->k > 64)
         return -2;
     if (!orc_block_bytes(ly->du_fmt) || !orc_block_bytes(ly->ex_fmt) ||
-        ly->du_fmt == ORC_Q8_1 || ly->ex_fmt == ORC_Q8_1)
+        ly->du_fmt == ORC_Q8_1 || ly->ex_fmt == ORC_Q8_1 || ly->du_fmt == ORC_NVFP4)
+        return -2;
+    if (ly->ex_fmt == ORC_NVFP4 && (!ly->gate_g || !ly->up_g || !ly->down_g ||
+                                    !(ly->act_gz > 0.0f) || !(ly->act_gh > 0.0f)))
         return -2;
     return 0;
 }
@@ -443,23 +616,36 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trac
     orc_qmatmul(ly->du_fmt, ly->D, L, H, xq, T, z);
     /* a3: router on the fp32 latent */
     orc_router_topk(z, ly->router_w, ly->router_bias, T, L, E, k, idx, w, lg);
-    /* a4: latent activations for the experts */
-    orc_quantize_q8_1(z, (int64_t)T * L, zq);
+    /* a4: latent activations for the experts (NVFP4 experts: NVFP4
+     * activations under the layer's static scale act_gz, R20) */
+    int nv = ly->ex_fmt == ORC_NVFP4;
+    if (nv) orc_quantize_nvfp4(z, (int64_t)T * L, ly->act_gz, zq);
+    else orc_quantize_q8_1(z, (int64_t)T * L, zq);
     /* a5 */
     orc_bucket(idx, T, k, E, counts, offsets, perm, pos);
     /* a6-a8, one (token, slot) pair at a time, in pair order */
     for (int p = 0; p < P && rc == 0; ++p) {
         int t = p / k, e = idx[p];
         if (!ly->gate[e] || !ly->up[e] || !ly->down[e]) { rc = -1; break; }
-        const uint8_t* zt = zq + (size_t)t * (L / 32) * 36;
-        orc_qmatmul(ly->ex_fmt, ly->gate[e], I, L, zt, 1, g);
-        orc_qmatmul(ly->ex_fmt, ly->up[e], I, L, zt, 1, u);
-        for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
-        orc_quantize_q8_1(h, I, hq);
-        orc_qmatmul(ly->ex_fmt, ly->down[e], L, I, hq, 1, o + (size_t)p * L);
+        if (nv) {
+            const uint8_t* zt = zq + (size_t)t * (L / 32) * 18;
+            orc_qmatmul_nvfp4(ly->gate[e], ly->gate_g[e], I, L, zt, ly->act_gz, 1, g);
+            orc_qmatmul_nvfp4(ly->up[e], ly->up_g[e], I, L, zt, ly->act_gz, 1, u);
+            for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
+            orc_quantize_nvfp4(h, I, ly->act_gh, hq);
+            orc_qmatmul_nvfp4(ly->down[e], ly->down_g[e], L, I, hq, ly->act_gh, 1, o + (size_t)p * L);
+        } else {
+            const uint8_t* zt = zq + (size_t)t * (L / 32) * 36;
+            orc_qmatmul(ly->ex_fmt, ly->gate[e], I, L, zt, 1, g);
+            orc_qmatmul(ly->ex_fmt, ly->up[e], I, L, zt, 1, u);
+            for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
+            orc_quantize_q8_1(h, I, hq);
+            orc_qmatmul(ly->ex_fmt, ly->down[e], L, I, hq, 1, o + (size_t)p * L);
+        }
+        const size_t hqb = (size_t)(I / 32) * (nv ? 18 : 36);
         if (tr && tr->g) memcpy(tr->g + (size_t)p * I, g, sizeof(float) * (size_t)I);
         if (tr && tr->u) memcpy(tr->u + (size_t)p * I, u, sizeof(float) * (size_t)I);
-        if (tr && tr->hq) memcpy(tr->hq + (size_t)p * (I / 32) * 36, hq, (size_t)(I / 32) * 36);
+        if (tr && tr->hq) memcpy(tr->hq + (size_t)p * hqb, hq, hqb);
     }
     if (rc == 0) {
         /* a9: weighted combine in rank order, then Q8_1 */
@@ -480,7 +666,7 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trac
         if (tr->logits) memcpy(tr->logits, lg, sizeof(float) * (size_t)T * E);
         if (tr->idx) memcpy(tr->idx, idx, sizeof(int32_t) * (size_t)P);
         if (tr->w) memcpy(tr->w, w, sizeof(float) * (size_t)P);
-        if (tr->zq) memcpy(tr->zq, zq, zqb);
+        if (tr->zq) memcpy(tr->zq, zq, nv ? (size_t)T * (L / 32) * 18 : zqb);
         if (tr->counts) memcpy(tr->counts, counts, sizeof(int32_t) * (size_t)E);
         if (tr->offsets) memcpy(tr->offsets, offsets, sizeof(int32_t) * (size_t)(E + 1));
         if (tr->perm) memcpy(tr->perm, perm, sizeof(int32_t) * (size_t)P);

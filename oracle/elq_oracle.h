@@ -56,6 +56,27 @@
  *      order from 0.
  *   R18 a NaN router logit ranks as -infinity, in the selection and in the
  *       softmax (ties still by lower id), so the chosen ids are always valid.
+ *
+ * NVFP4 latent experts (page "edge0-strata", section "Changes from upstream
+ * Strata": NVFP4 and Q3_K latent experts).  The pages name the format and
+ * nothing more; readings:
+ *   R19 E2M1 values (codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6; bit 3 the
+ *       sign) and E4M3 scales; conversions round to nearest with ties to the
+ *       even code and saturate finite values (6 and 448); a NaN or
+ *       non-positive scale input gives scale 0.
+ *   R20 a weight matrix (an expert's interleaved gate/up, or its down) has
+ *       one fp32 global scale g = amax / (6 * 448), 1 if all zero; the
+ *       experts' activations (the latent z and the SwiGLU output h) are NVFP4
+ *       too, each under a static fp32 global scale of the layer (act_gz for
+ *       z, act_gh for h), given with the weights as a calibrated checkpoint
+ *       carries it.  Per 16 values: s = e4m3(amax / 6 / g), code =
+ *       e2m1(x / (dec(s) * g)).  An 18-byte block holds 32 values: two
+ *       scales, then 16 bytes of codes (value 2j low nibble of byte j, 2j+1
+ *       high).
+ *   R21 row dot: per 16-value micro-block isum = sum (2w)(2a) (exact), sc =
+ *       dec(sw) * dec(sa), part = fmaf((float)isum, sc, part) over the 16
+ *       micro-blocks of a chunk of 8 blocks in order, acc = acc + part over
+ *       chunks, y = acc * ((g_w * g_a) * 0.25).
  */
 #ifndef ELQ_ORACLE_H
 #define ELQ_ORACLE_H
@@ -66,7 +87,7 @@
 extern "C" {
 #endif
 
-enum { ORC_Q4_0 = 2, ORC_Q8_0 = 8, ORC_Q8_1 = 9 };
+enum { ORC_Q4_0 = 2, ORC_Q8_0 = 8, ORC_Q8_1 = 9, ORC_NVFP4 = 100 };
 
 int      orc_block_bytes(int fmt);                /* 18, 34, 36; 0 if unknown */
 int64_t  orc_matrix_bytes(int fmt, int64_t rows, int64_t k);
@@ -105,6 +126,17 @@ void orc_router_topk(const float* z, const float* Wr, const float* bias,
 void orc_bucket(const int32_t* idx, int T, int k, int E,
                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos);
 
+/* NVFP4 (R19-R21) */
+uint8_t  orc_f32_to_e2m1(float v);
+float    orc_e2m1_to_f32(uint8_t c);
+uint8_t  orc_f32_to_e4m3(float v);
+float    orc_e4m3_to_f32(uint8_t b);
+float    orc_nvfp4_global(const float* x, int64_t n);
+void     orc_quantize_nvfp4(const float* x, int64_t n, float g, uint8_t* out);
+void     orc_dequantize_nvfp4(const uint8_t* blocks, int64_t n, float g, double* out);
+void     orc_qmatmul_nvfp4(const uint8_t* W, float gw, int N, int K, const uint8_t* X, float ga,
+                           int T, float* Y);
+
 /* One latent-MoE layer.  Weight matrices are row-major AoS blocks.
  * gate/up/down are arrays of E pointers; an expert no token selects may be
  * NULL. */
@@ -119,6 +151,13 @@ typedef struct {
     const uint8_t* const* gate; /* E x [I rows][L] */
     const uint8_t* const* up;   /* E x [I rows][L] */
     const uint8_t* const* down; /* E x [L rows][I] */
+    /* NVFP4 experts: each matrix's global scale (E entries each); gate and
+     * up of an expert share one (they are one interleaved matrix, R20) */
+    const float* gate_g;
+    const float* up_g;
+    const float* down_g;
+    float act_gz;               /* static global scales of the NVFP4 expert inputs */
+    float act_gh;
 } orc_layer;
 
 /* Optional intermediates; any pointer may be NULL. */

@@ -108,7 +108,7 @@ def permutation(seed: int, tid: int, n: int) -> torch.Tensor:
 # workloads
 
 F32, BF16 = "f32", "bf16"
-Q8_0, Q4_0 = "q8_0", "q4_0"
+Q8_0, Q4_0, NVFP4 = "q8_0", "q4_0", "nvfp4"
 
 
 @dataclass(frozen=True)
@@ -121,7 +121,7 @@ class Workload:
     E: int
     k: int
     I: int
-    fmt: str                 # weight format of D, U and the experts
+    fmt: str                 # weight format of D and U (and of the experts unless ex_fmt)
     x_dtype: str             # activation input dtype
     bias: str                # "none" | "normal" | "zipf"
     layers: int = 1
@@ -130,6 +130,11 @@ class Workload:
     zipf_c: float = 0.3
     residual: bool = False   # stack: x_{l+1} = x_l + y_l in fp32
     extra: dict = field(default_factory=dict)
+    ex_fmt: str = ""         # expert weight format when it differs from fmt
+
+    @property
+    def expert_fmt(self) -> str:
+        return self.ex_fmt or self.fmt
 
 
 WORKLOADS = {
@@ -143,12 +148,21 @@ WORKLOADS = {
     "verify": Workload("verify", 2, 6, 3072, 1280, 128, 8, 768, Q4_0, F32, "none"),
     # prefill: 2048 tokens, Zipf(1.1)-skewed router over the 128 experts
     "prefill": Workload("prefill", 3, 2048, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "zipf"),
+    # decode with NVFP4 latent experts (D/U stay Q8_0): the decode shapes
+    "decode_nvfp4": Workload("decode_nvfp4", 5, 1, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal",
+                             ex_fmt=NVFP4),
     # resident stack: 48 layers, 32 sequences decoding one token per step
     "stack": Workload("stack", 4, 32, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal",
                       layers=48, steps=64, residual=True),
 }
 
 WEIGHT_SIGMA = 0.02
+
+# Static fp32 global scales of the NVFP4 experts' inputs (the latent z and the
+# SwiGLU output h), as a calibrated checkpoint would carry them: 2^-6 puts
+# every micro-block of these workloads' activations in E4M3's normal range and
+# leaves room up to |x| = 6 * 448 / 64 = 42.
+NVFP4_ACT_GSCALE = 2.0 ** -6
 
 # tensor ids within a layer
 TID_X, TID_D, TID_U, TID_RW, TID_RB, TID_GATE, TID_UP, TID_DOWN, TID_ZIPF = range(9)
@@ -212,4 +226,6 @@ def layer_weights(wl: Workload, layer: int = 0, experts=None, device="cpu"):
     for e in es:
         gate[e], up[e], down[e] = expert_weights(wl, e, layer, device)
     w.update(gate=gate, up=up, down=down)
+    if wl.expert_fmt == NVFP4:
+        w.update(act_gz=NVFP4_ACT_GSCALE, act_gh=NVFP4_ACT_GSCALE)
     return w
