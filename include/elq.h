@@ -42,11 +42,23 @@
  *   Q4_0 : fp16 d, uint8 nib[16]                 x = d * (q - 8)      18 B
  *          byte j holds q[j] (low nibble) and q[j+16] (high nibble)
  *   Q8_1 : fp16 d, fp16 s, int8 q[32]            s = d * sum(q)       36 B
+ *   NVFP4: uint8 s[2], uint8 nib[16]          32 values as two micro-blocks  18 B
+ *          of 16; s[m] the E4M3 scale of micro-block m; byte j holds the
+ *          E2M1 code of value 2j (low nibble) and 2j+1 (high nibble); code
+ *          c (bit 3 the sign) stands for +-(0, 0.5, 1, 1.5, 2, 3, 4, 6)[c & 7];
+ *          x = e2m1(c) * e4m3(s[m]) * g, g the fp32 global scale of the
+ *          tensor ("edge0-strata/EDGE0.md", section "Changes from upstream
+ *          Strata": NVFP4 latent experts; the pages give no more, the layout
+ *          and the rules below are this library's reading)
  *   Quantisation of a block: amax = max |x|; Q8: d = amax / 127 (fp32,
  *   correctly rounded), q = round-half-away(x / d) (correctly rounded divide),
  *   d stored as fp16 (round to nearest even); Q4_0: m = the element of largest
  *   |x| (lowest index on ties), d = m / -8, q = clamp(round(x / d) + 8, 0, 15).
- *   A zero scale gives all-zero codes (Q4_0: 8).
+ *   A zero scale gives all-zero codes (Q4_0: 8).  NVFP4 under global scale
+ *   g: per micro-block s = e4m3(amax / 6 / g) (fp32 divides; round to nearest
+ *   even, saturating at 448), code = e2m1(x / (e4m3(s) * g)) (round to nearest
+ *   even, saturating at 6; a result that rounds to zero keeps the sign of a
+ *   negative input, -0 counts as +0); s = 0 gives zero codes.
  *
  * Arithmetic
  *   Block dot of a weight block with a Q8_1 block: isum = sum q_w * q_a (Q4_0:
@@ -58,6 +70,12 @@
  *   (16, 8, 4, 2, 1), plus the bias.  Top-k by logit, lower expert id first on
  *   ties; weights are the softmax over the k selected logits.  exp() is the
  *   library's own (Cody-Waite reduction, degree-7 Taylor polynomial).
+ *   NVFP4 experts: the activations they read (z, and h of SwiGLU) are
+ *   NVFP4 under the layer's static global scales act_gz and act_gh.  Per
+ *   micro-block isum = sum (2 c_w)(2 c_a) over the 16 doubled codes (exact),
+ *   part = fmaf((float)isum, e4m3(s_w) * e4m3(s_a), part) over the chunk's 16
+ *   micro-blocks in order, the chunks added as above, and the row's result is
+ *   acc * ((g_w * g_a) * 0.25).
  *   SwiGLU h = (g / (1 + exp(-g))) * u; the weighted combine sums
  *   fmaf(w_j, o_j, acc) over the k slots in rank order.
  *
@@ -72,7 +90,10 @@
  *         no-swizzle operand layout of the tcgen05 tensor cores.
  *         Q4_0 -- a 512-byte piece at q + t*nb*2048 + s*nb*512 + kb*512; row
  *         r's 16 nibble bytes at byte 16 r of the piece, in the block's order.
- *     d : fp16 scale at element t*nb*128 + s*nb*32 + kb*32 + r.
+ *         NVFP4 -- as Q4_0: row r's 16 code bytes at byte 16 r of a
+ *         512-byte piece.
+ *     d : fp16 scale at element t*nb*128 + s*nb*32 + kb*32 + r (NVFP4: the
+ *         block's two scale bytes, s[0] the low byte).
  *   So the 8 blocks of a 32-row slice that one warp of the decode kernels
  *   reads are one contiguous bulk copy.  q and d must be 256-byte aligned.
  *   The layer's matrices (and elq_latent_proj's) need k % 128 == 0.
@@ -84,6 +105,11 @@
  *            holds gate rows 64j .. 64j+63 then up rows 64j .. 64j+63.
  *            I % 64 == 0.
  *   down   : E * L rows x I; expert e owns rows [L e, L (e+1)).
+ *   NVFP4 experts (gate_up and down both ELQ_NVFP4; D and U Q8_0 or Q4_0):
+ *            gate_up.gs holds one global scale per expert (gs_rows = 2I),
+ *            down.gs one per expert (gs_rows = L); L % 256 == 0 and
+ *            I % 256 == 0; act_gz, act_gh > 0.  Such layers run for T <= 8
+ *            tokens (T * k <= 64) only; other T return ELQ_ERR_UNSUPPORTED.
  */
 #ifndef ELQ_H
 #define ELQ_H
@@ -110,17 +136,19 @@ typedef enum {                  /* GGUF type ids */
     ELQ_Q4_0 = 2,
     ELQ_Q8_0 = 8,
     ELQ_Q8_1 = 9,
-    ELQ_BF16 = 30
+    ELQ_BF16 = 30,
+    ELQ_NVFP4 = 100             /* not a GGUF id: this library's own */
 } elq_type;
 
 /* One quantised matrix in the tile-slab arena (device pointers q, d). */
 typedef struct {
-    int32_t fmt;                /* ELQ_Q8_0 or ELQ_Q4_0 */
+    int32_t fmt;                /* ELQ_Q8_0, ELQ_Q4_0, or ELQ_NVFP4 (expert matrices) */
     int32_t n_rows;             /* multiple of 128 */
     int32_t k;                  /* multiple of 32 */
-    int32_t reserved;
+    int32_t gs_rows;            /* NVFP4: rows that share one global scale; else 0 */
     const void* q;
     const void* d;
+    const float* gs;            /* NVFP4: device fp32 [n_rows / gs_rows], 4-byte aligned; else NULL */
 } elq_qmat;
 
 /* elq_layer.flags bits. */
@@ -144,6 +172,7 @@ typedef struct {
     const float* router_bias;   /* [E] or NULL */
     elq_qmat gate_up;           /* E*2I x L, interleaved by 64-row halves */
     elq_qmat down;              /* E*L x I */
+    float act_gz, act_gh;       /* NVFP4 experts: global scales of z and h; else unused */
 } elq_layer;
 
 /* ---- status ------------------------------------------------------------ */
@@ -163,12 +192,14 @@ size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k,
                        size_t* q_bytes, size_t* d_bytes);
 
 /* Repack row-major GGUF-style AoS blocks (device, n_rows x k/32 blocks of
- * 34 B (Q8_0) or 18 B (Q4_0), no alignment requirement) into the arena. */
+ * 34 B (Q8_0) or 18 B (Q4_0, NVFP4), no alignment requirement) into the
+ * arena.  NVFP4 global scales stay with the caller (elq_qmat.gs). */
 elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t k,
                           void* q_out, void* d_out, void* stream);
 
 /* Quantise fp32 weights (device, row-major n_rows x k) into the arena with the
- * format's own quantiser (block rules above). */
+ * format's own quantiser (block rules above).  Q8_0 and Q4_0; NVFP4 weights
+ * go through elq_quantize_nvfp4 and elq_arena_pack. */
 elq_status elq_quantize_weights(int32_t fmt, const float* w, int32_t n_rows, int32_t k,
                                 void* q_out, void* d_out, void* stream);
 
@@ -185,6 +216,13 @@ elq_status elq_quantize_gate_up(int32_t fmt, const float* gate, const float* up,
  * rows*cols/32 Q8_1 blocks (36 B each, row-major, 4-byte aligned). */
 elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_t cols,
                              void* out_q8_1, void* stream);
+
+/* NVFP4 quantiser under global scale g (> 0, finite): x device [rows][cols]
+ * fp32 (ELQ_F32) or bf16 (ELQ_BF16), cols % 32 == 0, 4-byte aligned; out
+ * device rows*cols/32 18-byte blocks, row-major, 2-byte aligned.  The
+ * layer's own NVFP4 activations are quantised by the same warp routine. */
+elq_status elq_quantize_nvfp4(const void* x, int32_t x_type, int64_t rows, int64_t cols, float g,
+                              void* out, void* stream);
 
 /* Router (a3): logits = W_r z + bias, top-k, softmax over the k.  z: device fp32
  * [T][L] (unquantised latent), w_router [E][L], bias [E] or NULL.  idx: device
@@ -245,7 +283,8 @@ elq_status elq_latent_proj_noalloc_status(void* stream);
 /* Grouped experts (a5-a9): bucketing, gate/up with SwiGLU and Q8_1 requant,
  * down, and the weighted combine.  z_q8_1: device T rows of L/32 Q8_1 blocks;
  * idx, weights: device [T][k] as elq_router_topk writes them; y_lat: device
- * fp32 [T][L].  Uses layer->L, E, k, I, gate_up and down. */
+ * fp32 [T][L].  Uses layer->L, E, k, I, gate_up and down.  NVFP4 experts
+ * (T <= 8, T * k <= 64): z is T rows of L/32 NVFP4 blocks under act_gz. */
 elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1,
                                    const int32_t* idx, const float* weights, int32_t T,
                                    float* y_lat, void* ws, size_t ws_bytes, void* stream);
@@ -304,6 +343,7 @@ elq_status elq_moe_layer_profiled(const elq_layer* layer, const void* x, int32_t
  * (int32 [E]), 7 offsets (int32 [E+1]), 8 perm (int32 [T*k]), 9 pos, 10 hq
  * (Q8_1 [T*k][I/32], by pair position), 11 o (fp32 [T*k][L], by position),
  * 12 y_lat (fp32 [T][L]), 13 ylq (Q8_1), 14 number of routed experts (int32).
+ * With NVFP4 experts zq and hq hold NVFP4 blocks (18 B) instead of Q8_1.
  * On the tensor-core path (T >= 16, all matrices Q8_0) hq and o are kept in
  * padded per-expert slots instead, and their views return ELQ_ERR_INVALID_ARG.
  * Sets *offset (bytes from the workspace start) and *bytes; returns ELQ_OK or

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <functional>
@@ -96,15 +97,25 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
 inline elq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ELQ_OK : ELQ_ERR_CUDA; }
 
 bool fmt_ok(int32_t f) { return f == ELQ_Q8_0 || f == ELQ_Q4_0; }
+// formats the arena holds (NVFP4 in the Q4_0 geometry: 16 code bytes and a
+// 16-bit scale word per row and block)
+bool arena_fmt_ok(int32_t f) { return fmt_ok(f) || f == ELQ_NVFP4; }
 int slab_bytes(int32_t f) { return f == ELQ_Q8_0 ? kQ80Slab : kQ40Slab; }
 
-elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k) {
+// nv_ok: the matrix may be NVFP4 (a layer's expert matrices), with a global
+// scale per gs_rows rows.
+elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k, bool nv_ok = false) {
     if (!w) return ELQ_ERR_INVALID_ARG;
-    if (!fmt_ok(w->fmt)) return ELQ_ERR_UNSUPPORTED;
+    if (!(fmt_ok(w->fmt) || (nv_ok && w->fmt == ELQ_NVFP4))) return ELQ_ERR_UNSUPPORTED;
     if (w->n_rows != rows || w->k != k || rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
     if (rows % kTileRows || k % 128) return ELQ_ERR_UNSUPPORTED;
     if (!w->q || !w->d) return ELQ_ERR_INVALID_ARG;
     if (!aligned(w->q, 256) || !aligned(w->d, 256)) return ELQ_ERR_ALIGNMENT;
+    if (w->fmt == ELQ_NVFP4) {
+        if (k % 256) return ELQ_ERR_UNSUPPORTED;   // whole 8-block chunks of 18-byte activation blocks
+        if (!w->gs || w->gs_rows <= 0 || rows % w->gs_rows) return ELQ_ERR_INVALID_ARG;
+        if (!aligned(w->gs, 4)) return ELQ_ERR_ALIGNMENT;
+    }
     return ELQ_OK;
 }
 
@@ -253,12 +264,14 @@ SPlan plan_s(int fmt, int x_mode, bool swiglu, int rows_per_group, int K, int gr
     // one stage of a CTA: the codes and scales of its cpc chunks, then each
     // token's activations over the same blocks
     const int codes = p.cpc * kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
-    const int ablock = x_mode == X_RAW_F32 ? 128 : x_mode == X_RAW_BF16 ? 64 : 36;
+    const int ablock = x_mode == X_RAW_F32 ? 128 : x_mode == X_RAW_BF16 ? 64 : fmt == ELQ_NVFP4 ? 18 : 36;
     p.scales_off = codes;
     p.acts_off = (int)round_up((size_t)codes + (size_t)p.cpc * kChunk * 64, 128);
     p.act_row = p.cpc * kChunk * ablock;
     p.stage_bytes = (int)round_up((size_t)p.acts_off + (size_t)T * p.act_row, 128);
-    p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)T * kChunk * 36, 128) : 0;
+    p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)T * kChunk * 36, 128)
+                      : fmt == ELQ_NVFP4                        ? (int)round_up((size_t)kSNvScratch, 128)
+                                                                : 0;
     const int pbuf = 2 * halves * p.nchunks * T * 128;
     const int route = routed ? (int)round_up((size_t)kSRouteBytes, 128) : 0;
     auto smem_for = [&](int st) { return kSHeader + st * p.stage_bytes + p.cpc * p.scratch_bytes + pbuf + route; };
@@ -326,6 +339,8 @@ cudaError_t launch_s_f(const SArgs& g, int x_mode, int out_mode, const SPlan& p,
     switch (x_mode * 16 + out_mode) {
     case X_RAW_BF16 * 16 + OUT_F32_Q81: return launch_s_t<FMT, X_RAW_BF16, OUT_F32_Q81>(g, p, s, pdl);
     case X_RAW_F32 * 16 + OUT_F32_Q81: return launch_s_t<FMT, X_RAW_F32, OUT_F32_Q81>(g, p, s, pdl);
+    case X_RAW_BF16 * 16 + OUT_F32_NV: return launch_s_t<FMT, X_RAW_BF16, OUT_F32_NV>(g, p, s, pdl);
+    case X_RAW_F32 * 16 + OUT_F32_NV: return launch_s_t<FMT, X_RAW_F32, OUT_F32_NV>(g, p, s, pdl);
     case X_Q81_TOKEN * 16 + OUT_F32: return launch_s_t<FMT, X_Q81_TOKEN, OUT_F32>(g, p, s, pdl);
     case X_Q81_TOKEN * 16 + OUT_F32_ADD: return launch_s_t<FMT, X_Q81_TOKEN, OUT_F32_ADD>(g, p, s, pdl);
     case X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU: return launch_s_t<FMT, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl);
@@ -353,6 +368,15 @@ cudaError_t launch_s(SArgs g, int fmt, int x_mode, int out_mode, const SPlan& p,
     const int64_t ctas = (int64_t)p.clusters * p.C;
     for (int r = 0; r < 3; ++r)
         g.pf_share[r] = g.pf[r] ? (int64_t)round_up((size_t)((g.pf_bytes[r] + ctas - 1) / ctas), 256) : 0;
+    if (fmt == ELQ_NVFP4) {
+        // NVFP4 expert projections only
+        switch (x_mode * 16 + out_mode) {
+        case X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU: return launch_s_t<kNV, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl);
+        case X_Q81_POSITION * 16 + OUT_F32_COMBINE:
+            return launch_s_t<kNV, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     return fmt == ELQ_Q8_0 ? launch_s_f<8>(g, x_mode, out_mode, p, s, pdl) : launch_s_f<2>(g, x_mode, out_mode, p, s, pdl);
 }
 
@@ -550,6 +574,7 @@ DecPlanH plan_dec(const elq_layer* ly, int T) {
     if (!(ly->flags & ELQ_LAYER_FUSED)) return d;
     if (T < 1 || T > kDecMaxT || (int64_t)T * ly->k > kDecMaxPairs) return d;
     if (ly->D.fmt != ly->U.fmt || ly->gate_up.fmt != ly->down.fmt) return d;
+    if (ly->gate_up.fmt == ELQ_NVFP4) return d;     // NVFP4 experts: the cluster GEMV path only
     if (ly->L / kTileRows > 64) return d;            // latent tiles the shared-memory mirror follows
     auto codes = [](int fmt) { return kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512); };
     const size_t acts = (size_t)T * kChunk * 36;
@@ -636,6 +661,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.rs_C = 1;
     while ((E + w.rs_C - 1) / w.rs_C > 4 && w.rs_C < kSMaxCluster) w.rs_C *= 2;
     w.rs_epc = (E + w.rs_C - 1) / w.rs_C;
+    // (NVFP4 experts take this path or none)
     if (!w.tc && !w.fused && w.raw && P <= kSMaxPairs && w.rs_epc <= kSMaxWarps &&
         rs_smem_bytes(T, L, E) + 16 <= kSSmemMax) {
         w.sd = plan_s(ly->D.fmt, dmode, false, L, H, 1, T, false);
@@ -739,8 +765,18 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     if ((s = check_qmat(&ly->D, L, H)) != ELQ_OK) return s;
     if ((s = check_qmat(&ly->U, H, L)) != ELQ_OK) return s;
     if ((int64_t)E * 2 * I > INT32_MAX || (int64_t)E * L > INT32_MAX) return ELQ_ERR_UNSUPPORTED;
-    if ((s = check_qmat(&ly->gate_up, E * 2 * I, L)) != ELQ_OK) return s;
-    if ((s = check_qmat(&ly->down, E * L, I)) != ELQ_OK) return s;
+    if ((s = check_qmat(&ly->gate_up, E * 2 * I, L, true)) != ELQ_OK) return s;
+    if ((s = check_qmat(&ly->down, E * L, I, true)) != ELQ_OK) return s;
+    if ((ly->gate_up.fmt == ELQ_NVFP4) != (ly->down.fmt == ELQ_NVFP4)) return ELQ_ERR_UNSUPPORTED;
+    if (ly->gate_up.fmt == ELQ_NVFP4) {
+        // one global scale per expert matrix; static activation scales
+        if (ly->gate_up.gs_rows != 2 * I || ly->down.gs_rows != L) return ELQ_ERR_INVALID_ARG;
+        if (!(ly->act_gz > 0.0f) || !(ly->act_gh > 0.0f) || !std::isfinite(ly->act_gz) ||
+            !std::isfinite(ly->act_gh))
+            return ELQ_ERR_INVALID_ARG;
+        // the cluster GEMV's token and pair bounds
+        if (T > kSMaxT || (int64_t)T * k > kSMaxPairs) return ELQ_ERR_UNSUPPORTED;
+    }
     if (!ly->router_w) return ELQ_ERR_INVALID_ARG;
     if (!aligned(ly->router_w, 16) || (ly->router_bias && !aligned(ly->router_bias, 4))) return ELQ_ERR_ALIGNMENT;
     return ELQ_OK;
@@ -849,6 +885,7 @@ SArgs gate_up_s(const elq_layer* ly, const LayerWs& w, int T, int route, const u
     g.grp = w.grp; g.gtok = w.gtok;
     g.x = zq;
     g.yq = w.hq; g.yq_ld = I / 32;
+    g.wgs = ly->gate_up.gs; g.ags = ly->act_gz; g.ogs = ly->act_gh;
     // the routed experts' down matrices, for the next kernel
     g.pfe_q = static_cast<const uint8_t*>(ly->down.q);
     g.pfe_d = reinterpret_cast<const uint8_t*>(ly->down.d);
@@ -878,6 +915,7 @@ SArgs down_s(const elq_layer* ly, const LayerWs& w, int T, int route, const floa
     h.x = w.hq;
     h.y = w.o; h.y_ld = L;
     h.cnt_comb = w.cnt_comb; h.ylat = y_lat; h.ylq = w.ylq; h.L = L;
+    h.wgs = ly->down.gs; h.ags = ly->act_gh;
     h.err = w.err;
     // the routing is complete before this kernel's upstream (gate/up) starts
     h.early = 1;
@@ -1095,10 +1133,10 @@ const char* elq_status_string(int32_t status) {
     }
 }
 
-int32_t elq_version(void) { return 1; }
+int32_t elq_version(void) { return 2; }
 
 size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k, size_t* q_bytes, size_t* d_bytes) {
-    if (!fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % 32) {
+    if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % 32) {
         if (q_bytes) *q_bytes = 0;
         if (d_bytes) *d_bytes = 0;
         return 0;
@@ -1112,7 +1150,7 @@ size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k, size_t* q_bytes, 
 
 elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t k, void* q_out, void* d_out,
                           void* stream) {
-    if (!fmt_ok(fmt)) return ELQ_ERR_UNSUPPORTED;
+    if (!arena_fmt_ok(fmt)) return ELQ_ERR_UNSUPPORTED;
     if (!aos || !q_out || !d_out || n_rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
     if (n_rows % kTileRows || k % 32) return ELQ_ERR_UNSUPPORTED;
     if (!aligned(q_out, 256) || !aligned(d_out, 256)) return ELQ_ERR_ALIGNMENT;
@@ -1122,7 +1160,7 @@ elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t 
     if (fmt == ELQ_Q8_0)
         k_arena_pack<8><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
                                              static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
-    else
+    else   // Q4_0, and NVFP4 in the same byte geometry
         k_arena_pack<2><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
                                              static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
     return cuda_status(cudaGetLastError());
@@ -1179,6 +1217,24 @@ elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_
                                   static_cast<uint8_t*>(out_q8_1)));
     return cuda_status(launch(k_quant_q8_1<false>, grid, dim3(256), 0, s, false, x, nblk,
                               static_cast<uint8_t*>(out_q8_1)));
+}
+
+elq_status elq_quantize_nvfp4(const void* x, int32_t x_type, int64_t rows, int64_t cols, float g, void* out,
+                              void* stream) {
+    if (x_type != ELQ_F32 && x_type != ELQ_BF16) return ELQ_ERR_UNSUPPORTED;
+    if (rows < 0 || cols <= 0 || !(g > 0.0f) || !std::isfinite(g)) return ELQ_ERR_INVALID_ARG;
+    if (cols % 32) return ELQ_ERR_UNSUPPORTED;
+    if (rows == 0) return ELQ_OK;
+    if (!x || !out) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(x, 4) || !aligned(out, 2)) return ELQ_ERR_ALIGNMENT;
+    const int64_t nblk = rows * (cols / 32);
+    const dim3 grid((unsigned)((nblk * 32 + 255) / 256));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (x_type == ELQ_BF16)
+        return cuda_status(launch(k_quant_nvfp4<true>, grid, dim3(256), 0, s, false, x, nblk, g,
+                                  static_cast<uint8_t*>(out)));
+    return cuda_status(launch(k_quant_nvfp4<false>, grid, dim3(256), 0, s, false, x, nblk, g,
+                              static_cast<uint8_t*>(out)));
 }
 
 elq_status elq_router_topk(const float* z, const float* w_router, const float* bias, int32_t T, int32_t L,
@@ -1284,6 +1340,13 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     const int E = layer->E, k = layer->k;
     const int64_t P = (int64_t)T * k;
     const int nw = 32;
+    const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
+    if (nv) {
+        const int gmax = (int)std::min<int64_t>(E, P);
+        if (!plan_s(ELQ_NVFP4, X_Q81_PAIR_TOKEN, true, 2 * layer->I, layer->L, gmax, T, true).ok ||
+            !plan_s(ELQ_NVFP4, X_Q81_POSITION, false, layer->L, layer->I, gmax, T, true).ok)
+            return ELQ_ERR_UNSUPPORTED;
+    }
     cudaError_t e = smem_optin(k_bucket, kRouterSmemMax, g_optin_bucket);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
     e = launch(k_bucket, dim3(1), dim3(nw * 32), (size_t)nw * E * 4, s, false, idx, (int)P, E, w.counts, w.offsets,
@@ -1383,10 +1446,11 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, 
                  I = layer->I;
     const void* p = nullptr;
     size_t n = 0;
+    const size_t ablk = layer->gate_up.fmt == ELQ_NVFP4 ? 18 : 36;   // the experts' activation blocks
     switch (which) {
     case 0: p = w.xq; n = Tz * (H / 32) * 36; break;
     case 1: p = w.z; n = Tz * L * 4; break;
-    case 2: p = w.zq; n = Tz * (L / 32) * 36; break;
+    case 2: p = w.zq; n = Tz * (L / 32) * ablk; break;
     case 3: p = w.logits; n = Tz * E * 4; break;
     case 4: p = w.idx; n = P * 4; break;
     case 5: p = w.wts; n = P * 4; break;
@@ -1394,7 +1458,7 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, 
     case 7: p = w.offsets; n = (E + 1) * 4; break;
     case 8: p = w.perm; n = P * 4; break;
     case 9: p = w.pos; n = P * 4; break;
-    case 10: p = w.tc ? nullptr : w.hq; n = P * (I / 32) * 36; break;
+    case 10: p = w.tc ? nullptr : w.hq; n = P * (I / 32) * ablk; break;
     case 11: p = w.tc ? nullptr : w.o; n = P * L * 4; break;
     case 12: p = w.ylat; n = Tz * L * 4; break;
     case 13: p = w.ylq; n = Tz * (L / 32) * 36; break;
@@ -1553,6 +1617,8 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     if (events && n_events < layer_kernels(layer, T) + 1) return ELQ_ERR_INVALID_ARG;
     if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
     LayerWs w = layer_layout(layer, T, ws, x_type);
+    const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
+    if (nv && !w.small) return ELQ_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1608,13 +1674,14 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         // the router rows and U, which later kernels of the layer read
         const int dmode = x_type == ELQ_BF16 ? X_RAW_BF16 : X_RAW_F32;
         SArgs gd = dense_s(&layer->D, T, x, H, w.z, w.zq, w.err);
+        gd.ogs = layer->act_gz;                 // NVFP4 experts: z's blocks under act_gz
         gd.pf[0] = reinterpret_cast<const uint8_t*>(layer->router_w);
         gd.pf_bytes[0] = (int64_t)E * L * 4;
         gd.pf[1] = static_cast<const uint8_t*>(layer->U.q);
         gd.pf_bytes[1] = (int64_t)(H / kTileRows) * (L / 32) * slab_bytes(layer->U.fmt);
         gd.pf[2] = static_cast<const uint8_t*>(layer->U.d);
         gd.pf_bytes[2] = (int64_t)(H / kTileRows) * (L / 32) * kScaleSlab;
-        if (launch_s(gd, layer->D.fmt, dmode, OUT_F32_Q81, w.sd, s, pdl) != cudaSuccess || !mark())
+        if (launch_s(gd, layer->D.fmt, dmode, nv ? OUT_F32_NV : OUT_F32_Q81, w.sd, s, pdl) != cudaSuccess || !mark())
             return ELQ_ERR_CUDA;
         // a3 + a5: the cluster router (logits, top-k, softmax, bucketing, group table)
         if (launch_route_small(layer, w, T, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;

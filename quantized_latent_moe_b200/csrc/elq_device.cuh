@@ -91,6 +91,77 @@ __device__ __forceinline__ void warp_quant_q8_1(float v, uint8_t* dst) {
     }
 }
 
+// ---- NVFP4: E2M1 codes under E4M3 micro-block scales ---------------------------
+
+constexpr int kNV = 100;           // format id of NVFP4 (ELQ_NVFP4)
+
+// The two E4M3 bytes of s (s[0] the low byte) as fp32, exactly (every E4M3
+// value is an fp16 value): the hardware conversion to fp16x2, then widening.
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t s) {
+    uint32_t h2;
+    const uint16_t s16 = (uint16_t)s;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(s16));
+    return make_float2(h2f((uint16_t)(h2 & 0xffffu)), h2f((uint16_t)(h2 >> 16)));
+}
+
+// fp32 -> E4M3 byte: round to nearest even, finite results saturating at 448
+// (the hardware's satfinite conversion); NaN and non-positive inputs give 0.
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+    if (!(x > 0.0f)) return 0u;
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return (uint32_t)(r & 0xffu);
+}
+
+// E2M1 codes of lo (low nibble) and hi (high nibble): round to nearest even,
+// saturating at 6.  -0 counts as +0 and a negative input that rounds to zero
+// keeps its sign bit, whatever the conversion does with signed zeros.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    lo = __fadd_rn(lo, 0.0f);
+    hi = __fadd_rn(hi, 0.0f);
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return (r & 0x77u) | (lo < 0.0f ? 0x08u : 0u) | (hi < 0.0f ? 0x80u : 0u);
+}
+
+// Doubled magnitudes (0, 1, 2, 3, 4, 6, 8, 12) of the four E2M1 codes in the
+// low 16 bits of c (code i in bits 4i .. 4i+3), one byte each, in order; a
+// code whose sign bit is set gives 0 (the byte permute's sign-replicating
+// selectors pick a table byte whose top bit is clear).
+__device__ __forceinline__ uint32_t e2m1x4_pos(uint32_t c) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(0x03020100u), "r"(0x0C080604u), "r"(c));
+    return r;
+}
+
+// Signed doubled values (2 * e2m1) of the four codes in the low 16 bits of c.
+__device__ __forceinline__ uint32_t e2m1x4_signed(uint32_t c) {
+    return __vsub4(e2m1x4_pos(c), e2m1x4_pos(c ^ 0x8888u));
+}
+
+// Quantise one 32-value block held one value per lane (lane i = element i)
+// into an NVFP4 block at dst (2-byte aligned) under global scale g: per
+// 16-lane half s = e4m3(amax / 6 / g), code = e2m1(x / (e4m3(s) * g)), zero
+// codes for a zero scale.
+__device__ __forceinline__ void warp_quant_nvfp4(float v, float g, uint8_t* dst) {
+    const int lane = threadIdx.x & 31;
+    float amax = fabsf(v);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const uint32_t s = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+    const float den = __fmul_rn(e4m3x2_to_f32(s).x, g);
+    const float x = den != 0.0f ? __fdiv_rn(v, den) : 0.0f;
+    const float xo = __shfl_down_sync(0xffffffffu, x, 1);     // value 2j+1, on lane 2j
+    const uint32_t byte = f32x2_to_e2m1x2(x, xo);             // code byte j, on lane 2j
+    const uint32_t b2 = __shfl_down_sync(0xffffffffu, byte, 2);
+    const uint32_t s1 = __shfl_sync(0xffffffffu, s, 16);
+    if ((lane & 3) == 0)
+        reinterpret_cast<uint16_t*>(dst + 2)[lane >> 2] = (uint16_t)((byte & 0xffu) | ((b2 & 0xffu) << 8));
+    if (lane == 0) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)(s | (s1 << 8));
+}
+
 // ---- bulk copies and mbarriers (sm_90+ PTX, used on sm_100a) ------------------
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

@@ -1,5 +1,6 @@
 // elq_kernels.cuh -- the layer's sm_100a kernels (decode/verify path):
 //   k_quant_q8_1      a1/a4  activation quantiser
+//   k_quant_nvfp4     NVFP4 quantiser (standalone entry point)
 //   k_quant_weights   arena preparation from fp32 weights
 //   k_arena_pack      arena preparation from GGUF-style AoS blocks
 //   k_router          a3 (+a5)  logits, top-k, softmax, bucketing
@@ -31,6 +32,22 @@ __global__ void __launch_bounds__(256) k_quant_q8_1(const void* __restrict__ x, 
         v = reinterpret_cast<const float*>(x)[blk * 32 + lane];
     warp_quant_q8_1(v, out + blk * 36);
     pdl_trigger();
+}
+
+// NVFP4 quantiser under global scale g: one warp per 32-value block (the
+// layer's NVFP4 activations use the same warp routine in their epilogues).
+template <bool kBF16>
+__global__ void __launch_bounds__(256) k_quant_nvfp4(const void* __restrict__ x, int64_t nblocks, float g,
+                                                     uint8_t* __restrict__ out) {
+    const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (blk >= nblocks) return;
+    float v;
+    if (kBF16)
+        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[blk * 32 + lane]);
+    else
+        v = reinterpret_cast<const float*>(x)[blk * 32 + lane];
+    warp_quant_nvfp4(v, g, out + blk * 18);
 }
 
 // ============================================================================
@@ -555,7 +572,9 @@ __global__ void __launch_bounds__(128) k_topk(const float* __restrict__ logits, 
 // ============================================================================
 constexpr int kTokMax = 32;        // tokens a unit stages at once
 
-enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2, OUT_F32_COMBINE = 3, OUT_F32_ADD = 4 };
+// OUT_F32_NV: fp32 rows and their NVFP4 blocks (the latent z of a layer with
+// NVFP4 experts; the cluster GEMV only).
+enum { OUT_F32 = 0, OUT_F32_Q81 = 1, OUT_SWIGLU = 2, OUT_F32_COMBINE = 3, OUT_F32_ADD = 4, OUT_F32_NV = 5 };
 enum { X_Q81_TOKEN = 0, X_Q81_PAIR_TOKEN = 1, X_Q81_POSITION = 2, X_RAW_F32 = 3, X_RAW_BF16 = 4 };
 
 struct WArgs {

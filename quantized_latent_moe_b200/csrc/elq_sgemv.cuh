@@ -105,6 +105,10 @@ struct SArgs {
     const uint8_t* pfe_q;
     const uint8_t* pfe_d;
     int64_t pfe_qs, pfe_ds;                      // bytes per expert (multiples of 256)
+    // NVFP4: global scales of the weights (one per group's expert, indexed by
+    // expert), of the input activations, and of the epilogue's NVFP4 output
+    const float* wgs;
+    float ags, ogs;
     int* err;
     uint64_t budget_ns;
     int early;               // weights and routing do not depend on the upstream grid
@@ -201,10 +205,11 @@ __device__ __forceinline__ SUnit s_unit(const SArgs& g, const uint8_t* rs, int i
     return u;
 }
 
-// Bytes of one activation block (32 values) in the input's form.
-template <int XM>
+// Bytes of one activation block (32 values) in the input's form: raw fp32 or
+// bf16, or quantised (NVFP4 for NVFP4 weights, else Q8_1).
+template <int FMT, int XM>
 __device__ __forceinline__ uint32_t s_act_block() {
-    return XM == X_RAW_F32 ? 128u : XM == X_RAW_BF16 ? 64u : 36u;
+    return XM == X_RAW_F32 ? 128u : XM == X_RAW_BF16 ? 64u : FMT == kNV ? 18u : 36u;
 }
 
 // The CTA's blocks of an item: [kb0, kb0 + nblk) of slice (tile, s), the
@@ -229,7 +234,7 @@ __device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, 
                                                 uint64_t* bar) {
     using SL = WSlice<FMT>;
     const uint32_t cb = (uint32_t)(r.nblk * SL::kCodes), sb = (uint32_t)(r.nblk * 64);
-    mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * (uint32_t)r.nblk * s_act_block<XM>());
+    mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * (uint32_t)r.nblk * s_act_block<FMT, XM>());
     bulk_g2s(stg, g.q + u.grp.x * g.q_gstride + ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
              cb, bar);
     bulk_g2s(stg + g.scales_off,
@@ -238,7 +243,7 @@ __device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, 
              sb, bar);
 }
 
-template <int XM>
+template <int FMT, int XM>
 __device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, const SUnit& u, const SRange& r,
                                              uint8_t* stg, uint64_t* bar) {
     const int lane = threadIdx.x & 31;
@@ -253,8 +258,8 @@ __device__ __forceinline__ void s_issue_acts(const SArgs& g, const uint8_t* rs, 
         else if (XM == X_RAW_BF16)
             src = static_cast<const uint8_t*>(g.x) + (row * g.x_row + (int64_t)r.kb0 * 32) * 2;
         else
-            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + r.kb0) * 36;
-        bulk_g2s(stg + g.acts_off + lane * g.act_row, src, (uint32_t)r.nblk * s_act_block<XM>(), bar);
+            src = static_cast<const uint8_t*>(g.x) + (row * g.nb + r.kb0) * (int64_t)s_act_block<FMT, XM>();
+        bulk_g2s(stg + g.acts_off + lane * g.act_row, src, (uint32_t)r.nblk * s_act_block<FMT, XM>(), bar);
     }
 }
 
@@ -345,7 +350,7 @@ __device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uin
     // this warp's chunk inside the CTA's stage
     const uint8_t* codes = stg + warp * kChunk * SL::kCodes;
     const uint16_t* scales = reinterpret_cast<const uint16_t*>(stg + g.scales_off) + warp * kChunk * 32;
-    const uint8_t* abase = stg + g.acts_off + warp * kChunk * s_act_block<XM>();
+    const uint8_t* abase = stg + g.acts_off + warp * kChunk * s_act_block<FMT, XM>();
     int astride = g.act_row;
     const int nt = u.grp.z;
     if (XM == X_RAW_F32 || XM == X_RAW_BF16) {
@@ -387,31 +392,114 @@ __device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uin
     }
 }
 
+// Scratch of the NVFP4 dot: per (token, block) of the chunk the activations'
+// 32 doubled codes as signed bytes, then separately their two scales.
+constexpr int kSNvScratch = kSMaxT * kChunk * 32 + kSMaxT * kChunk * 8;
+
+// The NVFP4 form of s_dots.  The warp first expands its tokens' activation
+// blocks (18-byte NVFP4) into signed doubled codes and fp32 scales in its
+// scratch; then, block by block, each lane expands its row's 32 codes once
+// into the doubled magnitudes of the positive and of the negative codes (byte
+// permutes) and takes, for every token, isum = dp4a(pos, a) - dp4a(neg, a)
+// per 16-value micro-block, and part = fmaf(isum, s_w * s_a, part) in
+// micro-block order.  The global scales are applied in the epilogue.
+template <int XM>
+__device__ __forceinline__ void s_dots_nv(const SArgs& g, const SUnit& u, const uint8_t* stg, uint8_t* scratch,
+                                          uint32_t dst) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const uint8_t* codes = stg + warp * kChunk * 512;
+    const uint16_t* scales = reinterpret_cast<const uint16_t*>(stg + g.scales_off) + warp * kChunk * 32;
+    const uint8_t* abase = stg + g.acts_off + warp * kChunk * 18;
+    const int nt = u.grp.z, kbn = u.kbn;
+    uint32_t* ap = reinterpret_cast<uint32_t*>(scratch);                          // [t][kb][8]
+    float2* as = reinterpret_cast<float2*>(scratch + kSMaxT * kChunk * 32);       // [t][kb]
+#pragma unroll 1
+    for (int i = lane; i < nt * kChunk * 9; i += 32) {
+        const int t = i / (kChunk * 9), r = i - t * (kChunk * 9);
+        const int kb = r / 9, j = r - kb * 9;
+        if (kb < kbn) {
+            const uint8_t* blk = abase + t * g.act_row + kb * 18;
+            const uint32_t v = *reinterpret_cast<const uint16_t*>(blk + (j < 8 ? 2 + 2 * j : 0));
+            if (j < 8) ap[(t * kChunk + kb) * 8 + j] = e2m1x4_signed(v);
+            else as[t * kChunk + kb] = e4m3x2_to_f32(v);
+        }
+    }
+    __syncwarp();
+    float part[kSMaxT];
+#pragma unroll
+    for (int t = 0; t < kSMaxT; ++t) part[t] = 0.0f;
+#pragma unroll 1
+    for (int kb = 0; kb < kbn; ++kb) {
+        const float2 sw = e4m3x2_to_f32(scales[kb * 32 + lane]);
+        // micro-block by micro-block (each token's chain keeps the block's order)
+#pragma unroll
+        for (int mb = 0; mb < 2; ++mb) {
+            const uint2 q = *reinterpret_cast<const uint2*>(codes + kb * 512 + lane * 16 + mb * 8);
+            const float swm = mb ? sw.y : sw.x;
+            uint32_t wp[4], wn[4];
+            wp[0] = e2m1x4_pos(q.x);
+            wp[1] = e2m1x4_pos(q.x >> 16);
+            wp[2] = e2m1x4_pos(q.y);
+            wp[3] = e2m1x4_pos(q.y >> 16);
+            wn[0] = e2m1x4_pos(q.x ^ 0x88888888u);
+            wn[1] = e2m1x4_pos((q.x ^ 0x88888888u) >> 16);
+            wn[2] = e2m1x4_pos(q.y ^ 0x88888888u);
+            wn[3] = e2m1x4_pos((q.y ^ 0x88888888u) >> 16);
+#pragma unroll
+            for (int t = 0; t < kSMaxT; ++t) {
+                if (t < nt) {
+                    const uint4 a = lds128(ap + (t * kChunk + kb) * 8 + mb * 4);
+                    const float2 sa = as[t * kChunk + kb];
+                    int ps = __dp4a((int)wp[0], (int)a.x, 0), ns = __dp4a((int)wn[0], (int)a.x, 0);
+                    ps = __dp4a((int)wp[1], (int)a.y, ps); ns = __dp4a((int)wn[1], (int)a.y, ns);
+                    ps = __dp4a((int)wp[2], (int)a.z, ps); ns = __dp4a((int)wn[2], (int)a.z, ns);
+                    ps = __dp4a((int)wp[3], (int)a.w, ps); ns = __dp4a((int)wn[3], (int)a.w, ns);
+                    part[t] = __fmaf_rn(__int2float_rn(ps - ns), __fmul_rn(swm, mb ? sa.y : sa.x), part[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kSMaxT; ++t)
+        if (t < nt) dsmem_st(dst + (uint32_t)((t * 32 + lane) * 4), part[t]);
+}
+
 // One out-of-line copy each of the epilogues' quantiser and SwiGLU.
 __device__ __noinline__ void s_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
+__device__ __noinline__ void s_quant_nv(float v, float g, uint8_t* dst) { warp_quant_nvfp4(v, g, dst); }
 __device__ __noinline__ float s_swiglu(float g, float u) { return __fmul_rn(silu_f32(g), u); }
 
 // The item's epilogue in the cluster's first CTA: per token (warps take
-// tokens in turn) the chunk partials in chunk order, then the output mode.
+// tokens in turn) the chunk partials in chunk order, then (NVFP4 weights) the
+// product of the global scales, then the output mode.
 // pb: this item's partial buffer [units][T][32].
-template <int OM>
+template <int FMT, int OM>
 __device__ void s_epilogue(const SArgs& g, const uint8_t* rs, const SUnit& u, const float* pb) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = blockDim.x >> 5;
     const int T = g.T;
     const int nt = u.grp.z;
     const int row = u.tile * kTileRows + u.s * 32 + lane;      // row of the group's matrix
+    // NVFP4: y = acc * ((g_w * g_a) * 0.25), the codes being doubled
+    const float gq = FMT == kNV ? __fmul_rn(__fmul_rn(__ldg(g.wgs + u.grp.x), g.ags), 0.25f) : 1.0f;
     for (int t = warp; t < nt; t += nw) {
         float acc = 0.0f;
 #pragma unroll 1
         for (int c = 0; c < g.nchunks; ++c) acc = __fadd_rn(acc, pb[(c * T + t) * 32 + lane]);
+        if (FMT == kNV) acc = __fmul_rn(acc, gq);
         const int64_t pp = (int64_t)u.grp.y + t;                // token (dense) or pair position
         if (OM == OUT_SWIGLU) {
             // the up slice's partials follow the gate slice's
             float up = 0.0f;
 #pragma unroll 1
             for (int c = 0; c < g.nchunks; ++c) up = __fadd_rn(up, pb[((g.nchunks + c) * T + t) * 32 + lane]);
-            s_quant(s_swiglu(acc, up), g.yq + (pp * g.yq_ld + u.tile * 2 + u.hb) * 36);
+            if (FMT == kNV) {
+                up = __fmul_rn(up, gq);
+                s_quant_nv(s_swiglu(acc, up), g.ogs, g.yq + (pp * g.yq_ld + u.tile * 2 + u.hb) * 18);
+            } else {
+                s_quant(s_swiglu(acc, up), g.yq + (pp * g.yq_ld + u.tile * 2 + u.hb) * 36);
+            }
             continue;
         }
         float* yr = g.y + pp * g.y_ld + row;
@@ -422,6 +510,8 @@ __device__ void s_epilogue(const SArgs& g, const uint8_t* rs, const SUnit& u, co
         *yr = acc;
         if (OM == OUT_F32_Q81) {
             s_quant(acc, g.yq + (pp * g.yq_ld + u.tile * 4 + u.s) * 36);
+        } else if (OM == OUT_F32_NV) {
+            s_quant_nv(acc, g.ogs, g.yq + (pp * g.yq_ld + u.tile * 4 + u.s) * 18);
         } else if (OM == OUT_F32_COMBINE) {
             // this pair's 32 rows of o are out: count them for the token; the
             // last of the token's k pairs combines this 32-row block
@@ -696,7 +786,7 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         const int item = cid + m * ncl;
         if (item >= n_items || !cta_has) return;
         const SUnit u = s_unit<OM>(g, rs, item, rank, 0);
-        s_issue_acts<XM>(g, rs, u, rng, stages + (m % S) * g.stage_bytes, &bars[m % S]);
+        s_issue_acts<FMT, XM>(g, rs, u, rng, stages + (m % S) * g.stage_bytes, &bars[m % S]);
     };
     // L2 prefetch of the fixed ranges a later kernel reads (by the last warp)
     auto prefetch_fixed = [&]() {
@@ -752,7 +842,9 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
             if (!__all_sync(kFull, got)) {
                 if (lane == 0) *bad = 1;
             } else {
-                s_dots<FMT, XM>(g, u, stg, scratch, pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128));
+                const uint32_t dst = pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128);
+                if constexpr (FMT == kNV) s_dots_nv<XM>(g, u, stg, scratch, dst);
+                else s_dots<FMT, XM>(g, u, stg, scratch, dst);
             }
         }
         // every chunk partial of the item is in the first CTA, and every warp
@@ -767,7 +859,7 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
             __syncwarp();
             issue_a(m + S);
         }
-        if (rank == 0) s_epilogue<OM>(g, rs, u, pbuf + (size_t)(m & 1) * units * g.T * 32);
+        if (rank == 0) s_epilogue<FMT, OM>(g, rs, u, pbuf + (size_t)(m & 1) * units * g.T * 32);
     }
     if (*bad && threadIdx.x == 0) {
         // drain: wait (bounded) for the last copies of every stage

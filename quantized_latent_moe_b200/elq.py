@@ -15,10 +15,10 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libelq.so")
 
-F32, Q4_0, Q8_0, Q8_1, BF16 = 0, 2, 8, 9, 30
+F32, Q4_0, Q8_0, Q8_1, BF16, NVFP4 = 0, 2, 8, 9, 30, 100
 LAYER_FUSED = 1            # elq_layer.flags: small T as one persistent kernel
-FMT = {"q8_0": Q8_0, "q4_0": Q4_0}
-SLAB = {Q8_0: 4096, Q4_0: 2048}
+FMT = {"q8_0": Q8_0, "q4_0": Q4_0, "nvfp4": NVFP4}
+SLAB = {Q8_0: 4096, Q4_0: 2048, NVFP4: 2048}
 
 
 class ElqError(RuntimeError):
@@ -29,14 +29,16 @@ class ElqError(RuntimeError):
 
 class QMat(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("n_rows", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("q", ctypes.c_void_p), ("d", ctypes.c_void_p)]
+                ("gs_rows", ctypes.c_int32), ("q", ctypes.c_void_p), ("d", ctypes.c_void_p),
+                ("gs", ctypes.c_void_p)]
 
 
 class LayerC(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("L", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("D", QMat), ("U", QMat), ("router_w", ctypes.c_void_p),
-                ("router_bias", ctypes.c_void_p), ("gate_up", QMat), ("down", QMat)]
+                ("router_bias", ctypes.c_void_p), ("gate_up", QMat), ("down", QMat),
+                ("act_gz", ctypes.c_float), ("act_gh", ctypes.c_float)]
 
 
 _L = None
@@ -50,6 +52,7 @@ SIGNATURES = {
     "elq_quantize_weights": (I32, [I32, V, I32, I32, V, V, V]),
     "elq_quantize_gate_up": (I32, [I32, V, V, I32, I32, I32, V, V, V]),
     "elq_quantize_q8_1": (I32, [V, I32, I64, I64, V, V]),
+    "elq_quantize_nvfp4": (I32, [V, I32, I64, I64, ctypes.c_float, V, V]),
     "elq_router_topk": (I32, [V, V, V, I32, I32, I32, I32, V, V, V, V]),
     "elq_route_bucket": (I32, [V, I32, I32, I32, V, V, V, V, V]),
     "elq_latent_proj_workspace_bytes": (SZ, [ctypes.POINTER(QMat), I32]),
@@ -118,13 +121,17 @@ def _dev_empty(nbytes: int, device, align: int = 256) -> torch.Tensor:
 class QMatrix:
     """One matrix in the device tile-slab arena (codes ``q`` and scales ``d``)."""
 
-    def __init__(self, fmt: int, n_rows: int, k: int, device="cuda"):
+    def __init__(self, fmt: int, n_rows: int, k: int, device="cuda", gs_rows: int = 0):
         qb, db = SZ(), SZ()
         if not _lib().elq_arena_bytes(fmt, n_rows, k, ctypes.byref(qb), ctypes.byref(db)):
             raise ElqError(-2, "elq_arena_bytes")
         self.fmt, self.n_rows, self.k = fmt, n_rows, k
         self.q = _dev_empty(qb.value, device)
         self.d = _dev_empty(db.value, device)
+        # NVFP4: one fp32 global scale per gs_rows rows (all rows by default)
+        self.gs_rows = (gs_rows or n_rows) if fmt == NVFP4 else 0
+        self.gs = (torch.ones(n_rows // self.gs_rows, dtype=torch.float32, device=device)
+                   if fmt == NVFP4 else None)
 
     @classmethod
     def from_f32(cls, w: torch.Tensor, fmt: int, stream=None) -> "QMatrix":
@@ -142,7 +149,8 @@ class QMatrix:
         return m
 
     def struct(self) -> QMat:
-        return QMat(self.fmt, self.n_rows, self.k, 0, self.q.data_ptr(), self.d.data_ptr())
+        return QMat(self.fmt, self.n_rows, self.k, self.gs_rows, self.q.data_ptr(), self.d.data_ptr(),
+                    None if self.gs is None else self.gs.data_ptr())
 
 
 class Layer:
@@ -155,13 +163,15 @@ class Layer:
         self.router_w = router_w.contiguous()
         self.router_bias = None if router_bias is None else router_bias.contiguous()
         self.flags = 0          # LAYER_FUSED: small T as one persistent kernel
+        # NVFP4 experts: static global scales of their inputs z and h
+        self.act_gz, self.act_gh = 1.0, 1.0
         self._ws = {}
 
     @classmethod
     def allocate(cls, H, L, E, k, I, du_fmt, ex_fmt, router_w, router_bias, device="cuda"):
         return cls(H, L, E, k, I, QMatrix(du_fmt, L, H, device), QMatrix(du_fmt, H, L, device),
-                   router_w, router_bias, QMatrix(ex_fmt, E * 2 * I, L, device),
-                   QMatrix(ex_fmt, E * L, I, device))
+                   router_w, router_bias, QMatrix(ex_fmt, E * 2 * I, L, device, gs_rows=2 * I),
+                   QMatrix(ex_fmt, E * L, I, device, gs_rows=L))
 
     def set_dense(self, D: torch.Tensor, U: torch.Tensor, stream=None):
         for m, w in ((self.D, D), (self.U, U)):
@@ -188,11 +198,44 @@ class Layer:
                                         ctypes.c_void_p(dn.d.data_ptr() + e0 * dd),
                                         _stream(stream)), "elq_quantize_weights")
 
+    def set_experts_nvfp4(self, e0: int, gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor,
+                          g_gate_up: torch.Tensor, g_down: torch.Tensor, stream=None):
+        """NVFP4 experts e0 .. e0+n-1 from fp32 gate/up [n, I, L] and down [n, L, I]
+        under the given per-expert global scales (fp32 [n] each): the library's
+        NVFP4 quantiser, then the arena packing (gate and up interleaved by
+        64-row halves)."""
+        n, I, L = gate.shape
+        gu, dn = self.gate_up, self.down
+        # interleave: tile j of expert e holds gate rows 64j.. then up rows 64j..
+        gi = torch.stack([gate.reshape(n, I // 64, 64, L), up.reshape(n, I // 64, 64, L)], dim=2)
+        gi = gi.reshape(n, 2 * I, L).contiguous()
+        aos_gu = torch.empty(n, 2 * I, L // 32 * 18, dtype=torch.uint8, device=gate.device)
+        aos_dn = torch.empty(n, L, I // 32 * 18, dtype=torch.uint8, device=gate.device)
+        for e in range(n):
+            _ck(_lib().elq_quantize_nvfp4(_ptr(gi[e]), F32, 2 * I, L, float(g_gate_up[e]), _ptr(aos_gu[e]),
+                                          _stream(stream)), "elq_quantize_nvfp4")
+            de = down[e].contiguous()
+            _ck(_lib().elq_quantize_nvfp4(_ptr(de), F32, L, I, float(g_down[e]), _ptr(aos_dn[e]),
+                                          _stream(stream)), "elq_quantize_nvfp4")
+        per_q = (2 * I // 128) * (L // 32) * SLAB[NVFP4]
+        per_d = (2 * I // 128) * (L // 32) * 256
+        _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_gu), n * 2 * I, L,
+                                  ctypes.c_void_p(gu.q.data_ptr() + e0 * per_q),
+                                  ctypes.c_void_p(gu.d.data_ptr() + e0 * per_d), _stream(stream)),
+            "elq_arena_pack")
+        dq = (L // 128) * (I // 32) * SLAB[NVFP4]
+        dd = (L // 128) * (I // 32) * 256
+        _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_dn), n * L, I, ctypes.c_void_p(dn.q.data_ptr() + e0 * dq),
+                                  ctypes.c_void_p(dn.d.data_ptr() + e0 * dd), _stream(stream)),
+            "elq_arena_pack")
+        gu.gs[e0:e0 + n].copy_(g_gate_up)
+        dn.gs[e0:e0 + n].copy_(g_down)
+
     def struct(self) -> LayerC:
         return LayerC(self.H, self.L, self.E, self.k, self.I, self.flags, self.D.struct(), self.U.struct(),
                       self.router_w.data_ptr(),
                       None if self.router_bias is None else self.router_bias.data_ptr(),
-                      self.gate_up.struct(), self.down.struct())
+                      self.gate_up.struct(), self.down.struct(), self.act_gz, self.act_gh)
 
     def kernel_count(self, T: int) -> int:
         s = self.struct()
@@ -247,6 +290,17 @@ def quantize_q8_1(x: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(rows, cols // 32 * 36, dtype=torch.uint8, device=x.device)
     _ck(_lib().elq_quantize_q8_1(_ptr(x), xt, rows, cols, _ptr(out), _stream(stream)),
         "elq_quantize_q8_1")
+    return out
+
+
+def quantize_nvfp4(x: torch.Tensor, g: float, stream=None) -> torch.Tensor:
+    """NVFP4 blocks (18 bytes per 32 values) of x [rows, cols] under global scale g."""
+    x = x.contiguous()
+    rows, cols = x.shape
+    xt = {torch.float32: F32, torch.bfloat16: BF16}[x.dtype]
+    out = torch.empty(rows, cols // 32 * 18, dtype=torch.uint8, device=x.device)
+    _ck(_lib().elq_quantize_nvfp4(_ptr(x), xt, rows, cols, float(g), _ptr(out), _stream(stream)),
+        "elq_quantize_nvfp4")
     return out
 
 

@@ -6,33 +6,50 @@ import torch
 
 from quantized_latent_moe_b200 import synth
 
-ORC_FMT = {"q8_0": 8, "q4_0": 2}
+ORC_FMT = {"q8_0": 8, "q4_0": 2, "nvfp4": 100}
+
+
+def nvfp4_globals(w: torch.Tensor) -> torch.Tensor:
+    """Per-matrix NVFP4 global scales of w [n, ...]: amax / 2688 (fp32), 1 for
+    an all-zero matrix -- computed here, on either side's device, from the
+    seeded fp32 weights."""
+    amax = w.reshape(w.shape[0], -1).abs().amax(dim=1)
+    g = amax / torch.tensor(2688.0, dtype=torch.float32, device=w.device)
+    return torch.where(amax > 0, g, torch.ones_like(g))
 
 
 def gpu_layer(wl, layer=0, device="cuda", expert_batch=16):
     from quantized_latent_moe_b200 import elq
     fmt = elq.FMT[wl.fmt]
+    efmt = elq.FMT[wl.expert_fmt]
     dw = synth.dense_weights(wl, layer, device=device)
     rb = dw["router_bias"]
-    ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, dw["router_w"],
+    ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, efmt, dw["router_w"],
                             None if rb is None else rb.to(device))
     ly.set_dense(dw["D"], dw["U"])
+    if efmt == elq.NVFP4:
+        ly.act_gz = ly.act_gh = synth.NVFP4_ACT_GSCALE
     for e0 in range(0, wl.E, expert_batch):
         es = range(e0, min(wl.E, e0 + expert_batch))
         ws = [synth.expert_weights(wl, e, layer, device=device) for e in es]
-        ly.set_experts(e0, torch.stack([w[0] for w in ws]), torch.stack([w[1] for w in ws]),
-                       torch.stack([w[2] for w in ws]))
+        g, u, d = (torch.stack([w[i] for w in ws]) for i in range(3))
+        if efmt == elq.NVFP4:
+            ly.set_experts_nvfp4(e0, g, u, d, nvfp4_globals(torch.cat([g, u], dim=1)), nvfp4_globals(d))
+        else:
+            ly.set_experts(e0, g, u, d)
+        del ws, g, u, d
     torch.cuda.synchronize()
     return ly
 
 
 def oracle_layer(orc, wl, layer=0, experts=None):
     """Oracle layer with only ``experts`` supplied (None = all)."""
-    fmt = ORC_FMT[wl.fmt]
     dw = synth.dense_weights(wl, layer)
     w = {k: (None if v is None else v.numpy()) for k, v in dw.items()}
     w["gate"] = None
-    ly = orc.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, w)
+    if wl.expert_fmt == synth.NVFP4:
+        w["act_gz"] = w["act_gh"] = synth.NVFP4_ACT_GSCALE
+    ly = orc.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, ORC_FMT[wl.fmt], ORC_FMT[wl.expert_fmt], w)
     if experts is None:
         experts = range(wl.E)
     add_experts(ly, wl, experts, layer)

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.elq_version() == 1
+    assert L.elq_version() == 2
     assert L.elq_status_string(0) == b"ok"
     assert L.elq_status_string(-4).startswith(b"workspace")
     assert L.elq_status_string(123) == b"unknown status"
@@ -110,6 +110,78 @@ def test_layer_validation(L):
     assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws_small, 1 << 30, None) == -1
     assert L.elq_moe_layer(None, x, 0, 4, y, ws_small, 1 << 30, None) == -1
     assert L.elq_moe_layer(ctypes.byref(good), x, 0, -1, y, ws_small, 1 << 30, None) == -1
+
+
+def _nv_layer(T_ok=True, **over):
+    """A layer with NVFP4 experts (Q8_0 D/U): global scales per expert matrix."""
+    ly = _layer(L_=256, I=256)
+    base = 1 << 25
+    ly.gate_up = elq.QMat(elq.NVFP4, 8 * 2 * 256, 256, 2 * 256, base, base + 4096, base + 8192)
+    ly.down = elq.QMat(elq.NVFP4, 8 * 256, 256, 256, base + 12288, base + 16384, base + 20480)
+    ly.act_gz, ly.act_gh = 2.0 ** -6, 2.0 ** -6
+    for k_, v in over.items():
+        setattr(ly, k_, v)
+    return ly
+
+
+def test_nvfp4_layer_validation(L):
+    x = ctypes.c_void_p(1 << 27)
+    y = ctypes.c_void_p(1 << 28)
+    ws = ctypes.c_void_p(1 << 26)
+    nv = _nv_layer()
+    # the cluster GEMV path, T <= 8 and T * k <= 64 only
+    for T in (1, 4, 8):
+        assert L.elq_layer_kernel_count(ctypes.byref(nv), T) == 5
+        assert L.elq_workspace_bytes(ctypes.byref(nv), T) > 0
+    for T in (9, 16, 64):
+        assert L.elq_layer_kernel_count(ctypes.byref(nv), T) == 0
+        assert L.elq_moe_layer(ctypes.byref(nv), x, 0, T, y, ws, 1 << 30, None) == -2
+    # the fused flag does not apply: still the five-kernel sequence
+    assert L.elq_layer_kernel_count(ctypes.byref(_nv_layer(flags=1)), 4) == 5
+    # global scales: present, one per expert matrix; activation scales positive
+    bad = _nv_layer()
+    bad.gate_up.gs = None
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -1
+    bad = _nv_layer()
+    bad.down.gs_rows = 128
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -1
+    bad = _nv_layer()
+    bad.down.gs = (1 << 25) + 20482
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -3
+    for v in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.elq_moe_layer(ctypes.byref(_nv_layer(act_gh=v)), x, 0, 1, y, ws, 1 << 30, None) == -1
+    # both expert matrices NVFP4 or neither; never D or U
+    bad = _nv_layer()
+    bad.down = _qm(8, 8 * 256, 256)
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -2
+    bad = _nv_layer()
+    bad.D = elq.QMat(elq.NVFP4, 256, 512, 256, 1 << 20, 2 << 20, 3 << 20)
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -2
+    # whole 8-block chunks: L and I multiples of 256
+    bad = _layer(L_=384, I=256)
+    base = 1 << 25
+    bad.gate_up = elq.QMat(elq.NVFP4, 8 * 512, 384, 512, base, base + 4096, base + 8192)
+    bad.down = elq.QMat(elq.NVFP4, 8 * 384, 256, 384, base + 12288, base + 16384, base + 20480)
+    bad.act_gz, bad.act_gh = 1.0, 1.0
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -2
+    # workspace still checked
+    assert L.elq_moe_layer(ctypes.byref(nv), x, 0, 1, y, ws, 16, None) == -4
+
+
+def test_nvfp4_arena_and_quantiser_validation(L):
+    q, d = elq.SZ(), elq.SZ()
+    # the Q4_0 byte geometry: 16 code bytes and a 16-bit scale word per row and block
+    assert L.elq_arena_bytes(elq.NVFP4, 2048, 1792, ctypes.byref(q), ctypes.byref(d)) == 2048 * 56 * 18
+    assert q.value == 2048 * 56 * 16 and d.value == 2048 * 56 * 2
+    x = ctypes.c_void_p(1 << 27)
+    out = ctypes.c_void_p(1 << 28)
+    assert L.elq_quantize_nvfp4(x, 0, 4, 64, 0.0, out, None) == -1
+    assert L.elq_quantize_nvfp4(x, 0, 4, 64, float("inf"), out, None) == -1
+    assert L.elq_quantize_nvfp4(x, 0, 4, 48, 1.0, out, None) == -2
+    assert L.elq_quantize_nvfp4(x, 7, 4, 64, 1.0, out, None) == -2
+    assert L.elq_quantize_nvfp4(x, 0, 4, 64, 1.0, ctypes.c_void_p((1 << 28) + 1), None) == -3
+    assert L.elq_quantize_nvfp4(None, 0, 0, 64, 1.0, None, None) == 0        # no rows: nothing to do
+    assert L.elq_quantize_weights(elq.NVFP4, x, 128, 64, out, out, None) == -2
 
 
 def test_stack_validation(L):
