@@ -44,7 +44,7 @@ KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "combine",
               "proj_U"]
 KERNELS_FUSED = ["layer"]
-KERNEL_NAMES = {"gate_up": {5: "k_sgemv<{fmt}> gate/up (cluster GEMV, +SwiGLU, Q8_1)",
+KERNEL_NAMES = {"gate_up": {5: "k_sgemv<{fmt}> gate/up (cluster GEMV, +SwiGLU, {afmt})",
                             6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
                             10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
@@ -79,8 +79,43 @@ def peaks():
 
 
 def workload_desc(wl):
+    wfmt = wl.fmt.upper() if wl.expert_fmt == wl.fmt else "%s D/U and %s expert" % (wl.fmt.upper(),
+                                                                                  wl.expert_fmt.upper())
     return ("T=%d, H=%d, L=%d, E=%d, top-%d, I=%d, %s weights, %s input, router bias %s"
-            % (wl.T, wl.H, wl.L, wl.E, wl.k, wl.I, wl.fmt.upper(), wl.x_dtype, wl.bias))
+            % (wl.T, wl.H, wl.L, wl.E, wl.k, wl.I, wfmt, wl.x_dtype, wl.bias))
+
+
+def nvfp4_globals(w):
+    """Per-matrix NVFP4 global scales of w [n, ...]: amax / 2688 in fp32 (1 if all zero)."""
+    import torch
+    amax = w.reshape(w.shape[0], -1).abs().amax(dim=1)
+    g = amax / torch.tensor(2688.0, dtype=torch.float32, device=w.device)
+    return torch.where(amax > 0, g, torch.ones_like(g))
+
+
+def build_layer(elq, synth, wl, li, dev, fused=False, batch=32):
+    """Layer li of the workload on device dev, quantised by the library."""
+    import torch
+    fmt, efmt = elq.FMT[wl.fmt], elq.FMT[wl.expert_fmt]
+    dw = synth.dense_weights(wl, li, device=dev)
+    rb = dw["router_bias"]
+    ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, efmt, dw["router_w"],
+                            None if rb is None else rb.to(dev), device=dev)
+    ly.set_dense(dw["D"], dw["U"])
+    if fused:
+        ly.flags = elq.LAYER_FUSED
+    if efmt == elq.NVFP4:
+        ly.act_gz = ly.act_gh = synth.NVFP4_ACT_GSCALE
+    for e0 in range(0, wl.E, batch):
+        n = min(batch, wl.E - e0)
+        ws_ = [synth.expert_weights(wl, e, li, device=dev) for e in range(e0, e0 + n)]
+        g, u, d = (torch.stack([w[i] for w in ws_]) for i in range(3))
+        if efmt == elq.NVFP4:
+            ly.set_experts_nvfp4(e0, g, u, d, nvfp4_globals(torch.cat([g, u], dim=1)), nvfp4_globals(d))
+        else:
+            ly.set_experts(e0, g, u, d)
+        del ws_, g, u, d
+    return ly
 
 
 # ---------------------------------------------------------------------------
@@ -141,7 +176,7 @@ def oracle_setup(wl, n_tokens, gen_device, tokens=None):
     import numpy as np
     import oracle
     from quantized_latent_moe_b200 import synth
-    fmt = {"q8_0": oracle.Q8_0, "q4_0": oracle.Q4_0}[wl.fmt]
+    fmts = {"q8_0": oracle.Q8_0, "q4_0": oracle.Q4_0, "nvfp4": oracle.NVFP4}
 
     def g(t):
         return t.to("cpu").numpy()
@@ -149,7 +184,9 @@ def oracle_setup(wl, n_tokens, gen_device, tokens=None):
     dw = synth.dense_weights(wl, 0, device=gen_device)
     w = {k: (None if v is None else g(v)) for k, v in dw.items()}
     w["gate"] = None
-    ly = oracle.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, w)
+    if wl.expert_fmt == synth.NVFP4:
+        w["act_gz"] = w["act_gh"] = synth.NVFP4_ACT_GSCALE
+    ly = oracle.Layer(wl.H, wl.L, wl.E, wl.k, wl.I, fmts[wl.fmt], fmts[wl.expert_fmt], w)
     xs = [g(synth.make_x(wl, step=s, T=tokens, device=gen_device).float()) for s in range(n_tokens)]
     need = set()
     for x in xs:
@@ -318,7 +355,7 @@ def traffic_for(kernel, workload):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    e = d.get(kernel)
+    e = d.get("%s@%s" % (kernel, workload)) or d.get(kernel)
     if not e or e.get("source_hash") != source_hash() or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
@@ -429,28 +466,10 @@ def run_elq(args):
         dist.barrier()
     elq.lib()
     wl = synth.WORKLOADS[args.workload]
-    fmt = elq.FMT[wl.fmt]
     stream = torch.cuda.current_stream()
 
     # distinct layer copies (layer index = copy + 8 * rank) and inputs
-    layers = []
-    for c in range(args.copies):
-        li = c + args.copies * rank
-        dw = synth.dense_weights(wl, li, device=dev)
-        rb = dw["router_bias"]
-        ly = elq.Layer.allocate(wl.H, wl.L, wl.E, wl.k, wl.I, fmt, fmt, dw["router_w"],
-                                None if rb is None else rb.to(dev), device=dev)
-        ly.set_dense(dw["D"], dw["U"])
-        if args.fused:
-            ly.flags = elq.LAYER_FUSED
-        for e0 in range(0, wl.E, 32):
-            n = min(32, wl.E - e0)
-            ws_ = [synth.expert_weights(wl, e, li, device=dev) for e in range(e0, e0 + n)]
-            ly.set_experts(e0, torch.stack([w[0] for w in ws_]), torch.stack([w[1] for w in ws_]),
-                           torch.stack([w[2] for w in ws_]))
-            del ws_
-        layers.append(ly)
-        del dw
+    layers = [build_layer(elq, synth, wl, c + args.copies * rank, dev, args.fused) for c in range(args.copies)]
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     S = args.inputs
@@ -562,10 +581,12 @@ def run_elq(args):
     dev_ms, e2e_ms = max_over_ranks([dev_ms, e2e_ms], world, dev)
 
     if rank == 0:
-        blk = 34 if wl.fmt == "q8_0" else 18
+        blk = 34 if wl.fmt == "q8_0" else 18              # D and U blocks
+        eblk = 34 if wl.expert_fmt == "q8_0" else 18      # expert blocks (Q4_0 and NVFP4: 18 B)
+        ablk = 18 if wl.expert_fmt == "nvfp4" else 36     # the experts' activation blocks
         nb_L, nb_H, nb_I = wl.L // 32, wl.H // 32, wl.I // 32
-        gu_w = act * 2 * wl.I * nb_L * blk
-        dn_w = act * wl.L * nb_I * blk
+        gu_w = act * 2 * wl.I * nb_L * eblk
+        dn_w = act * wl.L * nb_I * eblk
         du_w = (wl.L * nb_H + wl.H * nb_L) * blk
         rt_w = wl.E * wl.L * 4
         P = wl.T * wl.k
@@ -576,7 +597,7 @@ def run_elq(args):
         layer_bytes = gu_w + dn_w + du_w + rt_w
         # activations the layer must read or write once: x, y, and the Q8_1 rows between the steps
         x_bytes = wl.T * wl.H * (2 if wl.x_dtype == "bf16" else 4)
-        act_bytes = x_bytes + wl.T * wl.H * 4 + wl.T * nb_L * 36 * 2 + P * nb_I * 36
+        act_bytes = x_bytes + wl.T * wl.H * 4 + wl.T * nb_L * (36 + ablk) + P * nb_I * ablk
         if launches_per_step == 1:
             lay_ms = kern_ms[0]
             gu_ms = dn_ms = None
@@ -619,9 +640,12 @@ def run_elq(args):
                 "note": "each fraction = that bound's time / the launch's event-timed time; the epilogue bound "
                         "uses the measured fma.rn.f32x2 instruction rate"}
         else:
-            gu_bytes = gu_w + wl.T * nb_L * 36 + P * nb_I * 36           # weights + zq + hq
+            gu_bytes = gu_w + wl.T * nb_L * ablk + P * nb_I * ablk       # weights + zq + hq
             achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-            roof = {"bound": "hbm", "kernel": KERNEL_NAMES["gate_up"][launches_per_step].format(fmt=wl.fmt.upper()),
+            afmt = "NVFP4" if wl.expert_fmt == "nvfp4" else "Q8_1"
+            efmt = wl.expert_fmt.upper()
+            roof = {"bound": "hbm",
+                    "kernel": KERNEL_NAMES["gate_up"][launches_per_step].format(fmt=efmt, afmt=afmt),
                     "achieved": achieved,
                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
                     "traffic": traffic_for("gate_up", wl.name), "algorithmic_bytes_per_launch": gu_bytes}

@@ -392,17 +392,33 @@ __device__ __forceinline__ void s_dots(const SArgs& g, const SUnit& u, const uin
     }
 }
 
+// Sum over one 16-value micro-block of (2 w)(2 a): the row's 16 codes in
+// w0, w1 (codes 0..7, 8..15) against the 16 doubled activation values as
+// signed bytes in a (four per word, in order): the positive codes' doubled
+// magnitudes and the negative codes' (byte permutes of the code nibbles)
+// each in a dp4a chain, the second chain subtracted.
+__device__ __forceinline__ int nv_dot16(uint32_t w0, uint32_t w1, const uint4& a) {
+    const uint32_t n0 = w0 ^ 0x88888888u, n1 = w1 ^ 0x88888888u;
+    int p = __dp4a((int)e2m1x4_pos(w0), (int)a.x, 0);
+    int n = __dp4a((int)e2m1x4_pos(n0), (int)a.x, 0);
+    p = __dp4a((int)e2m1x4_pos(w0 >> 16), (int)a.y, p);
+    n = __dp4a((int)e2m1x4_pos(n0 >> 16), (int)a.y, n);
+    p = __dp4a((int)e2m1x4_pos(w1), (int)a.z, p);
+    n = __dp4a((int)e2m1x4_pos(n1), (int)a.z, n);
+    p = __dp4a((int)e2m1x4_pos(w1 >> 16), (int)a.w, p);
+    n = __dp4a((int)e2m1x4_pos(n1 >> 16), (int)a.w, n);
+    return p - n;
+}
+
 // Scratch of the NVFP4 dot: per (token, block) of the chunk the activations'
 // 32 doubled codes as signed bytes, then separately their two scales.
 constexpr int kSNvScratch = kSMaxT * kChunk * 32 + kSMaxT * kChunk * 8;
 
 // The NVFP4 form of s_dots.  The warp first expands its tokens' activation
 // blocks (18-byte NVFP4) into signed doubled codes and fp32 scales in its
-// scratch; then, block by block, each lane expands its row's 32 codes once
-// into the doubled magnitudes of the positive and of the negative codes (byte
-// permutes) and takes, for every token, isum = dp4a(pos, a) - dp4a(neg, a)
-// per 16-value micro-block, and part = fmaf(isum, s_w * s_a, part) in
-// micro-block order.  The global scales are applied in the epilogue.
+// scratch; then, token by token, each lane takes its row's 16 micro-block
+// sums (nv_dot16) and scale products s_w * s_a, and part = fmaf(isum, sc,
+// part) in micro-block order.  The global scales are applied in the epilogue.
 template <int XM>
 __device__ __forceinline__ void s_dots_nv(const SArgs& g, const SUnit& u, const uint8_t* stg, uint8_t* scratch,
                                           uint32_t dst) {
@@ -426,43 +442,39 @@ __device__ __forceinline__ void s_dots_nv(const SArgs& g, const SUnit& u, const 
         }
     }
     __syncwarp();
-    float part[kSMaxT];
-#pragma unroll
-    for (int t = 0; t < kSMaxT; ++t) part[t] = 0.0f;
 #pragma unroll 1
-    for (int kb = 0; kb < kbn; ++kb) {
-        const float2 sw = e4m3x2_to_f32(scales[kb * 32 + lane]);
-        // micro-block by micro-block (each token's chain keeps the block's order)
+    for (int t = 0; t < nt; ++t) {
+        float part = 0.0f;
+        // four blocks at a time: their 8 micro-block sums and scale products
+        // are independent (their loads in flight together), then the ordered
+        // chain of fused multiply-adds over them
 #pragma unroll
-        for (int mb = 0; mb < 2; ++mb) {
-            const uint2 q = *reinterpret_cast<const uint2*>(codes + kb * 512 + lane * 16 + mb * 8);
-            const float swm = mb ? sw.y : sw.x;
-            uint32_t wp[4], wn[4];
-            wp[0] = e2m1x4_pos(q.x);
-            wp[1] = e2m1x4_pos(q.x >> 16);
-            wp[2] = e2m1x4_pos(q.y);
-            wp[3] = e2m1x4_pos(q.y >> 16);
-            wn[0] = e2m1x4_pos(q.x ^ 0x88888888u);
-            wn[1] = e2m1x4_pos((q.x ^ 0x88888888u) >> 16);
-            wn[2] = e2m1x4_pos(q.y ^ 0x88888888u);
-            wn[3] = e2m1x4_pos((q.y ^ 0x88888888u) >> 16);
+        for (int h = 0; h < kChunk; h += 4) {
+            int isum[8];
+            float sc[8];
 #pragma unroll
-            for (int t = 0; t < kSMaxT; ++t) {
-                if (t < nt) {
-                    const uint4 a = lds128(ap + (t * kChunk + kb) * 8 + mb * 4);
+            for (int j = 0; j < 4; ++j) {
+                const int kb = h + j;
+                isum[2 * j] = isum[2 * j + 1] = 0;
+                sc[2 * j] = sc[2 * j + 1] = 0.0f;
+                if (kb < kbn) {
+                    const uint4 q = lds128(codes + kb * 512 + lane * 16);
+                    const float2 sw = e4m3x2_to_f32(scales[kb * 32 + lane]);
+                    const uint32_t* at = ap + (t * kChunk + kb) * 8;
+                    const uint4 a0 = lds128(at), a1 = lds128(at + 4);
                     const float2 sa = as[t * kChunk + kb];
-                    int ps = __dp4a((int)wp[0], (int)a.x, 0), ns = __dp4a((int)wn[0], (int)a.x, 0);
-                    ps = __dp4a((int)wp[1], (int)a.y, ps); ns = __dp4a((int)wn[1], (int)a.y, ns);
-                    ps = __dp4a((int)wp[2], (int)a.z, ps); ns = __dp4a((int)wn[2], (int)a.z, ns);
-                    ps = __dp4a((int)wp[3], (int)a.w, ps); ns = __dp4a((int)wn[3], (int)a.w, ns);
-                    part[t] = __fmaf_rn(__int2float_rn(ps - ns), __fmul_rn(swm, mb ? sa.y : sa.x), part[t]);
+                    isum[2 * j] = nv_dot16(q.x, q.y, a0);
+                    isum[2 * j + 1] = nv_dot16(q.z, q.w, a1);
+                    sc[2 * j] = __fmul_rn(sw.x, sa.x);
+                    sc[2 * j + 1] = __fmul_rn(sw.y, sa.y);
                 }
             }
-        }
-    }
 #pragma unroll
-    for (int t = 0; t < kSMaxT; ++t)
-        if (t < nt) dsmem_st(dst + (uint32_t)((t * 32 + lane) * 4), part[t]);
+            for (int i = 0; i < 8; ++i)
+                if (h + i / 2 < kbn) part = __fmaf_rn(__int2float_rn(isum[i]), sc[i], part);
+        }
+        dsmem_st(dst + (uint32_t)((t * 32 + lane) * 4), part);
+    }
 }
 
 // One out-of-line copy each of the epilogues' quantiser and SwiGLU.

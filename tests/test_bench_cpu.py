@@ -41,11 +41,13 @@ def test_traffic_null_once_sources_change(monkeypatch):
 
 def test_gemv_label_names_the_format():
     from quantized_latent_moe_b200 import synth
-    for wname in ("decode", "verify"):
+    for wname in ("decode", "verify", "decode_nvfp4"):
         wl = synth.WORKLOADS[wname]
-        label = bench.KERNEL_NAMES["gate_up"][5].format(fmt=wl.fmt.upper())
-        assert ("Q4_0" in label) == (wl.fmt == "q4_0"), label
-        assert ("Q8_0" in label) == (wl.fmt == "q8_0"), label
+        afmt = "NVFP4" if wl.expert_fmt == "nvfp4" else "Q8_1"
+        label = bench.KERNEL_NAMES["gate_up"][5].format(fmt=wl.expert_fmt.upper(), afmt=afmt)
+        assert ("Q4_0" in label) == (wl.expert_fmt == "q4_0"), label
+        assert ("Q8_0" in label) == (wl.expert_fmt == "q8_0"), label
+        assert label.count("NVFP4") == (2 if wl.expert_fmt == "nvfp4" else 0), label
 
 
 class _FakeGraph:
