@@ -43,10 +43,13 @@ KERNELS_SMALL_T = ["proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_LARGE_T = ["quant_x", "proj_D", "router", "gate_up", "down", "proj_U"]
 KERNELS_TC = ["quant_x", "pack_x", "proj_D", "router", "slot_map", "pack_z", "gate_up", "down", "combine",
               "proj_U"]
+KERNELS_NVTC = ["quant_x", "pack_x", "proj_D", "quant_z", "router", "slot_map", "pack_z", "gate_up", "down",
+                "combine", "proj_U"]
 KERNELS_FUSED = ["layer"]
 KERNEL_NAMES = {"gate_up": {5: "k_sgemv<{fmt}> gate/up (cluster GEMV, +SwiGLU, {afmt})",
                             6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
-                            10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)"},
+                            10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)",
+                            11: "k_nvgemm gate/up (tcgen05 kind::mxf4nvf4 block-scaled, +SwiGLU, NVFP4)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 
 
@@ -310,6 +313,39 @@ def tensor_peak_int8():
     return _INT8_PEAK
 
 
+_FP4_PEAK = None
+
+
+def tensor_peak_fp4():
+    """Dense fp4 block-scaled tensor-core peak (TFLOP/s), measured on this GPU:
+    one CTA per SM issuing back-to-back tcgen05.mma kind::mxf4nvf4 (M=128,
+    N=256, K=64) from shared memory into TMEM (elq_test_mma_nvf4_rate); the
+    best of five launches after a warm-up one (a burst figure)."""
+    global _FP4_PEAK
+    if _FP4_PEAK is not None:
+        return _FP4_PEAK
+    import torch
+    from quantized_latent_moe_b200 import elq
+    stream = torch.cuda.current_stream()
+    n_mma = 32768
+    flops = 2.0 * 128 * 256 * 64 * n_mma * elq.sm_count()
+    elq.test_mma_nvf4_rate(256)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _, err = elq.test_mma_nvf4_rate(n_mma)
+        e1.record(stream)
+        e1.synchronize()
+        if int(err.item()) != 0:
+            raise RuntimeError("fp4 rate kernel: a bounded wait ran out")
+        best = max(best, flops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    _FP4_PEAK = (best, "measured fp4 (tcgen05.mma kind::mxf4nvf4 block-scaled M128 N256 K64 loop, one CTA per SM, "
+                       "best of 5)")
+    return _FP4_PEAK
+
+
 _F32X2_RATE = None
 
 
@@ -493,7 +529,8 @@ def run_elq(args):
     graphs = GraphSet(G, step)
 
     launches_per_step = layers[0].kernel_count(wl.T)
-    KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 10: KERNELS_TC}[launches_per_step]
+    KERNELS = {1: KERNELS_FUSED, 5: KERNELS_SMALL_T, 6: KERNELS_LARGE_T, 10: KERNELS_TC,
+               11: KERNELS_NVTC}[launches_per_step]
     pos = graphs.run(args.warmup)
     # every graph the timed steps replay is captured, instantiated and
     # replayed once here: the timed region holds replays only
@@ -611,6 +648,23 @@ def run_elq(args):
             dn_ms = kern_ms[KERNELS.index("down")]
         if launches_per_step == 1:
             pass
+        elif launches_per_step == 11:
+            # block-scaled fp4 tensor cores: gate/up is a contraction, against the measured fp4 rate
+            gu_ops = 2.0 * (2 * wl.I) * P * wl.L
+            tpk, tkind = tensor_peak_fp4()
+            achieved = gu_ops / (gu_ms / 1e3) / 1e12
+            # HBM: the codes and the scale atoms of every routed expert, z's and h's packed rows
+            gu_io = act * 2 * wl.I * wl.L * (0.5 + 1.0 / 16) + P * wl.L * (0.5 + 1.0 / 16) + P * wl.I * (0.5 + 1.0 / 16)
+            t_tensor = gu_ops / (tpk * 1e12)
+            t_hbm = gu_io / (hbm_peak * 1e9)
+            t_meas = gu_ms / 1e3
+            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][11], "achieved": achieved, "peak": tpk,
+                    "peak_kind": tkind, "unit": "TFLOP/s (fp4)",
+                    "frac": achieved / tpk, "traffic": traffic_for("gate_up_nv", wl.name),
+                    "algorithmic_ops_per_launch": gu_ops, "algorithmic_bytes_per_launch": gu_io,
+                    "fractions": {"tensor": t_tensor / t_meas, "hbm": t_hbm / t_meas,
+                                  "max_bound": max(t_tensor, t_hbm) / t_meas,
+                                  "bound_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}}}
         elif launches_per_step == 10:
             # tensor-core path: gate/up is a contraction; int8 peak = measured bf16 x the nominal 2x ratio
             gu_ops = 2.0 * (2 * wl.I) * P * wl.L

@@ -92,8 +92,13 @@
  *         r's 16 nibble bytes at byte 16 r of the piece, in the block's order.
  *         NVFP4 -- as Q4_0: row r's 16 code bytes at byte 16 r of a
  *         512-byte piece.
- *     d : fp16 scale at element t*nb*128 + s*nb*32 + kb*32 + r (NVFP4: the
- *         block's two scale bytes, s[0] the low byte).
+ *     d : fp16 scale at element t*nb*128 + s*nb*32 + kb*32 + r.
+ *         NVFP4 (k % 64 == 0): tile t's scales start at element t*nb*256;
+ *         its first nb*128 elements hold the block's two scale bytes (s[0]
+ *         the low byte) in the order above, the next nb*256 bytes the same
+ *         bytes again as the tensor cores' scale-factor atoms: for blocks 2j
+ *         and 2j+1 one 512-byte atom, tile row m = 32 s + r's four scales
+ *         (block 2j s[0], s[1], block 2j+1 s[0], s[1]) at byte 16 r + 4 s.
  *   So the 8 blocks of a 32-row slice that one warp of the decode kernels
  *   reads are one contiguous bulk copy.  q and d must be 256-byte aligned.
  *   The layer's matrices (and elq_latent_proj's) need k % 128 == 0.
@@ -387,6 +392,12 @@ elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q
  * int32 [elq_sm_count()], one accumulator word per CTA; err: device int32,
  * zero before the call, ELQ_ERR_TIMEOUT's code 1 if a wait ran out. */
 elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
+
+/* The fp4 block-scaled tensor-core rate, for the NVFP4 experts' roofline: as
+ * elq_test_mma_i8_rate with n_mma (>= 1) tcgen05.mma kind::mxf4nvf4 of M =
+ * 128, N = 256, K = 64 (2 * 128 * 256 * 64 operations each) into one
+ * accumulator, the scale factors copied to TMEM once. */
+elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
 
 /* The packed fp32 rate, for the tensor-core epilogue's bound: 2 * SM count
  * CTAs of 1024 threads, each thread running n iterations of 8 independent

@@ -15,7 +15,7 @@
 #include "../../include/elq.h"
 #include "elq_decode.cuh"
 #include "elq_sgemv.cuh"
-#include "elq_tc.cuh"
+#include "elq_nvtc.cuh"
 
 using namespace elq;
 
@@ -623,8 +623,8 @@ struct LayerWs {
     int* sync;
     int4* grp;
     float* part_d;          // D chunk partials (fused path)
-    // tensor-core path
-    bool tc;
+    // tensor-core path (int8; nvtc: NVFP4 experts on the block-scaled MMA)
+    bool tc, nvtc;
     int64_t tstride, sstride;   // slots of the dense (tokens) and the expert (pairs, padded) B buffers
     uint8_t *bxq, *bzq, *bhq, *byq;
     float *bxd, *bzd, *bhd, *byd;
@@ -670,6 +670,10 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
         w.su = plan_s(ly->U.fmt, X_Q81_TOKEN, false, H, L, 1, T, false);
         w.small = w.sd.ok && w.sgu.ok && w.sdn.ok && w.su.ok;
     }
+    // NVFP4 experts beyond the cluster GEMV's sizes: D and U on the int8
+    // tensor cores, the experts on the block-scaled ones
+    w.nvtc = ly->gate_up.fmt == ELQ_NVFP4 && !w.small && ly->D.fmt == ELQ_Q8_0 && ly->U.fmt == ELQ_Q8_0;
+    const bool tcbuf = w.tc || w.nvtc;
     const size_t n_sync = w.fused ? (size_t)dec_sync_ints(T, L, I) : 0;
     const size_t n_cnt = 64 + (rblocks + 1) + w.pd.counter_ints + w.pgu.counter_ints + w.pdn.counter_ints +
                          w.pu.counter_ints + (size_t)T * (L / 32) + n_sync;
@@ -684,7 +688,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.cnt_u = adv(w.pu.counter_ints);
     w.cnt_comb = adv((size_t)T * (L / 32));     // per (token, 32-row block): covers the per-tile use too
     w.sync = w.fused ? adv(n_sync) : nullptr;
-    w.xq = w.raw ? nullptr : c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
+    w.xq = (w.raw && !w.nvtc) ? nullptr : c.take<uint8_t>(base, (size_t)T * (H / 32) * 36);
     w.z = c.take<float>(base, (size_t)T * L * 4);
     w.zq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
     w.logits = c.take<float>(base, (size_t)T * E * 4);
@@ -701,7 +705,9 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.ylat = c.take<float>(base, (size_t)T * L * 4);
     w.ylq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
     w.tstride = round16(T);
-    w.sstride = round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
+    // NVFP4: token tiles start on 64 slots and scale atoms cover 128
+    w.sstride = w.nvtc ? (int64_t)round_up((size_t)(P + 64 * (int64_t)std::min<int64_t>(E, P)), 128)
+                       : round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
     w.grp = nullptr;
     w.gtok = nullptr;
     w.part_d = nullptr;
@@ -721,7 +727,7 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
         w.bxd = w.bzd = w.bhd = w.byd = nullptr;
         w.slot_off = w.tt_off = w.pair_slot = nullptr;
         w.cnt_comb_tc = nullptr;
-    } else if (!w.tc) {
+    } else if (!tcbuf) {
         const size_t part = std::max(std::max(w.pd.partial_bytes, w.pgu.partial_bytes),
                                      std::max(w.pdn.partial_bytes, w.pu.partial_bytes));
         w.partial = c.take<float>(base, part);
@@ -774,8 +780,10 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
         if (!(ly->act_gz > 0.0f) || !(ly->act_gh > 0.0f) || !std::isfinite(ly->act_gz) ||
             !std::isfinite(ly->act_gh))
             return ELQ_ERR_INVALID_ARG;
-        // the cluster GEMV's token and pair bounds
-        if (T > kSMaxT || (int64_t)T * k > kSMaxPairs) return ELQ_ERR_UNSUPPORTED;
+        // beyond the cluster GEMV's token and pair bounds: the tensor-core
+        // path, which takes D and U in Q8_0 only
+        if ((T > kSMaxT || (int64_t)T * k > kSMaxPairs) && (ly->D.fmt != ELQ_Q8_0 || ly->U.fmt != ELQ_Q8_0))
+            return ELQ_ERR_UNSUPPORTED;
     }
     if (!ly->router_w) return ELQ_ERR_INVALID_ARG;
     if (!aligned(ly->router_w, 16) || (ly->router_bias && !aligned(ly->router_bias, 4))) return ELQ_ERR_ALIGNMENT;
@@ -877,7 +885,7 @@ SArgs gate_up_s(const elq_layer* ly, const LayerWs& w, int T, int route, const u
     g.d = static_cast<const uint16_t*>(ly->gate_up.d);
     g.nb = L / 32;
     g.q_gstride = (int64_t)(2 * I / kTileRows) * g.nb * slab_bytes(ly->gate_up.fmt);
-    g.d_gstride = (int64_t)(2 * I / kTileRows) * g.nb * kTileRows;
+    g.d_gstride = (int64_t)(2 * I / kTileRows) * d_tile_elems(ly->gate_up.fmt, g.nb);
     g.groups_max = (int)std::min<int64_t>(E, (int64_t)T * k);
     g.route = route;
     g.T = T; g.E = E; g.k = k;
@@ -890,7 +898,7 @@ SArgs gate_up_s(const elq_layer* ly, const LayerWs& w, int T, int route, const u
     g.pfe_q = static_cast<const uint8_t*>(ly->down.q);
     g.pfe_d = reinterpret_cast<const uint8_t*>(ly->down.d);
     g.pfe_qs = (int64_t)(L / kTileRows) * (I / 32) * slab_bytes(ly->down.fmt);
-    g.pfe_ds = (int64_t)(L / kTileRows) * (I / 32) * kScaleSlab;
+    g.pfe_ds = (int64_t)(L / kTileRows) * d_tile_elems(ly->down.fmt, I / 32) * 2;
     g.L = L;
     g.err = w.err;
     g.early = 0;
@@ -905,7 +913,7 @@ SArgs down_s(const elq_layer* ly, const LayerWs& w, int T, int route, const floa
     h.d = static_cast<const uint16_t*>(ly->down.d);
     h.nb = I / 32;
     h.q_gstride = (int64_t)(L / kTileRows) * h.nb * slab_bytes(ly->down.fmt);
-    h.d_gstride = (int64_t)(L / kTileRows) * h.nb * kTileRows;
+    h.d_gstride = (int64_t)(L / kTileRows) * d_tile_elems(ly->down.fmt, h.nb);
     h.groups_max = (int)std::min<int64_t>(E, (int64_t)T * k);
     h.route = route;
     h.T = T; h.E = E; h.k = k;
@@ -1044,7 +1052,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     const int P = T * k;
     if (launch(k_tc_route, dim3(1), dim3(1024), 0, s, pdl, (const int32_t*)w.offsets, (const int32_t*)w.act,
                (const int32_t*)w.n_act, (const int32_t*)w.idx, (const int32_t*)w.pos, P, E, w.slot_off, w.tt_off,
-               w.pair_slot) != cudaSuccess ||
+               w.pair_slot, 16) != cudaSuccess ||
         !mark())
         return ELQ_ERR_CUDA;
     PackArgs pa;
@@ -1103,6 +1111,98 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     return ELQ_OK;
 }
 
+// ---- NVFP4 experts on the block-scaled tensor cores --------------------------
+
+template <int OM>
+cudaError_t launch_nv_t(const NvArgs& g, cudaStream_t s, bool pdl) {
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_nvgemm<OM>, kNvSmem, optin);
+    if (e != cudaSuccess) return e;
+    return launch(k_nvgemm<OM>, dim3(sm_count()), dim3(kTcThreads), (size_t)kNvSmem, s, pdl, g);
+}
+
+// An expert projection: weights m (n_rows = E * rows per expert, k), the
+// activations packed in bq / sfb (K steps of 64 values, sstride slots).
+NvArgs nv_args(const elq_qmat* m, int E, const LayerWs& w, int T, const uint8_t* bq, const uint8_t* sfb, float ags,
+               bool& ok) {
+    NvArgs g;
+    std::memset(&g, 0, sizeof(g));
+    const int nb = m->k / 32;
+    g.d = static_cast<const uint8_t*>(m->d);
+    g.d_tile_bytes = d_tile_elems(ELQ_NVFP4, nb) * 2;
+    g.nb = nb;
+    g.nks = m->k / 64;
+    g.rtiles = m->n_rows / E / kTileRows;
+    g.act = w.act; g.n_act = w.n_act; g.slot_off = w.slot_off; g.offsets = w.offsets; g.tt_off = w.tt_off;
+    g.T = T;
+    g.sfb = sfb;
+    g.wgs = m->gs;
+    g.ags = ags;
+    g.sstride = w.sstride;
+    g.err = w.err;
+    g.budget_ns = kWaitBudgetNs;
+    const cuuint64_t tiles = (cuuint64_t)m->n_rows / kTileRows, nbu = (cuuint64_t)nb;
+    const cuuint64_t da[4] = {128, 4, nbu, tiles}, sa[3] = {nbu * 512, 512, nbu * 2048};
+    const cuuint32_t ba[4] = {128, 4, 2 * kNvKS, 1};
+    const cuuint64_t slots = (cuuint64_t)w.sstride;
+    const cuuint64_t db[3] = {64, slots / 8, (cuuint64_t)g.nks}, sb[2] = {256, slots * 32};
+    const cuuint32_t bb[3] = {64, kTcN / 8, kNvKS};
+    ok = encode_map(&g.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, m->q, da, sa, ba) &&
+         encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, bq, db, sb, bb);
+    return g;
+}
+
+// Slots from the routing, z packed, gate/up (+SwiGLU into the packed h),
+// down (o by slot), the weighted combine (y_lat, its Q8_1 rows, and the
+// packed buffer the U projection reads).  zq: NVFP4 rows under act_gz.
+elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const uint8_t* zq, const float* wts,
+                            float* y_lat, cudaStream_t s, bool pdl, const std::function<bool()>& mark) {
+    const int L = ly->L, E = ly->E, k = ly->k, I = ly->I;
+    const int P = T * k;
+    if (launch(k_tc_route, dim3(1), dim3(1024), 0, s, pdl, (const int32_t*)w.offsets, (const int32_t*)w.act,
+               (const int32_t*)w.n_act, (const int32_t*)w.idx, (const int32_t*)w.pos, P, E, w.slot_off, w.tt_off,
+               w.pair_slot, kTcN) != cudaSuccess ||
+        !mark())
+        return ELQ_ERR_CUDA;
+    NvPackArgs pk;
+    std::memset(&pk, 0, sizeof(pk));
+    pk.x = zq;
+    pk.nb = L / 32;
+    pk.nks = L / 64;
+    pk.offsets = w.offsets;
+    pk.slot_off = w.slot_off;
+    pk.perm = w.perm;
+    pk.kslots = k;
+    pk.E = E;
+    pk.bq = w.bzq;
+    pk.bsf = reinterpret_cast<uint8_t*>(w.bzd);
+    pk.sstride = w.sstride;
+    const int64_t n = w.sstride * pk.nks;
+    if (launch(k_pack_nv, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, pk) != cudaSuccess || !mark())
+        return ELQ_ERR_CUDA;
+    bool ok = false;
+    NvArgs g = nv_args(&ly->gate_up, E, w, T, w.bzq, reinterpret_cast<const uint8_t*>(w.bzd), ly->act_gz, ok);
+    if (!ok) return ELQ_ERR_CUDA;
+    g.hq = w.bhq;
+    g.hsf = reinterpret_cast<uint8_t*>(w.bhd);
+    g.h_nks = I / 64;
+    g.ogs = ly->act_gh;
+    if (launch_nv_t<NV_OUT_SWIGLU>(g, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    NvArgs h = nv_args(&ly->down, E, w, T, w.bhq, reinterpret_cast<const uint8_t*>(w.bhd), ly->act_gh, ok);
+    if (!ok) return ELQ_ERR_CUDA;
+    h.y = w.o;
+    h.y_ld = L;
+    if (launch_nv_t<NV_OUT_F32>(h, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+    CombArgs c;
+    std::memset(&c, 0, sizeof(c));
+    c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
+    c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
+    const int64_t warps = (int64_t)T * (L / 32);
+    if (launch(k_tc_combine, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+        return ELQ_ERR_CUDA;
+    return ELQ_OK;
+}
+
 bool layer_tc(const elq_layer* ly, int T) {
     return tc_path(ly->D.fmt, T) && tc_path(ly->U.fmt, T) && tc_path(ly->gate_up.fmt, T) && tc_path(ly->down.fmt, T);
 }
@@ -1110,6 +1210,10 @@ bool layer_tc(const elq_layer* ly, int T) {
 bool layer_fused(const elq_layer* ly, int T) { return !layer_tc(ly, T) && plan_dec(ly, T).ok; }
 
 int layer_kernels(const elq_layer* ly, int T) {
+    if (ly->gate_up.fmt == ELQ_NVFP4) {
+        const LayerWs w = layer_layout(ly, T, nullptr, ELQ_F32);
+        return w.small ? 5 : w.nvtc ? 11 : 0;
+    }
     if (layer_tc(ly, T)) return 10;
     if (layer_fused(ly, T)) return 1;
     return T <= kRawMaxT ? 5 : 6;
@@ -1136,13 +1240,14 @@ const char* elq_status_string(int32_t status) {
 int32_t elq_version(void) { return 2; }
 
 size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k, size_t* q_bytes, size_t* d_bytes) {
-    if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % 32) {
+    if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % (fmt == ELQ_NVFP4 ? 64 : 32)) {
         if (q_bytes) *q_bytes = 0;
         if (d_bytes) *d_bytes = 0;
         return 0;
     }
     const size_t slabs = (size_t)(n_rows / kTileRows) * (k / 32);
-    const size_t q = slabs * slab_bytes(fmt), d = slabs * kScaleSlab;
+    // NVFP4: each tile's scales twice (per row, and as the tensor cores' atoms)
+    const size_t q = slabs * slab_bytes(fmt), d = slabs * kScaleSlab * (fmt == ELQ_NVFP4 ? 2 : 1);
     if (q_bytes) *q_bytes = q;
     if (d_bytes) *d_bytes = d;
     return q + d;
@@ -1152,7 +1257,7 @@ elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t 
                           void* stream) {
     if (!arena_fmt_ok(fmt)) return ELQ_ERR_UNSUPPORTED;
     if (!aos || !q_out || !d_out || n_rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
-    if (n_rows % kTileRows || k % 32) return ELQ_ERR_UNSUPPORTED;
+    if (n_rows % kTileRows || k % (fmt == ELQ_NVFP4 ? 64 : 32)) return ELQ_ERR_UNSUPPORTED;
     if (!aligned(q_out, 256) || !aligned(d_out, 256)) return ELQ_ERR_ALIGNMENT;
     const int64_t n = (int64_t)n_rows * (k / 32);
     const dim3 grid((unsigned)((n + 255) / 256));
@@ -1160,7 +1265,10 @@ elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t 
     if (fmt == ELQ_Q8_0)
         k_arena_pack<8><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
                                              static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
-    else   // Q4_0, and NVFP4 in the same byte geometry
+    else if (fmt == ELQ_NVFP4)
+        k_arena_pack<kNV><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
+                                               static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
+    else
         k_arena_pack<2><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
                                              static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
     return cuda_status(cudaGetLastError());
@@ -1341,7 +1449,7 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     const int64_t P = (int64_t)T * k;
     const int nw = 32;
     const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
-    if (nv) {
+    if (nv && !w.nvtc) {
         const int gmax = (int)std::min<int64_t>(E, P);
         if (!plan_s(ELQ_NVFP4, X_Q81_PAIR_TOKEN, true, 2 * layer->I, layer->L, gmax, T, true).ok ||
             !plan_s(ELQ_NVFP4, X_Q81_POSITION, false, layer->L, layer->I, gmax, T, true).ok)
@@ -1363,6 +1471,11 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
             return cuda_status(launch_s(down_s(layer, w, T, ROUTE_ARRAYS, weights, y_lat), layer->down.fmt,
                                         X_Q81_POSITION, OUT_F32_COMBINE, pdn, s, true));
         }
+    }
+    if (w.nvtc) {
+        if (cudaMemcpyAsync(w.idx, idx, (size_t)P * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return ELQ_ERR_CUDA;
+        return run_experts_nvtc(layer, w, T, static_cast<const uint8_t*>(z_q8_1), weights, y_lat, s, true,
+                                []() { return true; });
     }
     if (w.tc) {
         // the slot map reads idx from the workspace copy the layer call would have
@@ -1458,8 +1571,8 @@ elq_status elq_workspace_view(const elq_layer* layer, int32_t T, int32_t which, 
     case 7: p = w.offsets; n = (E + 1) * 4; break;
     case 8: p = w.perm; n = P * 4; break;
     case 9: p = w.pos; n = P * 4; break;
-    case 10: p = w.tc ? nullptr : w.hq; n = P * (I / 32) * ablk; break;
-    case 11: p = w.tc ? nullptr : w.o; n = P * L * 4; break;
+    case 10: p = (w.tc || w.nvtc) ? nullptr : w.hq; n = P * (I / 32) * ablk; break;
+    case 11: p = (w.tc || w.nvtc) ? nullptr : w.o; n = P * L * 4; break;
     case 12: p = w.ylat; n = Tz * L * 4; break;
     case 13: p = w.ylq; n = Tz * (L / 32) * 36; break;
     case 14: p = w.n_act; n = 4; break;
@@ -1515,6 +1628,17 @@ elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void
     cudaError_t e = smem_optin(k_test_mma_i8_rate, kRateSmem, optin);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
     return cuda_status(launch(k_test_mma_i8_rate, dim3(sm_count()), dim3(128), (size_t)kRateSmem,
+                              static_cast<cudaStream_t>(stream), false, (int)n_mma, (int*)sink, (int*)err,
+                              kWaitBudgetNs));
+}
+
+elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream) {
+    if (n_mma < 1 || !sink || !err) return ELQ_ERR_INVALID_ARG;
+    static bool optin[kMaxDevices];
+    // the int8 rate kernel's shared-memory request: one CTA (and one TMEM allocation) per SM
+    cudaError_t e = smem_optin(k_test_mma_nvf4_rate, kRateSmem, optin);
+    if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    return cuda_status(launch(k_test_mma_nvf4_rate, dim3(sm_count()), dim3(128), (size_t)kRateSmem,
                               static_cast<cudaStream_t>(stream), false, (int)n_mma, (int*)sink, (int*)err,
                               kWaitBudgetNs));
 }
@@ -1618,7 +1742,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
     LayerWs w = layer_layout(layer, T, ws, x_type);
     const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
-    if (nv && !w.small) return ELQ_ERR_UNSUPPORTED;
+    if (nv && !w.small && !w.nvtc) return ELQ_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1635,6 +1759,43 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         st = run_fused(layer, w, x, x_type, T, y, s);
         if (st != ELQ_OK) return st;
         return mark() ? ELQ_OK : ELQ_ERR_CUDA;
+    }
+    if (w.nvtc) {
+        // NVFP4 experts, many tokens: a1 quantiser, packed x, D on the int8
+        // tensor cores (z), z's NVFP4 rows, router, the block-scaled experts, U
+        const int64_t nblk = (int64_t)T * (H / 32);
+        if (x_type == ELQ_BF16)
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        else
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+                       nblk, w.xq);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        PackArgs pa;
+        std::memset(&pa, 0, sizeof(pa));
+        pa.x = w.xq;
+        pa.nb = H / 32;
+        pa.mode = PACK_DENSE;
+        pa.T = T;
+        pa.bq = w.bxq;
+        pa.bd = w.bxd;
+        pa.bstride = w.tstride;
+        if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32, w.z, nullptr, w.err);
+        if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        const int64_t zblk = (int64_t)T * (L / 32);
+        e = launch(k_quant_nvfp4<false>, dim3((unsigned)((zblk * 32 + 255) / 256)), dim3(256), 0, s, pdl,
+                   (const void*)w.z, zblk, layer->act_gz, w.zq);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits,
+                          w.cnt_router, true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl);
+        if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        st = run_experts_nvtc(layer, w, T, w.zq, w.wts, w.ylat, s, pdl, mark);
+        if (st != ELQ_OK) return st;
+        TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, residual ? TC_OUT_F32_ADD : TC_OUT_F32, y,
+                             nullptr, w.err);
+        if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
+        return ELQ_OK;
     }
     if (w.tc) {
         // prefill: a1 quantiser, packed x, D on the tensor cores (z, zq), router,

@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) k_quant_q8_1(const void* __restrict__ x, 
 template <bool kBF16>
 __global__ void __launch_bounds__(256) k_quant_nvfp4(const void* __restrict__ x, int64_t nblocks, float g,
                                                      uint8_t* __restrict__ out) {
+    pdl_wait();
     const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (blk >= nblocks) return;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(256) k_quant_nvfp4(const void* __restrict__ x,
     else
         v = reinterpret_cast<const float*>(x)[blk * 32 + lane];
     warp_quant_nvfp4(v, g, out + blk * 18);
+    pdl_trigger();
 }
 
 // ============================================================================
@@ -129,6 +131,15 @@ __global__ void __launch_bounds__(256) k_quant_weights(const float* __restrict__
     }
 }
 
+// NVFP4 scales of a tile: nb*128 16-bit words (each row's two micro-block
+// scales per block, as Q4_0's fp16 scales), then the same bytes once more as
+// the tensor cores' scale-factor atoms: per pair of blocks (64 values) one
+// 512-byte atom, row m's four scales (blocks 2j, 2j+1, micro-blocks 0, 1) as
+// one 32-bit word at byte (m % 32) * 16 + (m / 32) * 4.
+__host__ __device__ constexpr int64_t d_tile_elems(int fmt, int nb) {
+    return (int64_t)nb * kTileRows * (fmt == kNV ? 2 : 1);
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(256) k_arena_pack(const uint8_t* __restrict__ aos, int n_rows, int k,
                                                     uint8_t* __restrict__ q, uint16_t* __restrict__ d) {
@@ -141,7 +152,13 @@ __global__ void __launch_bounds__(256) k_arena_pack(const uint8_t* __restrict__ 
     const uint8_t* src = aos + id * bb;
     const int64_t tile = row / kTileRows;
     const int slice = (int)(row % kTileRows) / 32, r = (int)(row % 32);
-    d[tile * nb * kTileRows + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r] = (uint16_t)(src[0] | (src[1] << 8));
+    const uint16_t sw = (uint16_t)(src[0] | (src[1] << 8));
+    d[tile * d_tile_elems(FMT, nb) + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r] = sw;
+    if (FMT == kNV) {
+        // the atom copy: row m = 32 slice + r, byte (kb % 2) * 2 of its word
+        uint8_t* atoms = reinterpret_cast<uint8_t*>(d + tile * d_tile_elems(FMT, nb) + (int64_t)nb * kTileRows);
+        *reinterpret_cast<uint16_t*>(atoms + (int64_t)(kb >> 1) * 512 + r * 16 + slice * 4 + (kb & 1) * 2) = sw;
+    }
     uint32_t words[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const int nq = (FMT == 8) ? 32 : 16;
     for (int i = 0; i < nq; ++i) words[i >> 2] |= (uint32_t)src[2 + i] << (8 * (i & 3));

@@ -1,0 +1,489 @@
+// elq_nvtc.cuh -- NVFP4 expert projections for many tokens on the tensor
+// cores: tcgen05.mma kind::mxf4nvf4 with block scales (E2M1 operands, one
+// E4M3 scale per 16 values of each operand), fp32 accumulators in TMEM.
+//
+// The block-scaled MMA applies both operands' micro-block scales inside the
+// tensor core and accumulates the whole K range in fp32, so the epilogue only
+// multiplies by the two global scales: there is no per-block rescale.  The
+// order of that fp32 accumulation is the hardware's, not the micro-block
+// chain of the GEMV path, so these results agree with the GEMV's to rounding,
+// not bit for bit.
+//
+// One MMA: M = 128 weight rows, N = up to 64 slots, K = 64 values (two
+// 32-value blocks).  Shared-memory operands, K-major without swizzle:
+//  A (weights): [block][slice][32 rows x 16 bytes], one tensor-map copy per
+//    stage from the arena; for the MMA of blocks 2j, 2j+1: LBO = 2048 bytes
+//    (the next 16-byte K chunk), SBO = 128 bytes (the next 8 rows).
+//  B (activations): pre-packed per K step as [slot/8][2][8][16] bytes
+//    (LBO = 128, SBO = 256), the Q8_1 B buffers' geometry.
+// Scale factors go shared memory -> TMEM with tcgen05.cp (32 lanes x 128
+// bits, repeated in all four lane quarters) from 512-byte atoms: row m's four
+// scales of a K step as one 32-bit word at byte (m % 32) * 16 + (m / 32) * 4.
+// The weights' atoms are stored in the arena; the activations' atoms are
+// written by the packing kernel and the SwiGLU epilogue, per 128 slots.
+//
+// CTA: warp 0 issues the copies, warp 1 the scale copies and the MMAs, warps
+// 2..17 drain the accumulators (4 TMEM lane quarters x 4 column quarters).
+#pragma once
+
+#include "elq_tc.cuh"
+
+namespace elq {
+
+// Instruction descriptor of kind::mxf4nvf4: E2M1 x E2M1 -> fp32, both
+// K-major, UE4M3 scales, dense K = 64.
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= (A x SFA) . (B x SFB)^T, scale factors in TMEM at sfa, sfb.
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Shared memory (a 512-byte atom: 32 rows of 16 bytes) -> TMEM columns
+// taddr .. taddr+3 of all 128 lanes (each lane quarter gets the same rows).
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, const void* atom) {
+    const uint64_t desc = umma_desc(atom, 128, 128);
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// Untiled bulk copy global -> shared on an mbarrier (16-byte aligned, size a
+// multiple of 16).  No multicast.
+__device__ __forceinline__ void bulk_g2s_nv(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    bulk_g2s(dst, src, bytes, bar);
+}
+
+constexpr int kNvKS = 4;                       // K steps (64 values each) per stage
+constexpr int kNvStages = 6;
+constexpr int kNvStageA = kNvKS * 4096;
+constexpr int kNvStageB = kNvKS * kTcN * 32;
+constexpr int kNvStageSfa = kNvKS * 512;
+constexpr int kNvStageSfb = kNvKS * 512;
+constexpr int kNvStage = kNvStageA + kNvStageB + kNvStageSfa + kNvStageSfb;
+constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kTcXchg;
+constexpr int kNvAccBufs = 2;                  // accumulators of kTcN columns
+constexpr int kNvSfCol = kNvAccBufs * kTcN;    // scale-factor columns: kNvKS x (SFA 4, SFB 4)
+constexpr int kNvTmemCols = 256;
+static_assert(kNvSfCol + kNvKS * 8 <= kNvTmemCols, "TMEM plan");
+
+enum { NV_OUT_F32 = 0, NV_OUT_SWIGLU = 1 };
+
+struct NvArgs {
+    // tm_a: weight codes, uint32 [tiles][nb][4 slices][128] with strides
+    //       (nb*2048, 512, nb*512) bytes; box [1][2 kNvKS][4][128] -> [block][slice][512 B]
+    // tm_b: packed activation codes, uint32 [K steps][slots/8][64]; box [kNvKS][8][64]
+    CUtensorMap tm_a, tm_b;
+    const uint8_t* d;           // weight scales of the arena (the atoms follow each tile's per-row scales)
+    int64_t d_tile_bytes;       // bytes of a tile's scales
+    int nb, nks, rtiles;        // blocks, K steps, row tiles per group
+    // groups: the routed experts (slot_off, offsets per expert, tt_off per active expert)
+    const int32_t* act;
+    const int32_t* n_act;
+    const int32_t* slot_off;
+    const int32_t* offsets;
+    const int32_t* tt_off;
+    int T;
+    const uint8_t* sfb;         // activation atoms: [slot/128][nks][512]
+    // global scales: weights (per expert) x the activations' static scale
+    const float* wgs;
+    float ags;
+    // outputs
+    float* y;                   // NV_OUT_F32: fp32 rows by slot
+    int64_t y_ld;
+    uint8_t* hq;                // NV_OUT_SWIGLU: the down projection's B codes
+    uint8_t* hsf;               //   and its activation atoms
+    int64_t sstride;            // slots of the B buffers (multiple of 128)
+    int h_nks;                  // K steps of h (I / 64)
+    float ogs;                  // the static scale of h
+    int* err;
+    uint64_t budget_ns;
+};
+
+__device__ __forceinline__ int nv_units(const NvArgs& g) { return __ldcg(g.tt_off + __ldcg(g.n_act)) * g.rtiles; }
+
+// Unit u: row tile rt of the routed expert whose token tiles hold u / rtiles
+// (the same order as the int8 path: a weight tile against all its expert's
+// token tiles in turn).
+__device__ __forceinline__ TcUnit nv_unit(const NvArgs& g, int u) {
+    TcUnit r;
+    const int q = u / g.rtiles;
+    const int na = __ldcg(g.n_act);
+    int lo = 0, hi = na;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldcg(g.tt_off + mid) <= q) lo = mid; else hi = mid;
+    }
+    r.e = __ldcg(g.act + lo);
+    const int base = __ldcg(g.tt_off + lo);
+    const int n_q = __ldcg(g.tt_off + lo + 1) - base;
+    const int v = u - base * g.rtiles;
+    r.rt = v / n_q;
+    const int tt = v - r.rt * n_q;
+    r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
+    const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
+    r.nvalid = min(kTcN, cnt - tt * kTcN);
+    r.ncols = (r.nvalid + 15) & ~15;
+    r.valid = r.nvalid > 0;
+    return r;
+}
+
+// ---- packing: NVFP4 rows (18-byte blocks) -> B codes and scale atoms ---------
+// Slot s of expert e (s - slot_off[e] < count(e)) holds the row of its pair
+// perm[offsets[e] + s - slot_off[e]] / k; other slots hold zeros.  One thread
+// per (slot, K step): the two blocks' 32 code bytes to [K step][slot/8][2][8][16],
+// their four scales as one word of the slot's atom.
+struct NvPackArgs {
+    const uint8_t* x;           // NVFP4 rows, nb blocks each
+    int nb, nks;
+    const int32_t* offsets;
+    const int32_t* slot_off;
+    const int32_t* perm;
+    int kslots, E;
+    uint8_t* bq;
+    uint8_t* bsf;
+    int64_t sstride;
+};
+
+__global__ void __launch_bounds__(256) k_pack_nv(NvPackArgs a) {
+    pdl_wait();
+    const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= a.sstride * a.nks) return;
+    const int64_t slot = id / a.nks;
+    const int ks = (int)(id % a.nks);
+    int lo = 0, hi = a.E;       // slot_off[lo] <= slot < slot_off[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldcg(a.slot_off + mid) <= slot) lo = mid; else hi = mid;
+    }
+    int64_t row = -1;
+    if (slot < __ldcg(a.slot_off + a.E)) {
+        const int i = (int)(slot - __ldcg(a.slot_off + lo));
+        const int n = __ldcg(a.offsets + lo + 1) - __ldcg(a.offsets + lo);
+        if (i < n) row = __ldcg(a.perm + __ldcg(a.offsets + lo) + i) / a.kslots;
+    }
+    uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sw = 0;
+    if (row >= 0) {
+        // two 18-byte blocks (2-byte aligned): scales, then 16 code bytes each
+        const uint16_t* src = reinterpret_cast<const uint16_t*>(a.x + (row * a.nb + 2 * ks) * 18);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const uint16_t* sb = src + 9 * b;
+            sw |= (uint32_t)__ldcg(sb) << (16 * b);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                c[4 * b + j] = (uint32_t)__ldcg(sb + 1 + 2 * j) | ((uint32_t)__ldcg(sb + 2 + 2 * j) << 16);
+        }
+    }
+    uint8_t* dst = a.bq + (int64_t)ks * a.sstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(c[0], c[1], c[2], c[3]);
+    *reinterpret_cast<uint4*>(dst + 128) = make_uint4(c[4], c[5], c[6], c[7]);
+    *reinterpret_cast<uint32_t*>(a.bsf + ((slot >> 7) * a.nks + ks) * 512 + (slot & 31) * 16 + ((slot >> 5) & 3) * 4) =
+        sw;
+    pdl_trigger();
+}
+
+// The h blocks of one (slot, 32-value block) from four lanes of eight values
+// each (lanes 2q, 2q+1 share micro-block q): NVFP4 under global scale gs,
+// written as the down projection's B codes and scale-atom bytes.
+__device__ __forceinline__ void nv_quant_h8(const float (&h)[8], bool on, float gs, int qd, int64_t slot, int kbh,
+                                            const NvArgs& g) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(h[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    const uint32_t s = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs));
+    const float den = __fmul_rn(e4m3x2_to_f32(s).x, gs);
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float x0 = den != 0.0f ? __fdiv_rn(h[i], den) : 0.0f;
+        const float x1 = den != 0.0f ? __fdiv_rn(h[i + 1], den) : 0.0f;
+        w |= f32x2_to_e2m1x2(x0, x1) << (4 * i);
+    }
+    if (on) {
+        const int ks = kbh >> 1;
+        uint8_t* dst = g.hq + (int64_t)ks * g.sstride * 32 + (slot >> 3) * 256 + (kbh & 1) * 128 + (slot & 7) * 16 +
+                       qd * 4;
+        *reinterpret_cast<uint32_t*>(dst) = w;
+        if ((qd & 1) == 0)
+            g.hsf[((slot >> 7) * g.h_nks + ks) * 512 + (slot & 31) * 16 + ((slot >> 5) & 3) * 4 + (kbh & 1) * 2 +
+                  (qd >> 1)] = (uint8_t)s;
+    }
+}
+
+// ---- the GEMM ------------------------------------------------------------------
+
+template <int OM>
+__global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant__ NvArgs g) {
+    extern __shared__ __align__(1024) uint8_t nvsm[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(nvsm);            // [stages]: copies landed
+    uint64_t* empty = full + kNvStages;                             // [stages]: MMAs done with them
+    uint64_t* tfull = empty + kNvStages;                            // [2]: a unit's accumulator complete
+    uint64_t* tempty = tfull + kNvAccBufs;                          // [2]: ... and drained
+    uint64_t* xfull = tempty + kNvAccBufs;
+    uint64_t* xempty = xfull + 1;
+    uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(xempty + 1);
+    int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
+    uint8_t* stages = nvsm + 1024;
+    float* xchg = reinterpret_cast<float*>(nvsm + 1024 + kNvStages * kNvStage);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kNvStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < kNvAccBufs; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kTcEpiWarps);
+        }
+        mbar_init(xfull, kTcEpiWarps);
+        mbar_init(xempty, kTcEpiWarps);
+        *abort_sm = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_sm, kNvTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_sm;
+    pdl_wait();
+
+    const int n_units = nv_units(g);
+    const int u0 = (int)((int64_t)n_units * blockIdx.x / gridDim.x);
+    const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
+    const int kstages = g.nks / kNvKS;
+    volatile int* abort_v = abort_sm;
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int it = 0;
+            for (int u = u0; u < u1 && !*abort_v; ++u) {
+                const TcUnit un = nv_unit(g, u);
+                if (!un.valid) continue;
+                const int tile = un.e * g.rtiles + un.rt;
+                const uint8_t* sfa = g.d + (int64_t)tile * g.d_tile_bytes + (int64_t)g.nb * 256;
+                const uint8_t* sfb = g.sfb + (int64_t)(un.slot0 >> 7) * g.nks * 512;
+                for (int ks = 0; ks < kstages; ++ks, ++it) {
+                    const int s = it % kNvStages;
+                    if (it >= kNvStages &&
+                        !mbar_wait_bounded(&empty[s], (uint32_t)((it / kNvStages - 1) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    uint8_t* st = stages + s * kNvStage;
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)kNvStage);
+                    tma_load_4d(st, &g.tm_a, 0, 0, ks * 2 * kNvKS, tile, &full[s]);
+                    tma_load_3d(st + kNvStageA, &g.tm_b, 0, un.slot0 >> 3, ks * kNvKS, &full[s]);
+                    bulk_g2s(st + kNvStageA + kNvStageB, sfa + (int64_t)ks * kNvKS * 512, kNvStageSfa, &full[s]);
+                    bulk_g2s(st + kNvStageA + kNvStageB + kNvStageSfa, sfb + (int64_t)ks * kNvKS * 512, kNvStageSfb,
+                             &full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- scale copies and MMAs ----------------
+        if (lane == 0) {
+            int it = 0, uc = 0;
+            const uint32_t sf = tmem + (uint32_t)kNvSfCol;
+            for (int u = u0; u < u1 && !*abort_v; ++u, ++uc) {
+                const TcUnit un = nv_unit(g, u);
+                if (!un.valid) {
+                    --uc;
+                    continue;
+                }
+                const int ab = uc % kNvAccBufs;
+                if (uc >= kNvAccBufs &&
+                    !mbar_wait_bounded(&tempty[ab], (uint32_t)((uc / kNvAccBufs - 1) & 1), g.err, g.budget_ns)) {
+                    *abort_v = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t idesc = umma_idesc_nvf4(128, un.ncols);
+                const uint32_t dacc = tmem + (uint32_t)(ab * kTcN);
+                const uint32_t bsub = (uint32_t)((un.slot0 & 127) >> 5);   // the tile's words of the slot atoms
+                for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
+                    const int s = it % kNvStages;
+                    if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kNvStages) & 1), g.err, g.budget_ns)) {
+                        *abort_v = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t* st = stages + s * kNvStage;
+                    for (int k = 0; k < kNvKS; ++k) {
+                        const uint32_t sfa_t = sf + (uint32_t)(k * 8), sfb_t = sfa_t + 4u;
+                        tmem_cp_atom(sfa_t, st + kNvStageA + kNvStageB + k * 512);
+                        tmem_cp_atom(sfb_t, st + kNvStageA + kNvStageB + kNvStageSfa + k * 512);
+                        const uint64_t adesc = umma_desc(st + k * 4096, 2048, 128);
+                        const uint64_t bdesc = umma_desc(st + kNvStageA + k * kTcN * 32, 128, 256);
+                        umma_nvf4(dacc, adesc, bdesc, idesc, sfa_t, sfb_t + bsub, (ks | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                umma_commit(&tfull[ab]);
+            }
+            // let the last MMAs finish before the TMEM is freed
+            if (uc > 0) {
+                const int last = uc - 1;
+                mbar_wait_bounded(&tfull[last % kNvAccBufs], (uint32_t)((last / kNvAccBufs) & 1), nullptr,
+                                  g.budget_ns);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int ew = warp - 2;
+        const int sp = warp & 3;                  // TMEM lane quarter
+        const int c0 = (ew >> 2) * kTcEpiCols;    // accumulator columns (slots) c0 .. c0+15
+        const int row = sp * 32 + lane;           // weight row within the tile
+        int uc = 0, xc = 0;
+        for (int u = u0; u < u1 && !*abort_v; ++u) {
+            const TcUnit un = nv_unit(g, u);
+            if (!un.valid) continue;
+            const int ab = uc % kNvAccBufs;
+            if (!warp_wait_bounded(&tfull[ab], (uint32_t)((uc / kNvAccBufs) & 1), g.err, g.budget_ns)) {
+                *abort_v = 1;
+                break;
+            }
+            ++uc;
+            tc_fence_after();
+            float acc[kTcEpiCols];
+            const bool active = c0 < un.ncols;
+            if (active) {
+                uint32_t rc[kTcEpiCols];
+                tmem_ld16(tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(ab * kTcN + c0), rc);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < kTcEpiCols; ++j) acc[j] = __uint_as_float(rc[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kTcEpiCols; ++j) acc[j] = 0.0f;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[ab]);
+            const float gq = __fmul_rn(__ldg(g.wgs + un.e), g.ags);
+#pragma unroll
+            for (int j = 0; j < kTcEpiCols; ++j) acc[j] = __fmul_rn(acc[j], gq);
+            const int nv = un.nvalid;
+            const int64_t slot0 = un.slot0;
+            if (OM == NV_OUT_SWIGLU) {
+                // transpose the tile through shared memory ([slot][row], padded), then four
+                // threads per (slot, h block): h row 32 hb + i takes gate row 32 hb + i and up
+                // row 64 + 32 hb + i of the tile
+                if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
+                    *abort_v = 1;
+                    break;
+                }
+#pragma unroll
+                for (int j = 0; j < kTcEpiCols; ++j) xchg[(c0 + j) * kTcXld + row] = acc[j];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xfull);
+                if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
+                    *abort_v = 1;
+                    break;
+                }
+                {
+                    const int task = ew * 32 + lane;          // 0 .. 511
+                    const int b = task >> 2, qd = task & 3;
+                    const int t = b >> 1, hb = b & 1;
+                    const bool on = t < nv;
+                    float h[8];
+                    if (on) {
+                        const float* gr = xchg + t * kTcXld + hb * 32 + qd * 8;
+                        const float* ur = gr + 64;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) h[i] = 0.0f;
+                    }
+                    nv_quant_h8(h, on, g.ogs, qd, slot0 + t, un.rt * 2 + hb, g);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xempty);
+                ++xc;
+                continue;
+            }
+#pragma unroll
+            for (int j = 0; j < kTcEpiCols; ++j) {
+                const int t = c0 + j;
+                if (t < nv) g.y[(slot0 + t) * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kNvTmemCols);
+    pdl_trigger();
+}
+
+// ---- measurement: the fp4 block-scaled tensor-core rate ------------------------
+//
+// One CTA per SM, one thread issuing n_mma tcgen05.mma kind::mxf4nvf4 (M = 128,
+// N = 256, K = 64, 2 * 128 * 256 * 64 operations each) from fixed shared-memory
+// operands and scale atoms (copied to TMEM once) into one accumulator, then a
+// bounded wait for them (ELQ_ERR_TIMEOUT's code 1 in *err if it runs out).
+constexpr int kRateNvSmem = 1024 + (128 + kRateN) * 32 + 2 * 512;
+
+__global__ void __launch_bounds__(128, 1) k_test_mma_nvf4_rate(int n_mma, int* sink, int* err, uint64_t budget_ns) {
+    extern __shared__ __align__(1024) uint8_t rnsm_[];
+    uint64_t* done = reinterpret_cast<uint64_t*>(rnsm_);
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(rnsm_ + 8);
+    uint8_t* a = rnsm_ + 1024;                // 128 x 32 bytes (64 E2M1 codes a row)
+    uint8_t* b = a + 128 * 32;                // 256 x 32 bytes
+    uint8_t* sf = b + kRateN * 32;            // two scale atoms (all 1.0)
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (128 + kRateN) * 32 / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(a)[i] = 0x22222222u;                     // every value 1.0
+    for (int i = threadIdx.x; i < 2 * 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sf)[i] = 0x38383838u;
+    if (threadIdx.x == 0) {
+        mbar_init(done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tbase;
+    if (threadIdx.x == 0) {
+        const uint32_t sfa = tmem + (uint32_t)kRateN, sfb = sfa + 4u;
+        tmem_cp_atom(sfa, sf);
+        tmem_cp_atom(sfb, sf + 512);
+        const uint32_t idesc = umma_idesc_nvf4(128, kRateN);
+        const uint64_t ad = umma_desc(a, 2048, 128), bd = umma_desc(b, 128, 256);
+        for (int i = 0; i < n_mma; ++i) umma_nvf4(tmem, ad, bd, idesc, sfa, sfb, i > 0 ? 1u : 0u);
+        umma_commit(done);
+    }
+    __syncwarp();
+    const bool ok = warp_wait_bounded(done, 0, err, budget_ns);
+    tc_fence_after();
+    if (warp == 0) {
+        uint32_t r[16];
+        tmem_ld16(tmem, r);
+        tmem_ld_wait();
+        if (ok && threadIdx.x == 0) sink[blockIdx.x] = (int)r[0];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace elq

@@ -238,7 +238,7 @@ __device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, 
     bulk_g2s(stg, g.q + u.grp.x * g.q_gstride + ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
              cb, bar);
     bulk_g2s(stg + g.scales_off,
-             g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows + (int64_t)u.s * g.nb * 32 +
+             g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) + (int64_t)u.s * g.nb * 32 +
                  (int64_t)r.kb0 * 32,
              sb, bar);
 }
@@ -596,7 +596,7 @@ __device__ __forceinline__ void s_prefetch_own(const SArgs& g, const uint8_t* rs
         bulk_prefetch_l2(g.q + u.grp.x * g.q_gstride +
                              ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
                          (uint32_t)(r.nblk * SL::kCodes));
-        bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + (int64_t)u.tile * g.nb * kTileRows + (int64_t)u.s * g.nb * 32 +
+        bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) + (int64_t)u.s * g.nb * 32 +
                              (int64_t)r.kb0 * 32,
                          (uint32_t)(r.nblk * 64));
     }

@@ -252,12 +252,14 @@ __global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
 constexpr int kTcN = 64;            // tokens per tile
 
 // ---- routing -> padded slots -------------------------------------------------
-// slot_off[e] = sum over e' < e of roundup(count(e'), 16); tt_off[a] = sum over
+// slot_off[e] = sum over e' < e of roundup(count(e'), align) (align 16, or 64
+// for the NVFP4 path, whose token tiles must start on 64 slots); tt_off[a] = sum over
 // active experts a' < a of ceil(count / 64); pair_slot[p] = the slot of pair p.
 // One CTA.
 __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const int32_t* act, const int32_t* n_act,
                                                    const int32_t* idx, const int32_t* pos, int P, int E,
-                                                   int32_t* slot_off, int32_t* tt_off, int32_t* pair_slot) {
+                                                   int32_t* slot_off, int32_t* tt_off, int32_t* pair_slot,
+                                                   int align) {
     pdl_wait();
     __shared__ int s_slot[1025];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
         const int per = (E + 31) / 32;
         const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
         int local = 0;
-        for (int e = e0; e < e1; ++e) local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + 15) & ~15;
+        for (int e = e0; e < e1; ++e) local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + align - 1) & -align;
         int incl = local;
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
         for (int e = e0; e < e1; ++e) {
             s_slot[e] = run;
             slot_off[e] = run;
-            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + 15) & ~15;
+            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + align - 1) & -align;
         }
         if (lane == 31) {
             s_slot[E] = incl;

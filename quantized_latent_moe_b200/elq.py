@@ -71,6 +71,7 @@ SIGNATURES = {
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
     "elq_test_expf": (I32, [V, V, I64, V]),
     "elq_test_mma_i8_rate": (I32, [I32, V, V, V]),
+    "elq_test_mma_nvf4_rate": (I32, [I32, V, V, V]),
     "elq_sm_count": (I32, []),
     "elq_test_f32x2_rate": (I32, [I32, V, V]),
     "elq_test_fused_timeout": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, ctypes.c_uint64, V]),
@@ -218,13 +219,13 @@ class Layer:
             _ck(_lib().elq_quantize_nvfp4(_ptr(de), F32, L, I, float(g_down[e]), _ptr(aos_dn[e]),
                                           _stream(stream)), "elq_quantize_nvfp4")
         per_q = (2 * I // 128) * (L // 32) * SLAB[NVFP4]
-        per_d = (2 * I // 128) * (L // 32) * 256
+        per_d = (2 * I // 128) * (L // 32) * 512      # per-row scales, then the scale atoms
         _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_gu), n * 2 * I, L,
                                   ctypes.c_void_p(gu.q.data_ptr() + e0 * per_q),
                                   ctypes.c_void_p(gu.d.data_ptr() + e0 * per_d), _stream(stream)),
             "elq_arena_pack")
         dq = (L // 128) * (I // 32) * SLAB[NVFP4]
-        dd = (L // 128) * (I // 32) * 256
+        dd = (L // 128) * (I // 32) * 512
         _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_dn), n * L, I, ctypes.c_void_p(dn.q.data_ptr() + e0 * dq),
                                   ctypes.c_void_p(dn.d.data_ptr() + e0 * dd), _stream(stream)),
             "elq_arena_pack")
@@ -469,6 +470,16 @@ def test_mma_i8_rate(n_mma: int, device="cuda", stream=None):
     sink = torch.zeros(n, dtype=torch.int32, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     _ck(_lib().elq_test_mma_i8_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_i8_rate")
+    return sink, err
+
+
+def test_mma_nvf4_rate(n_mma: int, device="cuda", stream=None):
+    """Launches the fp4 block-scaled tensor-core rate kernel
+    (elq_test_mma_nvf4_rate) on the current stream; returns (sink, err)."""
+    n = int(_lib().elq_sm_count())
+    sink = torch.zeros(n, dtype=torch.int32, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    _ck(_lib().elq_test_mma_nvf4_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_nvf4_rate")
     return sink, err
 
 

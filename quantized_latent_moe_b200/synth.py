@@ -151,6 +151,9 @@ WORKLOADS = {
     # decode with NVFP4 latent experts (D/U stay Q8_0): the decode shapes
     "decode_nvfp4": Workload("decode_nvfp4", 5, 1, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal",
                              ex_fmt=NVFP4),
+    # prefill with NVFP4 latent experts: the prefill shapes and router skew
+    "prefill_nvfp4": Workload("prefill_nvfp4", 6, 2048, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "zipf",
+                              ex_fmt=NVFP4),
     # resident stack: 48 layers, 32 sequences decoding one token per step
     "stack": Workload("stack", 4, 32, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal",
                       layers=48, steps=64, residual=True),

@@ -133,9 +133,17 @@ def test_nvfp4_layer_validation(L):
     for T in (1, 4, 8):
         assert L.elq_layer_kernel_count(ctypes.byref(nv), T) == 5
         assert L.elq_workspace_bytes(ctypes.byref(nv), T) > 0
+    # beyond: the block-scaled tensor cores (D and U on the int8 ones, Q8_0 only)
+    for T in (9, 16, 64, 2048):
+        assert L.elq_layer_kernel_count(ctypes.byref(nv), T) == 11
+        assert L.elq_workspace_bytes(ctypes.byref(nv), T) > 0
+    nv4 = _nv_layer()
+    nv4.D = _qm(2, 256, 512)
+    nv4.U = _qm(2, 512, 256)
+    assert L.elq_layer_kernel_count(ctypes.byref(nv4), 4) == 5
     for T in (9, 16, 64):
-        assert L.elq_layer_kernel_count(ctypes.byref(nv), T) == 0
-        assert L.elq_moe_layer(ctypes.byref(nv), x, 0, T, y, ws, 1 << 30, None) == -2
+        assert L.elq_layer_kernel_count(ctypes.byref(nv4), T) == 0
+        assert L.elq_moe_layer(ctypes.byref(nv4), x, 0, T, y, ws, 1 << 30, None) == -2
     # the fused flag does not apply: still the five-kernel sequence
     assert L.elq_layer_kernel_count(ctypes.byref(_nv_layer(flags=1)), 4) == 5
     # global scales: present, one per expert matrix; activation scales positive
@@ -170,9 +178,11 @@ def test_nvfp4_layer_validation(L):
 
 def test_nvfp4_arena_and_quantiser_validation(L):
     q, d = elq.SZ(), elq.SZ()
-    # the Q4_0 byte geometry: 16 code bytes and a 16-bit scale word per row and block
-    assert L.elq_arena_bytes(elq.NVFP4, 2048, 1792, ctypes.byref(q), ctypes.byref(d)) == 2048 * 56 * 18
-    assert q.value == 2048 * 56 * 16 and d.value == 2048 * 56 * 2
+    # the Q4_0 byte geometry (16 code bytes and a 16-bit scale word per row and
+    # block), the scales once more as the tensor cores' atoms
+    assert L.elq_arena_bytes(elq.NVFP4, 2048, 1792, ctypes.byref(q), ctypes.byref(d)) == 2048 * 56 * 20
+    assert q.value == 2048 * 56 * 16 and d.value == 2048 * 56 * 4
+    assert L.elq_arena_bytes(elq.NVFP4, 128, 96, None, None) == 0              # whole 64-value pairs only
     x = ctypes.c_void_p(1 << 27)
     out = ctypes.c_void_p(1 << 28)
     assert L.elq_quantize_nvfp4(x, 0, 4, 64, 0.0, out, None) == -1
