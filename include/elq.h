@@ -395,9 +395,11 @@ elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void
 
 /* The fp4 block-scaled tensor-core rate, for the NVFP4 experts' roofline: as
  * elq_test_mma_i8_rate with n_mma (>= 1) tcgen05.mma kind::mxf4nvf4 of M =
- * 128, N = 256, K = 64 (2 * 128 * 256 * 64 operations each) into one
- * accumulator, the scale factors copied to TMEM once. */
-elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
+ * 128, N = n_cols (16 .. 256, a multiple of 16), K = 64 (2 * 128 * n_cols * 64
+ * operations each) into one accumulator; the scale factors are copied to TMEM
+ * once, or before every MMA when cp_each is nonzero. */
+elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t n_cols, int32_t cp_each, int32_t* sink, int32_t* err,
+                                  void* stream);
 
 /* The packed fp32 rate, for the tensor-core epilogue's bound: 2 * SM count
  * CTAs of 1024 threads, each thread running n iterations of 8 independent

@@ -1632,15 +1632,17 @@ elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void
                               kWaitBudgetNs));
 }
 
-elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream) {
+elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t n_cols, int32_t cp_each, int32_t* sink, int32_t* err,
+                                  void* stream) {
     if (n_mma < 1 || !sink || !err) return ELQ_ERR_INVALID_ARG;
+    if (n_cols < 16 || n_cols > 256 || n_cols % 16) return ELQ_ERR_INVALID_ARG;
     static bool optin[kMaxDevices];
     // the int8 rate kernel's shared-memory request: one CTA (and one TMEM allocation) per SM
     cudaError_t e = smem_optin(k_test_mma_nvf4_rate, kRateSmem, optin);
     if (e != cudaSuccess) return ELQ_ERR_CUDA;
     return cuda_status(launch(k_test_mma_nvf4_rate, dim3(sm_count()), dim3(128), (size_t)kRateSmem,
-                              static_cast<cudaStream_t>(stream), false, (int)n_mma, (int*)sink, (int*)err,
-                              kWaitBudgetNs));
+                              static_cast<cudaStream_t>(stream), false, (int)n_mma, (int)n_cols, (int)(cp_each != 0),
+                              (int*)sink, (int*)err, kWaitBudgetNs));
 }
 
 elq_status elq_test_f32x2_rate(int32_t n, float* sink, void* stream) {

@@ -68,7 +68,7 @@ constexpr int kNvStageB = kNvKS * kTcN * 32;
 constexpr int kNvStageSfa = kNvKS * 512;
 constexpr int kNvStageSfb = kNvKS * 512;
 constexpr int kNvStage = kNvStageA + kNvStageB + kNvStageSfa + kNvStageSfb;
-constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kTcXchg;
+constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kTcXchg + kUnitsBytes;
 constexpr int kNvAccBufs = 2;                  // accumulators of kTcN columns
 constexpr int kNvSfCol = kNvAccBufs * kTcN;    // scale-factor columns: kNvKS x (SFA 4, SFB 4)
 constexpr int kNvTmemCols = 256;
@@ -112,7 +112,7 @@ __device__ __forceinline__ int nv_units(const NvArgs& g) { return __ldcg(g.tt_of
 // Unit u: row tile rt of the routed expert whose token tiles hold u / rtiles
 // (the same order as the int8 path: a weight tile against all its expert's
 // token tiles in turn).
-__device__ __forceinline__ TcUnit nv_unit(const NvArgs& g, int u) {
+__device__ __forceinline__ TcUnit tc_unit(const NvArgs& g, int u) {
     TcUnit r;
     const int q = u / g.rtiles;
     const int na = __ldcg(g.n_act);
@@ -234,6 +234,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
     int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
     uint8_t* stages = nvsm + 1024;
     float* xchg = reinterpret_cast<float*>(nvsm + 1024 + kNvStages * kNvStage);
+    TcUnit* su = reinterpret_cast<TcUnit*>(nvsm + 1024 + kNvStages * kNvStage + kTcXchg);
+    int* stt = reinterpret_cast<int*>(su + kUnitsSmem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -265,13 +267,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
     const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
     const int kstages = g.nks / kNvKS;
     volatile int* abort_v = abort_sm;
+    stage_units(g, u0, u1, su, stt);
+    auto unit_at = [&](int u) { return u - u0 < kUnitsSmem ? su[u - u0] : tc_unit(g, u); };
 
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
             int it = 0;
             for (int u = u0; u < u1 && !*abort_v; ++u) {
-                const TcUnit un = nv_unit(g, u);
+                const TcUnit un = unit_at(u);
                 if (!un.valid) continue;
                 const int tile = un.e * g.rtiles + un.rt;
                 const uint8_t* sfa = g.d + (int64_t)tile * g.d_tile_bytes + (int64_t)g.nb * 256;
@@ -299,7 +303,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
             int it = 0, uc = 0;
             const uint32_t sf = tmem + (uint32_t)kNvSfCol;
             for (int u = u0; u < u1 && !*abort_v; ++u, ++uc) {
-                const TcUnit un = nv_unit(g, u);
+                const TcUnit un = unit_at(u);
                 if (!un.valid) {
                     --uc;
                     continue;
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
         const int row = sp * 32 + lane;           // weight row within the tile
         int uc = 0, xc = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
-            const TcUnit un = nv_unit(g, u);
+            const TcUnit un = unit_at(u);
             if (!un.valid) continue;
             const int ab = uc % kNvAccBufs;
             if (!warp_wait_bounded(&tfull[ab], (uint32_t)((uc / kNvAccBufs) & 1), g.err, g.budget_ns)) {
@@ -433,12 +437,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
 // ---- measurement: the fp4 block-scaled tensor-core rate ------------------------
 //
 // One CTA per SM, one thread issuing n_mma tcgen05.mma kind::mxf4nvf4 (M = 128,
-// N = 256, K = 64, 2 * 128 * 256 * 64 operations each) from fixed shared-memory
-// operands and scale atoms (copied to TMEM once) into one accumulator, then a
-// bounded wait for them (ELQ_ERR_TIMEOUT's code 1 in *err if it runs out).
+// N = n_cols, K = 64, 2 * 128 * n_cols * 64 operations each) from fixed
+// shared-memory operands and scale atoms into one accumulator, then a bounded
+// wait for them (ELQ_ERR_TIMEOUT's code 1 in *err if it runs out).  The atoms
+// go to TMEM once, or (cp_each) before every MMA, as the GEMM's main loop
+// does.
 constexpr int kRateNvSmem = 1024 + (128 + kRateN) * 32 + 2 * 512;
 
-__global__ void __launch_bounds__(128, 1) k_test_mma_nvf4_rate(int n_mma, int* sink, int* err, uint64_t budget_ns) {
+__global__ void __launch_bounds__(128, 1) k_test_mma_nvf4_rate(int n_mma, int n_cols, int cp_each, int* sink, int* err,
+                                                               uint64_t budget_ns) {
     extern __shared__ __align__(1024) uint8_t rnsm_[];
     uint64_t* done = reinterpret_cast<uint64_t*>(rnsm_);
     uint32_t* tbase = reinterpret_cast<uint32_t*>(rnsm_ + 8);
@@ -466,9 +473,15 @@ __global__ void __launch_bounds__(128, 1) k_test_mma_nvf4_rate(int n_mma, int* s
         const uint32_t sfa = tmem + (uint32_t)kRateN, sfb = sfa + 4u;
         tmem_cp_atom(sfa, sf);
         tmem_cp_atom(sfb, sf + 512);
-        const uint32_t idesc = umma_idesc_nvf4(128, kRateN);
+        const uint32_t idesc = umma_idesc_nvf4(128, n_cols);
         const uint64_t ad = umma_desc(a, 2048, 128), bd = umma_desc(b, 128, 256);
-        for (int i = 0; i < n_mma; ++i) umma_nvf4(tmem, ad, bd, idesc, sfa, sfb, i > 0 ? 1u : 0u);
+        for (int i = 0; i < n_mma; ++i) {
+            if (cp_each) {
+                tmem_cp_atom(sfa, sf);
+                tmem_cp_atom(sfb, sf + 512);
+            }
+            umma_nvf4(tmem, ad, bd, idesc, sfa, sfb, i > 0 ? 1u : 0u);
+        }
         umma_commit(done);
     }
     __syncwarp();

@@ -330,7 +330,7 @@ constexpr int kTcStageDa = kTcKS * kTcN * 4;
 constexpr int kTcStage = kTcStageA + kTcStageB + kTcStageDw + kTcStageDa;
 constexpr int kTcXld = kTcTileRowsPad;
 constexpr int kTcXchg = kTcN * kTcXld * 4;                  // SwiGLU transpose: [token][row], padded rows
-constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg;
+constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg + 6144 + 4100;   // + the staged units
 static_assert(kTcEpiWarps * kTcEpiCols == 4 * kTcN, "the epilogue warps cover the 128 x 64 tile");
 
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
@@ -425,6 +425,57 @@ __device__ __forceinline__ TcUnit tc_unit(const TcArgs& g, int u) {
     return r;
 }
 
+// A CTA's units staged once in shared memory: every role then reads a unit
+// from there instead of repeating a binary search of dependent global loads
+// per unit (each one an L2 round trip).
+constexpr int kUnitsSmem = 256;
+constexpr int kUnitTableInts = 1025;        // tt_off[0 .. na], na <= 1024
+constexpr int kUnitsBytes = kUnitsSmem * (int)sizeof(TcUnit) + kUnitTableInts * 4;
+static_assert(kUnitsBytes == 6144 + 4100, "kTcSmem counts the staged units' bytes");
+
+// Expert unit u with the token-tile offsets in shared memory (stt = tt_off[0
+// .. na]): the search runs there; the expert, first slot and pair count take
+// two dependent global loads.
+template <class A>
+__device__ __forceinline__ TcUnit unit_staged(const A& g, int u, const int* stt, int na) {
+    TcUnit r;
+    const int q = u / g.rtiles;
+    int lo = 0, hi = na;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (stt[mid] <= q) lo = mid; else hi = mid;
+    }
+    r.e = __ldcg(g.act + lo);
+    const int base = stt[lo];
+    const int n_q = stt[lo + 1] - base;
+    const int v = u - base * g.rtiles;
+    r.rt = v / n_q;
+    const int tt = v - r.rt * n_q;
+    r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
+    const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
+    r.nvalid = min(kTcN, cnt - tt * kTcN);
+    r.ncols = (r.nvalid + 15) & ~15;
+    r.valid = r.nvalid > 0;
+    return r;
+}
+
+// The CTA's units [u0, u1) (the first kUnitsSmem) into su, all threads;
+// ends with a CTA barrier.  Dense launches (no routing) compute theirs
+// directly.
+template <class A>
+__device__ void stage_units(const A& g, int u0, int u1, TcUnit* su, int* stt) {
+    const int n = min(u1 - u0, kUnitsSmem);
+    const int na = g.act ? __ldcg(g.n_act) : 0;
+    if (g.act && na + 1 <= kUnitTableInts) {
+        for (int i = threadIdx.x; i <= na; i += blockDim.x) stt[i] = __ldcg(g.tt_off + i);
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = unit_staged(g, u0 + i, stt, na);
+    } else {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = tc_unit(g, u0 + i);
+    }
+    __syncthreads();
+}
+
 __device__ __forceinline__ int tc_units(const TcArgs& g) {
     if (!g.act) return ((g.T + kTcN - 1) / kTcN) * g.rtiles;
     return __ldcg(g.tt_off + __ldcg(g.n_act)) * g.rtiles;
@@ -450,6 +501,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
     int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
     uint8_t* stages = tcsm + 1024;
     float* xchg = reinterpret_cast<float*>(tcsm + 1024 + kTcStages * kTcStage);
+    TcUnit* su = reinterpret_cast<TcUnit*>(tcsm + 1024 + kTcStages * kTcStage + kTcXchg);
+    int* stt = reinterpret_cast<int*>(su + kUnitsSmem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -492,13 +545,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
     const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
     const int kstages = g.nb / kTcKS;
     volatile int* abort_v = abort_sm;
+    stage_units(g, u0, u1, su, stt);
+    auto unit_at = [&](int u) { return u - u0 < kUnitsSmem ? su[u - u0] : tc_unit(g, u); };
 
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
             int it = 0;
             for (int u = u0; u < u1 && !*abort_v; ++u) {
-                const TcUnit un = tc_unit(g, u);
+                const TcUnit un = unit_at(u);
                 if (!un.valid) continue;
                 const uint8_t* qa = g.q + un.e * g.q_gstride + (int64_t)un.rt * g.nb * 4096;
                 const uint16_t* da = g.d + un.e * g.d_gstride + (int64_t)un.rt * g.nb * kTileRows;
@@ -526,7 +581,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
         if (lane == 0) {
             int it = 0;
             for (int u = u0; u < u1 && !*abort_v; ++u) {
-                const TcUnit un = tc_unit(g, u);
+                const TcUnit un = unit_at(u);
                 if (!un.valid) continue;
                 const uint32_t idesc = umma_idesc_i8(128, un.ncols);
                 for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
@@ -565,7 +620,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
         const int row = sp * 32 + lane;       // weight row within the tile
         int it = 0, xc = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
-            const TcUnit un = tc_unit(g, u);
+            const TcUnit un = unit_at(u);
             if (!un.valid) continue;
             // accumulator pairs (columns 2j, 2j+1)
             uint64_t acc2[kTcEpiCols / 2], part2[kTcEpiCols / 2];

@@ -71,7 +71,7 @@ SIGNATURES = {
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
     "elq_test_expf": (I32, [V, V, I64, V]),
     "elq_test_mma_i8_rate": (I32, [I32, V, V, V]),
-    "elq_test_mma_nvf4_rate": (I32, [I32, V, V, V]),
+    "elq_test_mma_nvf4_rate": (I32, [I32, I32, I32, V, V, V]),
     "elq_sm_count": (I32, []),
     "elq_test_f32x2_rate": (I32, [I32, V, V]),
     "elq_test_fused_timeout": (I32, [ctypes.POINTER(LayerC), V, I32, I32, V, V, SZ, ctypes.c_uint64, V]),
@@ -473,13 +473,14 @@ def test_mma_i8_rate(n_mma: int, device="cuda", stream=None):
     return sink, err
 
 
-def test_mma_nvf4_rate(n_mma: int, device="cuda", stream=None):
+def test_mma_nvf4_rate(n_mma: int, n_cols: int = 256, cp_each: bool = False, device="cuda", stream=None):
     """Launches the fp4 block-scaled tensor-core rate kernel
     (elq_test_mma_nvf4_rate) on the current stream; returns (sink, err)."""
     n = int(_lib().elq_sm_count())
     sink = torch.zeros(n, dtype=torch.int32, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
-    _ck(_lib().elq_test_mma_nvf4_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_nvf4_rate")
+    _ck(_lib().elq_test_mma_nvf4_rate(n_mma, n_cols, int(cp_each), _ptr(sink), _ptr(err), _stream(stream)),
+        "elq_test_mma_nvf4_rate")
     return sink, err
 
 
