@@ -705,8 +705,8 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     w.ylat = c.take<float>(base, (size_t)T * L * 4);
     w.ylq = c.take<uint8_t>(base, (size_t)T * (L / 32) * 36);
     w.tstride = round16(T);
-    // NVFP4: token tiles start on 64 slots and scale atoms cover 128
-    w.sstride = w.nvtc ? (int64_t)round_up((size_t)(P + 64 * (int64_t)std::min<int64_t>(E, P)), 128)
+    // NVFP4: token tiles of 128 slots start on whole scale atoms
+    w.sstride = w.nvtc ? (int64_t)round_up((size_t)(P + kNvN * (int64_t)std::min<int64_t>(E, P)), 128)
                        : round16(P + 16 * (int64_t)std::min<int64_t>(E, P));
     w.grp = nullptr;
     w.gtok = nullptr;
@@ -1052,7 +1052,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     const int P = T * k;
     if (launch(k_tc_route, dim3(1), dim3(1024), 0, s, pdl, (const int32_t*)w.offsets, (const int32_t*)w.act,
                (const int32_t*)w.n_act, (const int32_t*)w.idx, (const int32_t*)w.pos, P, E, w.slot_off, w.tt_off,
-               w.pair_slot, 16) != cudaSuccess ||
+               w.pair_slot, 16, kTcN) != cudaSuccess ||
         !mark())
         return ELQ_ERR_CUDA;
     PackArgs pa;
@@ -1146,7 +1146,7 @@ NvArgs nv_args(const elq_qmat* m, int E, const LayerWs& w, int T, const uint8_t*
     const cuuint32_t ba[4] = {128, 4, 2 * kNvKS, 1};
     const cuuint64_t slots = (cuuint64_t)w.sstride;
     const cuuint64_t db[3] = {64, slots / 8, (cuuint64_t)g.nks}, sb[2] = {256, slots * 32};
-    const cuuint32_t bb[3] = {64, kTcN / 8, kNvKS};
+    const cuuint32_t bb[3] = {64, kNvN / 8, kNvKS};
     ok = encode_map(&g.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, m->q, da, sa, ba) &&
          encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, bq, db, sb, bb);
     return g;
@@ -1161,7 +1161,7 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     const int P = T * k;
     if (launch(k_tc_route, dim3(1), dim3(1024), 0, s, pdl, (const int32_t*)w.offsets, (const int32_t*)w.act,
                (const int32_t*)w.n_act, (const int32_t*)w.idx, (const int32_t*)w.pos, P, E, w.slot_off, w.tt_off,
-               w.pair_slot, kTcN) != cudaSuccess ||
+               w.pair_slot, kNvN, kNvN) != cudaSuccess ||
         !mark())
         return ELQ_ERR_CUDA;
     NvPackArgs pk;

@@ -9,8 +9,9 @@
 // chain of the GEMV path, so these results agree with the GEMV's to rounding,
 // not bit for bit.
 //
-// One MMA: M = 128 weight rows, N = up to 64 slots, K = 64 values (two
-// 32-value blocks).  Shared-memory operands, K-major without swizzle:
+// One MMA: M = 128 weight rows, N = up to 128 slots, K = 64 values (two
+// 32-value blocks).  An MMA of this shape costs the same issue time whatever
+// N, so token tiles are as wide as one scale atom (128 slots).  Shared-memory operands, K-major without swizzle:
 //  A (weights): [block][slice][32 rows x 16 bytes], one tensor-map copy per
 //    stage from the arena; for the MMA of blocks 2j, 2j+1: LBO = 2048 bytes
 //    (the next 16-byte K chunk), SBO = 128 bytes (the next 8 rows).
@@ -62,21 +63,28 @@ __device__ __forceinline__ void bulk_g2s_nv(void* dst, const void* src, uint32_t
 }
 
 constexpr int kNvKS = 4;                       // K steps (64 values each) per stage
-constexpr int kNvStages = 6;
+constexpr int kNvN = 128;                      // slots per token tile (one whole scale atom)
+constexpr int kNvStages = 4;
 constexpr int kNvStageA = kNvKS * 4096;
-constexpr int kNvStageB = kNvKS * kTcN * 32;
+constexpr int kNvStageB = kNvKS * kNvN * 32;
 constexpr int kNvStageSfa = kNvKS * 512;
 constexpr int kNvStageSfb = kNvKS * 512;
 constexpr int kNvStage = kNvStageA + kNvStageB + kNvStageSfa + kNvStageSfb;
-constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kTcXchg + kUnitsBytes;
-constexpr int kNvAccBufs = 2;                  // accumulators of kTcN columns
-constexpr int kNvSfCol = kNvAccBufs * kTcN;    // scale-factor columns: kNvKS x (SFA 4, SFB 4)
-constexpr int kNvTmemCols = 256;
+constexpr int kNvXld = 129;                    // SwiGLU exchange: [slot][128 rows], padded
+constexpr int kNvXchg = kNvN * kNvXld * 4;
+constexpr int kNvSmem = 1024 + kNvStages * kNvStage + kNvXchg + kUnitsBytes;
+constexpr int kNvAccBufs = 2;                  // accumulators of kNvN columns
+constexpr int kNvSfCol = kNvAccBufs * kNvN;    // scale-factor columns: kNvKS x (SFA 4, SFB 4)
+constexpr int kNvTmemCols = 512;
+constexpr int kNvEpiCols = 32;                 // accumulator columns per epilogue warp
 static_assert(kNvSfCol + kNvKS * 8 <= kNvTmemCols, "TMEM plan");
+static_assert(kTcEpiWarps / 4 * kNvEpiCols == kNvN, "the epilogue warps cover the 128 x 128 tile");
+static_assert(kNvSmem <= 227 * 1024, "shared memory plan");
 
 enum { NV_OUT_F32 = 0, NV_OUT_SWIGLU = 1 };
 
 struct NvArgs {
+    static constexpr int kN = kNvN;   // slots per token tile
     // tm_a: weight codes, uint32 [tiles][nb][4 slices][128] with strides
     //       (nb*2048, 512, nb*512) bytes; box [1][2 kNvKS][4][128] -> [block][slice][512 B]
     // tm_b: packed activation codes, uint32 [K steps][slots/8][64]; box [kNvKS][8][64]
@@ -127,9 +135,9 @@ __device__ __forceinline__ TcUnit tc_unit(const NvArgs& g, int u) {
     const int v = u - base * g.rtiles;
     r.rt = v / n_q;
     const int tt = v - r.rt * n_q;
-    r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
+    r.slot0 = __ldcg(g.slot_off + r.e) + tt * kNvN;
     const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
-    r.nvalid = min(kTcN, cnt - tt * kTcN);
+    r.nvalid = min(kNvN, cnt - tt * kNvN);
     r.ncols = (r.nvalid + 15) & ~15;
     r.valid = r.nvalid > 0;
     return r;
@@ -190,33 +198,29 @@ __global__ void __launch_bounds__(256) k_pack_nv(NvPackArgs a) {
     pdl_trigger();
 }
 
-// The h blocks of one (slot, 32-value block) from four lanes of eight values
-// each (lanes 2q, 2q+1 share micro-block q): NVFP4 under global scale gs,
-// written as the down projection's B codes and scale-atom bytes.
-__device__ __forceinline__ void nv_quant_h8(const float (&h)[8], bool on, float gs, int qd, int64_t slot, int kbh,
-                                            const NvArgs& g) {
+// One micro-block of h (16 values held by one thread): NVFP4 under global
+// scale gs (the rule of warp_quant_nvfp4), its 8 code bytes written into the
+// down projection's B codes (half of the slot's 16-byte chunk of block kbh)
+// and its scale byte into the slot's atom.
+__device__ __forceinline__ void nv_quant_h16(const float (&h)[16], float gs, int64_t slot, int kbh, int mb,
+                                             uint8_t* hq, uint8_t* hsf, int64_t sstride, int h_nks) {
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(h[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-    const uint32_t s = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs));
-    const float den = __fmul_rn(e4m3x2_to_f32(s).x, gs);
-    uint32_t w = 0;
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(h[i]));
+    const uint32_t sb = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs));
+    const float den = __fmul_rn(e4m3x2_to_f32(sb).x, gs);
+    uint32_t w[2] = {0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
+    for (int i = 0; i < 16; i += 2) {
         const float x0 = den != 0.0f ? __fdiv_rn(h[i], den) : 0.0f;
         const float x1 = den != 0.0f ? __fdiv_rn(h[i + 1], den) : 0.0f;
-        w |= f32x2_to_e2m1x2(x0, x1) << (4 * i);
+        w[i >> 3] |= f32x2_to_e2m1x2(x0, x1) << (4 * (i & 7));
     }
-    if (on) {
-        const int ks = kbh >> 1;
-        uint8_t* dst = g.hq + (int64_t)ks * g.sstride * 32 + (slot >> 3) * 256 + (kbh & 1) * 128 + (slot & 7) * 16 +
-                       qd * 4;
-        *reinterpret_cast<uint32_t*>(dst) = w;
-        if ((qd & 1) == 0)
-            g.hsf[((slot >> 7) * g.h_nks + ks) * 512 + (slot & 31) * 16 + ((slot >> 5) & 3) * 4 + (kbh & 1) * 2 +
-                  (qd >> 1)] = (uint8_t)s;
-    }
+    const int ks = kbh >> 1;
+    uint8_t* dst = hq + (int64_t)ks * sstride * 32 + (slot >> 3) * 256 + (kbh & 1) * 128 + (slot & 7) * 16 + mb * 8;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    hsf[((slot >> 7) * h_nks + ks) * 512 + (slot & 31) * 16 + ((slot >> 5) & 3) * 4 + (kbh & 1) * 2 + mb] =
+        (uint8_t)sb;
 }
 
 // ---- the GEMM ------------------------------------------------------------------
@@ -228,13 +232,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
     uint64_t* empty = full + kNvStages;                             // [stages]: MMAs done with them
     uint64_t* tfull = empty + kNvStages;                            // [2]: a unit's accumulator complete
     uint64_t* tempty = tfull + kNvAccBufs;                          // [2]: ... and drained
-    uint64_t* xfull = tempty + kNvAccBufs;
-    uint64_t* xempty = xfull + 1;
+    uint64_t* xfull = tempty + kNvAccBufs;                          // SwiGLU: up rows handed over
+    uint64_t* xempty = xfull + 1;                                   // ... and taken
     uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(xempty + 1);
     int* abort_sm = reinterpret_cast<int*>(tmem_base_sm + 1);
     uint8_t* stages = nvsm + 1024;
-    float* xchg = reinterpret_cast<float*>(nvsm + 1024 + kNvStages * kNvStage);
-    TcUnit* su = reinterpret_cast<TcUnit*>(nvsm + 1024 + kNvStages * kNvStage + kTcXchg);
+    float* xchg = reinterpret_cast<float*>(nvsm + 1024 + kNvStages * kNvStage);   // [slot][128 rows]
+    TcUnit* su = reinterpret_cast<TcUnit*>(nvsm + 1024 + kNvStages * kNvStage + kNvXchg);
     int* stt = reinterpret_cast<int*>(su + kUnitsSmem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -302,22 +306,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
         if (lane == 0) {
             int it = 0, uc = 0;
             const uint32_t sf = tmem + (uint32_t)kNvSfCol;
-            for (int u = u0; u < u1 && !*abort_v; ++u, ++uc) {
+            for (int u = u0; u < u1 && !*abort_v; ++u) {
                 const TcUnit un = unit_at(u);
-                if (!un.valid) {
-                    --uc;
-                    continue;
-                }
+                if (!un.valid) continue;
                 const int ab = uc % kNvAccBufs;
                 if (uc >= kNvAccBufs &&
                     !mbar_wait_bounded(&tempty[ab], (uint32_t)((uc / kNvAccBufs - 1) & 1), g.err, g.budget_ns)) {
                     *abort_v = 1;
                     break;
                 }
+                ++uc;
                 tc_fence_after();
                 const uint32_t idesc = umma_idesc_nvf4(128, un.ncols);
-                const uint32_t dacc = tmem + (uint32_t)(ab * kTcN);
-                const uint32_t bsub = (uint32_t)((un.slot0 & 127) >> 5);   // the tile's words of the slot atoms
+                const uint32_t dacc = tmem + (uint32_t)(ab * kNvN);
                 for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
                     const int s = it % kNvStages;
                     if (!mbar_wait_bounded(&full[s], (uint32_t)((it / kNvStages) & 1), g.err, g.budget_ns)) {
@@ -331,8 +332,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
                         tmem_cp_atom(sfa_t, st + kNvStageA + kNvStageB + k * 512);
                         tmem_cp_atom(sfb_t, st + kNvStageA + kNvStageB + kNvStageSfa + k * 512);
                         const uint64_t adesc = umma_desc(st + k * 4096, 2048, 128);
-                        const uint64_t bdesc = umma_desc(st + kNvStageA + k * kTcN * 32, 128, 256);
-                        umma_nvf4(dacc, adesc, bdesc, idesc, sfa_t, sfb_t + bsub, (ks | k) != 0 ? 1u : 0u);
+                        const uint64_t bdesc = umma_desc(st + kNvStageA + k * kNvN * 32, 128, 256);
+                        umma_nvf4(dacc, adesc, bdesc, idesc, sfa_t, sfb_t, (ks | k) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -347,10 +348,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
         }
     } else {
         // ---------------- epilogue ----------------
+        // warp: TMEM lane quarter sp (tile rows 32 sp ..), columns (slots) c0 .. c0 + 31
         const int ew = warp - 2;
-        const int sp = warp & 3;                  // TMEM lane quarter
-        const int c0 = (ew >> 2) * kTcEpiCols;    // accumulator columns (slots) c0 .. c0+15
-        const int row = sp * 32 + lane;           // weight row within the tile
+        const int sp = warp & 3;
+        const int c0 = (ew >> 2) * kNvEpiCols;
+        const int row = sp * 32 + lane;
         int uc = 0, xc = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
             const TcUnit un = unit_at(u);
@@ -362,36 +364,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
             }
             ++uc;
             tc_fence_after();
-            float acc[kTcEpiCols];
+            float acc[kNvEpiCols];
             const bool active = c0 < un.ncols;
             if (active) {
-                uint32_t rc[kTcEpiCols];
-                tmem_ld16(tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(ab * kTcN + c0), rc);
+                uint32_t rc[kNvEpiCols];
+                tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + (uint32_t)(ab * kNvN + c0), rc);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < kTcEpiCols; ++j) acc[j] = __uint_as_float(rc[j]);
+                for (int j = 0; j < kNvEpiCols; ++j) acc[j] = __uint_as_float(rc[j]);
             } else {
 #pragma unroll
-                for (int j = 0; j < kTcEpiCols; ++j) acc[j] = 0.0f;
+                for (int j = 0; j < kNvEpiCols; ++j) acc[j] = 0.0f;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[ab]);
             const float gq = __fmul_rn(__ldg(g.wgs + un.e), g.ags);
 #pragma unroll
-            for (int j = 0; j < kTcEpiCols; ++j) acc[j] = __fmul_rn(acc[j], gq);
+            for (int j = 0; j < kNvEpiCols; ++j) acc[j] = __fmul_rn(acc[j], gq);
             const int nv = un.nvalid;
             const int64_t slot0 = un.slot0;
             if (OM == NV_OUT_SWIGLU) {
-                // transpose the tile through shared memory ([slot][row], padded), then four
-                // threads per (slot, h block): h row 32 hb + i takes gate row 32 hb + i and up
-                // row 64 + 32 hb + i of the tile
+                // the tile through shared memory ([slot][row], padded), then two threads per
+                // (slot, h block), one micro-block of 16 values each: h row 32 hb + i takes gate
+                // row 32 hb + i and up row 64 + 32 hb + i of the tile
                 if (xc > 0 && !warp_wait_bounded(xempty, (uint32_t)((xc - 1) & 1), g.err, g.budget_ns)) {
                     *abort_v = 1;
                     break;
                 }
 #pragma unroll
-                for (int j = 0; j < kTcEpiCols; ++j) xchg[(c0 + j) * kTcXld + row] = acc[j];
+                for (int j = 0; j < kNvEpiCols; ++j) xchg[(c0 + j) * kNvXld + row] = acc[j];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(xfull);
                 if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
@@ -400,20 +402,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
                 }
                 {
                     const int task = ew * 32 + lane;          // 0 .. 511
-                    const int b = task >> 2, qd = task & 3;
+                    const int mb = task & 1, b = task >> 1;
                     const int t = b >> 1, hb = b & 1;
-                    const bool on = t < nv;
-                    float h[8];
-                    if (on) {
-                        const float* gr = xchg + t * kTcXld + hb * 32 + qd * 8;
+                    if (t < nv) {
+                        const float* gr = xchg + t * kNvXld + hb * 32 + mb * 16;
                         const float* ur = gr + 64;
+                        float h[16];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) h[i] = 0.0f;
+                        for (int i = 0; i < 16; ++i) h[i] = __fmul_rn(silu_f32(gr[i]), ur[i]);
+                        nv_quant_h16(h, g.ogs, slot0 + t, un.rt * 2 + hb, mb, g.hq, g.hsf, g.sstride, g.h_nks);
                     }
-                    nv_quant_h8(h, on, g.ogs, qd, slot0 + t, un.rt * 2 + hb, g);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(xempty);
@@ -421,7 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
                 continue;
             }
 #pragma unroll
-            for (int j = 0; j < kTcEpiCols; ++j) {
+            for (int j = 0; j < kNvEpiCols; ++j) {
                 const int t = c0 + j;
                 if (t < nv) g.y[(slot0 + t) * g.y_ld + (int64_t)un.rt * kTileRows + row] = acc[j];
             }

@@ -252,14 +252,15 @@ __global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
 constexpr int kTcN = 64;            // tokens per tile
 
 // ---- routing -> padded slots -------------------------------------------------
-// slot_off[e] = sum over e' < e of roundup(count(e'), align) (align 16, or 64
-// for the NVFP4 path, whose token tiles must start on 64 slots); tt_off[a] = sum over
-// active experts a' < a of ceil(count / 64); pair_slot[p] = the slot of pair p.
+// slot_off[e] = sum over e' < e of roundup(count(e'), align) (align 16, or 128
+// for the NVFP4 path, whose token tiles start on whole scale atoms); tt_off[a]
+// = sum over active experts a' < a of ceil(count / tile) (64, or 128 for
+// NVFP4); pair_slot[p] = the slot of pair p.
 // One CTA.
 __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const int32_t* act, const int32_t* n_act,
                                                    const int32_t* idx, const int32_t* pos, int P, int E,
                                                    int32_t* slot_off, int32_t* tt_off, int32_t* pair_slot,
-                                                   int align) {
+                                                   int align, int tile) {
     pdl_wait();
     __shared__ int s_slot[1025];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
         int local = 0;
         for (int a = a0; a < a1; ++a) {
             const int e = __ldcg(act + a);
-            local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + kTcN - 1) / kTcN;
+            local += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + tile - 1) / tile;
         }
         int incl = local;
         for (int o = 1; o < 32; o <<= 1) {
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
         for (int a = a0; a < a1; ++a) {
             tt_off[a] = run;
             const int e = __ldcg(act + a);
-            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + kTcN - 1) / kTcN;
+            run += (__ldcg(offsets + e + 1) - __ldcg(offsets + e) + tile - 1) / tile;
         }
         if (lane == 31) tt_off[na] = incl;
     }
@@ -336,6 +337,7 @@ static_assert(kTcEpiWarps * kTcEpiCols == 4 * kTcN, "the epilogue warps cover th
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
 
 struct TcArgs {
+    static constexpr int kN = kTcN;   // slots per token tile
     // tensor maps of one stage's four copies (host-encoded):
     //  tm_a : weight codes, uint32 [tiles][nb][4 slices][256] with strides
     //         (nb*4096, 1024, nb*1024) bytes; box [1][4][4][256] lands as
@@ -451,9 +453,9 @@ __device__ __forceinline__ TcUnit unit_staged(const A& g, int u, const int* stt,
     const int v = u - base * g.rtiles;
     r.rt = v / n_q;
     const int tt = v - r.rt * n_q;
-    r.slot0 = __ldcg(g.slot_off + r.e) + tt * kTcN;
+    r.slot0 = __ldcg(g.slot_off + r.e) + tt * A::kN;
     const int cnt = __ldcg(g.offsets + r.e + 1) - __ldcg(g.offsets + r.e);
-    r.nvalid = min(kTcN, cnt - tt * kTcN);
+    r.nvalid = min(A::kN, cnt - tt * A::kN);
     r.ncols = (r.nvalid + 15) & ~15;
     r.valid = r.nvalid > 0;
     return r;

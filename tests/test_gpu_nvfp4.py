@@ -158,10 +158,10 @@ def _check_tc(E, ly, T, tr):
     return v("y_lat").reshape(T, -1)
 
 
-@pytest.mark.parametrize("T", [9, 16, 63, 64, 65, 300])
+@pytest.mark.parametrize("T", [9, 16, 64, 127, 128, 129, 300])
 def test_nvfp4_tc_layer(E, orc, T):
     """The block-scaled tensor-core experts (eleven kernels), from just above
-    the GEMV's sizes through several 64-slot tiles per expert and ragged last
+    the GEMV's sizes through several 128-slot tiles per expert and ragged last
     tiles."""
     wl = NV_TINY
     ly = gpu_layer(wl)
