@@ -456,7 +456,7 @@ ProjWs proj_layout(const elq_qmat* w, int T, void* base, bool allow_tc = true) {
 bool g_optin_tc[kMaxDevices];
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s, bool pdl) {
-    const int64_t n = a.bstride * a.nb;
+    const int64_t n = (a.mode == PACK_DENSE ? a.bstride : (int64_t)a.P) * a.nb;
     return launch(k_pack_b, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, a);
 }
 
@@ -1060,11 +1060,9 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     pa.x = zq;
     pa.nb = L / 32;
     pa.mode = PACK_PAIRS;
-    pa.offsets = w.offsets;
-    pa.slot_off = w.slot_off;
-    pa.perm = w.perm;
+    pa.pair_slot = w.pair_slot;
+    pa.P = P;
     pa.kslots = k;
-    pa.E = E;
     pa.bq = w.bzq;
     pa.bd = w.bzd;
     pa.bstride = w.sstride;
@@ -1105,8 +1103,8 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
-    const int64_t warps = (int64_t)T * (L / 32);
-    if (launch(k_tc_combine, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+    const int64_t warps = (int64_t)T * (L / 32);   // one thread per (token, block)
+    if (launch(k_tc_combine, dim3((unsigned)((warps + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
         return ELQ_ERR_CUDA;
     return ELQ_OK;
 }
@@ -1169,15 +1167,13 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     pk.x = zq;
     pk.nb = L / 32;
     pk.nks = L / 64;
-    pk.offsets = w.offsets;
-    pk.slot_off = w.slot_off;
-    pk.perm = w.perm;
+    pk.pair_slot = w.pair_slot;
+    pk.P = P;
     pk.kslots = k;
-    pk.E = E;
     pk.bq = w.bzq;
     pk.bsf = reinterpret_cast<uint8_t*>(w.bzd);
     pk.sstride = w.sstride;
-    const int64_t n = w.sstride * pk.nks;
+    const int64_t n = (int64_t)P * pk.nks;
     if (launch(k_pack_nv, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, pk) != cudaSuccess || !mark())
         return ELQ_ERR_CUDA;
     bool ok = false;
@@ -1197,8 +1193,8 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
-    const int64_t warps = (int64_t)T * (L / 32);
-    if (launch(k_tc_combine, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+    const int64_t warps = (int64_t)T * (L / 32);   // one thread per (token, block)
+    if (launch(k_tc_combine, dim3((unsigned)((warps + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
         return ELQ_ERR_CUDA;
     return ELQ_OK;
 }
@@ -1318,7 +1314,7 @@ elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_
     if (!x || !out_q8_1) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x, 4) || !aligned(out_q8_1, 4)) return ELQ_ERR_ALIGNMENT;
     const int64_t nblk = rows * (cols / 32);
-    const dim3 grid((unsigned)((nblk * 32 + 255) / 256));
+    const dim3 grid((unsigned)((nblk + 255) / 256));   // one thread per block
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (x_type == ELQ_BF16)
         return cuda_status(launch(k_quant_q8_1<true>, grid, dim3(256), 0, s, false, x, nblk,
@@ -1767,10 +1763,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         // tensor cores (z), z's NVFP4 rows, router, the block-scaled experts, U
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         PackArgs pa;
@@ -1804,10 +1800,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         // then the tensor-core experts and U
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         PackArgs pa;
@@ -1872,10 +1868,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     } else {
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk * 32 + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         gd = dense_w(&layer->D, T, w.xq, X_Q81_TOKEN, 0, OUT_F32_Q81, w.z, w.zq, w.partial, w.cnt_d, w.err);

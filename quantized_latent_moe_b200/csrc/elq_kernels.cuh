@@ -16,21 +16,61 @@ namespace elq {
 constexpr unsigned kFull = 0xffffffffu;
 
 // ============================================================================
-// a1 / a4 -- Q8_1 activation quantiser: one warp per 32-value block.
+// a1 / a4 -- Q8_1 activation quantiser: one thread per 32-value block (the
+// block's 32 values in registers: amax, d = amax / 127, q = clamp(round(x /
+// d)), s = fp16(d * sum q); the same operations as the warp quantiser).
 // ============================================================================
 template <bool kBF16>
 __global__ void __launch_bounds__(256) k_quant_q8_1(const void* __restrict__ x, int64_t nblocks,
                                                     uint8_t* __restrict__ out) {
     pdl_wait();
-    const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (blk >= nblocks) return;
-    float v;
-    if (kBF16)
-        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[blk * 32 + lane]);
-    else
-        v = reinterpret_cast<const float*>(x)[blk * 32 + lane];
-    warp_quant_q8_1(v, out + blk * 36);
+    const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (blk < nblocks) {
+        float v[32];
+        if ((reinterpret_cast<uintptr_t>(x) & 15) != 0) {
+            // 4-byte aligned input: element loads
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = kBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[blk * 32 + i])
+                             : static_cast<const float*>(x)[blk * 32 + i];
+        } else if (kBF16) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + blk * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 w = __ldg(src + i);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
+                    v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+                }
+            }
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + blk * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 w = __ldg(src + i);
+                v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+            }
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const float d = __fdiv_rn(amax, 127.0f);
+        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            int q = 0;
+            if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f);
+            sum += q;
+            w[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+        }
+        uint32_t* o = reinterpret_cast<uint32_t*>(out + blk * 36);
+        o[0] = (uint32_t)f2h(d) | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[1 + i] = w[i];
+    }
     pdl_trigger();
 }
 

@@ -144,17 +144,15 @@ __device__ __forceinline__ TcUnit tc_unit(const NvArgs& g, int u) {
 }
 
 // ---- packing: NVFP4 rows (18-byte blocks) -> B codes and scale atoms ---------
-// Slot s of expert e (s - slot_off[e] < count(e)) holds the row of its pair
-// perm[offsets[e] + s - slot_off[e]] / k; other slots hold zeros.  One thread
-// per (slot, K step): the two blocks' 32 code bytes to [K step][slot/8][2][8][16],
-// their four scales as one word of the slot's atom.
+// Pair p (row p / k) goes to slot pair_slot[p]: per K step its two blocks' 32
+// code bytes to [K step][slot/8][2][8][16], their four scales as one word of
+// the slot's atom.  One thread per (pair, K step); padding slots are left as
+// they are (the GEMM's columns past a tile's pairs are unused).
 struct NvPackArgs {
     const uint8_t* x;           // NVFP4 rows, nb blocks each
     int nb, nks;
-    const int32_t* offsets;
-    const int32_t* slot_off;
-    const int32_t* perm;
-    int kslots, E;
+    const int32_t* pair_slot;
+    int P, kslots;
     uint8_t* bq;
     uint8_t* bsf;
     int64_t sstride;
@@ -163,22 +161,13 @@ struct NvPackArgs {
 __global__ void __launch_bounds__(256) k_pack_nv(NvPackArgs a) {
     pdl_wait();
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (id >= a.sstride * a.nks) return;
-    const int64_t slot = id / a.nks;
+    if (id >= (int64_t)a.P * a.nks) return;
+    const int64_t p = id / a.nks;
     const int ks = (int)(id % a.nks);
-    int lo = 0, hi = a.E;       // slot_off[lo] <= slot < slot_off[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldcg(a.slot_off + mid) <= slot) lo = mid; else hi = mid;
-    }
-    int64_t row = -1;
-    if (slot < __ldcg(a.slot_off + a.E)) {
-        const int i = (int)(slot - __ldcg(a.slot_off + lo));
-        const int n = __ldcg(a.offsets + lo + 1) - __ldcg(a.offsets + lo);
-        if (i < n) row = __ldcg(a.perm + __ldcg(a.offsets + lo) + i) / a.kslots;
-    }
+    const int64_t slot = __ldcg(a.pair_slot + p);
+    const int64_t row = p / a.kslots;
     uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sw = 0;
-    if (row >= 0) {
+    {
         // two 18-byte blocks (2-byte aligned): scales, then 16 code bytes each
         const uint16_t* src = reinterpret_cast<const uint16_t*>(a.x + (row * a.nb + 2 * ks) * 18);
 #pragma unroll

@@ -202,36 +202,29 @@ struct PackArgs {
     int nb;
     int mode;
     int T;                      // PACK_DENSE: rows 0 .. T-1 -> slots 0 .. T-1
-    // PACK_PAIRS: expert e's pairs perm[off[e] + i] go to slot slot_off[e] + i; row = pair / k
-    const int32_t* offsets;
-    const int32_t* slot_off;
-    const int32_t* perm;
-    int kslots, E;
+    // PACK_PAIRS: pair p (row p / k) goes to slot pair_slot[p]; padding slots
+    // are left as they are (the GEMM's columns past a tile's pairs are unused)
+    const int32_t* pair_slot;
+    int P, kslots;
     uint8_t* bq;
     float* bd;
     int64_t bstride;            // slots in the buffer (multiple of 16)
 };
 
-// One thread per (slot, block).
+// One thread per (slot, block) (dense), or per (pair, block).
 __global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
     pdl_wait();
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (id >= a.bstride * a.nb) return;
-    const int64_t slot = id / a.nb;
+    const int64_t n_items = a.mode == PACK_DENSE ? a.bstride : a.P;
+    if (id >= n_items * a.nb) return;
+    const int64_t item = id / a.nb;
     const int kb = (int)(id % a.nb);
-    int64_t row = -1;
+    int64_t row = -1, slot = item;
     if (a.mode == PACK_DENSE) {
-        if (slot < a.T) row = slot;
+        if (item < a.T) row = item;
     } else {
-        // the expert whose padded slot range holds this slot
-        int lo = 0, hi = a.E;   // slot_off[lo] <= slot < slot_off[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (__ldcg(a.slot_off + mid) <= slot) lo = mid; else hi = mid;
-        }
-        const int i = (int)(slot - __ldcg(a.slot_off + lo));
-        const int n = __ldcg(a.offsets + lo + 1) - __ldcg(a.offsets + lo);
-        if (i < n) row = __ldcg(a.perm + __ldcg(a.offsets + lo) + i) / a.kslots;
+        slot = __ldcg(a.pair_slot + item);
+        row = item / a.kslots;
     }
     uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
     float dd = 0.0f;
@@ -842,10 +835,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 
 // ---- a9 on the tensor-core path: the weighted combine --------------------------
 //
-// One warp per (token, 32-row latent block), lane = row: y_lat = fmaf(w_j,
-// o_j, y_lat) over the token's k pairs in rank order (o read by the pair's
-// slot), then its Q8_1 block, written both row-major (ylq) and into the
-// packed buffer the U projection reads (slot = token).
+// One thread per (token, 32-row latent block), its 32 rows in registers:
+// y_lat = fmaf(w_j, o_j, y_lat) over the token's k pairs in rank order (o
+// read by the pair's slot, 128 contiguous bytes a pair), then its Q8_1 block,
+// written both row-major (ylq) and into the packed buffer the U projection
+// reads (slot = token).
 struct CombArgs {
     const float* o;             // [slots][L] by slot
     const float* wts;           // [T][k]
@@ -861,34 +855,52 @@ struct CombArgs {
 __global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
     pdl_wait();
     pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int nbl = a.L / 32;
-    if (wid >= (int64_t)a.T * nbl) return;
-    const int t = (int)(wid / nbl), blk = (int)(wid - (int64_t)t * nbl);
-    float acc = 0.0f;
-    for (int j0 = 0; j0 < a.k; j0 += 8) {
-        float ov[8], wv[8];
+    if (id >= (int64_t)a.T * nbl) return;
+    const int t = (int)(id / nbl), blk = (int)(id - (int64_t)t * nbl);
+    float acc[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (j0 + q < a.k) {
-                const int pj = t * a.k + j0 + q;
-                wv[q] = __ldg(a.wts + pj);
-                ov[q] = __ldcg(a.o + (int64_t)__ldg(a.pair_slot + pj) * a.L + blk * 32 + lane);
-            }
+    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < a.k; ++j) {
+        const int pj = t * a.k + j;
+        const float wj = __ldg(a.wts + pj);
+        const float4* src = reinterpret_cast<const float4*>(a.o + (int64_t)__ldg(a.pair_slot + pj) * a.L + blk * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (j0 + q < a.k) acc = __fmaf_rn(wv[q], ov[q], acc);
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldcg(src + i);
+            acc[4 * i] = __fmaf_rn(wj, v.x, acc[4 * i]);
+            acc[4 * i + 1] = __fmaf_rn(wj, v.y, acc[4 * i + 1]);
+            acc[4 * i + 2] = __fmaf_rn(wj, v.z, acc[4 * i + 2]);
+            acc[4 * i + 3] = __fmaf_rn(wj, v.w, acc[4 * i + 3]);
+        }
     }
-    a.ylat[(int64_t)t * a.L + blk * 32 + lane] = acc;
-    uint8_t* qb = a.ylq + ((int64_t)t * nbl + blk) * 36;
-    warp_quant_q8_1(acc, qb);
-    __syncwarp();
-    // the same block, packed for the U projection
+    float4* yl = reinterpret_cast<float4*>(a.ylat + (int64_t)t * a.L + blk * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) yl[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+    // its Q8_1 block (the quantiser's rule), row-major and packed for the U projection
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+    const float d = __fdiv_rn(amax, 127.0f);
+    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        int q = 0;
+        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(acc[i], d)), -127.0f), 127.0f);
+        sum += q;
+        w[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+    }
+    const uint16_t dh = f2h(d);
+    uint32_t* qb = reinterpret_cast<uint32_t*>(a.ylq + ((int64_t)t * nbl + blk) * 36);
+    qb[0] = (uint32_t)dh | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qb[1 + i] = w[i];
     uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 32 + ((int64_t)t >> 3) * 256 + (t & 7) * 16;
-    if (lane < 8)
-        reinterpret_cast<uint32_t*>(dst + (lane >> 2) * 128)[lane & 3] = reinterpret_cast<const uint32_t*>(qb + 4)[lane];
-    if (lane == 0) a.cd[(int64_t)blk * a.cstride + t] = h2f(*reinterpret_cast<const uint16_t*>(qb));
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(dst + 128) = make_uint4(w[4], w[5], w[6], w[7]);
+    a.cd[(int64_t)blk * a.cstride + t] = h2f(dh);
 }
 
 // ---- measurement: the int8 tensor-core rate ------------------------------------
