@@ -3,7 +3,7 @@
 Only the tests, the package's ``smoke()`` check and the benchmark's CPU
 baseline leg may use this package.  The CUDA library never imports, links or
 calls it, and it imports nothing from the CUDA library.  What it computes is
-stated in ``elq_oracle.h`` (readings R1-R21) and written out in
+stated in ``elq_oracle.h`` (readings R1-R24) and written out in
 ``elq_oracle.c`` as plain loops; this module only builds the C file with gcc
 and marshals numpy arrays into it.
 """
@@ -20,8 +20,9 @@ SRC = os.path.join(HERE, "elq_oracle.c")
 HDR = os.path.join(HERE, "elq_oracle.h")
 LIB = os.path.join(HERE, "libelq_oracle.so")
 
-Q4_0, Q8_0, Q8_1, NVFP4 = 2, 8, 9, 100
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q8_1: 36, NVFP4: 18}
+Q4_0, Q5_1, Q8_0, Q8_1, Q4_K, Q5_K, NVFP4 = 2, 7, 8, 9, 12, 13, 100
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q8_1: 36, NVFP4: 18, Q5_1: 24}
+EXT = (Q5_1, Q4_K, Q5_K)           # expert formats given as GGUF blocks (R22-R24)
 
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC",
           "-shared", "-Wall", "-Wextra"]
@@ -91,6 +92,10 @@ def _declare(L):
                                          P, ctypes.POINTER(OrcTrace)]),
         "orc_route": (ctypes.c_int, [ctypes.POINTER(OrcLayer), P, ctypes.c_int, P, P]),
         "orc_arena_pack": (None, [ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, P]),
+        "orc_row_bytes": (I64, [ctypes.c_int, I64]),
+        "orc_dequantize_ext": (None, [ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P]),
+        "orc_block_ext": (None, [ctypes.c_int, P, ctypes.c_int, P, P, P, P, P]),
+        "orc_qmatmul_ext": (None, [ctypes.c_int, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P]),
         "orc_f32_to_e2m1": (ctypes.c_uint8, [F32]),
         "orc_e2m1_to_f32": (F32, [ctypes.c_uint8]),
         "orc_f32_to_e4m3": (ctypes.c_uint8, [F32]),
@@ -253,6 +258,39 @@ def qmatmul_nvfp4(W: np.ndarray, gw: float, N: int, K: int, Xq: np.ndarray, T: i
     return Y
 
 
+def row_bytes(fmt: int, k: int) -> int:
+    return int(lib().orc_row_bytes(fmt, k))
+
+
+def dequantize_ext(fmt: int, W: np.ndarray, N: int, K: int) -> np.ndarray:
+    """fp64 values of N rows of Q5_1 / Q4_K / Q5_K blocks (R22)."""
+    W = np.ascontiguousarray(W, np.uint8)
+    assert W.size == N * row_bytes(fmt, K)
+    out = np.empty((N, K), np.float64)
+    lib().orc_dequantize_ext(fmt, _p(W), N, K, _p(out))
+    return out
+
+
+def block_ext(fmt: int, row: np.ndarray, kb: int, ablk: np.ndarray):
+    """(isum, sumq, sd, sm) of 32-value block kb of a row against a Q8_1 block (R23, R24)."""
+    row = np.ascontiguousarray(row, np.uint8)
+    ablk = np.ascontiguousarray(ablk, np.uint8)
+    isum, sumq = ctypes.c_int32(), ctypes.c_int32()
+    sd, sm = ctypes.c_float(), ctypes.c_float()
+    lib().orc_block_ext(fmt, _p(row), kb, _p(ablk), ctypes.byref(isum), ctypes.byref(sumq), ctypes.byref(sd),
+                        ctypes.byref(sm))
+    return isum.value, sumq.value, sd.value, sm.value
+
+
+def qmatmul_ext(fmt: int, W: np.ndarray, N: int, K: int, Xq: np.ndarray, T: int) -> np.ndarray:
+    W = np.ascontiguousarray(W, np.uint8)
+    Xq = np.ascontiguousarray(Xq, np.uint8)
+    assert W.size == N * row_bytes(fmt, K) and Xq.size == T * (K // 32) * 36
+    Y = np.empty((T, N), np.float32)
+    lib().orc_qmatmul_ext(fmt, _p(W), N, K, _p(Xq), T, _p(Y))
+    return Y
+
+
 def arena_pack(fmt: int, aos: np.ndarray, n_rows: int, k: int):
     aos = np.ascontiguousarray(aos, np.uint8)
     nb = k // 32
@@ -292,6 +330,12 @@ class Layer:
         for e in experts:
             g = w["gate"][e] if w.get("gate") is not None else None
             if g is None:
+                continue
+            if self.ex_fmt in EXT:
+                # given as GGUF blocks (uint8 rows)
+                self.gate[e] = np.ascontiguousarray(g, np.uint8)
+                self.up[e] = np.ascontiguousarray(w["up"][e], np.uint8)
+                self.down[e] = np.ascontiguousarray(w["down"][e], np.uint8)
                 continue
             if self.ex_fmt == NVFP4:
                 gu = np.concatenate([_f32(g).ravel(), _f32(w["up"][e]).ravel()])

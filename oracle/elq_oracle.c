@@ -23,13 +23,22 @@ int orc_block_bytes(int fmt)
     case ORC_Q8_0: return 34;
     case ORC_Q8_1: return 36;
     case ORC_NVFP4: return 18;
+    case ORC_Q5_1: return 24;
     default: return 0;
     }
 }
 
+/* bytes of a row of k values (K-quants: super-blocks of 256) */
+int64_t orc_row_bytes(int fmt, int64_t k)
+{
+    if (fmt == ORC_Q4_K) return (k / 256) * 144;
+    if (fmt == ORC_Q5_K) return (k / 256) * 176;
+    return (k / 32) * (int64_t)orc_block_bytes(fmt);
+}
+
 int64_t orc_matrix_bytes(int fmt, int64_t rows, int64_t k)
 {
-    return rows * (k / 32) * (int64_t)orc_block_bytes(fmt);
+    return rows * orc_row_bytes(fmt, k);
 }
 
 /* fp32 -> fp16, round to nearest, ties to even (the loader's narrowing rule in
@@ -256,6 +265,137 @@ void orc_dequantize(int fmt, const uint8_t* blocks, int64_t n, double* out)
                 ob[j] = d * (double)((p[2 + j] & 0x0F) - 8);
                 ob[j + 16] = d * (double)((p[2 + j] >> 4) - 8);
             }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Q5_1 and the K-quants Q4_K, Q5_K ("Q8 0 support - Pull Request #255",    */
+/* follow-up commit "per-role format lists": the Q4_K / Q5_K / Q5_1 expert  */
+/* dots, Q5_1's min term on the sum of the quantised activations).  The     */
+/* block layouts are the GGUF formats the pages name (R22-R24 in            */
+/* elq_oracle.h).                                                            */
+
+/* Q5_1, 24-byte blocks of 32: fp16 d, fp16 m, uint32 qh, 16 code bytes.
+ * Value i: code q = (low nibble of byte i for i < 16, high nibble of byte
+ * i - 16 otherwise) + 16 * bit i of qh; x = d * q + m. */
+static int q51_code(const uint8_t* b, int i)
+{
+    uint32_t qh = (uint32_t)b[4] | ((uint32_t)b[5] << 8) | ((uint32_t)b[6] << 16) | ((uint32_t)b[7] << 24);
+    int lo = i < 16 ? (b[8 + i] & 0x0F) : (b[8 + i - 16] >> 4);
+    return lo | (int)(((qh >> i) & 1u) << 4);
+}
+
+/* K-quant super-block (256 values, 8 sub-blocks of 32): fp16 d, fp16 dmin,
+ * 12 bytes of 6-bit sub-block scales and mins, [Q5_K: 32 bytes qh], 128
+ * code bytes.  Sub-block j < 4: scale = byte j & 63, min = byte j+4 & 63;
+ * j >= 4: scale = (byte j+4 & 15) | (byte j-4 >> 6) << 4, min = (byte j+4 >>
+ * 4) | (byte j >> 6) << 4. */
+static void kq_scale_min(const uint8_t* sc, int j, int* scale, int* min)
+{
+    if (j < 4) {
+        *scale = sc[j] & 63;
+        *min = sc[j + 4] & 63;
+    } else {
+        *scale = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);
+        *min = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+    }
+}
+
+/* value i (0..255) of a super-block: code bytes 32p .. 32p+31 hold sub-block
+ * 2p (low nibbles) and 2p+1 (high nibbles), value l of each at byte 32p + l;
+ * Q5_K adds 16 * bit j of qh[l] for value l of sub-block j. */
+static int kq_code(int fmt, const uint8_t* b, int i)
+{
+    int j = i / 32, l = i % 32;
+    const uint8_t* qs = b + (fmt == ORC_Q5_K ? 48 : 16);
+    int q = (j & 1) ? (qs[32 * (j / 2) + l] >> 4) : (qs[32 * (j / 2) + l] & 0x0F);
+    if (fmt == ORC_Q5_K) q |= ((b[16 + l] >> j) & 1) << 4;
+    return q;
+}
+
+int orc_is_kquant(int fmt) { return fmt == ORC_Q4_K || fmt == ORC_Q5_K; }
+
+/* x of value i of a row (fp64) */
+static double ext_value(int fmt, const uint8_t* row, int64_t i)
+{
+    if (fmt == ORC_Q5_1) {
+        const uint8_t* b = row + 24 * (i / 32);
+        return (double)orc_f16_to_f32(get16(b)) * (double)q51_code(b, (int)(i % 32)) +
+               (double)orc_f16_to_f32(get16(b + 2));
+    }
+    const uint8_t* b = row + (fmt == ORC_Q5_K ? 176 : 144) * (i / 256);
+    int sc, mn;
+    kq_scale_min(b + 4, (int)(i % 256) / 32, &sc, &mn);
+    return (double)orc_f16_to_f32(get16(b)) * sc * kq_code(fmt, b, (int)(i % 256)) -
+           (double)orc_f16_to_f32(get16(b + 2)) * mn;
+}
+
+void orc_dequantize_ext(int fmt, const uint8_t* W, int N, int K, double* out)
+{
+    int64_t rb = orc_row_bytes(fmt, K);
+    for (int n = 0; n < N; ++n)
+        for (int64_t i = 0; i < K; ++i) out[(int64_t)n * K + i] = ext_value(fmt, W + n * rb, i);
+}
+
+/* R22-R24: per 32-value block kb of a row against Q8_1 block kb: isum = sum
+ * q_w q_a, sumq = sum q_a (exact integers); sd = fp32 scale product, sm = the
+ * min product; part = fmaf((float)isum, sd, part) then part = fmaf((float)sumq,
+ * sm, part), blocks in order within chunks of 8 (= one K-quant super-block),
+ * acc = acc + part over chunks.  Q5_1: sd = d_w * d_a, sm = m_w * d_a.
+ * K-quants: sd = (d * scale_j) * d_a, sm = -((dmin * min_j) * d_a). */
+void orc_block_ext(int fmt, const uint8_t* row, int kb, const uint8_t* a, int32_t* isum, int32_t* sumq,
+                   float* sd, float* sm)
+{
+    const int8_t* qa = (const int8_t*)(a + 4);
+    float da = orc_f16_to_f32(get16(a));
+    int32_t s = 0, z = 0;
+    if (fmt == ORC_Q5_1) {
+        const uint8_t* b = row + 24 * kb;
+        for (int i = 0; i < 32; ++i) {
+            s += q51_code(b, i) * (int32_t)qa[i];
+            z += qa[i];
+        }
+        *sd = orc_f16_to_f32(get16(b)) * da;
+        *sm = orc_f16_to_f32(get16(b + 2)) * da;
+    } else {
+        const uint8_t* b = row + (fmt == ORC_Q5_K ? 176 : 144) * (kb / 8);
+        int j = kb % 8, sc, mn;
+        kq_scale_min(b + 4, j, &sc, &mn);
+        for (int i = 0; i < 32; ++i) {
+            s += kq_code(fmt, b, 32 * j + i) * (int32_t)qa[i];
+            z += qa[i];
+        }
+        float dsc = orc_f16_to_f32(get16(b)) * (float)sc;
+        float dmn = orc_f16_to_f32(get16(b + 2)) * (float)mn;
+        *sd = dsc * da;
+        *sm = -(dmn * da);
+    }
+    *isum = s;
+    *sumq = z;
+}
+
+void orc_qmatmul_ext(int fmt, const uint8_t* W, int N, int K, const uint8_t* Xq, int T, float* Y)
+{
+    int nb = K / 32;
+    int64_t rb = orc_row_bytes(fmt, K);
+    for (int t = 0; t < T; ++t) {
+        const uint8_t* xr = Xq + (int64_t)t * nb * 36;
+        for (int n = 0; n < N; ++n) {
+            const uint8_t* wr = W + (int64_t)n * rb;
+            float acc = 0.0f;
+            for (int c = 0; c < nb; c += 8) {
+                float part = 0.0f;
+                for (int kb = c; kb < c + 8 && kb < nb; ++kb) {
+                    int32_t isum, sumq;
+                    float sd, sm;
+                    orc_block_ext(fmt, wr, kb, xr + (int64_t)kb * 36, &isum, &sumq, &sd, &sm);
+                    part = fmaf((float)isum, sd, part);
+                    part = fmaf((float)sumq, sm, part);
+                }
+                acc = acc + part;
+            }
+            Y[(int64_t)t * N + n] = acc;
         }
     }
 }
@@ -563,9 +703,11 @@ static int check_layer(const orc_layer* ly)
     if (ly->H % 32 || ly->L % 32 || ly->I % 32 || ly->E < 1 || ly->k < 1 ||
         ly->k > ly->E || ly->k > 64)
         return -2;
-    if (!orc_block_bytes(ly->du_fmt) || !orc_block_bytes(ly->ex_fmt) ||
-        ly->du_fmt == ORC_Q8_1 || ly->ex_fmt == ORC_Q8_1 || ly->du_fmt == ORC_NVFP4)
+    if (!orc_row_bytes(ly->du_fmt, 256) || !orc_row_bytes(ly->ex_fmt, 256) ||
+        ly->du_fmt == ORC_Q8_1 || ly->ex_fmt == ORC_Q8_1 || ly->du_fmt == ORC_NVFP4 ||
+        ly->du_fmt == ORC_Q5_1 || orc_is_kquant(ly->du_fmt))
         return -2;
+    if (orc_is_kquant(ly->ex_fmt) && (ly->L % 256 || ly->I % 256)) return -2;
     if (ly->ex_fmt == ORC_NVFP4 && (!ly->gate_g || !ly->up_g || !ly->down_g ||
                                     !(ly->act_gz > 0.0f) || !(ly->act_gh > 0.0f)))
         return -2;
@@ -619,6 +761,7 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trac
     /* a4: latent activations for the experts (NVFP4 experts: NVFP4
      * activations under the layer's static scale act_gz, R20) */
     int nv = ly->ex_fmt == ORC_NVFP4;
+    int ext = ly->ex_fmt == ORC_Q5_1 || orc_is_kquant(ly->ex_fmt);
     if (nv) orc_quantize_nvfp4(z, (int64_t)T * L, ly->act_gz, zq);
     else orc_quantize_q8_1(z, (int64_t)T * L, zq);
     /* a5 */
@@ -634,6 +777,13 @@ int orc_moe_layer(const orc_layer* ly, const float* x, int T, float* y, orc_trac
             for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
             orc_quantize_nvfp4(h, I, ly->act_gh, hq);
             orc_qmatmul_nvfp4(ly->down[e], ly->down_g[e], L, I, hq, ly->act_gh, 1, o + (size_t)p * L);
+        } else if (ext) {
+            const uint8_t* zt = zq + (size_t)t * (L / 32) * 36;
+            orc_qmatmul_ext(ly->ex_fmt, ly->gate[e], I, L, zt, 1, g);
+            orc_qmatmul_ext(ly->ex_fmt, ly->up[e], I, L, zt, 1, u);
+            for (int i = 0; i < I; ++i) h[i] = orc_silu(g[i]) * u[i];
+            orc_quantize_q8_1(h, I, hq);
+            orc_qmatmul_ext(ly->ex_fmt, ly->down[e], L, I, hq, 1, o + (size_t)p * L);
         } else {
             const uint8_t* zt = zq + (size_t)t * (L / 32) * 36;
             orc_qmatmul(ly->ex_fmt, ly->gate[e], I, L, zt, 1, g);

@@ -77,6 +77,23 @@
  *       dec(sw) * dec(sa), part = fmaf((float)isum, sc, part) over the 16
  *       micro-blocks of a chunk of 8 blocks in order, acc = acc + part over
  *       chunks, y = acc * ((g_w * g_a) * 0.25).
+ *
+ * Q5_1, Q4_K and Q5_K experts ("Q8 0 support - Pull Request #255 -
+ * Niko1221/Strata", follow-up commit "per-role format lists": the Q4_K, Q5_K
+ * and Q5_1 expert dots; Q5_1's min term multiplies the sum of the quantised
+ * activations, not the stored s).  The blocks are the GGUF layouts those
+ * names stand for; readings:
+ *   R22 Q5_1: x = d q + m, q = 4-bit code + 16 * its qh bit (q in 0..31).
+ *       Q4_K, Q5_K: super-blocks of 256 in 8 sub-blocks of 32 with 6-bit
+ *       scale_j and min_j; x = d scale_j q - dmin min_j.
+ *   R23 per 32-value block (a K-quant sub-block) against a Q8_1 block:
+ *       isum = sum q_w q_a and sumq = sum q_a, exact integers (the min term
+ *       takes the quantised sum for every one of these formats).
+ *   R24 order: part = fmaf((float)isum, sd, part), then part =
+ *       fmaf((float)sumq, sm, part), blocks in order within chunks of 8 (one
+ *       super-block), acc = acc + part over chunks.  Q5_1: sd = d_w d_a, sm =
+ *       m_w d_a; K-quants: sd = (d scale_j) d_a, sm = -((dmin min_j) d_a),
+ *       each product one fp32 multiply (d scale_j and dmin min_j are exact).
  */
 #ifndef ELQ_ORACLE_H
 #define ELQ_ORACLE_H
@@ -87,7 +104,7 @@
 extern "C" {
 #endif
 
-enum { ORC_Q4_0 = 2, ORC_Q8_0 = 8, ORC_Q8_1 = 9, ORC_NVFP4 = 100 };
+enum { ORC_Q4_0 = 2, ORC_Q5_1 = 7, ORC_Q8_0 = 8, ORC_Q8_1 = 9, ORC_Q4_K = 12, ORC_Q5_K = 13, ORC_NVFP4 = 100 };
 
 int      orc_block_bytes(int fmt);                /* 18, 34, 36; 0 if unknown */
 int64_t  orc_matrix_bytes(int fmt, int64_t rows, int64_t k);
@@ -136,6 +153,14 @@ void     orc_quantize_nvfp4(const float* x, int64_t n, float g, uint8_t* out);
 void     orc_dequantize_nvfp4(const uint8_t* blocks, int64_t n, float g, double* out);
 void     orc_qmatmul_nvfp4(const uint8_t* W, float gw, int N, int K, const uint8_t* X, float ga,
                            int T, float* Y);
+
+/* Q5_1 / Q4_K / Q5_K (R22-R24) */
+int64_t  orc_row_bytes(int fmt, int64_t k);
+int      orc_is_kquant(int fmt);
+void     orc_dequantize_ext(int fmt, const uint8_t* W, int N, int K, double* out);
+void     orc_block_ext(int fmt, const uint8_t* row, int kb, const uint8_t* a, int32_t* isum, int32_t* sumq,
+                       float* sd, float* sm);
+void     orc_qmatmul_ext(int fmt, const uint8_t* W, int N, int K, const uint8_t* Xq, int T, float* Y);
 
 /* One latent-MoE layer.  Weight matrices are row-major AoS blocks.
  * gate/up/down are arrays of E pointers; an expert no token selects may be

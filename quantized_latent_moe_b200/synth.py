@@ -105,6 +105,52 @@ def permutation(seed: int, tid: int, n: int) -> torch.Tensor:
 
 
 # ---------------------------------------------------------------------------
+# pre-quantised weights: GGUF blocks drawn directly (random codes, 6-bit
+# sub-block scales and mins, fp16 super-block scales in a fixed binade)
+
+Q5_1, Q4_K, Q5_K = "q5_1", "q4_k", "q5_k"
+EXT_ROW_BYTES = {Q5_1: (32, 24), Q4_K: (256, 144), Q5_K: (256, 176)}   # values, bytes per block
+# fp16 exponent fields of the block scales: (d, m or dmin), so that values
+# land within about +-0.1 and Q5_1's m is negative
+_EXT_FIELDS = {Q5_1: (4, 8), Q4_K: (1, 5), Q5_K: (1, 6)}
+
+
+def ext_row_bytes(fmt: str, k: int) -> int:
+    vals, nb = EXT_ROW_BYTES[fmt]
+    return k // vals * nb
+
+
+def ext_blocks(fmt: str, seed: int, tid: int, rows: int, k: int, row0: int = 0) -> torch.Tensor:
+    """uint8 [rows, row bytes] of GGUF blocks of format fmt (q5_1, q4_k, q5_k):
+    every byte from the counter hash, then each block's fp16 scale fields
+    set to a positive fp16 of exponent field f_d (d) and, for the second
+    field, f_m (negative for Q5_1's m, positive for the K-quants' dmin), the
+    fraction bits from the hash.  Rows row0 .. row0+rows-1 of the stream."""
+    vals, bb = EXT_ROW_BYTES[fmt]
+    rb = k // vals * bb
+    nw = rb // 4
+    w = words(seed, tid, row0 * nw, rows * nw, 0)
+    by = torch.stack([(w >> (8 * i)) & 0xFF for i in range(4)], dim=1).reshape(rows, k // vals, bb)
+    fd, fm = _EXT_FIELDS[fmt]
+    d = (fd << 10) | ((by[:, :, 0] | (by[:, :, 1] << 8)) & 0x3FF)
+    m = (fm << 10) | ((by[:, :, 2] | (by[:, :, 3] << 8)) & 0x3FF)
+    if fmt == Q5_1:
+        m = m | 0x8000
+    by[:, :, 0], by[:, :, 1] = d & 0xFF, d >> 8
+    by[:, :, 2], by[:, :, 3] = m & 0xFF, m >> 8
+    return by.reshape(rows, rb).to(torch.uint8)
+
+
+def expert_blocks(wl: "Workload", e: int, layer: int = 0):
+    """Expert e's gate [I, L], up [I, L] and down [L, I] as GGUF blocks of
+    the workload's expert format (uint8 rows)."""
+    fmt = wl.expert_fmt
+    return (ext_blocks(fmt, wl.seed, tid(layer, TID_GATE), wl.I, wl.L, row0=e * wl.I),
+            ext_blocks(fmt, wl.seed, tid(layer, TID_UP), wl.I, wl.L, row0=e * wl.I),
+            ext_blocks(fmt, wl.seed, tid(layer, TID_DOWN), wl.L, wl.I, row0=e * wl.L))
+
+
+# ---------------------------------------------------------------------------
 # workloads
 
 F32, BF16 = "f32", "bf16"
