@@ -141,6 +141,9 @@ typedef enum {                  /* GGUF type ids */
     ELQ_Q4_0 = 2,
     ELQ_Q8_0 = 8,
     ELQ_Q8_1 = 9,
+    ELQ_Q5_1 = 7,
+    ELQ_Q4_K = 12,
+    ELQ_Q5_K = 13,
     ELQ_BF16 = 30,
     ELQ_NVFP4 = 100             /* not a GGUF id: this library's own */
 } elq_type;

@@ -99,18 +99,23 @@ inline elq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ELQ_OK 
 bool fmt_ok(int32_t f) { return f == ELQ_Q8_0 || f == ELQ_Q4_0; }
 // formats the arena holds (NVFP4 in the Q4_0 geometry: 16 code bytes and a
 // 16-bit scale word per row and block)
-bool arena_fmt_ok(int32_t f) { return fmt_ok(f) || f == ELQ_NVFP4; }
-int slab_bytes(int32_t f) { return f == ELQ_Q8_0 ? kQ80Slab : kQ40Slab; }
+bool ext_fmt(int32_t f) { return f == ELQ_Q5_1 || f == ELQ_Q4_K || f == ELQ_Q5_K; }
+bool arena_fmt_ok(int32_t f) { return fmt_ok(f) || f == ELQ_NVFP4 || ext_fmt(f); }
+// codes per (tile, block): four slices' pieces (WSlice::kCodes each)
+int slab_bytes(int32_t f) { return f == ELQ_Q8_0 ? kQ80Slab : fmt_has_qh(f) ? 4 * 640 : kQ40Slab; }
+// k granularity of an arena matrix
+int arena_k_unit(int32_t f) { return f == ELQ_NVFP4 ? 64 : (f == ELQ_Q4_K || f == ELQ_Q5_K) ? 256 : 32; }
 
-// nv_ok: the matrix may be NVFP4 (a layer's expert matrices), with a global
-// scale per gs_rows rows.
-elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k, bool nv_ok = false) {
+// expert: the matrix may also be NVFP4 (with a global scale per gs_rows
+// rows), Q5_1, Q4_K or Q5_K (a layer's expert matrices).
+elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k, bool expert = false) {
     if (!w) return ELQ_ERR_INVALID_ARG;
-    if (!(fmt_ok(w->fmt) || (nv_ok && w->fmt == ELQ_NVFP4))) return ELQ_ERR_UNSUPPORTED;
+    if (!(fmt_ok(w->fmt) || (expert && (w->fmt == ELQ_NVFP4 || ext_fmt(w->fmt))))) return ELQ_ERR_UNSUPPORTED;
     if (w->n_rows != rows || w->k != k || rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
     if (rows % kTileRows || k % 128) return ELQ_ERR_UNSUPPORTED;
     if (!w->q || !w->d) return ELQ_ERR_INVALID_ARG;
     if (!aligned(w->q, 256) || !aligned(w->d, 256)) return ELQ_ERR_ALIGNMENT;
+    if ((w->fmt == ELQ_Q4_K || w->fmt == ELQ_Q5_K) && k % 256) return ELQ_ERR_UNSUPPORTED;   // whole super-blocks
     if (w->fmt == ELQ_NVFP4) {
         if (k % 256) return ELQ_ERR_UNSUPPORTED;   // whole 8-block chunks of 18-byte activation blocks
         if (!w->gs || w->gs_rows <= 0 || rows % w->gs_rows) return ELQ_ERR_INVALID_ARG;
@@ -263,10 +268,10 @@ SPlan plan_s(int fmt, int x_mode, bool swiglu, int rows_per_group, int K, int gr
     p.cpc = (p.nchunks + Cg - 1) / Cg;
     // one stage of a CTA: the codes and scales of its cpc chunks, then each
     // token's activations over the same blocks
-    const int codes = p.cpc * kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512);
+    const int codes = p.cpc * kChunk * (slab_bytes(fmt) / 4);
     const int ablock = x_mode == X_RAW_F32 ? 128 : x_mode == X_RAW_BF16 ? 64 : fmt == ELQ_NVFP4 ? 18 : 36;
     p.scales_off = codes;
-    p.acts_off = (int)round_up((size_t)codes + (size_t)p.cpc * kChunk * 64, 128);
+    p.acts_off = (int)round_up((size_t)codes + (size_t)p.cpc * kChunk * 64 * scale_units(fmt), 128);
     p.act_row = p.cpc * kChunk * ablock;
     p.stage_bytes = (int)round_up((size_t)p.acts_off + (size_t)T * p.act_row, 128);
     p.scratch_bytes = (x_mode == X_RAW_F32 || x_mode == X_RAW_BF16) ? (int)round_up((size_t)T * kChunk * 36, 128)
@@ -368,6 +373,24 @@ cudaError_t launch_s(SArgs g, int fmt, int x_mode, int out_mode, const SPlan& p,
     const int64_t ctas = (int64_t)p.clusters * p.C;
     for (int r = 0; r < 3; ++r)
         g.pf_share[r] = g.pf[r] ? (int64_t)round_up((size_t)((g.pf_bytes[r] + ctas - 1) / ctas), 256) : 0;
+    if (ext_fmt(fmt)) {
+        // Q5_1 / Q4_K / Q5_K expert projections only
+        const int sel = x_mode * 16 + out_mode;
+        if (sel != X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU && sel != X_Q81_POSITION * 16 + OUT_F32_COMBINE)
+            return cudaErrorInvalidValue;
+        const bool gu = sel == X_Q81_PAIR_TOKEN * 16 + OUT_SWIGLU;
+        switch (fmt) {
+        case ELQ_Q5_1:
+            return gu ? launch_s_t<kQ51, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
+                      : launch_s_t<kQ51, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+        case ELQ_Q4_K:
+            return gu ? launch_s_t<kQ4K, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
+                      : launch_s_t<kQ4K, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+        default:
+            return gu ? launch_s_t<kQ5K, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
+                      : launch_s_t<kQ5K, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+        }
+    }
     if (fmt == ELQ_NVFP4) {
         // NVFP4 expert projections only
         switch (x_mode * 16 + out_mode) {
@@ -574,7 +597,7 @@ DecPlanH plan_dec(const elq_layer* ly, int T) {
     if (!(ly->flags & ELQ_LAYER_FUSED)) return d;
     if (T < 1 || T > kDecMaxT || (int64_t)T * ly->k > kDecMaxPairs) return d;
     if (ly->D.fmt != ly->U.fmt || ly->gate_up.fmt != ly->down.fmt) return d;
-    if (ly->gate_up.fmt == ELQ_NVFP4) return d;     // NVFP4 experts: the cluster GEMV path only
+    if (ly->gate_up.fmt == ELQ_NVFP4 || ext_fmt(ly->gate_up.fmt)) return d;   // the cluster GEMV path only
     if (ly->L / kTileRows > 64) return d;            // latent tiles the shared-memory mirror follows
     auto codes = [](int fmt) { return kChunk * (fmt == ELQ_Q8_0 ? 1024 : 512); };
     const size_t acts = (size_t)T * kChunk * 36;
@@ -774,6 +797,10 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     if ((s = check_qmat(&ly->gate_up, E * 2 * I, L, true)) != ELQ_OK) return s;
     if ((s = check_qmat(&ly->down, E * L, I, true)) != ELQ_OK) return s;
     if ((ly->gate_up.fmt == ELQ_NVFP4) != (ly->down.fmt == ELQ_NVFP4)) return ELQ_ERR_UNSUPPORTED;
+    if ((ext_fmt(ly->gate_up.fmt) || ext_fmt(ly->down.fmt)) && ly->gate_up.fmt != ly->down.fmt)
+        return ELQ_ERR_UNSUPPORTED;
+    // Q5_1 / K-quant experts: the cluster GEMV's token and pair bounds only
+    if (ext_fmt(ly->gate_up.fmt) && (T > kSMaxT || (int64_t)T * k > kSMaxPairs)) return ELQ_ERR_UNSUPPORTED;
     if (ly->gate_up.fmt == ELQ_NVFP4) {
         // one global scale per expert matrix; static activation scales
         if (ly->gate_up.gs_rows != 2 * I || ly->down.gs_rows != L) return ELQ_ERR_INVALID_ARG;
@@ -1206,7 +1233,7 @@ bool layer_tc(const elq_layer* ly, int T) {
 bool layer_fused(const elq_layer* ly, int T) { return !layer_tc(ly, T) && plan_dec(ly, T).ok; }
 
 int layer_kernels(const elq_layer* ly, int T) {
-    if (ly->gate_up.fmt == ELQ_NVFP4) {
+    if (ly->gate_up.fmt == ELQ_NVFP4 || ext_fmt(ly->gate_up.fmt)) {
         const LayerWs w = layer_layout(ly, T, nullptr, ELQ_F32);
         return w.small ? 5 : w.nvtc ? 11 : 0;
     }
@@ -1236,14 +1263,14 @@ const char* elq_status_string(int32_t status) {
 int32_t elq_version(void) { return 2; }
 
 size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k, size_t* q_bytes, size_t* d_bytes) {
-    if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % (fmt == ELQ_NVFP4 ? 64 : 32)) {
+    if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % arena_k_unit(fmt)) {
         if (q_bytes) *q_bytes = 0;
         if (d_bytes) *d_bytes = 0;
         return 0;
     }
     const size_t slabs = (size_t)(n_rows / kTileRows) * (k / 32);
     // NVFP4: each tile's scales twice (per row, and as the tensor cores' atoms)
-    const size_t q = slabs * slab_bytes(fmt), d = slabs * kScaleSlab * (fmt == ELQ_NVFP4 ? 2 : 1);
+    const size_t q = slabs * slab_bytes(fmt), d = slabs * kScaleSlab * (fmt == ELQ_NVFP4 ? 2 : scale_units(fmt));
     if (q_bytes) *q_bytes = q;
     if (d_bytes) *d_bytes = d;
     return q + d;
@@ -1253,12 +1280,21 @@ elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t 
                           void* stream) {
     if (!arena_fmt_ok(fmt)) return ELQ_ERR_UNSUPPORTED;
     if (!aos || !q_out || !d_out || n_rows <= 0 || k <= 0) return ELQ_ERR_INVALID_ARG;
-    if (n_rows % kTileRows || k % (fmt == ELQ_NVFP4 ? 64 : 32)) return ELQ_ERR_UNSUPPORTED;
+    if (n_rows % kTileRows || k % arena_k_unit(fmt)) return ELQ_ERR_UNSUPPORTED;
     if (!aligned(q_out, 256) || !aligned(d_out, 256)) return ELQ_ERR_ALIGNMENT;
     const int64_t n = (int64_t)n_rows * (k / 32);
     const dim3 grid((unsigned)((n + 255) / 256));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (fmt == ELQ_Q8_0)
+    uint32_t* d32 = static_cast<uint32_t*>(d_out);
+    const uint8_t* src = static_cast<const uint8_t*>(aos);
+    uint8_t* q8 = static_cast<uint8_t*>(q_out);
+    if (fmt == ELQ_Q5_1)
+        k_arena_pack_ext<kQ51><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
+    else if (fmt == ELQ_Q4_K)
+        k_arena_pack_ext<kQ4K><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
+    else if (fmt == ELQ_Q5_K)
+        k_arena_pack_ext<kQ5K><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
+    else if (fmt == ELQ_Q8_0)
         k_arena_pack<8><<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(aos), n_rows, k,
                                              static_cast<uint8_t*>(q_out), static_cast<uint16_t*>(d_out));
     else if (fmt == ELQ_NVFP4)
@@ -1444,11 +1480,11 @@ elq_status elq_moe_experts_grouped(const elq_layer* layer, const void* z_q8_1, c
     const int E = layer->E, k = layer->k;
     const int64_t P = (int64_t)T * k;
     const int nw = 32;
-    const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
+    const bool nv = layer->gate_up.fmt == ELQ_NVFP4 || ext_fmt(layer->gate_up.fmt);
     if (nv && !w.nvtc) {
         const int gmax = (int)std::min<int64_t>(E, P);
-        if (!plan_s(ELQ_NVFP4, X_Q81_PAIR_TOKEN, true, 2 * layer->I, layer->L, gmax, T, true).ok ||
-            !plan_s(ELQ_NVFP4, X_Q81_POSITION, false, layer->L, layer->I, gmax, T, true).ok)
+        if (!plan_s(layer->gate_up.fmt, X_Q81_PAIR_TOKEN, true, 2 * layer->I, layer->L, gmax, T, true).ok ||
+            !plan_s(layer->down.fmt, X_Q81_POSITION, false, layer->L, layer->I, gmax, T, true).ok)
             return ELQ_ERR_UNSUPPORTED;
     }
     cudaError_t e = smem_optin(k_bucket, kRouterSmemMax, g_optin_bucket);
@@ -1740,7 +1776,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     if (!router_shape_ok(T, layer->L, layer->E)) return ELQ_ERR_UNSUPPORTED;
     LayerWs w = layer_layout(layer, T, ws, x_type);
     const bool nv = layer->gate_up.fmt == ELQ_NVFP4;
-    if (nv && !w.small && !w.nvtc) return ELQ_ERR_UNSUPPORTED;
+    if ((nv || ext_fmt(layer->gate_up.fmt)) && !w.small && !w.nvtc) return ELQ_ERR_UNSUPPORTED;
     if (!ws || ws_bytes < w.total) return ELQ_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return ELQ_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

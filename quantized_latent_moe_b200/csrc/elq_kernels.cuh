@@ -176,8 +176,67 @@ __global__ void __launch_bounds__(256) k_quant_weights(const float* __restrict__
 // the tensor cores' scale-factor atoms: per pair of blocks (64 values) one
 // 512-byte atom, row m's four scales (blocks 2j, 2j+1, micro-blocks 0, 1) as
 // one 32-bit word at byte (m % 32) * 16 + (m / 32) * 4.
+// In 16-bit units; Q5_1 / K-quant tiles hold a 32-bit word per (row, block).
 __host__ __device__ constexpr int64_t d_tile_elems(int fmt, int nb) {
-    return (int64_t)nb * kTileRows * (fmt == kNV ? 2 : 1);
+    return (int64_t)nb * kTileRows * (fmt == kNV ? 2 : scale_units(fmt));
+}
+
+// Q5_1 / Q4_K / Q5_K arena from GGUF blocks, one thread per (row, 32-value
+// block).  Per (tile, slice, block) piece: 32 rows of 16 code bytes (byte i:
+// value i in the low nibble, value i + 16 in the high one -- Q4_0's order, 4-bit
+// codes without an offset), then for Q5_1 / Q5_K 32 rows of a 32-bit word of
+// the codes' fifth bits (bit i for value i).  Scale word per (row, block):
+// Q5_1 fp16 d | fp16 m << 16; K-quants 6-bit scale | 6-bit min << 8 | (the
+// super-block's fp16 d in sub-block 0, its fp16 dmin in sub-block 1) << 16.
+template <int FMT>
+__global__ void __launch_bounds__(256) k_arena_pack_ext(const uint8_t* __restrict__ aos, int n_rows, int k,
+                                                        uint8_t* __restrict__ q, uint32_t* __restrict__ d) {
+    const int nb = k / 32;
+    const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= (int64_t)n_rows * nb) return;
+    const int64_t row = id / nb;
+    const int kb = (int)(id % nb);
+    const int64_t tile = row / kTileRows;
+    const int slice = (int)(row % kTileRows) / 32, r = (int)(row % 32);
+    constexpr int kPiece = fmt_has_qh(FMT) ? 640 : 512;
+    uint8_t codes[32];
+    uint32_t qh = 0, sw;
+    if (FMT == kQ51) {
+        const uint8_t* b = aos + (row * nb + kb) * 24;
+        for (int i = 0; i < 16; ++i) {
+            codes[i] = b[8 + i] & 15;
+            codes[i + 16] = b[8 + i] >> 4;
+        }
+        qh = (uint32_t)b[4] | ((uint32_t)b[5] << 8) | ((uint32_t)b[6] << 16) | ((uint32_t)b[7] << 24);
+        sw = (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
+    } else {
+        constexpr int kBB = FMT == kQ5K ? 176 : 144;
+        const uint8_t* b = aos + (row * (nb / 8) + kb / 8) * kBB;
+        const int j = kb % 8;
+        const uint8_t* sc = b + 4;
+        int scale, mn;
+        if (j < 4) {
+            scale = sc[j] & 63;
+            mn = sc[j + 4] & 63;
+        } else {
+            scale = (sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4);
+            mn = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+        }
+        const uint8_t* qs = b + (FMT == kQ5K ? 48 : 16) + 32 * (j / 2);
+        for (int l = 0; l < 32; ++l) codes[l] = (j & 1) ? (qs[l] >> 4) : (qs[l] & 15);
+        if (FMT == kQ5K)
+            for (int l = 0; l < 32; ++l) qh |= (uint32_t)((b[16 + l] >> j) & 1) << l;
+        uint32_t hi = 0;
+        if (j == 0) hi = (uint32_t)b[0] | ((uint32_t)b[1] << 8);
+        if (j == 1) hi = (uint32_t)b[2] | ((uint32_t)b[3] << 8);
+        sw = (uint32_t)scale | ((uint32_t)mn << 8) | (hi << 16);
+    }
+    uint32_t words[4] = {0, 0, 0, 0};
+    for (int i = 0; i < 16; ++i) words[i >> 2] |= (uint32_t)(codes[i] | (codes[i + 16] << 4)) << (8 * (i & 3));
+    uint8_t* piece = q + tile * nb * (4 * kPiece) + (int64_t)slice * nb * kPiece + (int64_t)kb * kPiece;
+    *reinterpret_cast<uint4*>(piece + r * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+    if (fmt_has_qh(FMT)) *reinterpret_cast<uint32_t*>(piece + 512 + r * 4) = qh;
+    d[tile * nb * kTileRows + (int64_t)slice * nb * 32 + (int64_t)kb * 32 + r] = sw;
 }
 
 template <int FMT>
@@ -676,7 +735,9 @@ struct WArgs {
 
 template <int FMT>
 struct WSlice {
-    static constexpr int kCodes = (FMT == 8) ? 1024 : 512;   // bytes per (slice, block)
+    // bytes per (slice, block): Q8_0 codes; 4-bit codes (Q4_0, NVFP4, Q4_K);
+    // 4-bit codes and a word of fifth bits per row (Q5_1, Q5_K)
+    static constexpr int kCodes = (FMT == 8) ? 1024 : fmt_has_qh(FMT) ? 640 : 512;
 };
 
 struct WUnit {

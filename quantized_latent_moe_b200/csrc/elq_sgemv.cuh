@@ -233,13 +233,14 @@ template <int FMT, int XM>
 __device__ __forceinline__ void s_issue_weights(const SArgs& g, const SUnit& u, const SRange& r, uint8_t* stg,
                                                 uint64_t* bar) {
     using SL = WSlice<FMT>;
-    const uint32_t cb = (uint32_t)(r.nblk * SL::kCodes), sb = (uint32_t)(r.nblk * 64);
+    constexpr int SU = scale_units(FMT);
+    const uint32_t cb = (uint32_t)(r.nblk * SL::kCodes), sb = (uint32_t)(r.nblk * 64 * SU);
     mbar_arrive_expect_tx(bar, cb + sb + (uint32_t)u.grp.z * (uint32_t)r.nblk * s_act_block<FMT, XM>());
     bulk_g2s(stg, g.q + u.grp.x * g.q_gstride + ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
              cb, bar);
     bulk_g2s(stg + g.scales_off,
-             g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) + (int64_t)u.s * g.nb * 32 +
-                 (int64_t)r.kb0 * 32,
+             g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) +
+                 ((int64_t)u.s * g.nb * 32 + (int64_t)r.kb0 * 32) * SU,
              sb, bar);
 }
 
@@ -408,6 +409,87 @@ __device__ __forceinline__ int nv_dot16(uint32_t w0, uint32_t w1, const uint4& a
     p = __dp4a((int)e2m1x4_pos(w1 >> 16), (int)a.w, p);
     n = __dp4a((int)e2m1x4_pos(n1 >> 16), (int)a.w, n);
     return p - n;
+}
+
+// Bit 4 of each byte of a word from 4 bits of x (bit b -> bit 8 b + 4).
+__device__ __forceinline__ uint32_t spread4_to_bit4(uint32_t x) {
+    return ((x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21)) << 4;
+}
+
+// The Q5_1 / Q4_K / Q5_K form of s_dots (Q8_1 activations): per block, the
+// row's codes (4-bit, plus the fifth bits) as unsigned bytes, isum = sum q_w
+// q_a and sumq = sum q_a (dp4a), and the block's two fp32 factors: Q5_1 sd =
+// d_w d_a, sm = m_w d_a; K-quants sd = (d scale) d_a, sm = -((dmin min) d_a),
+// d and dmin from the words of the chunk's (super-block's) first two blocks.
+// Then part = fmaf(isum, sd, part), part = fmaf(sumq, sm, part) per block in
+// order.
+template <int FMT, int XM>
+__device__ __forceinline__ void s_dots_ext(const SArgs& g, const SUnit& u, const uint8_t* stg, uint32_t dst) {
+    using SL = WSlice<FMT>;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const uint8_t* codes = stg + warp * kChunk * SL::kCodes;
+    const uint32_t* sw = reinterpret_cast<const uint32_t*>(stg + g.scales_off) + warp * kChunk * 32;
+    const uint8_t* abase = stg + g.acts_off + warp * kChunk * 36;
+    const int nt = u.grp.z;
+    float dk = 0.0f, dmk = 0.0f;
+    if (FMT != kQ51) {
+        dk = h2f((uint16_t)(sw[lane] >> 16));
+        dmk = h2f((uint16_t)(sw[32 + lane] >> 16));
+    }
+#pragma unroll 1
+    for (int t = 0; t < nt; ++t) {
+        const uint8_t* ab = abase + t * g.act_row;
+        float part = 0.0f;
+        // four blocks' sums and factors at a time, then their ordered fmafs
+#pragma unroll
+        for (int h = 0; h < kChunk; h += 4) {
+            int isum[4], sumq[4];
+            float sd[4], sm[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kb = h + i;
+                isum[i] = sumq[i] = 0;
+                sd[i] = sm[i] = 0.0f;
+                if (kb < u.kbn) {
+                    const uint4 c = lds128(codes + kb * SL::kCodes + lane * 16);
+                    const uint32_t v[4] = {c.x, c.y, c.z, c.w};
+                    uint32_t qh = 0;
+                    if (fmt_has_qh(FMT))
+                        qh = *reinterpret_cast<const uint32_t*>(codes + kb * SL::kCodes + 512 + lane * 4);
+                    const uint32_t* aw = reinterpret_cast<const uint32_t*>(ab + kb * 36);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t lo = v[j] & 0x0F0F0F0Fu, hi = (v[j] >> 4) & 0x0F0F0F0Fu;
+                        if (fmt_has_qh(FMT)) {
+                            lo |= spread4_to_bit4((qh >> (4 * j)) & 15u);
+                            hi |= spread4_to_bit4((qh >> (16 + 4 * j)) & 15u);
+                        }
+                        isum[i] = __dp4a((int)lo, (int)aw[1 + j], isum[i]);
+                        isum[i] = __dp4a((int)hi, (int)aw[5 + j], isum[i]);
+                        sumq[i] = __dp4a(0x01010101, (int)aw[1 + j], sumq[i]);
+                        sumq[i] = __dp4a(0x01010101, (int)aw[5 + j], sumq[i]);
+                    }
+                    const float da = h2f((uint16_t)(aw[0] & 0xffff));
+                    const uint32_t w = sw[kb * 32 + lane];
+                    if (FMT == kQ51) {
+                        sd[i] = __fmul_rn(h2f((uint16_t)(w & 0xffff)), da);
+                        sm[i] = __fmul_rn(h2f((uint16_t)(w >> 16)), da);
+                    } else {
+                        sd[i] = __fmul_rn(__fmul_rn(dk, (float)(w & 0xff)), da);
+                        sm[i] = -__fmul_rn(__fmul_rn(dmk, (float)((w >> 8) & 0xff)), da);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (h + i < u.kbn) {
+                    part = __fmaf_rn(__int2float_rn(isum[i]), sd[i], part);
+                    part = __fmaf_rn(__int2float_rn(sumq[i]), sm[i], part);
+                }
+        }
+        dsmem_st(dst + (uint32_t)((t * 32 + lane) * 4), part);
+    }
 }
 
 // Scratch of the NVFP4 dot: per (token, block) of the chunk the activations'
@@ -596,9 +678,9 @@ __device__ __forceinline__ void s_prefetch_own(const SArgs& g, const uint8_t* rs
         bulk_prefetch_l2(g.q + u.grp.x * g.q_gstride +
                              ((int64_t)u.tile * g.nb * 4 + (int64_t)u.s * g.nb + r.kb0) * SL::kCodes,
                          (uint32_t)(r.nblk * SL::kCodes));
-        bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) + (int64_t)u.s * g.nb * 32 +
-                             (int64_t)r.kb0 * 32,
-                         (uint32_t)(r.nblk * 64));
+        bulk_prefetch_l2(g.d + u.grp.x * g.d_gstride + u.tile * d_tile_elems(FMT, g.nb) +
+                             ((int64_t)u.s * g.nb * 32 + (int64_t)r.kb0 * 32) * scale_units(FMT),
+                         (uint32_t)(r.nblk * 64 * scale_units(FMT)));
     }
 }
 
@@ -856,6 +938,7 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
             } else {
                 const uint32_t dst = pb_lead + (uint32_t)(((m & 1) * units + uidx) * g.T * 128);
                 if constexpr (FMT == kNV) s_dots_nv<XM>(g, u, stg, scratch, dst);
+                else if constexpr (fmt_ext(FMT)) s_dots_ext<FMT, XM>(g, u, stg, dst);
                 else s_dots<FMT, XM>(g, u, stg, scratch, dst);
             }
         }

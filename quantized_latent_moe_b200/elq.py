@@ -15,10 +15,12 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libelq.so")
 
-F32, Q4_0, Q8_0, Q8_1, BF16, NVFP4 = 0, 2, 8, 9, 30, 100
+F32, Q4_0, Q5_1, Q8_0, Q8_1, Q4_K, Q5_K, BF16, NVFP4 = 0, 2, 7, 8, 9, 12, 13, 30, 100
 LAYER_FUSED = 1            # elq_layer.flags: small T as one persistent kernel
-FMT = {"q8_0": Q8_0, "q4_0": Q4_0, "nvfp4": NVFP4}
-SLAB = {Q8_0: 4096, Q4_0: 2048, NVFP4: 2048}
+FMT = {"q8_0": Q8_0, "q4_0": Q4_0, "nvfp4": NVFP4, "q5_1": Q5_1, "q4_k": Q4_K, "q5_k": Q5_K}
+SLAB = {Q8_0: 4096, Q4_0: 2048, NVFP4: 2048, Q5_1: 2560, Q4_K: 2048, Q5_K: 2560}   # code bytes per (tile, block)
+SCALE_SLAB = {NVFP4: 512, Q5_1: 512, Q4_K: 512, Q5_K: 512}                       # scale bytes per (tile, block)
+EXT = (Q5_1, Q4_K, Q5_K)
 
 
 class ElqError(RuntimeError):
@@ -219,18 +221,39 @@ class Layer:
             _ck(_lib().elq_quantize_nvfp4(_ptr(de), F32, L, I, float(g_down[e]), _ptr(aos_dn[e]),
                                           _stream(stream)), "elq_quantize_nvfp4")
         per_q = (2 * I // 128) * (L // 32) * SLAB[NVFP4]
-        per_d = (2 * I // 128) * (L // 32) * 512      # per-row scales, then the scale atoms
+        per_d = (2 * I // 128) * (L // 32) * SCALE_SLAB[NVFP4]   # per-row scales, then the scale atoms
         _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_gu), n * 2 * I, L,
                                   ctypes.c_void_p(gu.q.data_ptr() + e0 * per_q),
                                   ctypes.c_void_p(gu.d.data_ptr() + e0 * per_d), _stream(stream)),
             "elq_arena_pack")
         dq = (L // 128) * (I // 32) * SLAB[NVFP4]
-        dd = (L // 128) * (I // 32) * 512
+        dd = (L // 128) * (I // 32) * SCALE_SLAB[NVFP4]
         _ck(_lib().elq_arena_pack(NVFP4, _ptr(aos_dn), n * L, I, ctypes.c_void_p(dn.q.data_ptr() + e0 * dq),
                                   ctypes.c_void_p(dn.d.data_ptr() + e0 * dd), _stream(stream)),
             "elq_arena_pack")
         gu.gs[e0:e0 + n].copy_(g_gate_up)
         dn.gs[e0:e0 + n].copy_(g_down)
+
+    def set_expert_blocks(self, e0: int, gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor, stream=None):
+        """Experts e0 .. e0+n-1 from GGUF blocks (uint8 rows) of the layer's
+        expert format (Q5_1, Q4_K, Q5_K): gate / up [n, I, row bytes of L],
+        down [n, L, row bytes of I], packed into the arena (gate and up
+        interleaved by 64-row halves)."""
+        n, I = gate.shape[0], self.I
+        gu, dn = self.gate_up, self.down
+        rb = gate.shape[2]
+        gi = torch.stack([gate.reshape(n, I // 64, 64, rb), up.reshape(n, I // 64, 64, rb)], dim=2)
+        gi = gi.reshape(n * 2 * I, rb).contiguous()
+        per_q = (2 * I // 128) * (self.L // 32) * SLAB[gu.fmt]
+        per_d = (2 * I // 128) * (self.L // 32) * SCALE_SLAB[gu.fmt]
+        _ck(_lib().elq_arena_pack(gu.fmt, _ptr(gi), n * 2 * I, self.L,
+                                  ctypes.c_void_p(gu.q.data_ptr() + e0 * per_q),
+                                  ctypes.c_void_p(gu.d.data_ptr() + e0 * per_d), _stream(stream)), "elq_arena_pack")
+        dq = (self.L // 128) * (I // 32) * SLAB[dn.fmt]
+        dd = (self.L // 128) * (I // 32) * SCALE_SLAB[dn.fmt]
+        down = down.reshape(n * self.L, -1).contiguous()
+        _ck(_lib().elq_arena_pack(dn.fmt, _ptr(down), n * self.L, I, ctypes.c_void_p(dn.q.data_ptr() + e0 * dq),
+                                  ctypes.c_void_p(dn.d.data_ptr() + e0 * dd), _stream(stream)), "elq_arena_pack")
 
     def struct(self) -> LayerC:
         return LayerC(self.H, self.L, self.E, self.k, self.I, self.flags, self.D.struct(), self.U.struct(),

@@ -6,7 +6,8 @@ import torch
 
 from quantized_latent_moe_b200 import synth
 
-ORC_FMT = {"q8_0": 8, "q4_0": 2, "nvfp4": 100}
+ORC_FMT = {"q8_0": 8, "q4_0": 2, "nvfp4": 100, "q5_1": 7, "q4_k": 12, "q5_k": 13}
+EXT = ("q5_1", "q4_k", "q5_k")
 
 
 def nvfp4_globals(w: torch.Tensor) -> torch.Tensor:
@@ -31,6 +32,10 @@ def gpu_layer(wl, layer=0, device="cuda", expert_batch=16):
         ly.act_gz = ly.act_gh = synth.NVFP4_ACT_GSCALE
     for e0 in range(0, wl.E, expert_batch):
         es = range(e0, min(wl.E, e0 + expert_batch))
+        if wl.expert_fmt in EXT:
+            bs = [synth.expert_blocks(wl, e, layer) for e in es]
+            ly.set_expert_blocks(e0, *(torch.stack([b[i] for b in bs]).to(device) for i in range(3)))
+            continue
         ws = [synth.expert_weights(wl, e, layer, device=device) for e in es]
         g, u, d = (torch.stack([w[i] for w in ws]) for i in range(3))
         if efmt == elq.NVFP4:
@@ -62,7 +67,10 @@ def add_experts(ly, wl, experts, layer=0):
     d = [None] * wl.E
     for e in experts:
         if ly.gate[e] is None:
-            a, b, c = synth.expert_weights(wl, int(e), layer)
+            if wl.expert_fmt in EXT:
+                a, b, c = synth.expert_blocks(wl, int(e), layer)
+            else:
+                a, b, c = synth.expert_weights(wl, int(e), layer)
             g[e], u[e], d[e] = a.numpy(), b.numpy(), c.numpy()
     ly.set_experts({"gate": g, "up": u, "down": d}, [e for e in experts if g[e] is not None])
 

@@ -194,6 +194,39 @@ def test_nvfp4_arena_and_quantiser_validation(L):
     assert L.elq_quantize_weights(elq.NVFP4, x, 128, 64, out, out, None) == -2
 
 
+def test_ext_format_layer_validation(L):
+    """Q5_1 / Q4_K / Q5_K experts: the cluster GEMV path (T <= 8, T * k <= 64)
+    only; gate/up and down in one format; K-quant matrices in whole
+    256-value super-blocks."""
+    x = ctypes.c_void_p(1 << 27)
+    y = ctypes.c_void_p(1 << 28)
+    ws = ctypes.c_void_p(1 << 26)
+    q, d = elq.SZ(), elq.SZ()
+    assert L.elq_arena_bytes(elq.Q5_1, 128, 64, ctypes.byref(q), ctypes.byref(d)) == 128 * 2 * (20 + 4)
+    assert L.elq_arena_bytes(elq.Q4_K, 128, 256, ctypes.byref(q), ctypes.byref(d)) == 128 * 8 * (16 + 4)
+    assert L.elq_arena_bytes(elq.Q5_K, 128, 256, ctypes.byref(q), ctypes.byref(d)) == 128 * 8 * (20 + 4)
+    assert L.elq_arena_bytes(elq.Q4_K, 128, 128, None, None) == 0
+    for fmt in (elq.Q5_1, elq.Q4_K, elq.Q5_K):
+        ly = _layer(L_=256, I=256)
+        ly.gate_up = _qm(fmt, 8 * 2 * 256, 256)
+        ly.down = _qm(fmt, 8 * 256, 256)
+        for T in (1, 4, 8):
+            assert L.elq_layer_kernel_count(ctypes.byref(ly), T) == 5
+        for T in (9, 64):
+            assert L.elq_layer_kernel_count(ctypes.byref(ly), T) == 0
+            assert L.elq_moe_layer(ctypes.byref(ly), x, 0, T, y, ws, 1 << 30, None) == -2
+        mixed = _layer(L_=256, I=256)
+        mixed.gate_up = _qm(fmt, 8 * 2 * 256, 256)
+        assert L.elq_moe_layer(ctypes.byref(mixed), x, 0, 1, y, ws, 1 << 30, None) == -2
+        bad = _layer(fmt=8)
+        bad.D = _qm(fmt, 256, 512)
+        assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 1, y, ws, 1 << 30, None) == -2
+    kq = _layer(L_=384, I=256)
+    kq.gate_up = _qm(elq.Q4_K, 8 * 2 * 256, 384)
+    kq.down = _qm(elq.Q4_K, 8 * 384, 256)
+    assert L.elq_moe_layer(ctypes.byref(kq), x, 0, 1, y, ws, 1 << 30, None) == -2
+
+
 def test_stack_validation(L):
     ws = ctypes.c_void_p(1 << 26)
     x = ctypes.c_void_p(1 << 27)
