@@ -3,7 +3,7 @@
 Only the tests, the package's ``smoke()`` check and the benchmark's CPU
 baseline leg may use this package.  The CUDA library never imports, links or
 calls it, and it imports nothing from the CUDA library.  What it computes is
-stated in ``elq_oracle.h`` (readings R1-R24) and written out in
+stated in ``elq_oracle.h`` (readings R1-R25) and written out in
 ``elq_oracle.c`` as plain loops; this module only builds the C file with gcc
 and marshals numpy arrays into it.
 """
@@ -20,9 +20,9 @@ SRC = os.path.join(HERE, "elq_oracle.c")
 HDR = os.path.join(HERE, "elq_oracle.h")
 LIB = os.path.join(HERE, "libelq_oracle.so")
 
-Q4_0, Q5_1, Q8_0, Q8_1, Q4_K, Q5_K, NVFP4 = 2, 7, 8, 9, 12, 13, 100
+Q4_0, Q5_1, Q8_0, Q8_1, Q3_K, Q4_K, Q5_K, NVFP4 = 2, 7, 8, 9, 11, 12, 13, 100
 BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q8_1: 36, NVFP4: 18, Q5_1: 24}
-EXT = (Q5_1, Q4_K, Q5_K)           # expert formats given as GGUF blocks (R22-R24)
+EXT = (Q5_1, Q3_K, Q4_K, Q5_K)     # expert formats given as GGUF blocks (R22-R25)
 
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC",
           "-shared", "-Wall", "-Wextra"]

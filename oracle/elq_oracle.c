@@ -31,6 +31,7 @@ int orc_block_bytes(int fmt)
 /* bytes of a row of k values (K-quants: super-blocks of 256) */
 int64_t orc_row_bytes(int fmt, int64_t k)
 {
+    if (fmt == ORC_Q3_K) return (k / 256) * 110;
     if (fmt == ORC_Q4_K) return (k / 256) * 144;
     if (fmt == ORC_Q5_K) return (k / 256) * 176;
     return (k / 32) * (int64_t)orc_block_bytes(fmt);
@@ -314,11 +315,39 @@ static int kq_code(int fmt, const uint8_t* b, int i)
     return q;
 }
 
-int orc_is_kquant(int fmt) { return fmt == ORC_Q4_K || fmt == ORC_Q5_K; }
+int orc_is_kquant(int fmt) { return fmt == ORC_Q3_K || fmt == ORC_Q4_K || fmt == ORC_Q5_K; }
+
+/* Q3_K super-block (110 bytes, 256 values): hmask[32], qs[64], 12 bytes of
+ * 16 packed 6-bit scales, fp16 d last.  Value i = 128 n + 32 j + l (half n,
+ * bit pair j, l < 32): low two bits (qs[32 n + l] >> 2 j) & 3, high bit =
+ * bit (4 n + j) of hmask[l]; q = low - (high ? 0 : 4) in -4 .. 3.  Scale of
+ * the 16-value sub-block s = i / 16: four low bits from byte s (s < 8, low
+ * nibble) or byte s - 8 (high nibble), two high bits (byte 8 + s % 4 >> 2 (s /
+ * 4)) & 3; scale = that 6-bit value - 32.  x = d * scale * q. */
+static int q3k_code(const uint8_t* b, int i)
+{
+    int n = i / 128, j = (i % 128) / 32, l = i % 32;
+    int low = (b[32 + 32 * n + l] >> (2 * j)) & 3;
+    int high = (b[l] >> (4 * n + j)) & 1;
+    return low - (high ? 0 : 4);
+}
+
+static int q3k_scale(const uint8_t* b, int s)
+{
+    const uint8_t* sc = b + 96;
+    int low4 = s < 8 ? (sc[s] & 15) : (sc[s - 8] >> 4);
+    int hi2 = (sc[8 + s % 4] >> (2 * (s / 4))) & 3;
+    return (low4 | (hi2 << 4)) - 32;
+}
 
 /* x of value i of a row (fp64) */
 static double ext_value(int fmt, const uint8_t* row, int64_t i)
 {
+    if (fmt == ORC_Q3_K) {
+        const uint8_t* b = row + 110 * (i / 256);
+        int v = (int)(i % 256);
+        return (double)orc_f16_to_f32(get16(b + 108)) * q3k_scale(b, v / 16) * q3k_code(b, v);
+    }
     if (fmt == ORC_Q5_1) {
         const uint8_t* b = row + 24 * (i / 32);
         return (double)orc_f16_to_f32(get16(b)) * (double)q51_code(b, (int)(i % 32)) +
@@ -350,6 +379,22 @@ void orc_block_ext(int fmt, const uint8_t* row, int kb, const uint8_t* a, int32_
     const int8_t* qa = (const int8_t*)(a + 4);
     float da = orc_f16_to_f32(get16(a));
     int32_t s = 0, z = 0;
+    if (fmt == ORC_Q3_K) {
+        /* two 16-value sub-blocks: (isum, sd) of the first as (isum, sd),
+         * of the second as (sumq, sm), so that the R24 chain takes them in
+         * order (R25) */
+        const uint8_t* b = row + 110 * (kb / 8);
+        int j = kb % 8;
+        int32_t s0 = 0, s1 = 0;
+        for (int i = 0; i < 16; ++i) s0 += q3k_code(b, 32 * j + i) * (int32_t)qa[i];
+        for (int i = 16; i < 32; ++i) s1 += q3k_code(b, 32 * j + i) * (int32_t)qa[i];
+        float d = orc_f16_to_f32(get16(b + 108));
+        *isum = s0;
+        *sumq = s1;
+        *sd = (d * (float)q3k_scale(b, 2 * j)) * da;
+        *sm = (d * (float)q3k_scale(b, 2 * j + 1)) * da;
+        return;
+    }
     if (fmt == ORC_Q5_1) {
         const uint8_t* b = row + 24 * kb;
         for (int i = 0; i < 32; ++i) {

@@ -94,6 +94,17 @@
  *       super-block), acc = acc + part over chunks.  Q5_1: sd = d_w d_a, sm =
  *       m_w d_a; K-quants: sd = (d scale_j) d_a, sm = -((dmin min_j) d_a),
  *       each product one fp32 multiply (d scale_j and dmin min_j are exact).
+ *
+ * Q3_K experts ("edge0-strata/EDGE0.md", "Changes from upstream Strata":
+ * "NVFP4 and Q3_K latent experts"):
+ *   R25 the GGUF Q3_K super-block (256 values, 16 sub-blocks of 16 with
+ *       6-bit scales stored offset by 32, 3-bit codes as two low bits and a
+ *       high-bit mask, q = low - 4 when the high bit is clear); x = d scale q.
+ *       Per 32-value block the two 16-value halves: isum_h = sum q_w q_a
+ *       (exact), sd_h = (d scale_h) d_a; part = fmaf(isum_0, sd_0, part), then
+ *       part = fmaf(isum_1, sd_1, part), in the R8 chunk order (no min term).
+ *       orc_block_ext returns (isum_0, isum_1, sd_0, sd_1) in (isum, sumq,
+ *       sd, sm).
  */
 #ifndef ELQ_ORACLE_H
 #define ELQ_ORACLE_H
@@ -104,7 +115,8 @@
 extern "C" {
 #endif
 
-enum { ORC_Q4_0 = 2, ORC_Q5_1 = 7, ORC_Q8_0 = 8, ORC_Q8_1 = 9, ORC_Q4_K = 12, ORC_Q5_K = 13, ORC_NVFP4 = 100 };
+enum { ORC_Q4_0 = 2, ORC_Q5_1 = 7, ORC_Q8_0 = 8, ORC_Q8_1 = 9, ORC_Q3_K = 11, ORC_Q4_K = 12, ORC_Q5_K = 13,
+       ORC_NVFP4 = 100 };
 
 int      orc_block_bytes(int fmt);                /* 18, 34, 36; 0 if unknown */
 int64_t  orc_matrix_bytes(int fmt, int64_t rows, int64_t k);

@@ -108,11 +108,11 @@ def permutation(seed: int, tid: int, n: int) -> torch.Tensor:
 # pre-quantised weights: GGUF blocks drawn directly (random codes, 6-bit
 # sub-block scales and mins, fp16 super-block scales in a fixed binade)
 
-Q5_1, Q4_K, Q5_K = "q5_1", "q4_k", "q5_k"
-EXT_ROW_BYTES = {Q5_1: (32, 24), Q4_K: (256, 144), Q5_K: (256, 176)}   # values, bytes per block
+Q5_1, Q3_K, Q4_K, Q5_K = "q5_1", "q3_k", "q4_k", "q5_k"
+EXT_ROW_BYTES = {Q5_1: (32, 24), Q3_K: (256, 110), Q4_K: (256, 144), Q5_K: (256, 176)}   # values, bytes per block
 # fp16 exponent fields of the block scales: (d, m or dmin), so that values
 # land within about +-0.1 and Q5_1's m is negative
-_EXT_FIELDS = {Q5_1: (4, 8), Q4_K: (1, 5), Q5_K: (1, 6)}
+_EXT_FIELDS = {Q5_1: (4, 8), Q3_K: (5, None), Q4_K: (1, 5), Q5_K: (1, 6)}
 
 
 def ext_row_bytes(fmt: str, k: int) -> int:
@@ -121,17 +121,23 @@ def ext_row_bytes(fmt: str, k: int) -> int:
 
 
 def ext_blocks(fmt: str, seed: int, tid: int, rows: int, k: int, row0: int = 0) -> torch.Tensor:
-    """uint8 [rows, row bytes] of GGUF blocks of format fmt (q5_1, q4_k, q5_k):
+    """uint8 [rows, row bytes] of GGUF blocks of format fmt (q5_1, q3_k, q4_k, q5_k):
     every byte from the counter hash, then each block's fp16 scale fields
     set to a positive fp16 of exponent field f_d (d) and, for the second
     field, f_m (negative for Q5_1's m, positive for the K-quants' dmin), the
     fraction bits from the hash.  Rows row0 .. row0+rows-1 of the stream."""
     vals, bb = EXT_ROW_BYTES[fmt]
     rb = k // vals * bb
-    nw = rb // 4
+    nw = (rb + 3) // 4                    # hash words per row (the last one partly used)
     w = words(seed, tid, row0 * nw, rows * nw, 0)
-    by = torch.stack([(w >> (8 * i)) & 0xFF for i in range(4)], dim=1).reshape(rows, k // vals, bb)
+    by = torch.stack([(w >> (8 * i)) & 0xFF for i in range(4)], dim=1).reshape(rows, nw * 4)[:, :rb]
+    by = by.reshape(rows, k // vals, bb).clone()
     fd, fm = _EXT_FIELDS[fmt]
+    if fmt == Q3_K:
+        # the super-block scale d is the block's last two bytes
+        d = (fd << 10) | ((by[:, :, 108] | (by[:, :, 109] << 8)) & 0x3FF)
+        by[:, :, 108], by[:, :, 109] = d & 0xFF, d >> 8
+        return by.reshape(rows, rb).to(torch.uint8)
     d = (fd << 10) | ((by[:, :, 0] | (by[:, :, 1] << 8)) & 0x3FF)
     m = (fm << 10) | ((by[:, :, 2] | (by[:, :, 3] << 8)) & 0x3FF)
     if fmt == Q5_1:

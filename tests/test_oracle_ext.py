@@ -17,7 +17,7 @@ from quantized_latent_moe_b200 import synth
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
 EPS32 = 2.0 ** -24
-FMTS = {"q5_1": 7, "q4_k": 12, "q5_k": 13}
+FMTS = {"q5_1": 7, "q3_k": 11, "q4_k": 12, "q5_k": 13}
 
 
 def _fixture():
@@ -62,11 +62,33 @@ def _q51_expected(fx):
     return np.array(out)
 
 
+def _q3k_block(fx):
+    b = bytearray(range(32))                                       # hmask[l] = l
+    b += bytes(((3 * l + n) & 255) for n in range(2) for l in range(32))
+    b += bytes(fx["q3k_scales_bytes"])
+    b += struct.pack("<H", fx["q3k_d_bits"])
+    return np.frombuffer(bytes(b), np.uint8)
+
+
+def test_q3_k_worked_block(orc):
+    fx = _fixture()
+    blk = _q3k_block(fx)
+    assert blk.size == 110
+    vals = orc.dequantize_ext(orc.Q3_K, blk, 1, 256)[0]
+    for i, v in fx["q3k_spot"].items():
+        assert vals[int(i)] == v, i
+    # every value is 0.5 * scale(i / 16) * q with q in -4 .. 3 (the scale table by hand)
+    sc = np.repeat(np.array(fx["q3k_scale"], np.float64), 16)
+    q = vals / (0.5 * sc)
+    assert np.all(q == np.rint(q)) and q.min() >= -4 and q.max() <= 3
+
+
 def test_row_bytes_are_gguf_sizes(orc):
     assert orc.row_bytes(orc.Q5_1, 32) == 24
     assert orc.row_bytes(orc.Q4_K, 256) == 144
     assert orc.row_bytes(orc.Q5_K, 256) == 176
     assert orc.row_bytes(orc.Q4_K, 1792) == 7 * 144
+    assert orc.row_bytes(orc.Q3_K, 256) == 110
 
 
 def test_worked_blocks_decode(orc):
@@ -89,6 +111,13 @@ def _codes(name, row, K):
         lo = np.concatenate([b[:, 8:] & 15, b[:, 8:] >> 4], axis=1).astype(np.int64)
         bits = (qh[:, None] >> np.arange(32)[None, :]) & 1
         return (lo + 16 * bits).reshape(-1)
+    if name == "q3_k":
+        b = row.reshape(K // 256, 110).astype(np.int64)
+        i = np.arange(256)
+        n, j, l = i // 128, (i % 128) // 32, i % 32
+        low = (b[:, 32 + 32 * n + l] >> (2 * j)) & 3
+        high = (b[:, l] >> (4 * n + j)) & 1
+        return (low - 4 * (1 - high)).reshape(-1)
     bb = 176 if name == "q5_k" else 144
     b = row.reshape(K // 256, bb)
     qs = b[:, bb - 128:].reshape(-1, 4, 32).astype(np.int64)
@@ -99,7 +128,7 @@ def _codes(name, row, K):
     return q.reshape(-1)
 
 
-@pytest.mark.parametrize("name", ["q5_1", "q4_k", "q5_k"])
+@pytest.mark.parametrize("name", ["q5_1", "q3_k", "q4_k", "q5_k"])
 def test_block_sums_brute_force(orc, name):
     """isum and sumq are the exact integer sums of the codes with the
     activation codes (the min term's sum is the quantised one, not s / d)."""
@@ -110,13 +139,20 @@ def test_block_sums_brute_force(orc, name):
     rows = synth.ext_blocks(name, 3, fmt, 4, K).numpy()
     for n in range(4):
         qw_all = _codes(name, rows[n], K)
-        assert qw_all.min() >= 0 and qw_all.max() <= (15 if name == "q4_k" else 31)
+        lo, hi = {"q3_k": (-4, 3), "q4_k": (0, 15)}.get(name, (0, 31))
+        assert qw_all.min() >= lo and qw_all.max() <= hi
         a = _q81(orc, r, K)
         for kb in range(K // 32):
             isum, sumq, sd, sm = orc.block_ext(fmt, rows[n], kb, a[kb * 36:(kb + 1) * 36])
             qa = a[kb * 36 + 4:(kb + 1) * 36].view(np.int8).astype(np.int64)
+            qw = qw_all[kb * 32:(kb + 1) * 32]
+            if name == "q3_k":
+                # the two 16-value halves' sums (no min term)
+                assert isum == int((qw[:16] * qa[:16]).sum())
+                assert sumq == int((qw[16:] * qa[16:]).sum())
+                continue
             assert sumq == int(qa.sum())
-            assert isum == int((qw_all[kb * 32:(kb + 1) * 32] * qa).sum())
+            assert isum == int((qw * qa).sum())
     # the worked K block against an activation block of ones: sums per sub-block by hand
     a = orc.quantize(orc.Q8_1, np.full(256, 1.0, np.float32))       # every code 127
     kq = _kq_block(fx, False)
@@ -127,7 +163,8 @@ def test_block_sums_brute_force(orc, name):
 
 
 @pytest.mark.parametrize("name,N,K,T", [("q5_1", 3, 64, 1), ("q5_1", 5, 512, 2), ("q4_k", 4, 256, 1),
-                                        ("q4_k", 3, 1792, 2), ("q5_k", 4, 512, 3)])
+                                        ("q4_k", 3, 1792, 2), ("q5_k", 4, 512, 3), ("q3_k", 4, 256, 1),
+                                        ("q3_k", 3, 1792, 2)])
 def test_qmatmul_ext_vs_fp64(orc, name, N, K, T):
     fmt = FMTS[name]
     r = np.random.default_rng(N * K + T)
@@ -142,7 +179,7 @@ def test_qmatmul_ext_vs_fp64(orc, name, N, K, T):
     assert np.all(np.abs(Y - ref) <= gamma * (np.abs(Xd) @ np.abs(Wd).T) + 1e-30)
 
 
-@pytest.mark.parametrize("name", ["q5_1", "q4_k", "q5_k"])
+@pytest.mark.parametrize("name", ["q5_1", "q3_k", "q4_k", "q5_k"])
 def test_ext_layer_stages_vs_fp64(orc, name):
     wl = synth.Workload("ext_tiny", 12, 3, 512, 256, 8, 2, 256, synth.Q8_0, synth.F32, "normal", ex_fmt=name)
     fmt = FMTS[name]
