@@ -111,7 +111,7 @@ def build_layer(elq, synth, wl, li, dev, fused=False, batch=32):
         ly.act_gz = ly.act_gh = synth.NVFP4_ACT_GSCALE
     for e0 in range(0, wl.E, batch):
         n = min(batch, wl.E - e0)
-        if wl.expert_fmt in ("q5_1", "q4_k", "q5_k"):
+        if wl.expert_fmt in ("q5_1", "q3_k", "q4_k", "q5_k"):
             # pre-quantised GGUF blocks, packed into the arena
             bs = [synth.expert_blocks(wl, e, li) for e in range(e0, e0 + n)]
             ly.set_expert_blocks(e0, *(torch.stack([b[i] for b in bs]).to(dev) for i in range(3)))
@@ -186,7 +186,7 @@ def oracle_setup(wl, n_tokens, gen_device, tokens=None):
     import oracle
     from quantized_latent_moe_b200 import synth
     fmts = {"q8_0": oracle.Q8_0, "q4_0": oracle.Q4_0, "nvfp4": oracle.NVFP4, "q5_1": oracle.Q5_1,
-            "q4_k": oracle.Q4_K, "q5_k": oracle.Q5_K}
+            "q3_k": oracle.Q3_K, "q4_k": oracle.Q4_K, "q5_k": oracle.Q5_K}
 
     def g(t):
         return t.to("cpu").numpy()
@@ -204,7 +204,7 @@ def oracle_setup(wl, n_tokens, gen_device, tokens=None):
         need |= set(idx.reshape(-1).tolist())
     gate, up, down = [None] * wl.E, [None] * wl.E, [None] * wl.E
     for e in sorted(need):
-        if wl.expert_fmt in ("q5_1", "q4_k", "q5_k"):
+        if wl.expert_fmt in ("q5_1", "q3_k", "q4_k", "q5_k"):
             a, b, c = synth.expert_blocks(wl, e, 0)
         else:
             a, b, c = synth.expert_weights(wl, e, 0, device=gen_device)
@@ -631,7 +631,7 @@ def run_elq(args):
         blk = 34 if wl.fmt == "q8_0" else 18              # D and U blocks
         # expert bytes per 32 values as the kernels read them (GGUF sizes; the
         # K-quants' arena carries 20 B per 32 values: 16 codes + a scale word)
-        eblk = {"q8_0": 34, "q4_0": 18, "nvfp4": 18, "q5_1": 24, "q4_k": 20, "q5_k": 24}[wl.expert_fmt]
+        eblk = {"q8_0": 34, "q4_0": 18, "nvfp4": 18, "q5_1": 24, "q3_k": 20, "q4_k": 20, "q5_k": 24}[wl.expert_fmt]
         ablk = 18 if wl.expert_fmt == "nvfp4" else 36     # the experts' activation blocks
         nb_L, nb_H, nb_I = wl.L // 32, wl.H // 32, wl.I // 32
         gu_w = act * 2 * wl.I * nb_L * eblk

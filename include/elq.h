@@ -142,6 +142,7 @@ typedef enum {                  /* GGUF type ids */
     ELQ_Q8_0 = 8,
     ELQ_Q8_1 = 9,
     ELQ_Q5_1 = 7,
+    ELQ_Q3_K = 11,
     ELQ_Q4_K = 12,
     ELQ_Q5_K = 13,
     ELQ_BF16 = 30,

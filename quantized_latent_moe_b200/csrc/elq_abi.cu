@@ -99,12 +99,14 @@ inline elq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ELQ_OK 
 bool fmt_ok(int32_t f) { return f == ELQ_Q8_0 || f == ELQ_Q4_0; }
 // formats the arena holds (NVFP4 in the Q4_0 geometry: 16 code bytes and a
 // 16-bit scale word per row and block)
-bool ext_fmt(int32_t f) { return f == ELQ_Q5_1 || f == ELQ_Q4_K || f == ELQ_Q5_K; }
+bool ext_fmt(int32_t f) { return f == ELQ_Q5_1 || f == ELQ_Q3_K || f == ELQ_Q4_K || f == ELQ_Q5_K; }
 bool arena_fmt_ok(int32_t f) { return fmt_ok(f) || f == ELQ_NVFP4 || ext_fmt(f); }
 // codes per (tile, block): four slices' pieces (WSlice::kCodes each)
 int slab_bytes(int32_t f) { return f == ELQ_Q8_0 ? kQ80Slab : fmt_has_qh(f) ? 4 * 640 : kQ40Slab; }
 // k granularity of an arena matrix
-int arena_k_unit(int32_t f) { return f == ELQ_NVFP4 ? 64 : (f == ELQ_Q4_K || f == ELQ_Q5_K) ? 256 : 32; }
+int arena_k_unit(int32_t f) {
+    return f == ELQ_NVFP4 ? 64 : (f == ELQ_Q3_K || f == ELQ_Q4_K || f == ELQ_Q5_K) ? 256 : 32;
+}
 
 // expert: the matrix may also be NVFP4 (with a global scale per gs_rows
 // rows), Q5_1, Q4_K or Q5_K (a layer's expert matrices).
@@ -115,7 +117,8 @@ elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k, bool expert = 
     if (rows % kTileRows || k % 128) return ELQ_ERR_UNSUPPORTED;
     if (!w->q || !w->d) return ELQ_ERR_INVALID_ARG;
     if (!aligned(w->q, 256) || !aligned(w->d, 256)) return ELQ_ERR_ALIGNMENT;
-    if ((w->fmt == ELQ_Q4_K || w->fmt == ELQ_Q5_K) && k % 256) return ELQ_ERR_UNSUPPORTED;   // whole super-blocks
+    if ((w->fmt == ELQ_Q3_K || w->fmt == ELQ_Q4_K || w->fmt == ELQ_Q5_K) && k % 256)
+        return ELQ_ERR_UNSUPPORTED;   // whole super-blocks
     if (w->fmt == ELQ_NVFP4) {
         if (k % 256) return ELQ_ERR_UNSUPPORTED;   // whole 8-block chunks of 18-byte activation blocks
         if (!w->gs || w->gs_rows <= 0 || rows % w->gs_rows) return ELQ_ERR_INVALID_ARG;
@@ -383,6 +386,9 @@ cudaError_t launch_s(SArgs g, int fmt, int x_mode, int out_mode, const SPlan& p,
         case ELQ_Q5_1:
             return gu ? launch_s_t<kQ51, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
                       : launch_s_t<kQ51, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
+        case ELQ_Q3_K:
+            return gu ? launch_s_t<kQ3K, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
+                      : launch_s_t<kQ3K, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
         case ELQ_Q4_K:
             return gu ? launch_s_t<kQ4K, X_Q81_PAIR_TOKEN, OUT_SWIGLU>(g, p, s, pdl)
                       : launch_s_t<kQ4K, X_Q81_POSITION, OUT_F32_COMBINE>(g, p, s, pdl);
@@ -1290,6 +1296,8 @@ elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t 
     uint8_t* q8 = static_cast<uint8_t*>(q_out);
     if (fmt == ELQ_Q5_1)
         k_arena_pack_ext<kQ51><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
+    else if (fmt == ELQ_Q3_K)
+        k_arena_pack_ext<kQ3K><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
     else if (fmt == ELQ_Q4_K)
         k_arena_pack_ext<kQ4K><<<grid, 256, 0, s>>>(src, n_rows, k, q8, d32);
     else if (fmt == ELQ_Q5_K)

@@ -94,12 +94,15 @@ __device__ __forceinline__ void warp_quant_q8_1(float v, uint8_t* dst) {
 // ---- NVFP4: E2M1 codes under E4M3 micro-block scales ---------------------------
 
 constexpr int kNV = 100;           // format id of NVFP4 (ELQ_NVFP4)
-constexpr int kQ51 = 7, kQ4K = 12, kQ5K = 13;   // Q5_1, Q4_K, Q5_K (GGUF ids)
+constexpr int kQ51 = 7, kQ3K = 11, kQ4K = 12, kQ5K = 13;   // Q5_1, Q3_K, Q4_K, Q5_K (GGUF ids)
 
 // Formats whose arena scale word per (row, 32-value block) is 32 bits (two
-// 16-bit units): Q5_1 (fp16 d, fp16 m) and the K-quants (6-bit scale and
-// min, and the super-block's fp16 d or dmin in sub-blocks 0 and 1).
-__host__ __device__ constexpr bool fmt_ext(int fmt) { return fmt == kQ51 || fmt == kQ4K || fmt == kQ5K; }
+// 16-bit units): Q5_1 (fp16 d, fp16 m), Q4_K / Q5_K (6-bit scale and min,
+// and the super-block's fp16 d or dmin in sub-blocks 0 and 1), Q3_K (the two
+// 16-value halves' 6-bit scales, and d in sub-block 0).
+__host__ __device__ constexpr bool fmt_ext(int fmt) {
+    return fmt == kQ51 || fmt == kQ3K || fmt == kQ4K || fmt == kQ5K;
+}
 __host__ __device__ constexpr bool fmt_has_qh(int fmt) { return fmt == kQ51 || fmt == kQ5K; }
 __host__ __device__ constexpr int scale_units(int fmt) { return fmt_ext(fmt) ? 2 : 1; }
 

@@ -201,7 +201,26 @@ __global__ void __launch_bounds__(256) k_arena_pack_ext(const uint8_t* __restric
     constexpr int kPiece = fmt_has_qh(FMT) ? 640 : 512;
     uint8_t codes[32];
     uint32_t qh = 0, sw;
-    if (FMT == kQ51) {
+    if (FMT == kQ3K) {
+        // codes q in -4 .. 3 stored as q + 8 (Q4_0's offset); the halves' scales
+        const uint8_t* b = aos + (row * (nb / 8) + kb / 8) * 110;
+        const int j = kb % 8;
+        for (int l = 0; l < 32; ++l) {
+            const int i = 32 * j + l, n = i / 128, jj = (i % 128) / 32, ll = i % 32;
+            const int low = (b[32 + 32 * n + ll] >> (2 * jj)) & 3;
+            const int high = (b[ll] >> (4 * n + jj)) & 1;
+            codes[l] = (uint8_t)(low - (high ? 0 : 4) + 8);
+        }
+        uint32_t sc6[2];
+        for (int h = 0; h < 2; ++h) {
+            const int s = 2 * j + h;
+            const int low4 = s < 8 ? (b[96 + s] & 15) : (b[96 + s - 8] >> 4);
+            const int hi2 = (b[96 + 8 + s % 4] >> (2 * (s / 4))) & 3;
+            sc6[h] = (uint32_t)(low4 | (hi2 << 4));
+        }
+        const uint32_t hi = j == 0 ? ((uint32_t)b[108] | ((uint32_t)b[109] << 8)) : 0u;
+        sw = sc6[0] | (sc6[1] << 8) | (hi << 16);
+    } else if (FMT == kQ51) {
         const uint8_t* b = aos + (row * nb + kb) * 24;
         for (int i = 0; i < 16; ++i) {
             codes[i] = b[8 + i] & 15;

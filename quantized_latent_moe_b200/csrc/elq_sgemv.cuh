@@ -435,7 +435,7 @@ __device__ __forceinline__ void s_dots_ext(const SArgs& g, const SUnit& u, const
     float dk = 0.0f, dmk = 0.0f;
     if (FMT != kQ51) {
         dk = h2f((uint16_t)(sw[lane] >> 16));
-        dmk = h2f((uint16_t)(sw[32 + lane] >> 16));
+        if (FMT != kQ3K) dmk = h2f((uint16_t)(sw[32 + lane] >> 16));
     }
 #pragma unroll 1
     for (int t = 0; t < nt; ++t) {
@@ -465,6 +465,14 @@ __device__ __forceinline__ void s_dots_ext(const SArgs& g, const SUnit& u, const
                             lo |= spread4_to_bit4((qh >> (4 * j)) & 15u);
                             hi |= spread4_to_bit4((qh >> (16 + 4 * j)) & 15u);
                         }
+                        if (FMT == kQ3K) {
+                            // q + 8 -> q (signed bytes, no borrow between bytes); the halves' sums
+                            lo = ((lo | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
+                            hi = ((hi | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
+                            isum[i] = __dp4a((int)lo, (int)aw[1 + j], isum[i]);
+                            sumq[i] = __dp4a((int)hi, (int)aw[5 + j], sumq[i]);
+                            continue;
+                        }
                         isum[i] = __dp4a((int)lo, (int)aw[1 + j], isum[i]);
                         isum[i] = __dp4a((int)hi, (int)aw[5 + j], isum[i]);
                         sumq[i] = __dp4a(0x01010101, (int)aw[1 + j], sumq[i]);
@@ -472,7 +480,11 @@ __device__ __forceinline__ void s_dots_ext(const SArgs& g, const SUnit& u, const
                     }
                     const float da = h2f((uint16_t)(aw[0] & 0xffff));
                     const uint32_t w = sw[kb * 32 + lane];
-                    if (FMT == kQ51) {
+                    if (FMT == kQ3K) {
+                        // Q3_K: (isum, sd) for values 0..15, (sumq, sm) for 16..31 (no min term)
+                        sd[i] = __fmul_rn(__fmul_rn(dk, (float)((int)(w & 0xff) - 32)), da);
+                        sm[i] = __fmul_rn(__fmul_rn(dk, (float)((int)((w >> 8) & 0xff) - 32)), da);
+                    } else if (FMT == kQ51) {
                         sd[i] = __fmul_rn(h2f((uint16_t)(w & 0xffff)), da);
                         sm[i] = __fmul_rn(h2f((uint16_t)(w >> 16)), da);
                     } else {

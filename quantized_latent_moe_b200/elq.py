@@ -15,12 +15,12 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libelq.so")
 
-F32, Q4_0, Q5_1, Q8_0, Q8_1, Q4_K, Q5_K, BF16, NVFP4 = 0, 2, 7, 8, 9, 12, 13, 30, 100
+F32, Q4_0, Q5_1, Q8_0, Q8_1, Q3_K, Q4_K, Q5_K, BF16, NVFP4 = 0, 2, 7, 8, 9, 11, 12, 13, 30, 100
 LAYER_FUSED = 1            # elq_layer.flags: small T as one persistent kernel
-FMT = {"q8_0": Q8_0, "q4_0": Q4_0, "nvfp4": NVFP4, "q5_1": Q5_1, "q4_k": Q4_K, "q5_k": Q5_K}
-SLAB = {Q8_0: 4096, Q4_0: 2048, NVFP4: 2048, Q5_1: 2560, Q4_K: 2048, Q5_K: 2560}   # code bytes per (tile, block)
-SCALE_SLAB = {NVFP4: 512, Q5_1: 512, Q4_K: 512, Q5_K: 512}                       # scale bytes per (tile, block)
-EXT = (Q5_1, Q4_K, Q5_K)
+FMT = {"q8_0": Q8_0, "q4_0": Q4_0, "nvfp4": NVFP4, "q5_1": Q5_1, "q3_k": Q3_K, "q4_k": Q4_K, "q5_k": Q5_K}
+SLAB = {Q8_0: 4096, Q4_0: 2048, NVFP4: 2048, Q5_1: 2560, Q3_K: 2048, Q4_K: 2048, Q5_K: 2560}   # code bytes per (tile, block)
+SCALE_SLAB = {NVFP4: 512, Q5_1: 512, Q3_K: 512, Q4_K: 512, Q5_K: 512}                       # scale bytes per (tile, block)
+EXT = (Q5_1, Q3_K, Q4_K, Q5_K)
 
 
 class ElqError(RuntimeError):

@@ -208,6 +208,8 @@ WORKLOADS = {
                               ex_fmt=NVFP4),
     # decode with Q4_K latent experts (D/U Q8_0): the decode shapes
     "decode_q4_k": Workload("decode_q4_k", 7, 1, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal", ex_fmt="q4_k"),
+    # decode with Q3_K latent experts (D/U Q8_0): the decode shapes
+    "decode_q3_k": Workload("decode_q3_k", 8, 1, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal", ex_fmt="q3_k"),
     # resident stack: 48 layers, 32 sequences decoding one token per step
     "stack": Workload("stack", 4, 32, 4096, 1792, 128, 8, 1024, Q8_0, BF16, "normal",
                       layers=48, steps=64, residual=True),

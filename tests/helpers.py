@@ -6,8 +6,8 @@ import torch
 
 from quantized_latent_moe_b200 import synth
 
-ORC_FMT = {"q8_0": 8, "q4_0": 2, "nvfp4": 100, "q5_1": 7, "q4_k": 12, "q5_k": 13}
-EXT = ("q5_1", "q4_k", "q5_k")
+ORC_FMT = {"q8_0": 8, "q4_0": 2, "nvfp4": 100, "q5_1": 7, "q3_k": 11, "q4_k": 12, "q5_k": 13}
+EXT = ("q5_1", "q3_k", "q4_k", "q5_k")
 
 
 def nvfp4_globals(w: torch.Tensor) -> torch.Tensor:

@@ -1,8 +1,8 @@
-"""Parity of the Q5_1 / Q4_K / Q5_K expert path (through the C ABI) with the
-CPU oracle: the packed arena byte for byte against the layout the header
-states, and every intermediate and the output of layers with these experts
-bit-exact (both sides take the same per-block integer sums, the same fp32
-factor products and the same chunk order, R22-R24)."""
+"""Parity of the Q5_1 / Q3_K / Q4_K / Q5_K expert path (through the C ABI)
+with the CPU oracle: the packed arena byte for byte against the layout the
+header states, and every intermediate and the output of layers with these
+experts bit-exact (both sides take the same per-block integer sums, the same
+fp32 factor products and the same chunk order, R22-R25)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +11,7 @@ from quantized_latent_moe_b200 import synth
 from helpers import gpu_layer, oracle_forward, oracle_layer
 
 pytestmark = pytest.mark.gpu
-FMTS = ["q5_1", "q4_k", "q5_k"]
+FMTS = ["q5_1", "q3_k", "q4_k", "q5_k"]
 
 
 @pytest.fixture(scope="module")
@@ -35,7 +35,25 @@ def _expected_arena(name, blocks, n_rows, k):
         rb = blocks[row]
         t, sl, r = row // 128, (row % 128) // 32, row % 32
         for kb in range(nb):
-            if name == "q5_1":
+            if name == "q3_k":
+                b = rb[110 * (kb // 8):110 * (kb // 8) + 110].astype(np.int64)
+                j = kb % 8
+                codes = []
+                for l_ in range(32):
+                    i = 32 * j + l_
+                    n_, jj, ll = i // 128, (i % 128) // 32, i % 32
+                    low = (b[32 + 32 * n_ + ll] >> (2 * jj)) & 3
+                    high = (b[ll] >> (4 * n_ + jj)) & 1
+                    codes.append(int(low - (0 if high else 4) + 8))
+                sc6 = []
+                for h in range(2):
+                    s_ = 2 * j + h
+                    low4 = (b[96 + s_] & 15) if s_ < 8 else (b[96 + s_ - 8] >> 4)
+                    sc6.append(int(low4 | (((b[104 + s_ % 4] >> (2 * (s_ // 4))) & 3) << 4)))
+                hi = int(b[108]) | int(b[109]) << 8 if j == 0 else 0
+                sw = sc6[0] | sc6[1] << 8 | hi << 16
+                qh = 0
+            elif name == "q5_1":
                 b = rb[24 * kb:24 * kb + 24]
                 codes = [b[8 + i] & 15 for i in range(16)] + [b[8 + i] >> 4 for i in range(16)]
                 qh = int(struct.unpack("<I", bytes(b[4:8]))[0])
@@ -113,11 +131,12 @@ def test_ext_experts_grouped_exact(E, orc, name):
     assert np.array_equal(y_lat, tr["y_lat"])
 
 
-@pytest.mark.parametrize("T", [1, 8])
-def test_q4_k_decode_full_size(E, orc, T):
+@pytest.mark.parametrize("name,T", [("decode_q4_k", 1), ("decode_q4_k", 8), ("decode_q3_k", 1), ("decode_q3_k", 8)])
+def test_kquant_decode_full_size(E, orc, name, T):
     """The decode shapes (128 experts, top-8, L = 1792 = 7 super-blocks, I =
-    1024) with Q4_K experts: the whole output equals the oracle's."""
-    wl = synth.WORKLOADS["decode_q4_k"]
+    1024) with Q4_K and with Q3_K experts: the whole output equals the
+    oracle's."""
+    wl = synth.WORKLOADS[name]
     ly = gpu_layer(wl)
     x = synth.make_x(wl, T=T)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
