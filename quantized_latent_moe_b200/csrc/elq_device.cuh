@@ -230,6 +230,20 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about hint_ns pass, instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for an mbarrier phase: gives up after budget_ns of wall time
 // (and a hard cap on polls), records kErrTimeout in *err and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
@@ -237,8 +251,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 0; i < (1u << 26); ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 255 && global_timer_ns() - t0 > budget_ns) break;
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+        if ((i & 15) == 15 && global_timer_ns() - t0 > budget_ns) break;
     }
     if (err) atomicExch(err, kErrTimeout);
     return false;

@@ -165,7 +165,8 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 
 // Exact int32 -> fp32 for |s| < 2^22 without the (slow) conversion unit: the
 // integer s + 0x4B400000 is the bit pattern of the float 1.5 * 2^23 + s, so
-// one fp32 subtraction of 1.5 * 2^23 recovers s exactly.
+// one fp32 subtraction of 1.5 * 2^23 recovers s exactly.  Each block's MMA
+// writes a fresh int32 accumulator; the epilogue adds the seed as it reads it.
 constexpr uint32_t kAccSeed = 0x4B400000u;
 constexpr float kAccSeedF = 12582912.0f;
 
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
 
 // ---- the GEMM ------------------------------------------------------------------
 
-constexpr int kTcKS = 4;            // blocks per pipeline stage
+constexpr int kTcKS = 4;            // blocks per pipeline stage (and per accumulator group)
 constexpr int kTcTileRowsPad = 129; // padded row count of the SwiGLU transpose (no bank conflicts)
 constexpr int kTcStages = 6;
 constexpr int kTcBufs = 8;          // TMEM accumulators of kTcN columns (all 512 columns), two groups of kTcKS
@@ -522,17 +523,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_sm;
-    if (warp >= 2) {
-        // every accumulator starts at the seed: an MMA then leaves seed + isum,
-        // the bit pattern of the float 1.5 * 2^23 + isum (see kAccSeed)
-        const uint32_t tb = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(((warp - 2) >> 2) * kTcEpiCols);
-#pragma unroll
-        for (int b = 0; b < kTcBufs; ++b) tmem_st16_const(tb + (uint32_t)(b * kTcN), kAccSeed);
-        tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     pdl_wait();
 
     const int n_units = tc_units(g);
@@ -595,7 +585,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     for (int kl = 0; kl < kTcKS; ++kl) {
                         const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
                         const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
-                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 1u);
+                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 0u);
                     }
                     umma_commit(&tfull[gr]);
                     umma_commit(&empty[s]);
@@ -638,7 +628,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                 const uint16_t* dws = reinterpret_cast<const uint16_t*>(st + kTcStageA);
                 const float* das = reinterpret_cast<const float*>(st + kTcStageA + kTcStageDw + kTcStageB);
                 const uint32_t tb = tmem + tlane + (uint32_t)(gr * kTcKS * kTcN + c0);
-                // column groups past the tile's tokens hold no MMA result (and keep the seed)
+                // column groups past the tile's tokens hold no MMA result
                 if (active) {
 #pragma unroll
                     for (int kp = 0; kp < kTcKS; kp += 2) {
@@ -657,22 +647,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 #pragma unroll
                             for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
                                 const float4 dv = dak[j4];
-                                const uint64_t i0 = f2_sub(
-                                    f2_pack(__uint_as_float(rc[h][4 * j4]), __uint_as_float(rc[h][4 * j4 + 1])), seed2);
-                                const uint64_t i1 = f2_sub(
-                                    f2_pack(__uint_as_float(rc[h][4 * j4 + 2]), __uint_as_float(rc[h][4 * j4 + 3])), seed2);
+                                const uint64_t i0 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4] + kAccSeed),
+                                                                   __uint_as_float(rc[h][4 * j4 + 1] + kAccSeed)),
+                                                           seed2);
+                                const uint64_t i1 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4 + 2] + kAccSeed),
+                                                                   __uint_as_float(rc[h][4 * j4 + 3] + kAccSeed)),
+                                                           seed2);
                                 part2[2 * j4] = f2_fma(i0, f2_mul(dw2, f2_pack(dv.x, dv.y)), part2[2 * j4]);
                                 part2[2 * j4 + 1] = f2_fma(i1, f2_mul(dw2, f2_pack(dv.z, dv.w)), part2[2 * j4 + 1]);
                             }
                         }
                     }
-                    // the group's accumulators back to the seed for its next MMAs
-#pragma unroll
-                    for (int kl = 0; kl < kTcKS; ++kl) tmem_st16_const(tb + (uint32_t)(kl * kTcN), kAccSeed);
-                    tmem_st_wait();
                 }
-                // a run of 8 blocks ends with every second stage (and with the last)
-                if ((ks & 1) || ks == kstages - 1) {
+                // a run of 8 blocks ends with every (8 / kTcKS)-th stage (and with the last)
+                if ((ks + 1) % (kChunk / kTcKS) == 0 || ks == kstages - 1) {
 #pragma unroll
                     for (int j = 0; j < kTcEpiCols / 2; ++j) {
                         acc2[j] = f2_add(acc2[j], part2[j]);
