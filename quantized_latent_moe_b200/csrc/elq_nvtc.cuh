@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[ab]);
+            mbar_arrive_lane0(&tempty[ab], lane);
             const float gq = __fmul_rn(__ldg(g.wgs + un.e), g.ags);
 #pragma unroll
             for (int j = 0; j < kNvEpiCols; ++j) acc[j] = __fmul_rn(acc[j], gq);
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < kNvEpiCols; ++j) xchg[(c0 + j) * kNvXld + row] = acc[j];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(xfull);
+                mbar_arrive_lane0(xfull, lane);
                 if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
                     *abort_v = 1;
                     break;
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(xempty);
+                mbar_arrive_lane0(xempty, lane);
                 ++xc;
                 continue;
             }

@@ -60,6 +60,14 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
+// One arrival for the warp, by lane 0, as a predicated instruction (no branch).
+__device__ __forceinline__ void mbar_arrive_lane0(uint64_t* bar, int lane) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.s32 p, %1, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(
+            smem_addr(bar)),
+        "r"(lane)
+        : "memory");
+}
 
 // Tiled tensor copies global -> shared through a tensor map (a kernel
 // parameter), completing on an mbarrier's transaction count.  No multicast.
@@ -170,12 +178,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 constexpr uint32_t kAccSeed = 0x4B400000u;
 constexpr float kAccSeedF = 12582912.0f;
 
-// Bounded mbarrier wait taken by lane 0 for the whole warp (the result is the
-// same in every lane, so warp-collective instructions after it stay converged).
+// Bounded mbarrier wait of a whole warp: every lane polls (no divergent
+// branch around the poll loop) and the warp agrees on the outcome, so
+// warp-collective instructions after it stay converged.
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity, int* err, uint64_t budget_ns) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, err, budget_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, err, budget_ns) ? 1 : 0) != 0;
 }
 
 // Shared-memory matrix descriptor: K-major, no swizzle, version 1.
@@ -604,6 +611,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
         const int c0 = (ew >> 2) * kTcEpiCols;   // its accumulator columns (tokens) c0 .. c0+15
         const int row = sp * 32 + lane;       // weight row within the tile
         int it = 0, xc = 0;
+        int s = 0;                            // it % kTcStages and the parity of it / kTcStages
+        uint32_t sph = 0;
         for (int u = u0; u < u1 && !*abort_v; ++u) {
             const TcUnit un = unit_at(u);
             if (!un.valid) continue;
@@ -616,10 +625,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
             const uint32_t tlane = (uint32_t)(sp * 32) << 16;
             const uint64_t seed2 = f2_pack(kAccSeedF, kAccSeedF);
             for (int ks = 0; ks < kstages; ++ks, ++it) {
-                const int s = it % kTcStages, gr = it % kTcGroups;
+                const int gr = it % kTcGroups;
                 const uint8_t* st = stages + s * kTcStage;
                 // the stage's scales (bulk copies) and its accumulators (MMAs)
-                if (!warp_wait_bounded(&full[s], (uint32_t)((it / kTcStages) & 1), g.err, g.budget_ns) ||
+                if (!warp_wait_bounded(&full[s], sph, g.err, g.budget_ns) ||
                     !warp_wait_bounded(&tfull[gr], (uint32_t)((it / kTcGroups) & 1), g.err, g.budget_ns)) {
                     ok = false;
                     break;
@@ -669,9 +678,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&tempty[gr]);
-                    mbar_arrive(&empty[s]);
+                mbar_arrive_lane0(&tempty[gr], lane);
+                mbar_arrive_lane0(&empty[s], lane);
+                if (++s == kTcStages) {
+                    s = 0;
+                    sph ^= 1u;
                 }
             }
             float acc[kTcEpiCols];
@@ -695,7 +706,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < kTcEpiCols; ++j) xchg[(c0 + j) * kTcXld + row] = acc[j];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(xfull);
+                mbar_arrive_lane0(xfull, lane);
                 if (!warp_wait_bounded(xfull, (uint32_t)(xc & 1), g.err, g.budget_ns)) {
                     *abort_v = 1;
                     break;
@@ -744,7 +755,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(xempty);
+                mbar_arrive_lane0(xempty, lane);
                 ++xc;
                 continue;
             }
