@@ -56,7 +56,7 @@ cudaError_t smem_optin(K kern, int bytes, bool* done_per_dev) {
     return e;
 }
 
-bool g_optin_router[kMaxDevices], g_optin_bucket[kMaxDevices],
+bool g_optin_router[kMaxDevices], g_optin_router2[kMaxDevices], g_optin_bucket[kMaxDevices],
     g_optin_topk[kMaxDevices], g_optin_dec[4][kMaxDevices];
 
 // Cooperative launch: every CTA of the grid is resident at once.
@@ -823,19 +823,22 @@ elq_status check_layer(const elq_layer* ly, int32_t T) {
     return ELQ_OK;
 }
 
-// Router launch shape: 4 experts per CTA and one token block each while that
-// grid stays within two CTAs per SM; beyond, 16 experts per CTA and about one
-// CTA per SM, each streaming several token blocks.
+// Router launch shape: 4 experts per CTA (one per warp) and one token block
+// each while that grid stays within two CTAs per SM; beyond, 16 experts per
+// CTA (8 warps of two) and about one CTA per SM, each streaming several token
+// blocks.
 struct RouterShape {
-    int nw, gx, gy, stages;
+    int nw, epw, gx, gy, stages;
 };
 
 RouterShape router_shape(int T, int E) {
     RouterShape r;
     const int rblocks = (T + kRouterTok - 1) / kRouterTok;
     const int sms = sm_count();
-    r.nw = ((int64_t)rblocks * ((E + 3) / 4) <= 2 * (int64_t)sms) ? 4 : kRouterMaxWarps;
-    r.gx = (E + r.nw - 1) / r.nw;
+    const bool small = (int64_t)rblocks * ((E + 3) / 4) <= 2 * (int64_t)sms;
+    r.nw = small ? 4 : kRouterMaxWarps / 2;
+    r.epw = small ? 1 : 2;
+    r.gx = (E + r.nw * r.epw - 1) / (r.nw * r.epw);
     r.gy = r.nw == 4 ? rblocks : std::min(rblocks, std::max(1, sms / r.gx));
     r.stages = r.gy < rblocks ? 2 : 1;
     return r;
@@ -843,7 +846,8 @@ RouterShape router_shape(int T, int E) {
 
 size_t router_smem(int T, int L, int E) {
     const RouterShape r = router_shape(T, E);
-    return (size_t)r.stages * std::min(T, kRouterTok) * L * 4 + (size_t)r.nw * E * 4;
+    const int Lp = (L + 255) & ~255;   // the kernel's padded row stride
+    return (size_t)r.stages * std::min(T, kRouterTok) * Lp * 4 + (size_t)r.nw * E * 4;
 }
 
 bool router_shape_ok(int T, int L, int E) {
@@ -863,10 +867,15 @@ cudaError_t launch_router(const float* z, const float* w, const float* bias, int
     a.cnt_all = cnt ? cnt + rblocks : nullptr;
     a.do_bucket = do_bucket ? 1 : 0;
     a.counts = counts; a.offsets = offsets; a.perm = perm; a.pos = pos; a.act = act; a.n_act = n_act;
-    cudaError_t e = smem_optin(k_router, kRouterSmemMax, g_optin_router);
-    if (e != cudaSuccess) return e;
     const RouterShape r = router_shape(T, E);
-    return launch(k_router, dim3(r.gx, r.gy), dim3(r.nw * 32), router_smem(T, L, E), s, pdl, a);
+    if (r.epw == 2) {
+        cudaError_t e = smem_optin(k_router<2>, kRouterSmemMax, g_optin_router2);
+        if (e != cudaSuccess) return e;
+        return launch(k_router<2>, dim3(r.gx, r.gy), dim3(r.nw * 32), router_smem(T, L, E), s, pdl, a);
+    }
+    cudaError_t e = smem_optin(k_router<1>, kRouterSmemMax, g_optin_router);
+    if (e != cudaSuccess) return e;
+    return launch(k_router<1>, dim3(r.gx, r.gy), dim3(r.nw * 32), router_smem(T, L, E), s, pdl, a);
 }
 
 // Grouped gate/up over the routed pairs: SwiGLU epilogue into hq.

@@ -508,7 +508,38 @@ __device__ void bucket_warp_small(const int32_t* idx_sm, int P, int E, int32_t* 
     }
 }
 
-__global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
+// Warp sums of V values per lane (V a power of two, at most 32), each the same
+// xor-butterfly tree as V separate butterflies over offsets 16, 8, 4, 2, 1
+// (every level adds the two lanes' partials of the same value), but at each
+// of the first log2(V) levels a lane keeps only half of its values and trades
+// the other half with its partner: V - 1 + 5 - log2(V) shuffles instead of
+// 5 V.  On return lane l holds the total of value l >> (5 - log2(V)).
+template <int V>
+__device__ __forceinline__ float warp_sum_scatter(float (&p)[V], int lane) {
+    constexpr int LV = V >= 32 ? 5 : V >= 16 ? 4 : V >= 8 ? 3 : V >= 4 ? 2 : V >= 2 ? 1 : 0;
+    static_assert((1 << LV) == V, "V is a power of two <= 32");
+#pragma unroll
+    for (int st = 0; st < LV; ++st) {
+        const int o = 16 >> st, h = (V >> st) / 2;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = up ? p[i] : p[i + h];
+            const float keep = up ? p[i + h] : p[i];
+            p[i] = __fadd_rn(keep, __shfl_xor_sync(kFull, send, o));
+        }
+    }
+    float r = p[0];
+#pragma unroll
+    for (int o = 16 >> LV; o >= 1; o >>= 1) r = __fadd_rn(r, __shfl_xor_sync(kFull, r, o));
+    return r;
+}
+
+// EPW experts per warp (1 or 2): with 2, each latent value a lane reads from
+// shared memory feeds two experts' chains (half the shared-memory traffic per
+// logit, the bound of this loop), at twice the register-held weights.
+template <int EPW>
+__global__ void __launch_bounds__(EPW == 1 ? kRouterMaxWarps * 32 : kRouterMaxWarps * 16) k_router(RouterArgs a) {
     extern __shared__ __align__(128) float rsm[];   // [stages][<=8][L] latent rows, then [nw][E] scratch
     __shared__ int s_last, s_all;
     __shared__ int32_t s_idx[64];
@@ -522,31 +553,49 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
     const int nmine = (rblocks - (int)blockIdx.y + gy - 1) / gy;   // >= 1: gridDim.y <= rblocks
     const int stages = (gy < rblocks) ? 2 : 1;
     const int rows = min(a.T, kRouterTok);
-    float* scr = rsm + (size_t)stages * rows * L;
-    const int e = (int)blockIdx.x * nw + warp;
-    const bool has_e = e < E;
+    const int Lp = (L + 255) & ~255;                // shared row stride: whole chunks of 8 lane-strided values
+    float* scr = rsm + (size_t)stages * rows * Lp;
+    const int e0 = ((int)blockIdx.x * nw + warp) * EPW;   // this warp's experts e0 .. e0 + EPW - 1
+    const bool has_e = e0 < E;
     // the router rows do not depend on the upstream kernel: load them first
-    float wr[kRouterJ];
-    {
-        const float* wrow = a.w + (int64_t)(has_e ? e : 0) * L + lane;
+    float wr[EPW][kRouterJ];
+    float bias[EPW];
 #pragma unroll
-        for (int j = 0; j < kRouterJ; ++j) wr[j] = (has_e && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
+    for (int x = 0; x < EPW; ++x) {
+        const bool on = e0 + x < E;
+        const float* wrow = a.w + (int64_t)(on ? e0 + x : 0) * L + lane;
+#pragma unroll
+        for (int j = 0; j < kRouterJ; ++j) wr[x][j] = (on && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
+        bias[x] = (on && a.bias) ? __ldg(a.bias + e0 + x) : 0.0f;
     }
-    const float bias = (has_e && a.bias) ? __ldg(a.bias + e) : 0.0f;
     pdl_wait();
     pdl_trigger();
     // token block number i of this CTA into stage i % stages: one cp.async
     // group per block (an empty group past the last block keeps the count)
+    const int L4 = L >> 2;
     auto issue = [&](int i) {
         if (i < nmine) {
             const int t0 = ((int)blockIdx.y + i * gy) * kRouterTok;
-            const int n16 = min(kRouterTok, a.T - t0) * (L >> 2);
+            const int nr = min(kRouterTok, a.T - t0);
             const float* src = a.z + (int64_t)t0 * L;
-            float* dst = rsm + (size_t)(i & (stages - 1)) * rows * L;
-            for (int c = threadIdx.x; c < n16; c += blockDim.x) cp_async16(dst + 4 * c, src + 4 * c);
+            float* dst = rsm + (size_t)(i & (stages - 1)) * rows * Lp;
+            int r = (int)threadIdx.x / L4, c = (int)threadIdx.x - r * L4;
+            while (r < nr) {
+                cp_async16(dst + r * Lp + 4 * c, src + (int64_t)r * L + 4 * c);
+                c += (int)blockDim.x;
+                while (c >= L4) {
+                    c -= L4;
+                    ++r;
+                }
+            }
         }
         cp_async_commit();
     };
+    // the padding columns L .. Lp of every staged row are zeros (never copied into): a zero weight times
+    // a zero adds +0 to a chain that, started at +0, is never -0, so it leaves the chain's bits alone
+    if (Lp > L)
+        for (int q = threadIdx.x; q < stages * rows * (Lp - L); q += blockDim.x)
+            rsm[(q / (Lp - L)) * Lp + L + q % (Lp - L)] = 0.0f;
     issue(0);
     if (stages == 2) issue(1);
     const bool small = a.do_bucket && rblocks == 1 && a.T * a.k <= 64;
@@ -600,31 +649,46 @@ __global__ void __launch_bounds__(kRouterMaxWarps * 32) k_router(RouterArgs a) {
             cp_async_wait<0>();
         __syncthreads();
         if (has_e) {
-            const float* zs = rsm + (size_t)(i & (stages - 1)) * rows * L + lane;
-            for (int tt = 0; tt < nt; tt += 2) {
-                const float* z0 = zs + tt * L;
-                const float* z1 = zs + min(tt + 1, nt - 1) * L;
-                float p0 = 0.0f, p1 = 0.0f;
+            // four tokens by EPW experts per pass; lane l keeps the chains of the lane-strided
+            // values 32 j + l (R9), j in whole chunks of 8 (the rows are padded to 256)
+            constexpr int kTq = 4, kV = kTq * EPW;
+            const float* zs = rsm + (size_t)(i & (stages - 1)) * rows * Lp + lane;
+            const int nc = Lp >> 8;
+            for (int tt = 0; tt < nt; tt += kTq) {
+                const float* zr[kTq];
 #pragma unroll
-                for (int j = 0; j < kRouterJ; ++j) {
-                    if (j < nj) {
-                        p0 = __fmaf_rn(z0[32 * j], wr[j], p0);
-                        p1 = __fmaf_rn(z1[32 * j], wr[j], p1);
+                for (int q = 0; q < kTq; ++q) zr[q] = zs + min(tt + q, nt - 1) * Lp;
+                float p[kV];
+#pragma unroll
+                for (int v = 0; v < kV; ++v) p[v] = 0.0f;
+#pragma unroll
+                for (int c = 0; c < kRouterJ / 8; ++c) {
+                    if (c < nc) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int j = 8 * c + u;
+                            float zv[kTq];
+#pragma unroll
+                            for (int q = 0; q < kTq; ++q) zv[q] = zr[q][32 * j];
+#pragma unroll
+                            for (int q = 0; q < kTq; ++q)
+#pragma unroll
+                                for (int x = 0; x < EPW; ++x)
+                                    p[q * EPW + x] = __fmaf_rn(zv[q], wr[x][j], p[q * EPW + x]);
+                        }
                     }
                 }
+                // value v = q * EPW + x: token tt + q, expert e0 + x
+                float r = warp_sum_scatter<kV>(p, lane);
+                constexpr int kSh = 5 - (kV >= 32 ? 5 : kV >= 16 ? 4 : kV >= 8 ? 3 : kV >= 4 ? 2 : kV >= 2 ? 1 : 0);
+                const int v = lane >> kSh, q = v / EPW, x = v - q * EPW;
+                float bx = bias[0];
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    p0 = __fadd_rn(p0, __shfl_xor_sync(kFull, p0, o));
-                    p1 = __fadd_rn(p1, __shfl_xor_sync(kFull, p1, o));
-                }
-                if (a.bias) {
-                    p0 = __fadd_rn(p0, bias);
-                    p1 = __fadd_rn(p1, bias);
-                }
-                if (lane == 0) {
-                    a.logits[(int64_t)(t0 + tt) * E + e] = p0;
-                    if (tt + 1 < nt) a.logits[(int64_t)(t0 + tt + 1) * E + e] = p1;
-                }
+                for (int xx = 1; xx < EPW; ++xx)
+                    if (x == xx) bx = bias[xx];
+                if (a.bias) r = __fadd_rn(r, bx);
+                if ((lane & ((1 << kSh) - 1)) == 0 && tt + q < nt && e0 + x < E)
+                    a.logits[(int64_t)(t0 + tt + q) * E + e0 + x] = r;
             }
         }
         __syncthreads();                       // the stage is consumed: refill it

@@ -125,7 +125,8 @@ def test_latent_proj_exact(E, orc, fmt, N, K, T):
 
 @pytest.mark.parametrize("T,L,E_,k,bias", [(1, 1792, 128, 8, True), (6, 1280, 128, 8, False),
                                             (37, 256, 8, 2, False), (5, 64, 33, 32, True),
-                                            (300, 256, 128, 8, True), (2000, 64, 33, 32, True)])
+                                            (300, 256, 128, 8, True), (2000, 64, 33, 32, True),
+                                            (2048, 1792, 128, 8, True)])
 def test_router_exact(E, orc, T, L, E_, k, bias):
     z = _gen(7, T, (T, L), 1.3)
     W = _gen(7, 100 + L, (E_, L), 0.02)
