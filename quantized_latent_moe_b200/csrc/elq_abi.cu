@@ -485,7 +485,7 @@ ProjWs proj_layout(const elq_qmat* w, int T, void* base, bool allow_tc = true) {
 bool g_optin_tc[kMaxDevices];
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s, bool pdl) {
-    const int64_t n = (a.mode == PACK_DENSE ? a.bstride : (int64_t)a.P) * a.nb;
+    const int64_t n = a.bstride * a.nb;   // one thread per (block, slot)
     return launch(k_pack_b, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, a);
 }
 
@@ -1101,9 +1101,11 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     std::memset(&pa, 0, sizeof(pa));
     pa.x = zq;
     pa.nb = L / 32;
-    pa.mode = PACK_PAIRS;
-    pa.pair_slot = w.pair_slot;
-    pa.P = P;
+    pa.mode = PACK_SLOTS;
+    pa.slot_off = w.slot_off;
+    pa.offsets = w.offsets;
+    pa.perm = w.perm;
+    pa.E = E;
     pa.kslots = k;
     pa.bq = w.bzq;
     pa.bd = w.bzd;
@@ -1145,8 +1147,9 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
-    const int64_t warps = (int64_t)T * (L / 32);   // one thread per (token, block)
-    if (launch(k_tc_combine, dim3((unsigned)((warps + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+    const int64_t threads = (int64_t)T * ((L / 32 + 3) / 4) * 32;   // one warp per (token, 4 blocks)
+    if (launch(k_tc_combine, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess ||
+        !mark())
         return ELQ_ERR_CUDA;
     return ELQ_OK;
 }
@@ -1209,13 +1212,15 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     pk.x = zq;
     pk.nb = L / 32;
     pk.nks = L / 64;
-    pk.pair_slot = w.pair_slot;
-    pk.P = P;
+    pk.slot_off = w.slot_off;
+    pk.offsets = w.offsets;
+    pk.perm = w.perm;
+    pk.E = E;
     pk.kslots = k;
     pk.bq = w.bzq;
     pk.bsf = reinterpret_cast<uint8_t*>(w.bzd);
     pk.sstride = w.sstride;
-    const int64_t n = (int64_t)P * pk.nks;
+    const int64_t n = w.sstride * pk.nks;   // one thread per (K-step, slot)
     if (launch(k_pack_nv, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, pk) != cudaSuccess || !mark())
         return ELQ_ERR_CUDA;
     bool ok = false;
@@ -1235,8 +1240,9 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
-    const int64_t warps = (int64_t)T * (L / 32);   // one thread per (token, block)
-    if (launch(k_tc_combine, dim3((unsigned)((warps + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess || !mark())
+    const int64_t threads = (int64_t)T * ((L / 32 + 3) / 4) * 32;   // one warp per (token, 4 blocks)
+    if (launch(k_tc_combine, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess ||
+        !mark())
         return ELQ_ERR_CUDA;
     return ELQ_OK;
 }

@@ -151,32 +151,38 @@ __device__ __forceinline__ TcUnit tc_unit(const NvArgs& g, int u) {
 struct NvPackArgs {
     const uint8_t* x;           // NVFP4 rows, nb blocks each
     int nb, nks;
-    const int32_t* pair_slot;
-    int P, kslots;
+    const int32_t* slot_off;    // the slots of expert e: slot_off[e] .. slot_off[e+1]-1; from slot_off[E] on unused
+    const int32_t* offsets;     // its pairs: perm[offsets[e]] ..., row = pair / kslots; then zero slots
+    const int32_t* perm;
+    int E, kslots;
     uint8_t* bq;
     uint8_t* bsf;
     int64_t sstride;
 };
 
+// One thread per (K-step of 64, slot), slots fastest: the two 18-byte blocks
+// of the slot's row (zeros for padding) into its codes and scale atom.
 __global__ void __launch_bounds__(256) k_pack_nv(NvPackArgs a) {
+    __shared__ int s_off[1025];
     pdl_wait();
+    load_slot_off(s_off, a.slot_off, a.E);
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (id >= (int64_t)a.P * a.nks) return;
-    const int64_t p = id / a.nks;
-    const int ks = (int)(id % a.nks);
-    const int64_t slot = __ldcg(a.pair_slot + p);
-    const int64_t row = p / a.kslots;
+    if (id >= a.sstride * a.nks) return;
+    const int ks = (int)(id / a.sstride);
+    const int64_t slot = id - (int64_t)ks * a.sstride;
+    if (slot >= s_off[a.E]) return;
+    const int64_t row = slot_row_of(s_off, a.E, slot, a.offsets, a.perm, a.kslots);
     uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sw = 0;
-    {
+    if (row >= 0) {
         // two 18-byte blocks (2-byte aligned): scales, then 16 code bytes each
         const uint16_t* src = reinterpret_cast<const uint16_t*>(a.x + (row * a.nb + 2 * ks) * 18);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
             const uint16_t* sb = src + 9 * b;
-            sw |= (uint32_t)__ldcg(sb) << (16 * b);
+            sw |= (uint32_t)__ldg(sb) << (16 * b);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                c[4 * b + j] = (uint32_t)__ldcg(sb + 1 + 2 * j) | ((uint32_t)__ldcg(sb + 2 + 2 * j) << 16);
+                c[4 * b + j] = (uint32_t)__ldg(sb + 1 + 2 * j) | ((uint32_t)__ldg(sb + 2 + 2 * j) << 16);
         }
     }
     uint8_t* dst = a.bq + (int64_t)ks * a.sstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;

@@ -203,44 +203,76 @@ __host__ __device__ constexpr uint32_t umma_idesc_i8(int M, int N) {
 // bq + kb*bstride*32 + (s/8)*256 + (c/16)*128 + (s%8)*16 + c%16, its scale at
 // bd[kb*bstride + s].  Slots without a row hold zeros.
 
-enum { PACK_DENSE = 0, PACK_PAIRS = 1 };
+enum { PACK_DENSE = 0, PACK_SLOTS = 1 };
 
 struct PackArgs {
     const uint8_t* x;           // Q8_1 AoS rows, nb blocks each
     int nb;
     int mode;
     int T;                      // PACK_DENSE: rows 0 .. T-1 -> slots 0 .. T-1
-    // PACK_PAIRS: pair p (row p / k) goes to slot pair_slot[p]; padding slots
-    // are left as they are (the GEMM's columns past a tile's pairs are unused)
-    const int32_t* pair_slot;
-    int P, kslots;
+    // PACK_SLOTS: the slots of expert e are slot_off[e] .. slot_off[e+1]-1,
+    // its pairs (perm[offsets[e]] ..., row = pair / kslots) then zeros; slots
+    // from slot_off[E] on are past the routed tiles and stay as they are
+    const int32_t* slot_off;
+    const int32_t* offsets;
+    const int32_t* perm;
+    int E, kslots;
     uint8_t* bq;
     float* bd;
     int64_t bstride;            // slots in the buffer (multiple of 16)
 };
 
-// One thread per (slot, block) (dense), or per (pair, block).
+// Shared copy of slot_off[0 .. E] for slot_row_of (E <= 1024).
+__device__ __forceinline__ void load_slot_off(int* s_off, const int32_t* slot_off, int E) {
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = __ldcg(slot_off + i);
+    __syncthreads();
+}
+
+// The token row of the pair in slot `slot` (< slot_off[E]), or -1 for a
+// padding slot: the expert is the last e with slot_off[e] <= slot.
+__device__ __forceinline__ int64_t slot_row_of(const int* s_off, int E, int64_t slot, const int32_t* offsets,
+                                               const int32_t* perm, int kslots) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_off[mid] <= slot) lo = mid;
+        else hi = mid;
+    }
+    const int r = (int)(slot - s_off[lo]);
+    const int o0 = __ldg(offsets + lo), cnt = __ldg(offsets + lo + 1) - o0;
+    return r < cnt ? __ldg(perm + o0 + r) / kslots : -1;
+}
+
+// PACK_SLOTS: one thread per (block, slot), slots fastest: a warp writes 32
+// consecutive slots of one block (1 KB of codes and 128 B of scales,
+// contiguous) and reads its rows' 36-byte blocks through L1.  PACK_DENSE: one
+// thread per (slot, block), blocks fastest (a warp reads 32 consecutive blocks
+// of a row).
 __global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
+    __shared__ int s_off[1025];
     pdl_wait();
+    if (a.mode != PACK_DENSE) load_slot_off(s_off, a.slot_off, a.E);
     const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t n_items = a.mode == PACK_DENSE ? a.bstride : a.P;
-    if (id >= n_items * a.nb) return;
-    const int64_t item = id / a.nb;
-    const int kb = (int)(id % a.nb);
-    int64_t row = -1, slot = item;
+    if (id >= a.bstride * a.nb) return;
+    int kb;
+    int64_t slot, row;
     if (a.mode == PACK_DENSE) {
-        if (item < a.T) row = item;
+        slot = id / a.nb;
+        kb = (int)(id - slot * a.nb);
+        row = slot < a.T ? slot : -1;
     } else {
-        slot = __ldcg(a.pair_slot + item);
-        row = item / a.kslots;
+        kb = (int)(id / a.bstride);
+        slot = id - (int64_t)kb * a.bstride;
+        if (slot >= s_off[a.E]) return;
+        row = slot_row_of(s_off, a.E, slot, a.offsets, a.perm, a.kslots);
     }
     uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
     float dd = 0.0f;
     if (row >= 0) {
         const uint32_t* src = reinterpret_cast<const uint32_t*>(a.x + (row * a.nb + kb) * 36);
-        const uint32_t w0 = __ldcg(src);
-        lo4 = make_uint4(__ldcg(src + 1), __ldcg(src + 2), __ldcg(src + 3), __ldcg(src + 4));
-        hi4 = make_uint4(__ldcg(src + 5), __ldcg(src + 6), __ldcg(src + 7), __ldcg(src + 8));
+        const uint32_t w0 = __ldg(src);
+        lo4 = make_uint4(__ldg(src + 1), __ldg(src + 2), __ldg(src + 3), __ldg(src + 4));
+        hi4 = make_uint4(__ldg(src + 5), __ldg(src + 6), __ldg(src + 7), __ldg(src + 8));
         dd = h2f((uint16_t)(w0 & 0xffff));
     }
     uint8_t* dst = a.bq + (int64_t)kb * a.bstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
@@ -834,9 +866,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 
 // ---- a9 on the tensor-core path: the weighted combine --------------------------
 //
-// One thread per (token, 32-row latent block), its 32 rows in registers:
-// y_lat = fmaf(w_j, o_j, y_lat) over the token's k pairs in rank order (o
-// read by the pair's slot, 128 contiguous bytes a pair), then its Q8_1 block,
+// One warp per (token, 4 consecutive 32-row latent blocks): lane l keeps the 4
+// rows 4 (l % 8) .. +3 of block l / 8, so each read of a pair's o row is 512
+// contiguous bytes for the warp.  Every row is y_lat = fmaf(w_j, o_j, y_lat)
+// over the token's k pairs in rank order (o read by the pair's slot), then
+// the Q8_1 block of each 8-lane group (amax and code sum by three shuffles),
 // written both row-major (ylq) and into the packed buffer the U projection
 // reads (slot = token).
 struct CombArgs {
@@ -854,52 +888,56 @@ struct CombArgs {
 __global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
     pdl_wait();
     pdl_trigger();
-    const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int nbl = a.L / 32;
-    if (id >= (int64_t)a.T * nbl) return;
-    const int t = (int)(id / nbl), blk = (int)(id - (int64_t)t * nbl);
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+    const int lane = threadIdx.x & 31;
+    const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nbl = a.L / 32, nch = (nbl + 3) / 4;
+    if (task >= (int64_t)a.T * nch) return;          // whole warps
+    const int t = (int)(task / nch), c = (int)(task - (int64_t)t * nch);
+    const int blk = 4 * c + (lane >> 3), m = lane & 7;
+    const bool on = blk < nbl;
+    const int64_t col = (int64_t)blk * 32 + 4 * m;   // this lane's first row
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 4
     for (int j = 0; j < a.k; ++j) {
         const int pj = t * a.k + j;
         const float wj = __ldg(a.wts + pj);
-        const float4* src = reinterpret_cast<const float4*>(a.o + (int64_t)__ldg(a.pair_slot + pj) * a.L + blk * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 v = __ldcg(src + i);
-            acc[4 * i] = __fmaf_rn(wj, v.x, acc[4 * i]);
-            acc[4 * i + 1] = __fmaf_rn(wj, v.y, acc[4 * i + 1]);
-            acc[4 * i + 2] = __fmaf_rn(wj, v.z, acc[4 * i + 2]);
-            acc[4 * i + 3] = __fmaf_rn(wj, v.w, acc[4 * i + 3]);
+        const int64_t slot = __ldg(a.pair_slot + pj);
+        if (on) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.o + slot * a.L + col));
+            acc.x = __fmaf_rn(wj, v.x, acc.x);
+            acc.y = __fmaf_rn(wj, v.y, acc.y);
+            acc.z = __fmaf_rn(wj, v.z, acc.z);
+            acc.w = __fmaf_rn(wj, v.w, acc.w);
         }
     }
-    float4* yl = reinterpret_cast<float4*>(a.ylat + (int64_t)t * a.L + blk * 32);
+    if (on) *reinterpret_cast<float4*>(a.ylat + (int64_t)t * a.L + col) = acc;
+    // the block's Q8_1 (the quantiser's rule) over its 8-lane group
+    float amax = fmaxf(fmaxf(fabsf(acc.x), fabsf(acc.y)), fmaxf(fabsf(acc.z), fabsf(acc.w)));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) yl[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-    // its Q8_1 block (the quantiser's rule), row-major and packed for the U projection
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
     const float d = __fdiv_rn(amax, 127.0f);
-    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const float av[4] = {acc.x, acc.y, acc.z, acc.w};
+    uint32_t wv = 0;
     int sum = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 4; ++i) {
         int q = 0;
-        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(acc[i], d)), -127.0f), 127.0f);
+        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(av[i], d)), -127.0f), 127.0f);
         sum += q;
-        w[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+        wv |= (uint32_t)(q & 0xff) << (8 * i);
     }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) sum += __shfl_xor_sync(kFull, sum, o);
+    if (!on) return;
     const uint16_t dh = f2h(d);
     uint32_t* qb = reinterpret_cast<uint32_t*>(a.ylq + ((int64_t)t * nbl + blk) * 36);
-    qb[0] = (uint32_t)dh | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qb[1 + i] = w[i];
+    qb[1 + m] = wv;
     uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 32 + ((int64_t)t >> 3) * 256 + (t & 7) * 16;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(dst + 128) = make_uint4(w[4], w[5], w[6], w[7]);
-    a.cd[(int64_t)blk * a.cstride + t] = h2f(dh);
+    *reinterpret_cast<uint32_t*>(dst + (m < 4 ? 4 * m : 128 + 4 * (m - 4))) = wv;
+    if (m == 0) {
+        qb[0] = (uint32_t)dh | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
+        a.cd[(int64_t)blk * a.cstride + t] = h2f(dh);
+    }
 }
 
 // ---- measurement: the int8 tensor-core rate ------------------------------------
