@@ -936,11 +936,6 @@ SArgs gate_up_s(const elq_layer* ly, const LayerWs& w, int T, int route, const u
     g.x = zq;
     g.yq = w.hq; g.yq_ld = I / 32;
     g.wgs = ly->gate_up.gs; g.ags = ly->act_gz; g.ogs = ly->act_gh;
-    // the routed experts' down matrices, for the next kernel
-    g.pfe_q = static_cast<const uint8_t*>(ly->down.q);
-    g.pfe_d = reinterpret_cast<const uint8_t*>(ly->down.d);
-    g.pfe_qs = (int64_t)(L / kTileRows) * (I / 32) * slab_bytes(ly->down.fmt);
-    g.pfe_ds = (int64_t)(L / kTileRows) * d_tile_elems(ly->down.fmt, I / 32) * 2;
     g.L = L;
     g.err = w.err;
     g.early = 0;

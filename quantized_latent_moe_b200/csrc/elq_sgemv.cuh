@@ -19,9 +19,10 @@
 // each warp keeps up to two items' copies in flight.  Weights that do not
 // depend on the upstream kernel are requested before the grid dependency
 // wait.  Each CTA also asks L2 to prefetch its share of weights a later
-// kernel of the layer reads (the router rows and U during D; the routed
-// experts' down matrices during gate/up), so that those kernels find them in
-// L2.
+// kernel of the layer reads (the router rows and U during D), so that those
+// kernels find them in L2.  (The routed experts' down matrices are not
+// prefetched during gate/up: the down projection requests its weights before
+// its own grid dependency wait, and the extra traffic only slowed gate/up.)
 //
 // Routing.  k_route_small (one cluster) computes the router logits, gathers
 // them in its first CTA through distributed shared memory, and there takes
@@ -65,6 +66,15 @@ __device__ __forceinline__ void dsmem_st(uint32_t a, float v) {
 __device__ __forceinline__ void cluster_barrier() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// The two halves of a cluster barrier that only has to establish that every
+// CTA of the cluster is running (nothing to publish): arrive early, wait just
+// before the first distributed shared-memory access.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 struct SArgs {
     // weights: codes of slice s of tile t, blocks 8c .. 8c+7, of group e at
@@ -98,13 +108,10 @@ struct SArgs {
     float* ylat;
     uint8_t* ylq;
     int L;
-    // L2 prefetch: up to three fixed ranges, and one per-expert pair of ranges
+    // L2 prefetch: up to three fixed ranges
     const uint8_t* pf[3];
     int64_t pf_bytes[3];
     int64_t pf_share[3];                         // bytes per CTA (a multiple of 256)
-    const uint8_t* pfe_q;
-    const uint8_t* pfe_d;
-    int64_t pfe_qs, pfe_ds;                      // bytes per expert (multiples of 256)
     // NVFP4: global scales of the weights (one per group's expert, indexed by
     // expert), of the input activations, and of the epilogue's NVFP4 output
     const float* wgs;
@@ -656,26 +663,6 @@ __device__ void s_epilogue(const SArgs& g, const uint8_t* rs, const SUnit& u, co
     }
 }
 
-// Prefetch into L2 this CTA's share of the routed experts' ranges (group a's
-// expert e: bytes [0, len) at base + e * len; len a multiple of 256; groups
-// taken in order, the total split evenly over the grid's CTAs).
-__device__ __forceinline__ void s_prefetch_experts(const SArgs& g, const uint8_t* rs, int na, const uint8_t* base,
-                                                   int64_t len) {
-    const uint32_t len_u = (uint32_t)(len >> 8);
-    const uint32_t total_u = (uint32_t)na * len_u;
-    const uint32_t share_u = (total_u + gridDim.x - 1) / gridDim.x;
-    uint32_t lo = blockIdx.x * share_u;
-    const uint32_t hi = min(total_u, lo + share_u);
-    while (lo < hi) {
-        const uint32_t a = lo / len_u;
-        const uint32_t end = min(hi, (a + 1) * len_u);
-        const int e = sgroup(g, rs, (int)a).x;
-        const int64_t off = (int64_t)(lo - a * len_u) << 8;
-        l2_prefetch_range(base + (int64_t)e * len, off, off + ((int64_t)(end - lo) << 8));
-        lo = end;
-    }
-}
-
 // Prefetch into L2 this CTA's weights in every item of its cluster from `m0`
 // on (the items the ring has not requested yet), so that HBM streams them
 // while the ring works through the earlier ones.  Thread 0.
@@ -750,13 +737,15 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 1) k_route_small(RSArgs a) {
         for (int j = 0; j < kRouterJ; ++j) wr[j] = (has_e && j < nj) ? __ldg(wrow + 32 * j) : 0.0f;
     }
     const float bias = (has_e && a.bias) ? __ldg(a.bias + e) : 0.0f;
-    // every CTA of the cluster is running before any distributed store
-    if (a.C > 1) cluster_barrier();
+    // every CTA of the cluster is running before any distributed store: the
+    // arrival goes out now, the wait comes after z is staged
+    if (a.C > 1) cluster_arrive_relaxed();
     pdl_wait();
     pdl_trigger();
     for (int i = threadIdx.x; i < T * L / 4; i += blockDim.x)
         reinterpret_cast<float4*>(zs)[i] = __ldcg(reinterpret_cast<const float4*>(a.z) + i);
     __syncthreads();
+    if (a.C > 1) cluster_wait();
     if (has_e) {
         const uint32_t lg_lead = a.C > 1 ? dsmem_map(smem_addr(lg), 0) : smem_addr(lg);
         for (int t = 0; t < T; ++t) {
@@ -875,9 +864,12 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         *bad = 0;
         fence_barrier_init();
     }
+    __syncthreads();
     // every CTA of the cluster is running (its shared memory may be written
-    // by the others) before the first distributed shared-memory store
-    if (g.C > 1) cluster_barrier(); else __syncthreads();
+    // by the others) before the first distributed shared-memory store: the
+    // arrival goes out now, the wait comes before the first item's dots
+    if (g.C > 1) cluster_arrive_relaxed();
+    bool cl_pending = g.C > 1;
 
     int n_items = 0;
     int issued = -1;                 // thread 0: the last item whose copies went out
@@ -930,11 +922,6 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
             if (lane == 0) s_prefetch_own<FMT, OM>(g, rs, n_items, cid, ncl, S, rank);
         }
         prefetch_fixed();
-        if (g.pfe_q && warp == (int)(blockDim.x >> 5) - 1 && lane < 2) {
-            const int na = s_n_groups(g, rs);
-            if (lane == 0) s_prefetch_experts(g, rs, na, g.pfe_q, g.pfe_qs);
-            else s_prefetch_experts(g, rs, na, g.pfe_d, g.pfe_ds);
-        }
     }
 
     for (int m = 0;; ++m) {
@@ -943,6 +930,10 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         const int st = m % S;
         const SUnit u = s_unit<OM>(g, rs, item, rank, warp);
         const uint8_t* stg = stages + st * g.stage_bytes;
+        if (cl_pending) {
+            cluster_wait();
+            cl_pending = false;
+        }
         if (u.has && !*bad) {
             const bool got = mbar_wait_bounded(&bars[st], (uint32_t)((m / S) & 1), g.err, g.budget_ns);
             if (!__all_sync(kFull, got)) {
@@ -968,6 +959,7 @@ __global__ void __launch_bounds__(kSMaxWarps * 32, 2) k_sgemv(SArgs g) {
         }
         if (rank == 0) s_epilogue<FMT, OM>(g, rs, u, pbuf + (size_t)(m & 1) * units * g.T * 32);
     }
+    if (cl_pending) cluster_wait();   // no item: the arrival is still matched
     if (*bad && threadIdx.x == 0) {
         // drain: wait (bounded) for the last copies of every stage
         for (int m = (issued - S + 1 > 0 ? issued - S + 1 : 0); m <= issued; ++m)
