@@ -18,7 +18,7 @@ def _entries():
 
 def test_traffic_entries_name_workload_and_sources():
     for name, e in _entries().items():
-        assert e["workload"] in ("decode", "verify", "prefill", "stack", "tiny"), name
+        assert e["workload"] in ("decode", "verify", "prefill", "prefill_nvfp4", "stack", "tiny"), name
         assert len(e["source_hash"]) == 16, name
         assert e["dram_bytes_per_launch"] > 0, name
 
