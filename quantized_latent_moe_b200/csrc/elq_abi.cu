@@ -1368,7 +1368,7 @@ elq_status elq_quantize_q8_1(const void* x, int32_t x_type, int64_t rows, int64_
     if (!x || !out_q8_1) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x, 4) || !aligned(out_q8_1, 4)) return ELQ_ERR_ALIGNMENT;
     const int64_t nblk = rows * (cols / 32);
-    const dim3 grid((unsigned)((nblk + 255) / 256));   // one thread per block
+    const dim3 grid((unsigned)((4 * nblk + 255) / 256));   // four threads per block
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (x_type == ELQ_BF16)
         return cuda_status(launch(k_quant_q8_1<true>, grid, dim3(256), 0, s, false, x, nblk,
@@ -1386,7 +1386,7 @@ elq_status elq_quantize_nvfp4(const void* x, int32_t x_type, int64_t rows, int64
     if (!x || !out) return ELQ_ERR_INVALID_ARG;
     if (!aligned(x, 4) || !aligned(out, 2)) return ELQ_ERR_ALIGNMENT;
     const int64_t nblk = rows * (cols / 32);
-    const dim3 grid((unsigned)((nblk * 32 + 255) / 256));
+    const dim3 grid((unsigned)((nblk * 4 + 255) / 256));   // four threads per block
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (x_type == ELQ_BF16)
         return cuda_status(launch(k_quant_nvfp4<true>, grid, dim3(256), 0, s, false, x, nblk, g,
@@ -1817,10 +1817,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         // tensor cores (z), z's NVFP4 rows, router, the block-scaled experts, U
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         PackArgs pa;
@@ -1836,7 +1836,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32, w.z, nullptr, w.err);
         if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         const int64_t zblk = (int64_t)T * (L / 32);
-        e = launch(k_quant_nvfp4<false>, dim3((unsigned)((zblk * 32 + 255) / 256)), dim3(256), 0, s, pdl,
+        e = launch(k_quant_nvfp4<false>, dim3((unsigned)((zblk * 4 + 255) / 256)), dim3(256), 0, s, pdl,
                    (const void*)w.z, zblk, layer->act_gz, w.zq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits,
@@ -1854,10 +1854,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         // then the tensor-core experts and U
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         PackArgs pa;
@@ -1922,10 +1922,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
     } else {
         const int64_t nblk = (int64_t)T * (H / 32);
         if (x_type == ELQ_BF16)
-            e = launch(k_quant_q8_1<true>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<true>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         else
-            e = launch(k_quant_q8_1<false>, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, false, x,
+            e = launch(k_quant_q8_1<false>, dim3((unsigned)((4 * nblk + 255) / 256)), dim3(256), 0, s, false, x,
                        nblk, w.xq);
         if (e != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         gd = dense_w(&layer->D, T, w.xq, X_Q81_TOKEN, 0, OUT_F32_Q81, w.z, w.zq, w.partial, w.cnt_d, w.err);

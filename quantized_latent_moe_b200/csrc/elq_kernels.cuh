@@ -16,79 +16,121 @@ namespace elq {
 constexpr unsigned kFull = 0xffffffffu;
 
 // ============================================================================
-// a1 / a4 -- Q8_1 activation quantiser: one thread per 32-value block (the
-// block's 32 values in registers: amax, d = amax / 127, q = clamp(round(x /
-// d)), s = fp16(d * sum q); the same operations as the warp quantiser).
+// a1 / a4 -- Q8_1 activation quantiser: four lanes per 32-value block, eight
+// values each (a warp reads 512 contiguous bytes of bf16): amax and the code
+// sum over the four lanes, d = amax / 127, q = clamp(round(x / d)), s =
+// fp16(d * sum q); the same operations as the warp quantiser.
 // ============================================================================
 template <bool kBF16>
 __global__ void __launch_bounds__(256) k_quant_q8_1(const void* __restrict__ x, int64_t nblocks,
                                                     uint8_t* __restrict__ out) {
     pdl_wait();
-    const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (blk < nblocks) {
-        float v[32];
-        if ((reinterpret_cast<uintptr_t>(x) & 15) != 0) {
-            // 4-byte aligned input: element loads
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t blk = tid >> 2;      // four lanes per block, eight values each
+    const int q4 = (int)(tid & 3);
+    const bool on = blk < nblocks;
+    float v[8];
+    if (!on) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                v[i] = kBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[blk * 32 + i])
-                             : static_cast<const float*>(x)[blk * 32 + i];
-        } else if (kBF16) {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + blk * 32);
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    } else if ((reinterpret_cast<uintptr_t>(x) & 15) != 0) {
+        // 4-byte aligned input: element loads
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 w = __ldg(src + i);
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int i = 0; i < 8; ++i)
+            v[i] = kBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[blk * 32 + 8 * q4 + i])
+                         : static_cast<const float*>(x)[blk * 32 + 8 * q4 + i];
+    } else if (kBF16) {
+        // a warp reads 512 contiguous bytes
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + blk * 32) + q4);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
-                    v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
-                }
-            }
-        } else {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + blk * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 w = __ldg(src + i);
-                v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
-            }
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = __uint_as_float(ws[j] << 16);
+            v[2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
         }
-        float amax = 0.0f;
+    } else {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + blk * 32) + 2 * q4;
+        const float4 a = __ldg(src), b = __ldg(src + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    // the block's amax and code sum over its four lanes (order-free: a max and an integer sum)
+    float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-        const float d = __fdiv_rn(amax, 127.0f);
-        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        int sum = 0;
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const float d = __fdiv_rn(amax, 127.0f);
+    uint32_t w0 = 0, w1 = 0;
+    int sum = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            int q = 0;
-            if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f);
-            sum += q;
-            w[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
-        }
+    for (int i = 0; i < 8; ++i) {
+        int q = 0;
+        if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f);
+        sum += q;
+        if (i < 4) w0 |= (uint32_t)(q & 0xff) << (8 * i);
+        else w1 |= (uint32_t)(q & 0xff) << (8 * (i - 4));
+    }
+    sum += __shfl_xor_sync(kFull, sum, 1);
+    sum += __shfl_xor_sync(kFull, sum, 2);
+    if (on) {
         uint32_t* o = reinterpret_cast<uint32_t*>(out + blk * 36);
-        o[0] = (uint32_t)f2h(d) | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[1 + i] = w[i];
+        o[1 + 2 * q4] = w0;
+        o[2 + 2 * q4] = w1;
+        if (q4 == 0) o[0] = (uint32_t)f2h(d) | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
     }
     pdl_trigger();
 }
 
-// NVFP4 quantiser under global scale g: one warp per 32-value block (the
-// layer's NVFP4 activations use the same warp routine in their epilogues).
+// NVFP4 quantiser under global scale g: four lanes per 32-value block, eight
+// values each (two lanes per 16-value micro-block), the same operations per
+// value as warp_quant_nvfp4 (the layer's epilogues): s = e4m3(amax / 6 / g),
+// den = s * g, codes e2m1(x / den) in pairs.
 template <bool kBF16>
 __global__ void __launch_bounds__(256) k_quant_nvfp4(const void* __restrict__ x, int64_t nblocks, float g,
                                                      uint8_t* __restrict__ out) {
     pdl_wait();
-    const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (blk >= nblocks) return;
-    float v;
-    if (kBF16)
-        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[blk * 32 + lane]);
-    else
-        v = reinterpret_cast<const float*>(x)[blk * 32 + lane];
-    warp_quant_nvfp4(v, g, out + blk * 18);
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t blk = tid >> 2;
+    const int q4 = (int)(tid & 3);
+    const bool on = blk < nblocks;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    if (on) {
+        const int64_t e0 = blk * 32 + 8 * q4;
+        if (!kBF16 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + e0);
+            const float4 a = __ldg(src), b = __ldg(src + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                v[i] = kBF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[e0 + i])
+                             : static_cast<const float*>(x)[e0 + i];
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));          // the micro-block's two lanes
+    const uint32_t sc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+    const float den = __fmul_rn(e4m3x2_to_f32(sc).x, g);
+    uint32_t codes = 0;                                             // code bytes 4 q4 .. 4 q4 + 3
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float xa = den != 0.0f ? __fdiv_rn(v[2 * j], den) : 0.0f;
+        const float xb = den != 0.0f ? __fdiv_rn(v[2 * j + 1], den) : 0.0f;
+        codes |= (f32x2_to_e2m1x2(xa, xb) & 0xffu) << (8 * j);
+    }
+    const uint32_t sc1 = __shfl_sync(kFull, sc, (threadIdx.x & 31 & ~3) | 2);   // micro-block 1's scale
+    if (on) {
+        uint16_t* dst = reinterpret_cast<uint16_t*>(out + blk * 18);            // 2-byte aligned
+        dst[1 + 2 * q4] = (uint16_t)(codes & 0xffffu);
+        dst[2 + 2 * q4] = (uint16_t)(codes >> 16);
+        if (q4 == 0) dst[0] = (uint16_t)(sc | (sc1 << 8));
+    }
     pdl_trigger();
 }
 
