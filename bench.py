@@ -48,7 +48,7 @@ KERNELS_NVTC = ["quant_x", "pack_x", "proj_D", "quant_z", "router", "slot_map", 
 KERNELS_FUSED = ["layer"]
 KERNEL_NAMES = {"gate_up": {5: "k_sgemv<{fmt}> gate/up (cluster GEMV, +SwiGLU, {afmt})",
                             6: "k_wgemv<{fmt}> gate/up (+SwiGLU, Q8_1)",
-                            10: "k_tcgemm gate/up (tcgen05 kind::i8, +SwiGLU)",
+                            10: "k_tcgemm gate/up (tcgen05 kind::{kind}, +SwiGLU)",
                             11: "k_nvgemm gate/up (tcgen05 kind::mxf4nvf4 block-scaled, +SwiGLU, NVFP4)"},
                 "layer": {1: "k_decode_layer (the whole layer: D, router, gate/up, down + combine, U; one launch)"}}
 
@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--inputs", type=int, default=64, help="distinct inputs rotated over")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bounded CPU-baseline sample")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--f16", default="auto", choices=["auto", "on", "off"],
+                    help="fp16 codes for the tensor-core GEMMs (auto: on for T >= 16)")
     ap.add_argument("--fused", action="store_true",
                     help="small T as the single persistent kernel instead of the separate-kernel sequence")
     ap.add_argument("--no-clocks", action="store_true",
@@ -96,8 +98,18 @@ def nvfp4_globals(w):
     return torch.where(amax > 0, g, torch.ones_like(g))
 
 
-def build_layer(elq, synth, wl, li, dev, fused=False, batch=32):
-    """Layer li of the workload on device dev, quantised by the library."""
+def use_f16(args, wl):
+    """The fp16-operand tensor-core GEMMs: on for the workloads whose calls
+    take the tensor-core path (T >= 16), unless --f16 says otherwise."""
+    if args.f16 != "auto":
+        return args.f16 == "on"
+    return wl.T >= 16
+
+
+def build_layer(elq, synth, wl, li, dev, fused=False, batch=32, f16=False):
+    """Layer li of the workload on device dev, quantised by the library
+    (f16: also the fp16 codes of its Q8_0 matrices, for the fp16-operand
+    tensor-core GEMMs)."""
     import torch
     fmt, efmt = elq.FMT[wl.fmt], elq.FMT[wl.expert_fmt]
     dw = synth.dense_weights(wl, li, device=dev)
@@ -124,6 +136,8 @@ def build_layer(elq, synth, wl, li, dev, fused=False, batch=32):
         else:
             ly.set_experts(e0, g, u, d)
         del ws_, g, u, d
+    if f16:
+        ly.enable_f16()
     return ly
 
 
@@ -323,6 +337,36 @@ def tensor_peak_int8():
     return _INT8_PEAK
 
 
+_F16_PEAK = None
+
+
+def tensor_peak_f16():
+    """Dense fp16 tensor-core peak (TFLOP/s), measured as tensor_peak_int8 is,
+    with tcgen05.mma kind::f16 (M=128, N=256, K=16; elq_test_mma_f16_rate)."""
+    global _F16_PEAK
+    if _F16_PEAK is not None:
+        return _F16_PEAK
+    import torch
+    from quantized_latent_moe_b200 import elq
+    stream = torch.cuda.current_stream()
+    n_mma = 32768
+    ops = 2.0 * 128 * 256 * 16 * n_mma * elq.sm_count()
+    elq.test_mma_f16_rate(256)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _, err = elq.test_mma_f16_rate(n_mma)
+        e1.record(stream)
+        e1.synchronize()
+        if int(err.item()) != 0:
+            raise RuntimeError("fp16 rate kernel: a bounded wait ran out")
+        best = max(best, ops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    _F16_PEAK = (best, "measured fp16 (tcgen05.mma kind::f16 M128 N256 K16 loop, one CTA per SM, best of 5)")
+    return _F16_PEAK
+
+
 _FP4_PEAK = None
 
 
@@ -515,7 +559,8 @@ def run_elq(args):
     stream = torch.cuda.current_stream()
 
     # distinct layer copies (layer index = copy + 8 * rank) and inputs
-    layers = [build_layer(elq, synth, wl, c + args.copies * rank, dev, args.fused) for c in range(args.copies)]
+    layers = [build_layer(elq, synth, wl, c + args.copies * rank, dev, args.fused, f16=use_f16(args, wl))
+              for c in range(args.copies)]
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     S = args.inputs
@@ -678,25 +723,30 @@ def run_elq(args):
                                   "max_bound": max(t_tensor, t_hbm) / t_meas,
                                   "bound_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6}}}
         elif launches_per_step == 10:
-            # tensor-core path: gate/up is a contraction; int8 peak = measured bf16 x the nominal 2x ratio
+            # tensor-core path: gate/up is a contraction, on int8 or on fp16-widened codes (the
+            # peak of the MMA kind that ran, measured here)
             gu_ops = 2.0 * (2 * wl.I) * P * wl.L
-            tpk, tkind = tensor_peak_int8()
+            f16 = use_f16(args, wl)
+            tpk, tkind = tensor_peak_f16() if f16 else tensor_peak_int8()
             achieved = gu_ops / (gu_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][10], "achieved": achieved, "peak": tpk,
-                    "peak_kind": tkind, "unit": "TOPS (int8)", "frac": achieved / tpk,
+            roof = {"bound": "tensor", "kernel": KERNEL_NAMES["gate_up"][10].format(kind="f16" if f16 else "i8"),
+                    "achieved": achieved, "peak": tpk, "peak_kind": tkind,
+                    "unit": "TFLOP/s (fp16 operands)" if f16 else "TOPS (int8)", "frac": achieved / tpk,
                     "traffic": traffic_for("gate_up_tc", wl.name), "algorithmic_ops_per_launch": gu_ops,
                     "algorithmic_bytes_per_launch": gu_w}
-            # the launch's three bounds: int8 tensor ops, HBM bytes, and the
-            # fp32 epilogue (per 32-value block of every output element one
-            # int-to-float subtract, one scale product and one fused
-            # multiply-add, as packed pairs: 1.5 fma.rn.f32x2-rate
+            # the launch's three bounds: tensor ops, HBM bytes (fp16 codes: the
+            # weights' code bytes twice), and the fp32 epilogue (per 32-value
+            # block of every output element one scale product and one fused
+            # multiply-add, plus with int8 accumulators the int-to-float
+            # subtract, as packed pairs: 1.0 or 1.5 fma.rn.f32x2-rate
             # instructions per element-block)
-            gu_io = gu_w + wl.T * nb_L * 36 + P * nb_I * 36
+            gu_codes = float(wl.E) * (2 * wl.I) * wl.L
+            gu_io = gu_w + (gu_codes if f16 else 0.0) + wl.T * nb_L * 36 + P * nb_I * 36
             elem_blocks = float(P) * (2 * wl.I) * nb_L
             f2r = f32x2_rate()
             t_tensor = gu_ops / (tpk * 1e12)
             t_hbm = gu_io / (hbm_peak * 1e9)
-            t_epi = elem_blocks * 1.5 / f2r
+            t_epi = elem_blocks * (1.0 if f16 else 1.5) / f2r
             t_meas = gu_ms / 1e3
             roof["fractions"] = {
                 "tensor": t_tensor / t_meas, "hbm": t_hbm / t_meas, "epilogue": t_epi / t_meas,
@@ -718,11 +768,14 @@ def run_elq(args):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dev_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16" if (use_f16(args, wl) and launches_per_step in (10, 11)) else "int8",
             "data": "synthetic (seeded counter-hash normals; random-init weights of the layer's shape)",
             "config": {"workload": "%s: %s" % (wl.name, workload_desc(wl)),
                        "global_batch": wl.T * world, "parallelism": "replicas" if world > 1 else "1 GPU",
                        "layer_copies": args.copies, "inputs": S,
+                       "tc_operands": ("fp16-widened codes (kind::f16)" if use_f16(args, wl) else "int8 codes")
+                       if launches_per_step in (10, 11) else None,
                        "l2": "inputs larger than L2: %d layer copies x ~%.0f MB touched per step rotate, "
                              "%.0f MB between reuses of a layer (L2 126 MB)"
                              % (args.copies, layer_bytes / 1e6, (args.copies - 1) * layer_bytes / 1e6),

@@ -158,6 +158,11 @@ typedef struct {
     const void* q;
     const void* d;
     const float* gs;            /* NVFP4: device fp32 [n_rows / gs_rows], 4-byte aligned; else NULL */
+    const void* q16;            /* optional, Q8_0 only: the codes widened to fp16 (elq_pack_f16), 256-byte
+                                 * aligned.  When every int8 tensor-core matrix of a layer call carries
+                                 * it, the T >= 16 path multiplies fp16 operands (tcgen05 kind::f16,
+                                 * fp32 accumulators that hold each block's integer sum exactly) instead
+                                 * of int8 ones; the results are the same bits.  NULL: int8. */
 } elq_qmat;
 
 /* elq_layer.flags bits. */
@@ -205,6 +210,18 @@ size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k,
  * arena.  NVFP4 global scales stay with the caller (elq_qmat.gs). */
 elq_status elq_arena_pack(int32_t fmt, const void* aos, int32_t n_rows, int32_t k,
                           void* q_out, void* d_out, void* stream);
+
+/* The fp16 codes of a Q8_0 arena matrix (elq_qmat.q16): 2 * n_rows * k bytes,
+ * or 0 for another format.  Block-major: per (128-row tile, 32-value block),
+ * tile-major then block, 8 KB laid out [code / 16][row / 8][(code % 16) / 8]
+ * [row % 8][8 fp16] -- per 16-value half of the block the no-swizzle K-major
+ * operand of one fp16 MMA (experts: each expert's 2x its code bytes). */
+size_t elq_f16_bytes(const elq_qmat* w);
+
+/* Fill q16 (device, elq_f16_bytes(w) bytes, 256-byte aligned) from w's
+ * arena codes: every code c becomes the fp16 value c (exact).  Stream order;
+ * w->q16 is not read. */
+elq_status elq_pack_f16(const elq_qmat* w, void* q16, void* stream);
 
 /* Quantise fp32 weights (device, row-major n_rows x k) into the arena with the
  * format's own quantiser (block rules above).  Q8_0 and Q4_0; NVFP4 weights
@@ -396,6 +413,11 @@ elq_status elq_test_block_isums(int32_t wfmt, const void* w_aos, const void* x_q
  * int32 [elq_sm_count()], one accumulator word per CTA; err: device int32,
  * zero before the call, ELQ_ERR_TIMEOUT's code 1 if a wait ran out. */
 elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
+
+/* The fp16 tensor-core rate, for the roofline of the fp16-operand GEMMs: as
+ * elq_test_mma_i8_rate with tcgen05.mma kind::f16 of M = 128, N = 256, K = 16
+ * (2 * 128 * 256 * 16 = 1048576 operations each, fp32 accumulators). */
+elq_status elq_test_mma_f16_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream);
 
 /* The fp4 block-scaled tensor-core rate, for the NVFP4 experts' roofline: as
  * elq_test_mma_i8_rate with n_mma (>= 1) tcgen05.mma kind::mxf4nvf4 of M =

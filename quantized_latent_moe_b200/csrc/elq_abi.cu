@@ -124,6 +124,10 @@ elq_status check_qmat(const elq_qmat* w, int32_t rows, int32_t k, bool expert = 
         if (!w->gs || w->gs_rows <= 0 || rows % w->gs_rows) return ELQ_ERR_INVALID_ARG;
         if (!aligned(w->gs, 4)) return ELQ_ERR_ALIGNMENT;
     }
+    if (w->q16) {
+        if (w->fmt != ELQ_Q8_0) return ELQ_ERR_UNSUPPORTED;
+        if (!aligned(w->q16, 256)) return ELQ_ERR_ALIGNMENT;
+    }
     return ELQ_OK;
 }
 
@@ -490,12 +494,12 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s, bool pdl) {
 }
 
 // One kernel per output mode: each launch carries only its own epilogue.
-template <int OM>
+template <int OM, bool F16>
 cudaError_t launch_tc_t(const TcArgs& g, cudaStream_t s, bool pdl) {
     static bool optin[kMaxDevices];
-    cudaError_t e = smem_optin(k_tcgemm<OM>, kTcSmem, optin);
+    cudaError_t e = smem_optin(k_tcgemm<OM, F16>, tc_smem(F16), optin);
     if (e != cudaSuccess) return e;
-    return launch(k_tcgemm<OM>, dim3(sm_count()), dim3(kTcThreads), (size_t)kTcSmem, s, pdl, g);
+    return launch(k_tcgemm<OM, F16>, dim3(sm_count()), dim3(kTcThreads), (size_t)tc_smem(F16), s, pdl, g);
 }
 
 // The driver's tensor-map encoder, looked up once through the runtime.
@@ -533,23 +537,37 @@ bool tc_maps(TcArgs& g, int n_groups) {
     const cuuint32_t bdd[4] = {32, 4, kTcKS, 1};
     const cuuint64_t db[3] = {64, slots / 8, nb}, sb[2] = {256, slots * 32};
     const cuuint32_t bb[3] = {64, kTcN / 8, kTcKS};
+    // fp16 codes: [nb][2 halves][slots/8][64 words]
+    const cuuint64_t db16[4] = {64, slots / 8, 2, nb}, sb16[3] = {256, slots * 32, slots * 64};
+    const cuuint32_t bb16[4] = {64, kTcN / 8, 2, kTcKS};
     const cuuint64_t dbd[2] = {slots, nb}, sbd[1] = {slots * 4};
     const cuuint32_t bbd[2] = {kTcN, kTcKS};
+    const bool bmap = g.q16 ? encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.bq, db16, sb16, bb16)
+                            : encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, g.bq, db, sb, bb);
     return encode_map(&g.tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, g.q, da, sa, ba) &&
-           encode_map(&g.tm_d, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, g.d, dd, sd, bdd) &&
-           encode_map(&g.tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, g.bq, db, sb, bb) &&
+           encode_map(&g.tm_d, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, g.d, dd, sd, bdd) && bmap &&
            encode_map(&g.tm_bd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, g.bd, dbd, sbd, bbd);
 }
 
 cudaError_t launch_tc(TcArgs g, cudaStream_t s, bool pdl) {
     g.budget_ns = kWaitBudgetNs;
     if (!tc_maps(g, g.n_groups)) return cudaErrorInvalidValue;
+    // fp16 operands (kind::f16) when the matrix carries its fp16 codes; int8 (kind::i8) otherwise
+    if (g.q16) {
+        switch (g.out_mode) {
+        case TC_OUT_F32: return launch_tc_t<TC_OUT_F32, true>(g, s, pdl);
+        case TC_OUT_F32_Q81: return launch_tc_t<TC_OUT_F32_Q81, true>(g, s, pdl);
+        case TC_OUT_SWIGLU: return launch_tc_t<TC_OUT_SWIGLU, true>(g, s, pdl);
+        case TC_OUT_F32_ADD: return launch_tc_t<TC_OUT_F32_ADD, true>(g, s, pdl);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     switch (g.out_mode) {
-    case TC_OUT_F32: return launch_tc_t<TC_OUT_F32>(g, s, pdl);
-    case TC_OUT_F32_Q81: return launch_tc_t<TC_OUT_F32_Q81>(g, s, pdl);
-    case TC_OUT_SWIGLU: return launch_tc_t<TC_OUT_SWIGLU>(g, s, pdl);
-    case TC_OUT_F32_COMBINE: return launch_tc_t<TC_OUT_F32_COMBINE>(g, s, pdl);
-    case TC_OUT_F32_ADD: return launch_tc_t<TC_OUT_F32_ADD>(g, s, pdl);
+    case TC_OUT_F32: return launch_tc_t<TC_OUT_F32, false>(g, s, pdl);
+    case TC_OUT_F32_Q81: return launch_tc_t<TC_OUT_F32_Q81, false>(g, s, pdl);
+    case TC_OUT_SWIGLU: return launch_tc_t<TC_OUT_SWIGLU, false>(g, s, pdl);
+    case TC_OUT_F32_COMBINE: return launch_tc_t<TC_OUT_F32_COMBINE, false>(g, s, pdl);
+    case TC_OUT_F32_ADD: return launch_tc_t<TC_OUT_F32_ADD, false>(g, s, pdl);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -654,6 +672,7 @@ struct LayerWs {
     float* part_d;          // D chunk partials (fused path)
     // tensor-core path (int8; nvtc: NVFP4 experts on the block-scaled MMA)
     bool tc, nvtc;
+    bool f16;               // tensor-core GEMMs on fp16-widened codes (every such matrix carries q16)
     int64_t tstride, sstride;   // slots of the dense (tokens) and the expert (pairs, padded) B buffers
     uint8_t *bxq, *bzq, *bhq, *byq;
     float *bxd, *bzd, *bhd, *byd;
@@ -703,6 +722,11 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     // tensor cores, the experts on the block-scaled ones
     w.nvtc = ly->gate_up.fmt == ELQ_NVFP4 && !w.small && ly->D.fmt == ELQ_Q8_0 && ly->U.fmt == ELQ_Q8_0;
     const bool tcbuf = w.tc || w.nvtc;
+    // fp16-operand GEMMs when every int8 tensor-core matrix of the path carries its fp16 codes
+    w.f16 = (w.tc && ly->D.q16 && ly->U.q16 && ly->gate_up.q16 && ly->down.q16) ||
+            (w.nvtc && ly->D.q16 && ly->U.q16);
+    const size_t cx = w.f16 ? 64 : 32;                     // bytes of a block's codes in the B buffers
+    const size_t ce = (w.f16 && w.tc) ? 64 : 32;           // ... of the expert B buffers (NVFP4: packed codes)
     const size_t n_sync = w.fused ? (size_t)dec_sync_ints(T, L, I) : 0;
     const size_t n_cnt = 64 + (rblocks + 1) + w.pd.counter_ints + w.pgu.counter_ints + w.pdn.counter_ints +
                          w.pu.counter_ints + (size_t)T * (L / 32) + n_sync;
@@ -767,13 +791,13 @@ LayerWs layer_layout(const elq_layer* ly, int T, void* base, int x_type) {
     } else {
         w.partial = nullptr;
         const int nbH = H / 32, nbL = L / 32, nbI = I / 32;
-        w.bxq = c.take<uint8_t>(base, (size_t)nbH * w.tstride * 32);
+        w.bxq = c.take<uint8_t>(base, (size_t)nbH * w.tstride * cx);
         w.bxd = c.take<float>(base, (size_t)nbH * w.tstride * 4);
-        w.bzq = c.take<uint8_t>(base, (size_t)nbL * w.sstride * 32);
+        w.bzq = c.take<uint8_t>(base, (size_t)nbL * w.sstride * ce);
         w.bzd = c.take<float>(base, (size_t)nbL * w.sstride * 4);
-        w.bhq = c.take<uint8_t>(base, (size_t)nbI * w.sstride * 32);
+        w.bhq = c.take<uint8_t>(base, (size_t)nbI * w.sstride * ce);
         w.bhd = c.take<float>(base, (size_t)nbI * w.sstride * 4);
-        w.byq = c.take<uint8_t>(base, (size_t)nbL * w.tstride * 32);
+        w.byq = c.take<uint8_t>(base, (size_t)nbL * w.tstride * cx);
         w.byd = c.take<float>(base, (size_t)nbL * w.tstride * 4);
         w.slot_off = c.take<int32_t>(base, (size_t)(E + 1) * 4);
         w.tt_off = c.take<int32_t>(base, (size_t)(E + 1) * 4);
@@ -1105,6 +1129,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     pa.bq = w.bzq;
     pa.bd = w.bzd;
     pa.bstride = w.sstride;
+    pa.f16 = w.f16 ? 1 : 0;
     if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
     TcArgs g;
     std::memset(&g, 0, sizeof(g));
@@ -1115,6 +1140,8 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     g.n_groups = E;
     g.q_gstride = (int64_t)g.rtiles * g.nb * kQ80Slab;
     g.d_gstride = (int64_t)g.rtiles * g.nb * kTileRows;
+    g.q16 = w.f16 ? static_cast<const uint8_t*>(ly->gate_up.q16) : nullptr;
+    g.q16_gstride = 2 * g.q_gstride;
     g.act = w.act; g.n_act = w.n_act; g.slot_off = w.slot_off; g.offsets = w.offsets; g.tt_off = w.tt_off;
     g.T = T;
     g.bq = w.bzq; g.bd = w.bzd; g.bstride = w.sstride;
@@ -1131,6 +1158,8 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     h.n_groups = E;
     h.q_gstride = (int64_t)h.rtiles * h.nb * kQ80Slab;
     h.d_gstride = (int64_t)h.rtiles * h.nb * kTileRows;
+    h.q16 = w.f16 ? static_cast<const uint8_t*>(ly->down.q16) : nullptr;
+    h.q16_gstride = 2 * h.q_gstride;
     h.act = w.act; h.n_act = w.n_act; h.slot_off = w.slot_off; h.offsets = w.offsets; h.tt_off = w.tt_off;
     h.T = T;
     h.bq = w.bhq; h.bd = w.bhd; h.bstride = w.sstride;
@@ -1142,6 +1171,7 @@ elq_status run_experts_tc(const elq_layer* ly, const LayerWs& w, int T, const ui
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
+    c.f16 = w.f16 ? 1 : 0;
     const int64_t threads = (int64_t)T * ((L / 32 + 3) / 4) * 32;   // one warp per (token, 4 blocks)
     if (launch(k_tc_combine, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess ||
         !mark())
@@ -1235,6 +1265,7 @@ elq_status run_experts_nvtc(const elq_layer* ly, const LayerWs& w, int T, const 
     std::memset(&c, 0, sizeof(c));
     c.o = w.o; c.wts = wts; c.pair_slot = w.pair_slot; c.T = T; c.L = L; c.k = k;
     c.ylat = y_lat; c.ylq = w.ylq; c.cq = w.byq; c.cd = w.byd; c.cstride = w.tstride;
+    c.f16 = w.f16 ? 1 : 0;
     const int64_t threads = (int64_t)T * ((L / 32 + 3) / 4) * 32;   // one warp per (token, 4 blocks)
     if (launch(k_tc_combine, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, pdl, c) != cudaSuccess ||
         !mark())
@@ -1276,7 +1307,23 @@ const char* elq_status_string(int32_t status) {
     }
 }
 
-int32_t elq_version(void) { return 2; }
+int32_t elq_version(void) { return 3; }
+
+size_t elq_f16_bytes(const elq_qmat* w) {
+    if (!w || w->fmt != ELQ_Q8_0 || w->n_rows <= 0 || w->k <= 0) return 0;
+    return (size_t)w->n_rows * (size_t)w->k * 2;
+}
+
+elq_status elq_pack_f16(const elq_qmat* w, void* q16, void* stream) {
+    if (!w || !q16 || !w->q) return ELQ_ERR_INVALID_ARG;
+    if (w->fmt != ELQ_Q8_0) return ELQ_ERR_UNSUPPORTED;
+    if (w->n_rows <= 0 || w->k <= 0 || w->n_rows % kTileRows || w->k % 32) return ELQ_ERR_INVALID_ARG;
+    if (!aligned(w->q, 256) || !aligned(q16, 256)) return ELQ_ERR_ALIGNMENT;
+    const int64_t pieces = (int64_t)w->n_rows * w->k / 16;   // 16-byte pieces of the int8 codes
+    return cuda_status(launch(k_arena_f16, dim3((unsigned)((pieces + 255) / 256)), dim3(256), 0,
+                              static_cast<cudaStream_t>(stream), false, static_cast<const uint8_t*>(w->q), pieces,
+                              (int)(w->k / 32), static_cast<uint8_t*>(q16)));
+}
 
 size_t elq_arena_bytes(int32_t fmt, int32_t n_rows, int32_t k, size_t* q_bytes, size_t* d_bytes) {
     if (!arena_fmt_ok(fmt) || n_rows <= 0 || k <= 0 || n_rows % kTileRows || k % arena_k_unit(fmt)) {
@@ -1682,6 +1729,16 @@ elq_status elq_test_mma_i8_rate(int32_t n_mma, int32_t* sink, int32_t* err, void
                               kWaitBudgetNs));
 }
 
+elq_status elq_test_mma_f16_rate(int32_t n_mma, int32_t* sink, int32_t* err, void* stream) {
+    if (n_mma < 2 || !sink || !err) return ELQ_ERR_INVALID_ARG;
+    static bool optin[kMaxDevices];
+    cudaError_t e = smem_optin(k_test_mma_f16_rate, kRateSmem, optin);
+    if (e != cudaSuccess) return ELQ_ERR_CUDA;
+    return cuda_status(launch(k_test_mma_f16_rate, dim3(sm_count()), dim3(128), (size_t)kRateSmem,
+                              static_cast<cudaStream_t>(stream), false, (int)n_mma, (int*)sink, (int*)err,
+                              kWaitBudgetNs));
+}
+
 elq_status elq_test_mma_nvf4_rate(int32_t n_mma, int32_t n_cols, int32_t cp_each, int32_t* sink, int32_t* err,
                                   void* stream) {
     if (n_mma < 1 || !sink || !err) return ELQ_ERR_INVALID_ARG;
@@ -1832,8 +1889,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         pa.bq = w.bxq;
         pa.bd = w.bxd;
         pa.bstride = w.tstride;
+        pa.f16 = w.f16 ? 1 : 0;
         if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32, w.z, nullptr, w.err);
+        gd.q16 = w.f16 ? static_cast<const uint8_t*>(layer->D.q16) : nullptr;
         if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         const int64_t zblk = (int64_t)T * (L / 32);
         e = launch(k_quant_nvfp4<false>, dim3((unsigned)((zblk * 4 + 255) / 256)), dim3(256), 0, s, pdl,
@@ -1846,6 +1905,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         if (st != ELQ_OK) return st;
         TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, residual ? TC_OUT_F32_ADD : TC_OUT_F32, y,
                              nullptr, w.err);
+        gu.q16 = w.f16 ? static_cast<const uint8_t*>(layer->U.q16) : nullptr;
         if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         return ELQ_OK;
     }
@@ -1869,8 +1929,10 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         pa.bq = w.bxq;
         pa.bd = w.bxd;
         pa.bstride = w.tstride;
+        pa.f16 = w.f16 ? 1 : 0;
         if (launch_pack(pa, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         TcArgs gd = dense_tc(&layer->D, T, w.bxq, w.bxd, w.tstride, TC_OUT_F32_Q81, w.z, w.zq, w.err);
+        gd.q16 = w.f16 ? static_cast<const uint8_t*>(layer->D.q16) : nullptr;
         if (launch_tc(gd, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         e = launch_router(w.z, layer->router_w, layer->router_bias, T, L, E, k, w.idx, w.wts, w.logits,
                           w.cnt_router, true, w.counts, w.offsets, w.perm, w.pos, w.act, w.n_act, s, pdl);
@@ -1879,6 +1941,7 @@ elq_status run_layer(const elq_layer* layer, const void* x, int32_t x_type, int3
         if (st != ELQ_OK) return st;
         TcArgs gu = dense_tc(&layer->U, T, w.byq, w.byd, w.tstride, residual ? TC_OUT_F32_ADD : TC_OUT_F32, y,
                              nullptr, w.err);
+        gu.q16 = w.f16 ? static_cast<const uint8_t*>(layer->U.q16) : nullptr;
         if (launch_tc(gu, s, pdl) != cudaSuccess || !mark()) return ELQ_ERR_CUDA;
         return ELQ_OK;
     }

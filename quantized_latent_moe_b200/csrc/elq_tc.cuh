@@ -51,6 +51,16 @@ __device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
         : "memory");
 }
+// D (fp32 in TMEM) = A * B (+ D when acc != 0), fp16 operands, K = 16.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
 // Arrive (once) on an mbarrier when all MMAs this thread issued so far are done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -171,6 +181,18 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     return r;
 }
 
+// Two small integers (|q| <= 2048, exact in fp16) as an fp16 pair, q0 in the low half.
+__device__ __forceinline__ uint32_t h2_pack_int(int q0, int q1) {
+    return (uint32_t)__half_as_ushort(__int2half_rn(q0)) | ((uint32_t)__half_as_ushort(__int2half_rn(q1)) << 16);
+}
+
+// Eight signed 8-bit codes (w0 bytes 0..3, then w1) as eight fp16, in order.
+__device__ __forceinline__ uint4 h8_from_i8(uint32_t w0, uint32_t w1) {
+    auto b = [](uint32_t w, int i) { return (int)(int8_t)(uint8_t)(w >> (8 * i)); };
+    return make_uint4(h2_pack_int(b(w0, 0), b(w0, 1)), h2_pack_int(b(w0, 2), b(w0, 3)),
+                      h2_pack_int(b(w1, 0), b(w1, 1)), h2_pack_int(b(w1, 2), b(w1, 3)));
+}
+
 // Exact int32 -> fp32 for |s| < 2^22 without the (slow) conversion unit: the
 // integer s + 0x4B400000 is the bit pattern of the float 1.5 * 2^23 + s, so
 // one fp32 subtraction of 1.5 * 2^23 recovers s exactly.  Each block's MMA
@@ -196,6 +218,10 @@ __device__ __forceinline__ uint64_t umma_desc(const void* p, uint32_t lbo, uint3
 __host__ __device__ constexpr uint32_t umma_idesc_i8(int M, int N) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor: f16 x f16 -> f32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 
 // ---- B buffers: Q8_1 rows -> canonical slots ---------------------------------
 //
@@ -220,6 +246,7 @@ struct PackArgs {
     uint8_t* bq;
     float* bd;
     int64_t bstride;            // slots in the buffer (multiple of 16)
+    int f16;                    // codes widened to fp16 (the kind::f16 operand layout)
 };
 
 // Shared copy of slot_off[0 .. E] for slot_row_of (E <= 1024).
@@ -275,11 +302,43 @@ __global__ void __launch_bounds__(256) k_pack_b(PackArgs a) {
         hi4 = make_uint4(__ldg(src + 5), __ldg(src + 6), __ldg(src + 7), __ldg(src + 8));
         dd = h2f((uint16_t)(w0 & 0xffff));
     }
-    uint8_t* dst = a.bq + (int64_t)kb * a.bstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
-    *reinterpret_cast<uint4*>(dst) = lo4;
-    *reinterpret_cast<uint4*>(dst + 128) = hi4;
+    if (a.f16) {
+        // half h (codes 16 h .. 16 h + 15) of the block: two 16-byte core-matrix rows of fp16
+        uint8_t* dst = a.bq + (int64_t)kb * a.bstride * 64 + (slot >> 3) * 256 + (slot & 7) * 16;
+        uint8_t* dst1 = dst + a.bstride * 32;
+        *reinterpret_cast<uint4*>(dst) = h8_from_i8(lo4.x, lo4.y);
+        *reinterpret_cast<uint4*>(dst + 128) = h8_from_i8(lo4.z, lo4.w);
+        *reinterpret_cast<uint4*>(dst1) = h8_from_i8(hi4.x, hi4.y);
+        *reinterpret_cast<uint4*>(dst1 + 128) = h8_from_i8(hi4.z, hi4.w);
+    } else {
+        uint8_t* dst = a.bq + (int64_t)kb * a.bstride * 32 + (slot >> 3) * 256 + (slot & 7) * 16;
+        *reinterpret_cast<uint4*>(dst) = lo4;
+        *reinterpret_cast<uint4*>(dst + 128) = hi4;
+    }
     a.bd[(int64_t)kb * a.bstride + slot] = dd;
     pdl_trigger();
+}
+
+// fp16 copy of a Q8_0 arena's codes for the kind::f16 GEMM.  The int8 arena
+// holds a 128-row tile slice-major -- [slice s][block][1 KB], the 1 KB of 32
+// rows as [row/8][code/16][row%8][16] -- and the copy block-major: per (tile,
+// block) 8 KB, [code/16][row/8][(code%16)/8][row%8][8 fp16] (per K = 16 half
+// of the block, the no-swizzle K-major operand of one MMA).  One thread per
+// 16-byte piece of the int8 arena.
+__global__ void __launch_bounds__(256) k_arena_f16(const uint8_t* __restrict__ q, int64_t n_pieces, int nb,
+                                                   uint8_t* __restrict__ q16) {
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= n_pieces) return;
+    const int64_t per_tile = (int64_t)nb * 256;     // pieces of a tile: 4 slices x nb blocks x 64
+    const int64_t tile = p / per_tile;
+    const int rem = (int)(p - tile * per_tile);
+    const int sl = rem / (nb * 64), rem2 = rem - sl * nb * 64;
+    const int kb = rem2 >> 6, pi = rem2 & 63;
+    const int r8 = 4 * sl + (pi >> 4), hh = (pi >> 3) & 1, r = pi & 7;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(q) + p);
+    uint8_t* dst = q16 + (tile * nb + kb) * 8192 + hh * 4096 + r8 * 256 + r * 16;
+    *reinterpret_cast<uint4*>(dst) = h8_from_i8(w.x, w.y);
+    *reinterpret_cast<uint4*>(dst + 128) = h8_from_i8(w.z, w.w);
 }
 
 constexpr int kTcN = 64;            // tokens per tile
@@ -351,20 +410,29 @@ __global__ void __launch_bounds__(1024) k_tc_route(const int32_t* offsets, const
 
 constexpr int kTcKS = 4;            // blocks per pipeline stage (and per accumulator group)
 constexpr int kTcTileRowsPad = 129; // padded row count of the SwiGLU transpose (no bank conflicts)
-constexpr int kTcStages = 6;
 constexpr int kTcBufs = 8;          // TMEM accumulators of kTcN columns (all 512 columns), two groups of kTcKS
 constexpr int kTcGroups = kTcBufs / kTcKS;
 constexpr int kTcEpiWarps = 16;     // epilogue warps: 4 TMEM lane quarters x 4 column quarters
 constexpr int kTcEpiCols = 16;      // accumulator columns (tokens) per epilogue warp
 constexpr int kTcThreads = 32 * (2 + kTcEpiWarps);
-constexpr int kTcStageA = kTcKS * 4096;
-constexpr int kTcStageB = kTcKS * kTcN * 32;
 constexpr int kTcStageDw = kTcKS * kTileRows * 2;
 constexpr int kTcStageDa = kTcKS * kTcN * 4;
-constexpr int kTcStage = kTcStageA + kTcStageB + kTcStageDw + kTcStageDa;
 constexpr int kTcXld = kTcTileRowsPad;
 constexpr int kTcXchg = kTcN * kTcXld * 4;                  // SwiGLU transpose: [token][row], padded rows
-constexpr int kTcSmem = 1024 + kTcStages * kTcStage + kTcXchg + 6144 + 4100;   // + the staged units
+// One pipeline stage: weight codes (A), weight scales, activation codes (B),
+// activation scales.  The codes are int8 (kind::i8 MMAs), or the same
+// integers widened to fp16 (kind::f16 MMAs, fp32 accumulators that hold the
+// block sums exactly: every product and partial sum is an integer below 2^24).
+__host__ __device__ constexpr int tc_stage_a(bool f16) { return kTcKS * (f16 ? 8192 : 4096); }
+__host__ __device__ constexpr int tc_stage_b(bool f16) { return kTcKS * kTcN * (f16 ? 64 : 32); }
+__host__ __device__ constexpr int tc_stage(bool f16) {
+    return tc_stage_a(f16) + kTcStageDw + tc_stage_b(f16) + kTcStageDa;
+}
+__host__ __device__ constexpr int tc_nstages(bool f16) { return f16 ? 3 : 6; }
+__host__ __device__ constexpr int tc_smem(bool f16) {
+    return 1024 + tc_nstages(f16) * tc_stage(f16) + kTcXchg + 6144 + 4100;   // + the staged units
+}
+static_assert(tc_smem(true) <= 227 * 1024 && tc_smem(false) <= 227 * 1024, "one CTA per SM");
 static_assert(kTcEpiWarps * kTcEpiCols == 4 * kTcN, "the epilogue warps cover the 128 x 64 tile");
 
 enum { TC_OUT_F32 = 0, TC_OUT_F32_Q81 = 1, TC_OUT_SWIGLU = 2, TC_OUT_F32_COMBINE = 3, TC_OUT_F32_ADD = 4 };
@@ -377,11 +445,15 @@ struct TcArgs {
     //         [block][slice][1 KB], the MMA's A layout
     //  tm_d : weight scales, uint16 [tiles][nb][4][32]; box -> [block][slice][32]
     //  tm_b : packed activation codes, uint32 [nb][slots/8][64]; box [4][8][64]
+    //         (fp16 codes: uint32 [nb][2][slots/8][64]; box [4][2][8][64])
     //  tm_bd: activation scales, fp32 [nb][slots]; box [4][64]
+    // (fp16 codes: the weight codes come from q16 by one bulk copy a stage)
     CUtensorMap tm_a, tm_d, tm_b, tm_bd;
     const uint8_t* q;           // weight arena of group 0
     const uint16_t* d;
     int64_t q_gstride, d_gstride;
+    const uint8_t* q16;         // fp16 codes (kind::f16 launches): [tiles][nb][2][16][2][8][8] fp16
+    int64_t q16_gstride;
     int nb, rtiles;
     int n_groups;               // matrices in the arena (the experts, or 1)
     // groups: dense (act == NULL: one group of T tokens in slots 0 .. T-1) or
@@ -466,7 +538,7 @@ __device__ __forceinline__ TcUnit tc_unit(const TcArgs& g, int u) {
 constexpr int kUnitsSmem = 256;
 constexpr int kUnitTableInts = 1025;        // tt_off[0 .. na], na <= 1024
 constexpr int kUnitsBytes = kUnitsSmem * (int)sizeof(TcUnit) + kUnitTableInts * 4;
-static_assert(kUnitsBytes == 6144 + 4100, "kTcSmem counts the staged units' bytes");
+static_assert(kUnitsBytes == 6144 + 4100, "tc_smem counts the staged units' bytes");
 
 // Expert unit u with the token-tile offsets in shared memory (stt = tt_off[0
 // .. na]): the search runs there; the expert, first slot and pair count take
@@ -523,8 +595,10 @@ __device__ __forceinline__ int tc_units(const TcArgs& g) {
 __device__ __noinline__ void tc_quant(float v, uint8_t* dst) { warp_quant_q8_1(v, dst); }
 
 
-template <int OM>
+template <int OM, bool F16>
 __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant__ TcArgs g) {
+    constexpr int kTcStages = tc_nstages(F16), kTcStage = tc_stage(F16);
+    constexpr int kTcStageA = tc_stage_a(F16), kTcStageB = tc_stage_b(F16);
     extern __shared__ __align__(1024) uint8_t tcsm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(tcsm);            // [stages]
     uint64_t* empty = full + kTcStages;                             // [stages]
@@ -592,9 +666,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     mbar_arrive_expect_tx(&full[s], (uint32_t)kTcStage);
                     const int kb0 = ks * kTcKS;
                     const int tile = un.e * g.rtiles + un.rt;
-                    tma_load_4d(st, &g.tm_a, 0, 0, kb0, tile, &full[s]);
+                    if constexpr (F16) {
+                        bulk_g2s(st, g.q16 + un.e * g.q16_gstride + ((int64_t)un.rt * g.nb + kb0) * 8192,
+                                 (uint32_t)kTcStageA, &full[s]);
+                    } else {
+                        tma_load_4d(st, &g.tm_a, 0, 0, kb0, tile, &full[s]);
+                    }
                     tma_load_4d(st + kTcStageA, &g.tm_d, 0, 0, kb0, tile, &full[s]);
-                    tma_load_3d(st + kTcStageA + kTcStageDw, &g.tm_b, 0, un.slot0 >> 3, kb0, &full[s]);
+                    if constexpr (F16)
+                        tma_load_4d(st + kTcStageA + kTcStageDw, &g.tm_b, 0, un.slot0 >> 3, 0, kb0, &full[s]);
+                    else
+                        tma_load_3d(st + kTcStageA + kTcStageDw, &g.tm_b, 0, un.slot0 >> 3, kb0, &full[s]);
                     tma_load_2d(st + kTcStageA + kTcStageDw + kTcStageB, &g.tm_bd, un.slot0, kb0, &full[s]);
                 }
             }
@@ -607,7 +689,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
             for (int u = u0; u < u1 && !*abort_v; ++u) {
                 const TcUnit un = unit_at(u);
                 if (!un.valid) continue;
-                const uint32_t idesc = umma_idesc_i8(128, un.ncols);
+                const uint32_t idesc = F16 ? umma_idesc_f16(128, un.ncols) : umma_idesc_i8(128, un.ncols);
                 for (int ks = 0; ks < kstages && !*abort_v; ++ks, ++it) {
                     const int s = it % kTcStages, gr = it % kTcGroups;
                     if (it >= kTcGroups &&
@@ -622,9 +704,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     tc_fence_after();
                     const uint8_t* st = stages + s * kTcStage;
                     for (int kl = 0; kl < kTcKS; ++kl) {
-                        const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
-                        const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
-                        umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 0u);
+                        if constexpr (F16) {
+                            // a block = two K = 16 halves, 4 KB of A and 2 KB of B each
+                            for (int h = 0; h < 2; ++h) {
+                                const uint64_t adesc = umma_desc(st + (kl * 2 + h) * 4096, 128, 256);
+                                const uint64_t bdesc =
+                                    umma_desc(st + kTcStageA + kTcStageDw + (kl * 2 + h) * kTcN * 32, 128, 256);
+                                umma_f16(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc,
+                                         (uint32_t)h);
+                            }
+                        } else {
+                            const uint64_t adesc = umma_desc(st + kl * 4096, 128, 256);
+                            const uint64_t bdesc = umma_desc(st + kTcStageA + kTcStageDw + kl * kTcN * 32, 128, 256);
+                            umma_i8(tmem + (uint32_t)((gr * kTcKS + kl) * kTcN), adesc, bdesc, idesc, 0u);
+                        }
                     }
                     umma_commit(&tfull[gr]);
                     umma_commit(&empty[s]);
@@ -688,12 +781,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
 #pragma unroll
                             for (int j4 = 0; j4 < kTcEpiCols / 4; ++j4) {
                                 const float4 dv = dak[j4];
-                                const uint64_t i0 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4] + kAccSeed),
-                                                                   __uint_as_float(rc[h][4 * j4 + 1] + kAccSeed)),
-                                                           seed2);
-                                const uint64_t i1 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4 + 2] + kAccSeed),
-                                                                   __uint_as_float(rc[h][4 * j4 + 3] + kAccSeed)),
-                                                           seed2);
+                                uint64_t i0, i1;
+                                if constexpr (F16) {
+                                    // fp32 accumulators: the block sums themselves
+                                    i0 = f2_pack(__uint_as_float(rc[h][4 * j4]), __uint_as_float(rc[h][4 * j4 + 1]));
+                                    i1 = f2_pack(__uint_as_float(rc[h][4 * j4 + 2]),
+                                                 __uint_as_float(rc[h][4 * j4 + 3]));
+                                } else {
+                                    i0 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4] + kAccSeed),
+                                                        __uint_as_float(rc[h][4 * j4 + 1] + kAccSeed)),
+                                                seed2);
+                                    i1 = f2_sub(f2_pack(__uint_as_float(rc[h][4 * j4 + 2] + kAccSeed),
+                                                        __uint_as_float(rc[h][4 * j4 + 3] + kAccSeed)),
+                                                seed2);
+                                }
                                 part2[2 * j4] = f2_fma(i0, f2_mul(dw2, f2_pack(dv.x, dv.y)), part2[2 * j4]);
                                 part2[2 * j4 + 1] = f2_fma(i1, f2_mul(dw2, f2_pack(dv.z, dv.w)), part2[2 * j4 + 1]);
                             }
@@ -768,20 +869,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
                     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
                     const float d = __fdiv_rn(amax, 127.0f);
                     uint32_t w0 = 0, w1 = 0;
+                    int qv[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         int q = 0;
                         if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(h[i], d)), -127.0f), 127.0f);
+                        qv[i] = q;
                         if (i < 4) w0 |= (uint32_t)(q & 0xff) << (8 * i);
                         else w1 |= (uint32_t)(q & 0xff) << (8 * (i - 4));
                     }
                     if (on) {
                         const int64_t slot = slot0 + t;
                         const int kbh = un.rt * 2 + hb;
-                        // codes 8 qd .. 8 qd + 7 of the slot's 32: first or second 16-byte half, low or high 8 bytes
-                        uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 32 + (slot >> 3) * 256 + (qd >> 1) * 128 +
-                                       (slot & 7) * 16 + (qd & 1) * 8;
-                        *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+                        if constexpr (F16) {
+                            // codes 8 qd .. 8 qd + 7 as fp16: half qd / 2 of the block, core matrix qd % 2
+                            uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 64 + (int64_t)(qd >> 1) * g.cstride * 32 +
+                                           (slot >> 3) * 256 + (qd & 1) * 128 + (slot & 7) * 16;
+                            *reinterpret_cast<uint4*>(dst) = make_uint4(h2_pack_int(qv[0], qv[1]), h2_pack_int(qv[2], qv[3]),
+                                                                        h2_pack_int(qv[4], qv[5]), h2_pack_int(qv[6], qv[7]));
+                        } else {
+                            // codes 8 qd .. 8 qd + 7 of the slot's 32: first or second 16-byte half, low or high 8 bytes
+                            uint8_t* dst = g.cq + (int64_t)kbh * g.cstride * 32 + (slot >> 3) * 256 + (qd >> 1) * 128 +
+                                           (slot & 7) * 16 + (qd & 1) * 8;
+                            *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+                        }
                         // the activation scale as the down projection reads it: fp32 of the stored fp16
                         if (qd == 0) g.cd[(int64_t)kbh * g.cstride + slot] = __half2float(__float2half_rn(d));
                     }
@@ -880,9 +991,10 @@ struct CombArgs {
     int T, L, k;
     float* ylat;                // [T][L]
     uint8_t* ylq;               // [T][L/32] Q8_1
-    uint8_t* cq;                // packed codes [L/32][cstride]
+    uint8_t* cq;                // packed codes [L/32][cstride] (fp16 codes: [L/32][2][cstride] x 32 B)
     float* cd;                  // packed scales [L/32][cstride]
     int64_t cstride;
+    int f16;                    // codes widened to fp16 (the kind::f16 operand layout)
 };
 
 __global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
@@ -919,10 +1031,12 @@ __global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
     const float av[4] = {acc.x, acc.y, acc.z, acc.w};
     uint32_t wv = 0;
     int sum = 0;
+    int qv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         int q = 0;
         if (d != 0.0f) q = (int)fminf(fmaxf(roundf(__fdiv_rn(av[i], d)), -127.0f), 127.0f);
+        qv[i] = q;
         sum += q;
         wv |= (uint32_t)(q & 0xff) << (8 * i);
     }
@@ -932,8 +1046,15 @@ __global__ void __launch_bounds__(256) k_tc_combine(CombArgs a) {
     const uint16_t dh = f2h(d);
     uint32_t* qb = reinterpret_cast<uint32_t*>(a.ylq + ((int64_t)t * nbl + blk) * 36);
     qb[1 + m] = wv;
-    uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 32 + ((int64_t)t >> 3) * 256 + (t & 7) * 16;
-    *reinterpret_cast<uint32_t*>(dst + (m < 4 ? 4 * m : 128 + 4 * (m - 4))) = wv;
+    if (a.f16) {
+        // codes 4 m .. 4 m + 3 as fp16: half m / 4 of the block, core matrix (m / 2) % 2, its 8-byte half m % 2
+        uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 64 + (int64_t)(m >> 2) * a.cstride * 32 +
+                       ((int64_t)t >> 3) * 256 + ((m >> 1) & 1) * 128 + (t & 7) * 16 + (m & 1) * 8;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(h2_pack_int(qv[0], qv[1]), h2_pack_int(qv[2], qv[3]));
+    } else {
+        uint8_t* dst = a.cq + (int64_t)blk * a.cstride * 32 + ((int64_t)t >> 3) * 256 + (t & 7) * 16;
+        *reinterpret_cast<uint32_t*>(dst + (m < 4 ? 4 * m : 128 + 4 * (m - 4))) = wv;
+    }
     if (m == 0) {
         qb[0] = (uint32_t)dh | ((uint32_t)f2h(__fmul_rn(d, (float)sum)) << 16);
         a.cd[(int64_t)blk * a.cstride + t] = h2f(dh);
@@ -979,6 +1100,55 @@ __global__ void __launch_bounds__(128, 1) k_test_mma_i8_rate(int n_mma, int* sin
         const uint64_t ad = umma_desc(a, 128, 256), bd = umma_desc(b, 128, 256);
         for (int i = 0; i < n_mma; ++i)
             umma_i8(tmem + (uint32_t)((i & 1) * kRateN), ad, bd, idesc, i >= 2 ? 1u : 0u);
+        umma_commit(done);
+    }
+    __syncwarp();
+    const bool ok = warp_wait_bounded(done, 0, err, budget_ns);
+    tc_fence_after();
+    if (warp == 0) {
+        uint32_t r[16];
+        tmem_ld16(tmem, r);
+        tmem_ld_wait();
+        if (ok && threadIdx.x == 0) sink[blockIdx.x] = (int)r[0];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 2 * kRateN);
+}
+
+// ---- measurement: the fp16 tensor-core rate ------------------------------------
+//
+// As k_test_mma_i8_rate, with tcgen05.mma kind::f16 of M=128, N=256, K=16
+// (fp16 operands holding small integers, fp32 accumulators): the peak of the
+// fp16-operand GEMMs.
+__global__ void __launch_bounds__(128, 1) k_test_mma_f16_rate(int n_mma, int* sink, int* err, uint64_t budget_ns) {
+    extern __shared__ __align__(1024) uint8_t rsm16_[];
+    uint64_t* done = reinterpret_cast<uint64_t*>(rsm16_);
+    uint32_t* tbase = reinterpret_cast<uint32_t*>(rsm16_ + 8);
+    uint8_t* a = rsm16_ + 1024;               // 128 x 16 fp16 (4 KB)
+    uint8_t* b = a + 128 * 32;                // 256 x 16 fp16 (8 KB)
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (128 + kRateN) * 32 / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(a)[i] = h2_pack_int((i & 7) + 1, (i & 3) - 2);
+    if (threadIdx.x == 0) {
+        mbar_init(done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase, 2 * kRateN);
+        tmem_relinquish();
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tbase;
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = umma_idesc_f16(128, kRateN);
+        const uint64_t ad = umma_desc(a, 128, 256), bd = umma_desc(b, 128, 256);
+        for (int i = 0; i < n_mma; ++i)
+            umma_f16(tmem + (uint32_t)((i & 1) * kRateN), ad, bd, idesc, i >= 2 ? 1u : 0u);
         umma_commit(done);
     }
     __syncwarp();

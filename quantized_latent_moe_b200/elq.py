@@ -32,7 +32,7 @@ class ElqError(RuntimeError):
 class QMat(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("n_rows", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("gs_rows", ctypes.c_int32), ("q", ctypes.c_void_p), ("d", ctypes.c_void_p),
-                ("gs", ctypes.c_void_p)]
+                ("gs", ctypes.c_void_p), ("q16", ctypes.c_void_p)]
 
 
 class LayerC(ctypes.Structure):
@@ -51,6 +51,8 @@ SIGNATURES = {
     "elq_version": (I32, []),
     "elq_arena_bytes": (SZ, [I32, I32, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "elq_arena_pack": (I32, [I32, V, I32, I32, V, V, V]),
+    "elq_f16_bytes": (SZ, [V]),
+    "elq_pack_f16": (I32, [V, V, V]),
     "elq_quantize_weights": (I32, [I32, V, I32, I32, V, V, V]),
     "elq_quantize_gate_up": (I32, [I32, V, V, I32, I32, I32, V, V, V]),
     "elq_quantize_q8_1": (I32, [V, I32, I64, I64, V, V]),
@@ -73,6 +75,7 @@ SIGNATURES = {
     "elq_test_block_isums": (I32, [I32, V, V, I64, V, V, V]),
     "elq_test_expf": (I32, [V, V, I64, V]),
     "elq_test_mma_i8_rate": (I32, [I32, V, V, V]),
+    "elq_test_mma_f16_rate": (I32, [I32, V, V, V]),
     "elq_test_mma_nvf4_rate": (I32, [I32, I32, I32, V, V, V]),
     "elq_sm_count": (I32, []),
     "elq_test_f32x2_rate": (I32, [I32, V, V]),
@@ -135,6 +138,7 @@ class QMatrix:
         self.gs_rows = (gs_rows or n_rows) if fmt == NVFP4 else 0
         self.gs = (torch.ones(n_rows // self.gs_rows, dtype=torch.float32, device=device)
                    if fmt == NVFP4 else None)
+        self.q16 = None         # fp16 codes for the fp16-operand tensor-core GEMMs (Q8_0), or None
 
     @classmethod
     def from_f32(cls, w: torch.Tensor, fmt: int, stream=None) -> "QMatrix":
@@ -153,7 +157,22 @@ class QMatrix:
 
     def struct(self) -> QMat:
         return QMat(self.fmt, self.n_rows, self.k, self.gs_rows, self.q.data_ptr(), self.d.data_ptr(),
-                    None if self.gs is None else self.gs.data_ptr())
+                    None if self.gs is None else self.gs.data_ptr(),
+                    None if self.q16 is None else self.q16.data_ptr())
+
+    def pack_f16(self, stream=None) -> "QMatrix":
+        """Fills ``q16`` with the codes widened to fp16 (elq_pack_f16); Q8_0 only."""
+        m = self.struct()
+        m.q16 = None
+        n = _lib().elq_f16_bytes(ctypes.byref(m))
+        if not n:
+            raise ElqError(-2, "elq_f16_bytes")
+        self.q16 = _dev_empty(n, self.q.device)
+        _ck(_lib().elq_pack_f16(ctypes.byref(m), _ptr(self.q16), _stream(stream)), "elq_pack_f16")
+        return self
+
+    def drop_f16(self):
+        self.q16 = None
 
 
 class Layer:
@@ -175,6 +194,22 @@ class Layer:
         return cls(H, L, E, k, I, QMatrix(du_fmt, L, H, device), QMatrix(du_fmt, H, L, device),
                    router_w, router_bias, QMatrix(ex_fmt, E * 2 * I, L, device, gs_rows=2 * I),
                    QMatrix(ex_fmt, E * L, I, device, gs_rows=L))
+
+    def enable_f16(self, stream=None):
+        """Builds the fp16 codes of every Q8_0 matrix of the layer, so that calls
+        with T >= 16 multiply fp16 operands (same results; twice the codes' bytes
+        held in addition)."""
+        for m in (self.D, self.U, self.gate_up, self.down):
+            if m.fmt == FMT["q8_0"]:
+                m.pack_f16(stream)
+        self._ws = {}
+        return self
+
+    def disable_f16(self):
+        for m in (self.D, self.U, self.gate_up, self.down):
+            m.drop_f16()
+        self._ws = {}
+        return self
 
     def set_dense(self, D: torch.Tensor, U: torch.Tensor, stream=None):
         for m, w in ((self.D, D), (self.U, U)):
@@ -493,6 +528,16 @@ def test_mma_i8_rate(n_mma: int, device="cuda", stream=None):
     sink = torch.zeros(n, dtype=torch.int32, device=device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     _ck(_lib().elq_test_mma_i8_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_i8_rate")
+    return sink, err
+
+
+def test_mma_f16_rate(n_mma: int, device="cuda", stream=None):
+    """Launches the fp16 tensor-core rate kernel (elq_test_mma_f16_rate) on the
+    current stream; returns (sink, err) device tensors.  The caller times it."""
+    n = int(_lib().elq_sm_count())
+    sink = torch.zeros(n, dtype=torch.int32, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    _ck(_lib().elq_test_mma_f16_rate(n_mma, _ptr(sink), _ptr(err), _stream(stream)), "elq_test_mma_f16_rate")
     return sink, err
 
 

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.elq_version() == 2
+    assert L.elq_version() == 3
     assert L.elq_status_string(0) == b"ok"
     assert L.elq_status_string(-4).startswith(b"workspace")
     assert L.elq_status_string(123) == b"unknown status"

@@ -158,13 +158,16 @@ def _check_tc(E, ly, T, tr):
     return v("y_lat").reshape(T, -1)
 
 
-@pytest.mark.parametrize("T", [9, 16, 64, 127, 128, 129, 300])
-def test_nvfp4_tc_layer(E, orc, T):
+@pytest.mark.parametrize("T,f16", [(9, False), (16, False), (64, False), (127, False), (128, False),
+                                   (129, False), (300, False), (16, True), (129, True)])
+def test_nvfp4_tc_layer(E, orc, T, f16):
     """The block-scaled tensor-core experts (eleven kernels), from just above
     the GEMV's sizes through several 128-slot tiles per expert and ragged last
-    tiles."""
+    tiles; D and U on int8 or fp16-widened codes."""
     wl = NV_TINY
     ly = gpu_layer(wl)
+    if f16:
+        ly.enable_f16()
     assert ly.kernel_count(T) == 11
     ol = oracle_layer(orc, wl)
     x = synth.make_x(wl, T=T)

@@ -1,5 +1,6 @@
-"""Parity of the tensor-core path (tcgen05 kind::i8, T >= 16, Q8_0 weights)
-with the CPU oracle, through the C ABI."""
+"""Parity of the tensor-core path (tcgen05 kind::i8, or kind::f16 on the
+codes widened to fp16, T >= 16, Q8_0 weights) with the CPU oracle, through
+the C ABI."""
 import numpy as np
 import pytest
 import torch
@@ -30,10 +31,34 @@ def test_tc_latent_proj_exact(E, orc, N, K, T):
     assert np.array_equal(y, ref)
 
 
+def test_f16_codes_layout(E):
+    """elq_pack_f16 against the layout the header states, built here from the
+    quantised weights' codes: per (tile, block) [code/16][row/8][(code%16)/8]
+    [row%8][8 fp16], the value of row r's code c of the block."""
+    n_rows, k = 256, 128
+    W = synth.normal(23, 7, (n_rows, k), 0.02)
+    m = E.QMatrix.from_f32(W.cuda(), 8).pack_f16()
+    # the codes by row, independent of the int8 arena: the Q8_0 quantiser's blocks
+    import oracle
+    oracle.lib()
+    codes = np.frombuffer(oracle.quantize(8, W.numpy()).tobytes(), np.uint8).reshape(n_rows, k // 32, 34)[:, :, 2:]
+    codes = codes.view(np.int8)
+    got = m.q16.cpu().numpy().view(np.float16).reshape(n_rows // 128, k // 32, 4096)
+    exp = np.zeros_like(got)
+    for r in range(128):
+        for c in range(32):
+            dst = ((c // 16) * 4096 + (r // 8) * 256 + ((c % 16) // 8) * 128 + (r % 8) * 16 + (c % 8) * 2) // 2
+            exp[:, :, dst] = codes[r::128, :, c].astype(np.float16).reshape(n_rows // 128, k // 32)
+    assert np.array_equal(got, exp)
+
+
+@pytest.mark.parametrize("f16", [False, True], ids=["i8", "f16"])
 @pytest.mark.parametrize("T", [64, 100, 257])
-def test_tc_layer_tiny_exact(E, orc, T):
+def test_tc_layer_tiny_exact(E, orc, T, f16):
     wl = synth.WORKLOADS["tiny"]
     ly = gpu_layer(wl)
+    if f16:
+        ly.enable_f16()
     assert ly.kernel_count(T) == 10
     x = synth.make_x(wl, T=T)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
@@ -51,10 +76,13 @@ def test_tc_layer_tiny_exact(E, orc, T):
     assert np.array_equal(y, tr["y"])
 
 
-def test_tc_experts_grouped_exact(E, orc):
+@pytest.mark.parametrize("f16", [False, True], ids=["i8", "f16"])
+def test_tc_experts_grouped_exact(E, orc, f16):
     wl = synth.WORKLOADS["tiny"]
     T = 96
     ly = gpu_layer(wl)
+    if f16:
+        ly.enable_f16()
     ol = oracle_layer(orc, wl)
     tr = ol.forward(synth.make_x(wl, T=T).numpy(), trace=True)
     y_lat = E.moe_experts_grouped(ly, torch.from_numpy(tr["zq"]).cuda(), torch.from_numpy(tr["idx"]).cuda(),
@@ -69,7 +97,8 @@ def _threads(fn, parts):
         return list(ex.map(fn, parts))
 
 
-def test_tc_prefill_full_size(E, orc):
+@pytest.mark.parametrize("f16", [False, True], ids=["i8", "f16"])
+def test_tc_prefill_full_size(E, orc, f16):
     """The prefill workload at full size (T=2048, 128 experts, Zipf-skewed
     router), through the layer call:
      - z and its Q8_1 rows for all 2048 tokens against the oracle's quantised
@@ -84,6 +113,8 @@ def test_tc_prefill_full_size(E, orc):
        and 2047."""
     wl = synth.WORKLOADS["prefill"]
     ly = gpu_layer(wl)
+    if f16:
+        ly.enable_f16()
     x = synth.make_x(wl)
     y = E.moe_layer(ly, x.cuda()).cpu().numpy()
     assert E.workspace_status(ly.workspace(wl.T)) == 0
