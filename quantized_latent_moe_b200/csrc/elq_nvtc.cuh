@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_nvgemm(const __grid_constant_
     const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
     const int kstages = g.nks / kNvKS;
     volatile int* abort_v = abort_sm;
-    stage_units(g, u0, u1, su, stt);
+    stage_units(g, u0, 1, u1 - u0, su, stt);
     auto unit_at = [&](int u) { return u - u0 < kUnitsSmem ? su[u - u0] : tc_unit(g, u); };
 
     if (warp == 0) {

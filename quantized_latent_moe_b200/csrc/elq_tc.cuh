@@ -566,19 +566,19 @@ __device__ __forceinline__ TcUnit unit_staged(const A& g, int u, const int* stt,
     return r;
 }
 
-// The CTA's units [u0, u1) (the first kUnitsSmem) into su, all threads;
-// ends with a CTA barrier.  Dense launches (no routing) compute theirs
-// directly.
+// The CTA's units u0 + i * step, i < n (the first kUnitsSmem) into su, all
+// threads; ends with a CTA barrier.  Dense launches (no routing) compute
+// theirs directly.
 template <class A>
-__device__ void stage_units(const A& g, int u0, int u1, TcUnit* su, int* stt) {
-    const int n = min(u1 - u0, kUnitsSmem);
+__device__ void stage_units(const A& g, int u0, int step, int n_all, TcUnit* su, int* stt) {
+    const int n = min(n_all, kUnitsSmem);
     const int na = g.act ? __ldcg(g.n_act) : 0;
     if (g.act && na + 1 <= kUnitTableInts) {
         for (int i = threadIdx.x; i <= na; i += blockDim.x) stt[i] = __ldcg(g.tt_off + i);
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = unit_staged(g, u0 + i, stt, na);
+        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = unit_staged(g, u0 + i * step, stt, na);
     } else {
-        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = tc_unit(g, u0 + i);
+        for (int i = threadIdx.x; i < n; i += blockDim.x) su[i] = tc_unit(g, u0 + i * step);
     }
     __syncthreads();
 }
@@ -639,12 +639,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tcgemm(const __grid_constant_
     pdl_wait();
 
     const int n_units = tc_units(g);
-    const int u0 = (int)((int64_t)n_units * blockIdx.x / gridDim.x);
-    const int u1 = (int)((int64_t)n_units * (blockIdx.x + 1) / gridDim.x);
+    // CTA b takes units b, b + grid, b + 2 grid, ...: at any moment the CTAs work on neighbouring
+    // units, so a weight row tile (the units of one row tile are consecutive) and an activation
+    // tile are read by several CTAs together and come from L2 after the first (loop index u: the
+    // CTA's i-th unit)
+    const int n_mine = n_units > (int)blockIdx.x ? (n_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                                                 : 0;
+    const int u0 = 0, u1 = n_mine;
     const int kstages = g.nb / kTcKS;
     volatile int* abort_v = abort_sm;
-    stage_units(g, u0, u1, su, stt);
-    auto unit_at = [&](int u) { return u - u0 < kUnitsSmem ? su[u - u0] : tc_unit(g, u); };
+    stage_units(g, (int)blockIdx.x, (int)gridDim.x, n_mine, su, stt);
+    auto unit_at = [&](int i) {
+        return i < kUnitsSmem ? su[i] : tc_unit(g, (int)blockIdx.x + i * (int)gridDim.x);
+    };
 
     if (warp == 0) {
         // ---------------- producer ----------------
