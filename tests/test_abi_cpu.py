@@ -291,3 +291,57 @@ def test_other_entry_validation(L):
     assert L.elq_quantize_gate_up(8, p, p, 2, 96, 64, p, p, None) == -2
     assert L.elq_test_block_isums(9, p, p, 4, p, p, None) == -2
     assert L.elq_workspace_status(None, None) == -1
+
+
+def _with_q16(ly, names=("D", "U", "gate_up", "down"), base=1 << 29):
+    for i, n in enumerate(names):
+        m = getattr(ly, n)
+        m.q16 = base + i * (1 << 24)
+        setattr(ly, n, m)
+    return ly
+
+
+def test_f16_codes_validation(L):
+    """The fp16 codes of a matrix: their size, the formats that may carry them,
+    their alignment, and the workspace of a tensor-core call that uses them
+    (the B operands' codes take twice the bytes)."""
+    assert L.elq_f16_bytes(ctypes.byref(_qm(8, 256, 512))) == 256 * 512 * 2
+    assert L.elq_f16_bytes(ctypes.byref(_qm(2, 256, 512))) == 0          # Q4_0 has none
+    assert L.elq_f16_bytes(None) == 0
+    q16 = ctypes.c_void_p(1 << 29)
+    assert L.elq_pack_f16(ctypes.byref(_qm(2, 256, 512)), q16, None) == -2
+    assert L.elq_pack_f16(ctypes.byref(_qm(8, 256, 512)), ctypes.c_void_p((1 << 29) + 16), None) == -3
+    assert L.elq_pack_f16(ctypes.byref(_qm(8, 256, 512)), None, None) == -1
+    assert L.elq_pack_f16(None, q16, None) == -1
+    x = ctypes.c_void_p(1 << 27)
+    y = ctypes.c_void_p(1 << 28)
+    ws = ctypes.c_void_p(1 << 26)
+    good = _with_q16(_layer())
+    # the same launch sequence; a bigger workspace only where the tensor-core path runs
+    assert L.elq_layer_kernel_count(ctypes.byref(good), 64) == 10
+    assert L.elq_workspace_bytes(ctypes.byref(good), 64) > L.elq_workspace_bytes(ctypes.byref(_layer()), 64)
+    assert L.elq_workspace_bytes(ctypes.byref(good), 4) == L.elq_workspace_bytes(ctypes.byref(_layer()), 4)
+    # only some matrices with fp16 codes: the int8 GEMMs, the int8 workspace
+    part = _with_q16(_layer(), names=("D", "U"))
+    assert L.elq_workspace_bytes(ctypes.byref(part), 64) == L.elq_workspace_bytes(ctypes.byref(_layer()), 64)
+    # fp16 codes on a Q4_0 matrix, or misaligned: refused before any launch
+    bad = _with_q16(_layer(fmt=2), names=("D",))
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws, 1 << 30, None) == -2
+    bad = _with_q16(_layer(), names=("U",), base=(1 << 29) + 64)
+    assert L.elq_moe_layer(ctypes.byref(bad), x, 0, 4, y, ws, 1 << 30, None) == -3
+
+
+def test_bench_f16_choice():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_latent_moe_b200 import synth
+
+    class A:
+        f16 = "auto"
+    a = A()
+    assert bench.use_f16(a, synth.WORKLOADS["prefill"]) and not bench.use_f16(a, synth.WORKLOADS["decode"])
+    a.f16 = "off"
+    assert not bench.use_f16(a, synth.WORKLOADS["prefill"])
+    a.f16 = "on"
+    assert bench.use_f16(a, synth.WORKLOADS["decode"])
