@@ -9,6 +9,13 @@ experts top-8, expert FFN I=1024, Q8_0 weights, bf16 input, router bias
 N(0, 1) per expert.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl elq|reference]
+                  [--workload decode|verify|prefill|prefill_nvfp4|decode_nvfp4|decode_q4_k|decode_q3_k|stack|tiny]
+                  [--f16 auto|on|off]
+
+--f16: the layers also hold their Q8_0 codes widened to fp16, so that calls
+taking the tensor-core path (T >= 16) multiply fp16 operands into exact fp32
+accumulators (the same results); auto = on for the workloads with T >= 16
+except the 48-layer stack (whose copies would take ~70 GB more).
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 synchronize on both sides, timed with CUDA events on the launching stream; the
